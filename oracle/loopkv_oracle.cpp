@@ -1,0 +1,442 @@
+// LoopKV oracle: a plain, slow, single-threaded CPU restatement of what the
+// LoopKV decode path computes.  TEST INFRASTRUCTURE ONLY: the tests, the
+// smoke check and the benchmark's CPU-baseline leg may call it; the product
+// path never does.  It shares no code, header, table or constant with the
+// CUDA library.
+//
+// Source of the method: "LoopKV: Loop-Aware KV Cache Compression for Serving
+// Looped Transformers", section 概要 (the abstract):
+//   * each (loop, layer) cell keeps 4-bit codes, 2-bit codes, or reuses the
+//     final loop's KV (SHARE);
+//   * a 4-bit value is read as its high 2 bits, and its low 2 bits are
+//     fetched only where the loop's own attention weights need 4-bit
+//     precision.
+// The abstract leaves the arithmetic open; this file takes these readings:
+//   R1 asymmetric min/max quantization as in "KIVI: A Tuning-Free Asymmetric
+//      2bit Quantization for KV Cache": keys per channel over a group of 32
+//      tokens, values per token over groups of 32 channels, fp32 scale and
+//      zero point (zero = group minimum), codes rounded half-to-even;
+//   R2 the IEEE fp32 operations that produce a code are fixed:
+//      scale = (max - min) / qmax, code = rne((x - min) / scale), no fused
+//      multiply-add, -0 zero point stored as +0, scale 0 => all codes 0;
+//   R3 a 4-bit code q splits as hi = q >> 2 (high plane), lo = q & 3 (low
+//      plane); a high-plane-only read reconstructs 4*hi + 1.5;
+//   R4 a token of a 4-bit cell whose softmax weight p >= tau gets hi+lo, all
+//      others hi only; keys are always read at stored precision;
+//   R5 fewer than 32 recent tokens stay in a bf16 residual; the residual is
+//      quantized as a group the moment it holds 32 tokens;
+//   R6 a SHARE cell of length n attends over the final loop's stored
+//      positions [0, n-1) plus its own current bf16 key and value;
+//   R7 softmax scale 1/sqrt(D) unless given; one query per KV head.
+// All attention arithmetic is fp64 (dequantized values, scores, softmax,
+// weighted sum).  Quantization is fp32 because the codes are defined by it.
+//
+// Build: g++ -O2 -std=c++17 -ffp-contract=off -fno-fast-math -shared -fPIC
+// (no contraction and no fast-math, so the fp32 steps are the IEEE ones).
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+namespace {
+
+constexpr int kG = 32;  // group size (R1)
+
+enum Kind { KIND_Q4 = 0, KIND_Q2 = 1, KIND_SHARE = 2, KIND_BF16 = 3 };
+
+float bf16_to_float(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+// One group of 32 fp32 values -> codes, scale, zero (R1, R2).
+void quantize_group(const float* x, int bits, uint8_t* code, float* scale,
+                    float* zero) {
+  const int qmax = (1 << bits) - 1;
+  float mn = x[0], mx = x[0];
+  for (int i = 1; i < kG; ++i) {
+    if (x[i] < mn) mn = x[i];
+    if (x[i] > mx) mx = x[i];
+  }
+  const float range = mx - mn;               // fp32, round to nearest
+  const float s = range / static_cast<float>(qmax);
+  for (int i = 0; i < kG; ++i) {
+    if (s == 0.0f) {
+      code[i] = 0;
+      continue;
+    }
+    const float shifted = x[i] - mn;          // fp32
+    const float ratio = shifted / s;          // fp32
+    float r = std::nearbyint(ratio);          // default mode: half to even
+    if (r < 0.0f) r = 0.0f;
+    if (r > static_cast<float>(qmax)) r = static_cast<float>(qmax);
+    code[i] = static_cast<uint8_t>(r);
+  }
+  *scale = s;
+  *zero = (mn == 0.0f) ? 0.0f : mn;  // canonical +0
+}
+
+// State of one (cell, sequence, head) unit after some appends.
+struct Unit {
+  int kind = 0, D = 0, cap = 0, n = 0;
+  // KIND_Q4 / KIND_Q2: quantized groups and the bf16 residual (R5).
+  std::vector<uint8_t> kq;   // [qtok][D] key codes
+  std::vector<float> ks, kz; // [qtok/32][D] per-channel key scale, zero
+  std::vector<uint8_t> vq;   // [qtok][D] value codes
+  std::vector<float> vs, vz; // [qtok][D/32] per-token value scale, zero
+  std::vector<uint16_t> rk, rv;  // residual [R][D] bf16 bits
+  // KIND_BF16: every token raw.
+  std::vector<uint16_t> bk, bv;  // [n][D]
+  // KIND_SHARE: the current token only.
+  std::vector<uint16_t> ck, cv;  // [D]
+
+  int qtok() const { return (kind == KIND_Q4 || kind == KIND_Q2) ? n - residual() : 0; }
+  int residual() const { return static_cast<int>(rk.size()) / D; }
+  int bits() const { return kind == KIND_Q4 ? 4 : 2; }
+
+  void flush_group() {
+    // keys: per channel over the 32 residual tokens
+    const int g = static_cast<int>(ks.size()) / D;
+    const size_t tok0 = kq.size() / D;
+    kq.resize((tok0 + kG) * D);
+    vq.resize((tok0 + kG) * D);
+    ks.resize((g + 1) * D);
+    kz.resize((g + 1) * D);
+    vs.resize((tok0 + kG) * (D / kG));
+    vz.resize((tok0 + kG) * (D / kG));
+    float x[kG];
+    uint8_t c[kG];
+    for (int d = 0; d < D; ++d) {
+      for (int i = 0; i < kG; ++i) x[i] = bf16_to_float(rk[i * D + d]);
+      quantize_group(x, bits(), c, &ks[g * D + d], &kz[g * D + d]);
+      for (int i = 0; i < kG; ++i) kq[(tok0 + i) * D + d] = c[i];
+    }
+    // values: per token over groups of 32 channels
+    for (int i = 0; i < kG; ++i) {
+      for (int j = 0; j < D / kG; ++j) {
+        for (int e = 0; e < kG; ++e) x[e] = bf16_to_float(rv[i * D + j * kG + e]);
+        const size_t t = tok0 + i;
+        quantize_group(x, bits(), c, &vs[t * (D / kG) + j], &vz[t * (D / kG) + j]);
+        for (int e = 0; e < kG; ++e) vq[t * D + j * kG + e] = c[e];
+      }
+    }
+    rk.clear();
+    rv.clear();
+  }
+
+  // Append one token (bf16 bits) following R5 / R6.
+  void append_token(const uint16_t* k, const uint16_t* v) {
+    if (kind == KIND_SHARE) {
+      ck.assign(k, k + D);
+      cv.assign(v, v + D);
+    } else if (kind == KIND_BF16) {
+      bk.insert(bk.end(), k, k + D);
+      bv.insert(bv.end(), v, v + D);
+    } else {
+      rk.insert(rk.end(), k, k + D);
+      rv.insert(rv.end(), v, v + D);
+      if (residual() == kG) flush_group();
+    }
+    ++n;
+  }
+};
+
+size_t round128(size_t x) { return (x + 127) / 128 * 128; }
+
+// Canonical per-unit region layout (the one the CUDA library writes).
+// Offsets in bytes from the start of the unit's region.
+struct Layout {
+  size_t k_hi = 0, k_lo = 0, k_meta = 0, v_hi = 0, v_lo = 0, v_meta = 0;
+  size_t res_k = 0, res_v = 0, cur_k = 0, cur_v = 0, raw_k = 0, raw_v = 0;
+  size_t total = 0;
+};
+
+Layout make_layout(int kind, int D, int cap) {
+  Layout L;
+  const size_t ng = static_cast<size_t>(cap / kG);
+  const size_t kblock = ng * 8 * D;           // one key plane or key meta
+  const size_t vblock = ng * kG * (D / 4);    // one value plane or value meta
+  const size_t rblock = static_cast<size_t>(kG) * D * 2;
+  size_t off = 0;
+  if (kind == KIND_Q4 || kind == KIND_Q2) {
+    L.k_hi = off; off += round128(kblock);
+    if (kind == KIND_Q4) { L.k_lo = off; off += round128(kblock); }
+    L.k_meta = off; off += round128(kblock);
+    L.v_hi = off; off += round128(vblock);
+    if (kind == KIND_Q4) { L.v_lo = off; off += round128(vblock); }
+    L.v_meta = off; off += round128(vblock);
+    L.res_k = off; off += rblock;
+    L.res_v = off; off += rblock;
+  } else if (kind == KIND_SHARE) {
+    L.cur_k = off; off += round128(static_cast<size_t>(D) * 2);
+    L.cur_v = off; off += round128(static_cast<size_t>(D) * 2);
+  } else {
+    L.raw_k = off; off += round128(static_cast<size_t>(cap) * D * 2);
+    L.raw_v = off; off += round128(static_cast<size_t>(cap) * D * 2);
+  }
+  L.total = off;
+  return L;
+}
+
+void put_bytes(uint8_t* out, uint8_t* valid, size_t off, const void* src, size_t n) {
+  std::memcpy(out + off, src, n);
+  std::memset(valid + off, 1, n);
+}
+
+}  // namespace
+
+extern "C" {
+
+// ---- quantizer -------------------------------------------------------------
+void orc_quantize_group(const float* x, int bits, uint8_t* code, float* scale,
+                        float* zero) {
+  quantize_group(x, bits, code, scale, zero);
+}
+
+// ---- unit state ------------------------------------------------------------
+void* orc_unit_new(int kind, int D, int cap) {
+  if (kind < 0 || kind > 3 || (D != 64 && D != 128) || cap < 0) return nullptr;
+  Unit* u = new Unit();
+  u->kind = kind;
+  u->D = D;
+  u->cap = cap;
+  return u;
+}
+
+void orc_unit_free(void* p) { delete static_cast<Unit*>(p); }
+
+int orc_unit_len(const void* p) { return static_cast<const Unit*>(p)->n; }
+
+// Append n_new tokens given as bf16 bits [n_new][D] each.  Returns 0, or -1
+// when the capacity would be exceeded (nothing is appended then).
+int orc_unit_append(void* p, const uint16_t* k, const uint16_t* v, int n_new) {
+  Unit* u = static_cast<Unit*>(p);
+  if (n_new < 0) return -1;
+  if (u->kind != KIND_SHARE && u->n + n_new > u->cap) return -1;
+  for (int t = 0; t < n_new; ++t)
+    u->append_token(k + static_cast<size_t>(t) * u->D, v + static_cast<size_t>(t) * u->D);
+  return 0;
+}
+
+// Quantized state, for tests: key codes [qtok][D], key scale/zero [qtok/32][D],
+// value codes [qtok][D], value scale/zero [qtok][D/32].  Any pointer may be
+// null.  Returns qtok.
+int orc_unit_export(const void* p, uint8_t* kq, float* ks, float* kz, uint8_t* vq,
+                    float* vs, float* vz) {
+  const Unit* u = static_cast<const Unit*>(p);
+  if (kq) std::copy(u->kq.begin(), u->kq.end(), kq);
+  if (ks) std::copy(u->ks.begin(), u->ks.end(), ks);
+  if (kz) std::copy(u->kz.begin(), u->kz.end(), kz);
+  if (vq) std::copy(u->vq.begin(), u->vq.end(), vq);
+  if (vs) std::copy(u->vs.begin(), u->vs.end(), vs);
+  if (vz) std::copy(u->vz.begin(), u->vz.end(), vz);
+  return u->qtok();
+}
+
+size_t orc_region_bytes(int kind, int D, int cap) { return make_layout(kind, D, cap).total; }
+
+// Write the unit's bytes in the canonical layout; valid[i] = 1 for every byte
+// the layout defines at the unit's current length (unused groups and residual
+// slots stay 0 in both arrays).  Returns 0, or -1 on a size mismatch.
+int orc_unit_serialize(const void* p, uint8_t* out, uint8_t* valid, size_t bytes) {
+  const Unit* u = static_cast<const Unit*>(p);
+  const int D = u->D;
+  const Layout L = make_layout(u->kind, D, u->cap);
+  if (bytes != L.total) return -1;
+  std::memset(out, 0, bytes);
+  std::memset(valid, 0, bytes);
+  if (u->kind == KIND_SHARE) {
+    if (u->n > 0) {
+      put_bytes(out, valid, L.cur_k, u->ck.data(), D * 2);
+      put_bytes(out, valid, L.cur_v, u->cv.data(), D * 2);
+    }
+    return 0;
+  }
+  if (u->kind == KIND_BF16) {
+    put_bytes(out, valid, L.raw_k, u->bk.data(), u->bk.size() * 2);
+    put_bytes(out, valid, L.raw_v, u->bv.data(), u->bv.size() * 2);
+    return 0;
+  }
+  const bool q4 = u->kind == KIND_Q4;
+  const int ngq = u->qtok() / kG;
+  for (int g = 0; g < ngq; ++g) {
+    // key planes: [g][chunk of 64 channels][token][4 words of 16 codes]
+    for (int c = 0; c < D / 64; ++c) {
+      for (int t = 0; t < kG; ++t) {
+        for (int w = 0; w < 4; ++w) {
+          uint32_t hi = 0, lo = 0;
+          for (int j = 0; j < 16; ++j) {
+            const int d = 64 * c + 16 * w + j;
+            const uint32_t q = u->kq[static_cast<size_t>(g * kG + t) * D + d];
+            const uint32_t plane_hi = q4 ? (q >> 2) : q;
+            hi |= (plane_hi & 3u) << (2 * j);
+            lo |= (q & 3u) << (2 * j);
+          }
+          const size_t off = static_cast<size_t>(g) * 8 * D + c * 512 + t * 16 + w * 4;
+          put_bytes(out, valid, L.k_hi + off, &hi, 4);
+          if (q4) put_bytes(out, valid, L.k_lo + off, &lo, 4);
+        }
+      }
+    }
+    // key meta: scale[D] then zero[D]
+    put_bytes(out, valid, L.k_meta + static_cast<size_t>(g) * 8 * D, &u->ks[g * D], 4 * D);
+    put_bytes(out, valid, L.k_meta + static_cast<size_t>(g) * 8 * D + 4 * D, &u->kz[g * D], 4 * D);
+  }
+  for (int t = 0; t < u->qtok(); ++t) {
+    // value planes: [token][D/16 words]
+    for (int w = 0; w < D / 16; ++w) {
+      uint32_t hi = 0, lo = 0;
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t q = u->vq[static_cast<size_t>(t) * D + 16 * w + j];
+        const uint32_t plane_hi = q4 ? (q >> 2) : q;
+        hi |= (plane_hi & 3u) << (2 * j);
+        lo |= (q & 3u) << (2 * j);
+      }
+      const size_t off = static_cast<size_t>(t) * (D / 4) + w * 4;
+      put_bytes(out, valid, L.v_hi + off, &hi, 4);
+      if (q4) put_bytes(out, valid, L.v_lo + off, &lo, 4);
+    }
+    // value meta: (scale_j, zero_j) pairs
+    for (int j = 0; j < D / kG; ++j) {
+      const size_t off = static_cast<size_t>(t) * (D / 4) + j * 8;
+      put_bytes(out, valid, L.v_meta + off, &u->vs[t * (D / kG) + j], 4);
+      put_bytes(out, valid, L.v_meta + off + 4, &u->vz[t * (D / kG) + j], 4);
+    }
+  }
+  for (int r = 0; r < u->residual(); ++r) {
+    put_bytes(out, valid, L.res_k + static_cast<size_t>(r) * D * 2, &u->rk[r * D], D * 2);
+    put_bytes(out, valid, L.res_v + static_cast<size_t>(r) * D * 2, &u->rv[r * D], D * 2);
+  }
+  return 0;
+}
+
+// ---- decode ----------------------------------------------------------------
+// Decode one unit.  own: the unit; src: the final loop's unit of the same
+// layer, sequence and head when own is SHARE (else ignored).  q: bf16 bits
+// [D].  sm_scale <= 0 means 1/sqrt(D).
+// Outputs: out[D]; *lse (natural log); mask words, one per 32 positions of the
+// data cell's quantized range, bit j of word g = position 32g+j selected
+// (only when the data cell is 4-bit); *nsel; slack[D] (nullable) = sum over
+// 4-bit positions with |p - tau| <= band of p * scale_v * |lo - 1.5|, the most
+// a disagreement on those positions can move each output.
+// *n_mask_words receives the number of mask words written; weights (nullable)
+// receives the softmax weight of every attended position, own current last.
+// Returns 0, or -1 on invalid input (no positions, SHARE without a source,
+// SHARE longer than its source allows).
+int orc_decode(const void* own_p, const void* src_p, const uint16_t* q,
+               double tau, double sm_scale, double band, double* out,
+               double* lse, uint32_t* mask, int* n_mask_words, int* nsel,
+               double* slack, double* weights) {
+  const Unit* own = static_cast<const Unit*>(own_p);
+  const Unit* src = static_cast<const Unit*>(src_p);
+  const int D = own->D;
+  const Unit* data = own;
+  int n_att = own->n;
+  const bool share = own->kind == KIND_SHARE;
+  if (share) {
+    if (src == nullptr || src->kind == KIND_SHARE || src->D != D) return -1;
+    data = src;
+    n_att = own->n - 1;  // R6
+    if (own->n < 1 || n_att > src->n) return -1;
+  }
+  if (n_att + (share ? 1 : 0) < 1) return -1;
+  if (sm_scale <= 0.0) sm_scale = 1.0 / std::sqrt(static_cast<double>(D));
+
+  std::vector<double> qd(D);
+  for (int d = 0; d < D; ++d) qd[d] = static_cast<double>(bf16_to_float(q[d]));
+
+  const bool quant = data->kind == KIND_Q4 || data->kind == KIND_Q2;
+  const int qtok = quant ? data->qtok() : 0;
+  const int npos = n_att + (share ? 1 : 0);
+
+  // dequantized key of a position (fp64)
+  std::vector<double> khat(D);
+  auto key_of = [&](int pos) {
+    if (share && pos == n_att) {
+      for (int d = 0; d < D; ++d) khat[d] = bf16_to_float(own->ck[d]);
+    } else if (data->kind == KIND_BF16) {
+      for (int d = 0; d < D; ++d) khat[d] = bf16_to_float(data->bk[static_cast<size_t>(pos) * D + d]);
+    } else if (pos < qtok) {
+      const int g = pos / kG;
+      for (int d = 0; d < D; ++d)
+        khat[d] = static_cast<double>(data->ks[g * D + d]) *
+                      data->kq[static_cast<size_t>(pos) * D + d] +
+                  static_cast<double>(data->kz[g * D + d]);
+    } else {
+      const int r = pos - qtok;
+      for (int d = 0; d < D; ++d) khat[d] = bf16_to_float(data->rk[static_cast<size_t>(r) * D + d]);
+    }
+  };
+
+  // scores and softmax
+  std::vector<double> s(npos), p(npos);
+  double smax = -INFINITY;
+  for (int pos = 0; pos < npos; ++pos) {
+    key_of(pos);
+    double acc = 0.0;
+    for (int d = 0; d < D; ++d) acc += qd[d] * khat[d];
+    s[pos] = sm_scale * acc;
+    smax = std::max(smax, s[pos]);
+  }
+  double sum = 0.0;
+  for (int pos = 0; pos < npos; ++pos) sum += std::exp(s[pos] - smax);
+  const double l = smax + std::log(sum);
+  for (int pos = 0; pos < npos; ++pos) p[pos] = std::exp(s[pos] - l);
+  *lse = l;
+  if (weights) std::copy(p.begin(), p.end(), weights);
+
+  // selection mask over the 4-bit quantized positions (R4)
+  const bool q4 = data->kind == KIND_Q4;
+  const int nq_att = q4 ? std::min(n_att, qtok) : 0;
+  const int nwords = (nq_att + kG - 1) / kG;
+  for (int w = 0; w < nwords; ++w) mask[w] = 0;
+  int count = 0;
+  std::vector<char> sel(npos, 0);
+  for (int pos = 0; pos < nq_att; ++pos) {
+    if (p[pos] >= tau) {
+      sel[pos] = 1;
+      mask[pos / kG] |= 1u << (pos % kG);
+      ++count;
+    }
+  }
+  *n_mask_words = nwords;
+  *nsel = count;
+
+  // weighted values
+  for (int d = 0; d < D; ++d) out[d] = 0.0;
+  if (slack) for (int d = 0; d < D; ++d) slack[d] = 0.0;
+  for (int pos = 0; pos < npos; ++pos) {
+    for (int d = 0; d < D; ++d) {
+      double v;
+      if (share && pos == n_att) {
+        v = bf16_to_float(own->cv[d]);
+      } else if (data->kind == KIND_BF16) {
+        v = bf16_to_float(data->bv[static_cast<size_t>(pos) * D + d]);
+      } else if (pos < qtok) {
+        const int j = d / kG;
+        const double sc = data->vs[static_cast<size_t>(pos) * (D / kG) + j];
+        const double ze = data->vz[static_cast<size_t>(pos) * (D / kG) + j];
+        const int code = data->vq[static_cast<size_t>(pos) * D + d];
+        if (q4) {
+          const int hi = code >> 2, lo = code & 3;
+          const double low_part = sel[pos] ? static_cast<double>(lo) : 1.5;  // R3
+          v = sc * (4.0 * hi + low_part) + ze;
+          if (slack && std::fabs(p[pos] - tau) <= band)
+            slack[d] += p[pos] * sc * std::fabs(lo - 1.5);
+        } else {
+          v = sc * code + ze;
+        }
+      } else {
+        v = bf16_to_float(data->rv[static_cast<size_t>(pos - qtok) * D + d]);
+      }
+      out[d] += p[pos] * v;
+    }
+  }
+  return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,158 @@
+"""ctypes wrapper around the C++ oracle (test infrastructure only).
+
+Every function here forwards to ``loopkv_oracle.cpp``; nothing is computed in
+Python beyond array allocation.  Arrays of bf16 values travel as their raw
+16-bit patterns (``numpy.uint16``).
+"""
+
+import ctypes
+import dataclasses
+
+import numpy as np
+
+from . import build as _build
+
+KIND_Q4, KIND_Q2, KIND_SHARE, KIND_BF16 = 0, 1, 2, 3
+G = 32
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(_build.build())
+    P = ctypes.c_void_p
+    lib.orc_quantize_group.argtypes = [P, ctypes.c_int, P, P, P]
+    lib.orc_quantize_group.restype = None
+    lib.orc_unit_new.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.orc_unit_new.restype = P
+    lib.orc_unit_free.argtypes = [P]
+    lib.orc_unit_free.restype = None
+    lib.orc_unit_len.argtypes = [P]
+    lib.orc_unit_len.restype = ctypes.c_int
+    lib.orc_unit_append.argtypes = [P, P, P, ctypes.c_int]
+    lib.orc_unit_append.restype = ctypes.c_int
+    lib.orc_unit_export.argtypes = [P, P, P, P, P, P, P]
+    lib.orc_unit_export.restype = ctypes.c_int
+    lib.orc_region_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.orc_region_bytes.restype = ctypes.c_size_t
+    lib.orc_unit_serialize.argtypes = [P, P, P, ctypes.c_size_t]
+    lib.orc_unit_serialize.restype = ctypes.c_int
+    lib.orc_decode.argtypes = [P, P, P, ctypes.c_double, ctypes.c_double,
+                               ctypes.c_double, P, P, P, P, P, P, P]
+    lib.orc_decode.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def quantize_group(x, bits):
+    """Quantize 32 fp32 values at ``bits`` (4 or 2) -> (codes u8[32], scale, zero)."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    assert x.shape == (G,)
+    code = np.zeros(G, np.uint8)
+    scale = np.zeros(1, np.float32)
+    zero = np.zeros(1, np.float32)
+    lib.orc_quantize_group(_ptr(x), bits, _ptr(code), _ptr(scale), _ptr(zero))
+    return code, scale[0], zero[0]
+
+
+def region_bytes(kind, D, cap):
+    """Bytes of one unit's region in the canonical cache layout."""
+    return int(_load().orc_region_bytes(kind, D, cap))
+
+
+class OracleUnit:
+    """One (cell, sequence, head) unit: its cache state after appends."""
+
+    def __init__(self, kind, D, cap):
+        lib = _load()
+        self._lib = lib  # free with the library that made the handle
+        self._h = lib.orc_unit_new(kind, D, cap)
+        if not self._h:
+            raise ValueError("bad unit kind=%r D=%r cap=%r" % (kind, D, cap))
+        self.kind, self.D, self.cap = kind, D, cap
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            self._lib.orc_unit_free(h)
+            self._h = None
+
+    @property
+    def n(self):
+        return int(self._lib.orc_unit_len(self._h))
+
+    def append(self, k_bits, v_bits):
+        """Append tokens given as bf16 bit patterns of shape [n_new, D]."""
+        k = np.ascontiguousarray(k_bits, dtype=np.uint16).reshape(-1, self.D)
+        v = np.ascontiguousarray(v_bits, dtype=np.uint16).reshape(-1, self.D)
+        assert k.shape == v.shape
+        rc = self._lib.orc_unit_append(self._h, _ptr(k), _ptr(v), k.shape[0])
+        if rc != 0:
+            raise ValueError("oracle append rejected (capacity)")
+
+    def export(self):
+        """Quantized state: dict of key/value codes, scales and zero points."""
+        qtok = self._lib.orc_unit_export(self._h, None, None, None, None, None, None)
+        D = self.D
+        kq = np.zeros((qtok, D), np.uint8)
+        ks = np.zeros((qtok // G, D), np.float32)
+        kz = np.zeros((qtok // G, D), np.float32)
+        vq = np.zeros((qtok, D), np.uint8)
+        vs = np.zeros((qtok, D // G), np.float32)
+        vz = np.zeros((qtok, D // G), np.float32)
+        self._lib.orc_unit_export(self._h, _ptr(kq), _ptr(ks), _ptr(kz), _ptr(vq),
+                             _ptr(vs), _ptr(vz))
+        return dict(qtok=qtok, kq=kq, ks=ks, kz=kz, vq=vq, vs=vs, vz=vz)
+
+    def serialize(self):
+        """(bytes u8[R], valid u8[R]) of the unit in the canonical layout."""
+        nbytes = region_bytes(self.kind, self.D, self.cap)
+        out = np.zeros(nbytes, np.uint8)
+        valid = np.zeros(nbytes, np.uint8)
+        rc = self._lib.orc_unit_serialize(self._h, _ptr(out), _ptr(valid), nbytes)
+        assert rc == 0
+        return out, valid
+
+
+@dataclasses.dataclass
+class DecodeResult:
+    out: np.ndarray      # fp64 [D]
+    lse: float           # natural log
+    mask: np.ndarray     # uint32 words over the 4-bit positions
+    nsel: int
+    slack: np.ndarray    # fp64 [D]
+    weights: np.ndarray  # fp64 softmax weight per attended position
+
+
+def decode(unit, q_bits, tau, src=None, sm_scale=0.0, band=1e-6):
+    """Decode one unit for the query ``q_bits`` (bf16 bits [D]).
+
+    ``src`` is the final loop's unit of the same layer, sequence and head when
+    ``unit`` is a SHARE unit.
+    """
+    D = unit.D
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16).reshape(D)
+    npos = unit.n
+    out = np.zeros(D, np.float64)
+    slack = np.zeros(D, np.float64)
+    weights = np.zeros(max(npos, 1), np.float64)
+    lse = np.zeros(1, np.float64)
+    mask = np.zeros(max(npos // G + 2, 1), np.uint32)
+    nw = np.zeros(1, np.int32)
+    nsel = np.zeros(1, np.int32)
+    rc = unit._lib.orc_decode(unit._h, None if src is None else src._h, _ptr(q),
+                         float(tau), float(sm_scale), float(band), _ptr(out),
+                         _ptr(lse), _ptr(mask), _ptr(nw), _ptr(nsel),
+                         _ptr(slack), _ptr(weights))
+    if rc != 0:
+        raise ValueError("oracle decode rejected its input")
+    return DecodeResult(out=out, lse=float(lse[0]), mask=mask[: nw[0]].copy(),
+                        nsel=int(nsel[0]), slack=slack, weights=weights[:npos])

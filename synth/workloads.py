@@ -1,0 +1,258 @@
+"""Seeded synthetic workloads for the LoopKV decode path (host side).
+
+A workload fixes the cell grid (loops x layers), heads, head dim, batch,
+per-sequence lengths, the per-cell storage plan and tau, and the recipe of
+every raw key, value and query.  Every value is a pure function of
+(seed, stream, counters) through Philox4x32-10 (``philox.py``), so the GPU
+twin in ``csrc/synth.cu`` produces the same bits and either side can
+regenerate any slice.  No LoopKV arithmetic lives here.
+
+Cells are indexed loop-major: cell = loop * n_layers + layer.  The final loop
+is loop n_loops - 1; a SHARE cell at (loop, layer) reuses cell
+(n_loops - 1, layer).
+
+Recipes (the shapes follow a 1.4B-parameter looped model at 4K-16K context):
+  keys    "lognormal": N(0,1) times a per-(cell, head, channel) factor
+          exp(N(0,1)); "outlier": N(0,1), with 4 channels per (cell, head)
+          scaled by 10.
+  values  N(0,1).
+  queries "sum3": the sum of the raw keys at 3 distinct random attended
+          positions plus 0.5 * N(0,1); "peaked": 2 * the raw key at one random
+          attended position plus N(0,1).  Attended positions of a SHARE unit
+          of length n are the final loop's positions [0, n-1) and its own
+          position n-1.
+N(0,1) is the Irwin-Hall stand-in of ``philox.normal_from_bits``.  Sums and
+products are fp32 round-to-nearest, then rounded once to bf16.
+"""
+
+import dataclasses
+
+import numpy as np
+
+from . import philox as px
+
+Q4, Q2, SHARE, BF16 = 0, 1, 2, 3
+KIND_NAMES = {Q4: "Q4", Q2: "Q2", SHARE: "SHARE", BF16: "BF16"}
+
+# Philox key word 1 selects the stream; key word 0 is the workload seed.
+STREAM_K, STREAM_V, STREAM_QNOISE, STREAM_QPOS = 1, 2, 3, 4
+STREAM_CHSCALE, STREAM_PLAN, STREAM_LEN, STREAM_OUTLIER = 5, 6, 7, 8
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    n_loops: int
+    n_layers: int
+    n_heads: int
+    head_dim: int
+    batch: int
+    seed: int
+    kinds: np.ndarray        # uint8 [cells], loop-major
+    tau: float
+    lengths: np.ndarray      # int32 [batch]: tokens cached per cell after the build
+    capacity: np.ndarray     # int32 [batch]
+    key_dist: str            # "lognormal" | "outlier"
+    query_mode: str          # "sum3" | "peaked"
+    chscale: np.ndarray      # float32 [cells, heads, head_dim]
+    description: str = ""
+
+    @property
+    def n_cells(self):
+        return self.n_loops * self.n_layers
+
+    def source_cell(self, cell):
+        """Cell whose KV a SHARE cell reuses: the final loop, same layer."""
+        return (self.n_loops - 1) * self.n_layers + cell % self.n_layers
+
+    def data_cell(self, cell):
+        return self.source_cell(cell) if self.kinds[cell] == SHARE else cell
+
+    def cells_of_loop(self, loop):
+        return list(range(loop * self.n_layers, (loop + 1) * self.n_layers))
+
+
+# ---------------------------------------------------------------- raw streams
+
+def _unit_word(wl, b, h):
+    return np.uint32(h + wl.n_heads * b)
+
+
+def raw_keys(wl, cell, b, h, t0, t1):
+    """bf16 bits [t1-t0, D] of the raw keys of (cell, b, h) at positions t0..t1-1."""
+    D = wl.head_dim
+    t = np.arange(t0, t1, dtype=np.uint32)[:, None]
+    d = np.arange(D, dtype=np.uint32)[None, :]
+    u = px.philox4x32(t, d, _unit_word(wl, b, h), np.uint32(cell), wl.seed, STREAM_K)
+    z = px.normal_from_bits(*u)
+    x = (z * wl.chscale[cell, h][None, :]).astype(np.float32)
+    return px.float_to_bf16_bits(x)
+
+
+def raw_values(wl, cell, b, h, t0, t1):
+    """bf16 bits [t1-t0, D] of the raw values of (cell, b, h)."""
+    D = wl.head_dim
+    t = np.arange(t0, t1, dtype=np.uint32)[:, None]
+    d = np.arange(D, dtype=np.uint32)[None, :]
+    u = px.philox4x32(t, d, _unit_word(wl, b, h), np.uint32(cell), wl.seed, STREAM_V)
+    return px.float_to_bf16_bits(px.normal_from_bits(*u))
+
+
+def query_positions(wl, cell, b, h, n):
+    """Attended positions the query of a unit of length n is built from."""
+    u = px.philox4x32(np.uint32(n), np.uint32(0), _unit_word(wl, b, h), np.uint32(cell),
+                      wl.seed, STREAM_QPOS)
+    u = [int(x) for x in u]
+    want = 3 if wl.query_mode == "sum3" else 1
+    k = min(want, n)
+    picks = []
+    for i in range(k):
+        r = int(px.uniform_index(np.uint32(u[i]), n - i))
+        for p in sorted(picks):  # skip the positions already taken
+            if r >= p:
+                r += 1
+        picks.append(r)
+    return picks
+
+
+def query(wl, cell, b, h, n):
+    """bf16 bits [D] of the query of unit (cell, b, h) when it holds n tokens."""
+    D = wl.head_dim
+    share = wl.kinds[cell] == SHARE
+    keys = []
+    for p in query_positions(wl, cell, b, h, n):
+        src = wl.source_cell(cell) if (share and p < n - 1) else cell
+        keys.append(px.bf16_bits_to_float(raw_keys(wl, src, b, h, p, p + 1)[0]))
+    d = np.arange(D, dtype=np.uint32)
+    u = px.philox4x32(np.uint32(n), d, _unit_word(wl, b, h), np.uint32(cell), wl.seed,
+                      STREAM_QNOISE)
+    z = px.normal_from_bits(*u)
+    if wl.query_mode == "sum3":
+        acc = np.zeros(D, np.float32)
+        for kv in keys:
+            acc = (acc + kv).astype(np.float32)
+        x = (acc + (np.float32(0.5) * z).astype(np.float32)).astype(np.float32)
+    else:
+        x = ((np.float32(2.0) * keys[0]).astype(np.float32) + z).astype(np.float32)
+    return px.float_to_bf16_bits(x)
+
+
+# ------------------------------------------------------------------ tables
+
+def _permutation(seed, n, purpose):
+    u = px.philox4x32(np.arange(n, dtype=np.uint32), np.uint32(purpose), 0, 0, seed,
+                      STREAM_PLAN)[0]
+    return np.argsort(u.astype(np.int64) * 4096 + np.arange(n), kind="stable")
+
+
+def percent_plan(seed, n_loops, n_layers, pct_q4, pct_share, final_all_q4=False):
+    """Seeded plan with round(pct * cells) Q4 and SHARE cells, the rest Q2.
+
+    SHARE cells are drawn from the non-final loops only.  With final_all_q4
+    the final loop is all Q4 and the percentages apply to the other loops.
+    """
+    cells = n_loops * n_layers
+    kinds = np.full(cells, Q2, np.uint8)
+    nonfinal = np.arange((n_loops - 1) * n_layers)
+    if final_all_q4:
+        kinds[(n_loops - 1) * n_layers:] = Q4
+        pool = nonfinal
+        n_share = int(round(pct_share * len(pool)))
+        n_q4 = int(round(pct_q4 * len(pool)))
+        perm = pool[_permutation(seed, len(pool), 1)]
+        kinds[perm[:n_share]] = SHARE
+        kinds[perm[n_share:n_share + n_q4]] = Q4
+        return kinds
+    n_share = int(round(pct_share * cells))
+    n_q4 = int(round(pct_q4 * cells))
+    perm = nonfinal[_permutation(seed, len(nonfinal), 1)]
+    kinds[perm[:n_share]] = SHARE
+    rest = np.array([c for c in range(cells) if kinds[c] != SHARE])
+    rest = rest[_permutation(seed, len(rest), 2)]
+    kinds[rest[:n_q4]] = Q4
+    return kinds
+
+
+def lognormal_chscale(seed, cells, H, D):
+    d = np.arange(D, dtype=np.uint32)[None, None, :]
+    h = np.arange(H, dtype=np.uint32)[None, :, None]
+    c = np.arange(cells, dtype=np.uint32)[:, None, None]
+    z = px.normal_from_bits(*px.philox4x32(d, h, c, 0, seed, STREAM_CHSCALE))
+    return np.exp(z.astype(np.float64)).astype(np.float32)
+
+
+def outlier_chscale(seed, cells, H, D, n_out=4, factor=10.0):
+    out = np.ones((cells, H, D), np.float32)
+    d = np.arange(D, dtype=np.uint32)
+    for c in range(cells):
+        for h in range(H):
+            u = px.philox4x32(d, np.uint32(h), np.uint32(c), 0, seed, STREAM_OUTLIER)[0]
+            idx = np.argsort(u.astype(np.int64) * 256 + d, kind="stable")[:n_out]
+            out[c, h, idx] = factor
+    return out
+
+
+def round_up(x, m):
+    return (np.asarray(x) + m - 1) // m * m
+
+
+# --------------------------------------------------------------- the configs
+
+def make(config, **over):
+    """Workload for config 0, 1, 2, "3a".."3d" or 4; keyword args override fields."""
+    config = str(config)
+    if config == "0":
+        # plan given as [[Q4, Q2], [SHARE, Q4]] indexed [layer][loop]
+        kinds = np.array([Q4, SHARE, Q2, Q4], np.uint8)  # loop-major
+        wl = Workload("tiny", 2, 2, 2, 64, 1, 0, kinds, 0.01,
+                      np.array([256], np.int32), np.array([256 + 64], np.int32),
+                      "lognormal", "sum3", lognormal_chscale(0, 4, 2, 64),
+                      "2 loops x 2 layers, batch 1, 2 heads, D 64, 256 tokens")
+    elif config == "1":
+        kinds = percent_plan(1, 4, 24, 0.5, 0.2)
+        wl = Workload("single-4k", 4, 24, 16, 128, 1, 1, kinds, 0.005,
+                      np.array([4096 + 17], np.int32), round_up([4096 + 17 + 64], 32).astype(np.int32),
+                      "lognormal", "sum3", lognormal_chscale(1, 96, 16, 128),
+                      "4x24 cells, 16 heads, D 128, batch 1, 4096 + 17 tokens")
+    elif config == "2" or config.startswith("3"):
+        kinds = percent_plan(2, 4, 24, 0.35, 0.30, final_all_q4=True)
+        tau = 0.002
+        name = "batched-16k"
+        if config.startswith("3"):
+            sub = config[1:]
+            if sub == "a":
+                kinds, tau = np.full(96, Q4, np.uint8), 0.0
+            elif sub == "b":
+                kinds = np.full(96, Q4, np.uint8)
+            elif sub == "c":
+                kinds = np.full(96, Q2, np.uint8)
+            elif sub == "d":
+                kinds = np.full(96, BF16, np.uint8)
+            else:
+                raise ValueError(config)
+            name = "ablation-" + sub
+        wl = Workload(name, 4, 24, 16, 128, 32, 2, kinds, tau,
+                      np.full(32, 16384, np.int32), np.full(32, 16384 + 64, np.int32),
+                      "outlier", "peaked", outlier_chscale(2, 96, 16, 128),
+                      "4x24 cells, 16 heads, D 128, batch 32, 16384 tokens")
+    elif config == "4":
+        B = 64
+        u = px.philox4x32(np.arange(B, dtype=np.uint32), 0, 0, 0, 4, STREAM_LEN)
+        ctx = 1024 + px.uniform_index(u[0], 16384 - 1024 + 1)
+        res = px.uniform_index(u[1], 32)
+        lengths = (ctx // 32 * 32 + res).astype(np.int32)
+        kinds = percent_plan(4, 4, 32, 0.40, 0.25)
+        wl = Workload("ragged-append", 4, 32, 32, 128, B, 4, kinds, 0.003, lengths,
+                      round_up(lengths + 64, 32).astype(np.int32),
+                      "lognormal", "sum3", lognormal_chscale(4, 128, 32, 128),
+                      "4x32 cells, 32 heads, D 128, batch 64, ragged 1K-16K")
+    else:
+        raise ValueError("unknown config %r" % config)
+    for k, v in over.items():
+        setattr(wl, k, v)
+    return wl
+
+
+def unit_length(wl, cell, b):
+    """Tokens a unit of this cell holds after the build (all cells alike)."""
+    return int(wl.lengths[b])

@@ -1,0 +1,383 @@
+"""Pins that tie the CPU oracle to facts outside itself.
+
+Each ``pin_*`` function raises AssertionError when the oracle disagrees with
+a hand-worked example, a closed form, brute force, or a textbook attention
+routine (``torch.nn.functional.scaled_dot_product_attention`` in fp64) on a
+special case the LoopKV decode reduces to.  ``test_oracle_pins.py`` runs them
+against the oracle; ``test_oracle_mutants.py`` runs them against copies of the
+oracle with a mistake planted, each of which must fail at least one pin.
+
+Method: "LoopKV: Loop-Aware KV Cache Compression for Serving Looped
+Transformers", section 概要; quantizer as in "KIVI: A Tuning-Free Asymmetric
+2bit Quantization for KV Cache" (keys per channel, values per token, groups
+of 32, asymmetric min/max, round half to even).
+"""
+
+import numpy as np
+import torch
+
+from oracle import oracle as orc
+from synth import philox as px
+
+G = 32
+
+
+def bf16(x):
+    return px.float_to_bf16_bits(np.asarray(x, np.float32))
+
+
+def f32(bits):
+    return px.bf16_bits_to_float(bits)
+
+
+def sdpa(q, k, v, scale):
+    """Textbook softmax attention in fp64 (library routine)."""
+    q = torch.tensor(np.asarray(q, np.float64)).view(1, 1, 1, -1)
+    k = torch.tensor(np.asarray(k, np.float64))[None, None]
+    v = torch.tensor(np.asarray(v, np.float64))[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=scale).view(-1).numpy()
+
+
+def rng_bits(seed, shape, scale=1.0):
+    """Seeded bf16 bit patterns from the shared input generator."""
+    n = int(np.prod(shape))
+    u = px.philox4x32(np.arange(n, dtype=np.uint32), 0, 0, 0, seed, 99)
+    z = px.normal_from_bits(*u).reshape(shape) * np.float32(scale)
+    return bf16(z)
+
+
+# ------------------------------------------------------------ quantizer pins
+
+def pin_quantize_q2_ties():
+    # range [0, 3] at 2 bits: scale 1, zero 0; 0.5 -> 0 and 2.5 -> 2 (ties to
+    # even), 1.5 -> 2.
+    x = np.zeros(G, np.float32)
+    x[:7] = [0.0, 3.0, 0.5, 1.5, 2.5, 1.0, 2.0]
+    code, s, z = orc.quantize_group(x, 2)
+    assert s == np.float32(1.0) and z == np.float32(0.0), (s, z)
+    assert list(code[:7]) == [0, 3, 0, 2, 2, 1, 2], code[:7]
+    assert (code[7:] == 0).all()
+
+
+def pin_quantize_q4_ties():
+    # range [0, 15] at 4 bits: scale 1; 7.5 -> 8, 8.5 -> 8, 0.25 -> 0, 14.75 -> 15
+    x = np.zeros(G, np.float32)
+    x[:16] = np.arange(16)
+    x[16:20] = [7.5, 8.5, 0.25, 14.75]
+    code, s, z = orc.quantize_group(x, 4)
+    assert s == np.float32(1.0) and z == np.float32(0.0)
+    assert list(code[:16]) == list(range(16))
+    assert list(code[16:20]) == [8, 8, 0, 15], code[16:20]
+
+
+def pin_quantize_fp32_scale():
+    # group {-1, 1, 0...} at 4 bits: scale = fl32(2/15) = 0.13333334, and
+    # (0 - (-1)) / scale = 7.4999995 in fp32, so 0 maps to code 7 (the exact
+    # ratio 7.5 would give 8): the division uses the stored fp32 scale.
+    x = np.zeros(G, np.float32)
+    x[0], x[1] = -1.0, 1.0
+    code, s, z = orc.quantize_group(x, 4)
+    assert s == np.float32(2.0) / np.float32(15.0)
+    assert z == np.float32(-1.0)
+    assert code[0] == 0 and code[1] == 15 and (code[2:] == 7).all(), code
+
+
+def pin_quantize_degenerate():
+    # constant group: scale 0, all codes 0, zero = the constant
+    x = np.full(G, 3.25, np.float32)
+    code, s, z = orc.quantize_group(x, 4)
+    assert s == 0.0 and z == np.float32(3.25) and (code == 0).all()
+    # a group of signed zeros stores a +0 zero point
+    x = np.full(G, -0.0, np.float32)
+    code, s, z = orc.quantize_group(x, 2)
+    assert s == 0.0 and (code == 0).all() and np.signbit(z) == False  # noqa: E712
+
+
+def pin_quantize_brute_force():
+    # every code is a nearest grid point of zero + scale * q, q in [0, qmax];
+    # the extremes map to 0 and qmax; reconstruction error <= scale / 2.
+    for bits in (2, 4):
+        qmax = (1 << bits) - 1
+        for seed in range(40):
+            scale_in = [0.01, 1.0, 37.0, 1e-3][seed % 4]
+            x = f32(rng_bits(1000 + seed, (G,), scale_in)) + np.float32(seed % 3)
+            code, s, z = orc.quantize_group(x, bits)
+            xd = x.astype(np.float64)
+            assert z == x.min() or (z == 0 and x.min() == 0)
+            assert abs(float(s) * qmax - (xd.max() - xd.min())) <= 4e-7 * (xd.max() - xd.min()) + 1e-30
+            grid = float(z) + float(s) * np.arange(qmax + 1)
+            err = np.abs(xd[:, None] - grid[None, :])
+            best = err.min(axis=1)
+            mine = err[np.arange(G), code.astype(int)]
+            assert (mine <= best + 1e-6 * max(float(s), 1e-30)).all(), (bits, seed)
+            assert (mine <= float(s) / 2 * (1 + 1e-6) + 1e-30).all()
+            assert code[np.argmin(x)] == 0 and code[np.argmax(x)] == qmax
+
+
+# ------------------------------------------------------- append / layout pins
+
+def pin_pack_worked_example():
+    # One 4-bit group, D = 64.  Key channel d (0..15) holds d at token 0, 0 at
+    # token 1 and 15 at token 2, so its codes over the group are d, 0, 15.
+    # Value token t holds channels 0..15 = 0..15 and channels 16..31 = 15.
+    # Codes 0..15 on channels 0..15 pack to high word 0xFFAA5500 and low word
+    # 0xE4E4E4E4 (code j in bits 2j..2j+1).
+    D = 64
+    k = np.zeros((G, D), np.float32)
+    k[0, :16] = np.arange(16)
+    k[2, :16] = 15.0
+    v = np.zeros((G, D), np.float32)
+    v[:, :16] = np.arange(16)
+    v[:, 16:32] = 15.0
+    u = orc.OracleUnit(orc.KIND_Q4, D, 64)
+    u.append(bf16(k), bf16(v))
+    out, valid = u.serialize()
+    words = out.view(np.uint32)
+    kblock = (64 // G) * 8 * D
+    vblock = (64 // G) * G * (D // 4)
+    # key planes: group 0, chunk 0, token 0, word 0
+    assert words[0] == 0xFFAA5500, hex(words[0])
+    assert words[kblock // 4] == 0xE4E4E4E4, hex(words[kblock // 4])
+    # key meta: scale[D] then zero[D]; channel 3 spans [0, 15] -> scale 1
+    meta = out[2 * kblock: 3 * kblock].view(np.float32)
+    assert meta[3] == 1.0 and meta[D + 3] == 0.0
+    # value planes: token 0 words 0 and 1
+    vh = (3 * kblock) // 4
+    vl = (3 * kblock + vblock) // 4
+    assert words[vh] == 0xFFAA5500 and words[vh + 1] == 0xFFFFFFFF
+    assert words[vl] == 0xE4E4E4E4 and words[vl + 1] == 0xFFFFFFFF
+    # value meta: (scale, zero) pairs per 32 channels of token 0
+    vm = out[3 * kblock + 2 * vblock: 3 * kblock + 2 * vblock + 16].view(np.float32)
+    assert vm[0] == 1.0 and vm[1] == 0.0
+    # one filled group: three key blocks and three value blocks of it
+    assert valid.sum() == 3 * 8 * D + 3 * G * (D // 4)
+
+
+def pin_axes():
+    # Keys are quantized per channel over tokens and values per token over
+    # channels: with every channel of token t equal to t, each key channel
+    # spans [0, 31] (scale fl32(31/15)) while each value group is constant
+    # (scale 0, zero = t).
+    D = 64
+    x = np.repeat(np.arange(G, dtype=np.float32)[:, None], D, axis=1)
+    u = orc.OracleUnit(orc.KIND_Q4, D, 64)
+    u.append(bf16(x), bf16(x))
+    st = u.export()
+    assert st["qtok"] == G
+    assert (st["ks"] == np.float32(31.0) / np.float32(15.0)).all()
+    assert (st["kz"] == 0).all()
+    assert (st["vs"] == 0).all() and (st["vz"][:, 0] == np.arange(G)).all()
+    assert (st["kq"][:, 0] == np.rint(np.arange(G) / (np.float32(31.0) / np.float32(15.0)))).all()
+
+
+def pin_flush_and_bulk():
+    # The residual flushes exactly when it holds 32 tokens, and appending one
+    # token at a time gives the same bytes as one bulk append.
+    D = 64
+    k = rng_bits(7, (100, D))
+    v = rng_bits(8, (100, D))
+    a = orc.OracleUnit(orc.KIND_Q4, D, 128)
+    for t in range(100):
+        a.append(k[t:t + 1], v[t:t + 1])
+        qtok = a.export()["qtok"]
+        assert qtok == (t + 1) // G * G, (t, qtok)
+    b = orc.OracleUnit(orc.KIND_Q4, D, 128)
+    b.append(k[:45], v[:45])
+    b.append(k[45:], v[45:])
+    assert a.n == b.n == 100
+    oa, va = a.serialize()
+    ob, vb = b.serialize()
+    assert (oa == ob).all() and (va == vb).all()
+    # capacity is enforced
+    c = orc.OracleUnit(orc.KIND_Q2, D, 64)
+    c.append(k[:64], v[:64])
+    try:
+        c.append(k[:1], v[:1])
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("capacity not enforced")
+
+
+# ------------------------------------------------------------------ decode pins
+
+def dequant_keys(st, res_k):
+    """Keys of a quantized unit as the decode must see them (stored precision)."""
+    qtok = st["qtok"]
+    g = np.arange(qtok) // G
+    kk = st["ks"][g].astype(np.float64) * st["kq"] + st["kz"][g].astype(np.float64)
+    return np.concatenate([kk, f32(res_k).astype(np.float64)]) if len(res_k) else kk
+
+
+def dequant_values(st, res_v, mode):
+    """Values: mode 'full' (all code bits), 'hi' (high plane + 1.5), 'q2'."""
+    qtok = st["qtok"]
+    D = st["vq"].shape[1]
+    s = np.repeat(st["vs"].astype(np.float64), G, axis=1)[:, :D]
+    z = np.repeat(st["vz"].astype(np.float64), G, axis=1)[:, :D]
+    c = st["vq"].astype(np.float64)
+    if mode == "hi":
+        c = 4.0 * (st["vq"] >> 2) + 1.5
+    vv = s * c + z
+    return np.concatenate([vv, f32(res_v).astype(np.float64)]) if len(res_v) else vv
+
+
+def _unit(kind, D, n, seed, cap=None, kscale=1.0):
+    k = rng_bits(seed, (n, D), kscale)
+    v = rng_bits(seed + 1, (n, D))
+    u = orc.OracleUnit(kind, D, cap or (n + 64))
+    u.append(k, v)
+    return u, k, v
+
+
+def pin_bf16_is_textbook():
+    D = 64
+    for n in (1, 5, 50):
+        u, k, v = _unit(orc.KIND_BF16, D, n, 20 + n)
+        q = rng_bits(30 + n, (D,), 2.0)
+        r = orc.decode(u, q, tau=0.01)
+        ref = sdpa(f32(q), f32(k), f32(v), 1 / np.sqrt(D))
+        assert np.abs(r.out - ref).max() < 1e-12, np.abs(r.out - ref).max()
+        assert abs(r.weights.sum() - 1.0) < 1e-12
+        assert r.nsel == 0 and len(r.mask) == 0
+
+
+def pin_tau_zero_is_full_4bit():
+    D = 64
+    n = 70  # two groups and 6 residual tokens
+    u, k, v = _unit(orc.KIND_Q4, D, n, 40)
+    st = u.export()
+    q = rng_bits(41, (D,), 2.0)
+    r = orc.decode(u, q, tau=0.0)
+    ref = sdpa(f32(q), dequant_keys(st, k[64:]), dequant_values(st, v[64:], "full"),
+               1 / np.sqrt(D))
+    assert np.abs(r.out - ref).max() < 1e-12
+    assert r.nsel == 64 and list(r.mask) == [0xFFFFFFFF, 0xFFFFFFFF]
+
+
+def pin_tau_above_one_is_high_plane():
+    D = 64
+    n = 70
+    u, k, v = _unit(orc.KIND_Q4, D, n, 42)
+    st = u.export()
+    q = rng_bits(43, (D,), 2.0)
+    r = orc.decode(u, q, tau=1.5)
+    ref = sdpa(f32(q), dequant_keys(st, k[64:]), dequant_values(st, v[64:], "hi"),
+               1 / np.sqrt(D))
+    assert np.abs(r.out - ref).max() < 1e-12
+    assert r.nsel == 0 and (r.mask == 0).all()
+
+
+def pin_q2_is_plain_dequant():
+    D = 128
+    n = 96 + 31
+    u, k, v = _unit(orc.KIND_Q2, D, n, 44)
+    st = u.export()
+    q = rng_bits(45, (D,), 2.0)
+    r = orc.decode(u, q, tau=0.0)
+    ref = sdpa(f32(q), dequant_keys(st, k[96:]), dequant_values(st, v[96:], "full"),
+               1 / np.sqrt(D))
+    assert np.abs(r.out - ref).max() < 1e-12
+    assert r.nsel == 0
+
+
+def pin_share_reads_final_loop():
+    # A SHARE unit of length n attends over the source's positions [0, n-1)
+    # as the source stores them, plus its own current token.
+    D = 64
+    for n_src, n_own in ((100, 90), (100, 101), (96, 97), (64, 40), (5, 3)):
+        src, ks_, vs_ = _unit(orc.KIND_Q4, D, n_src, 50 + n_own)
+        own = orc.OracleUnit(orc.KIND_SHARE, D, 0)
+        kown = rng_bits(60 + n_own, (n_own, D))
+        vown = rng_bits(61 + n_own, (n_own, D))
+        own.append(kown, vown)
+        assert own.n == n_own
+        st = src.export()
+        qtok = st["qtok"]
+        kk = dequant_keys(st, ks_[qtok:])[: n_own - 1]
+        vv = dequant_values(st, vs_[qtok:], "full")[: n_own - 1]
+        keys = np.concatenate([kk, f32(kown[-1:]).astype(np.float64)])
+        vals = np.concatenate([vv, f32(vown[-1:]).astype(np.float64)])
+        q = rng_bits(70 + n_own, (D,), 2.0)
+        r = orc.decode(own, q, tau=0.0, src=src)
+        ref = sdpa(f32(q), keys, vals, 1 / np.sqrt(D))
+        assert np.abs(r.out - ref).max() < 1e-12, (n_src, n_own)
+        assert r.nsel == min(n_own - 1, qtok)
+    # a SHARE unit cannot read past the source's length
+    src, _, _ = _unit(orc.KIND_Q4, D, 10, 80)
+    own = orc.OracleUnit(orc.KIND_SHARE, D, 0)
+    own.append(rng_bits(81, (12, D)), rng_bits(82, (12, D)))
+    try:
+        orc.decode(own, rng_bits(83, (D,)), tau=0.0, src=src)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("SHARE past its source accepted")
+
+
+def pin_high_plane_worked_example():
+    # 32 tokens with equal keys (key scale 0, so every weight is 1/32).  Each
+    # value token is 0 on channel 0, 15 on channel 1, 13 on channel 2 and 0
+    # elsewhere in its first 32 channels: scale 1, zero 0, channel 2 code 13 =
+    # (hi 3, lo 1).  Full precision gives 13; high plane only gives 13.5.
+    # Channel 1 (code 15 = hi 3, lo 3) reads 13.5 from the high plane alone,
+    # channel 0 (code 0) reads 1.5.
+    D = 64
+    k = np.full((G, D), 0.5, np.float32)
+    v = np.zeros((G, D), np.float32)
+    v[:, 1], v[:, 2] = 15.0, 13.0
+    u = orc.OracleUnit(orc.KIND_Q4, D, 64)
+    u.append(bf16(k), bf16(v))
+    q = bf16(np.ones(D, np.float32))
+    hi_only = orc.decode(u, q, tau=0.5)
+    full = orc.decode(u, q, tau=0.01)
+    assert abs(hi_only.out[2] - 13.5) < 1e-12 and abs(full.out[2] - 13.0) < 1e-12
+    assert abs(hi_only.out[1] - 13.5) < 1e-12 and abs(hi_only.out[0] - 1.5) < 1e-12
+    assert abs(full.out[1] - 15.0) < 1e-12 and abs(full.out[0]) < 1e-12
+    assert hi_only.nsel == 0 and full.nsel == G
+    # equal scores: lse = s + log(32) with s = sum(q * 0.5) / sqrt(D)
+    s = 0.5 * D / np.sqrt(D)
+    assert abs(full.lse - (s + np.log(G))) < 1e-12
+    assert np.allclose(full.weights, 1.0 / G, atol=1e-15)
+
+
+def pin_mask_properties():
+    # N_sel <= floor(1/tau); the selected set shrinks as tau grows; a token is
+    # selected exactly when its weight reaches tau (ties included).
+    D = 128
+    n = 32 * 20 + 7
+    u, _, _ = _unit(orc.KIND_Q4, D, n, 90, kscale=3.0)
+    q = rng_bits(91, (D,), 3.0)
+    prev = None
+    for tau in (0.0005, 0.001, 0.002, 0.005, 0.01, 0.05, 0.2):
+        r = orc.decode(u, q, tau=tau)
+        assert r.nsel <= int(np.floor(1.0 / tau) + 1e-9)
+        assert abs(r.weights.sum() - 1.0) < 1e-12
+        bits = np.unpackbits(r.mask.view(np.uint8), bitorder="little")[: n // G * G]
+        assert bits.sum() == r.nsel
+        if prev is not None:
+            assert ((bits & ~prev) == 0).all()
+        prev = bits
+    r = orc.decode(u, q, tau=0.0)
+    w = r.weights[5]
+    r2 = orc.decode(u, q, tau=float(w))
+    assert (r2.mask[0] >> 5) & 1 == 1
+
+
+ALL_PINS = [
+    pin_quantize_q2_ties,
+    pin_quantize_q4_ties,
+    pin_quantize_fp32_scale,
+    pin_quantize_degenerate,
+    pin_quantize_brute_force,
+    pin_pack_worked_example,
+    pin_axes,
+    pin_flush_and_bulk,
+    pin_bf16_is_textbook,
+    pin_tau_zero_is_full_4bit,
+    pin_tau_above_one_is_high_plane,
+    pin_q2_is_plain_dequant,
+    pin_share_reads_final_loop,
+    pin_high_plane_worked_example,
+    pin_mask_properties,
+]

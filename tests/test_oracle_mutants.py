@@ -1,0 +1,76 @@
+"""Plant one mistake at a time in a copy of the CPU oracle and check that the
+pins catch it.  Shows the pins would notice a dropped term, a wrong sign,
+index or operand, or a wrong constant.  CPU only; the planted copies are
+compiled into a temporary directory and never touch the real oracle."""
+
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+from oracle import build as obuild
+from oracle import oracle as orc
+from tests import oracle_pins
+
+# (name, text in the oracle, replacement)
+MUTANTS = [
+    ("qmax off by one", "const int qmax = (1 << bits) - 1;", "const int qmax = (1 << bits);"),
+    ("offset by max", "const float shifted = x[i] - mn;", "const float shifted = x[i] - mx;"),
+    ("truncate", "float r = std::nearbyint(ratio);", "float r = std::floor(ratio);"),
+    ("zero sign kept", "*zero = (mn == 0.0f) ? 0.0f : mn;", "*zero = mn;"),
+    ("value axis transposed", "x[e] = bf16_to_float(rv[i * D + j * kG + e]);",
+     "x[e] = bf16_to_float(rv[e * D + j * kG + i]);"),
+    ("late flush", "if (residual() == kG) flush_group();",
+     "if (residual() == kG + 1) flush_group();"),
+    ("code order reversed", "hi |= (plane_hi & 3u) << (2 * j);",
+     "hi |= (plane_hi & 3u) << (2 * (15 - j));"),
+    ("key index shifted", "for (int d = 0; d < D; ++d) acc += qd[d] * khat[d];",
+     "for (int d = 0; d < D; ++d) acc += qd[d] * khat[(d + 1) % D];"),
+    ("softmax not normalised", "p[pos] = std::exp(s[pos] - l);",
+     "p[pos] = std::exp(s[pos] - smax);"),
+    ("share reads its own slot", "n_att = own->n - 1;  // R6", "n_att = own->n;  // R6"),
+    ("high plane weight", "v = sc * (4.0 * hi + low_part) + ze;",
+     "v = sc * (2.0 * hi + low_part) + ze;"),
+    ("high-plane midpoint", "sel[pos] ? static_cast<double>(lo) : 1.5",
+     "sel[pos] ? static_cast<double>(lo) : 2.0"),
+    ("zero point dropped", "v = sc * code + ze;", "v = sc * code;"),
+    ("tie not selected", "if (p[pos] >= tau) {", "if (p[pos] > tau) {"),
+    ("sign of zero point", "static_cast<double>(data->kz[g * D + d]);",
+     "-static_cast<double>(data->kz[g * D + d]);"),
+]
+
+
+def _compile(src_text, path):
+    cpp = path + ".cpp"
+    with open(cpp, "w") as f:
+        f.write(src_text)
+    subprocess.check_call(["g++", *obuild.FLAGS, cpp, "-o", path])
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(name, old, new, monkeypatch):
+    src = open(obuild.SRC).read()
+    assert src.count(old) >= 1, "mutation site not found: %s" % name
+    mutated = src.replace(old, new, 1)
+    with tempfile.TemporaryDirectory() as tmp:
+        lib = os.path.join(tmp, "libmutant.so")
+        _compile(mutated, lib)
+        monkeypatch.setattr(orc, "_lib", None)
+        monkeypatch.setattr(obuild, "build", lambda force=False: lib)
+        failed = []
+        for pin in oracle_pins.ALL_PINS:
+            try:
+                pin()
+            except Exception as e:  # AssertionError or a rejected input
+                failed.append((pin.__name__, type(e).__name__))
+        monkeypatch.setattr(orc, "_lib", None)
+    assert failed, "planted mistake %r passed every pin" % name
+
+
+def test_real_oracle_passes_all_pins():
+    orc._lib = None
+    for pin in oracle_pins.ALL_PINS:
+        pin()
+    assert isinstance(orc._load(), ctypes.CDLL)
