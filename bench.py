@@ -1,0 +1,463 @@
+"""Benchmark of the LoopKV decode step on B200.
+
+Workload: the batched long-context decode of a 1.4B-shaped looped model
+(4 loops x 24 layers, 16 KV heads, head dim 128, batch 32, 16384 cached
+tokens per sequence; loop 3 all 4-bit, loops 0-2 35% 4-bit / 35% 2-bit /
+30% SHARE; tau 0.002; keys with 4 outlier channels at 10x, peaked queries;
+synthetic, seeded).  One step appends one new token to every cell and
+decodes every cell, in serving order (loops 0-2, then loop 3), for all 32
+sequences and 16 heads: 96 cell-steps.
+
+Prints one JSON line.  ``value`` is cell-steps/s over all ranks, timed on
+the device with CUDA events (max over ranks) with the KV cache resident in
+HBM (105 GB, far larger than L2).  ``e2e`` repeats the step through the
+public API with each step's inputs copied from pinned host memory and the
+outputs read back inside the timed region.  ``roofline`` reports the decode
+kernel's algorithmic bytes over its measured time against the measured HBM
+copy bandwidth.  ``--impl reference`` times the CPU oracle instead.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn loop×layer cell-steps/s; achieved HBM GB/s vs ~8 TB/s roofline"
+UNIT = "cell-steps/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="loopkv", choices=["loopkv", "reference"])
+    ap.add_argument("--config", default="2")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU work budget of the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mp = json.load(f)
+        return float(mp["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def per_token_head_bytes(kind, D):
+    """Bytes one quantized token of one head occupies in the planes + meta."""
+    if kind == 0:
+        return 5 * D // 4      # K_hi, K_lo, K_meta, V_hi, V_meta (V_lo counted per selection)
+    if kind == 1:
+        return 4 * D // 4      # K_hi, K_meta, V_hi, V_meta
+    return 4 * D               # bf16 key + value
+
+
+def decode_bytes(wl, cells, lens_own, lens_src, nsel_total):
+    """Algorithmic HBM bytes of one decode launch over `cells`.
+
+    Per unit: each attended position at its storage's per-token bytes (bf16
+    residual and the SHARE current token at 4D bytes), the low-plane rows of
+    the selected positions (D/4 each), the query (2D) and the output (4D).
+    """
+    D, H = wl.head_dim, wl.n_heads
+    total = 0
+    for c in cells:
+        share = wl.kinds[c] == 2
+        dk = int(wl.kinds[wl.data_cell(c)])
+        for b, n in enumerate(lens_own):
+            n_att = n - 1 if share else n
+            n_src = lens_src[b] if share else n
+            if dk == 3:
+                q, r = 0, n_att
+            else:
+                qtok = n_src // 32 * 32
+                q = min(n_att, qtok)
+                r = n_att - q
+            tok = q * per_token_head_bytes(dk, D) + r * 4 * D + (4 * D if share else 0)
+            total += H * (tok + 2 * D + 4 * D)
+    return total + nsel_total * (D // 4)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_src):
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
+    when it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_hash") != source_hash(kernel_src):
+        return None
+    return rec.get("bytes_per_full_launch")
+
+
+# --------------------------------------------------------- oracle baseline
+
+def oracle_baseline(config, seconds, seqs_global):
+    """Time the CPU oracle on a fixed sample of the workload's units.
+
+    Returns (cell-steps/s, sample description, cores).  A cell-step is B x H
+    unit decodes, so the rate is units/s divided by B * H.
+    """
+    from oracle import oracle as orc
+    from synth import workloads as W
+    wl = W.make(config)
+    n = int(wl.lengths[0])
+    rng = np.random.default_rng(0)
+    picks = []
+    for kind in (0, 1, 2):
+        cs = [c for c in range(wl.n_cells) if wl.kinds[c] == kind]
+        if cs:
+            picks.append((int(rng.choice(cs)), int(rng.integers(wl.batch)),
+                          int(rng.integers(wl.n_heads))))
+    units = []
+    for c, b, h in picks:
+        b = int(seqs_global[b])
+        kind = int(wl.kinds[c])
+        cap = int(wl.capacity[0])
+        own = orc.OracleUnit(kind, wl.head_dim, cap)
+        src = None
+        if kind == 2:
+            k = np.zeros((n + 1, wl.head_dim), np.uint16)
+            v = np.zeros_like(k)
+            k[-1] = W.raw_keys(wl, c, b, h, n, n + 1)[0]
+            v[-1] = W.raw_values(wl, c, b, h, n, n + 1)[0]
+            own.append(k, v)
+            sc = wl.source_cell(c)
+            src = orc.OracleUnit(int(wl.kinds[sc]), wl.head_dim, cap)
+            src.append(W.raw_keys(wl, sc, b, h, 0, n), W.raw_values(wl, sc, b, h, 0, n))
+            q = W.query(wl, c, b, h, n + 1)
+        else:
+            own.append(W.raw_keys(wl, c, b, h, 0, n + 1), W.raw_values(wl, c, b, h, 0, n + 1))
+            q = W.query(wl, c, b, h, n + 1)
+        units.append((own, src, q))
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        for own, src, q in units:
+            orc.decode(own, q, wl.tau, src=src)
+            done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    rate_units = done / el
+    desc = ("%d oracle decodes of %d sampled units (Q4, Q2, SHARE; %d tokens each, "
+            "%d-token contexts) in %.1f s on 1 core; cell-steps/s = units/s / (%d seqs x %d heads)"
+            % (done, len(units), n + 1, n + 1, el, wl.batch, wl.n_heads))
+    return rate_units / (wl.batch * wl.n_heads), desc, 1
+
+
+# -------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from synth import workloads as W
+    wl = W.make(args.config)
+    budget = max(1.0, min(args.cpu_seconds, 6.0))
+    vals = []
+    desc = ""
+    for _ in range(args.warmup):
+        oracle_baseline(args.config, 0.5, list(range(wl.batch)))
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        v, desc, cores = oracle_baseline(args.config, budget / max(1, args.steps) + 0.2,
+                                         list(range(wl.batch)))
+        vals.append(v)
+    wall = time.perf_counter() - t_all
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * wl.n_cells / value if value > 0 else None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "batched-16k (4x24 cells, 16 KV heads, D128, batch 32, 16384 "
+                               "tokens, tau 0.002)", "impl": "CPU oracle (fp64 C++)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": wall,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main arm
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from loop_aware_quantized_b200 import Plan, steps
+    from synth import workloads as W
+    from synth.gpu import DeviceGenerator
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+
+    wl = W.make(args.config)
+    B, H, D = wl.batch, wl.n_heads, wl.head_dim
+    # weak scaling: every rank serves its own batch of B sequences
+    seqs = list(range(rank * B, (rank + 1) * B))
+    n0 = wl.lengths[:B].astype(np.int32)
+    total_steps = args.warmup + args.steps + (0 if args.no_e2e else args.warmup + args.steps)
+    cap = np.full(B, int(n0.max()) + total_steps + 32, np.int32)
+    cap = (cap + 31) // 32 * 32
+    plan = Plan(wl.n_loops, wl.n_layers, H, D, cap, wl.kinds, wl.tau, device=dev)
+    gen = DeviceGenerator(wl, dev)
+
+    # build the cache: every token of every cell through the append kernel
+    t_build = time.perf_counter()
+    kbuf = vbuf = None
+    for c in range(wl.n_cells):
+        kbuf, vbuf = gen.kv([c], seqs, np.zeros(B, np.int32), int(n0.max()), k=kbuf, v=vbuf)
+        plan.append([c], kbuf, vbuf, n_new=n0)
+    del kbuf, vbuf
+    torch.cuda.synchronize()
+    build_s = time.perf_counter() - t_build
+    torch.cuda.empty_cache()
+
+    phase = steps.phases(wl.n_loops, wl.n_layers)
+
+    def step_inputs(s):
+        """Inputs of step s: the token at position n0 + s of every cell, and the
+        queries of units holding n0 + s + 1 tokens."""
+        q, k, v = [], [], []
+        for cells in phase:
+            kk, vv = gen.kv(list(cells), seqs, n0 + s, 1)
+            k.append(kk)
+            v.append(vv)
+            q.append(gen.queries(list(cells), seqs, np.tile(n0 + s + 1, (len(cells), 1))))
+        return q, k, v
+
+    n_dev_steps = args.warmup + args.steps
+    inputs = [step_inputs(s) for s in range(n_dev_steps)]
+    outs = [torch.empty((len(c), B, H, D), dtype=torch.float32, device=dev) for c in phase]
+    nsels = [[torch.zeros((len(c), B, H), dtype=torch.int32, device=dev) for c in phase]
+             for _ in range(args.steps)]
+    stream = torch.cuda.current_stream()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in phase] for _ in range(args.steps)]
+
+    for s in range(args.warmup):
+        q, k, v = inputs[s]
+        steps.decode_step(plan, phase, q, k, v, outs)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        q, k, v = inputs[args.warmup + i]
+        steps.decode_step(plan, phase, q, k, v, outs, nsel=nsels[i], events=ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = sum(a.elapsed_time(b) for row in ev for (a, b) in row)
+    plan.check()
+
+    # algorithmic bytes of every decode launch in the timed region
+    dec_bytes = 0
+    for i in range(args.steps):
+        s = args.warmup + i
+        for pi, cells in enumerate(phase):
+            lens_own = n0 + s + 1
+            # non-final loops decode before the final loop's append of this step
+            lens_src = n0 + s if pi == 0 else n0 + s + 1
+            dec_bytes += decode_bytes(wl, cells, lens_own, lens_src, int(nsels[i][pi].sum()))
+
+    t = torch.tensor([elapsed_ms, dec_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, dec_ms = float(t[0]), float(t[1])
+    ms_per_step = elapsed_ms / args.steps
+    value = wl.n_cells * world / (ms_per_step / 1000.0)
+    launches_per_step = 3 * len(phase)   # append + length commit + decode per phase
+
+    # ---- end to end through the API: pinned host inputs in, outputs out
+    e2e = None
+    if not args.no_e2e:
+        host_in = []
+        for s in range(args.steps):
+            q, k, v = step_inputs(n_dev_steps + s)
+            host_in.append([[x.cpu().pin_memory() for x in grp] for grp in (q, k, v)])
+        dq = [torch.empty_like(x) for x in inputs[0][0]]
+        dk = [torch.empty_like(x) for x in inputs[0][1]]
+        dv = [torch.empty_like(x) for x in inputs[0][2]]
+        host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        h2d = sum(x.numel() * x.element_size() for grp in host_in[0] for x in grp)
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(args.steps):
+            hq, hk, hv = host_in[s]
+            for dst, src in zip(dq + dk + dv, hq + hk + hv):
+                dst.copy_(src, non_blocking=True)
+            steps.decode_step(plan, phase, dq, dk, dv, outs)
+            for dst, src in zip(host_out, outs):
+                dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te[0]) / args.steps
+        e2e = {"value": wl.n_cells * world / (e2e_ms / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms}
+        plan.check()
+
+    peak, peak_kind = measured_peaks()
+    achieved = dec_bytes / (dec_ms / 1000.0) / 1e9 if dec_ms > 0 else 0.0
+    n_dec_launches = args.steps * len(phase)
+    kernel_src = [os.path.join(ROOT, "loop_aware_quantized_b200", "csrc", f)
+                  for f in ("decode.cu", "loopkv_internal.cuh")]
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": ncu_traffic(kernel_src),
+                "peak_kind": peak_kind + " copy bandwidth",
+                "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                "kernel": "loopkv decode", "bytes_per_launch": dec_bytes / n_dec_launches,
+                "ms_per_launch": dec_ms / n_dec_launches}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, cores = oracle_baseline(args.config, args.cpu_seconds, seqs)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u2/u4 codes, fp32 accumulate", "data": "synthetic",
+            "config": {"workload": "batched-16k: 4 loops x 24 layers, 16 KV heads, head dim "
+                                   "128, batch 32 per GPU, 16384 cached tokens + 1 appended "
+                                   "per step, plan loop3 Q4 / loops0-2 35% Q4 35% Q2 30% SHARE,"
+                                   " tau 0.002",
+                       "step": "append 1 token + decode, every cell, serving order",
+                       "global_batch": B * world, "seq_len": int(n0[0]),
+                       "parallelism": "dp%d (independent sequences)" % world,
+                       "l2": "inputs larger than L2 (KV cache %.1f GB)" % (plan.cache_bytes / 1e9),
+                       "build_s": build_s},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,214 @@
+/*
+ * loopkv.h - C ABI of the LoopKV decode library for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  "LoopKV: Loop-Aware KV Cache Compression for Serving
+ * Looped Transformers", section 概要 (abstract): a looped transformer keeps
+ * one KV cache per (loop, layer) cell; a plan gives every cell 4-bit storage,
+ * 2-bit storage, or reuse of the final loop's KV (SHARE); during decoding
+ * each loop reads the high 2 bits of every 4-bit value and fetches the low
+ * 2 bits only where its own attention weights need 4-bit precision; one
+ * fused kernel runs the plan.  The abstract fixes no arithmetic; this
+ * library takes these readings (the CPU oracle under oracle/ takes the same):
+ *   - asymmetric min/max quantization as in "KIVI: A Tuning-Free Asymmetric
+ *     2bit Quantization for KV Cache": keys per channel over groups of 32
+ *     tokens, values per token over groups of 32 channels, fp32 scale =
+ *     (max - min) / qmax and zero point = min, codes rounded half to even,
+ *     all in IEEE fp32 without fused multiply-add; scale 0 gives codes 0;
+ *   - a 4-bit code q is kept as two 2-bit planes, hi = q >> 2 and
+ *     lo = q & 3; reading hi alone reconstructs scale * (4*hi + 1.5) + zero;
+ *   - a value of a 4-bit cell uses hi and lo when its softmax weight
+ *     p >= tau, else hi only; keys are always read at stored precision;
+ *   - fewer than 32 recent tokens stay in a bf16 residual, quantized as a
+ *     group the moment it holds 32;
+ *   - a SHARE cell of length n attends over the final loop's stored
+ *     positions [0, n-1) (same layer, sequence and head) plus its own
+ *     current bf16 key and value;
+ *   - softmax scale 1/sqrt(head_dim) unless given; one query per KV head.
+ * LOOPKV_BF16 (raw bf16 cells) exists for ablations and checks.
+ *
+ * Terms.  cells = n_loops * n_layers, indexed loop-major (cell = loop *
+ * n_layers + layer).  A unit is one (cell, sequence, head).  Tokens of a
+ * unit are positions 0..n-1.
+ *
+ * Memory.  The caller owns every device buffer (table, cache, inputs and
+ * outputs) and every stream; the library allocates no device memory and
+ * owns only the host-side plan handle, which holds a host copy of the
+ * per-(cell, sequence) lengths.  Device pointers must be 16-byte aligned;
+ * the cache must be 256-byte aligned.  Streams are passed as `void*` and
+ * mean `cudaStream_t` (NULL = the legacy default stream).  bf16 data travel
+ * as their 16-bit patterns (`uint16_t`).
+ *
+ * Errors.  Every call returns a status.  Argument, plan and capacity errors
+ * are found on the host, from the host copy of the lengths, before anything
+ * is launched; the device state is then untouched.  A failed launch returns
+ * LOOPKV_ERR_CUDA.  Kernels never trap: an inconsistency they detect (which
+ * the host checks should make impossible) sets a bit in a status word inside
+ * the table, skips the affected unit, and is reported by loopkv_check().
+ *
+ * Asynchrony.  loopkv_append, loopkv_decode and loopkv_set_lengths only
+ * enqueue work on the given stream and return.  A plan handle must not be
+ * used from two host threads at once.
+ *
+ * Cache layout (canonical, part of the contract).  The cache is one buffer;
+ * cell c, sequence b, head h owns a region at loopkv_unit_region().  With
+ * capacity C tokens and NG = C / 32 (integer division) groups, a LOOPKV_Q4
+ * region holds, in order, each block a multiple of 128 bytes:
+ *   K_hi  [NG][D/64][32 tokens][4 words]   2-bit codes, channel 64c+16w+j of
+ *                                           the token in bits 2j..2j+1 of word w
+ *   K_lo  [NG][D/64][32][4]                 low planes, same arrangement
+ *   K_meta[NG]{scale[D], zero[D]}           fp32, per channel of the group
+ *   V_hi  [NG*32 tokens][D/16 words]        channel 16w+j in bits 2j..2j+1
+ *   V_lo  [NG*32][D/16]
+ *   V_meta[NG*32]{(scale, zero) x D/32}     fp32 pairs per 32 channels
+ *   res_K [32][D], res_V [32][D]            bf16 residual; slot r holds
+ *                                           position 32*floor(n/32) + r
+ * LOOPKV_Q2 has the same blocks without K_lo and V_lo; its "hi" planes hold
+ * the 2-bit codes.  LOOPKV_SHARE holds cur_K[D], cur_V[D] (bf16, each block
+ * rounded up to 128 bytes).  LOOPKV_BF16 holds K[C][D] then V[C][D] (bf16,
+ * each rounded up to 128 bytes).
+ */
+#ifndef LOOPKV_H_
+#define LOOPKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LOOPKV_OK = 0,
+  LOOPKV_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad cell index ... */
+  LOOPKV_ERR_PLAN = 2,        /* plan descriptor is not a valid plan */
+  LOOPKV_ERR_CAPACITY = 3,    /* an append would exceed a unit's capacity */
+  LOOPKV_ERR_UNSUPPORTED = 4, /* valid request outside what is implemented */
+  LOOPKV_ERR_CUDA = 5,        /* a CUDA call failed */
+  LOOPKV_ERR_DEVICE = 6       /* a kernel flagged an inconsistency */
+} loopkv_status;
+
+typedef enum {
+  LOOPKV_Q4 = 0,    /* 4-bit codes kept as hi and lo 2-bit planes */
+  LOOPKV_Q2 = 1,    /* 2-bit codes */
+  LOOPKV_SHARE = 2, /* reuse the final loop's KV; keeps its current token */
+  LOOPKV_BF16 = 3   /* raw bf16 (ablation / checks) */
+} loopkv_kind;
+
+/* Largest number of cells one loopkv_append / loopkv_decode call may name. */
+#define LOOPKV_MAX_CELLS_PER_CALL 256
+/* Largest batch (sequences) a plan may hold. */
+#define LOOPKV_MAX_BATCH 256
+
+typedef struct {
+  int32_t n_loops;        /* >= 1 */
+  int32_t n_layers;       /* >= 1; n_loops * n_layers <= 4096 */
+  int32_t n_kv_heads;     /* >= 1 */
+  int32_t head_dim;       /* 64 or 128 */
+  int32_t max_batch;      /* 1 .. LOOPKV_MAX_BATCH */
+  const int32_t* capacity;/* host [max_batch]: tokens each unit of sequence b
+                             can hold, 0 .. 2^20 */
+  const uint8_t* kinds;   /* host [n_loops * n_layers], loop-major,
+                             loopkv_kind values; LOOPKV_SHARE only in loops
+                             < n_loops - 1 */
+  float tau;              /* low-plane threshold on the softmax weight, >= 0 */
+  float sm_scale;         /* softmax scale; <= 0 means 1/sqrt(head_dim) */
+} loopkv_plan_desc;
+
+typedef struct {
+  size_t table_bytes; /* device plan table (cells, lengths, status word) */
+  size_t cache_bytes; /* device KV cache in the canonical layout */
+} loopkv_sizes;
+
+typedef struct loopkv_plan loopkv_plan; /* opaque host handle */
+
+/* Validate a plan and report the device memory it needs.
+ * Errors: LOOPKV_ERR_INVALID_ARG (null), LOOPKV_ERR_PLAN (bad kinds, SHARE
+ * in the final loop, head_dim not 64/128, sizes out of range). */
+loopkv_status loopkv_plan_query(const loopkv_plan_desc* desc, loopkv_sizes* sizes);
+
+/* Bind a plan to caller-allocated device memory.  Writes the plan table to
+ * d_table (table_bytes >= the queried size) on `stream` and sets every
+ * length to 0.  The cache contents need no initialisation.  The descriptor's
+ * host arrays are copied; the handle keeps the pointers d_table and d_cache,
+ * which must stay valid until loopkv_plan_free.  On success *out receives a
+ * new handle. */
+loopkv_status loopkv_plan_load(const loopkv_plan_desc* desc, void* d_table, size_t table_bytes,
+                               void* d_cache, size_t cache_bytes, void* stream,
+                               loopkv_plan** out);
+
+/* Release the host handle (device memory stays the caller's). NULL is a no-op. */
+void loopkv_plan_free(loopkv_plan* plan);
+
+/* Append tokens: the LoopKV cache update (quantize, split into bit planes,
+ * store).  For every listed cell c = h_cells[i], sequence b < batch and head
+ * h, tokens t < h_n_new[b] of
+ *     d_k, d_v: bf16 [n_cells][batch][n_kv_heads][n_new_max][head_dim]
+ * become positions len+t of the unit (len = the unit's length before the
+ * call).  Q4/Q2 cells: tokens enter the bf16 residual; each time it holds 32
+ * tokens they are quantized as one group (keys per channel, values per token
+ * per 32 channels) into the planes.  SHARE cells keep only the last appended
+ * token as their current key and value.  BF16 cells store tokens raw.
+ * Lengths grow by h_n_new[b].  h_cells: distinct cell indices; h_n_new: host
+ * [batch], each 0 .. n_new_max.
+ * Errors (nothing launched): LOOPKV_ERR_INVALID_ARG, LOOPKV_ERR_CAPACITY
+ * (len + n_new > capacity for a non-SHARE unit). */
+loopkv_status loopkv_append(loopkv_plan* plan, const int32_t* h_cells, int32_t n_cells,
+                            int32_t batch, const int32_t* h_n_new, int32_t n_new_max,
+                            const uint16_t* d_k, const uint16_t* d_v, void* stream);
+
+/* Decode attention: the fused LoopKV read of the plan.  For every listed
+ * cell c = h_cells[i], sequence b < batch and head h, with query
+ *     d_q: bf16 [n_cells][batch][n_kv_heads][head_dim]
+ * computes over the unit's attended positions (its own n tokens; for a SHARE
+ * unit of length n, the final loop's stored positions [0, n-1) and its own
+ * current token) the scores sm_scale * <q, k>, with keys dequantized at their
+ * stored precision, their softmax p, the selection p >= tau over 4-bit
+ * quantized positions, and
+ *     d_out: fp32 [n_cells][batch][n_kv_heads][head_dim] = sum_t p_t * v_t
+ * with v_t at 4-bit precision where selected, high plane only otherwise,
+ * 2-bit, or bf16 as stored.  Optional outputs (NULL to skip):
+ *     d_lse : fp32 [n_cells][batch][n_kv_heads], natural-log logsumexp
+ *     d_mask: uint32 [n_cells][batch][n_kv_heads][mask_words]; bit j of
+ *             word g = position 32g+j was selected; words
+ *             0 .. ceil(nq/32)-1 are written, nq = 4-bit positions attended
+ *     d_nsel: int32 [n_cells][batch][n_kv_heads], number of selected positions
+ * Every unit must hold n >= 1 tokens; a SHARE unit needs its source to hold
+ * at least n-1.  SHARE units read the source as it is stored when the kernel
+ * runs (decode a loop before appending to the final loop for serving order).
+ * Errors (nothing launched): LOOPKV_ERR_INVALID_ARG, LOOPKV_ERR_UNSUPPORTED
+ * (a unit longer than the kernel's limit). */
+loopkv_status loopkv_decode(loopkv_plan* plan, const int32_t* h_cells, int32_t n_cells,
+                            int32_t batch, const uint16_t* d_q, float* d_out, float* d_lse,
+                            uint32_t* d_mask, int32_t mask_words, int32_t* d_nsel,
+                            void* stream);
+
+/* Set the lengths of (cell, sequence) pairs: h_len is host [n_cells][batch]
+ * for the listed cells.  Allowed per unit: 0 (reset), or any value that
+ * keeps every stored position valid: new <= old and, for Q4/Q2 cells,
+ * new >= 32*floor(old/32) (drop residual tokens only) or new a multiple of
+ * 32 (drop whole groups); SHARE cells: new == old (only the current
+ * token is kept, so a SHARE unit can only be reset).  For rollback and reuse
+ * of sequence slots.  Errors: LOOPKV_ERR_INVALID_ARG. */
+loopkv_status loopkv_set_lengths(loopkv_plan* plan, const int32_t* h_cells, int32_t n_cells,
+                                 int32_t batch, const int32_t* h_len, void* stream);
+
+/* Host copy of the lengths: h_len receives [n_loops*n_layers][max_batch]. */
+loopkv_status loopkv_get_lengths(const loopkv_plan* plan, int32_t* h_len);
+
+/* Byte offset (from the cache base) and size of the region of unit
+ * (cell, seq, head) in the canonical layout. */
+loopkv_status loopkv_unit_region(const loopkv_plan* plan, int32_t cell, int32_t seq,
+                                 int32_t head, uint64_t* offset, uint64_t* bytes);
+
+/* Wait for `stream`, then read and clear the device status word.
+ * Returns LOOPKV_ERR_DEVICE if a kernel flagged an inconsistency. */
+loopkv_status loopkv_check(loopkv_plan* plan, void* stream);
+
+/* Static description of a status code. */
+const char* loopkv_status_string(loopkv_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOOPKV_H_ */

@@ -1,0 +1,293 @@
+// LoopKV cache append for sm_100a: quantize, split into bit planes, store.
+//
+// "LoopKV: Loop-Aware KV Cache Compression for Serving Looped Transformers",
+// section 概要: a cell keeps 4-bit storage (read as a high and a low 2-bit
+// plane), 2-bit storage, or reuses the final loop's KV.  Quantization is
+// asymmetric min/max as in "KIVI: A Tuning-Free Asymmetric 2bit
+// Quantization for KV Cache": keys per channel over a group of 32 tokens,
+// values per token over groups of 32 channels; the fp32 steps
+//   scale = (max - min) / qmax,  code = rne((x - min) / scale)
+// are done with explicit round-to-nearest intrinsics (no contraction), so the
+// codes are the ones any IEEE implementation of the same steps produces.
+//
+// One CTA per (cell, sequence, head) unit.  New tokens fill the bf16
+// residual; every 32-position group that becomes complete is quantized by
+// one warp through a padded shared-memory tile, then the remaining tokens
+// are written to the residual.  Lengths are advanced by a second, tiny
+// kernel once every head of the unit has read the old length.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "loopkv_internal.cuh"
+
+namespace loopkv {
+namespace {
+
+constexpr int kAppendThreads = 128;
+constexpr int kAppendWarps = kAppendThreads / 32;
+
+// Quantize x (fp32) of a 32-value group: returns the code, given the
+// group's min and scale.  scale == 0 gives 0.
+__device__ __forceinline__ uint32_t quant_code(float x, float mn, float scale, int qmax) {
+  if (scale == 0.0f) return 0u;
+  const float r = __fdiv_rn(__fsub_rn(x, mn), scale);
+  int c = __float2int_rn(r);  // round half to even
+  c = c < 0 ? 0 : (c > qmax ? qmax : c);
+  return (uint32_t)c;
+}
+
+// A zero range stores scale +0 whatever the signs of zero min / max.
+__device__ __forceinline__ float group_scale(float mn, float mx, int qmax) {
+  const float range = __fsub_rn(mx, mn);
+  return range == 0.0f ? 0.0f : __fdiv_rn(range, (float)qmax);
+}
+
+__device__ __forceinline__ float canon_zero(float mn) { return mn == 0.0f ? 0.0f : mn; }
+
+__device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+template <int D>
+__global__ void __launch_bounds__(kAppendThreads)
+append_kernel(const AppendParams p, const CellList cl) {
+  constexpr int TROW = D + 2;     // bf16 per padded tile row
+  constexpr int CROW = D + 16;    // bytes per padded code row
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint16_t* tk = reinterpret_cast<uint16_t*>(sm) + warp * (2 * 32 * TROW);
+  uint16_t* tv = tk + 32 * TROW;
+  uint8_t* codes = sm + kAppendWarps * (2 * 32 * TROW) * 2 + warp * (32 * CROW);
+
+  const int H = p.n_heads;
+  const int h = blockIdx.x % H;
+  const int b = (blockIdx.x / H) % p.batch;
+  const int ci = blockIdx.x / (H * p.batch);
+  const int cell = cl.cell[ci];
+  const int n_new = p.n_new[b];
+  if (n_new <= 0) return;
+
+  const TableHeader* hdr = reinterpret_cast<const TableHeader*>(p.table);
+  const DevCell* cells = reinterpret_cast<const DevCell*>(p.table + table_cells_offset());
+  const DevSeq* seqs = reinterpret_cast<const DevSeq*>(p.table + table_seqs_offset(hdr->n_cells));
+  const DevCell c = cells[cell];
+  const DevSeq s = seqs[(size_t)cell * hdr->max_batch + b];
+  const int kind = c.kind;
+  const int n_old = s.len;
+  if (n_old < 0 || (kind != LOOPKV_SHARE && n_old + n_new > s.cap)) {
+    if (threadIdx.x == 0) atomicOr(reinterpret_cast<uint32_t*>(p.table), kStatusLength);
+    return;
+  }
+  uint8_t* base = p.cache + s.offset + (size_t)h * s.stride;
+  const UnitLayout L = unit_layout(kind, D, s.cap);
+  const size_t in_off = (((size_t)ci * p.batch + b) * H + h) * (size_t)p.n_new_max * D;
+  const uint16_t* kin = p.k + in_off;
+  const uint16_t* vin = p.v + in_off;
+
+  if (kind == LOOPKV_SHARE) {
+    // keep only the last appended token as the current one
+    const uint4* ks = reinterpret_cast<const uint4*>(kin + (size_t)(n_new - 1) * D);
+    const uint4* vs = reinterpret_cast<const uint4*>(vin + (size_t)(n_new - 1) * D);
+    for (int i = threadIdx.x; i < D / 8; i += kAppendThreads) {
+      reinterpret_cast<uint4*>(base + L.cur_k)[i] = ks[i];
+      reinterpret_cast<uint4*>(base + L.cur_v)[i] = vs[i];
+    }
+    return;
+  }
+  if (kind == LOOPKV_BF16) {
+    const size_t n16 = (size_t)n_new * D / 8;
+    uint4* kd = reinterpret_cast<uint4*>(base + L.raw_k + (size_t)n_old * D * 2);
+    uint4* vd = reinterpret_cast<uint4*>(base + L.raw_v + (size_t)n_old * D * 2);
+    for (size_t i = threadIdx.x; i < n16; i += kAppendThreads) {
+      const size_t t = i / (D / 8), cc = i % (D / 8);
+      kd[i] = reinterpret_cast<const uint4*>(kin + t * D)[cc];
+      vd[i] = reinterpret_cast<const uint4*>(vin + t * D)[cc];
+    }
+    return;
+  }
+
+  const bool q4 = kind == LOOPKV_Q4;
+  const int qmax = q4 ? 15 : 3;
+  const int qtok0 = n_old / kGroup * kGroup;
+  const int n1 = n_old + n_new;
+  const int qtok1 = n1 / kGroup * kGroup;
+  const uint16_t* resk = reinterpret_cast<const uint16_t*>(base + L.res_k);
+  const uint16_t* resv = reinterpret_cast<const uint16_t*>(base + L.res_v);
+
+  for (int g = qtok0 / kGroup + warp; g < qtok1 / kGroup; g += kAppendWarps) {
+    // gather the group's 32 tokens: residual slots first, then new tokens
+    for (int i = lane; i < 32 * (D / 2); i += 32) {
+      const int t = i / (D / 2), cc = i % (D / 2);
+      const int pos = g * kGroup + t;
+      const uint32_t* ksrc;
+      const uint32_t* vsrc;
+      if (pos < n_old) {
+        ksrc = reinterpret_cast<const uint32_t*>(resk + (size_t)(pos - qtok0) * D);
+        vsrc = reinterpret_cast<const uint32_t*>(resv + (size_t)(pos - qtok0) * D);
+      } else {
+        ksrc = reinterpret_cast<const uint32_t*>(kin + (size_t)(pos - n_old) * D);
+        vsrc = reinterpret_cast<const uint32_t*>(vin + (size_t)(pos - n_old) * D);
+      }
+      reinterpret_cast<uint32_t*>(tk + t * TROW)[cc] = ksrc[cc];
+      reinterpret_cast<uint32_t*>(tv + t * TROW)[cc] = vsrc[cc];
+    }
+    __syncwarp();
+
+    // keys: per channel over the 32 tokens
+    float* kmeta = reinterpret_cast<float*>(base + L.k_meta + (size_t)g * 8 * D);
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const int d = lane + 32 * i;
+      float mn = bf16f(tk[d]), mx = mn;
+      for (int t = 1; t < 32; ++t) {
+        const float x = bf16f(tk[t * TROW + d]);
+        mn = fminf(mn, x);
+        mx = fmaxf(mx, x);
+      }
+      const float sc = group_scale(mn, mx, qmax);
+      for (int t = 0; t < 32; ++t)
+        codes[t * CROW + d] = (uint8_t)quant_code(bf16f(tk[t * TROW + d]), mn, sc, qmax);
+      kmeta[d] = sc;
+      kmeta[D + d] = canon_zero(mn);
+    }
+    __syncwarp();
+    // pack: lane = token; chunk c of 64 channels -> 4 words per plane
+#pragma unroll
+    for (int cc = 0; cc < D / 64; ++cc) {
+      uint32_t hiw[4], low[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint4 cw = *reinterpret_cast<const uint4*>(codes + lane * CROW + 64 * cc + 16 * w);
+        const uint32_t bytes[4] = {cw.x, cw.y, cw.z, cw.w};
+        uint32_t hv = 0, lv = 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t q = (bytes[j / 4] >> (8 * (j % 4))) & 0xFFu;
+          hv |= ((q4 ? (q >> 2) : q) & 3u) << (2 * j);
+          lv |= (q & 3u) << (2 * j);
+        }
+        hiw[w] = hv;
+        low[w] = lv;
+      }
+      const size_t off = (size_t)g * 8 * D + cc * 512 + lane * 16;
+      *reinterpret_cast<uint4*>(base + L.k_hi + off) = make_uint4(hiw[0], hiw[1], hiw[2], hiw[3]);
+      if (q4) *reinterpret_cast<uint4*>(base + L.k_lo + off) = make_uint4(low[0], low[1], low[2], low[3]);
+    }
+
+    // values: lane = token, per group of 32 channels
+    {
+      const int t = lane;
+      const size_t tpos = (size_t)g * kGroup + t;
+      uint32_t hiw[D / 16], low[D / 16];
+      float meta[D / 16];
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        const uint32_t* row = reinterpret_cast<const uint32_t*>(tv + t * TROW + 32 * j);
+        float mn = bf16f(tv[t * TROW + 32 * j]), mx = mn;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const uint32_t w2 = row[e];
+          const float a = __uint_as_float(w2 << 16), bb = __uint_as_float(w2 & 0xFFFF0000u);
+          mn = fminf(mn, fminf(a, bb));
+          mx = fmaxf(mx, fmaxf(a, bb));
+        }
+        const float sc = group_scale(mn, mx, qmax);
+        uint32_t hv0 = 0, lv0 = 0, hv1 = 0, lv1 = 0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const uint32_t w2 = row[e];
+          const uint32_t qa = quant_code(__uint_as_float(w2 << 16), mn, sc, qmax);
+          const uint32_t qb = quant_code(__uint_as_float(w2 & 0xFFFF0000u), mn, sc, qmax);
+          // channels 2e and 2e+1 of the group; word 0 holds channels 0..15
+          const int ja = (2 * e) % 16, jb = (2 * e + 1) % 16;
+          const uint32_t ha = (q4 ? (qa >> 2) : qa) & 3u, hb = (q4 ? (qb >> 2) : qb) & 3u;
+          if (e < 8) {
+            hv0 |= (ha << (2 * ja)) | (hb << (2 * jb));
+            lv0 |= ((qa & 3u) << (2 * ja)) | ((qb & 3u) << (2 * jb));
+          } else {
+            hv1 |= (ha << (2 * ja)) | (hb << (2 * jb));
+            lv1 |= ((qa & 3u) << (2 * ja)) | ((qb & 3u) << (2 * jb));
+          }
+        }
+        hiw[2 * j] = hv0;
+        hiw[2 * j + 1] = hv1;
+        low[2 * j] = lv0;
+        low[2 * j + 1] = lv1;
+        meta[2 * j] = sc;
+        meta[2 * j + 1] = canon_zero(mn);
+      }
+      uint4* vh = reinterpret_cast<uint4*>(base + L.v_hi + tpos * (D / 4));
+      uint4* vl = reinterpret_cast<uint4*>(base + L.v_lo + tpos * (D / 4));
+      float4* vm = reinterpret_cast<float4*>(base + L.v_meta + tpos * (D / 4));
+#pragma unroll
+      for (int i = 0; i < D / 64; ++i) {
+        vh[i] = make_uint4(hiw[4 * i], hiw[4 * i + 1], hiw[4 * i + 2], hiw[4 * i + 3]);
+        if (q4) vl[i] = make_uint4(low[4 * i], low[4 * i + 1], low[4 * i + 2], low[4 * i + 3]);
+        vm[i] = make_float4(meta[4 * i], meta[4 * i + 1], meta[4 * i + 2], meta[4 * i + 3]);
+      }
+    }
+    __syncwarp();
+  }
+  __syncthreads();  // flushed groups have read the old residual
+
+  // remaining tokens go to the residual
+  const int r_first = (qtok1 > qtok0) ? qtok1 : n_old;  // first position to write
+  uint8_t* rk = base + L.res_k;
+  uint8_t* rv = base + L.res_v;
+  const int nres = n1 - r_first;
+  for (int i = threadIdx.x; i < nres * (D / 8); i += kAppendThreads) {
+    const int t = i / (D / 8), cc = i % (D / 8);
+    const int pos = r_first + t;
+    const int slot = pos - qtok1;
+    reinterpret_cast<uint4*>(rk + (size_t)slot * D * 2)[cc] =
+        reinterpret_cast<const uint4*>(kin + (size_t)(pos - n_old) * D)[cc];
+    reinterpret_cast<uint4*>(rv + (size_t)slot * D * 2)[cc] =
+        reinterpret_cast<const uint4*>(vin + (size_t)(pos - n_old) * D)[cc];
+  }
+}
+
+__global__ void commit_lengths_kernel(uint8_t* table, const CellList cl, int n_cells, int batch,
+                                      const AppendParams p) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_cells * batch) return;
+  const int ci = i / batch, b = i % batch;
+  const TableHeader* hdr = reinterpret_cast<const TableHeader*>(table);
+  DevSeq* seqs = reinterpret_cast<DevSeq*>(table + table_seqs_offset(hdr->n_cells));
+  seqs[(size_t)cl.cell[ci] * hdr->max_batch + b].len += p.n_new[b];
+}
+
+template <int D>
+size_t append_smem() {
+  return (size_t)kAppendWarps * (2 * 32 * (D + 2) * 2 + 32 * (D + 16));
+}
+
+template <int D>
+int launch_append_t(const AppendParams& p, const CellList& cells, cudaStream_t stream) {
+  const size_t smem = append_smem<D>();
+  cudaError_t e = cudaFuncSetAttribute(append_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return (int)e;
+  const long long units = (long long)p.n_cells * p.batch * p.n_heads;
+  append_kernel<D><<<(unsigned)units, kAppendThreads, smem, stream>>>(p, cells);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_append(const AppendParams& p, const CellList& cells, void* stream, int head_dim) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (head_dim == 64) return launch_append_t<64>(p, cells, s);
+  return launch_append_t<128>(p, cells, s);
+}
+
+int launch_commit_lengths(uint8_t* table, const CellList& cells, int n_cells, int batch,
+                          const int32_t* n_new, void* stream) {
+  AppendParams p{};
+  for (int b = 0; b < batch; ++b) p.n_new[b] = n_new[b];
+  const int n = n_cells * batch;
+  commit_lengths_kernel<<<(n + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      table, cells, n_cells, batch, p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace loopkv

@@ -1,0 +1,287 @@
+"""Python binding of the LoopKV C ABI (``include/loopkv.h``).
+
+Argument marshalling only: every step of append and decode runs in the CUDA
+library ``libloopkv.so`` built in-tree for sm_100a.  PyTorch supplies device
+memory and streams.  Importing this module on a machine where the library is
+missing raises immediately; there is no other code path.
+
+Low-level functions carry the C names (``loopkv_plan_query``,
+``loopkv_append`` ...) and take raw pointers; ``Plan`` wraps a plan handle
+together with the torch tensors that hold its table and cache.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libloopkv.so")
+
+LOOPKV_Q4, LOOPKV_Q2, LOOPKV_SHARE, LOOPKV_BF16 = 0, 1, 2, 3
+LOOPKV_MAX_CELLS_PER_CALL = 256
+LOOPKV_MAX_BATCH = 256
+
+STATUS = {
+    0: "LOOPKV_OK",
+    1: "LOOPKV_ERR_INVALID_ARG",
+    2: "LOOPKV_ERR_PLAN",
+    3: "LOOPKV_ERR_CAPACITY",
+    4: "LOOPKV_ERR_UNSUPPORTED",
+    5: "LOOPKV_ERR_CUDA",
+    6: "LOOPKV_ERR_DEVICE",
+}
+
+
+class LoopKVError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s: %s (%s)" % (where, STATUS.get(status, status),
+                                          loopkv_status_string(status)))
+
+
+class loopkv_plan_desc(ctypes.Structure):
+    _fields_ = [
+        ("n_loops", ctypes.c_int32),
+        ("n_layers", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("max_batch", ctypes.c_int32),
+        ("capacity", ctypes.POINTER(ctypes.c_int32)),
+        ("kinds", ctypes.POINTER(ctypes.c_uint8)),
+        ("tau", ctypes.c_float),
+        ("sm_scale", ctypes.c_float),
+    ]
+
+
+class loopkv_sizes(ctypes.Structure):
+    _fields_ = [("table_bytes", ctypes.c_size_t), ("cache_bytes", ctypes.c_size_t)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            "libloopkv.so is missing (%s); build it with "
+            "`python loop_aware_quantized_b200/build.py`" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    I32 = ctypes.c_int32
+    st = ctypes.c_int
+    sig = {
+        "loopkv_plan_query": (st, [ctypes.POINTER(loopkv_plan_desc), ctypes.POINTER(loopkv_sizes)]),
+        "loopkv_plan_load": (st, [ctypes.POINTER(loopkv_plan_desc), P, ctypes.c_size_t, P,
+                                  ctypes.c_size_t, P, ctypes.POINTER(P)]),
+        "loopkv_plan_free": (None, [P]),
+        "loopkv_append": (st, [P, P, I32, I32, P, I32, P, P, P]),
+        "loopkv_decode": (st, [P, P, I32, I32, P, P, P, P, I32, P, P]),
+        "loopkv_set_lengths": (st, [P, P, I32, I32, P, P]),
+        "loopkv_get_lengths": (st, [P, P]),
+        "loopkv_unit_region": (st, [P, I32, I32, I32, ctypes.POINTER(ctypes.c_uint64),
+                                    ctypes.POINTER(ctypes.c_uint64)]),
+        "loopkv_check": (st, [P, P]),
+        "loopkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+# ----------------------------------------------------------- C-named calls
+
+def loopkv_status_string(status):
+    return _lib.loopkv_status_string(int(status)).decode()
+
+
+def loopkv_plan_query(desc):
+    sizes = loopkv_sizes()
+    ref = None if desc is None else ctypes.byref(desc)
+    return _lib.loopkv_plan_query(ref, ctypes.byref(sizes)), sizes
+
+
+def loopkv_plan_load(desc, d_table, table_bytes, d_cache, cache_bytes, stream):
+    handle = ctypes.c_void_p()
+    rc = _lib.loopkv_plan_load(ctypes.byref(desc), d_table, table_bytes, d_cache, cache_bytes,
+                               stream, ctypes.byref(handle))
+    return rc, handle
+
+
+def loopkv_plan_free(handle):
+    _lib.loopkv_plan_free(handle)
+
+
+def loopkv_append(handle, h_cells, n_cells, batch, h_n_new, n_new_max, d_k, d_v, stream):
+    return _lib.loopkv_append(handle, h_cells, n_cells, batch, h_n_new, n_new_max, d_k, d_v,
+                              stream)
+
+
+def loopkv_decode(handle, h_cells, n_cells, batch, d_q, d_out, d_lse, d_mask, mask_words,
+                  d_nsel, stream):
+    return _lib.loopkv_decode(handle, h_cells, n_cells, batch, d_q, d_out, d_lse, d_mask,
+                              mask_words, d_nsel, stream)
+
+
+def loopkv_set_lengths(handle, h_cells, n_cells, batch, h_len, stream):
+    return _lib.loopkv_set_lengths(handle, h_cells, n_cells, batch, h_len, stream)
+
+
+def loopkv_get_lengths(handle, h_len):
+    return _lib.loopkv_get_lengths(handle, h_len)
+
+
+def loopkv_unit_region(handle, cell, seq, head):
+    off = ctypes.c_uint64()
+    nbytes = ctypes.c_uint64()
+    rc = _lib.loopkv_unit_region(handle, cell, seq, head, ctypes.byref(off), ctypes.byref(nbytes))
+    return rc, off.value, nbytes.value
+
+
+def loopkv_check(handle, stream):
+    return _lib.loopkv_check(handle, stream)
+
+
+# ------------------------------------------------------------------ helpers
+
+def _np_ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc, where):
+    if rc != 0:
+        raise LoopKVError(rc, where)
+
+
+def make_desc(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau, sm_scale=0.0):
+    """Build a loopkv_plan_desc; returns (desc, keepalive arrays)."""
+    cap = np.ascontiguousarray(capacity, dtype=np.int32)
+    kinds = np.ascontiguousarray(kinds, dtype=np.uint8)
+    d = loopkv_plan_desc()
+    d.n_loops, d.n_layers, d.n_kv_heads, d.head_dim = n_loops, n_layers, n_kv_heads, head_dim
+    d.max_batch = int(cap.size)
+    d.capacity = cap.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    d.kinds = kinds.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+    d.tau = float(tau)
+    d.sm_scale = float(sm_scale)
+    return d, (cap, kinds)
+
+
+def query_sizes(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau=0.0):
+    """(table_bytes, cache_bytes) a plan needs; raises LoopKVError if invalid."""
+    d, keep = make_desc(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau)
+    rc, sizes = loopkv_plan_query(d)
+    _check(rc, "loopkv_plan_query")
+    return int(sizes.table_bytes), int(sizes.cache_bytes)
+
+
+class Plan:
+    """A loaded LoopKV plan with its device table and cache (torch tensors)."""
+
+    def __init__(self, n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau,
+                 sm_scale=0.0, device="cuda", stream=None):
+        import torch
+        self.n_loops, self.n_layers = n_loops, n_layers
+        self.n_cells = n_loops * n_layers
+        self.n_heads, self.head_dim = n_kv_heads, head_dim
+        self.capacity = np.ascontiguousarray(capacity, dtype=np.int32)
+        self.max_batch = int(self.capacity.size)
+        self.kinds = np.ascontiguousarray(kinds, dtype=np.uint8)
+        self.tau = float(tau)
+        d, keep = make_desc(n_loops, n_layers, n_kv_heads, head_dim, self.capacity, self.kinds,
+                            tau, sm_scale)
+        rc, sizes = loopkv_plan_query(d)
+        _check(rc, "loopkv_plan_query")
+        self.table_bytes, self.cache_bytes = int(sizes.table_bytes), int(sizes.cache_bytes)
+        self.table = torch.empty(self.table_bytes, dtype=torch.uint8, device=device)
+        self.cache = torch.empty(max(self.cache_bytes, 256), dtype=torch.uint8, device=device)
+        self._handle = None
+        rc, h = loopkv_plan_load(d, _ptr(self.table), self.table_bytes, _ptr(self.cache),
+                                 self.cache_bytes, _stream_handle(stream))
+        _check(rc, "loopkv_plan_load")
+        self._handle = h
+
+    def close(self):
+        if getattr(self, "_handle", None):
+            loopkv_plan_free(self._handle)
+            self._handle = None
+
+    def __del__(self):
+        self.close()
+
+    @property
+    def handle(self):
+        return self._handle
+
+    def source_cell(self, cell):
+        return (self.n_loops - 1) * self.n_layers + cell % self.n_layers
+
+    def append(self, cells, k, v, n_new=None, stream=None):
+        """k, v: bf16 [n_cells, batch, H, n_new_max, D] on the device."""
+        import torch
+        cells = np.ascontiguousarray(cells, dtype=np.int32)
+        assert k.dtype == torch.bfloat16 and v.dtype == torch.bfloat16
+        assert k.is_contiguous() and v.is_contiguous() and k.shape == v.shape
+        nc, batch, H, nmax, D = k.shape
+        assert nc == cells.size and H == self.n_heads and D == self.head_dim
+        if n_new is None:
+            n_new = np.full(batch, nmax, np.int32)
+        n_new = np.ascontiguousarray(n_new, dtype=np.int32)
+        rc = loopkv_append(self._handle, _np_ptr(cells), int(cells.size), int(batch),
+                           _np_ptr(n_new), int(nmax), _ptr(k), _ptr(v), _stream_handle(stream))
+        _check(rc, "loopkv_append")
+
+    def decode(self, cells, q, out=None, lse=None, mask=None, nsel=None, stream=None):
+        """q: bf16 [n_cells, batch, H, D] on the device; returns out (fp32, same shape)."""
+        import torch
+        cells = np.ascontiguousarray(cells, dtype=np.int32)
+        assert q.dtype == torch.bfloat16 and q.is_contiguous()
+        nc, batch, H, D = q.shape
+        assert nc == cells.size and H == self.n_heads and D == self.head_dim
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        mask_words = 0 if mask is None else int(mask.shape[-1])
+        rc = loopkv_decode(self._handle, _np_ptr(cells), int(cells.size), int(batch), _ptr(q),
+                           _ptr(out), _ptr(lse), _ptr(mask), mask_words, _ptr(nsel),
+                           _stream_handle(stream))
+        _check(rc, "loopkv_decode")
+        return out
+
+    def set_lengths(self, cells, lengths, stream=None):
+        cells = np.ascontiguousarray(cells, dtype=np.int32)
+        lengths = np.ascontiguousarray(lengths, dtype=np.int32)
+        batch = lengths.shape[-1]
+        rc = loopkv_set_lengths(self._handle, _np_ptr(cells), int(cells.size), int(batch),
+                                _np_ptr(lengths), _stream_handle(stream))
+        _check(rc, "loopkv_set_lengths")
+
+    def lengths(self):
+        out = np.zeros((self.n_cells, self.max_batch), np.int32)
+        _check(loopkv_get_lengths(self._handle, _np_ptr(out)), "loopkv_get_lengths")
+        return out
+
+    def unit_region(self, cell, seq, head):
+        rc, off, nbytes = loopkv_unit_region(self._handle, cell, seq, head)
+        _check(rc, "loopkv_unit_region")
+        return off, nbytes
+
+    def unit_bytes(self, cell, seq, head):
+        """Device bytes of a unit's region (a uint8 view into the cache)."""
+        off, nbytes = self.unit_region(cell, seq, head)
+        return self.cache[off:off + nbytes]
+
+    def check(self, stream=None):
+        _check(loopkv_check(self._handle, _stream_handle(stream)), "loopkv_check")

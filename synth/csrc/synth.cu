@@ -1,0 +1,174 @@
+// GPU twin of synth/philox.py and synth/workloads.py: the seeded synthetic
+// keys, values and queries, generated on the device so that inputs of
+// hundreds of GB never cross PCIe.  Same counters, same fp32 round-to-nearest
+// steps, same bf16 rounding as the host generator, hence the same bits.
+//
+// Philox4x32-10: Salmon, Moraes, Dror and Shaw, "Parallel Random Numbers: As
+// Easy as 1, 2, 3" (SC'11).  This file holds no LoopKV arithmetic.
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace {
+
+constexpr uint32_t kStreamK = 1, kStreamV = 2, kStreamQNoise = 3, kStreamQPos = 4;
+
+struct U4 {
+  uint32_t x, y, z, w;
+};
+
+__device__ __forceinline__ U4 philox(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                     uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+    const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n1 = lo1, n2 = hi0 ^ c3 ^ k1, n3 = lo0;
+    c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+  }
+  return U4{c0, c1, c2, c3};
+}
+
+// Sum of the eight 16-bit halves, centred, times the unit-variance scale.
+__device__ __forceinline__ float normal_from(U4 u, float nscale) {
+  const int s = (int)((u.x & 0xFFFFu) + (u.x >> 16) + (u.y & 0xFFFFu) + (u.y >> 16) +
+                      (u.z & 0xFFFFu) + (u.z >> 16) + (u.w & 0xFFFFu) + (u.w >> 16));
+  return __fmul_rn((float)(s - 262140), nscale);
+}
+
+__device__ __forceinline__ uint16_t to_bf16_bits(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+__device__ __forceinline__ float from_bf16_bits(uint16_t b) {
+  return __uint_as_float((uint32_t)b << 16);
+}
+
+__device__ __forceinline__ uint16_t key_bits(int cell, int b, int h, uint32_t t, int d, int H, int D,
+                                             const float* chscale, uint32_t seed, float nscale) {
+  const U4 u = philox(t, (uint32_t)d, (uint32_t)(h + H * b), (uint32_t)cell, seed, kStreamK);
+  const float z = normal_from(u, nscale);
+  return to_bf16_bits(__fmul_rn(z, chscale[((size_t)cell * H + h) * D + d]));
+}
+
+// out[c][b][h][i][d] for positions t0[b] + i, i < T.
+__global__ void gen_kv_kernel(uint16_t* __restrict__ k, uint16_t* __restrict__ v,
+                              const int32_t* __restrict__ cells, const int32_t* __restrict__ seqs,
+                              const int32_t* __restrict__ t0, int n_cells, int batch, int H, int D,
+                              int T, int table_cells, const float* __restrict__ chscale,
+                              uint32_t seed, float nscale) {
+  const size_t total = (size_t)n_cells * batch * H * T * D;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int d = (int)(i % D);
+    size_t r = i / D;
+    const int ti = (int)(r % T);
+    r /= T;
+    const int h = (int)(r % H);
+    r /= H;
+    const int bl = (int)(r % batch);
+    const int c = (int)(r / batch);
+    const int cell = cells[c], b = seqs[bl];
+    if (cell < 0 || cell >= table_cells) continue;  // host passes valid ids; never index past the table
+    const uint32_t t = (uint32_t)(t0[bl] + ti);
+    if (k) k[i] = key_bits(cell, b, h, t, d, H, D, chscale, seed, nscale);
+    if (v) {
+      const U4 u = philox(t, (uint32_t)d, (uint32_t)(h + H * b), (uint32_t)cell, seed, kStreamV);
+      v[i] = to_bf16_bits(normal_from(u, nscale));
+    }
+  }
+}
+
+// One warp per (c, b, h) query; lanes over channels.
+// mode 0: sum of raw keys at 3 distinct attended positions + 0.5 * N(0,1)
+// mode 1: 2 * raw key at one attended position + N(0,1)
+__global__ void gen_q_kernel(uint16_t* __restrict__ q, const int32_t* __restrict__ cells,
+                             const int32_t* __restrict__ srcs, const int32_t* __restrict__ seqs,
+                             const int32_t* __restrict__ lens, int n_cells, int batch, int H, int D,
+                             int mode, int table_cells, const float* __restrict__ chscale,
+                             uint32_t seed, float nscale) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_cells * batch * H) return;
+  const int h = warp % H;
+  const int bl = (warp / H) % batch;
+  const int c = warp / (H * batch);
+  const int cell = cells[c], src = srcs[c], b = seqs[bl];
+  const int n = lens[c * batch + bl];
+  if (cell < 0 || cell >= table_cells || src < 0 || src >= table_cells) return;
+  const bool share = src != cell;
+  const U4 u = philox((uint32_t)n, 0u, (uint32_t)(h + H * b), (uint32_t)cell, seed, kStreamQPos);
+  const uint32_t uu[3] = {u.x, u.y, u.z};
+  const int want = mode == 0 ? 3 : 1;
+  const int kcount = n < want ? n : want;
+  int picks[3] = {0, 0, 0};
+  for (int i = 0; i < kcount; ++i) {
+    int r = (int)(((uint64_t)uu[i] * (uint64_t)(n - i)) >> 32);
+    // skip the positions already taken, in ascending order
+    int a0 = picks[0], a1 = picks[1];
+    if (i == 2 && a1 < a0) { const int tmp = a0; a0 = a1; a1 = tmp; }
+    if (i >= 1 && r >= a0) ++r;
+    if (i >= 2 && r >= a1) ++r;
+    picks[i] = r;
+  }
+  for (int d = lane; d < D; d += 32) {
+    float key[3] = {0.f, 0.f, 0.f};
+    for (int i = 0; i < kcount; ++i) {
+      const int p = picks[i];
+      const int kc = (share && p < n - 1) ? src : cell;
+      key[i] = from_bf16_bits(key_bits(kc, b, h, (uint32_t)p, d, H, D, chscale, seed, nscale));
+    }
+    const U4 un = philox((uint32_t)n, (uint32_t)d, (uint32_t)(h + H * b), (uint32_t)cell, seed,
+                         kStreamQNoise);
+    const float z = normal_from(un, nscale);
+    float x;
+    if (mode == 0) {
+      float acc = 0.f;
+      for (int i = 0; i < kcount; ++i) acc = __fadd_rn(acc, key[i]);
+      x = __fadd_rn(acc, __fmul_rn(0.5f, z));
+    } else {
+      x = __fadd_rn(__fmul_rn(2.0f, key[0]), z);
+    }
+    q[(size_t)warp * D + d] = to_bf16_bits(x);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int synth_gen_kv(uint16_t* k, uint16_t* v, const int32_t* d_cells, const int32_t* d_seqs,
+                 const int32_t* d_t0, int n_cells, int batch, int H, int D, int T,
+                 int table_cells, const float* d_chscale, uint32_t seed, float nscale,
+                 void* stream) {
+  const size_t total = (size_t)n_cells * batch * H * T * D;
+  if (total == 0) return 0;
+  const int threads = 256;
+  size_t blocks = (total + threads - 1) / threads;
+  if (blocks > 148 * 64) blocks = 148 * 64;
+  gen_kv_kernel<<<(unsigned)blocks, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      k, v, d_cells, d_seqs, d_t0, n_cells, batch, H, D, T, table_cells, d_chscale, seed, nscale);
+  return (int)cudaGetLastError();
+}
+
+int synth_gen_q(uint16_t* q, const int32_t* d_cells, const int32_t* d_srcs, const int32_t* d_seqs,
+                const int32_t* d_lens, int n_cells, int batch, int H, int D, int mode,
+                int table_cells, const float* d_chscale, uint32_t seed, float nscale,
+                void* stream) {
+  const long long warps = (long long)n_cells * batch * H;
+  if (warps == 0) return 0;
+  const int threads = 256;
+  const long long blocks = (warps * 32 + threads - 1) / threads;
+  gen_q_kernel<<<(unsigned)blocks, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      q, d_cells, d_srcs, d_seqs, d_lens, n_cells, batch, H, D, mode, table_cells, d_chscale, seed,
+      nscale);
+  return (int)cudaGetLastError();
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+"""Device-side generation of the synthetic workloads (``csrc/synth.cu``).
+
+Produces the same bits as ``workloads.raw_keys`` / ``raw_values`` / ``query``
+on the host.  Torch provides the device buffers.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import philox as px
+from . import workloads as W
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libloopkv_synth.so")
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libloopkv_synth.so is missing; run `python synth/build.py`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        lib.synth_gen_kv.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, ctypes.c_uint32,
+                                     ctypes.c_float, P]
+        lib.synth_gen_kv.restype = I
+        lib.synth_gen_q.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, ctypes.c_uint32,
+                                    ctypes.c_float, P]
+        lib.synth_gen_q.restype = I
+        _lib = lib
+    return _lib
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+class DeviceGenerator:
+    """Generates a workload's raw keys, values and queries on a CUDA device."""
+
+    def __init__(self, wl, device="cuda"):
+        import torch
+        self.wl = wl
+        self.device = torch.device(device)
+        self.chscale = torch.from_numpy(np.ascontiguousarray(wl.chscale)).to(self.device)
+        self.nscale = float(px.NORMAL_SCALE)
+
+    def _i32(self, a):
+        import torch
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(self.device)
+
+    def kv(self, cells, seqs, t0, T, k=None, v=None, stream=None):
+        """bf16 [n_cells, len(seqs), H, T, D] keys and values at positions t0[b] + i."""
+        import torch
+        wl = self.wl
+        shape = (len(cells), len(seqs), wl.n_heads, T, wl.head_dim)
+        if k is None:
+            k = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+        if v is None:
+            v = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+        s = torch.cuda.current_stream() if stream is None else stream
+        # the index tensors must outlive the launch (a freed block is reused
+        # by the next allocation before the kernel runs)
+        d_cells, d_seqs, d_t0 = self._i32(cells), self._i32(seqs), self._i32(t0)
+        rc = _load().synth_gen_kv(_p(k), _p(v), _p(d_cells), _p(d_seqs), _p(d_t0), len(cells),
+                                  len(seqs), wl.n_heads, wl.head_dim, T, wl.n_cells,
+                                  _p(self.chscale),
+                                  wl.seed, self.nscale, ctypes.c_void_p(s.cuda_stream))
+        s.synchronize()
+        del d_cells, d_seqs, d_t0
+        assert rc == 0, rc
+        return k, v
+
+    def queries(self, cells, seqs, lens, out=None, stream=None):
+        """bf16 [n_cells, len(seqs), H, D]; lens [n_cells, len(seqs)] = unit lengths."""
+        import torch
+        wl = self.wl
+        srcs = [wl.data_cell(c) for c in cells]
+        shape = (len(cells), len(seqs), wl.n_heads, wl.head_dim)
+        if out is None:
+            out = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+        mode = 0 if wl.query_mode == "sum3" else 1
+        s = torch.cuda.current_stream() if stream is None else stream
+        d_cells, d_srcs, d_seqs = self._i32(cells), self._i32(srcs), self._i32(seqs)
+        d_lens = self._i32(np.asarray(lens).reshape(-1))
+        rc = _load().synth_gen_q(_p(out), _p(d_cells), _p(d_srcs), _p(d_seqs), _p(d_lens),
+                                 len(cells), len(seqs), wl.n_heads, wl.head_dim, mode,
+                                 wl.n_cells, _p(self.chscale), wl.seed, self.nscale,
+                                 ctypes.c_void_p(s.cuda_stream))
+        s.synchronize()
+        del d_cells, d_srcs, d_seqs, d_lens
+        assert rc == 0, rc
+        return out
+
+
+def host_kv(wl, cell, b, h, t0, t1):
+    """Host twin: (keys, values) bf16 bits [t1 - t0, D]."""
+    return W.raw_keys(wl, cell, b, h, t0, t1), W.raw_values(wl, cell, b, h, t0, t1)

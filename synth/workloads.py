@@ -256,3 +256,20 @@ def make(config, **over):
 def unit_length(wl, cell, b):
     """Tokens a unit of this cell holds after the build (all cells alike)."""
     return int(wl.lengths[b])
+
+
+def custom(n_loops, n_layers, n_heads, head_dim, kinds, lengths, capacity, tau, seed=9,
+           key_dist="lognormal", query_mode="sum3"):
+    """A small workload with an explicit plan and lengths (edge-case tests).
+
+    All arguments are plain values or tuples so the spec can be hashed and
+    sent to worker processes.
+    """
+    cells = n_loops * n_layers
+    if key_dist == "lognormal":
+        ch = lognormal_chscale(seed, cells, n_heads, head_dim)
+    else:
+        ch = outlier_chscale(seed, cells, n_heads, head_dim)
+    return Workload("custom", n_loops, n_layers, n_heads, head_dim, len(lengths), seed,
+                    np.array(kinds, np.uint8), float(tau), np.array(lengths, np.int32),
+                    np.array(capacity, np.int32), key_dist, query_mode, ch, "edge case")

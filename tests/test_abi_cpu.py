@@ -1,0 +1,122 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every function
+include/loopkv.h declares, and validates plans on the host.  No CUDA call is
+made here (plan_query, status strings and argument checks are host-only)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "loopkv.h")
+
+
+@pytest.fixture(scope="module")
+def lk():
+    from loop_aware_quantized_b200 import build
+    build.build()
+    from loop_aware_quantized_b200 import loopkv
+    return loopkv
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:loopkv_status|void|const char\*)\s+(loopkv_\w+)\s*\(",
+                                 text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("loopkv_plan_query", "loopkv_plan_load", "loopkv_plan_free",
+                     "loopkv_append", "loopkv_decode", "loopkv_set_lengths",
+                     "loopkv_check", "loopkv_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lk):
+    lib = ctypes.CDLL(lk.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lk):
+    for code in range(7):
+        assert lk.loopkv_status_string(code)
+    assert lk.loopkv_status_string(99) == "unknown status"
+
+
+def _query(lk, **kw):
+    base = dict(n_loops=2, n_layers=2, n_kv_heads=2, head_dim=64, capacity=[64, 96],
+                kinds=[0, 2, 1, 0], tau=0.01)
+    base.update(kw)
+    d, keep = lk.make_desc(base["n_loops"], base["n_layers"], base["n_kv_heads"],
+                           base["head_dim"], base["capacity"], base["kinds"], base["tau"])
+    rc, sizes = lk.loopkv_plan_query(d)
+    return rc, sizes
+
+
+def test_plan_query_rejects_invalid_plans(lk):
+    assert _query(lk)[0] == 0
+    assert _query(lk, kinds=[0, 0, 2, 0])[0] == 2          # SHARE in the final loop
+    assert _query(lk, n_loops=1, n_layers=4, kinds=[0, 2, 0, 0])[0] == 2
+    assert _query(lk, kinds=[0, 4, 1, 0])[0] == 2          # unknown kind
+    assert _query(lk, head_dim=96)[0] == 2
+    assert _query(lk, tau=-1.0)[0] == 2
+    assert _query(lk, tau=float("nan"))[0] == 2
+    assert _query(lk, capacity=[-1, 3])[0] == 2
+    assert _query(lk, capacity=[1 << 21, 3])[0] == 2
+    assert _query(lk, capacity=list(range(300)))[0] == 2   # max_batch > 256
+    rc, _ = lk.loopkv_plan_query(None)
+    assert rc == 1
+
+
+def test_plan_load_checks_arguments_before_any_device_work(lk):
+    d, keep = lk.make_desc(2, 2, 2, 64, [64, 96], [0, 2, 1, 0], 0.01)
+    rc, h = lk.loopkv_plan_load(d, None, 0, None, 0, None)
+    assert rc == 1 and not h.value
+    rc, h = lk.loopkv_plan_load(d, ctypes.c_void_p(16), 1, None, 0, None)  # table too small
+    assert rc == 1
+    rc, h = lk.loopkv_plan_load(d, ctypes.c_void_p(4096), 1 << 20, ctypes.c_void_p(4096 + 8),
+                                1 << 30, None)                           # cache misaligned
+    assert rc == 1
+
+
+def test_calls_on_a_null_plan_fail_cleanly(lk):
+    cells = np.zeros(1, np.int32)
+    n_new = np.ones(1, np.int32)
+    p = lk._np_ptr
+    assert lk.loopkv_append(None, p(cells), 1, 1, p(n_new), 1, None, None, None) == 1
+    assert lk.loopkv_decode(None, p(cells), 1, 1, None, None, None, None, 0, None, None) == 1
+    assert lk.loopkv_set_lengths(None, p(cells), 1, 1, p(n_new), None) == 1
+    assert lk.loopkv_check(None, None) == 1
+    assert lk.loopkv_unit_region(None, 0, 0, 0)[0] == 1
+    lk.loopkv_plan_free(None)
+
+
+def test_cache_size_matches_the_oracle_layout(lk):
+    """Two independent implementations of the canonical layout agree on every
+    unit's region size (library plan_query vs oracle region_bytes)."""
+    from oracle import oracle as orc
+    from synth import workloads as W
+    for config in ("0", "1", "2", "4"):
+        wl = W.make(config)
+        rc, sizes = _query(lk, n_loops=wl.n_loops, n_layers=wl.n_layers, n_kv_heads=wl.n_heads,
+                           head_dim=wl.head_dim, capacity=wl.capacity, kinds=wl.kinds,
+                           tau=wl.tau)
+        assert rc == 0
+        total = 0
+        for c in range(wl.n_cells):
+            for b in range(wl.batch):
+                total += wl.n_heads * orc.region_bytes(int(wl.kinds[c]), wl.head_dim,
+                                                       int(wl.capacity[b]))
+        assert total == sizes.cache_bytes, config
+
+
+def test_config2_cache_fits_one_b200(lk):
+    from synth import workloads as W
+    wl = W.make("2")
+    rc, sizes = _query(lk, n_loops=4, n_layers=24, n_kv_heads=16, head_dim=128,
+                       capacity=wl.capacity, kinds=wl.kinds, tau=wl.tau)
+    assert rc == 0 and sizes.cache_bytes < 120e9

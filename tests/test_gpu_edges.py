@@ -1,0 +1,161 @@
+"""Edge cases of the CUDA path against the CPU oracle (needs a B200): group
+boundaries, one-token units, SHARE over partial groups and residuals,
+token-by-token vs bulk append, rollback, tau extremes, argument errors."""
+
+import numpy as np
+import pytest
+
+from synth import workloads as W
+from tests import gpu_harness as GH
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+Q4, Q2, SH, BF = W.Q4, W.Q2, W.SHARE, W.BF16
+
+
+@pytest.fixture(scope="module")
+def pool():
+    p = P.make_pool(8)
+    yield p
+    p.terminate()
+
+
+def _spec(D, kinds, lengths, tau, n_loops=2, n_layers=2, H=2, extra=64):
+    cap = tuple(int((n + extra + 31) // 32 * 32) for n in lengths)
+    return (n_loops, n_layers, H, D, tuple(kinds), tuple(lengths), cap, tau)
+
+
+def _check_spec(spec, pool, dev, token_by_token=False, src_lengths=None):
+    """Build all cells of a custom workload, decode every unit, oracle-check all."""
+    import torch
+    from synth.gpu import DeviceGenerator
+    wl = W.custom(*spec)
+    seqs = list(range(wl.batch))
+    plan = GH.make_plan(wl, seqs)
+    gen = DeviceGenerator(wl, dev)
+    cells = list(range(wl.n_cells))
+    if token_by_token:
+        T = int(wl.lengths.max())
+        for t in range(T):
+            n_new = (wl.lengths > t).astype(np.int32)
+            k, v = gen.kv(cells, seqs, np.full(len(seqs), t, np.int32), 1)
+            plan.append(cells, k, v, n_new=n_new)
+    else:
+        GH.build_cache(wl, plan, gen, seqs, wl.lengths)
+    lens = np.tile(wl.lengths, (wl.n_cells, 1)).astype(np.int32)
+    res = GH.decode_all(wl, plan, gen, seqs, cells, lens, dev)
+    plan.check()
+    units = [(c, b, h) for c in cells for b in seqs for h in range(wl.n_heads)]
+    n_of = lambda c, b: int(wl.lengths[b])  # noqa: E731
+    GH.compare(spec, wl, plan, res, cells, seqs, units, n_of, n_of, pool)
+    torch.cuda.synchronize()
+    return plan
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_group_boundaries(pool, cuda_device, D):
+    # lengths around group edges; SHARE sources of the same length
+    lengths = (1, 2, 31, 32, 33, 63, 64, 65, 97)
+    for kinds in ((Q4, SH, Q2, Q4), (Q2, SH, Q4, Q2), (BF, SH, Q4, BF), (Q4, Q2, BF, Q4)):
+        _check_spec(_spec(D, kinds, lengths, 0.01), pool, cuda_device)
+
+
+@pytest.mark.parametrize("tau", [0.0, 0.03, 2.0])
+def test_tau_extremes(pool, cuda_device, tau):
+    _check_spec(_spec(128, (Q4, SH, Q2, Q4), (40, 300, 1000), tau), pool, cuda_device)
+
+
+def test_token_by_token_append_matches_oracle(pool, cuda_device):
+    _check_spec(_spec(64, (Q4, SH, Q2, Q4), (1, 31, 32, 70), 0.02), pool, cuda_device,
+                token_by_token=True)
+
+
+def test_share_with_longer_source(pool, cuda_device):
+    """SHARE unit shorter than its source: reads [0, n-1) of the source only,
+    across the source's quantized groups and residual."""
+    import torch
+    from synth.gpu import DeviceGenerator
+    spec = _spec(128, (SH, SH, Q4, Q2), (50, 70, 129), 0.01)
+    wl = W.custom(*spec)
+    seqs = [0, 1, 2]
+    plan = GH.make_plan(wl, seqs)
+    gen = DeviceGenerator(wl, cuda_device)
+    src_extra = np.array([7, 30, 40], np.int32)   # the final loop is ahead
+    GH.build_cache(wl, plan, gen, seqs, wl.lengths, cells=[0, 1])
+    GH.build_cache(wl, plan, gen, seqs, wl.lengths + src_extra, cells=[2, 3])
+    cells = [0, 1]
+    lens = np.tile(wl.lengths, (2, 1)).astype(np.int32)
+    res = GH.decode_all(wl, plan, gen, seqs, cells, lens, cuda_device)
+    plan.check()
+    units = [(ci, b, h) for ci in range(2) for b in seqs for h in range(wl.n_heads)]
+    own = lambda c, b: int(wl.lengths[b])  # noqa: E731
+    src = lambda c, b: int(wl.lengths[b] + src_extra[b])  # noqa: E731
+    GH.compare(spec, wl, plan, res, cells, seqs, units, own, src, pool)
+    torch.cuda.synchronize()
+
+
+def test_rollback_then_append(pool, cuda_device):
+    """set_lengths drops residual tokens or whole groups; appending again
+    rewrites those positions and the state equals a fresh build."""
+    from synth.gpu import DeviceGenerator
+    spec = _spec(64, (Q4, Q2, Q2, Q4), (45, 96, 70), 0.02)
+    wl = W.custom(*spec)
+    seqs = [0, 1, 2]
+    plan = GH.make_plan(wl, seqs)
+    gen = DeviceGenerator(wl, cuda_device)
+    cells = list(range(wl.n_cells))
+    GH.build_cache(wl, plan, gen, seqs, wl.lengths)
+    # roll back: seq0 into its residual (45 -> 40), seq1 by two groups (96 -> 32),
+    # seq2 to 0 (reset)
+    back = np.array([40, 32, 0], np.int32)
+    plan.set_lengths(cells, np.tile(back, (len(cells), 1)))
+    assert (plan.lengths()[:, :3] == back).all()
+    # re-append the same tokens
+    T = int((wl.lengths - back).max())
+    k, v = gen.kv([0], seqs, back, T)
+    for c in cells:
+        kk, vv = gen.kv([c], seqs, back, T)
+        plan.append([c], kk, vv, n_new=(wl.lengths - back).astype(np.int32))
+    lens = np.tile(wl.lengths, (wl.n_cells, 1)).astype(np.int32)
+    res = GH.decode_all(wl, plan, gen, seqs, cells, lens, cuda_device)
+    plan.check()
+    units = [(c, b, h) for c in cells for b in seqs for h in range(wl.n_heads)]
+    n_of = lambda c, b: int(wl.lengths[b])  # noqa: E731
+    GH.compare(spec, wl, plan, res, cells, seqs, units, n_of, n_of, pool)
+
+
+def test_argument_errors(cuda_device):
+    import torch
+    from loop_aware_quantized_b200 import LoopKVError
+    from synth.gpu import DeviceGenerator
+    spec = _spec(64, (Q4, SH, Q2, Q4), (40, 40), 0.01, extra=0)
+    wl = W.custom(*spec)
+    plan = GH.make_plan(wl, [0, 1])
+    gen = DeviceGenerator(wl, cuda_device)
+    k, v = gen.kv([0], [0, 1], np.zeros(2, np.int32), 40)
+    plan.append([0], k, v)
+    # capacity: 40 + 40 > 64
+    with pytest.raises(LoopKVError) as e:
+        plan.append([0], k, v)
+    assert e.value.status == 3
+    assert (plan.lengths()[0, :2] == 40).all()
+    # duplicate / out-of-range cells
+    with pytest.raises(LoopKVError):
+        plan.append([0, 0], torch.cat([k, k]), torch.cat([v, v]))
+    with pytest.raises(LoopKVError):
+        plan.decode([7], torch.zeros((1, 2, 2, 64), dtype=torch.bfloat16, device=cuda_device))
+    # decoding an empty unit is rejected
+    with pytest.raises(LoopKVError):
+        plan.decode([2], torch.zeros((1, 2, 2, 64), dtype=torch.bfloat16, device=cuda_device))
+    # SHARE unit longer than its source + 1 is rejected (cell 3 is empty)
+    plan.append([1], k, v)
+    with pytest.raises(LoopKVError):
+        plan.decode([1], torch.zeros((1, 2, 2, 64), dtype=torch.bfloat16, device=cuda_device))
+    # rollback rules: SHARE cannot be shortened
+    with pytest.raises(LoopKVError):
+        plan.set_lengths([1], np.array([[39, 40]], np.int32))
+    # empty append is a no-op
+    plan.append([0], k, v, n_new=np.zeros(2, np.int32))
+    assert (plan.lengths()[0, :2] == 40).all()
+    plan.check()
