@@ -48,6 +48,9 @@ def parse():
                     help="CPU work budget of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="sequences per GPU (default: the workload's batch); smaller "
+                         "batches are for profiling captures only")
     return ap.parse_args()
 
 
@@ -84,8 +87,9 @@ def decode_bytes(wl, cells, lens_own, lens_src, nsel_total):
         share = wl.kinds[c] == 2
         dk = int(wl.kinds[wl.data_cell(c)])
         for b, n in enumerate(lens_own):
+            n = int(n)
             n_att = n - 1 if share else n
-            n_src = lens_src[b] if share else n
+            n_src = int(lens_src[b]) if share else n
             if dk == 3:
                 q, r = 0, n_att
             else:
@@ -94,7 +98,7 @@ def decode_bytes(wl, cells, lens_own, lens_src, nsel_total):
                 r = n_att - q
             tok = q * per_token_head_bytes(dk, D) + r * 4 * D + (4 * D if share else 0)
             total += H * (tok + 2 * D + 4 * D)
-    return total + nsel_total * (D // 4)
+    return int(total) + int(nsel_total) * (D // 4)
 
 
 class ClockSampler:
@@ -151,6 +155,22 @@ class ClockSampler:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def shard_sequences(rank, batch):
+    """Global sequence ids a rank serves: weak scaling, `batch` sequences per
+    rank, disjoint across ranks (so every rank decodes different data)."""
+    return list(range(rank * batch, (rank + 1) * batch))
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise max of a list of floats over all ranks (timing)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
 
 
 def source_hash(paths):
@@ -292,9 +312,13 @@ def main():
                                 device_id=dev)
 
     wl = W.make(args.config)
+    if args.batch:
+        wl.batch = args.batch
+        wl.lengths = wl.lengths[:args.batch]
+        wl.capacity = wl.capacity[:args.batch]
     B, H, D = wl.batch, wl.n_heads, wl.head_dim
     # weak scaling: every rank serves its own batch of B sequences
-    seqs = list(range(rank * B, (rank + 1) * B))
+    seqs = shard_sequences(rank, B)
     n0 = wl.lengths[:B].astype(np.int32)
     total_steps = args.warmup + args.steps + (0 if args.no_e2e else args.warmup + args.steps)
     cap = np.full(B, int(n0.max()) + total_steps + 32, np.int32)
@@ -370,10 +394,7 @@ def main():
             lens_src = n0 + s if pi == 0 else n0 + s + 1
             dec_bytes += decode_bytes(wl, cells, lens_own, lens_src, int(nsels[i][pi].sum()))
 
-    t = torch.tensor([elapsed_ms, dec_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, dec_ms = float(t[0]), float(t[1])
+    elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], world, dev)
     ms_per_step = elapsed_ms / args.steps
     value = wl.n_cells * world / (ms_per_step / 1000.0)
     launches_per_step = 3 * len(phase)   # append + length commit + decode per phase
@@ -406,10 +427,7 @@ def main():
                 dst.copy_(src, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te[0]) / args.steps
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0] / args.steps
         e2e = {"value": wl.n_cells * world / (e2e_ms / 1000.0), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms}
@@ -439,9 +457,9 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "u2/u4 codes, fp32 accumulate", "data": "synthetic",
             "config": {"workload": "batched-16k: 4 loops x 24 layers, 16 KV heads, head dim "
-                                   "128, batch 32 per GPU, 16384 cached tokens + 1 appended "
-                                   "per step, plan loop3 Q4 / loops0-2 35% Q4 35% Q2 30% SHARE,"
-                                   " tau 0.002",
+                                   "128, batch %d per GPU, 16384 cached tokens + 1 appended "
+                                   "per step, plan loop3 Q4 / loops0-2 35%% Q4 35%% Q2 30%% "
+                                   "SHARE, tau 0.002" % B,
                        "step": "append 1 token + decode, every cell, serving order",
                        "global_batch": B * world, "seq_len": int(n0[0]),
                        "parallelism": "dp%d (independent sequences)" % world,

@@ -65,9 +65,79 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return r;
 }
 
-// Small integer (0..15) as float: exponent trick, exact.
-__device__ __forceinline__ float code_f(uint32_t c) {
-  return __uint_as_float(0x4B000000u | c) - 8388608.0f;
+// Packed fp32 pair arithmetic (sm_100): one instruction for two lanes of
+// work.  Round to nearest, no flush to zero.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("add.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<unsigned long long&>(d))
+      : "l"(reinterpret_cast<unsigned long long&>(a)),
+        "l"(reinterpret_cast<unsigned long long&>(b)));
+  return d;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(reinterpret_cast<unsigned long long&>(d))
+      : "l"(reinterpret_cast<unsigned long long&>(a)),
+        "l"(reinterpret_cast<unsigned long long&>(b)),
+        "l"(reinterpret_cast<unsigned long long&>(c)));
+  return d;
+}
+
+// A code field of `bits` bits at bit offset `off` (off + bits <= 23) of w,
+// as the exact float 2^(23-off) + code: the field becomes the low mantissa
+// bits of a float whose exponent makes one mantissa step worth 1.  A single
+// logic op; subtracting 2^(23-off) afterwards leaves the code exactly.
+template <int off, int bits>
+__device__ __forceinline__ float code_plus_pow2(uint32_t w) {
+  static_assert(off + bits <= 23, "field must stay inside the mantissa");
+  constexpr uint32_t mask = ((1u << bits) - 1u) << off;
+  constexpr uint32_t expo = (uint32_t)(150 - off) << 23;
+  return __uint_as_float((w & mask) | expo);
+}
+template <int off>
+__device__ __forceinline__ constexpr float pow2_of() {
+  return (float)(1u << (23 - off));
+}
+
+// 16 two-bit codes of w (code j in bits 2j..2j+1) -> 8 pairs (code 2i,
+// code 2i+1) as floats, exactly.
+__device__ __forceinline__ void codes2_to_pairs(uint32_t w, float2 (&out)[8]) {
+  const uint32_t y = w >> 12;  // codes 6..15 move to fields 0..9 (bits <= 19)
+#define LKV_PAIR(i, src_a, off_a, src_b, off_b)                                          \
+  out[i] = add2(make_float2(code_plus_pow2<off_a, 2>(src_a), code_plus_pow2<off_b, 2>(src_b)), \
+                make_float2(-pow2_of<off_a>(), -pow2_of<off_b>()));
+  LKV_PAIR(0, w, 0, w, 2)
+  LKV_PAIR(1, w, 4, w, 6)
+  LKV_PAIR(2, w, 8, w, 10)
+  LKV_PAIR(3, y, 0, y, 2)      // codes 6, 7
+  LKV_PAIR(4, y, 4, y, 6)      // codes 8, 9
+  LKV_PAIR(5, y, 8, y, 10)     // codes 10, 11
+  LKV_PAIR(6, y, 12, y, 14)    // codes 12, 13
+  LKV_PAIR(7, y, 16, y, 18)    // codes 14, 15
+#undef LKV_PAIR
+}
+
+// Hi and lo planes of 16 four-bit codes -> 8 pairs (q_2i, q_2i+1), q = 4hi+lo.
+// Bitwise merge into two words of nibbles: even codes (nibble m = code 2m)
+// and odd codes (nibble m = code 2m+1).
+__device__ __forceinline__ void codes4_to_pairs(uint32_t hi, uint32_t lo, float2 (&out)[8]) {
+  const uint32_t even = ((hi << 2) & 0xCCCCCCCCu) | (lo & 0x33333333u);
+  const uint32_t odd = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
+  const uint32_t even_h = even >> 12, odd_h = odd >> 12;  // nibbles 3..7 -> 0..4
+#define LKV_NIB(i, e, o, off)                                                    \
+  out[i] = add2(make_float2(code_plus_pow2<off, 4>(e), code_plus_pow2<off, 4>(o)), \
+                make_float2(-pow2_of<off>(), -pow2_of<off>()));
+  LKV_NIB(0, even, odd, 0)
+  LKV_NIB(1, even, odd, 4)
+  LKV_NIB(2, even, odd, 8)
+  LKV_NIB(3, even_h, odd_h, 0)
+  LKV_NIB(4, even_h, odd_h, 4)
+  LKV_NIB(5, even_h, odd_h, 8)
+  LKV_NIB(6, even_h, odd_h, 12)
+  LKV_NIB(7, even_h, odd_h, 16)
+#undef LKV_NIB
 }
 
 struct Unit {
@@ -147,41 +217,135 @@ __device__ __forceinline__ float dot_bf16(const uint8_t* row, const float* q_s) 
 }
 
 // Score of one quantized token: sum_d qs_d * code_d over the token's packed
-// planes (K_hi[g][chunk][token][4 words], same for K_lo).
+// planes (16-byte rows h[c], l[c] of K_hi / K_lo for chunk c of 64 channels).
 template <int D, bool Q4>
-__device__ __forceinline__ float dot_codes(const uint8_t* khi, const uint8_t* klo,
-                                           const float* qs) {
-  float acc = 0.f;
+__device__ __forceinline__ float dot_codes(const uint4 (&h)[D / 64], const uint4 (&l)[D / 64],
+                                           const float2* qs2) {
+  float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < D / 64; ++c) {
-    const uint4 h = ld_stream(khi + c * 512);
-    uint4 l = make_uint4(0, 0, 0, 0);
-    if (Q4) l = ld_stream(klo + c * 512);
-    const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
-    const uint32_t lw[4] = {l.x, l.y, l.z, l.w};
+    const uint32_t hw[4] = {h[c].x, h[c].y, h[c].z, h[c].w};
+    const uint32_t lw[4] = {l[c].x, l[c].y, l[c].z, l[c].w};
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
+      float2 v[8];
+      if (Q4) codes4_to_pairs(hw[w], lw[w], v);
+      else codes2_to_pairs(hw[w], v);
+      const float4* q4p = reinterpret_cast<const float4*>(qs2 + 32 * c + 8 * w);
 #pragma unroll
-      for (int j4 = 0; j4 < 4; ++j4) {
-        const float4 s = *reinterpret_cast<const float4*>(qs + 64 * c + 16 * w + 4 * j4);
-        const float sv[4] = {s.x, s.y, s.z, s.w};
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int j = 4 * j4 + jj;
-          uint32_t code = (hw[w] >> (2 * j)) & 3u;
-          if (Q4) code = (code << 2) | ((lw[w] >> (2 * j)) & 3u);
-          acc = fmaf(sv[jj], code_f(code), acc);
-        }
+      for (int i = 0; i < 4; ++i) {
+        const float4 qq = q4p[i];
+        acc = fma2(make_float2(qq.x, qq.y), v[2 * i], acc);
+        acc = fma2(make_float2(qq.z, qq.w), v[2 * i + 1], acc);
       }
     }
   }
-  return acc;
+  return acc.x + acc.y;
+}
+
+// Per-lane load of one 32-token key group: the lane's token rows of the
+// planes and the lane's D/32 channels of the group's scale / zero point.
+template <int D>
+struct KGroup {
+  uint4 h[D / 64], l[D / 64];
+  float sc[D / 32], zr[D / 32];
+};
+
+template <int D, bool Q4>
+__device__ __forceinline__ void load_kgroup(KGroup<D>& g, const uint8_t* data, const UnitLayout& L,
+                                            int bk, int lane) {
+  const size_t goff = (size_t)bk * 8 * D;
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) {
+    g.h[c] = ld_stream(data + L.k_hi + goff + c * 512 + lane * 16);
+    g.l[c] = Q4 ? ld_stream(data + L.k_lo + goff + c * 512 + lane * 16) : make_uint4(0, 0, 0, 0);
+  }
+  const float* meta = reinterpret_cast<const float*>(data + L.k_meta + goff);
+  if constexpr (D == 128) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(meta) + lane);
+    const float4 z = __ldg(reinterpret_cast<const float4*>(meta + D) + lane);
+    g.sc[0] = a.x; g.sc[1] = a.y; g.sc[2] = a.z; g.sc[3] = a.w;
+    g.zr[0] = z.x; g.zr[1] = z.y; g.zr[2] = z.z; g.zr[3] = z.w;
+  } else {
+    const float2 a = __ldg(reinterpret_cast<const float2*>(meta) + lane);
+    const float2 z = __ldg(reinterpret_cast<const float2*>(meta + D) + lane);
+    g.sc[0] = a.x; g.sc[1] = a.y;
+    g.zr[0] = z.x; g.zr[1] = z.y;
+  }
+}
+
+// Pass 1 over the CTA's quantized key groups [b_begin, b_end), warp-strided,
+// with the next group's loads in flight while the current one is scored.
+template <int D, bool Q4>
+__device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end, int p0, int p1,
+                                          const float* q_s, float* qs, float* sc, float sscale,
+                                          int warp, int lane) {
+  constexpr int CPL = D / 32;  // channels per lane for the q fold
+  float lmax = -INFINITY;
+  int bk = b_begin + warp;
+  if (bk >= b_end) return lmax;
+  float qv[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) qv[i] = q_s[CPL * lane + i];
+  KGroup<D> cur, nxt;
+  load_kgroup<D, Q4>(cur, u.data, u.Ld, bk, lane);
+  for (; bk < b_end; bk += kWarps) {
+    const bool more = bk + kWarps < b_end;
+    if (more) load_kgroup<D, Q4>(nxt, u.data, u.Ld, bk + kWarps, lane);
+    // fold q into the group's key scale / zero point
+    float cpart = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      qs[CPL * lane + i] = qv[i] * cur.sc[i];
+      cpart = fmaf(qv[i], cur.zr[i], cpart);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o);
+    __syncwarp();
+    const int pos = bk * 32 + lane;
+    if (pos < u.nq && pos < p1) {
+      const float dot = dot_codes<D, Q4>(cur.h, cur.l, reinterpret_cast<const float2*>(qs));
+      const float s = (dot + cpart) * sscale;
+      sc[pos - p0] = s;
+      lmax = fmaxf(lmax, s);
+    }
+    __syncwarp();
+    if (more) cur = nxt;
+  }
+  return lmax;
+}
+
+// Value accumulation of one quantized token half-row (64 channels): acc +=
+// (m * p * scale_j) * code for the lane's two 32-channel groups.
+__device__ __forceinline__ void value_codes(float2 (&acc)[32], const uint4 hw4, float a0, float a1) {
+  const uint32_t hw[4] = {hw4.x, hw4.y, hw4.z, hw4.w};
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    float2 v[8];
+    codes2_to_pairs(hw[w], v);
+    const float a = (w < 2) ? a0 : a1;
+    const float2 aa = make_float2(a, a);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[8 * w + i] = fma2(aa, v[i], acc[8 * w + i]);
+  }
+}
+
+__device__ __forceinline__ void value_raw(float2 (&acc)[32], const uint8_t* row, float pt) {
+  const float2 pp = make_float2(pt, pt);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 w = ldg128(row + c * 16);
+    acc[4 * c + 0] = fma2(pp, make_float2(bf16_lo(w.x), bf16_hi(w.x)), acc[4 * c + 0]);
+    acc[4 * c + 1] = fma2(pp, make_float2(bf16_lo(w.y), bf16_hi(w.y)), acc[4 * c + 1]);
+    acc[4 * c + 2] = fma2(pp, make_float2(bf16_lo(w.z), bf16_hi(w.z)), acc[4 * c + 2]);
+    acc[4 * c + 3] = fma2(pp, make_float2(bf16_lo(w.w), bf16_hi(w.w)), acc[4 * c + 3]);
+  }
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p, const CellList cl) {
-  constexpr int LPT = D / 64;       // lanes per token in pass 2
+  constexpr int LPT = D / 64;       // lanes per token in pass 2 (64 channels per lane)
   constexpr int TPI = 32 / LPT;     // tokens per warp iteration in pass 2
   extern __shared__ __align__(16) float smem[];
   float* q_s = smem;                                  // [D]
@@ -189,7 +353,9 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   float* red = qs_all + kWarps * D;                   // [kWarps][D]
   float* o_s = red + kWarps * D;                      // [D]
   float* misc = o_s + D;                              // [64]
-  float* sc = misc + 64;                              // [slots]
+  int* lst = reinterpret_cast<int*>(misc + 64);       // [kWarps][32]
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(lst + kWarps * 32);  // [slots / 32]
+  float* sc = reinterpret_cast<float*>(mask_s + p.slots / 32);        // [slots]
 
   const int split = p.split;
   const int rank = blockIdx.x % split;
@@ -228,43 +394,20 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   const bool q4 = u.data_kind == LOOPKV_Q4;
   float* qs = qs_all + warp * D;
   const float sscale = p.score_scale;
+  const int blk0 = p0 / 32;
+  const int blk1 = (p1 + 31) / 32;
+  const int nqb = quant ? (u.nq + 31) / 32 : 0;     // blocks holding quantized positions
+  const int qend = min(blk1, nqb);
 
   // ------------------------------------------------------------- pass 1
   float lmax = -INFINITY;
-  const int blk0 = p0 / 32;
-  const int blk1 = (p1 + 31) / 32;
-  for (int bk = blk0 + warp; bk < blk1; bk += kWarps) {
-    const int pos = bk * 32 + lane;
-    const bool active = pos < p1;
-    float s = -INFINITY;
-    if (quant && bk * 32 < u.nq) {
-      // fold q with the group's key scale / zero point
-      const uint8_t* meta = u.data + u.Ld.k_meta + (size_t)bk * 8 * D;
-      float cpart = 0.f;
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i) {
-        const int d = lane + 32 * i;
-        const float sc_d = __ldg(reinterpret_cast<const float*>(meta) + d);
-        const float z_d = __ldg(reinterpret_cast<const float*>(meta) + D + d);
-        qs[d] = q_s[d] * sc_d;
-        cpart = fmaf(q_s[d], z_d, cpart);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o);
-      __syncwarp();
-      if (active && pos < u.nq) {
-        const uint8_t* khi = u.data + u.Ld.k_hi + (size_t)bk * 8 * D + lane * 16;
-        const uint8_t* klo = u.data + u.Ld.k_lo + (size_t)bk * 8 * D + lane * 16;
-        const float dot = q4 ? dot_codes<D, true>(khi, klo, qs) : dot_codes<D, false>(khi, klo, qs);
-        s = (dot + cpart) * sscale;
-      }
-      __syncwarp();
-    }
-    if (active && pos >= u.nq) s = dot_bf16<D>(raw_row(u, pos, D, false), q_s) * sscale;
-    if (active) {
-      sc[pos - p0] = s;
-      lmax = fmaxf(lmax, s);
-    }
+  if (q4) lmax = key_pass<D, true>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, warp, lane);
+  else if (quant) lmax = key_pass<D, false>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, warp, lane);
+  // bf16 positions: residual, raw cells, the SHARE current token
+  for (int pos = max(p0, u.nq) + 32 * warp + lane; pos < p1; pos += 32 * kWarps) {
+    const float s = dot_bf16<D>(raw_row(u, pos, D, false), q_s) * sscale;
+    sc[pos - p0] = s;
+    lmax = fmaxf(lmax, s);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
@@ -298,10 +441,7 @@ decode_kernel(const DecodeParams p, const CellList cl) {
     if (tid == 0) { misc[16] = m_r; misc[17] = l_r; }
     cluster.sync();
     M = -INFINITY;
-    for (int r = 0; r < split; ++r) {
-      const float* rm = cluster.map_shared_rank(misc, r);
-      M = fmaxf(M, rm[16]);
-    }
+    for (int r = 0; r < split; ++r) M = fmaxf(M, cluster.map_shared_rank(misc, r)[16]);
     L = 0.f;
     for (int r = 0; r < split; ++r) {
       const float* rm = cluster.map_shared_rank(misc, r);
@@ -312,91 +452,97 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   const float tau = p.tau;
 
   // ------------------------------------------------------------- pass 2
-  float acc[64];
+  float2 acc[32];
 #pragma unroll
-  for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+  for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.f, 0.f);
   float g0 = 0.f, g1 = 0.f;  // per-group constants of the lane's two 32-channel groups
   int nsel = 0;
   const int hf = lane % LPT;
   const size_t vrow = D / 4;  // bytes per token of a value plane / value meta
+  const float hmul = q4 ? 4.f : 1.f;
+  const int qlim = min(p1, u.nq);
   for (int bk = blk0 + warp; bk < blk1; bk += kWarps) {
     const int pos = bk * 32 + lane;
     const bool active = pos < p1;
     const float pw = active ? sc[pos - p0] * f : 0.f;
-    const bool sel = q4 && active && pos < u.nq && pw >= tau;
+    const bool sel = q4 && pos < qlim && pw >= tau;
     const uint32_t ballot = __ballot_sync(0xffffffffu, sel);
     nsel += __popc(ballot);
-    if (p.mask != nullptr && lane == 0 && bk * 32 < u.nq && q4)
-      p.mask[uidx * p.mask_words + bk] = ballot;
-#pragma unroll 1
+    if (lane == 0) {
+      mask_s[bk - blk0] = ballot;
+      if (p.mask != nullptr && q4 && bk < nqb) p.mask[uidx * p.mask_words + bk] = ballot;
+    }
+    // load both token iterations' rows first, then accumulate
+    uint4 hw[LPT];
+    float4 mt[LPT];
+    int tq[LPT];
+#pragma unroll
+    for (int it = 0; it < LPT; ++it) {
+      const int tpos = bk * 32 + it * TPI + lane / LPT;
+      tq[it] = tpos;
+      if (tpos < qlim) {
+        hw[it] = ld_stream(u.data + u.Ld.v_hi + (size_t)tpos * vrow + hf * 16);
+        mt[it] = ldg128f(u.data + u.Ld.v_meta + (size_t)tpos * vrow + hf * 16);
+      }
+    }
+#pragma unroll
     for (int it = 0; it < LPT; ++it) {
       const int tk = it * TPI + lane / LPT;
-      const int tpos = bk * 32 + tk;
       const float pt = __shfl_sync(0xffffffffu, pw, tk);
-      if (tpos >= p1) continue;
-      if (quant && tpos < u.nq) {
-        const uint8_t* vh = u.data + u.Ld.v_hi + (size_t)tpos * vrow + hf * 16;
-        const uint8_t* vm = u.data + u.Ld.v_meta + (size_t)tpos * vrow + hf * 16;
-        const uint4 hw4 = ld_stream(vh);
-        const float4 mt = ldg128f(vm);  // (scale, zero) of the lane's two groups
-        const float ps0 = pt * mt.x, ps1 = pt * mt.z;
+      const int tpos = tq[it];
+      if (tpos < qlim) {
         const bool tsel = (ballot >> tk) & 1u;
-        uint4 lw4 = make_uint4(0, 0, 0, 0);
-        if (q4) {
-          if (tsel) {
-            lw4 = ld_stream(u.data + u.Ld.v_lo + (size_t)tpos * vrow + hf * 16);
-            g0 = fmaf(pt, mt.y, g0);
-            g1 = fmaf(pt, mt.w, g1);
-          } else {
-            g0 += fmaf(1.5f, ps0, pt * mt.y);
-            g1 += fmaf(1.5f, ps1, pt * mt.w);
-          }
-        } else {
-          g0 = fmaf(pt, mt.y, g0);
-          g1 = fmaf(pt, mt.w, g1);
-        }
-        const uint32_t hw[4] = {hw4.x, hw4.y, hw4.z, hw4.w};
-        const uint32_t lw[4] = {lw4.x, lw4.y, lw4.z, lw4.w};
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float ps = (w < 2) ? ps0 : ps1;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            uint32_t code = (hw[w] >> (2 * j)) & 3u;
-            if (q4) code = (code << 2) | ((lw[w] >> (2 * j)) & 3u);
-            acc[16 * w + j] = fmaf(ps, code_f(code), acc[16 * w + j]);
-          }
-        }
-      } else {
-        const uint8_t* row = raw_row(u, tpos, D, true) + hf * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 w = ldg128(row + c * 16);
-          acc[8 * c + 0] = fmaf(pt, bf16_lo(w.x), acc[8 * c + 0]);
-          acc[8 * c + 1] = fmaf(pt, bf16_hi(w.x), acc[8 * c + 1]);
-          acc[8 * c + 2] = fmaf(pt, bf16_lo(w.y), acc[8 * c + 2]);
-          acc[8 * c + 3] = fmaf(pt, bf16_hi(w.y), acc[8 * c + 3]);
-          acc[8 * c + 4] = fmaf(pt, bf16_lo(w.z), acc[8 * c + 4]);
-          acc[8 * c + 5] = fmaf(pt, bf16_hi(w.z), acc[8 * c + 5]);
-          acc[8 * c + 6] = fmaf(pt, bf16_lo(w.w), acc[8 * c + 6]);
-          acc[8 * c + 7] = fmaf(pt, bf16_hi(w.w), acc[8 * c + 7]);
+        const float ps0 = pt * mt[it].x, ps1 = pt * mt[it].z;
+        // unselected 4-bit tokens read hi alone: scale * (4 hi + 1.5) + zero
+        const float mid = (q4 && !tsel) ? 1.5f : 0.f;
+        g0 += fmaf(mid, ps0, pt * mt[it].y);
+        g1 += fmaf(mid, ps1, pt * mt[it].w);
+        value_codes(acc, hw[it], hmul * ps0, hmul * ps1);
+      } else if (tpos < p1) {
+        value_raw(acc, raw_row(u, tpos, D, true) + hf * 128, pt);
+      }
+    }
+  }
+  // low planes of the selected tokens: acc += p * scale * lo
+  if (q4) {
+    __syncthreads();  // mask_s complete
+    int* my = lst + warp * 32;
+    for (int bk = blk0 + warp; bk < qend; bk += kWarps) {
+      const uint32_t word = mask_s[bk - blk0];
+      if (word == 0u) continue;
+      if ((word >> lane) & 1u) my[__popc(word & ((1u << lane) - 1u))] = lane;
+      __syncwarp();
+      const int n = __popc(word);
+      for (int k0 = 0; k0 < n; k0 += TPI) {
+        const int kk = k0 + lane / LPT;
+        if (kk < n) {
+          const int tpos = bk * 32 + my[kk];
+          const float pt = sc[tpos - p0] * f;
+          const uint4 lw = ld_stream(u.data + u.Ld.v_lo + (size_t)tpos * vrow + hf * 16);
+          const float4 m4 = ldg128f(u.data + u.Ld.v_meta + (size_t)tpos * vrow + hf * 16);
+          value_codes(acc, lw, pt * m4.x, pt * m4.z);
         }
       }
+      __syncwarp();
     }
   }
   // per-group constants, then reduce over the lanes that share a channel half
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] += g0;
+  for (int i = 0; i < 16; ++i) { acc[i].x += g0; acc[i].y += g0; }
 #pragma unroll
-  for (int i = 32; i < 64; ++i) acc[i] += g1;
+  for (int i = 16; i < 32; ++i) { acc[i].x += g1; acc[i].y += g1; }
 #pragma unroll
-  for (int i = 0; i < 64; ++i) {
+  for (int i = 0; i < 32; ++i) {
 #pragma unroll
-    for (int o = 16; o >= LPT; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    for (int o = 16; o >= LPT; o >>= 1) {
+      acc[i].x += __shfl_xor_sync(0xffffffffu, acc[i].x, o);
+      acc[i].y += __shfl_xor_sync(0xffffffffu, acc[i].y, o);
+    }
   }
   if (lane < LPT) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) red[warp * D + lane * 64 + i] = acc[i];
+    for (int i = 0; i < 32; ++i)
+      reinterpret_cast<float2*>(red + warp * D + lane * 64)[i] = acc[i];
   }
   if (lane == 0) misc[24 + warp] = __int_as_float(nsel);
   __syncthreads();
@@ -441,7 +587,7 @@ decode_kernel(const DecodeParams p, const CellList cl) {
 
 template <int D>
 size_t decode_smem(int slots) {
-  return sizeof(float) * (size_t)(D + 2 * kWarps * D + D + 64 + slots);
+  return sizeof(float) * (size_t)(D + 2 * kWarps * D + D + 64 + kWarps * 32 + slots / 32 + slots);
 }
 
 template <int D>

@@ -110,8 +110,11 @@ def test_config2_batched_16k(pool, dev):
 @pytest.mark.parametrize("sub", ["a", "b", "c", "d"])
 def test_config3_ablation(pool, dev, sub):
     # every cell of an ablation plan has the same kind: 8 cells of the
-    # 16K batch-32 shape are enough to cover it
-    _run_decode_only("3" + sub, pool, dev, cells=[0, 13, 30, 47, 50, 71, 80, 95], n_sample=12)
+    # 16K shape cover it.  The all-bf16 plan (412 GB for the whole batch)
+    # runs on a 4-sequence slice of the batch.
+    seqs = [0, 9, 22, 31] if sub == "d" else None
+    _run_decode_only("3" + sub, pool, dev, cells=[0, 13, 30, 47, 50, 71, 80, 95], seqs=seqs,
+                     n_sample=12)
 
 
 def test_config4_ragged_serving_steps(pool, dev):
