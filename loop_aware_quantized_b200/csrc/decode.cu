@@ -85,60 +85,57 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   return d;
 }
 
-// A code field of `bits` bits at bit offset `off` (off + bits <= 23) of w,
-// as the exact float 2^(23-off) + code: the field becomes the low mantissa
-// bits of a float whose exponent makes one mantissa step worth 1.  A single
-// logic op; subtracting 2^(23-off) afterwards leaves the code exactly.
+// Codes to floats, exactly, at one logic op per code.  A field of `bits`
+// bits at bit offset `off` (off + bits <= 23) of a word w becomes the float
+// 2^23 + code * 2^off: the word's field is placed in the mantissa of a float
+// whose exponent word `expo` (the bits of 2^23) arrives in a register, so the
+// mask is the logic op's only immediate.  Subtracting 2^23 (exact) leaves
+// code * 2^off; the power of two is folded into the weights (keys) or
+// removed from the accumulators at the end (values).
 template <int off, int bits>
-__device__ __forceinline__ float code_plus_pow2(uint32_t w) {
+__device__ __forceinline__ float field_f(uint32_t w, uint32_t expo) {
   static_assert(off + bits <= 23, "field must stay inside the mantissa");
-  constexpr uint32_t mask = ((1u << bits) - 1u) << off;
-  constexpr uint32_t expo = (uint32_t)(150 - off) << 23;
-  return __uint_as_float((w & mask) | expo);
-}
-template <int off>
-__device__ __forceinline__ constexpr float pow2_of() {
-  return (float)(1u << (23 - off));
+  return __uint_as_float((w & (((1u << bits) - 1u) << off)) | expo);
 }
 
-// 16 two-bit codes of w (code j in bits 2j..2j+1) -> 8 pairs (code 2i,
-// code 2i+1) as floats, exactly.
-__device__ __forceinline__ void codes2_to_pairs(uint32_t w, float2 (&out)[8]) {
-  const uint32_t y = w >> 12;  // codes 6..15 move to fields 0..9 (bits <= 19)
-#define LKV_PAIR(i, src_a, off_a, src_b, off_b)                                          \
-  out[i] = add2(make_float2(code_plus_pow2<off_a, 2>(src_a), code_plus_pow2<off_b, 2>(src_b)), \
-                make_float2(-pow2_of<off_a>(), -pow2_of<off_b>()));
-  LKV_PAIR(0, w, 0, w, 2)
-  LKV_PAIR(1, w, 4, w, 6)
-  LKV_PAIR(2, w, 8, w, 10)
-  LKV_PAIR(3, y, 0, y, 2)      // codes 6, 7
-  LKV_PAIR(4, y, 4, y, 6)      // codes 8, 9
-  LKV_PAIR(5, y, 8, y, 10)     // codes 10, 11
-  LKV_PAIR(6, y, 12, y, 14)    // codes 12, 13
-  LKV_PAIR(7, y, 16, y, 18)    // codes 14, 15
-#undef LKV_PAIR
+// 16 two-bit codes of w (code j in bits 2j..2j+1) -> 8 pairs
+// (code 2i * 2^o(2i), code 2i+1 * 2^o(2i+1)), o(j) = 2j for j < 6, 2(j-6) else.
+__device__ __forceinline__ void codes2_to_pairs(uint32_t w, uint32_t expo, float2 neg,
+                                                float2 (&out)[8]) {
+  const uint32_t y = w >> 12;
+  out[0] = add2(make_float2(field_f<0, 2>(w, expo), field_f<2, 2>(w, expo)), neg);
+  out[1] = add2(make_float2(field_f<4, 2>(w, expo), field_f<6, 2>(w, expo)), neg);
+  out[2] = add2(make_float2(field_f<8, 2>(w, expo), field_f<10, 2>(w, expo)), neg);
+  out[3] = add2(make_float2(field_f<0, 2>(y, expo), field_f<2, 2>(y, expo)), neg);
+  out[4] = add2(make_float2(field_f<4, 2>(y, expo), field_f<6, 2>(y, expo)), neg);
+  out[5] = add2(make_float2(field_f<8, 2>(y, expo), field_f<10, 2>(y, expo)), neg);
+  out[6] = add2(make_float2(field_f<12, 2>(y, expo), field_f<14, 2>(y, expo)), neg);
+  out[7] = add2(make_float2(field_f<16, 2>(y, expo), field_f<18, 2>(y, expo)), neg);
 }
+// Bit offset a two-bit code j of a word ends up at in codes2_to_pairs.
+__host__ __device__ constexpr int code2_off(int j) { return j < 6 ? 2 * j : 2 * (j - 6); }
 
-// Hi and lo planes of 16 four-bit codes -> 8 pairs (q_2i, q_2i+1), q = 4hi+lo.
-// Bitwise merge into two words of nibbles: even codes (nibble m = code 2m)
-// and odd codes (nibble m = code 2m+1).
-__device__ __forceinline__ void codes4_to_pairs(uint32_t hi, uint32_t lo, float2 (&out)[8]) {
+// Hi and lo planes of 16 four-bit codes -> 8 pairs (q_2m * 2^o(m), q_2m+1 *
+// 2^o(m)), q = 4hi + lo, o(m) = 4m for m < 3, 4(m-3) else.  The planes are
+// merged into a word of even codes (nibble m = code 2m) and one of odd codes.
+__device__ __forceinline__ void codes4_to_pairs(uint32_t hi, uint32_t lo, uint32_t expo,
+                                                float2 neg, float2 (&out)[8]) {
   const uint32_t even = ((hi << 2) & 0xCCCCCCCCu) | (lo & 0x33333333u);
   const uint32_t odd = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
-  const uint32_t even_h = even >> 12, odd_h = odd >> 12;  // nibbles 3..7 -> 0..4
-#define LKV_NIB(i, e, o, off)                                                    \
-  out[i] = add2(make_float2(code_plus_pow2<off, 4>(e), code_plus_pow2<off, 4>(o)), \
-                make_float2(-pow2_of<off>(), -pow2_of<off>()));
-  LKV_NIB(0, even, odd, 0)
-  LKV_NIB(1, even, odd, 4)
-  LKV_NIB(2, even, odd, 8)
-  LKV_NIB(3, even_h, odd_h, 0)
-  LKV_NIB(4, even_h, odd_h, 4)
-  LKV_NIB(5, even_h, odd_h, 8)
-  LKV_NIB(6, even_h, odd_h, 12)
-  LKV_NIB(7, even_h, odd_h, 16)
-#undef LKV_NIB
+  const uint32_t eh = even >> 12, oh = odd >> 12;
+  out[0] = add2(make_float2(field_f<0, 4>(even, expo), field_f<0, 4>(odd, expo)), neg);
+  out[1] = add2(make_float2(field_f<4, 4>(even, expo), field_f<4, 4>(odd, expo)), neg);
+  out[2] = add2(make_float2(field_f<8, 4>(even, expo), field_f<8, 4>(odd, expo)), neg);
+  out[3] = add2(make_float2(field_f<0, 4>(eh, expo), field_f<0, 4>(oh, expo)), neg);
+  out[4] = add2(make_float2(field_f<4, 4>(eh, expo), field_f<4, 4>(oh, expo)), neg);
+  out[5] = add2(make_float2(field_f<8, 4>(eh, expo), field_f<8, 4>(oh, expo)), neg);
+  out[6] = add2(make_float2(field_f<12, 4>(eh, expo), field_f<12, 4>(oh, expo)), neg);
+  out[7] = add2(make_float2(field_f<16, 4>(eh, expo), field_f<16, 4>(oh, expo)), neg);
 }
+__host__ __device__ constexpr int code4_off(int m) { return m < 3 ? 4 * m : 4 * (m - 3); }
+
+// 2^-k as a float, k in [0, 126].
+__device__ __forceinline__ float pow2_neg(int k) { return __int_as_float((127 - k) << 23); }
 
 struct Unit {
   int own_kind, data_kind;
@@ -220,7 +217,7 @@ __device__ __forceinline__ float dot_bf16(const uint8_t* row, const float* q_s) 
 // planes (16-byte rows h[c], l[c] of K_hi / K_lo for chunk c of 64 channels).
 template <int D, bool Q4>
 __device__ __forceinline__ float dot_codes(const uint4 (&h)[D / 64], const uint4 (&l)[D / 64],
-                                           const float2* qs2) {
+                                           const float2* qs2, uint32_t expo, float2 neg) {
   float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < D / 64; ++c) {
@@ -229,8 +226,8 @@ __device__ __forceinline__ float dot_codes(const uint4 (&h)[D / 64], const uint4
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       float2 v[8];
-      if (Q4) codes4_to_pairs(hw[w], lw[w], v);
-      else codes2_to_pairs(hw[w], v);
+      if (Q4) codes4_to_pairs(hw[w], lw[w], expo, neg, v);
+      else codes2_to_pairs(hw[w], expo, neg, v);
       const float4* q4p = reinterpret_cast<const float4*>(qs2 + 32 * c + 8 * w);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -279,14 +276,23 @@ __device__ __forceinline__ void load_kgroup(KGroup<D>& g, const uint8_t* data, c
 template <int D, bool Q4>
 __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end, int p0, int p1,
                                           const float* q_s, float* qs, float* sc, float sscale,
-                                          int warp, int lane) {
+                                          uint32_t expo, float2 neg, int warp, int lane) {
   constexpr int CPL = D / 32;  // channels per lane for the q fold
   float lmax = -INFINITY;
   int bk = b_begin + warp;
   if (bk >= b_end) return lmax;
+  // q of the lane's channels, times 2^-o: o is the bit offset the channel's
+  // code keeps after conversion (see codes4_to_pairs / codes2_to_pairs)
   float qv[CPL];
 #pragma unroll
-  for (int i = 0; i < CPL; ++i) qv[i] = q_s[CPL * lane + i];
+  for (int i = 0; i < CPL; ++i) {
+    const int j = (CPL * lane + i) & 15;
+    qv[i] = q_s[CPL * lane + i] * pow2_neg(Q4 ? code4_off(j >> 1) : code2_off(j));
+  }
+  // the zero-point fold uses q itself
+  float qz[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) qz[i] = q_s[CPL * lane + i];
   KGroup<D> cur, nxt;
   load_kgroup<D, Q4>(cur, u.data, u.Ld, bk, lane);
   for (; bk < b_end; bk += kWarps) {
@@ -297,14 +303,14 @@ __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end,
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
       qs[CPL * lane + i] = qv[i] * cur.sc[i];
-      cpart = fmaf(qv[i], cur.zr[i], cpart);
+      cpart = fmaf(qz[i], cur.zr[i], cpart);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o);
     __syncwarp();
     const int pos = bk * 32 + lane;
     if (pos < u.nq && pos < p1) {
-      const float dot = dot_codes<D, Q4>(cur.h, cur.l, reinterpret_cast<const float2*>(qs));
+      const float dot = dot_codes<D, Q4>(cur.h, cur.l, reinterpret_cast<const float2*>(qs), expo, neg);
       const float s = (dot + cpart) * sscale;
       sc[pos - p0] = s;
       lmax = fmaxf(lmax, s);
@@ -316,13 +322,15 @@ __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end,
 }
 
 // Value accumulation of one quantized token half-row (64 channels): acc +=
-// (m * p * scale_j) * code for the lane's two 32-channel groups.
-__device__ __forceinline__ void value_codes(float2 (&acc)[32], const uint4 hw4, float a0, float a1) {
+// (a_j) * code * 2^o for the lane's two 32-channel groups (a0 for words 0-1,
+// a1 for words 2-3); the 2^o of each channel is removed once at the end.
+__device__ __forceinline__ void value_codes(float2 (&acc)[32], const uint4 hw4, float a0, float a1,
+                                            uint32_t expo, float2 neg) {
   const uint32_t hw[4] = {hw4.x, hw4.y, hw4.z, hw4.w};
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     float2 v[8];
-    codes2_to_pairs(hw[w], v);
+    codes2_to_pairs(hw[w], expo, neg, v);
     const float a = (w < 2) ? a0 : a1;
     const float2 aa = make_float2(a, a);
 #pragma unroll
@@ -330,15 +338,21 @@ __device__ __forceinline__ void value_codes(float2 (&acc)[32], const uint4 hw4, 
   }
 }
 
+// bf16 value row (64 channels) with weight pt, in the accumulators' scaled
+// representation (channel j of a 16-channel word carries 2^o(j)).
 __device__ __forceinline__ void value_raw(float2 (&acc)[32], const uint8_t* row, float pt) {
-  const float2 pp = make_float2(pt, pt);
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const uint4 w = ldg128(row + c * 16);
-    acc[4 * c + 0] = fma2(pp, make_float2(bf16_lo(w.x), bf16_hi(w.x)), acc[4 * c + 0]);
-    acc[4 * c + 1] = fma2(pp, make_float2(bf16_lo(w.y), bf16_hi(w.y)), acc[4 * c + 1]);
-    acc[4 * c + 2] = fma2(pp, make_float2(bf16_lo(w.z), bf16_hi(w.z)), acc[4 * c + 2]);
-    acc[4 * c + 3] = fma2(pp, make_float2(bf16_lo(w.w), bf16_hi(w.w)), acc[4 * c + 3]);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int pair = 4 * c + k;          // channels 2*pair, 2*pair+1
+      const int j = (2 * pair) & 15;       // position inside the 16-channel word
+      const float2 wt = make_float2(pt * (float)(1u << code2_off(j)),
+                                    pt * (float)(1u << code2_off(j + 1)));
+      acc[pair] = fma2(wt, make_float2(bf16_lo(ws[k]), bf16_hi(ws[k])), acc[pair]);
+    }
   }
 }
 
@@ -401,8 +415,11 @@ decode_kernel(const DecodeParams p, const CellList cl) {
 
   // ------------------------------------------------------------- pass 1
   float lmax = -INFINITY;
-  if (q4) lmax = key_pass<D, true>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, warp, lane);
-  else if (quant) lmax = key_pass<D, false>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, warp, lane);
+  const uint32_t expo = p.code_expo;
+  const float2 neg = make_float2(p.code_neg, p.code_neg);
+  if (q4) lmax = key_pass<D, true>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, expo, neg, warp, lane);
+  else if (quant)
+    lmax = key_pass<D, false>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, expo, neg, warp, lane);
   // bf16 positions: residual, raw cells, the SHARE current token
   for (int pos = max(p0, u.nq) + 32 * warp + lane; pos < p1; pos += 32 * kWarps) {
     const float s = dot_bf16<D>(raw_row(u, pos, D, false), q_s) * sscale;
@@ -497,7 +514,7 @@ decode_kernel(const DecodeParams p, const CellList cl) {
         const float mid = (q4 && !tsel) ? 1.5f : 0.f;
         g0 += fmaf(mid, ps0, pt * mt[it].y);
         g1 += fmaf(mid, ps1, pt * mt[it].w);
-        value_codes(acc, hw[it], hmul * ps0, hmul * ps1);
+        value_codes(acc, hw[it], hmul * ps0, hmul * ps1, expo, neg);
       } else if (tpos < p1) {
         value_raw(acc, raw_row(u, tpos, D, true) + hf * 128, pt);
       }
@@ -520,17 +537,20 @@ decode_kernel(const DecodeParams p, const CellList cl) {
           const float pt = sc[tpos - p0] * f;
           const uint4 lw = ld_stream(u.data + u.Ld.v_lo + (size_t)tpos * vrow + hf * 16);
           const float4 m4 = ldg128f(u.data + u.Ld.v_meta + (size_t)tpos * vrow + hf * 16);
-          value_codes(acc, lw, pt * m4.x, pt * m4.z);
+          value_codes(acc, lw, pt * m4.x, pt * m4.z, expo, neg);
         }
       }
       __syncwarp();
     }
   }
-  // per-group constants, then reduce over the lanes that share a channel half
+  // undo the per-channel 2^o of the code conversion, add the per-group
+  // constants, then reduce over the lanes that share a channel half
 #pragma unroll
-  for (int i = 0; i < 16; ++i) { acc[i].x += g0; acc[i].y += g0; }
-#pragma unroll
-  for (int i = 16; i < 32; ++i) { acc[i].x += g1; acc[i].y += g1; }
+  for (int i = 0; i < 32; ++i) {
+    const int j = (2 * i) & 15;
+    acc[i].x = fmaf(acc[i].x, pow2_neg(code2_off(j)), i < 16 ? g0 : g1);
+    acc[i].y = fmaf(acc[i].y, pow2_neg(code2_off(j + 1)), i < 16 ? g0 : g1);
+  }
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
 #pragma unroll
