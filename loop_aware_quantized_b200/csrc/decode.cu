@@ -45,6 +45,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxSlots = 24576;  // score slots per CTA (96 KB)
 constexpr int kMaxSplit = 8;      // portable cluster size
+constexpr int kListCap = 64;      // per-warp list of selected positions awaiting their low plane
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -218,7 +219,10 @@ __device__ __forceinline__ float dot_bf16(const uint8_t* row, const float* q_s) 
 template <int D, bool Q4>
 __device__ __forceinline__ float dot_codes(const uint4 (&h)[D / 64], const uint4 (&l)[D / 64],
                                            const float2* qs2, uint32_t expo, float2 neg) {
-  float2 acc = make_float2(0.f, 0.f);
+  // four independent accumulators keep the fma chain short
+  float2 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < D / 64; ++c) {
     const uint32_t hw[4] = {h[c].x, h[c].y, h[c].z, h[c].w};
@@ -232,12 +236,13 @@ __device__ __forceinline__ float dot_codes(const uint4 (&h)[D / 64], const uint4
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float4 qq = q4p[i];
-        acc = fma2(make_float2(qq.x, qq.y), v[2 * i], acc);
-        acc = fma2(make_float2(qq.z, qq.w), v[2 * i + 1], acc);
+        acc[(2 * i) & 3] = fma2(make_float2(qq.x, qq.y), v[2 * i], acc[(2 * i) & 3]);
+        acc[(2 * i + 1) & 3] = fma2(make_float2(qq.z, qq.w), v[2 * i + 1], acc[(2 * i + 1) & 3]);
       }
     }
   }
-  return acc.x + acc.y;
+  const float2 a = add2(acc[0], acc[1]), b = add2(acc[2], acc[3]);
+  return (a.x + b.x) + (a.y + b.y);
 }
 
 // Per-lane load of one 32-token key group: the lane's token rows of the
@@ -356,6 +361,27 @@ __device__ __forceinline__ void value_raw(float2 (&acc)[32], const uint8_t* row,
   }
 }
 
+// Low planes of queued selected positions: acc += p * scale * lo, TPI
+// positions per warp iteration (LPT lanes per position, 64 channels each).
+template <int D, int LPT>
+__device__ __forceinline__ void low_planes(float2 (&acc)[32], const Unit& u, const int* list,
+                                           int n, const float* sc, int p0, float f,
+                                           uint32_t expo, float2 neg, int lane) {
+  constexpr int TPI = 32 / LPT;
+  const int hf = lane % LPT;
+  for (int k0 = 0; k0 < n; k0 += TPI) {
+    const int kk = k0 + lane / LPT;
+    if (kk < n) {
+      const int tpos = list[kk];
+      const float pt = sc[tpos - p0] * f;
+      const uint4 lw = ld_stream(u.data + u.Ld.v_lo + (size_t)tpos * (D / 4) + hf * 16);
+      const float4 m4 = ldg128f(u.data + u.Ld.v_meta + (size_t)tpos * (D / 4) + hf * 16);
+      value_codes(acc, lw, pt * m4.x, pt * m4.z, expo, neg);
+    }
+  }
+  __syncwarp();
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p, const CellList cl) {
@@ -367,8 +393,8 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   float* red = qs_all + kWarps * D;                   // [kWarps][D]
   float* o_s = red + kWarps * D;                      // [D]
   float* misc = o_s + D;                              // [64]
-  int* lst = reinterpret_cast<int*>(misc + 64);       // [kWarps][32]
-  uint32_t* mask_s = reinterpret_cast<uint32_t*>(lst + kWarps * 32);  // [slots / 32]
+  int* lst = reinterpret_cast<int*>(misc + 64);       // [kWarps][kListCap] selected positions
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(lst + kWarps * kListCap);  // [slots / 32]
   float* sc = reinterpret_cast<float*>(mask_s + p.slots / 32);        // [slots]
 
   const int split = p.split;
@@ -520,28 +546,26 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       }
     }
   }
-  // low planes of the selected tokens: acc += p * scale * lo
+  // low planes of the selected tokens: acc += p * scale * lo.  The warp
+  // gathers its selected positions into a list and processes them TPI at a
+  // time, so the cost follows the number of selected tokens.
   if (q4) {
     __syncthreads();  // mask_s complete
-    int* my = lst + warp * 32;
+    int* my = lst + warp * kListCap;
+    int nlist = 0;
     for (int bk = blk0 + warp; bk < qend; bk += kWarps) {
       const uint32_t word = mask_s[bk - blk0];
       if (word == 0u) continue;
-      if ((word >> lane) & 1u) my[__popc(word & ((1u << lane) - 1u))] = lane;
-      __syncwarp();
-      const int n = __popc(word);
-      for (int k0 = 0; k0 < n; k0 += TPI) {
-        const int kk = k0 + lane / LPT;
-        if (kk < n) {
-          const int tpos = bk * 32 + my[kk];
-          const float pt = sc[tpos - p0] * f;
-          const uint4 lw = ld_stream(u.data + u.Ld.v_lo + (size_t)tpos * vrow + hf * 16);
-          const float4 m4 = ldg128f(u.data + u.Ld.v_meta + (size_t)tpos * vrow + hf * 16);
-          value_codes(acc, lw, pt * m4.x, pt * m4.z, expo, neg);
-        }
+      const int cnt = __popc(word);
+      if (nlist + cnt > kListCap) {
+        low_planes<D, LPT>(acc, u, my, nlist, sc, p0, f, expo, neg, lane);
+        nlist = 0;
       }
+      if ((word >> lane) & 1u) my[nlist + __popc(word & ((1u << lane) - 1u))] = bk * 32 + lane;
+      nlist += cnt;
       __syncwarp();
     }
+    if (nlist > 0) low_planes<D, LPT>(acc, u, my, nlist, sc, p0, f, expo, neg, lane);
   }
   // undo the per-channel 2^o of the code conversion, add the per-group
   // constants, then reduce over the lanes that share a channel half
@@ -607,7 +631,7 @@ decode_kernel(const DecodeParams p, const CellList cl) {
 
 template <int D>
 size_t decode_smem(int slots) {
-  return sizeof(float) * (size_t)(D + 2 * kWarps * D + D + 64 + kWarps * 32 + slots / 32 + slots);
+  return sizeof(float) * (size_t)(D + 2 * kWarps * D + D + 64 + kWarps * kListCap + slots / 32 + slots);
 }
 
 template <int D>
