@@ -182,17 +182,21 @@ def source_hash(paths):
 
 
 def ncu_traffic(kernel_src):
-    """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
-    when it was taken on the current kernel source; else None."""
+    """DRAM bytes / algorithmic bytes of the decode kernel from the committed ncu
+    capture (profiles/decode_traffic.json), when it was taken on the current
+    kernel source; else None.  Traffic grows with the units a launch
+    processes, so a full launch moves this ratio times its algorithmic bytes."""
+    rec_paths = ["loop_aware_quantized_b200/csrc/decode.cu",
+                 "loop_aware_quantized_b200/csrc/loopkv_internal.cuh"]
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("source_hash") != source_hash(kernel_src):
+    if rec.get("source_hash") != source_hash([os.path.join(ROOT, p) for p in rec_paths]):
         return None
-    return rec.get("bytes_per_full_launch")
+    return rec.get("traffic_over_algorithmic")
 
 
 # --------------------------------------------------------- oracle baseline
@@ -438,8 +442,10 @@ def main():
     n_dec_launches = args.steps * len(phase)
     kernel_src = [os.path.join(ROOT, "loop_aware_quantized_b200", "csrc", f)
                   for f in ("decode.cu", "loopkv_internal.cuh")]
+    tr = ncu_traffic(kernel_src)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": ncu_traffic(kernel_src),
+                "frac": achieved / peak,
+                "traffic": None if tr is None else tr * dec_bytes / n_dec_launches,
                 "peak_kind": peak_kind + " copy bandwidth",
                 "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                 "kernel": "loopkv decode", "bytes_per_launch": dec_bytes / n_dec_launches,
