@@ -253,75 +253,102 @@ struct KGroup {
   float sc[D / 32], zr[D / 32];
 };
 
+// Lane pointers into one group: kh -> the lane's K_hi row of chunk 0,
+// lo_off -> K_lo - K_hi, km -> the lane's scales (zeros D floats further).
 template <int D, bool Q4>
-__device__ __forceinline__ void load_kgroup(KGroup<D>& g, const uint8_t* data, const UnitLayout& L,
-                                            int bk, int lane) {
-  const size_t goff = (size_t)bk * 8 * D;
+__device__ __forceinline__ void load_kgroup(KGroup<D>& g, const uint8_t* kh, size_t lo_off,
+                                            const float* km) {
 #pragma unroll
   for (int c = 0; c < D / 64; ++c) {
-    g.h[c] = ld_stream(data + L.k_hi + goff + c * 512 + lane * 16);
-    g.l[c] = Q4 ? ld_stream(data + L.k_lo + goff + c * 512 + lane * 16) : make_uint4(0, 0, 0, 0);
+    g.h[c] = ld_stream(kh + c * 512);
+    g.l[c] = Q4 ? ld_stream(kh + lo_off + c * 512) : make_uint4(0, 0, 0, 0);
   }
-  const float* meta = reinterpret_cast<const float*>(data + L.k_meta + goff);
   if constexpr (D == 128) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(meta) + lane);
-    const float4 z = __ldg(reinterpret_cast<const float4*>(meta + D) + lane);
+    const float4 a = __ldg(reinterpret_cast<const float4*>(km));
+    const float4 z = __ldg(reinterpret_cast<const float4*>(km + D));
     g.sc[0] = a.x; g.sc[1] = a.y; g.sc[2] = a.z; g.sc[3] = a.w;
     g.zr[0] = z.x; g.zr[1] = z.y; g.zr[2] = z.z; g.zr[3] = z.w;
   } else {
-    const float2 a = __ldg(reinterpret_cast<const float2*>(meta) + lane);
-    const float2 z = __ldg(reinterpret_cast<const float2*>(meta + D) + lane);
+    const float2 a = __ldg(reinterpret_cast<const float2*>(km));
+    const float2 z = __ldg(reinterpret_cast<const float2*>(km + D));
     g.sc[0] = a.x; g.sc[1] = a.y;
     g.zr[0] = z.x; g.zr[1] = z.y;
   }
 }
 
-// Pass 1 over the CTA's quantized key groups [b_begin, b_end), warp-strided,
-// with the next group's loads in flight while the current one is scored.
+// Score one group held in registers; returns the lane's score (or -inf).
+template <int D, bool Q4>
+__device__ __forceinline__ float key_group(const KGroup<D>& g, const float (&qv)[D / 32],
+                                           const float (&qz)[D / 32], float* qs, int pos,
+                                           int qlim, float sscale, uint32_t expo, float2 neg,
+                                           int lane) {
+  constexpr int CPL = D / 32;
+  // fold q into the group's key scale / zero point
+  float cpart = 0.f;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) {
+    qs[CPL * lane + i] = qv[i] * g.sc[i];
+    cpart = fmaf(qz[i], g.zr[i], cpart);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o);
+  __syncwarp();
+  float s = -INFINITY;
+  if (pos < qlim) {
+    const float dot = dot_codes<D, Q4>(g.h, g.l, reinterpret_cast<const float2*>(qs), expo, neg);
+    s = (dot + cpart) * sscale;
+  }
+  __syncwarp();
+  return s;
+}
+
+// Pass 1 over the CTA's quantized key groups [b_begin, b_end), warp-strided.
+// Two register buffers alternate, so the next group's loads are in flight
+// while the current one is scored, without copies between them.
 template <int D, bool Q4>
 __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end, int p0, int p1,
                                           const float* q_s, float* qs, float* sc, float sscale,
                                           uint32_t expo, float2 neg, int warp, int lane) {
   constexpr int CPL = D / 32;  // channels per lane for the q fold
   float lmax = -INFINITY;
-  int bk = b_begin + warp;
-  if (bk >= b_end) return lmax;
+  const int first = b_begin + warp;
+  if (first >= b_end) return lmax;
   // q of the lane's channels, times 2^-o: o is the bit offset the channel's
   // code keeps after conversion (see codes4_to_pairs / codes2_to_pairs)
-  float qv[CPL];
+  float qv[CPL], qz[CPL];
 #pragma unroll
   for (int i = 0; i < CPL; ++i) {
     const int j = (CPL * lane + i) & 15;
-    qv[i] = q_s[CPL * lane + i] * pow2_neg(Q4 ? code4_off(j >> 1) : code2_off(j));
+    qz[i] = q_s[CPL * lane + i];
+    qv[i] = qz[i] * pow2_neg(Q4 ? code4_off(j >> 1) : code2_off(j));
   }
-  // the zero-point fold uses q itself
-  float qz[CPL];
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) qz[i] = q_s[CPL * lane + i];
-  KGroup<D> cur, nxt;
-  load_kgroup<D, Q4>(cur, u.data, u.Ld, bk, lane);
-  for (; bk < b_end; bk += kWarps) {
-    const bool more = bk + kWarps < b_end;
-    if (more) load_kgroup<D, Q4>(nxt, u.data, u.Ld, bk + kWarps, lane);
-    // fold q into the group's key scale / zero point
-    float cpart = 0.f;
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      qs[CPL * lane + i] = qv[i] * cur.sc[i];
-      cpart = fmaf(qz[i], cur.zr[i], cpart);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o);
-    __syncwarp();
-    const int pos = bk * 32 + lane;
-    if (pos < u.nq && pos < p1) {
-      const float dot = dot_codes<D, Q4>(cur.h, cur.l, reinterpret_cast<const float2*>(qs), expo, neg);
-      const float s = (dot + cpart) * sscale;
-      sc[pos - p0] = s;
-      lmax = fmaxf(lmax, s);
-    }
-    __syncwarp();
-    if (more) cur = nxt;
+  const int qlim = min(p1, u.nq);
+  constexpr size_t G = 8 * D;                       // bytes of one group in each block
+  constexpr size_t STEP = (size_t)kWarps * G;       // a warp's stride between its groups
+  const uint8_t* kh = u.data + u.Ld.k_hi + (size_t)first * G + lane * 16;
+  const size_t lo_off = u.Ld.k_lo - u.Ld.k_hi;
+  const float* km = reinterpret_cast<const float*>(u.data + u.Ld.k_meta + (size_t)first * G) +
+                    CPL * lane;
+  KGroup<D> a, b;
+  load_kgroup<D, Q4>(a, kh, lo_off, km);
+  int bk = first;
+  for (;;) {
+    const bool hasb = bk + kWarps < b_end;
+    if (hasb) load_kgroup<D, Q4>(b, kh + STEP, lo_off, km + STEP / 4);
+    float s = key_group<D, Q4>(a, qv, qz, qs, bk * 32 + lane, qlim, sscale, expo, neg, lane);
+    if (bk * 32 + lane < qlim) { sc[bk * 32 + lane - p0] = s; lmax = fmaxf(lmax, s); }
+    if (!hasb) break;
+    bk += kWarps;
+    kh += STEP;
+    km += STEP / 4;
+    const bool hasa = bk + kWarps < b_end;
+    if (hasa) load_kgroup<D, Q4>(a, kh + STEP, lo_off, km + STEP / 4);
+    s = key_group<D, Q4>(b, qv, qz, qs, bk * 32 + lane, qlim, sscale, expo, neg, lane);
+    if (bk * 32 + lane < qlim) { sc[bk * 32 + lane - p0] = s; lmax = fmaxf(lmax, s); }
+    if (!hasa) break;
+    bk += kWarps;
+    kh += STEP;
+    km += STEP / 4;
   }
   return lmax;
 }
@@ -385,8 +412,6 @@ __device__ __forceinline__ void low_planes(float2 (&acc)[32], const Unit& u, con
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p, const CellList cl) {
-  constexpr int LPT = D / 64;       // lanes per token in pass 2 (64 channels per lane)
-  constexpr int TPI = 32 / LPT;     // tokens per warp iteration in pass 2
   extern __shared__ __align__(16) float smem[];
   float* q_s = smem;                                  // [D]
   float* qs_all = q_s + D;                            // [kWarps][D]
@@ -446,6 +471,26 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   if (q4) lmax = key_pass<D, true>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, expo, neg, warp, lane);
   else if (quant)
     lmax = key_pass<D, false>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, expo, neg, warp, lane);
+  // the warp's first value block is requested now, ahead of the softmax merge
+  constexpr int LPT = D / 64;       // lanes per token in pass 2 (64 channels per lane)
+  constexpr int TPI = 32 / LPT;     // tokens per warp iteration in pass 2
+  const int hf = lane % LPT;
+  const size_t vrow = D / 4;  // bytes per token of a value plane / value meta
+  const int qlim = min(p1, u.nq);
+  const size_t row0 = ((size_t)(blk0 + warp) * 32 + lane / LPT) * vrow + hf * 16;
+  const uint8_t* vh = u.data + u.Ld.v_hi + row0;
+  const uint8_t* vm = u.data + u.Ld.v_meta + row0;
+  constexpr size_t VSTEP = (size_t)kWarps * 32 * (D / 4);
+  auto full_block = [&](int bk) { return (bk + 1) * 32 <= qlim; };
+  uint4 nh[LPT];
+  float4 nm[LPT];
+  if (blk0 + warp < blk1 && full_block(blk0 + warp)) {
+#pragma unroll
+    for (int it = 0; it < LPT; ++it) {
+      nh[it] = ld_stream(vh + it * TPI * vrow);
+      nm[it] = ldg128f(vm + it * TPI * vrow);
+    }
+  }
   // bf16 positions: residual, raw cells, the SHARE current token
   for (int pos = max(p0, u.nq) + 32 * warp + lane; pos < p1; pos += 32 * kWarps) {
     const float s = dot_bf16<D>(raw_row(u, pos, D, false), q_s) * sscale;
@@ -500,11 +545,11 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.f, 0.f);
   float g0 = 0.f, g1 = 0.f;  // per-group constants of the lane's two 32-channel groups
   int nsel = 0;
-  const int hf = lane % LPT;
-  const size_t vrow = D / 4;  // bytes per token of a value plane / value meta
+  // 4-bit high plane: weight 4 * p * scale; its missing low bits read as 1.5,
+  // i.e. + 1.5 * p * scale = 0.375 * (4 * p * scale) per unselected token
   const float hmul = q4 ? 4.f : 1.f;
-  const int qlim = min(p1, u.nq);
-  for (int bk = blk0 + warp; bk < blk1; bk += kWarps) {
+  const float mid_unsel = q4 ? 0.375f : 0.f;
+  for (int bk = blk0 + warp; bk < blk1; bk += kWarps, vh += VSTEP, vm += VSTEP) {
     const int pos = bk * 32 + lane;
     const bool active = pos < p1;
     const float pw = active ? sc[pos - p0] * f : 0.f;
@@ -515,34 +560,47 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       mask_s[bk - blk0] = ballot;
       if (p.mask != nullptr && q4 && bk < nqb) p.mask[uidx * p.mask_words + bk] = ballot;
     }
-    // load both token iterations' rows first, then accumulate
-    uint4 hw[LPT];
-    float4 mt[LPT];
-    int tq[LPT];
+    if (full_block(bk)) {
+      // a full quantized block: rows arrived with the previous iteration
+      uint4 hw[LPT];
+      float4 mt[LPT];
 #pragma unroll
-    for (int it = 0; it < LPT; ++it) {
-      const int tpos = bk * 32 + it * TPI + lane / LPT;
-      tq[it] = tpos;
-      if (tpos < qlim) {
-        hw[it] = ld_stream(u.data + u.Ld.v_hi + (size_t)tpos * vrow + hf * 16);
-        mt[it] = ldg128f(u.data + u.Ld.v_meta + (size_t)tpos * vrow + hf * 16);
+      for (int it = 0; it < LPT; ++it) { hw[it] = nh[it]; mt[it] = nm[it]; }
+      if (bk + kWarps < blk1 && full_block(bk + kWarps)) {
+#pragma unroll
+        for (int it = 0; it < LPT; ++it) {
+          nh[it] = ld_stream(vh + VSTEP + it * TPI * vrow);
+          nm[it] = ldg128f(vm + VSTEP + it * TPI * vrow);
+        }
       }
-    }
 #pragma unroll
-    for (int it = 0; it < LPT; ++it) {
-      const int tk = it * TPI + lane / LPT;
-      const float pt = __shfl_sync(0xffffffffu, pw, tk);
-      const int tpos = tq[it];
-      if (tpos < qlim) {
-        const bool tsel = (ballot >> tk) & 1u;
-        const float ps0 = pt * mt[it].x, ps1 = pt * mt[it].z;
-        // unselected 4-bit tokens read hi alone: scale * (4 hi + 1.5) + zero
-        const float mid = (q4 && !tsel) ? 1.5f : 0.f;
-        g0 += fmaf(mid, ps0, pt * mt[it].y);
-        g1 += fmaf(mid, ps1, pt * mt[it].w);
-        value_codes(acc, hw[it], hmul * ps0, hmul * ps1, expo, neg);
-      } else if (tpos < p1) {
-        value_raw(acc, raw_row(u, tpos, D, true) + hf * 128, pt);
+      for (int it = 0; it < LPT; ++it) {
+        const int tk = it * TPI + lane / LPT;
+        const float pt = __shfl_sync(0xffffffffu, pw, tk);
+        const float mid = ((ballot >> tk) & 1u) ? 0.f : mid_unsel;
+        const float a0 = (hmul * pt) * mt[it].x, a1 = (hmul * pt) * mt[it].z;
+        g0 = fmaf(mid, a0, fmaf(pt, mt[it].y, g0));
+        g1 = fmaf(mid, a1, fmaf(pt, mt[it].w, g1));
+        value_codes(acc, hw[it], a0, a1, expo, neg);
+      }
+    } else {
+      // partial block: quantized tokens below qlim, bf16 ones up to p1
+#pragma unroll
+      for (int it = 0; it < LPT; ++it) {
+        const int tk = it * TPI + lane / LPT;
+        const float pt = __shfl_sync(0xffffffffu, pw, tk);
+        const int tpos = bk * 32 + tk;
+        if (tpos < qlim) {
+          const uint4 hwv = ld_stream(vh + it * TPI * vrow);
+          const float4 mtv = ldg128f(vm + it * TPI * vrow);
+          const float mid = ((ballot >> tk) & 1u) ? 0.f : mid_unsel;
+          const float a0 = (hmul * pt) * mtv.x, a1 = (hmul * pt) * mtv.z;
+          g0 = fmaf(mid, a0, fmaf(pt, mtv.y, g0));
+          g1 = fmaf(mid, a1, fmaf(pt, mtv.w, g1));
+          value_codes(acc, hwv, a0, a1, expo, neg);
+        } else if (tpos < p1) {
+          value_raw(acc, raw_row(u, tpos, D, true) + hf * 128, pt);
+        }
       }
     }
   }
@@ -550,7 +608,7 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   // gathers its selected positions into a list and processes them TPI at a
   // time, so the cost follows the number of selected tokens.
   if (q4) {
-    __syncthreads();  // mask_s complete
+    __syncwarp();  // the warp reads only the mask words its own lane 0 wrote
     int* my = lst + warp * kListCap;
     int nlist = 0;
     for (int bk = blk0 + warp; bk < qend; bk += kWarps) {
