@@ -157,6 +157,18 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def workload_text(wl, B):
+    """One-line description of the benched workload."""
+    k = wl.kinds
+    plan = "plan %d Q4 / %d Q2 / %d SHARE / %d BF16 cells" % (
+        (k == 0).sum(), (k == 1).sum(), (k == 2).sum(), (k == 3).sum())
+    ctx = ("%d cached tokens" % int(wl.lengths[0]) if len(set(wl.lengths[:B].tolist())) == 1
+           else "ragged %d-%d cached tokens" % (int(wl.lengths[:B].min()), int(wl.lengths[:B].max())))
+    return ("%s: %d loops x %d layers, %d KV heads, head dim %d, batch %d per GPU, %s + 1 "
+            "appended per step, %s, tau %g" % (wl.name, wl.n_loops, wl.n_layers, wl.n_heads,
+                                              wl.head_dim, B, ctx, plan, wl.tau))
+
+
 def shard_sequences(rank, batch):
     """Global sequence ids a rank serves: weak scaling, `batch` sequences per
     rank, disjoint across ranks (so every rank decodes different data)."""
@@ -462,10 +474,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "u2/u4 codes, fp32 accumulate", "data": "synthetic",
-            "config": {"workload": "batched-16k: 4 loops x 24 layers, 16 KV heads, head dim "
-                                   "128, batch %d per GPU, 16384 cached tokens + 1 appended "
-                                   "per step, plan loop3 Q4 / loops0-2 35%% Q4 35%% Q2 30%% "
-                                   "SHARE, tau 0.002" % B,
+            "config": {"workload": workload_text(wl, B),
                        "step": "append 1 token + decode, every cell, serving order",
                        "global_batch": B * world, "seq_len": int(n0[0]),
                        "parallelism": "dp%d (independent sequences)" % world,

@@ -409,7 +409,9 @@ __device__ __forceinline__ void low_planes(float2 (&acc)[32], const Unit& u, con
   __syncwarp();
 }
 
-template <int D>
+// DENSE_LO: tau <= 0, every 4-bit token takes its low plane (read densely in
+// the value loop); otherwise low planes come from the selected-position list.
+template <int D, bool DENSE_LO>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p, const CellList cl) {
   extern __shared__ __align__(16) float smem[];
@@ -549,6 +551,10 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   // i.e. + 1.5 * p * scale = 0.375 * (4 * p * scale) per unselected token
   const float hmul = q4 ? 4.f : 1.f;
   const float mid_unsel = q4 ? 0.375f : 0.f;
+  // tau <= 0 selects every 4-bit token: the low planes are read with the high
+  // ones in this loop instead of through the selected-position list
+  const bool dense_lo = DENSE_LO && q4;
+  const size_t lo_off = u.Ld.v_lo - u.Ld.v_hi;
   for (int bk = blk0 + warp; bk < blk1; bk += kWarps, vh += VSTEP, vm += VSTEP) {
     const int pos = bk * 32 + lane;
     const bool active = pos < p1;
@@ -582,6 +588,8 @@ decode_kernel(const DecodeParams p, const CellList cl) {
         g0 = fmaf(mid, a0, fmaf(pt, mt[it].y, g0));
         g1 = fmaf(mid, a1, fmaf(pt, mt[it].w, g1));
         value_codes(acc, hw[it], a0, a1, expo, neg);
+        if (dense_lo)
+          value_codes(acc, ld_stream(vh + lo_off + it * TPI * vrow), 0.25f * a0, 0.25f * a1, expo, neg);
       }
     } else {
       // partial block: quantized tokens below qlim, bf16 ones up to p1
@@ -598,6 +606,9 @@ decode_kernel(const DecodeParams p, const CellList cl) {
           g0 = fmaf(mid, a0, fmaf(pt, mtv.y, g0));
           g1 = fmaf(mid, a1, fmaf(pt, mtv.w, g1));
           value_codes(acc, hwv, a0, a1, expo, neg);
+          if (dense_lo)
+            value_codes(acc, ld_stream(vh + lo_off + it * TPI * vrow), 0.25f * a0, 0.25f * a1, expo,
+                        neg);
         } else if (tpos < p1) {
           value_raw(acc, raw_row(u, tpos, D, true) + hf * 128, pt);
         }
@@ -607,7 +618,7 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   // low planes of the selected tokens: acc += p * scale * lo.  The warp
   // gathers its selected positions into a list and processes them TPI at a
   // time, so the cost follows the number of selected tokens.
-  if (q4) {
+  if (q4 && !dense_lo) {
     __syncwarp();  // the warp reads only the mask words its own lane 0 wrote
     int* my = lst + warp * kListCap;
     int nlist = 0;
@@ -692,10 +703,10 @@ size_t decode_smem(int slots) {
   return sizeof(float) * (size_t)(D + 2 * kWarps * D + D + 64 + kWarps * kListCap + slots / 32 + slots);
 }
 
-template <int D>
+template <int D, bool DENSE_LO>
 int launch_decode_t(const DecodeParams& p, const CellList& cells, cudaStream_t stream) {
   const size_t smem = decode_smem<D>(p.slots);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, DENSE_LO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_cells * p.batch * p.n_heads;
@@ -715,7 +726,7 @@ int launch_decode_t(const DecodeParams& p, const CellList& cells, cudaStream_t s
   }
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<D>, p, cells);
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, DENSE_LO>, p, cells);
   return (int)e;
 }
 
@@ -726,8 +737,9 @@ int decode_max_split() { return kMaxSplit; }
 
 int launch_decode(const DecodeParams& p, const CellList& cells, void* stream, int head_dim) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (head_dim == 64) return launch_decode_t<64>(p, cells, s);
-  return launch_decode_t<128>(p, cells, s);
+  const bool dense = !(p.tau > 0.f);
+  if (head_dim == 64) return dense ? launch_decode_t<64, true>(p, cells, s) : launch_decode_t<64, false>(p, cells, s);
+  return dense ? launch_decode_t<128, true>(p, cells, s) : launch_decode_t<128, false>(p, cells, s);
 }
 
 }  // namespace loopkv
