@@ -12,10 +12,10 @@
 // workspace is needed.  The scores of the CTA's range stay in shared memory
 // between the two passes:
 //   pass 1  keys: per 32-token group, q is folded with the group's per-channel
-//           key scales (qs_d = q_d * scale_d) and zero points
-//           (c = sum_d q_d * zero_d), then each lane (one token) forms
-//           sum_d qs_d * code_d + c from its packed planes.  Scores are kept
-//           in log2 units.
+//           key scales into integer weights under one power of two, and
+//           integer tensor-core products (mma.sync, u8 codes x s8 weight
+//           digits) give sum_d qs_d * code_d exactly; the zero points add
+//           c = sum_d q_d * zero_d.  Scores are kept in log2 units.
 //   softmax the CTA's max and sum of exponentials, merged across the cluster
 //           into the unit's logsumexp.
 //   pass 2  values: lane = position computes p and the selection p >= tau
@@ -26,8 +26,8 @@
 //           token is loaded only when the token is selected.
 //   combine warp shuffles reduce the per-token partial outputs, shared
 //           memory reduces across warps, DSMEM across the cluster.
-// No tensor cores: one query per KV head makes this a stream over the
-// cache, bound by HBM bandwidth.
+// The value pass and the softmax run on the FMA / ALU pipes; the kernel as a
+// whole streams the cache once, bound by HBM bandwidth.
 
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
@@ -116,25 +116,6 @@ __device__ __forceinline__ void codes2_to_pairs(uint32_t w, uint32_t expo, float
 // Bit offset a two-bit code j of a word ends up at in codes2_to_pairs.
 __host__ __device__ constexpr int code2_off(int j) { return j < 6 ? 2 * j : 2 * (j - 6); }
 
-// Hi and lo planes of 16 four-bit codes -> 8 pairs (q_2m * 2^o(m), q_2m+1 *
-// 2^o(m)), q = 4hi + lo, o(m) = 4m for m < 3, 4(m-3) else.  The planes are
-// merged into a word of even codes (nibble m = code 2m) and one of odd codes.
-__device__ __forceinline__ void codes4_to_pairs(uint32_t hi, uint32_t lo, uint32_t expo,
-                                                float2 neg, float2 (&out)[8]) {
-  const uint32_t even = ((hi << 2) & 0xCCCCCCCCu) | (lo & 0x33333333u);
-  const uint32_t odd = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
-  const uint32_t eh = even >> 12, oh = odd >> 12;
-  out[0] = add2(make_float2(field_f<0, 4>(even, expo), field_f<0, 4>(odd, expo)), neg);
-  out[1] = add2(make_float2(field_f<4, 4>(even, expo), field_f<4, 4>(odd, expo)), neg);
-  out[2] = add2(make_float2(field_f<8, 4>(even, expo), field_f<8, 4>(odd, expo)), neg);
-  out[3] = add2(make_float2(field_f<0, 4>(eh, expo), field_f<0, 4>(oh, expo)), neg);
-  out[4] = add2(make_float2(field_f<4, 4>(eh, expo), field_f<4, 4>(oh, expo)), neg);
-  out[5] = add2(make_float2(field_f<8, 4>(eh, expo), field_f<8, 4>(oh, expo)), neg);
-  out[6] = add2(make_float2(field_f<12, 4>(eh, expo), field_f<12, 4>(oh, expo)), neg);
-  out[7] = add2(make_float2(field_f<16, 4>(eh, expo), field_f<16, 4>(oh, expo)), neg);
-}
-__host__ __device__ constexpr int code4_off(int m) { return m < 3 ? 4 * m : 4 * (m - 3); }
-
 // 2^-k as a float, k in [0, 126].
 __device__ __forceinline__ float pow2_neg(int k) { return __int_as_float((127 - k) << 23); }
 
@@ -214,140 +195,238 @@ __device__ __forceinline__ float dot_bf16(const uint8_t* row, const float* q_s) 
   return acc;
 }
 
-// Score of one quantized token: sum_d qs_d * code_d over the token's packed
-// planes (16-byte rows h[c], l[c] of K_hi / K_lo for chunk c of 64 channels).
-template <int D, bool Q4>
-__device__ __forceinline__ float dot_codes(const uint4 (&h)[D / 64], const uint4 (&l)[D / 64],
-                                           const float2* qs2, uint32_t expo, float2 neg) {
-  // four independent accumulators keep the fma chain short
-  float2 acc[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int c = 0; c < D / 64; ++c) {
-    const uint32_t hw[4] = {h[c].x, h[c].y, h[c].z, h[c].w};
-    const uint32_t lw[4] = {l[c].x, l[c].y, l[c].z, l[c].w};
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      float2 v[8];
-      if (Q4) codes4_to_pairs(hw[w], lw[w], expo, neg, v);
-      else codes2_to_pairs(hw[w], expo, neg, v);
-      const float4* q4p = reinterpret_cast<const float4*>(qs2 + 32 * c + 8 * w);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 qq = q4p[i];
-        acc[(2 * i) & 3] = fma2(make_float2(qq.x, qq.y), v[2 * i], acc[(2 * i) & 3]);
-        acc[(2 * i + 1) & 3] = fma2(make_float2(qq.z, qq.w), v[2 * i + 1], acc[(2 * i + 1) & 3]);
-      }
-    }
-  }
-  const float2 a = add2(acc[0], acc[1]), b = add2(acc[2], acc[3]);
-  return (a.x + b.x) + (a.y + b.y);
+// ---------------------------------------------------------------- keys
+//
+// Key scores with integer tensor-core products (mma.sync m16n8k32, u8 x s8,
+// s32 accumulate).  For a 32-token group the folded weights qs_d = q_d *
+// scale_d share one power of two 2^E chosen from the group's largest |qs|,
+// W_d = rint(qs_d * 2^E) with |W_d| < 2^26, so sum_d W_d * code_d is exact
+// in integers and the score is that sum * 2^-E + sum_d q_d * zero_d.
+//
+// A operand (16 tokens x 32 bytes): the hi / lo planes of a 16-channel word
+// merge into two nibble words (even channels, odd channels); a byte of a
+// nibble word holds two codes, c_lo + 16 c_hi.  Two products cover both
+// codes without unpacking them: A_X = the nibble word against X = W(c_lo's
+// channel), A_Y = (nibble word & 0xF0F0F0F0) = 16 c_hi against
+// Y = W(c_hi's channel) - 16 W(c_lo's channel); then
+//   A_X . X + (A_Y . Y) / 16 = sum c_lo W_lo + sum c_hi W_hi.
+// B operand (32 bytes x 8 columns): X and Y as four signed base-256 digits
+// each, X's digits in columns 0-3 and Y's in columns 4-7; the X product
+// sees Y's columns as zero and the Y product X's, so both accumulate into
+// one fragment.  Digits: b_p = byte p of (W + 0x80808080) read as u8, minus
+// 128 (exact for |W| < 0x7F7F7F7F).
+//
+// Lane (g, t) = (lane / 4, lane % 4) holds tokens g + 8j (j = 0..3) of the
+// group: M tile j / 2, row g or g + 8.  K tile kt takes from lane t the
+// plane word w = (D / 64) t + kt of each of its tokens (16 channels), so a
+// K tile is 64 channels and a lane's words are contiguous in a row.
+
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Per-lane load of one 32-token key group: the lane's token rows of the
-// planes and the lane's D/32 channels of the group's scale / zero point.
+__device__ __forceinline__ uint2 ld_stream2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_stream1(const void* p) {
+  uint32_t r;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+
+// One lane's share of a 32-token key group.
 template <int D>
-struct KGroup {
-  uint4 h[D / 64], l[D / 64];
-  float sc[D / 32], zr[D / 32];
+struct KTile {
+  uint32_t h[4][D / 64], l[4][D / 64];  // token g + 8j: the lane's plane words
+  float4 sc, zr;                        // scale / zero of channels 4 lane .. 4 lane + 3
 };
 
-// Lane pointers into one group: kh -> the lane's K_hi row of chunk 0,
-// lo_off -> K_lo - K_hi, km -> the lane's scales (zeros D floats further).
+// kb -> the lane's K_hi words of token g; lo_off = K_lo - K_hi; km -> the
+// lane's four scales (zeros D floats further); meta: the lane folds channels.
 template <int D, bool Q4>
-__device__ __forceinline__ void load_kgroup(KGroup<D>& g, const uint8_t* kh, size_t lo_off,
-                                            const float* km) {
+__device__ __forceinline__ void load_ktile(KTile<D>& k, const uint8_t* kb, size_t lo_off,
+                                           const float* km, bool meta) {
 #pragma unroll
-  for (int c = 0; c < D / 64; ++c) {
-    g.h[c] = ld_stream(kh + c * 512);
-    g.l[c] = Q4 ? ld_stream(kh + lo_off + c * 512) : make_uint4(0, 0, 0, 0);
+  for (int j = 0; j < 4; ++j) {
+    if constexpr (D == 128) {
+      const uint2 hw = ld_stream2(kb + j * 128);
+      k.h[j][0] = hw.x; k.h[j][1] = hw.y;
+      if (Q4) {
+        const uint2 lw = ld_stream2(kb + lo_off + j * 128);
+        k.l[j][0] = lw.x; k.l[j][1] = lw.y;
+      } else {
+        k.l[j][0] = 0u; k.l[j][1] = 0u;
+      }
+    } else {
+      k.h[j][0] = ld_stream1(kb + j * 128);
+      k.l[j][0] = Q4 ? ld_stream1(kb + lo_off + j * 128) : 0u;
+    }
   }
-  if constexpr (D == 128) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(km));
-    const float4 z = __ldg(reinterpret_cast<const float4*>(km + D));
-    g.sc[0] = a.x; g.sc[1] = a.y; g.sc[2] = a.z; g.sc[3] = a.w;
-    g.zr[0] = z.x; g.zr[1] = z.y; g.zr[2] = z.z; g.zr[3] = z.w;
+  if (meta) {
+    k.sc = __ldg(reinterpret_cast<const float4*>(km));
+    k.zr = __ldg(reinterpret_cast<const float4*>(km + D));
   } else {
-    const float2 a = __ldg(reinterpret_cast<const float2*>(km));
-    const float2 z = __ldg(reinterpret_cast<const float2*>(km + D));
-    g.sc[0] = a.x; g.sc[1] = a.y;
-    g.zr[0] = z.x; g.zr[1] = z.y;
+    k.sc = make_float4(0.f, 0.f, 0.f, 0.f);
+    k.zr = k.sc;
   }
 }
 
-// Score one group held in registers; returns the lane's score (or -inf).
+// Nibble words of a 16-channel plane word: byte b of `ev` holds the codes of
+// channels 4b (low nibble) and 4b + 2 (high), byte b of `od` channels 4b + 1
+// and 4b + 3.  q = 4 hi + lo for 4-bit keys, q = hi for 2-bit keys.
+template <bool Q4>
+__device__ __forceinline__ void nibble_words(uint32_t hi, uint32_t lo, uint32_t& ev, uint32_t& od) {
+  if (Q4) {
+    ev = ((hi << 2) & 0xCCCCCCCCu) | (lo & 0x33333333u);
+    od = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
+  } else {
+    ev = hi & 0x33333333u;
+    od = (hi >> 2) & 0x33333333u;
+  }
+}
+
+// Scores one group; stores the scores of positions below qlim into sc and
+// returns their max.  stage: the warp's 64 * (D / 64) ints of staging.
 template <int D, bool Q4>
-__device__ __forceinline__ float key_group(const KGroup<D>& g, const float (&qv)[D / 32],
-                                           const float (&qz)[D / 32], float* qs, int pos,
-                                           int qlim, float sscale, uint32_t expo, float2 neg,
-                                           int lane) {
-  constexpr int CPL = D / 32;
-  // fold q into the group's key scale / zero point
-  float cpart = 0.f;
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) {
-    qs[CPL * lane + i] = qv[i] * g.sc[i];
-    cpart = fmaf(qz[i], g.zr[i], cpart);
+__device__ __forceinline__ float key_group(const KTile<D>& k, float4 qv, int* stage, int gpos0,
+                                           int qlim, int p0, float* sc, float sscale, int lane) {
+  constexpr int KT = D / 64;
+  const int g = lane >> 2, t = lane & 3;
+  // fold q into the scales; the zero-point term
+  const float q0 = qv.x * k.sc.x, q1 = qv.y * k.sc.y, q2 = qv.z * k.sc.z, q3 = qv.w * k.sc.w;
+  float cpart = fmaf(qv.w, k.zr.w, fmaf(qv.z, k.zr.z, fmaf(qv.y, k.zr.y, qv.x * k.zr.x)));
+  // the group's power of two: max|qs| * F < 2^26
+  const float amax = fmaxf(fmaxf(fabsf(q0), fabsf(q1)), fmaxf(fabsf(q2), fabsf(q3)));
+  const uint32_t mbits = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+  const int fexp = min(279 - (int)(mbits >> 23), 253);
+  const float F = __int_as_float(fexp << 23);
+  const float Finv = __int_as_float((254 - fexp) << 23);
+  const int w0 = __float2int_rn(q0 * F), w1 = __float2int_rn(q1 * F);
+  const int w2 = __float2int_rn(q2 * F), w3 = __float2int_rn(q3 * F);
+  if (lane < D / 4) {
+    // channels 4 lane + {0,1,2,3}: byte (lane % 4) of plane word lane / 4
+    const int w = lane >> 2, b = lane & 3;
+    const int base = (w % KT) * 16 + (w / KT) * 4 + b;
+    constexpr uint32_t kBias = 0x80808080u;
+    stage[base] = (int)((uint32_t)w0 + kBias);                       // X, even word
+    stage[base + 16 * KT] = (int)((uint32_t)(w2 - 16 * w0) + kBias);  // Y, even word
+    stage[base + 32 * KT] = (int)((uint32_t)w1 + kBias);             // X, odd word
+    stage[base + 48 * KT] = (int)((uint32_t)(w3 - 16 * w1) + kBias);  // Y, odd word
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o);
   __syncwarp();
-  float s = -INFINITY;
-  if (pos < qlim) {
-    const float dot = dot_codes<D, Q4>(g.h, g.l, reinterpret_cast<const float2*>(qs), expo, neg);
-    s = (dot + cpart) * sscale;
+  // B fragments: column g, bytes k = 4t..4t+3 (b0) and 16+4t.. (b1)
+  const uint32_t pl = (uint32_t)(g & 3);
+  const uint32_t selp = pl | ((pl + 4u) << 4) | (pl << 8) | ((pl + 4u) << 12);
+  const uint32_t mx = g < 4 ? 0xFFFFFFFFu : 0u;
+  uint32_t bx[KT][2], by[KT][2];
+#pragma unroll
+  for (int kt = 0; kt < KT; ++kt) {
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      const int4 iv = *reinterpret_cast<const int4*>(
+          stage + ((part * 2 + (g >> 2)) * KT + kt) * 16 + t * 4);
+      const uint32_t lo2 = __byte_perm((uint32_t)iv.x, (uint32_t)iv.y, selp);
+      const uint32_t hi2 = __byte_perm((uint32_t)iv.z, (uint32_t)iv.w, selp);
+      const uint32_t dg = __byte_perm(lo2, hi2, 0x5410u) ^ 0x80808080u;
+      bx[kt][part] = dg & mx;
+      by[kt][part] = dg & ~mx;
+    }
   }
-  __syncwarp();
-  return s;
+  // products: fragment j / 2 holds tokens g + 8 (j & ~1) and g + 8 (j | 1)
+  int acc[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[mt][i] = 0;
+#pragma unroll
+    for (int kt = 0; kt < KT; ++kt) {
+      uint32_t e0, o0, e1, o1;
+      nibble_words<Q4>(k.h[2 * mt][kt], k.l[2 * mt][kt], e0, o0);
+      nibble_words<Q4>(k.h[2 * mt + 1][kt], k.l[2 * mt + 1][kt], e1, o1);
+      mma_u8s8(acc[mt], e0, e1, o0, o1, bx[kt][0], bx[kt][1]);
+      mma_u8s8(acc[mt], e0 & 0xF0F0F0F0u, e1 & 0xF0F0F0F0u, o0 & 0xF0F0F0F0u, o1 & 0xF0F0F0F0u,
+               by[kt][0], by[kt][1]);
+    }
+  }
+  // lane t holds digit columns 2t, 2t+1: X digits 0-1, 2-3 (t = 0, 1), Y
+  // digits 0-1, 2-3 (t = 2, 3); weight them and sum over the quad
+  const float fac = (t == 0) ? 1.f : (t == 1) ? 65536.f : (t == 2) ? 0.0625f : 4096.f;
+  float r[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int* c = acc[j >> 1] + 2 * (j & 1);
+    r[j] = (float)(c[0] + (c[1] << 8)) * fac;
+  }
+  // reduce-scatter over the quad: lane t ends with row rho(t) = {0, 2, 1, 3}[t]
+  const bool odd = t & 1;
+  float k0 = odd ? r[2] : r[0], k1 = odd ? r[3] : r[1];
+  const float s0 = odd ? r[0] : r[2], s1 = odd ? r[1] : r[3];
+  k0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+  k1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+  const bool up = t & 2;
+  float tot = up ? k1 : k0;
+  tot += __shfl_xor_sync(0xffffffffu, up ? k0 : k1, 2);
+  const int rho = (odd ? 2 : 0) + (up ? 1 : 0);
+  const int pos = gpos0 + g + 8 * rho;
+  float lmax = -INFINITY;
+  if (pos < qlim) {
+    const float s = fmaf(tot, Finv * sscale, cpart * sscale);
+    sc[pos - p0] = s;
+    lmax = s;
+  }
+  return lmax;
 }
 
 // Pass 1 over the CTA's quantized key groups [b_begin, b_end), warp-strided.
 // Two register buffers alternate, so the next group's loads are in flight
-// while the current one is scored, without copies between them.
+// while the current one is scored.  Staging alternates between two halves
+// of the warp's area so one __syncwarp per group suffices.
 template <int D, bool Q4>
 __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end, int p0, int p1,
-                                          const float* q_s, float* qs, float* sc, float sscale,
-                                          uint32_t expo, float2 neg, int warp, int lane) {
-  constexpr int CPL = D / 32;  // channels per lane for the q fold
+                                          const float* q_s, int* stage, float* sc, float sscale,
+                                          int warp, int lane) {
   float lmax = -INFINITY;
   const int first = b_begin + warp;
   if (first >= b_end) return lmax;
-  // q of the lane's channels, times 2^-o: o is the bit offset the channel's
-  // code keeps after conversion (see codes4_to_pairs / codes2_to_pairs)
-  float qv[CPL], qz[CPL];
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) {
-    const int j = (CPL * lane + i) & 15;
-    qz[i] = q_s[CPL * lane + i];
-    qv[i] = qz[i] * pow2_neg(Q4 ? code4_off(j >> 1) : code2_off(j));
-  }
+  const bool meta = lane < D / 4;
+  const float4 qv = meta ? *reinterpret_cast<const float4*>(q_s + 4 * lane)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
   const int qlim = min(p1, u.nq);
-  constexpr size_t G = 8 * D;                       // bytes of one group in each block
-  constexpr size_t STEP = (size_t)kWarps * G;       // a warp's stride between its groups
-  const uint8_t* kh = u.data + u.Ld.k_hi + (size_t)first * G + lane * 16;
+  const int g = lane >> 2, t = lane & 3;
+  constexpr size_t G = 8 * D;                  // bytes of one group in each block
+  constexpr size_t STEP = (size_t)kWarps * G;  // a warp's stride between its groups
+  constexpr int SH = 64 * (D / 64);            // ints of one staging half
+  const size_t lane_off = (D == 128) ? (size_t)(t >> 1) * 512 + g * 16 + (t & 1) * 8
+                                     : (size_t)g * 16 + t * 4;
+  const uint8_t* kb = u.data + u.Ld.k_hi + (size_t)first * G + lane_off;
   const size_t lo_off = u.Ld.k_lo - u.Ld.k_hi;
   const float* km = reinterpret_cast<const float*>(u.data + u.Ld.k_meta + (size_t)first * G) +
-                    CPL * lane;
-  KGroup<D> a, b;
-  load_kgroup<D, Q4>(a, kh, lo_off, km);
+                    (meta ? 4 * lane : 0);
+  KTile<D> a, b;
+  load_ktile<D, Q4>(a, kb, lo_off, km, meta);
   int bk = first;
   for (;;) {
     const bool hasb = bk + kWarps < b_end;
-    if (hasb) load_kgroup<D, Q4>(b, kh + STEP, lo_off, km + STEP / 4);
-    float s = key_group<D, Q4>(a, qv, qz, qs, bk * 32 + lane, qlim, sscale, expo, neg, lane);
-    if (bk * 32 + lane < qlim) { sc[bk * 32 + lane - p0] = s; lmax = fmaxf(lmax, s); }
+    if (hasb) load_ktile<D, Q4>(b, kb + STEP, lo_off, km + STEP / 4, meta);
+    lmax = fmaxf(lmax, key_group<D, Q4>(a, qv, stage, bk * 32, qlim, p0, sc, sscale, lane));
     if (!hasb) break;
     bk += kWarps;
-    kh += STEP;
+    kb += STEP;
     km += STEP / 4;
     const bool hasa = bk + kWarps < b_end;
-    if (hasa) load_kgroup<D, Q4>(a, kh + STEP, lo_off, km + STEP / 4);
-    s = key_group<D, Q4>(b, qv, qz, qs, bk * 32 + lane, qlim, sscale, expo, neg, lane);
-    if (bk * 32 + lane < qlim) { sc[bk * 32 + lane - p0] = s; lmax = fmaxf(lmax, s); }
+    if (hasa) load_ktile<D, Q4>(a, kb + STEP, lo_off, km + STEP / 4, meta);
+    lmax = fmaxf(lmax, key_group<D, Q4>(b, qv, stage + SH, bk * 32, qlim, p0, sc, sscale, lane));
     if (!hasa) break;
     bk += kWarps;
-    kh += STEP;
+    kb += STEP;
     km += STEP / 4;
   }
   return lmax;
@@ -416,8 +495,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p, const CellList cl) {
   extern __shared__ __align__(16) float smem[];
   float* q_s = smem;                                  // [D]
-  float* qs_all = q_s + D;                            // [kWarps][D]
-  float* red = qs_all + kWarps * D;                   // [kWarps][D]
+  float* kstage = q_s + D;                            // [kWarps][D] key-weight staging, pass 1
+  float* red = kstage + kWarps * D;                   // [kWarps][D] (pass 1 staging continues here)
   float* o_s = red + kWarps * D;                      // [D]
   float* misc = o_s + D;                              // [64]
   int* lst = reinterpret_cast<int*>(misc + 64);       // [kWarps][kListCap] selected positions
@@ -459,7 +538,7 @@ decode_kernel(const DecodeParams p, const CellList cl) {
 
   const bool quant = u.data_kind == LOOPKV_Q4 || u.data_kind == LOOPKV_Q2;
   const bool q4 = u.data_kind == LOOPKV_Q4;
-  float* qs = qs_all + warp * D;
+  int* stage = reinterpret_cast<int*>(kstage) + warp * 2 * D;  // 2 D ints per warp
   const float sscale = p.score_scale;
   const int blk0 = p0 / 32;
   const int blk1 = (p1 + 31) / 32;
@@ -470,9 +549,8 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   float lmax = -INFINITY;
   const uint32_t expo = p.code_expo;
   const float2 neg = make_float2(p.code_neg, p.code_neg);
-  if (q4) lmax = key_pass<D, true>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, expo, neg, warp, lane);
-  else if (quant)
-    lmax = key_pass<D, false>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, expo, neg, warp, lane);
+  if (q4) lmax = key_pass<D, true>(u, blk0, qend, p0, p1, q_s, stage, sc, sscale, warp, lane);
+  else if (quant) lmax = key_pass<D, false>(u, blk0, qend, p0, p1, q_s, stage, sc, sscale, warp, lane);
   // the warp's first value block is requested now, ahead of the softmax merge
   constexpr int LPT = D / 64;       // lanes per token in pass 2 (64 channels per lane)
   constexpr int TPI = 32 / LPT;     // tokens per warp iteration in pass 2
