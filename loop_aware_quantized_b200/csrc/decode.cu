@@ -18,16 +18,18 @@
 //           c = sum_d q_d * zero_d.  Scores are kept in log2 units.
 //   softmax the CTA's max and sum of exponentials, merged across the cluster
 //           into the unit's logsumexp.
-//   pass 2  values: lane = position computes p and the selection p >= tau
-//           (a warp ballot gives the mask word of the group); lanes then
-//           work per token (64 channels per lane) accumulating
-//           p * scale * code in fp32 and the per-group constant
-//           p * (zero [+ 1.5 * scale]) separately; the low plane row of a
-//           token is loaded only when the token is selected.
+//   pass 2  values: p and the selection p >= tau per block (a warp ballot
+//           gives the mask word); the high planes of the quantized blocks
+//           go through integer tensor-core products against the weights
+//           hmul * p * scale (channel-major planes, contraction over
+//           tokens), the per-group constants p * (zero [+ 1.5 * scale])
+//           are summed in fp32; the low planes of the selected tokens and
+//           the bf16 positions are accumulated in fp32, lane = 64 channels
+//           of a token, so a low-plane row is read only when selected.
 //   combine warp shuffles reduce the per-token partial outputs, shared
 //           memory reduces across warps, DSMEM across the cluster.
-// The value pass and the softmax run on the FMA / ALU pipes; the kernel as a
-// whole streams the cache once, bound by HBM bandwidth.
+// The kernel streams the cache once: HBM bandwidth and memory latency bound
+// it, with the per-code arithmetic on the tensor cores.
 
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
@@ -240,6 +242,18 @@ __device__ __forceinline__ uint32_t ld_stream1(const void* p) {
   return r;
 }
 
+// Streams run ahead of use: the next group of a warp is loaded into
+// registers while the current one is processed, and the group kAheadK /
+// kAheadV groups ahead (0: none) is requested into L2, one 128-byte line per
+// lane; kPreV value groups of each warp are requested before the softmax.
+constexpr int kAheadK = 1;
+constexpr int kAheadV = 1;
+constexpr int kPreV = 2;
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // One lane's share of a 32-token key group.
 template <int D>
 struct KTile {
@@ -410,12 +424,20 @@ __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end,
   const size_t lo_off = u.Ld.k_lo - u.Ld.k_hi;
   const float* km = reinterpret_cast<const float*>(u.data + u.Ld.k_meta + (size_t)first * G) +
                     (meta ? 4 * lane : 0);
+  // L2 prefetch: lane -> line (lane % (D / 16)) of block K_hi, K_lo or K_meta
+  constexpr int LINES = D / 16;
+  const int pblk = lane / LINES;
+  const bool pon = pblk < (Q4 ? 3 : 2);
+  const uint8_t* pf = u.data + (pblk == 0 ? u.Ld.k_hi : (Q4 && pblk == 1) ? u.Ld.k_lo : u.Ld.k_meta) +
+                      (size_t)(lane % LINES) * 128;
   KTile<D> a, b;
   load_ktile<D, Q4>(a, kb, lo_off, km, meta);
   int bk = first;
   for (;;) {
     const bool hasb = bk + kWarps < b_end;
     if (hasb) load_ktile<D, Q4>(b, kb + STEP, lo_off, km + STEP / 4, meta);
+    if (kAheadK > 0 && pon && bk + kAheadK * kWarps < b_end)
+      prefetch_l2(pf + (size_t)(bk + kAheadK * kWarps) * G);
     lmax = fmaxf(lmax, key_group<D, Q4>(a, qv, stage, bk * 32, qlim, p0, sc, sscale, lane));
     if (!hasb) break;
     bk += kWarps;
@@ -423,6 +445,8 @@ __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end,
     km += STEP / 4;
     const bool hasa = bk + kWarps < b_end;
     if (hasa) load_ktile<D, Q4>(a, kb + STEP, lo_off, km + STEP / 4, meta);
+    if (kAheadK > 0 && pon && bk + kAheadK * kWarps < b_end)
+      prefetch_l2(pf + (size_t)(bk + kAheadK * kWarps) * G);
     lmax = fmaxf(lmax, key_group<D, Q4>(b, qv, stage + SH, bk * 32, qlim, p0, sc, sscale, lane));
     if (!hasa) break;
     bk += kWarps;
@@ -488,9 +512,217 @@ __device__ __forceinline__ void low_planes(float2 (&acc)[32], const Unit& u, con
   __syncwarp();
 }
 
-// DENSE_LO: tau <= 0, every 4-bit token takes its low plane (read densely in
-// the value loop); otherwise low planes come from the selected-position list.
-template <int D, bool DENSE_LO>
+// ---------------------------------------------------------------- values
+//
+// High planes of the quantized value blocks on the tensor cores
+// (mma.sync m16n8k16, u8 x s8, s32 accumulate):
+//   out_c += sum_T a_{T,G} * hi_{T,c},  a_{T,G} = hmul * p_T * scale_{T,G},
+// G = c / 32 the channel's value group.  M = 16 channels, K = 16 bytes = the
+// 32 tokens of a group (two codes per byte), N = 8 digit columns.  Lane
+// (g, t) supplies channels 8i + g (i = 0..D/8-1) of tokens 16 (t >> 1) ..
+// 16 (t >> 1) + 15, whose words are contiguous in the group's channel-major
+// block.  Even t takes the codes at bits 0-1 / 4-5 of each byte (tokens 4b
+// and 4b + 2 of the half), odd t those at bits 2-3 / 6-7 (tokens 4b + 1 and
+// 4b + 3, at four times their value); the weights of even-t bytes carry the
+// factor 4 instead, so every product comes out 4x and no code is shifted.
+// Byte k = 4t + b pairs tokens T_lo = 16 (t >> 1) + 4b + (t & 1) and
+// T_hi = T_lo + 2, with X = w(T_lo), Y = w(T_hi) - 16 w(T_lo) as for the keys.
+//
+// The integer weights share one power of two per channel group for the whole
+// pass, so the products accumulate in int32 across groups.  It is chosen from
+// hmul * f * max(scale) of the first group (p <= f for every token) with two
+// bits of headroom, and chosen again, after folding the accumulators into
+// fp32, only when a later group's weights outgrow it.
+
+__device__ __forceinline__ void mma16_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm("mma.sync.aligned.m16n8k16.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+// One lane's share of a 32-token value group.
+template <int D>
+struct VTile {
+  uint4 w[D / 32];  // high-plane words i = 0..D/8-1 (channel 8i + g)
+  float4 m[D / 64];  // meta row of token `lane`: (scale, zero) x D/32
+};
+
+template <int D>
+__device__ __forceinline__ void load_vtile(VTile<D>& v, const uint8_t* vh, const float* vm) {
+#pragma unroll
+  for (int i = 0; i < D / 32; ++i) v.w[i] = ld_stream(vh + 16 * i);
+#pragma unroll
+  for (int i = 0; i < D / 64; ++i) v.m[i] = __ldg(reinterpret_cast<const float4*>(vm) + i);
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4& q, int j) {
+  return j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w;
+}
+
+// The lane's 128-byte line of group 0 for L2 prefetches of the value high
+// plane (lanes 0 .. D/16 - 1) and value meta (the next D/16 lanes), else null;
+// group i's line is 8 D i bytes further.
+template <int D>
+__device__ __forceinline__ const uint8_t* vgroup_line(const Unit& u, int lane) {
+  constexpr int LINES = D / 16;
+  if (lane >= 2 * LINES) return nullptr;
+  return u.data + (lane < LINES ? u.Ld.v_hi : u.Ld.v_meta) + (size_t)(lane % LINES) * 128;
+}
+
+// Pass over the warp's quantized blocks [b_begin, b_end) (warp-strided).
+// vo[G]: lane (g, t)'s total for channel 32 G + 8 t + g (scaled by 2^o = 1);
+// cst[G]: the lane's share (token = lane) of sum_T p_T (zero + mid scale).
+template <int D>
+__device__ __forceinline__ void value_high_pass(const Unit& u, int b_begin, int b_end, int p0,
+                                                int qlim, int blk0, const float* sc,
+                                                const uint32_t* mask_s, float f, float hmul,
+                                                float mid_unsel, int* stage, float (&vo)[D / 32],
+                                                float (&cst)[D / 32], int warp, int lane) {
+  constexpr int NG = D / 32;
+  const int first = b_begin + warp;
+  if (first >= b_end) return;
+  const int g = lane >> 2, t = lane & 3;
+  // consumer side: operand masks, B column digit, digit weights of columns 2t, 2t+1
+  const uint32_t m1 = (t & 1) ? 0xCCCCCCCCu : 0x33333333u;
+  const uint32_t m2 = (t & 1) ? 0xC0C0C0C0u : 0x30303030u;
+  const uint32_t pl = (uint32_t)(g & 3);
+  const uint32_t selp = pl | ((pl + 4u) << 4) | (pl << 8) | ((pl + 4u) << 12);
+  const uint32_t mx = g < 4 ? 0xFFFFFFFFu : 0u;
+  const float fac = ((t == 0) ? 1.f : (t == 1) ? 65536.f : (t == 2) ? 0.0625f : 4096.f) * 0.25f;
+  // producer side: lane = token T; T_lo lanes (T % 4 < 2) stage the X / Y pair
+  const float mtok = (lane & 1) ? 1.f : 4.f;
+  const float hm = hmul * mtok;
+  const float mid_m = mid_unsel / mtok;
+  const bool tlo = (lane & 2) == 0;
+  const int kslot = (2 * (lane >> 4) + (lane & 1)) * 4 + ((lane >> 2) & 3);
+  constexpr uint32_t kBias = 0x80808080u;
+
+  int acc[NG][2][4];
+#pragma unroll
+  for (int G = 0; G < NG; ++G)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[G][i >> 2][i & 3] = 0;
+  float F[NG];
+#pragma unroll
+  for (int G = 0; G < NG; ++G) F[G] = 0.f;
+  bool fresh = true;
+
+  auto flush = [&]() {
+#pragma unroll
+    for (int G = 0; G < NG; ++G) {
+      const float sG = fac * __int_as_float((254 - (int)(__float_as_uint(F[G]) >> 23)) << 23);
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float x = fmaf((float)acc[G][mt][2 * h + 1], 256.f, (float)acc[G][mt][2 * h]) * sG;
+          x += __shfl_xor_sync(0xffffffffu, x, 1);
+          x += __shfl_xor_sync(0xffffffffu, x, 2);
+          if (2 * mt + h == t) vo[G] += x;
+          acc[G][mt][2 * h] = 0;
+          acc[G][mt][2 * h + 1] = 0;
+        }
+      }
+    }
+  };
+
+  auto body = [&](const VTile<D>& v, int bk, int* st) {
+    const int pos = bk * 32 + lane;
+    const bool valid = pos < qlim;
+    const float pw = valid ? sc[pos - p0] * f : 0.f;
+    const bool sel = (mask_s[bk - blk0] >> lane) & 1u;
+    const float hp = hm * pw;
+    const float mid = sel ? 0.f : mid_m;
+    float a[NG];
+    int w[NG];
+    int wmax = 0;
+#pragma unroll
+    for (int G = 0; G < NG; ++G) {
+      const float4 mm = v.m[G >> 1];
+      const float s = (G & 1) ? mm.z : mm.x, z = (G & 1) ? mm.w : mm.y;
+      a[G] = hp * s;
+      cst[G] = fmaf(mid, a[G], fmaf(pw, z, cst[G]));
+      w[G] = __float2int_rn(a[G] * F[G]);
+      wmax = max(wmax, w[G]);
+    }
+    if (__any_sync(0xffffffffu, fresh || wmax >= (1 << 26))) {
+      if (!fresh) flush();
+#pragma unroll
+      for (int G = 0; G < NG; ++G) {
+        const float4 mm = v.m[G >> 1];
+        const float s = valid ? ((G & 1) ? mm.z : mm.x) : 0.f;
+        const uint32_t smax = __reduce_max_sync(0xffffffffu, __float_as_uint(s));
+        const float x = hmul * f * __uint_as_float(smax);
+        const int fexp = min(275 - (int)(__float_as_uint(x) >> 23), 253);
+        F[G] = __int_as_float(fexp << 23);
+        w[G] = __float2int_rn(a[G] * F[G]);
+      }
+      fresh = false;
+    }
+#pragma unroll
+    for (int G = 0; G < NG; ++G) {
+      const int wp = __shfl_down_sync(0xffffffffu, w[G], 2);
+      if (tlo) {
+        st[G * 32 + kslot] = (int)((uint32_t)w[G] + kBias);
+        st[G * 32 + 16 + kslot] = (int)((uint32_t)(wp - 16 * w[G]) + kBias);
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int G = 0; G < NG; ++G) {
+      const int4 iv = *reinterpret_cast<const int4*>(st + G * 32 + (g >> 2) * 16 + 4 * t);
+      const uint32_t lo2 = __byte_perm((uint32_t)iv.x, (uint32_t)iv.y, selp);
+      const uint32_t hi2 = __byte_perm((uint32_t)iv.z, (uint32_t)iv.w, selp);
+      const uint32_t dg = __byte_perm(lo2, hi2, 0x5410u) ^ 0x80808080u;
+      const uint32_t bx = dg & mx, by = dg & ~mx;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int i0 = 4 * G + 2 * mt;
+        const uint32_t w0 = word_of(v.w[i0 >> 2], i0 & 3);
+        const uint32_t w1 = word_of(v.w[i0 >> 2], (i0 & 3) + 1);
+        mma16_u8s8(acc[G][mt], w0 & m1, w1 & m1, bx);
+        mma16_u8s8(acc[G][mt], w0 & m2, w1 & m2, by);
+      }
+    }
+  };
+
+  constexpr size_t GB = 8 * D;                        // bytes of a group's high-plane block
+  constexpr size_t VSTEP = (size_t)kWarps * GB;       // a warp's stride between its groups
+  constexpr size_t MSTEP = (size_t)kWarps * 32 * (D / 16);  // same, in meta floats
+  const uint8_t* vh = u.data + u.Ld.v_hi + (size_t)first * GB + (size_t)(g * 2 + (t >> 1)) * (D / 2);
+  const float* vm = reinterpret_cast<const float*>(u.data + u.Ld.v_meta) +
+                    ((size_t)first * 32 + lane) * (D / 16);
+  const uint8_t* pf = vgroup_line<D>(u, lane);
+  VTile<D> va, vb;
+  load_vtile<D>(va, vh, vm);
+  int bk = first;
+  for (;;) {
+    const bool hasb = bk + kWarps < b_end;
+    if (hasb) load_vtile<D>(vb, vh + VSTEP, vm + MSTEP);
+    if (kAheadV > 0 && pf != nullptr && bk + kAheadV * kWarps < b_end)
+      prefetch_l2(pf + (size_t)(bk + kAheadV * kWarps) * GB);
+    body(va, bk, stage);
+    if (!hasb) break;
+    bk += kWarps;
+    vh += VSTEP;
+    vm += MSTEP;
+    const bool hasa = bk + kWarps < b_end;
+    if (hasa) load_vtile<D>(va, vh + VSTEP, vm + MSTEP);
+    if (kAheadV > 0 && pf != nullptr && bk + kAheadV * kWarps < b_end)
+      prefetch_l2(pf + (size_t)(bk + kAheadV * kWarps) * GB);
+    body(vb, bk, stage + NG * 32);
+    if (!hasa) break;
+    bk += kWarps;
+    vh += VSTEP;
+    vm += MSTEP;
+  }
+  flush();
+}
+
+// tau <= 0 selects every 4-bit token: the low-plane list pass then covers
+// them all.
+template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p, const CellList cl) {
   extern __shared__ __align__(16) float smem[];
@@ -551,25 +783,12 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   const float2 neg = make_float2(p.code_neg, p.code_neg);
   if (q4) lmax = key_pass<D, true>(u, blk0, qend, p0, p1, q_s, stage, sc, sscale, warp, lane);
   else if (quant) lmax = key_pass<D, false>(u, blk0, qend, p0, p1, q_s, stage, sc, sscale, warp, lane);
-  // the warp's first value block is requested now, ahead of the softmax merge
-  constexpr int LPT = D / 64;       // lanes per token in pass 2 (64 channels per lane)
-  constexpr int TPI = 32 / LPT;     // tokens per warp iteration in pass 2
-  const int hf = lane % LPT;
-  const size_t vrow = D / 4;  // bytes per token of a value plane / value meta
-  const int qlim = min(p1, u.nq);
-  const size_t row0 = ((size_t)(blk0 + warp) * 32 + lane / LPT) * vrow + hf * 16;
-  const uint8_t* vh = u.data + u.Ld.v_hi + row0;
-  const uint8_t* vm = u.data + u.Ld.v_meta + row0;
-  constexpr size_t VSTEP = (size_t)kWarps * 32 * (D / 4);
-  auto full_block = [&](int bk) { return (bk + 1) * 32 <= qlim; };
-  uint4 nh[LPT];
-  float4 nm[LPT];
-  if (blk0 + warp < blk1 && full_block(blk0 + warp)) {
-#pragma unroll
-    for (int it = 0; it < LPT; ++it) {
-      nh[it] = ld_stream(vh + it * TPI * vrow);
-      nm[it] = ldg128f(vm + it * TPI * vrow);
-    }
+  // the warp's first value groups go to L2 ahead of the softmax merge
+  if (quant) {
+    const uint8_t* pf = vgroup_line<D>(u, lane);
+    if (pf != nullptr)
+      for (int j = 0; j < kPreV; ++j)
+        if (blk0 + warp + j * kWarps < qend) prefetch_l2(pf + (size_t)(blk0 + warp + j * kWarps) * 8 * D);
   }
   // bf16 positions: residual, raw cells, the SHARE current token
   for (int pos = max(p0, u.nq) + 32 * warp + lane; pos < p1; pos += 32 * kWarps) {
@@ -620,23 +839,12 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   const float tau = p.tau;
 
   // ------------------------------------------------------------- pass 2
-  float2 acc[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.f, 0.f);
-  float g0 = 0.f, g1 = 0.f;  // per-group constants of the lane's two 32-channel groups
+  const int qlim = min(p1, u.nq);
+  // selection: p >= tau on the quantized 4-bit positions, a ballot per block
   int nsel = 0;
-  // 4-bit high plane: weight 4 * p * scale; its missing low bits read as 1.5,
-  // i.e. + 1.5 * p * scale = 0.375 * (4 * p * scale) per unselected token
-  const float hmul = q4 ? 4.f : 1.f;
-  const float mid_unsel = q4 ? 0.375f : 0.f;
-  // tau <= 0 selects every 4-bit token: the low planes are read with the high
-  // ones in this loop instead of through the selected-position list
-  const bool dense_lo = DENSE_LO && q4;
-  const size_t lo_off = u.Ld.v_lo - u.Ld.v_hi;
-  for (int bk = blk0 + warp; bk < blk1; bk += kWarps, vh += VSTEP, vm += VSTEP) {
+  for (int bk = blk0 + warp; bk < blk1; bk += kWarps) {
     const int pos = bk * 32 + lane;
-    const bool active = pos < p1;
-    const float pw = active ? sc[pos - p0] * f : 0.f;
+    const float pw = pos < p1 ? sc[pos - p0] * f : 0.f;
     const bool sel = q4 && pos < qlim && pw >= tau;
     const uint32_t ballot = __ballot_sync(0xffffffffu, sel);
     nsel += __popc(ballot);
@@ -644,60 +852,45 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       mask_s[bk - blk0] = ballot;
       if (p.mask != nullptr && q4 && bk < nqb) p.mask[uidx * p.mask_words + bk] = ballot;
     }
-    if (full_block(bk)) {
-      // a full quantized block: rows arrived with the previous iteration
-      uint4 hw[LPT];
-      float4 mt[LPT];
+  }
+  __syncwarp();  // the warp reads back only the mask words its own lane 0 wrote
+
+  // high planes on the tensor cores.  A 4-bit high plane has weight
+  // 4 * p * scale; its missing low bits read as 1.5, i.e. + 1.5 * p * scale =
+  // 0.375 * (4 * p * scale) per unselected token, folded into the constants.
+  float vo[D / 32], cst[D / 32];
 #pragma unroll
-      for (int it = 0; it < LPT; ++it) { hw[it] = nh[it]; mt[it] = nm[it]; }
-      if (bk + kWarps < blk1 && full_block(bk + kWarps)) {
+  for (int i = 0; i < D / 32; ++i) { vo[i] = 0.f; cst[i] = 0.f; }
+  if (quant)
+    value_high_pass<D>(u, blk0, qend, p0, qlim, blk0, sc, mask_s, f, q4 ? 4.f : 1.f,
+                       q4 ? 0.375f : 0.f, stage, vo, cst, warp, lane);
+
+  // fp32 part, lane = 64 channels of a token: bf16 positions (residual, raw
+  // cells, the SHARE current token) and the low planes of selected tokens
+  constexpr int LPT = D / 64;       // lanes per token (64 channels per lane)
+  constexpr int TPI = 32 / LPT;     // tokens per warp iteration
+  const int hf = lane % LPT;
+  float2 acc[32];
 #pragma unroll
-        for (int it = 0; it < LPT; ++it) {
-          nh[it] = ld_stream(vh + VSTEP + it * TPI * vrow);
-          nm[it] = ldg128f(vm + VSTEP + it * TPI * vrow);
-        }
-      }
-#pragma unroll
-      for (int it = 0; it < LPT; ++it) {
-        const int tk = it * TPI + lane / LPT;
-        const float pt = __shfl_sync(0xffffffffu, pw, tk);
-        const float mid = ((ballot >> tk) & 1u) ? 0.f : mid_unsel;
-        const float a0 = (hmul * pt) * mt[it].x, a1 = (hmul * pt) * mt[it].z;
-        g0 = fmaf(mid, a0, fmaf(pt, mt[it].y, g0));
-        g1 = fmaf(mid, a1, fmaf(pt, mt[it].w, g1));
-        value_codes(acc, hw[it], a0, a1, expo, neg);
-        if (dense_lo)
-          value_codes(acc, ld_stream(vh + lo_off + it * TPI * vrow), 0.25f * a0, 0.25f * a1, expo, neg);
-      }
-    } else {
-      // partial block: quantized tokens below qlim, bf16 ones up to p1
+  for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.f, 0.f);
+  const int raw0 = max(p0, u.nq);
+  if (raw0 < p1) {
+    for (int bk = max(blk0, raw0 / 32) + warp; bk < blk1; bk += kWarps) {
+      const int pos = bk * 32 + lane;
+      const float pw = pos < p1 ? sc[pos - p0] * f : 0.f;
 #pragma unroll
       for (int it = 0; it < LPT; ++it) {
         const int tk = it * TPI + lane / LPT;
         const float pt = __shfl_sync(0xffffffffu, pw, tk);
         const int tpos = bk * 32 + tk;
-        if (tpos < qlim) {
-          const uint4 hwv = ld_stream(vh + it * TPI * vrow);
-          const float4 mtv = ldg128f(vm + it * TPI * vrow);
-          const float mid = ((ballot >> tk) & 1u) ? 0.f : mid_unsel;
-          const float a0 = (hmul * pt) * mtv.x, a1 = (hmul * pt) * mtv.z;
-          g0 = fmaf(mid, a0, fmaf(pt, mtv.y, g0));
-          g1 = fmaf(mid, a1, fmaf(pt, mtv.w, g1));
-          value_codes(acc, hwv, a0, a1, expo, neg);
-          if (dense_lo)
-            value_codes(acc, ld_stream(vh + lo_off + it * TPI * vrow), 0.25f * a0, 0.25f * a1, expo,
-                        neg);
-        } else if (tpos < p1) {
-          value_raw(acc, raw_row(u, tpos, D, true) + hf * 128, pt);
-        }
+        if (tpos >= raw0 && tpos < p1) value_raw(acc, raw_row(u, tpos, D, true) + hf * 128, pt);
       }
     }
   }
   // low planes of the selected tokens: acc += p * scale * lo.  The warp
   // gathers its selected positions into a list and processes them TPI at a
   // time, so the cost follows the number of selected tokens.
-  if (q4 && !dense_lo) {
-    __syncwarp();  // the warp reads only the mask words its own lane 0 wrote
+  if (q4) {
     int* my = lst + warp * kListCap;
     int nlist = 0;
     for (int bk = blk0 + warp; bk < qend; bk += kWarps) {
@@ -714,13 +907,13 @@ decode_kernel(const DecodeParams p, const CellList cl) {
     }
     if (nlist > 0) low_planes<D, LPT>(acc, u, my, nlist, sc, p0, f, expo, neg, lane);
   }
-  // undo the per-channel 2^o of the code conversion, add the per-group
-  // constants, then reduce over the lanes that share a channel half
+  // undo the per-channel 2^o of the fp32 part's code conversion, then reduce
+  // over the lanes that share a channel half
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const int j = (2 * i) & 15;
-    acc[i].x = fmaf(acc[i].x, pow2_neg(code2_off(j)), i < 16 ? g0 : g1);
-    acc[i].y = fmaf(acc[i].y, pow2_neg(code2_off(j + 1)), i < 16 ? g0 : g1);
+    acc[i].x *= pow2_neg(code2_off(j));
+    acc[i].y *= pow2_neg(code2_off(j + 1));
   }
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
@@ -730,11 +923,21 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       acc[i].y += __shfl_xor_sync(0xffffffffu, acc[i].y, o);
     }
   }
+#pragma unroll
+  for (int i = 0; i < D / 32; ++i)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cst[i] += __shfl_xor_sync(0xffffffffu, cst[i], o);
+  __syncthreads();  // every warp is done with its staging, which spans red
   if (lane < LPT) {
 #pragma unroll
     for (int i = 0; i < 32; ++i)
       reinterpret_cast<float2*>(red + warp * D + lane * 64)[i] = acc[i];
   }
+  __syncwarp();
+  // the tensor-core part and the per-group constants: lane (g, t) owns
+  // channel 32 G + 8 t + g of each value group G
+#pragma unroll
+  for (int i = 0; i < D / 32; ++i) red[warp * D + 32 * i + 8 * (lane & 3) + (lane >> 2)] += vo[i] + cst[i];
   if (lane == 0) misc[24 + warp] = __int_as_float(nsel);
   __syncthreads();
   for (int d = tid; d < D; d += kThreads) {
@@ -781,10 +984,10 @@ size_t decode_smem(int slots) {
   return sizeof(float) * (size_t)(D + 2 * kWarps * D + D + 64 + kWarps * kListCap + slots / 32 + slots);
 }
 
-template <int D, bool DENSE_LO>
+template <int D>
 int launch_decode_t(const DecodeParams& p, const CellList& cells, cudaStream_t stream) {
   const size_t smem = decode_smem<D>(p.slots);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, DENSE_LO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_cells * p.batch * p.n_heads;
@@ -804,7 +1007,7 @@ int launch_decode_t(const DecodeParams& p, const CellList& cells, cudaStream_t s
   }
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, DENSE_LO>, p, cells);
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<D>, p, cells);
   return (int)e;
 }
 
@@ -815,9 +1018,8 @@ int decode_max_split() { return kMaxSplit; }
 
 int launch_decode(const DecodeParams& p, const CellList& cells, void* stream, int head_dim) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool dense = !(p.tau > 0.f);
-  if (head_dim == 64) return dense ? launch_decode_t<64, true>(p, cells, s) : launch_decode_t<64, false>(p, cells, s);
-  return dense ? launch_decode_t<128, true>(p, cells, s) : launch_decode_t<128, false>(p, cells, s);
+  if (head_dim == 64) return launch_decode_t<64>(p, cells, s);
+  return launch_decode_t<128>(p, cells, s);
 }
 
 }  // namespace loopkv
