@@ -57,18 +57,11 @@
  *                                           the token in bits 2j..2j+1 of word w
  *   K_lo  [NG][D/64][32][4]                 low planes, same arrangement
  *   K_meta[NG]{scale[D], zero[D]}           fp32, per channel of the group
- *   V_hi  [NG][8][2][D/8 words]             channel-major inside a group: word
- *                                           (c%8, h, c/8) holds channel c of
- *                                           tokens 32g+16h+j in bits 2j..2j+1
- *   V_lo  [NG*32 tokens][D/16 words]        row-major: channel 16w+j of the
- *                                           token in bits 2j..2j+1 of word w
+ *   V_hi  [NG*32 tokens][D/16 words]        channel 16w+j in bits 2j..2j+1
+ *   V_lo  [NG*32][D/16]
  *   V_meta[NG*32]{(scale, zero) x D/32}     fp32 pairs per 32 channels
  *   res_K [32][D], res_V [32][D]            bf16 residual; slot r holds
  *                                           position 32*floor(n/32) + r
- * The value high plane is channel-major so that a word holds one channel of
- * 16 consecutive tokens (the contraction over tokens in decode packs them into
- * tensor-core operands); the low plane stays row-major, so the low codes of
- * one selected token are one contiguous D/4-byte row.
  * LOOPKV_Q2 has the same blocks without K_lo and V_lo; its "hi" planes hold
  * the 2-bit codes.  LOOPKV_SHARE holds cur_K[D], cur_V[D] (bf16, each block
  * rounded up to 128 bytes).  LOOPKV_BF16 holds K[C][D] then V[C][D] (bf16,

@@ -48,15 +48,6 @@ __device__ __forceinline__ float canon_zero(float mn) { return mn == 0.0f ? 0.0f
 
 __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
-// The low 16 bits of x to the even bit positions of a word (bit i -> 2i).
-__device__ __forceinline__ uint32_t spread_even(uint32_t x) {
-  x &= 0xFFFFu;
-  x = (x | (x << 8)) & 0x00FF00FFu;
-  x = (x | (x << 4)) & 0x0F0F0F0Fu;
-  x = (x | (x << 2)) & 0x33333333u;
-  return (x | (x << 1)) & 0x55555555u;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kAppendThreads)
 append_kernel(const AppendParams p, const CellList cl) {
@@ -225,32 +216,14 @@ append_kernel(const AppendParams p, const CellList cl) {
         meta[2 * j] = sc;
         meta[2 * j + 1] = canon_zero(mn);
       }
+      uint4* vh = reinterpret_cast<uint4*>(base + L.v_hi + tpos * (D / 4));
       uint4* vl = reinterpret_cast<uint4*>(base + L.v_lo + tpos * (D / 4));
       float4* vm = reinterpret_cast<float4*>(base + L.v_meta + tpos * (D / 4));
 #pragma unroll
       for (int i = 0; i < D / 64; ++i) {
+        vh[i] = make_uint4(hiw[4 * i], hiw[4 * i + 1], hiw[4 * i + 2], hiw[4 * i + 3]);
         if (q4) vl[i] = make_uint4(low[4 * i], low[4 * i + 1], low[4 * i + 2], low[4 * i + 3]);
         vm[i] = make_float4(meta[4 * i], meta[4 * i + 1], meta[4 * i + 2], meta[4 * i + 3]);
-      }
-      // high plane, channel-major: two ballots per channel collect the 32
-      // tokens' high codes; lane c % 32 keeps channel c's pair of masks and
-      // writes its words (tokens 16h .. 16h + 15, token j in bits 2j..2j+1)
-      uint32_t m0[D / 32], m1[D / 32];
-#pragma unroll
-      for (int c = 0; c < D; ++c) {
-        const uint32_t code = (hiw[c / 16] >> (2 * (c % 16))) & 3u;
-        const uint32_t b0 = __ballot_sync(0xffffffffu, code & 1u);
-        const uint32_t b1 = __ballot_sync(0xffffffffu, code & 2u);
-        if (lane == c % 32) { m0[c / 32] = b0; m1[c / 32] = b1; }
-      }
-      uint32_t* vhw = reinterpret_cast<uint32_t*>(base + L.v_hi + (size_t)g * 8 * D);
-#pragma unroll
-      for (int k = 0; k < D / 32; ++k) {
-        const int c = lane + 32 * k;
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          vhw[((c % 8) * 2 + h) * (D / 8) + c / 8] =
-              spread_even(m0[k] >> (16 * h)) | (spread_even(m1[k] >> (16 * h)) << 1);
       }
     }
     __syncwarp();

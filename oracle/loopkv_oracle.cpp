@@ -286,31 +286,18 @@ int orc_unit_serialize(const void* p, uint8_t* out, uint8_t* valid, size_t bytes
     put_bytes(out, valid, L.k_meta + static_cast<size_t>(g) * 8 * D, &u->ks[g * D], 4 * D);
     put_bytes(out, valid, L.k_meta + static_cast<size_t>(g) * 8 * D + 4 * D, &u->kz[g * D], 4 * D);
   }
-  // value high plane: per group, channel-major words of 16 tokens.  Word
-  // ((c % 8) * 2 + h) * (D / 8) + c / 8 of group g holds channel c of tokens
-  // 32 g + 16 h + j (j = 0..15) in bits 2j..2j+1.
-  for (int g = 0; g < u->qtok() / kG; ++g) {
-    for (int c = 0; c < D; ++c) {
-      for (int h = 0; h < 2; ++h) {
-        uint32_t hi = 0;
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t q = u->vq[static_cast<size_t>(g * kG + 16 * h + j) * D + c];
-          hi |= ((q4 ? (q >> 2) : q) & 3u) << (2 * j);
-        }
-        const size_t word = static_cast<size_t>((c % 8) * 2 + h) * (D / 8) + c / 8;
-        put_bytes(out, valid, L.v_hi + static_cast<size_t>(g) * 8 * D + 4 * word, &hi, 4);
-      }
-    }
-  }
   for (int t = 0; t < u->qtok(); ++t) {
-    // value low plane: [token][D/16 words], channel 16w + j in bits 2j..2j+1
+    // value planes: [token][D/16 words]
     for (int w = 0; w < D / 16; ++w) {
-      uint32_t lo = 0;
+      uint32_t hi = 0, lo = 0;
       for (int j = 0; j < 16; ++j) {
         const uint32_t q = u->vq[static_cast<size_t>(t) * D + 16 * w + j];
+        const uint32_t plane_hi = q4 ? (q >> 2) : q;
+        hi |= (plane_hi & 3u) << (2 * j);
         lo |= (q & 3u) << (2 * j);
       }
       const size_t off = static_cast<size_t>(t) * (D / 4) + w * 4;
+      put_bytes(out, valid, L.v_hi + off, &hi, 4);
       if (q4) put_bytes(out, valid, L.v_lo + off, &lo, 4);
     }
     // value meta: (scale_j, zero_j) pairs
