@@ -17,6 +17,8 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
+    # decode converts codes to floats as exact subnormals: keep them
+    "-ftz=false", "-prec-div=true", "-prec-sqrt=true",
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
     "--expt-relaxed-constexpr",

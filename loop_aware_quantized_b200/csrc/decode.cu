@@ -87,56 +87,60 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 }
 
 // Codes to floats, exactly, at one logic op per code.  A field of `bits`
-// bits at bit offset `off` (off + bits <= 23) of a word w becomes the float
-// 2^23 + code * 2^off: the word's field is placed in the mantissa of a float
-// whose exponent word `expo` (the bits of 2^23) arrives in a register, so the
-// mask is the logic op's only immediate.  Subtracting 2^23 (exact) leaves
-// code * 2^off; the power of two is folded into the weights (keys) or
-// removed from the accumulators at the end (values).
+// bits at bit offset `off` (off + bits <= 23) of a word, masked in place so
+// that the float's exponent field stays zero, is the subnormal float
+// code * 2^(off - 149): exact, with no implicit leading one to cancel.  The
+// weights carry 2^(kSub - off), so every product is an ordinary normal float
+// code * weight * 2^(kSub - 149); the FMA units take subnormal operands at
+// full rate and the build keeps them (no flush to zero).  Keys fold
+// 2^(kSub - off) into the folded query, values carry 2^kSub in their weights
+// and remove 2^(off + kSub - 149) from each channel's accumulator at the end.
+constexpr int kSub = 100;
+
 template <int off, int bits>
-__device__ __forceinline__ float field_f(uint32_t w, uint32_t expo) {
+__device__ __forceinline__ float field_f(uint32_t w) {
   static_assert(off + bits <= 23, "field must stay inside the mantissa");
-  return __uint_as_float((w & (((1u << bits) - 1u) << off)) | expo);
+  return __uint_as_float(w & (((1u << bits) - 1u) << off));
 }
 
 // 16 two-bit codes of w (code j in bits 2j..2j+1) -> 8 pairs
-// (code 2i * 2^o(2i), code 2i+1 * 2^o(2i+1)), o(j) = 2j for j < 6, 2(j-6) else.
-__device__ __forceinline__ void codes2_to_pairs(uint32_t w, uint32_t expo, float2 neg,
-                                                float2 (&out)[8]) {
+// (code 2i * 2^(o(2i) - 149), code 2i+1 * 2^(o(2i+1) - 149)),
+// o(j) = 2j for j < 6, 2(j-6) else.
+__device__ __forceinline__ void codes2_to_pairs(uint32_t w, float2 (&out)[8]) {
   const uint32_t y = w >> 12;
-  out[0] = add2(make_float2(field_f<0, 2>(w, expo), field_f<2, 2>(w, expo)), neg);
-  out[1] = add2(make_float2(field_f<4, 2>(w, expo), field_f<6, 2>(w, expo)), neg);
-  out[2] = add2(make_float2(field_f<8, 2>(w, expo), field_f<10, 2>(w, expo)), neg);
-  out[3] = add2(make_float2(field_f<0, 2>(y, expo), field_f<2, 2>(y, expo)), neg);
-  out[4] = add2(make_float2(field_f<4, 2>(y, expo), field_f<6, 2>(y, expo)), neg);
-  out[5] = add2(make_float2(field_f<8, 2>(y, expo), field_f<10, 2>(y, expo)), neg);
-  out[6] = add2(make_float2(field_f<12, 2>(y, expo), field_f<14, 2>(y, expo)), neg);
-  out[7] = add2(make_float2(field_f<16, 2>(y, expo), field_f<18, 2>(y, expo)), neg);
+  out[0] = make_float2(field_f<0, 2>(w), field_f<2, 2>(w));
+  out[1] = make_float2(field_f<4, 2>(w), field_f<6, 2>(w));
+  out[2] = make_float2(field_f<8, 2>(w), field_f<10, 2>(w));
+  out[3] = make_float2(field_f<0, 2>(y), field_f<2, 2>(y));
+  out[4] = make_float2(field_f<4, 2>(y), field_f<6, 2>(y));
+  out[5] = make_float2(field_f<8, 2>(y), field_f<10, 2>(y));
+  out[6] = make_float2(field_f<12, 2>(y), field_f<14, 2>(y));
+  out[7] = make_float2(field_f<16, 2>(y), field_f<18, 2>(y));
 }
 // Bit offset a two-bit code j of a word ends up at in codes2_to_pairs.
 __host__ __device__ constexpr int code2_off(int j) { return j < 6 ? 2 * j : 2 * (j - 6); }
 
-// Hi and lo planes of 16 four-bit codes -> 8 pairs (q_2m * 2^o(m), q_2m+1 *
-// 2^o(m)), q = 4hi + lo, o(m) = 4m for m < 3, 4(m-3) else.  The planes are
-// merged into a word of even codes (nibble m = code 2m) and one of odd codes.
-__device__ __forceinline__ void codes4_to_pairs(uint32_t hi, uint32_t lo, uint32_t expo,
-                                                float2 neg, float2 (&out)[8]) {
+// Hi and lo planes of 16 four-bit codes -> 8 pairs (q_2m * 2^(o(m) - 149),
+// q_2m+1 * 2^(o(m) - 149)), q = 4hi + lo, o(m) = 4m for m < 3, 4(m-3) else.
+// The planes are merged into a word of even codes (nibble m = code 2m) and
+// one of odd codes.
+__device__ __forceinline__ void codes4_to_pairs(uint32_t hi, uint32_t lo, float2 (&out)[8]) {
   const uint32_t even = ((hi << 2) & 0xCCCCCCCCu) | (lo & 0x33333333u);
   const uint32_t odd = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
   const uint32_t eh = even >> 12, oh = odd >> 12;
-  out[0] = add2(make_float2(field_f<0, 4>(even, expo), field_f<0, 4>(odd, expo)), neg);
-  out[1] = add2(make_float2(field_f<4, 4>(even, expo), field_f<4, 4>(odd, expo)), neg);
-  out[2] = add2(make_float2(field_f<8, 4>(even, expo), field_f<8, 4>(odd, expo)), neg);
-  out[3] = add2(make_float2(field_f<0, 4>(eh, expo), field_f<0, 4>(oh, expo)), neg);
-  out[4] = add2(make_float2(field_f<4, 4>(eh, expo), field_f<4, 4>(oh, expo)), neg);
-  out[5] = add2(make_float2(field_f<8, 4>(eh, expo), field_f<8, 4>(oh, expo)), neg);
-  out[6] = add2(make_float2(field_f<12, 4>(eh, expo), field_f<12, 4>(oh, expo)), neg);
-  out[7] = add2(make_float2(field_f<16, 4>(eh, expo), field_f<16, 4>(oh, expo)), neg);
+  out[0] = make_float2(field_f<0, 4>(even), field_f<0, 4>(odd));
+  out[1] = make_float2(field_f<4, 4>(even), field_f<4, 4>(odd));
+  out[2] = make_float2(field_f<8, 4>(even), field_f<8, 4>(odd));
+  out[3] = make_float2(field_f<0, 4>(eh), field_f<0, 4>(oh));
+  out[4] = make_float2(field_f<4, 4>(eh), field_f<4, 4>(oh));
+  out[5] = make_float2(field_f<8, 4>(eh), field_f<8, 4>(oh));
+  out[6] = make_float2(field_f<12, 4>(eh), field_f<12, 4>(oh));
+  out[7] = make_float2(field_f<16, 4>(eh), field_f<16, 4>(oh));
 }
 __host__ __device__ constexpr int code4_off(int m) { return m < 3 ? 4 * m : 4 * (m - 3); }
 
-// 2^-k as a float, k in [0, 126].
-__device__ __forceinline__ float pow2_neg(int k) { return __int_as_float((127 - k) << 23); }
+// 2^k as a float, k in [-126, 127].
+__device__ __forceinline__ float pow2(int k) { return __int_as_float((127 + k) << 23); }
 
 struct Unit {
   int own_kind, data_kind;
@@ -218,7 +222,7 @@ __device__ __forceinline__ float dot_bf16(const uint8_t* row, const float* q_s) 
 // planes (16-byte rows h[c], l[c] of K_hi / K_lo for chunk c of 64 channels).
 template <int D, bool Q4>
 __device__ __forceinline__ float dot_codes(const uint4 (&h)[D / 64], const uint4 (&l)[D / 64],
-                                           const float2* qs2, uint32_t expo, float2 neg) {
+                                           const float2* qs2) {
   // four independent accumulators keep the fma chain short
   float2 acc[4];
 #pragma unroll
@@ -230,8 +234,8 @@ __device__ __forceinline__ float dot_codes(const uint4 (&h)[D / 64], const uint4
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       float2 v[8];
-      if (Q4) codes4_to_pairs(hw[w], lw[w], expo, neg, v);
-      else codes2_to_pairs(hw[w], expo, neg, v);
+      if (Q4) codes4_to_pairs(hw[w], lw[w], v);
+      else codes2_to_pairs(hw[w], v);
       const float4* q4p = reinterpret_cast<const float4*>(qs2 + 32 * c + 8 * w);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -280,7 +284,7 @@ __device__ __forceinline__ void load_kgroup(KGroup<D>& g, const uint8_t* kh, siz
 template <int D, bool Q4>
 __device__ __forceinline__ float key_group(const KGroup<D>& g, const float (&qv)[D / 32],
                                            const float (&qz)[D / 32], float* qs, int pos,
-                                           int qlim, float sscale, uint32_t expo, float2 neg,
+                                           int qlim, float sscale,
                                            int lane) {
   constexpr int CPL = D / 32;
   // fold q into the group's key scale / zero point
@@ -295,8 +299,8 @@ __device__ __forceinline__ float key_group(const KGroup<D>& g, const float (&qv)
   __syncwarp();
   float s = -INFINITY;
   if (pos < qlim) {
-    const float dot = dot_codes<D, Q4>(g.h, g.l, reinterpret_cast<const float2*>(qs), expo, neg);
-    s = (dot + cpart) * sscale;
+    const float dot = dot_codes<D, Q4>(g.h, g.l, reinterpret_cast<const float2*>(qs));
+    s = fmaf(dot, pow2(149 - kSub) * sscale, cpart * sscale);
   }
   __syncwarp();
   return s;
@@ -308,7 +312,7 @@ __device__ __forceinline__ float key_group(const KGroup<D>& g, const float (&qv)
 template <int D, bool Q4>
 __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end, int p0, int p1,
                                           const float* q_s, float* qs, float* sc, float sscale,
-                                          uint32_t expo, float2 neg, int warp, int lane) {
+                                          int warp, int lane) {
   constexpr int CPL = D / 32;  // channels per lane for the q fold
   float lmax = -INFINITY;
   const int first = b_begin + warp;
@@ -320,7 +324,7 @@ __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end,
   for (int i = 0; i < CPL; ++i) {
     const int j = (CPL * lane + i) & 15;
     qz[i] = q_s[CPL * lane + i];
-    qv[i] = qz[i] * pow2_neg(Q4 ? code4_off(j >> 1) : code2_off(j));
+    qv[i] = qz[i] * pow2(kSub - (Q4 ? code4_off(j >> 1) : code2_off(j)));
   }
   const int qlim = min(p1, u.nq);
   constexpr size_t G = 8 * D;                       // bytes of one group in each block
@@ -335,7 +339,7 @@ __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end,
   for (;;) {
     const bool hasb = bk + kWarps < b_end;
     if (hasb) load_kgroup<D, Q4>(b, kh + STEP, lo_off, km + STEP / 4);
-    float s = key_group<D, Q4>(a, qv, qz, qs, bk * 32 + lane, qlim, sscale, expo, neg, lane);
+    float s = key_group<D, Q4>(a, qv, qz, qs, bk * 32 + lane, qlim, sscale, lane);
     if (bk * 32 + lane < qlim) { sc[bk * 32 + lane - p0] = s; lmax = fmaxf(lmax, s); }
     if (!hasb) break;
     bk += kWarps;
@@ -343,7 +347,7 @@ __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end,
     km += STEP / 4;
     const bool hasa = bk + kWarps < b_end;
     if (hasa) load_kgroup<D, Q4>(a, kh + STEP, lo_off, km + STEP / 4);
-    s = key_group<D, Q4>(b, qv, qz, qs, bk * 32 + lane, qlim, sscale, expo, neg, lane);
+    s = key_group<D, Q4>(b, qv, qz, qs, bk * 32 + lane, qlim, sscale, lane);
     if (bk * 32 + lane < qlim) { sc[bk * 32 + lane - p0] = s; lmax = fmaxf(lmax, s); }
     if (!hasa) break;
     bk += kWarps;
@@ -356,13 +360,12 @@ __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end,
 // Value accumulation of one quantized token half-row (64 channels): acc +=
 // (a_j) * code * 2^o for the lane's two 32-channel groups (a0 for words 0-1,
 // a1 for words 2-3); the 2^o of each channel is removed once at the end.
-__device__ __forceinline__ void value_codes(float2 (&acc)[32], const uint4 hw4, float a0, float a1,
-                                            uint32_t expo, float2 neg) {
+__device__ __forceinline__ void value_codes(float2 (&acc)[32], const uint4 hw4, float a0, float a1) {
   const uint32_t hw[4] = {hw4.x, hw4.y, hw4.z, hw4.w};
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     float2 v[8];
-    codes2_to_pairs(hw[w], expo, neg, v);
+    codes2_to_pairs(hw[w], v);
     const float a = (w < 2) ? a0 : a1;
     const float2 aa = make_float2(a, a);
 #pragma unroll
@@ -381,8 +384,8 @@ __device__ __forceinline__ void value_raw(float2 (&acc)[32], const uint8_t* row,
     for (int k = 0; k < 4; ++k) {
       const int pair = 4 * c + k;          // channels 2*pair, 2*pair+1
       const int j = (2 * pair) & 15;       // position inside the 16-channel word
-      const float2 wt = make_float2(pt * (float)(1u << code2_off(j)),
-                                    pt * (float)(1u << code2_off(j + 1)));
+      const float2 wt = make_float2(pt * pow2(code2_off(j) + kSub - 149),
+                                    pt * pow2(code2_off(j + 1) + kSub - 149));
       acc[pair] = fma2(wt, make_float2(bf16_lo(ws[k]), bf16_hi(ws[k])), acc[pair]);
     }
   }
@@ -392,8 +395,7 @@ __device__ __forceinline__ void value_raw(float2 (&acc)[32], const uint8_t* row,
 // positions per warp iteration (LPT lanes per position, 64 channels each).
 template <int D, int LPT>
 __device__ __forceinline__ void low_planes(float2 (&acc)[32], const Unit& u, const int* list,
-                                           int n, const float* sc, int p0, float f,
-                                           uint32_t expo, float2 neg, int lane) {
+                                           int n, const float* sc, int p0, float f, int lane) {
   constexpr int TPI = 32 / LPT;
   const int hf = lane % LPT;
   for (int k0 = 0; k0 < n; k0 += TPI) {
@@ -403,7 +405,7 @@ __device__ __forceinline__ void low_planes(float2 (&acc)[32], const Unit& u, con
       const float pt = sc[tpos - p0] * f;
       const uint4 lw = ld_stream(u.data + u.Ld.v_lo + (size_t)tpos * (D / 4) + hf * 16);
       const float4 m4 = ldg128f(u.data + u.Ld.v_meta + (size_t)tpos * (D / 4) + hf * 16);
-      value_codes(acc, lw, pt * m4.x, pt * m4.z, expo, neg);
+      value_codes(acc, lw, pt * m4.x, pt * m4.z);
     }
   }
   __syncwarp();
@@ -468,11 +470,9 @@ decode_kernel(const DecodeParams p, const CellList cl) {
 
   // ------------------------------------------------------------- pass 1
   float lmax = -INFINITY;
-  const uint32_t expo = p.code_expo;
-  const float2 neg = make_float2(p.code_neg, p.code_neg);
-  if (q4) lmax = key_pass<D, true>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, expo, neg, warp, lane);
+  if (q4) lmax = key_pass<D, true>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, warp, lane);
   else if (quant)
-    lmax = key_pass<D, false>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, expo, neg, warp, lane);
+    lmax = key_pass<D, false>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, warp, lane);
   // the warp's first value block is requested now, ahead of the softmax merge
   constexpr int LPT = D / 64;       // lanes per token in pass 2 (64 channels per lane)
   constexpr int TPI = 32 / LPT;     // tokens per warp iteration in pass 2
@@ -549,8 +549,11 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   int nsel = 0;
   // 4-bit high plane: weight 4 * p * scale; its missing low bits read as 1.5,
   // i.e. + 1.5 * p * scale = 0.375 * (4 * p * scale) per unselected token
-  const float hmul = q4 ? 4.f : 1.f;
-  const float mid_unsel = q4 ? 0.375f : 0.f;
+  // (the value weights carry 2^kSub for the code conversion; mid_unsel takes
+  // it back out for the constants)
+  const float hmul = (q4 ? 4.f : 1.f) * pow2(kSub);
+  const float mid_unsel = q4 ? 0.375f * pow2(-kSub) : 0.f;
+  const float fsub = f * pow2(kSub);  // e -> p * 2^kSub for the low planes
   // tau <= 0 selects every 4-bit token: the low planes are read with the high
   // ones in this loop instead of through the selected-position list
   const bool dense_lo = DENSE_LO && q4;
@@ -587,9 +590,9 @@ decode_kernel(const DecodeParams p, const CellList cl) {
         const float a0 = (hmul * pt) * mt[it].x, a1 = (hmul * pt) * mt[it].z;
         g0 = fmaf(mid, a0, fmaf(pt, mt[it].y, g0));
         g1 = fmaf(mid, a1, fmaf(pt, mt[it].w, g1));
-        value_codes(acc, hw[it], a0, a1, expo, neg);
+        value_codes(acc, hw[it], a0, a1);
         if (dense_lo)
-          value_codes(acc, ld_stream(vh + lo_off + it * TPI * vrow), 0.25f * a0, 0.25f * a1, expo, neg);
+          value_codes(acc, ld_stream(vh + lo_off + it * TPI * vrow), 0.25f * a0, 0.25f * a1);
       }
     } else {
       // partial block: quantized tokens below qlim, bf16 ones up to p1
@@ -605,10 +608,9 @@ decode_kernel(const DecodeParams p, const CellList cl) {
           const float a0 = (hmul * pt) * mtv.x, a1 = (hmul * pt) * mtv.z;
           g0 = fmaf(mid, a0, fmaf(pt, mtv.y, g0));
           g1 = fmaf(mid, a1, fmaf(pt, mtv.w, g1));
-          value_codes(acc, hwv, a0, a1, expo, neg);
+          value_codes(acc, hwv, a0, a1);
           if (dense_lo)
-            value_codes(acc, ld_stream(vh + lo_off + it * TPI * vrow), 0.25f * a0, 0.25f * a1, expo,
-                        neg);
+            value_codes(acc, ld_stream(vh + lo_off + it * TPI * vrow), 0.25f * a0, 0.25f * a1);
         } else if (tpos < p1) {
           value_raw(acc, raw_row(u, tpos, D, true) + hf * 128, pt);
         }
@@ -627,22 +629,22 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       if (word == 0u) continue;
       const int cnt = __popc(word);
       if (nlist + cnt > kListCap) {
-        low_planes<D, LPT>(acc, u, my, nlist, sc, p0, f, expo, neg, lane);
+        low_planes<D, LPT>(acc, u, my, nlist, sc, p0, fsub, lane);
         nlist = 0;
       }
       if ((word >> lane) & 1u) my[nlist + __popc(word & ((1u << lane) - 1u))] = bk * 32 + lane;
       nlist += cnt;
       __syncwarp();
     }
-    if (nlist > 0) low_planes<D, LPT>(acc, u, my, nlist, sc, p0, f, expo, neg, lane);
+    if (nlist > 0) low_planes<D, LPT>(acc, u, my, nlist, sc, p0, fsub, lane);
   }
   // undo the per-channel 2^o of the code conversion, add the per-group
   // constants, then reduce over the lanes that share a channel half
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const int j = (2 * i) & 15;
-    acc[i].x = fmaf(acc[i].x, pow2_neg(code2_off(j)), i < 16 ? g0 : g1);
-    acc[i].y = fmaf(acc[i].y, pow2_neg(code2_off(j + 1)), i < 16 ? g0 : g1);
+    acc[i].x = fmaf(acc[i].x, pow2(149 - kSub - code2_off(j)), i < 16 ? g0 : g1);
+    acc[i].y = fmaf(acc[i].y, pow2(149 - kSub - code2_off(j + 1)), i < 16 ? g0 : g1);
   }
 #pragma unroll
   for (int i = 0; i < 32; ++i) {

@@ -115,8 +115,6 @@ struct DecodeParams {
   int32_t slots;               // score slots per CTA (multiple of 32)
   float tau;
   float score_scale;           // sm_scale * log2(e): scores are kept in log2 units
-  uint32_t code_expo;          // bits of 2^23 (0x4B000000): exponent word of the code conversion
-  float code_neg;              // -2^23
 };
 
 // Launchers (decode.cu / append.cu).  Return cudaGetLastError() as int.

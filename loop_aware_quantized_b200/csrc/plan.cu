@@ -275,8 +275,6 @@ loopkv_status loopkv_decode(loopkv_plan* p, const int32_t* h_cells, int32_t n_ce
   dp.slots = slots_for(split);
   dp.tau = p->tau;
   dp.score_scale = p->sm_scale * 1.4426950408889634f;
-  dp.code_expo = 0x4B000000u;  // 2^23: a code field in the mantissa counts in units of 2^off
-  dp.code_neg = -8388608.0f;
   return from_cuda(launch_decode(dp, cl, stream, p->D));
 }
 
