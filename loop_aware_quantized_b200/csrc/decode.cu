@@ -139,6 +139,16 @@ __device__ __forceinline__ void codes4_to_pairs(uint32_t hi, uint32_t lo, float2
 }
 __host__ __device__ constexpr int code4_off(int m) { return m < 3 ? 4 * m : 4 * (m - 3); }
 
+// Streams run ahead of use: a warp's next group is loaded into registers
+// while the current one is processed, and its lines are also requested
+// into L2 (prefetch.global.L2) right after those loads.
+constexpr int kAheadK = 1;
+constexpr int kAheadV = 1;
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // 2^k as a float, k in [-126, 127].
 __device__ __forceinline__ float pow2(int k) { return __int_as_float((127 + k) << 23); }
 
@@ -306,6 +316,21 @@ __device__ __forceinline__ float key_group(const KGroup<D>& g, const float (&qv)
   return s;
 }
 
+// L2 requests for one key group by a lane with lane % 8 == 0: kh -> the
+// lane's K_hi row of chunk 0 (16 lane bytes into the group's block, so the
+// lanes 0, 8, 16, 24 start the chunk's four lines), km -> its scales.
+template <int D, bool Q4>
+__device__ __forceinline__ void prefetch_kgroup(const uint8_t* kh, size_t lo_off, const float* km) {
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) {
+    prefetch_l2(kh + c * 512);
+    if (Q4) prefetch_l2(kh + lo_off + c * 512);
+  }
+  // meta block: scales then zeros, D floats each; km is CPL lane floats in
+  prefetch_l2(km);
+  prefetch_l2(km + D);
+}
+
 // Pass 1 over the CTA's quantized key groups [b_begin, b_end), warp-strided.
 // Two register buffers alternate, so the next group's loads are in flight
 // while the current one is scored, without copies between them.
@@ -333,12 +358,14 @@ __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end,
   const size_t lo_off = u.Ld.k_lo - u.Ld.k_hi;
   const float* km = reinterpret_cast<const float*>(u.data + u.Ld.k_meta + (size_t)first * G) +
                     CPL * lane;
+  const bool pon = (lane & 7) == 0;  // lanes whose row pointers start a line
   KGroup<D> a, b;
   load_kgroup<D, Q4>(a, kh, lo_off, km);
   int bk = first;
   for (;;) {
     const bool hasb = bk + kWarps < b_end;
     if (hasb) load_kgroup<D, Q4>(b, kh + STEP, lo_off, km + STEP / 4);
+    if (kAheadK > 0 && pon && hasb) prefetch_kgroup<D, Q4>(kh + kAheadK * STEP, lo_off, km + kAheadK * STEP / 4);
     float s = key_group<D, Q4>(a, qv, qz, qs, bk * 32 + lane, qlim, sscale, lane);
     if (bk * 32 + lane < qlim) { sc[bk * 32 + lane - p0] = s; lmax = fmaxf(lmax, s); }
     if (!hasb) break;
@@ -347,6 +374,7 @@ __device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end,
     km += STEP / 4;
     const bool hasa = bk + kWarps < b_end;
     if (hasa) load_kgroup<D, Q4>(a, kh + STEP, lo_off, km + STEP / 4);
+    if (kAheadK > 0 && pon && hasa) prefetch_kgroup<D, Q4>(kh + kAheadK * STEP, lo_off, km + kAheadK * STEP / 4);
     s = key_group<D, Q4>(b, qv, qz, qs, bk * 32 + lane, qlim, sscale, lane);
     if (bk * 32 + lane < qlim) { sc[bk * 32 + lane - p0] = s; lmax = fmaxf(lmax, s); }
     if (!hasa) break;
@@ -580,6 +608,13 @@ decode_kernel(const DecodeParams p, const CellList cl) {
         for (int it = 0; it < LPT; ++it) {
           nh[it] = ld_stream(vh + VSTEP + it * TPI * vrow);
           nm[it] = ldg128f(vm + VSTEP + it * TPI * vrow);
+        }
+        if (kAheadV > 0 && (lane & 7) == 0) {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            prefetch_l2(vh + kAheadV * VSTEP + c * 512);
+            prefetch_l2(vm + kAheadV * VSTEP + c * 512);
+          }
         }
       }
 #pragma unroll
