@@ -27,7 +27,12 @@
 //      quantized as a group the moment it holds 32 tokens;
 //   R6 a SHARE cell of length n attends over the final loop's stored
 //      positions [0, n-1) plus its own current bf16 key and value;
-//   R7 softmax scale 1/sqrt(D) unless given; one query per KV head.
+//   R7 softmax scale 1/sqrt(D) unless given;
+//   R8 several query heads may share a KV head (grouped-query attention):
+//      each head has its own scores, softmax and output; a token's low
+//      plane is fetched for the group when any head's weight reaches tau,
+//      and every head of the group reconstructs that token with it (the
+//      selection is the union over the group's heads).
 // All attention arithmetic is fp64 (dequantized values, scores, softmax,
 // weighted sum).  Quantization is fp32 because the codes are defined by it.
 //
@@ -315,25 +320,29 @@ int orc_unit_serialize(const void* p, uint8_t* out, uint8_t* valid, size_t bytes
 }
 
 // ---- decode ----------------------------------------------------------------
-// Decode one unit.  own: the unit; src: the final loop's unit of the same
-// layer, sequence and head when own is SHARE (else ignored).  q: bf16 bits
-// [D].  sm_scale <= 0 means 1/sqrt(D).
-// Outputs: out[D]; *lse (natural log); mask words, one per 32 positions of the
-// data cell's quantized range, bit j of word g = position 32g+j selected
-// (only when the data cell is 4-bit); *nsel; slack[D] (nullable) = sum over
-// 4-bit positions with |p - tau| <= band of p * scale_v * |lo - 1.5|, the most
-// a disagreement on those positions can move each output.
-// *n_mask_words receives the number of mask words written; weights (nullable)
-// receives the softmax weight of every attended position, own current last.
+// Decode one unit for a group of g query heads that share its keys and
+// values (R8; g = 1 is plain one-query decode).  own: the unit; src: the final
+// loop's unit of the same layer, sequence and head when own is SHARE (else
+// ignored).  q: bf16 bits [g][D].  sm_scale <= 0 means 1/sqrt(D).
+// Outputs: out[g][D]; lse[g] (natural log); mask words, one per 32 positions
+// of the data cell's quantized range, bit j of word w = position 32w+j
+// selected by some head (only when the data cell is 4-bit); *nsel (selected
+// positions); slack[g][D] (nullable) = for head r, the sum over 4-bit
+// positions where some head's weight is within band of tau of
+// p_r * scale_v * |lo - 1.5|, the most a disagreement on those positions can
+// move each output.  *n_mask_words receives the number of mask words
+// written; weights[g][npos] (nullable) receives every head's softmax weight
+// of every attended position, own current last.
 // Returns 0, or -1 on invalid input (no positions, SHARE without a source,
-// SHARE longer than its source allows).
-int orc_decode(const void* own_p, const void* src_p, const uint16_t* q,
-               double tau, double sm_scale, double band, double* out,
-               double* lse, uint32_t* mask, int* n_mask_words, int* nsel,
-               double* slack, double* weights) {
+// SHARE longer than its source allows, g < 1).
+int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, int g,
+                     double tau, double sm_scale, double band, double* out, double* lse,
+                     uint32_t* mask, int* n_mask_words, int* nsel, double* slack,
+                     double* weights) {
   const Unit* own = static_cast<const Unit*>(own_p);
   const Unit* src = static_cast<const Unit*>(src_p);
   const int D = own->D;
+  if (g < 1) return -1;
   const Unit* data = own;
   int n_att = own->n;
   const bool share = own->kind == KIND_SHARE;
@@ -346,8 +355,8 @@ int orc_decode(const void* own_p, const void* src_p, const uint16_t* q,
   if (n_att + (share ? 1 : 0) < 1) return -1;
   if (sm_scale <= 0.0) sm_scale = 1.0 / std::sqrt(static_cast<double>(D));
 
-  std::vector<double> qd(D);
-  for (int d = 0; d < D; ++d) qd[d] = static_cast<double>(bf16_to_float(q[d]));
+  std::vector<double> qd(static_cast<size_t>(g) * D);
+  for (int i = 0; i < g * D; ++i) qd[i] = static_cast<double>(bf16_to_float(q[i]));
 
   const bool quant = data->kind == KIND_Q4 || data->kind == KIND_Q2;
   const int qtok = quant ? data->qtok() : 0;
@@ -361,44 +370,52 @@ int orc_decode(const void* own_p, const void* src_p, const uint16_t* q,
     } else if (data->kind == KIND_BF16) {
       for (int d = 0; d < D; ++d) khat[d] = bf16_to_float(data->bk[static_cast<size_t>(pos) * D + d]);
     } else if (pos < qtok) {
-      const int g = pos / kG;
+      const int gr = pos / kG;
       for (int d = 0; d < D; ++d)
-        khat[d] = static_cast<double>(data->ks[g * D + d]) *
+        khat[d] = static_cast<double>(data->ks[gr * D + d]) *
                       data->kq[static_cast<size_t>(pos) * D + d] +
-                  static_cast<double>(data->kz[g * D + d]);
+                  static_cast<double>(data->kz[gr * D + d]);
     } else {
       const int r = pos - qtok;
       for (int d = 0; d < D; ++d) khat[d] = bf16_to_float(data->rk[static_cast<size_t>(r) * D + d]);
     }
   };
 
-  // scores and softmax
-  std::vector<double> s(npos), p(npos);
-  double smax = -INFINITY;
-  for (int pos = 0; pos < npos; ++pos) {
-    key_of(pos);
-    double acc = 0.0;
-    for (int d = 0; d < D; ++d) acc += qd[d] * khat[d];
-    s[pos] = sm_scale * acc;
-    smax = std::max(smax, s[pos]);
+  // scores and softmax, per head
+  std::vector<double> p(static_cast<size_t>(g) * npos);
+  std::vector<double> s(npos);
+  for (int h = 0; h < g; ++h) {
+    const double* qh = &qd[static_cast<size_t>(h) * D];
+    double smax = -INFINITY;
+    for (int pos = 0; pos < npos; ++pos) {
+      key_of(pos);
+      double acc = 0.0;
+      for (int d = 0; d < D; ++d) acc += qh[d] * khat[d];
+      s[pos] = sm_scale * acc;
+      smax = std::max(smax, s[pos]);
+    }
+    double sum = 0.0;
+    for (int pos = 0; pos < npos; ++pos) sum += std::exp(s[pos] - smax);
+    const double l = smax + std::log(sum);
+    for (int pos = 0; pos < npos; ++pos) p[static_cast<size_t>(h) * npos + pos] = std::exp(s[pos] - l);
+    lse[h] = l;
   }
-  double sum = 0.0;
-  for (int pos = 0; pos < npos; ++pos) sum += std::exp(s[pos] - smax);
-  const double l = smax + std::log(sum);
-  for (int pos = 0; pos < npos; ++pos) p[pos] = std::exp(s[pos] - l);
-  *lse = l;
   if (weights) std::copy(p.begin(), p.end(), weights);
 
-  // selection mask over the 4-bit quantized positions (R4)
+  // selection over the 4-bit quantized positions: any head (R4, R8)
   const bool q4 = data->kind == KIND_Q4;
   const int nq_att = q4 ? std::min(n_att, qtok) : 0;
   const int nwords = (nq_att + kG - 1) / kG;
   for (int w = 0; w < nwords; ++w) mask[w] = 0;
   int count = 0;
-  std::vector<char> sel(npos, 0);
+  std::vector<char> sel(npos, 0), near(npos, 0);
   for (int pos = 0; pos < nq_att; ++pos) {
-    if (p[pos] >= tau) {
-      sel[pos] = 1;
+    for (int h = 0; h < g; ++h) {
+      const double ph = p[static_cast<size_t>(h) * npos + pos];
+      if (ph >= tau) sel[pos] = 1;
+      if (std::fabs(ph - tau) <= band) near[pos] = 1;
+    }
+    if (sel[pos]) {
       mask[pos / kG] |= 1u << (pos % kG);
       ++count;
     }
@@ -406,12 +423,13 @@ int orc_decode(const void* own_p, const void* src_p, const uint16_t* q,
   *n_mask_words = nwords;
   *nsel = count;
 
-  // weighted values
-  for (int d = 0; d < D; ++d) out[d] = 0.0;
-  if (slack) for (int d = 0; d < D; ++d) slack[d] = 0.0;
+  // weighted values, per head
+  for (int i = 0; i < g * D; ++i) out[i] = 0.0;
+  if (slack) for (int i = 0; i < g * D; ++i) slack[i] = 0.0;
   for (int pos = 0; pos < npos; ++pos) {
     for (int d = 0; d < D; ++d) {
       double v;
+      double dev = 0.0;  // |lo - 1.5| * scale: the most the selection moves v
       if (share && pos == n_att) {
         v = bf16_to_float(own->cv[d]);
       } else if (data->kind == KIND_BF16) {
@@ -425,18 +443,31 @@ int orc_decode(const void* own_p, const void* src_p, const uint16_t* q,
           const int hi = code >> 2, lo = code & 3;
           const double low_part = sel[pos] ? static_cast<double>(lo) : 1.5;  // R3
           v = sc * (4.0 * hi + low_part) + ze;
-          if (slack && std::fabs(p[pos] - tau) <= band)
-            slack[d] += p[pos] * sc * std::fabs(lo - 1.5);
+          dev = sc * std::fabs(lo - 1.5);
         } else {
           v = sc * code + ze;
         }
       } else {
         v = bf16_to_float(data->rv[static_cast<size_t>(pos - qtok) * D + d]);
       }
-      out[d] += p[pos] * v;
+      for (int h = 0; h < g; ++h) {
+        const double ph = p[static_cast<size_t>(h) * npos + pos];
+        out[static_cast<size_t>(h) * D + d] += ph * v;
+        if (slack && near[pos]) slack[static_cast<size_t>(h) * D + d] += ph * dev;
+      }
     }
   }
   return 0;
+}
+
+// One query head (g = 1): q bf16 bits [D], out[D], *lse, slack[D] and
+// weights[npos] as in orc_decode_group.
+int orc_decode(const void* own_p, const void* src_p, const uint16_t* q,
+               double tau, double sm_scale, double band, double* out,
+               double* lse, uint32_t* mask, int* n_mask_words, int* nsel,
+               double* slack, double* weights) {
+  return orc_decode_group(own_p, src_p, q, 1, tau, sm_scale, band, out, lse, mask,
+                          n_mask_words, nsel, slack, weights);
 }
 
 }  // extern "C"

@@ -43,6 +43,9 @@ def _load():
     lib.orc_decode.argtypes = [P, P, P, ctypes.c_double, ctypes.c_double,
                                ctypes.c_double, P, P, P, P, P, P, P]
     lib.orc_decode.restype = ctypes.c_int
+    lib.orc_decode_group.argtypes = [P, P, P, ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                     ctypes.c_double, P, P, P, P, P, P, P]
+    lib.orc_decode_group.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -143,7 +146,8 @@ def decode(unit, q_bits, tau, src=None, sm_scale=0.0, band=1e-6):
     npos = unit.n
     out = np.zeros(D, np.float64)
     slack = np.zeros(D, np.float64)
-    weights = np.zeros(max(npos, 1), np.float64)
+    # slack beyond npos: a planted mistake in a test copy may write more
+    weights = np.zeros(npos + 2, np.float64)
     lse = np.zeros(1, np.float64)
     mask = np.zeros(max(npos // G + 2, 1), np.uint32)
     nw = np.zeros(1, np.int32)
@@ -156,3 +160,39 @@ def decode(unit, q_bits, tau, src=None, sm_scale=0.0, band=1e-6):
         raise ValueError("oracle decode rejected its input")
     return DecodeResult(out=out, lse=float(lse[0]), mask=mask[: nw[0]].copy(),
                         nsel=int(nsel[0]), slack=slack, weights=weights[:npos])
+
+
+@dataclasses.dataclass
+class GroupDecodeResult:
+    out: np.ndarray      # fp64 [g][D]
+    lse: np.ndarray      # fp64 [g], natural log
+    mask: np.ndarray     # uint32 words over the 4-bit positions (union over heads)
+    nsel: int
+    slack: np.ndarray    # fp64 [g][D]
+    weights: np.ndarray  # fp64 [g][npos]
+
+
+def decode_group(unit, q_bits, tau, src=None, sm_scale=0.0, band=1e-6):
+    """Decode one unit for a group of query heads sharing its keys and values.
+
+    ``q_bits``: bf16 bits [g][D].  The selection is the union over the heads.
+    """
+    D = unit.D
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16).reshape(-1, D)
+    g = q.shape[0]
+    npos = unit.n
+    out = np.zeros((g, D), np.float64)
+    slack = np.zeros((g, D), np.float64)
+    weights = np.zeros(g * (npos + 2), np.float64)  # slack as in decode()
+    lse = np.zeros(g, np.float64)
+    mask = np.zeros(max(npos // G + 2, 1), np.uint32)
+    nw = np.zeros(1, np.int32)
+    nsel = np.zeros(1, np.int32)
+    rc = unit._lib.orc_decode_group(unit._h, None if src is None else src._h, _ptr(q), g,
+                                    float(tau), float(sm_scale), float(band), _ptr(out),
+                                    _ptr(lse), _ptr(mask), _ptr(nw), _ptr(nsel),
+                                    _ptr(slack), _ptr(weights))
+    if rc != 0:
+        raise ValueError("oracle decode rejected its input")
+    return GroupDecodeResult(out=out, lse=lse, mask=mask[: nw[0]].copy(), nsel=int(nsel[0]),
+                             slack=slack, weights=weights[: g * npos].reshape(g, npos).copy())

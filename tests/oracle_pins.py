@@ -315,6 +315,64 @@ def pin_share_reads_final_loop():
         raise AssertionError("SHARE past its source accepted")
 
 
+def _mask_bits(words, n):
+    """Selection per position [n] from mask words (bit j of word w = 32w + j)."""
+    out = np.zeros(n, bool)
+    for w, word in enumerate(np.asarray(words, np.uint64)):
+        for j in range(32):
+            if 32 * w + j < n and (int(word) >> j) & 1:
+                out[32 * w + j] = True
+    return out
+
+
+def pin_group_query_heads():
+    # Grouped-query decode: each head of the group has its own softmax and
+    # output; the low planes fetched for the group are the ones any head
+    # selects, and every head reconstructs those tokens at 4 bits.  So, head
+    # by head: the weights and lse equal a one-query decode, the mask is the
+    # union of the heads' own masks, and the output differs from the
+    # one-query decode by exactly p * scale * (lo - 1.5) summed over the
+    # tokens selected by other heads only.
+    D = 64
+    u, k, v = _unit(orc.KIND_Q4, D, 150, 90)
+    kf = f32(k)
+    q = np.stack([bf16(3.0 * kf[t]) for t in (10, 70, 100)])   # peaks on three tokens
+    tau = 0.01
+    r = orc.decode_group(u, q, tau)
+    st = u.export()
+    qtok = st["qtok"]
+    lo = (st["vq"].astype(np.int64) & 3) - 1.5                     # [qtok][D]
+    sc = np.repeat(st["vs"].astype(np.float64), G, axis=1)        # [qtok][D]
+    grp = _mask_bits(r.mask, qtok)
+    union = np.zeros_like(r.mask)
+    nsel_heads = []
+    for h in range(q.shape[0]):
+        one = orc.decode(u, q[h], tau)
+        assert np.array_equal(r.weights[h], one.weights) and r.lse[h] == one.lse
+        union |= one.mask
+        nsel_heads.append(one.nsel)
+        extra = grp & ~_mask_bits(one.mask, qtok)
+        delta = (r.weights[h][:qtok, None] * sc * lo * extra[:, None]).sum(0)
+        assert np.abs(r.out[h] - one.out - delta).max() < 1e-12, h
+    assert np.array_equal(r.mask, union)
+    assert r.nsel == int(grp.sum()) and r.nsel > max(nsel_heads)
+    # tau = 0 (every token) and tau > 1 (none) leave nothing to share
+    for t in (0.0, 2.0):
+        r2 = orc.decode_group(u, q, t)
+        for h in range(q.shape[0]):
+            assert np.array_equal(r2.out[h], orc.decode(u, q[h], t).out)
+    # a group of one head is the one-query decode
+    r1, o1 = orc.decode_group(u, q[:1], tau), orc.decode(u, q[0], tau)
+    assert np.array_equal(r1.out[0], o1.out) and np.array_equal(r1.mask, o1.mask)
+    assert r1.nsel == o1.nsel and np.array_equal(r1.slack[0], o1.slack)
+    # SHARE units group the same way over the final loop's positions
+    own = orc.OracleUnit(orc.KIND_SHARE, D, 0)
+    own.append(rng_bits(95, (120, D)), rng_bits(96, (120, D)))
+    rs = orc.decode_group(own, q, tau, src=u)
+    for h in range(q.shape[0]):
+        assert np.array_equal(rs.weights[h], orc.decode(own, q[h], tau, src=u).weights)
+
+
 def pin_high_plane_worked_example():
     # 32 tokens with equal keys (key scale 0, so every weight is 1/32).  Each
     # value token is 0 on channel 0, 15 on channel 1, 13 on channel 2 and 0
@@ -380,4 +438,5 @@ ALL_PINS = [
     pin_share_reads_final_loop,
     pin_high_plane_worked_example,
     pin_mask_properties,
+    pin_group_query_heads,
 ]

@@ -26,19 +26,23 @@ MUTANTS = [
      "if (residual() == kG + 1) flush_group();"),
     ("code order reversed", "hi |= (plane_hi & 3u) << (2 * j);",
      "hi |= (plane_hi & 3u) << (2 * (15 - j));"),
-    ("key index shifted", "for (int d = 0; d < D; ++d) acc += qd[d] * khat[d];",
-     "for (int d = 0; d < D; ++d) acc += qd[d] * khat[(d + 1) % D];"),
-    ("softmax not normalised", "p[pos] = std::exp(s[pos] - l);",
-     "p[pos] = std::exp(s[pos] - smax);"),
+    ("key index shifted", "for (int d = 0; d < D; ++d) acc += qh[d] * khat[d];",
+     "for (int d = 0; d < D; ++d) acc += qh[d] * khat[(d + 1) % D];"),
+    ("softmax not normalised", "p[static_cast<size_t>(h) * npos + pos] = std::exp(s[pos] - l);",
+     "p[static_cast<size_t>(h) * npos + pos] = std::exp(s[pos] - smax);"),
     ("share reads its own slot", "n_att = own->n - 1;  // R6", "n_att = own->n;  // R6"),
     ("high plane weight", "v = sc * (4.0 * hi + low_part) + ze;",
      "v = sc * (2.0 * hi + low_part) + ze;"),
     ("high-plane midpoint", "sel[pos] ? static_cast<double>(lo) : 1.5",
      "sel[pos] ? static_cast<double>(lo) : 2.0"),
     ("zero point dropped", "v = sc * code + ze;", "v = sc * code;"),
-    ("tie not selected", "if (p[pos] >= tau) {", "if (p[pos] > tau) {"),
-    ("sign of zero point", "static_cast<double>(data->kz[g * D + d]);",
-     "-static_cast<double>(data->kz[g * D + d]);"),
+    ("tie not selected", "if (ph >= tau) sel[pos] = 1;", "if (ph > tau) sel[pos] = 1;"),
+    ("selection from one head only", "if (ph >= tau) sel[pos] = 1;",
+     "if (ph >= tau && h == 0) sel[pos] = 1;"),
+    ("query heads share one query", "const double* qh = &qd[static_cast<size_t>(h) * D];",
+     "const double* qh = &qd[0];"),
+    ("sign of zero point", "static_cast<double>(data->kz[gr * D + d]);",
+     "-static_cast<double>(data->kz[gr * D + d]);"),
 ]
 
 
