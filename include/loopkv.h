@@ -112,6 +112,10 @@ typedef struct {
                              < n_loops - 1 */
   float tau;              /* low-plane threshold on the softmax weight, >= 0 */
   float sm_scale;         /* softmax scale; <= 0 means 1/sqrt(head_dim) */
+  int32_t q_per_kv;       /* query heads per KV head (grouped-query
+                             attention): 1, 2 or 4; 0 means 1.  The heads of
+                             a group share the KV head's reads; see
+                             loopkv_decode for their selection. */
 } loopkv_plan_desc;
 
 typedef struct {
@@ -157,19 +161,22 @@ loopkv_status loopkv_append(loopkv_plan* plan, const int32_t* h_cells, int32_t n
                             const uint16_t* d_k, const uint16_t* d_v, void* stream);
 
 /* Decode attention: the fused LoopKV read of the plan.  For every listed
- * cell c = h_cells[i], sequence b < batch and head h, with query
- *     d_q: bf16 [n_cells][batch][n_kv_heads][head_dim]
+ * cell c = h_cells[i], sequence b < batch, KV head h and query head r <
+ * g = q_per_kv of h's group, with queries
+ *     d_q: bf16 [n_cells][batch][n_kv_heads][g][head_dim]
  * computes over the unit's attended positions (its own n tokens; for a SHARE
  * unit of length n, the final loop's stored positions [0, n-1) and its own
- * current token) the scores sm_scale * <q, k>, with keys dequantized at their
- * stored precision, their softmax p, the selection p >= tau over 4-bit
- * quantized positions, and
- *     d_out: fp32 [n_cells][batch][n_kv_heads][head_dim] = sum_t p_t * v_t
+ * current token) the scores sm_scale * <q_r, k>, with keys dequantized at
+ * their stored precision, each query's softmax p_r, the selection of the
+ * 4-bit quantized positions where some query of the group has p_r >= tau
+ * (one query: p >= tau; the KV head's low plane is read once for the whole
+ * group, and every query of the group uses what was read), and
+ *     d_out: fp32 [n_cells][batch][n_kv_heads][g][head_dim] = sum_t p_r,t v_t
  * with v_t at 4-bit precision where selected, high plane only otherwise,
  * 2-bit, or bf16 as stored.  Optional outputs (NULL to skip):
- *     d_lse : fp32 [n_cells][batch][n_kv_heads], natural-log logsumexp
+ *     d_lse : fp32 [n_cells][batch][n_kv_heads][g], natural-log logsumexp
  *     d_mask: uint32 [n_cells][batch][n_kv_heads][mask_words]; bit j of
- *             word g = position 32g+j was selected; words
+ *             word w = position 32w+j was selected; words
  *             0 .. ceil(nq/32)-1 are written, nq = 4-bit positions attended
  *     d_nsel: int32 [n_cells][batch][n_kv_heads], number of selected positions
  * Every unit must hold n >= 1 tokens; a SHARE unit needs its source to hold

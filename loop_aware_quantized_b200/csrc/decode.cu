@@ -208,35 +208,47 @@ __device__ __forceinline__ const uint8_t* raw_row(const Unit& u, int pos, int D,
   return u.data + (value ? u.Ld.res_v : u.Ld.res_k) + (size_t)(pos - u.qtok) * D * 2;
 }
 
-template <int D>
-__device__ __forceinline__ float dot_bf16(const uint8_t* row, const float* q_s) {
-  float acc = 0.f;
+// bf16 key row dotted with the G queries of the group (q_s: [G][D] fp32).
+template <int D, int G>
+__device__ __forceinline__ void dot_bf16(const uint8_t* row, const float* q_s, float (&out)[G]) {
+#pragma unroll
+  for (int r = 0; r < G; ++r) out[r] = 0.f;
 #pragma unroll
   for (int c = 0; c < D / 8; ++c) {
     const uint4 w = ldg128(row + c * 16);
-    const float4 qa = *reinterpret_cast<const float4*>(q_s + 8 * c);
-    const float4 qb = *reinterpret_cast<const float4*>(q_s + 8 * c + 4);
-    acc = fmaf(qa.x, bf16_lo(w.x), acc);
-    acc = fmaf(qa.y, bf16_hi(w.x), acc);
-    acc = fmaf(qa.z, bf16_lo(w.y), acc);
-    acc = fmaf(qa.w, bf16_hi(w.y), acc);
-    acc = fmaf(qb.x, bf16_lo(w.z), acc);
-    acc = fmaf(qb.y, bf16_hi(w.z), acc);
-    acc = fmaf(qb.z, bf16_lo(w.w), acc);
-    acc = fmaf(qb.w, bf16_hi(w.w), acc);
+    const float k[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                        bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      const float4 qa = *reinterpret_cast<const float4*>(q_s + r * D + 8 * c);
+      const float4 qb = *reinterpret_cast<const float4*>(q_s + r * D + 8 * c + 4);
+      float acc = out[r];
+      acc = fmaf(qa.x, k[0], acc);
+      acc = fmaf(qa.y, k[1], acc);
+      acc = fmaf(qa.z, k[2], acc);
+      acc = fmaf(qa.w, k[3], acc);
+      acc = fmaf(qb.x, k[4], acc);
+      acc = fmaf(qb.y, k[5], acc);
+      acc = fmaf(qb.z, k[6], acc);
+      acc = fmaf(qb.w, k[7], acc);
+      out[r] = acc;
+    }
   }
-  return acc;
 }
 
-// Score of one quantized token: sum_d qs_d * code_d over the token's packed
-// planes (16-byte rows h[c], l[c] of K_hi / K_lo for chunk c of 64 channels).
-template <int D, bool Q4>
-__device__ __forceinline__ float dot_codes(const uint4 (&h)[D / 64], const uint4 (&l)[D / 64],
-                                           const float2* qs2) {
-  // four independent accumulators keep the fma chain short
-  float2 acc[4];
+// Scores of one quantized token for the G queries: sum_d qs_d * code_d over
+// the token's packed planes (16-byte rows h[c], l[c] of K_hi / K_lo for chunk
+// c of 64 channels); the codes are converted once and serve every query.
+// qs2: the warp's staged q * scale, [G][D] as float pairs.
+template <int D, bool Q4, int G>
+__device__ __forceinline__ void dot_codes(const uint4 (&h)[D / 64], const uint4 (&l)[D / 64],
+                                          const float2* qs2, float (&dot)[G]) {
+  // four independent accumulators per query keep the fma chains short
+  float2 acc[G][4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+  for (int r = 0; r < G; ++r)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[r][k] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < D / 64; ++c) {
     const uint32_t hw[4] = {h[c].x, h[c].y, h[c].z, h[c].w};
@@ -246,17 +258,24 @@ __device__ __forceinline__ float dot_codes(const uint4 (&h)[D / 64], const uint4
       float2 v[8];
       if (Q4) codes4_to_pairs(hw[w], lw[w], v);
       else codes2_to_pairs(hw[w], v);
-      const float4* q4p = reinterpret_cast<const float4*>(qs2 + 32 * c + 8 * w);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 qq = q4p[i];
-        acc[(2 * i) & 3] = fma2(make_float2(qq.x, qq.y), v[2 * i], acc[(2 * i) & 3]);
-        acc[(2 * i + 1) & 3] = fma2(make_float2(qq.z, qq.w), v[2 * i + 1], acc[(2 * i + 1) & 3]);
+      for (int r = 0; r < G; ++r) {
+        const float4* q4p = reinterpret_cast<const float4*>(qs2 + r * (D / 2) + 32 * c + 8 * w);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 qq = q4p[i];
+          acc[r][(2 * i) & 3] = fma2(make_float2(qq.x, qq.y), v[2 * i], acc[r][(2 * i) & 3]);
+          acc[r][(2 * i + 1) & 3] =
+              fma2(make_float2(qq.z, qq.w), v[2 * i + 1], acc[r][(2 * i + 1) & 3]);
+        }
       }
     }
   }
-  const float2 a = add2(acc[0], acc[1]), b = add2(acc[2], acc[3]);
-  return (a.x + b.x) + (a.y + b.y);
+#pragma unroll
+  for (int r = 0; r < G; ++r) {
+    const float2 a = add2(acc[r][0], acc[r][1]), b = add2(acc[r][2], acc[r][3]);
+    dot[r] = (a.x + b.x) + (a.y + b.y);
+  }
 }
 
 // Per-lane load of one 32-token key group: the lane's token rows of the
@@ -290,30 +309,38 @@ __device__ __forceinline__ void load_kgroup(KGroup<D>& g, const uint8_t* kh, siz
   }
 }
 
-// Score one group held in registers; returns the lane's score (or -inf).
-template <int D, bool Q4>
-__device__ __forceinline__ float key_group(const KGroup<D>& g, const float (&qv)[D / 32],
-                                           const float (&qz)[D / 32], float* qs, int pos,
-                                           int qlim, float sscale,
-                                           int lane) {
+// Score one group held in registers for the G queries; s[r] = the lane's
+// score for query r (or -inf past qlim).
+template <int D, bool Q4, int G>
+__device__ __forceinline__ void key_group(const KGroup<D>& g, const float (&qv)[G][D / 32],
+                                          const float (&qz)[G][D / 32], float* qs, int pos,
+                                          int qlim, float sscale, int lane, float (&s)[G]) {
   constexpr int CPL = D / 32;
-  // fold q into the group's key scale / zero point
-  float cpart = 0.f;
+  // fold each query into the group's key scale / zero point
+  float cpart[G];
 #pragma unroll
-  for (int i = 0; i < CPL; ++i) {
-    qs[CPL * lane + i] = qv[i] * g.sc[i];
-    cpart = fmaf(qz[i], g.zr[i], cpart);
+  for (int r = 0; r < G; ++r) {
+    cpart[r] = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      qs[r * D + CPL * lane + i] = qv[r][i] * g.sc[i];
+      cpart[r] = fmaf(qz[r][i], g.zr[i], cpart[r]);
+    }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o);
+  for (int r = 0; r < G; ++r)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cpart[r] += __shfl_xor_sync(0xffffffffu, cpart[r], o);
   __syncwarp();
-  float s = -INFINITY;
+#pragma unroll
+  for (int r = 0; r < G; ++r) s[r] = -INFINITY;
   if (pos < qlim) {
-    const float dot = dot_codes<D, Q4>(g.h, g.l, reinterpret_cast<const float2*>(qs));
-    s = fmaf(dot, pow2(149 - kSub) * sscale, cpart * sscale);
+    float dot[G];
+    dot_codes<D, Q4, G>(g.h, g.l, reinterpret_cast<const float2*>(qs), dot);
+#pragma unroll
+    for (int r = 0; r < G; ++r) s[r] = fmaf(dot[r], pow2(149 - kSub) * sscale, cpart[r] * sscale);
   }
   __syncwarp();
-  return s;
 }
 
 // L2 requests for one key group by a lane with lane % 8 == 0: kh -> the
@@ -333,126 +360,221 @@ __device__ __forceinline__ void prefetch_kgroup(const uint8_t* kh, size_t lo_off
 
 // Pass 1 over the CTA's quantized key groups [b_begin, b_end), warp-strided.
 // Two register buffers alternate, so the next group's loads are in flight
-// while the current one is scored, without copies between them.
-template <int D, bool Q4>
-__device__ __forceinline__ float key_pass(const Unit& u, int b_begin, int b_end, int p0, int p1,
-                                          const float* q_s, float* qs, float* sc, float sscale,
-                                          int warp, int lane) {
+// while the current one is scored, without copies between them.  Scores of
+// query r go to sc[r * S + pos - p0]; lmax[r] is raised to their maximum.
+template <int D, bool Q4, int G>
+__device__ __forceinline__ void key_pass(const Unit& u, int b_begin, int b_end, int p0, int p1,
+                                         const float* q_s, float* qs, float* sc, int S,
+                                         float sscale, int warp, int lane, float (&lmax)[G]) {
   constexpr int CPL = D / 32;  // channels per lane for the q fold
-  float lmax = -INFINITY;
   const int first = b_begin + warp;
-  if (first >= b_end) return lmax;
-  // q of the lane's channels, times 2^-o: o is the bit offset the channel's
-  // code keeps after conversion (see codes4_to_pairs / codes2_to_pairs)
-  float qv[CPL], qz[CPL];
+  if (first >= b_end) return;
+  // q of the lane's channels, times 2^(kSub - o): o is the bit offset the
+  // channel's code keeps after conversion (see codes4_to_pairs / codes2_to_pairs)
+  float qv[G][CPL], qz[G][CPL];
 #pragma unroll
-  for (int i = 0; i < CPL; ++i) {
-    const int j = (CPL * lane + i) & 15;
-    qz[i] = q_s[CPL * lane + i];
-    qv[i] = qz[i] * pow2(kSub - (Q4 ? code4_off(j >> 1) : code2_off(j)));
-  }
+  for (int r = 0; r < G; ++r)
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const int j = (CPL * lane + i) & 15;
+      qz[r][i] = q_s[r * D + CPL * lane + i];
+      qv[r][i] = qz[r][i] * pow2(kSub - (Q4 ? code4_off(j >> 1) : code2_off(j)));
+    }
   const int qlim = min(p1, u.nq);
-  constexpr size_t G = 8 * D;                       // bytes of one group in each block
-  constexpr size_t STEP = (size_t)kWarps * G;       // a warp's stride between its groups
-  const uint8_t* kh = u.data + u.Ld.k_hi + (size_t)first * G + lane * 16;
+  constexpr size_t GB = 8 * D;                      // bytes of one group in each block
+  constexpr size_t STEP = (size_t)kWarps * GB;      // a warp's stride between its groups
+  const uint8_t* kh = u.data + u.Ld.k_hi + (size_t)first * GB + lane * 16;
   const size_t lo_off = u.Ld.k_lo - u.Ld.k_hi;
-  const float* km = reinterpret_cast<const float*>(u.data + u.Ld.k_meta + (size_t)first * G) +
+  const float* km = reinterpret_cast<const float*>(u.data + u.Ld.k_meta + (size_t)first * GB) +
                     CPL * lane;
   const bool pon = (lane & 7) == 0;  // lanes whose row pointers start a line
   KGroup<D> a, b;
   load_kgroup<D, Q4>(a, kh, lo_off, km);
   int bk = first;
+  float s[G];
   for (;;) {
     const bool hasb = bk + kWarps < b_end;
     if (hasb) load_kgroup<D, Q4>(b, kh + STEP, lo_off, km + STEP / 4);
-    if (kAheadK > 0 && pon && hasb) prefetch_kgroup<D, Q4>(kh + kAheadK * STEP, lo_off, km + kAheadK * STEP / 4);
-    float s = key_group<D, Q4>(a, qv, qz, qs, bk * 32 + lane, qlim, sscale, lane);
-    if (bk * 32 + lane < qlim) { sc[bk * 32 + lane - p0] = s; lmax = fmaxf(lmax, s); }
+    if (kAheadK > 0 && pon && hasb)
+      prefetch_kgroup<D, Q4>(kh + kAheadK * STEP, lo_off, km + kAheadK * STEP / 4);
+    key_group<D, Q4, G>(a, qv, qz, qs, bk * 32 + lane, qlim, sscale, lane, s);
+    if (bk * 32 + lane < qlim) {
+#pragma unroll
+      for (int r = 0; r < G; ++r) {
+        sc[r * S + bk * 32 + lane - p0] = s[r];
+        lmax[r] = fmaxf(lmax[r], s[r]);
+      }
+    }
     if (!hasb) break;
     bk += kWarps;
     kh += STEP;
     km += STEP / 4;
     const bool hasa = bk + kWarps < b_end;
     if (hasa) load_kgroup<D, Q4>(a, kh + STEP, lo_off, km + STEP / 4);
-    if (kAheadK > 0 && pon && hasa) prefetch_kgroup<D, Q4>(kh + kAheadK * STEP, lo_off, km + kAheadK * STEP / 4);
-    s = key_group<D, Q4>(b, qv, qz, qs, bk * 32 + lane, qlim, sscale, lane);
-    if (bk * 32 + lane < qlim) { sc[bk * 32 + lane - p0] = s; lmax = fmaxf(lmax, s); }
+    if (kAheadK > 0 && pon && hasa)
+      prefetch_kgroup<D, Q4>(kh + kAheadK * STEP, lo_off, km + kAheadK * STEP / 4);
+    key_group<D, Q4, G>(b, qv, qz, qs, bk * 32 + lane, qlim, sscale, lane, s);
+    if (bk * 32 + lane < qlim) {
+#pragma unroll
+      for (int r = 0; r < G; ++r) {
+        sc[r * S + bk * 32 + lane - p0] = s[r];
+        lmax[r] = fmaxf(lmax[r], s[r]);
+      }
+    }
     if (!hasa) break;
     bk += kWarps;
     kh += STEP;
     km += STEP / 4;
   }
-  return lmax;
 }
 
-// Value accumulation of one quantized token half-row (64 channels): acc +=
-// (a_j) * code * 2^o for the lane's two 32-channel groups (a0 for words 0-1,
-// a1 for words 2-3); the 2^o of each channel is removed once at the end.
-__device__ __forceinline__ void value_codes(float2 (&acc)[32], const uint4 hw4, float a0, float a1) {
-  const uint32_t hw[4] = {hw4.x, hw4.y, hw4.z, hw4.w};
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    float2 v[8];
-    codes2_to_pairs(hw[w], v);
-    const float a = (w < 2) ? a0 : a1;
-    const float2 aa = make_float2(a, a);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[8 * w + i] = fma2(aa, v[i], acc[8 * w + i]);
+// A lane's share of a token's value row in pass 2: with G queries per KV
+// head, LPT = (D / 64) * G lanes share a token and each holds CH = 64 / G
+// channels for every query (G * CH / 2 = 32 accumulator pairs): NW plane
+// words, NGRP 32-channel value groups.
+template <int G>
+struct VShare {
+  static constexpr int CH = 64 / G;
+  static constexpr int NW = CH / 16;
+  static constexpr int NGRP = CH >= 32 ? CH / 32 : 1;
+};
+
+__device__ __forceinline__ uint2 ld_stream2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_stream1(const void* p) {
+  uint32_t r;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+
+// NW plane words of a value row (16 NW bytes, 16-byte aligned for NW = 4).
+template <int NW>
+__device__ __forceinline__ void load_words(uint32_t (&w)[NW], const uint8_t* p) {
+  if constexpr (NW == 4) {
+    const uint4 x = ld_stream(p);
+    w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+  } else if constexpr (NW == 2) {
+    const uint2 x = ld_stream2(p);
+    w[0] = x.x; w[1] = x.y;
+  } else {
+    w[0] = ld_stream1(p);
   }
 }
 
-// bf16 value row (64 channels) with weight pt, in the accumulators' scaled
-// representation (channel j of a 16-channel word carries 2^o(j)).
-__device__ __forceinline__ void value_raw(float2 (&acc)[32], const uint8_t* row, float pt) {
+// (scale, zero) of NGRP value groups of a meta row.
+template <int NGRP>
+__device__ __forceinline__ void load_meta(float (&m)[2 * NGRP], const uint8_t* p) {
+  if constexpr (NGRP == 2) {
+    const float4 x = ldg128f(p);
+    m[0] = x.x; m[1] = x.y; m[2] = x.z; m[3] = x.w;
+  } else {
+    const float2 x = __ldg(reinterpret_cast<const float2*>(p));
+    m[0] = x.x; m[1] = x.y;
+  }
+}
+
+// Value accumulation of the lane's share of one quantized token row:
+// acc[r] += a[r][group] * code * 2^(o - 149) per channel, one conversion per
+// code for all G queries; the per-channel power of two is removed once at
+// the end.
+template <int G>
+__device__ __forceinline__ void value_codes(float2 (&acc)[G][32 / G],
+                                            const uint32_t (&w)[VShare<G>::NW],
+                                            const float (&a)[G][VShare<G>::NGRP]) {
+  constexpr int NW = VShare<G>::NW;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint4 w = ldg128(row + c * 16);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  for (int wi = 0; wi < NW; ++wi) {
+    float2 v[8];
+    codes2_to_pairs(w[wi], v);
+    constexpr int kPerGroup = 2;  // 16-channel words per 32-channel group
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int pair = 4 * c + k;          // channels 2*pair, 2*pair+1
-      const int j = (2 * pair) & 15;       // position inside the 16-channel word
-      const float2 wt = make_float2(pt * pow2(code2_off(j) + kSub - 149),
-                                    pt * pow2(code2_off(j + 1) + kSub - 149));
-      acc[pair] = fma2(wt, make_float2(bf16_lo(ws[k]), bf16_hi(ws[k])), acc[pair]);
+    for (int r = 0; r < G; ++r) {
+      const float aw = a[r][wi / kPerGroup];
+      const float2 aa = make_float2(aw, aw);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[r][8 * wi + i] = fma2(aa, v[i], acc[r][8 * wi + i]);
     }
   }
 }
 
-// Low planes of queued selected positions: acc += p * scale * lo, TPI
-// positions per warp iteration (LPT lanes per position, 64 channels each).
-template <int D, int LPT>
-__device__ __forceinline__ void low_planes(float2 (&acc)[32], const Unit& u, const int* list,
-                                           int n, const float* sc, int p0, float f, int lane) {
+// bf16 value row (the lane's CH channels) with weight pt[r] per query, in the
+// accumulators' scaled representation (channel j of a 16-channel word
+// carries 2^(o(j) + kSub - 149)).
+template <int G>
+__device__ __forceinline__ void value_raw(float2 (&acc)[G][32 / G], const uint8_t* row,
+                                          const float (&pt)[G]) {
+  constexpr int CH = VShare<G>::CH;
+#pragma unroll
+  for (int c = 0; c < CH / 8; ++c) {
+    const uint4 w = ldg128(row + c * 16);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int pair = 4 * c + k;          // channels 2*pair, 2*pair+1 of the lane's share
+      const int j = (2 * pair) & 15;       // position inside the 16-channel word
+      const float2 x = make_float2(bf16_lo(ws[k]), bf16_hi(ws[k]));
+#pragma unroll
+      for (int r = 0; r < G; ++r) {
+        const float2 wt = make_float2(pt[r] * pow2(code2_off(j) + kSub - 149),
+                                      pt[r] * pow2(code2_off(j + 1) + kSub - 149));
+        acc[r][pair] = fma2(wt, x, acc[r][pair]);
+      }
+    }
+  }
+}
+
+// Low planes of queued selected positions: acc[r] += p_r * scale * lo, TPI
+// positions per warp iteration (LPT lanes per position).  fs[r] turns the
+// stored exponential of query r into p_r * 2^kSub.
+template <int D, int G, int LPT>
+__device__ __forceinline__ void low_planes(float2 (&acc)[G][32 / G], const Unit& u,
+                                           const int* list, int n, const float* sc, int S,
+                                           int p0, const float (&fs)[G], int lane) {
+  using VS = VShare<G>;
   constexpr int TPI = 32 / LPT;
   const int hf = lane % LPT;
   for (int k0 = 0; k0 < n; k0 += TPI) {
     const int kk = k0 + lane / LPT;
     if (kk < n) {
       const int tpos = list[kk];
-      const float pt = sc[tpos - p0] * f;
-      const uint4 lw = ld_stream(u.data + u.Ld.v_lo + (size_t)tpos * (D / 4) + hf * 16);
-      const float4 m4 = ldg128f(u.data + u.Ld.v_meta + (size_t)tpos * (D / 4) + hf * 16);
-      value_codes(acc, lw, pt * m4.x, pt * m4.z);
+      uint32_t lw[VS::NW];
+      float m[2 * VS::NGRP];
+      load_words<VS::NW>(lw, u.data + u.Ld.v_lo + (size_t)tpos * (D / 4) + hf * (VS::CH / 4));
+      load_meta<VS::NGRP>(m, u.data + u.Ld.v_meta + (size_t)tpos * (D / 4) + (hf * VS::CH / 32) * 8);
+      float a[G][VS::NGRP];
+#pragma unroll
+      for (int r = 0; r < G; ++r) {
+        const float pt = sc[r * S + tpos - p0] * fs[r];
+#pragma unroll
+        for (int gi = 0; gi < VS::NGRP; ++gi) a[r][gi] = pt * m[2 * gi];
+      }
+      value_codes<G>(acc, lw, a);
     }
   }
   __syncwarp();
 }
 
-// DENSE_LO: tau <= 0, every 4-bit token takes its low plane (read densely in
-// the value loop); otherwise low planes come from the selected-position list.
-template <int D, bool DENSE_LO>
+// One CTA per (unit, split) for a group of G query heads sharing the unit's
+// KV head.  DENSE_LO: tau <= 0, every 4-bit token takes its low plane (read
+// densely in the value loop); otherwise low planes come from the
+// selected-position list.
+template <int D, int G, bool DENSE_LO>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p, const CellList cl) {
+  using VS = VShare<G>;
+  const int S = p.slots;  // score slots per query
   extern __shared__ __align__(16) float smem[];
-  float* q_s = smem;                                  // [D]
-  float* qs_all = q_s + D;                            // [kWarps][D]
-  float* red = qs_all + kWarps * D;                   // [kWarps][D]
-  float* o_s = red + kWarps * D;                      // [D]
-  float* misc = o_s + D;                              // [64]
-  int* lst = reinterpret_cast<int*>(misc + 64);       // [kWarps][kListCap] selected positions
-  uint32_t* mask_s = reinterpret_cast<uint32_t*>(lst + kWarps * kListCap);  // [slots / 32]
-  float* sc = reinterpret_cast<float*>(mask_s + p.slots / 32);        // [slots]
+  float* q_s = smem;                                  // [G][D]
+  float* qs_all = q_s + G * D;                        // [kWarps][G][D]
+  float* red = qs_all + kWarps * G * D;               // [kWarps][G][D]
+  float* o_s = red + kWarps * G * D;                  // [G][D]
+  float* misc = o_s + G * D;                          // [128]
+  int* lst = reinterpret_cast<int*>(misc + 128);      // [kWarps][kListCap] selected positions
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(lst + kWarps * kListCap);  // [S / 32]
+  float* sc = reinterpret_cast<float*>(mask_s + S / 32);                    // [G][S]
 
   const int split = p.split;
   const int rank = blockIdx.x % split;
@@ -476,20 +598,20 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   const int chunk = ((u.npos + split - 1) / split + 31) / 32 * 32;
   const int p0 = rank * chunk;
   const int p1 = min(u.npos, p0 + chunk);
-  if (chunk > p.slots) {
+  if (chunk > S) {
     if (tid == 0 && rank == 0)
       atomicOr(reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.table)), kStatusRange);
     return;
   }
 
-  // query -> fp32 shared
-  const uint16_t* qg = p.q + uidx * D;
-  for (int d = tid; d < D; d += kThreads) q_s[d] = __uint_as_float((uint32_t)qg[d] << 16);
+  // the group's queries -> fp32 shared
+  const uint16_t* qg = p.q + uidx * G * D;
+  for (int d = tid; d < G * D; d += kThreads) q_s[d] = __uint_as_float((uint32_t)qg[d] << 16);
   __syncthreads();
 
   const bool quant = u.data_kind == LOOPKV_Q4 || u.data_kind == LOOPKV_Q2;
   const bool q4 = u.data_kind == LOOPKV_Q4;
-  float* qs = qs_all + warp * D;
+  float* qs = qs_all + warp * G * D;
   const float sscale = p.score_scale;
   const int blk0 = p0 / 32;
   const int blk1 = (p1 + 31) / 32;
@@ -497,83 +619,121 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   const int qend = min(blk1, nqb);
 
   // ------------------------------------------------------------- pass 1
-  float lmax = -INFINITY;
-  if (q4) lmax = key_pass<D, true>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, warp, lane);
-  else if (quant)
-    lmax = key_pass<D, false>(u, blk0, qend, p0, p1, q_s, qs, sc, sscale, warp, lane);
+  float lmax[G];
+#pragma unroll
+  for (int r = 0; r < G; ++r) lmax[r] = -INFINITY;
+  if (q4) key_pass<D, true, G>(u, blk0, qend, p0, p1, q_s, qs, sc, S, sscale, warp, lane, lmax);
+  else if (quant) key_pass<D, false, G>(u, blk0, qend, p0, p1, q_s, qs, sc, S, sscale, warp, lane, lmax);
   // the warp's first value block is requested now, ahead of the softmax merge
-  constexpr int LPT = D / 64;       // lanes per token in pass 2 (64 channels per lane)
-  constexpr int TPI = 32 / LPT;     // tokens per warp iteration in pass 2
+  constexpr int LPT = (D / 64) * G;  // lanes per token in pass 2
+  constexpr int TPI = 32 / LPT;      // tokens per warp iteration in pass 2
   const int hf = lane % LPT;
   const size_t vrow = D / 4;  // bytes per token of a value plane / value meta
   const int qlim = min(p1, u.nq);
-  const size_t row0 = ((size_t)(blk0 + warp) * 32 + lane / LPT) * vrow + hf * 16;
-  const uint8_t* vh = u.data + u.Ld.v_hi + row0;
-  const uint8_t* vm = u.data + u.Ld.v_meta + row0;
+  const size_t trow = ((size_t)(blk0 + warp) * 32 + lane / LPT) * vrow;
+  const uint8_t* vh = u.data + u.Ld.v_hi + trow + hf * (VS::CH / 4);
+  const uint8_t* vm = u.data + u.Ld.v_meta + trow + (hf * VS::CH / 32) * 8;
   constexpr size_t VSTEP = (size_t)kWarps * 32 * (D / 4);
   auto full_block = [&](int bk) { return (bk + 1) * 32 <= qlim; };
-  uint4 nh[LPT];
-  float4 nm[LPT];
+  uint32_t nh[LPT][VS::NW];
+  float nm[LPT][2 * VS::NGRP];
   if (blk0 + warp < blk1 && full_block(blk0 + warp)) {
 #pragma unroll
     for (int it = 0; it < LPT; ++it) {
-      nh[it] = ld_stream(vh + it * TPI * vrow);
-      nm[it] = ldg128f(vm + it * TPI * vrow);
+      load_words<VS::NW>(nh[it], vh + it * TPI * vrow);
+      load_meta<VS::NGRP>(nm[it], vm + it * TPI * vrow);
     }
   }
   // bf16 positions: residual, raw cells, the SHARE current token
   for (int pos = max(p0, u.nq) + 32 * warp + lane; pos < p1; pos += 32 * kWarps) {
-    const float s = dot_bf16<D>(raw_row(u, pos, D, false), q_s) * sscale;
-    sc[pos - p0] = s;
-    lmax = fmaxf(lmax, s);
-  }
+    float s[G];
+    dot_bf16<D, G>(raw_row(u, pos, D, false), q_s, s);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-  if (lane == 0) misc[warp] = lmax;
-  __syncthreads();
-  float m_r = misc[0];
-#pragma unroll
-  for (int w = 1; w < kWarps; ++w) m_r = fmaxf(m_r, misc[w]);
-
-  // exponentials relative to the CTA max, and their sum
-  float lsum = 0.f;
-  for (int i = tid; i < p1 - p0; i += kThreads) {
-    const float e = exp2f(sc[i] - m_r);
-    sc[i] = e;
-    lsum += e;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  __syncthreads();  // everyone has read misc[]
-  if (lane == 0) misc[8 + warp] = lsum;
-  __syncthreads();
-  float l_r = 0.f;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) l_r += misc[8 + w];
-  if (p1 <= p0) { m_r = -INFINITY; l_r = 0.f; }
-
-  // merge across the cluster: unit logsumexp (log2 units)
-  float M = m_r, L = l_r;
-  if (split > 1) {
-    cg::cluster_group cluster = cg::this_cluster();
-    if (tid == 0) { misc[16] = m_r; misc[17] = l_r; }
-    cluster.sync();
-    M = -INFINITY;
-    for (int r = 0; r < split; ++r) M = fmaxf(M, cluster.map_shared_rank(misc, r)[16]);
-    L = 0.f;
-    for (int r = 0; r < split; ++r) {
-      const float* rm = cluster.map_shared_rank(misc, r);
-      if (rm[17] > 0.f) L += rm[17] * exp2f(rm[16] - M);
+    for (int r = 0; r < G; ++r) {
+      sc[r * S + pos - p0] = s[r] * sscale;
+      lmax[r] = fmaxf(lmax[r], s[r] * sscale);
     }
   }
-  const float f = (l_r > 0.f) ? exp2f(m_r - M) / L : 0.f;  // e -> p
+#pragma unroll
+  for (int r = 0; r < G; ++r) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax[r] = fmaxf(lmax[r], __shfl_xor_sync(0xffffffffu, lmax[r], o));
+    if (lane == 0) misc[warp * G + r] = lmax[r];
+  }
+  __syncthreads();
+  float m_r[G];
+#pragma unroll
+  for (int r = 0; r < G; ++r) {
+    m_r[r] = misc[r];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) m_r[r] = fmaxf(m_r[r], misc[w * G + r]);
+  }
+
+  // exponentials relative to the CTA max, and their sum, per query
+  float lsum[G];
+#pragma unroll
+  for (int r = 0; r < G; ++r) {
+    lsum[r] = 0.f;
+    for (int i = tid; i < p1 - p0; i += kThreads) {
+      const float e = exp2f(sc[r * S + i] - m_r[r]);
+      sc[r * S + i] = e;
+      lsum[r] += e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lsum[r] += __shfl_xor_sync(0xffffffffu, lsum[r], o);
+    if (lane == 0) misc[32 + warp * G + r] = lsum[r];
+  }
+  __syncthreads();
+  float l_r[G];
+#pragma unroll
+  for (int r = 0; r < G; ++r) {
+    l_r[r] = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) l_r[r] += misc[32 + w * G + r];
+    if (p1 <= p0) { m_r[r] = -INFINITY; l_r[r] = 0.f; }
+  }
+
+  // merge across the cluster: the unit's logsumexp per query (log2 units)
+  float M[G], L[G];
+#pragma unroll
+  for (int r = 0; r < G; ++r) { M[r] = m_r[r]; L[r] = l_r[r]; }
+  if (split > 1) {
+    cg::cluster_group cluster = cg::this_cluster();
+    if (tid == 0) {
+#pragma unroll
+      for (int r = 0; r < G; ++r) { misc[64 + r] = m_r[r]; misc[72 + r] = l_r[r]; }
+    }
+    cluster.sync();
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      M[r] = -INFINITY;
+      for (int k = 0; k < split; ++k) M[r] = fmaxf(M[r], cluster.map_shared_rank(misc, k)[64 + r]);
+      L[r] = 0.f;
+      for (int k = 0; k < split; ++k) {
+        const float* rm = cluster.map_shared_rank(misc, k);
+        if (rm[72 + r] > 0.f) L[r] += rm[72 + r] * exp2f(rm[64 + r] - M[r]);
+      }
+    }
+  }
+  float f[G], fsub[G];  // e -> p, and p * 2^kSub for the low planes
+#pragma unroll
+  for (int r = 0; r < G; ++r) {
+    f[r] = (l_r[r] > 0.f) ? exp2f(m_r[r] - M[r]) / L[r] : 0.f;
+    fsub[r] = f[r] * pow2(kSub);
+  }
   const float tau = p.tau;
 
   // ------------------------------------------------------------- pass 2
-  float2 acc[32];
+  float2 acc[G][32 / G];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.f, 0.f);
-  float g0 = 0.f, g1 = 0.f;  // per-group constants of the lane's two 32-channel groups
+  for (int r = 0; r < G; ++r)
+#pragma unroll
+    for (int i = 0; i < 32 / G; ++i) acc[r][i] = make_float2(0.f, 0.f);
+  float gc[G][VS::NGRP];  // per-group constants of the lane's value groups, per query
+#pragma unroll
+  for (int r = 0; r < G; ++r)
+#pragma unroll
+    for (int gi = 0; gi < VS::NGRP; ++gi) gc[r][gi] = 0.f;
   int nsel = 0;
   // 4-bit high plane: weight 4 * p * scale; its missing low bits read as 1.5,
   // i.e. + 1.5 * p * scale = 0.375 * (4 * p * scale) per unselected token
@@ -581,16 +741,43 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   // it back out for the constants)
   const float hmul = (q4 ? 4.f : 1.f) * pow2(kSub);
   const float mid_unsel = q4 ? 0.375f * pow2(-kSub) : 0.f;
-  const float fsub = f * pow2(kSub);  // e -> p * 2^kSub for the low planes
   // tau <= 0 selects every 4-bit token: the low planes are read with the high
   // ones in this loop instead of through the selected-position list
   const bool dense_lo = DENSE_LO && q4;
   const size_t lo_off = u.Ld.v_lo - u.Ld.v_hi;
+  // one token-row share of a full or partial block, for every query
+  auto token_share = [&](const uint32_t (&hw)[VS::NW], const float (&mt)[2 * VS::NGRP],
+                         const float (&pt)[G], float mid, const uint8_t* lo_row) {
+    float a[G][VS::NGRP];
+#pragma unroll
+    for (int r = 0; r < G; ++r)
+#pragma unroll
+      for (int gi = 0; gi < VS::NGRP; ++gi) {
+        a[r][gi] = (hmul * pt[r]) * mt[2 * gi];
+        gc[r][gi] = fmaf(mid, a[r][gi], fmaf(pt[r], mt[2 * gi + 1], gc[r][gi]));
+      }
+    value_codes<G>(acc, hw, a);
+    if (dense_lo) {
+      uint32_t lw[VS::NW];
+      load_words<VS::NW>(lw, lo_row);
+#pragma unroll
+      for (int r = 0; r < G; ++r)
+#pragma unroll
+        for (int gi = 0; gi < VS::NGRP; ++gi) a[r][gi] *= 0.25f;
+      value_codes<G>(acc, lw, a);
+    }
+  };
   for (int bk = blk0 + warp; bk < blk1; bk += kWarps, vh += VSTEP, vm += VSTEP) {
     const int pos = bk * 32 + lane;
     const bool active = pos < p1;
-    const float pw = active ? sc[pos - p0] * f : 0.f;
-    const bool sel = q4 && pos < qlim && pw >= tau;
+    float pw[G];
+    bool any = false;
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      pw[r] = active ? sc[r * S + pos - p0] * f[r] : 0.f;
+      any = any || pw[r] >= tau;
+    }
+    const bool sel = q4 && pos < qlim && any;
     const uint32_t ballot = __ballot_sync(0xffffffffu, sel);
     nsel += __popc(ballot);
     if (lane == 0) {
@@ -599,17 +786,24 @@ decode_kernel(const DecodeParams p, const CellList cl) {
     }
     if (full_block(bk)) {
       // a full quantized block: rows arrived with the previous iteration
-      uint4 hw[LPT];
-      float4 mt[LPT];
+      uint32_t hw[LPT][VS::NW];
+      float mt[LPT][2 * VS::NGRP];
 #pragma unroll
-      for (int it = 0; it < LPT; ++it) { hw[it] = nh[it]; mt[it] = nm[it]; }
+      for (int it = 0; it < LPT; ++it) {
+#pragma unroll
+        for (int k = 0; k < VS::NW; ++k) hw[it][k] = nh[it][k];
+#pragma unroll
+        for (int k = 0; k < 2 * VS::NGRP; ++k) mt[it][k] = nm[it][k];
+      }
       if (bk + kWarps < blk1 && full_block(bk + kWarps)) {
 #pragma unroll
         for (int it = 0; it < LPT; ++it) {
-          nh[it] = ld_stream(vh + VSTEP + it * TPI * vrow);
-          nm[it] = ldg128f(vm + VSTEP + it * TPI * vrow);
+          load_words<VS::NW>(nh[it], vh + VSTEP + it * TPI * vrow);
+          load_meta<VS::NGRP>(nm[it], vm + VSTEP + it * TPI * vrow);
         }
-        if (kAheadV > 0 && (lane & 7) == 0) {
+        // vh sits 16 lane bytes into the block's rows when G = 1, so lanes
+        // with lane % 8 == 0 start its lines
+        if (G == 1 && kAheadV > 0 && (lane & 7) == 0) {
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
             prefetch_l2(vh + kAheadV * VSTEP + c * 512);
@@ -620,34 +814,30 @@ decode_kernel(const DecodeParams p, const CellList cl) {
 #pragma unroll
       for (int it = 0; it < LPT; ++it) {
         const int tk = it * TPI + lane / LPT;
-        const float pt = __shfl_sync(0xffffffffu, pw, tk);
+        float pt[G];
+#pragma unroll
+        for (int r = 0; r < G; ++r) pt[r] = __shfl_sync(0xffffffffu, pw[r], tk);
         const float mid = ((ballot >> tk) & 1u) ? 0.f : mid_unsel;
-        const float a0 = (hmul * pt) * mt[it].x, a1 = (hmul * pt) * mt[it].z;
-        g0 = fmaf(mid, a0, fmaf(pt, mt[it].y, g0));
-        g1 = fmaf(mid, a1, fmaf(pt, mt[it].w, g1));
-        value_codes(acc, hw[it], a0, a1);
-        if (dense_lo)
-          value_codes(acc, ld_stream(vh + lo_off + it * TPI * vrow), 0.25f * a0, 0.25f * a1);
+        token_share(hw[it], mt[it], pt, mid, vh + lo_off + it * TPI * vrow);
       }
     } else {
       // partial block: quantized tokens below qlim, bf16 ones up to p1
 #pragma unroll
       for (int it = 0; it < LPT; ++it) {
         const int tk = it * TPI + lane / LPT;
-        const float pt = __shfl_sync(0xffffffffu, pw, tk);
+        float pt[G];
+#pragma unroll
+        for (int r = 0; r < G; ++r) pt[r] = __shfl_sync(0xffffffffu, pw[r], tk);
         const int tpos = bk * 32 + tk;
         if (tpos < qlim) {
-          const uint4 hwv = ld_stream(vh + it * TPI * vrow);
-          const float4 mtv = ldg128f(vm + it * TPI * vrow);
+          uint32_t hwv[VS::NW];
+          float mtv[2 * VS::NGRP];
+          load_words<VS::NW>(hwv, vh + it * TPI * vrow);
+          load_meta<VS::NGRP>(mtv, vm + it * TPI * vrow);
           const float mid = ((ballot >> tk) & 1u) ? 0.f : mid_unsel;
-          const float a0 = (hmul * pt) * mtv.x, a1 = (hmul * pt) * mtv.z;
-          g0 = fmaf(mid, a0, fmaf(pt, mtv.y, g0));
-          g1 = fmaf(mid, a1, fmaf(pt, mtv.w, g1));
-          value_codes(acc, hwv, a0, a1);
-          if (dense_lo)
-            value_codes(acc, ld_stream(vh + lo_off + it * TPI * vrow), 0.25f * a0, 0.25f * a1);
+          token_share(hwv, mtv, pt, mid, vh + lo_off + it * TPI * vrow);
         } else if (tpos < p1) {
-          value_raw(acc, raw_row(u, tpos, D, true) + hf * 128, pt);
+          value_raw<G>(acc, raw_row(u, tpos, D, true) + hf * VS::CH * 2, pt);
         }
       }
     }
@@ -664,48 +854,55 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       if (word == 0u) continue;
       const int cnt = __popc(word);
       if (nlist + cnt > kListCap) {
-        low_planes<D, LPT>(acc, u, my, nlist, sc, p0, fsub, lane);
+        low_planes<D, G, LPT>(acc, u, my, nlist, sc, S, p0, fsub, lane);
         nlist = 0;
       }
       if ((word >> lane) & 1u) my[nlist + __popc(word & ((1u << lane) - 1u))] = bk * 32 + lane;
       nlist += cnt;
       __syncwarp();
     }
-    if (nlist > 0) low_planes<D, LPT>(acc, u, my, nlist, sc, p0, fsub, lane);
+    if (nlist > 0) low_planes<D, G, LPT>(acc, u, my, nlist, sc, S, p0, fsub, lane);
   }
   // undo the per-channel 2^o of the code conversion, add the per-group
-  // constants, then reduce over the lanes that share a channel half
+  // constants, then reduce over the lanes that share a channel range
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int j = (2 * i) & 15;
-    acc[i].x = fmaf(acc[i].x, pow2(149 - kSub - code2_off(j)), i < 16 ? g0 : g1);
-    acc[i].y = fmaf(acc[i].y, pow2(149 - kSub - code2_off(j + 1)), i < 16 ? g0 : g1);
-  }
+  for (int r = 0; r < G; ++r)
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-#pragma unroll
-    for (int o = 16; o >= LPT; o >>= 1) {
-      acc[i].x += __shfl_xor_sync(0xffffffffu, acc[i].x, o);
-      acc[i].y += __shfl_xor_sync(0xffffffffu, acc[i].y, o);
+    for (int i = 0; i < 32 / G; ++i) {
+      const int j = (2 * i) & 15;
+      const float gcon = gc[r][(2 * i) / 32];
+      acc[r][i].x = fmaf(acc[r][i].x, pow2(149 - kSub - code2_off(j)), gcon);
+      acc[r][i].y = fmaf(acc[r][i].y, pow2(149 - kSub - code2_off(j + 1)), gcon);
     }
-  }
+#pragma unroll
+  for (int r = 0; r < G; ++r)
+#pragma unroll
+    for (int i = 0; i < 32 / G; ++i) {
+#pragma unroll
+      for (int o = 16; o >= LPT; o >>= 1) {
+        acc[r][i].x += __shfl_xor_sync(0xffffffffu, acc[r][i].x, o);
+        acc[r][i].y += __shfl_xor_sync(0xffffffffu, acc[r][i].y, o);
+      }
+    }
   if (lane < LPT) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      reinterpret_cast<float2*>(red + warp * D + lane * 64)[i] = acc[i];
+    for (int r = 0; r < G; ++r)
+#pragma unroll
+      for (int i = 0; i < 32 / G; ++i)
+        reinterpret_cast<float2*>(red + (warp * G + r) * D + lane * VS::CH)[i] = acc[r][i];
   }
-  if (lane == 0) misc[24 + warp] = __int_as_float(nsel);
+  if (lane == 0) misc[80 + warp] = __int_as_float(nsel);
   __syncthreads();
-  for (int d = tid; d < D; d += kThreads) {
+  for (int d = tid; d < G * D; d += kThreads) {
     float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) o += red[w * D + d];
+    for (int w = 0; w < kWarps; ++w) o += red[w * G * D + d];
     o_s[d] = o;
   }
   if (tid == 0) {
     int t = 0;
-    for (int w = 0; w < kWarps; ++w) t += __float_as_int(misc[24 + w]);
-    misc[32] = __int_as_float(t);
+    for (int w = 0; w < kWarps; ++w) t += __float_as_int(misc[80 + w]);
+    misc[88] = __int_as_float(t);
   }
   __syncthreads();
 
@@ -713,38 +910,46 @@ decode_kernel(const DecodeParams p, const CellList cl) {
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     if (rank == 0) {
-      for (int d = tid; d < D; d += kThreads) {
+      for (int d = tid; d < G * D; d += kThreads) {
         float o = 0.f;
-        for (int r = 0; r < split; ++r) o += cluster.map_shared_rank(o_s, r)[d];
-        p.out[uidx * D + d] = o;
+        for (int k = 0; k < split; ++k) o += cluster.map_shared_rank(o_s, k)[d];
+        p.out[uidx * G * D + d] = o;
       }
       if (tid == 0) {
         int t = 0;
-        for (int r = 0; r < split; ++r) t += __float_as_int(cluster.map_shared_rank(misc, r)[32]);
+        for (int k = 0; k < split; ++k) t += __float_as_int(cluster.map_shared_rank(misc, k)[88]);
         if (p.nsel) p.nsel[uidx] = t;
-        if (p.lse) p.lse[uidx] = (M + log2f(L)) * 0.69314718055994531f;
+        if (p.lse) {
+#pragma unroll
+          for (int r = 0; r < G; ++r) p.lse[uidx * G + r] = (M[r] + log2f(L[r])) * 0.69314718055994531f;
+        }
       }
     }
     cluster.sync();  // keep every CTA's shared memory alive until rank 0 has read it
   } else {
-    for (int d = tid; d < D; d += kThreads) p.out[uidx * D + d] = o_s[d];
+    for (int d = tid; d < G * D; d += kThreads) p.out[uidx * G * D + d] = o_s[d];
     if (tid == 0) {
-      if (p.nsel) p.nsel[uidx] = __float_as_int(misc[32]);
-      if (p.lse) p.lse[uidx] = (M + log2f(L)) * 0.69314718055994531f;
+      if (p.nsel) p.nsel[uidx] = __float_as_int(misc[88]);
+      if (p.lse) {
+#pragma unroll
+        for (int r = 0; r < G; ++r) p.lse[uidx * G + r] = (M[r] + log2f(L[r])) * 0.69314718055994531f;
+      }
     }
   }
 }
 
-template <int D>
-size_t decode_smem(int slots) {
-  return sizeof(float) * (size_t)(D + 2 * kWarps * D + D + 64 + kWarps * kListCap + slots / 32 + slots);
+// Shared memory of one CTA for S score slots per query.
+template <int D, int G>
+constexpr size_t decode_smem(int S) {
+  return sizeof(float) * ((size_t)G * D * (2 + 2 * kWarps) + 128 + kWarps * kListCap + S / 32 +
+                          (size_t)G * S);
 }
 
-template <int D, bool DENSE_LO>
+template <int D, int G, bool DENSE_LO>
 int launch_decode_t(const DecodeParams& p, const CellList& cells, cudaStream_t stream) {
-  const size_t smem = decode_smem<D>(p.slots);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, DENSE_LO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const size_t smem = decode_smem<D, G>(p.slots);
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, DENSE_LO>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_cells * p.batch * p.n_heads;
   cudaLaunchConfig_t cfg{};
@@ -763,20 +968,47 @@ int launch_decode_t(const DecodeParams& p, const CellList& cells, cudaStream_t s
   }
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, DENSE_LO>, p, cells);
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, G, DENSE_LO>, p, cells);
   return (int)e;
+}
+
+template <int D, int G>
+int launch_decode_g(const DecodeParams& p, const CellList& cells, cudaStream_t s) {
+  const bool dense = !(p.tau > 0.f);
+  return dense ? launch_decode_t<D, G, true>(p, cells, s) : launch_decode_t<D, G, false>(p, cells, s);
+}
+
+template <int D>
+int launch_decode_d(const DecodeParams& p, const CellList& cells, cudaStream_t s) {
+  if (p.group == 2) return launch_decode_g<D, 2>(p, cells, s);
+  if (p.group == 4) return launch_decode_g<D, 4>(p, cells, s);
+  return launch_decode_g<D, 1>(p, cells, s);
+}
+
+// Largest score slots per query that keep two CTAs on an SM (at most
+// kMaxSlots in all), for a group of G queries.
+template <int D, int G>
+constexpr int max_slots_g() {
+  constexpr size_t kBudget = 113 * 1024;  // bytes of shared memory per CTA for two CTAs per SM
+  constexpr size_t fixed = decode_smem<D, G>(0);
+  constexpr size_t per_query = (kBudget - fixed) / sizeof(float);  // G * S + S / 32 <= this
+  constexpr size_t s = per_query * 32 / (32 * G + 1) / 32 * 32;
+  return (int)(s * G > (size_t)kMaxSlots ? kMaxSlots / G : s);
 }
 
 }  // namespace
 
-int decode_max_slots(int) { return kMaxSlots; }
+int decode_max_slots(int head_dim, int group) {
+  if (head_dim == 64)
+    return group == 4 ? max_slots_g<64, 4>() : group == 2 ? max_slots_g<64, 2>() : max_slots_g<64, 1>();
+  return group == 4 ? max_slots_g<128, 4>() : group == 2 ? max_slots_g<128, 2>() : max_slots_g<128, 1>();
+}
 int decode_max_split() { return kMaxSplit; }
 
 int launch_decode(const DecodeParams& p, const CellList& cells, void* stream, int head_dim) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool dense = !(p.tau > 0.f);
-  if (head_dim == 64) return dense ? launch_decode_t<64, true>(p, cells, s) : launch_decode_t<64, false>(p, cells, s);
-  return dense ? launch_decode_t<128, true>(p, cells, s) : launch_decode_t<128, false>(p, cells, s);
+  if (head_dim == 64) return launch_decode_d<64>(p, cells, s);
+  return launch_decode_d<128>(p, cells, s);
 }
 
 }  // namespace loopkv

@@ -104,15 +104,16 @@ struct AppendParams {
 struct DecodeParams {
   const uint8_t* table;
   const uint8_t* cache;
-  const uint16_t* q;           // [n_cells][batch][H][D]
-  float* out;                  // [n_cells][batch][H][D]
-  float* lse;                  // nullable [n_cells][batch][H]
+  const uint16_t* q;           // [n_cells][batch][H][group][D]
+  float* out;                  // [n_cells][batch][H][group][D]
+  float* lse;                  // nullable [n_cells][batch][H][group]
   uint32_t* mask;              // nullable [n_cells][batch][H][mask_words]
   int32_t* nsel;               // nullable [n_cells][batch][H]
   int32_t mask_words;
   int32_t n_cells, batch, n_heads;
+  int32_t group;               // query heads per KV head: 1, 2 or 4
   int32_t split;               // CTAs per unit (a thread-block cluster when > 1)
-  int32_t slots;               // score slots per CTA (multiple of 32)
+  int32_t slots;               // score slots per query per CTA (multiple of 32)
   float tau;
   float score_scale;           // sm_scale * log2(e): scores are kept in log2 units
 };
@@ -122,7 +123,7 @@ int launch_append(const AppendParams& p, const CellList& cells, void* stream, in
 int launch_commit_lengths(uint8_t* table, const CellList& cells, int n_cells, int batch,
                           const int32_t* n_new, void* stream);
 int launch_decode(const DecodeParams& p, const CellList& cells, void* stream, int head_dim);
-int decode_max_slots(int head_dim);     // largest per-CTA score slots the kernel accepts
+int decode_max_slots(int head_dim, int group);  // largest per-query score slots per CTA
 int decode_max_split();                 // largest cluster size used
 
 }  // namespace loopkv

@@ -16,6 +16,7 @@ using namespace loopkv;
 
 struct loopkv_plan {
   int n_loops = 0, n_layers = 0, n_cells = 0, H = 0, D = 0, max_batch = 0;
+  int group = 1;                  // query heads per KV head
   float tau = 0.f, sm_scale = 0.f;
   std::vector<uint8_t> kinds;     // [cells]
   std::vector<int32_t> cap;       // [max_batch]
@@ -48,6 +49,8 @@ loopkv_status validate_desc(const loopkv_plan_desc* d) {
   if (d->n_kv_heads > (1 << 16)) return LOOPKV_ERR_PLAN;
   if (!(d->tau >= 0.f) || !std::isfinite(d->tau)) return LOOPKV_ERR_PLAN;
   if (!std::isfinite(d->sm_scale)) return LOOPKV_ERR_PLAN;
+  if (d->q_per_kv != 0 && d->q_per_kv != 1 && d->q_per_kv != 2 && d->q_per_kv != 4)
+    return LOOPKV_ERR_PLAN;
   for (int b = 0; b < d->max_batch; ++b)
     if (d->capacity[b] < 0 || d->capacity[b] > kMaxCapacity) return LOOPKV_ERR_PLAN;
   const int cells = d->n_loops * d->n_layers;
@@ -121,6 +124,7 @@ loopkv_status loopkv_plan_load(const loopkv_plan_desc* desc, void* d_table, size
   p->n_layers = desc->n_layers;
   p->n_cells = desc->n_loops * desc->n_layers;
   p->H = desc->n_kv_heads;
+  p->group = desc->q_per_kv > 1 ? desc->q_per_kv : 1;
   p->D = desc->head_dim;
   p->max_batch = desc->max_batch;
   p->tau = desc->tau;
@@ -244,8 +248,9 @@ loopkv_status loopkv_decode(loopkv_plan* p, const int32_t* h_cells, int32_t n_ce
   if (d_mask != nullptr && (mask_words < 0 || !aligned16(d_mask))) return LOOPKV_ERR_INVALID_ARG;
 
   // Split a unit over a cluster of CTAs when its positions do not fit one
-  // CTA's score slots, or when there are too few units to fill the GPU.
-  const int max_slots = decode_max_slots(p->D);
+  // CTA's score slots (per query of the group), or when there are too few
+  // units to fill the GPU.
+  const int max_slots = decode_max_slots(p->D, p->group);
   const long long units = (long long)n_cells * batch * p->H;
   int split = 1;
   auto slots_for = [&](int s) { return ((npos_max + s - 1) / s + 31) / 32 * 32; };
@@ -271,6 +276,7 @@ loopkv_status loopkv_decode(loopkv_plan* p, const int32_t* h_cells, int32_t n_ce
   dp.n_cells = n_cells;
   dp.batch = batch;
   dp.n_heads = p->H;
+  dp.group = p->group;
   dp.split = split;
   dp.slots = slots_for(split);
   dp.tau = p->tau;

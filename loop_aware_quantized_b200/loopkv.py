@@ -52,6 +52,7 @@ class loopkv_plan_desc(ctypes.Structure):
         ("kinds", ctypes.POINTER(ctypes.c_uint8)),
         ("tau", ctypes.c_float),
         ("sm_scale", ctypes.c_float),
+        ("q_per_kv", ctypes.c_int32),
     ]
 
 
@@ -167,7 +168,8 @@ def _check(rc, where):
         raise LoopKVError(rc, where)
 
 
-def make_desc(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau, sm_scale=0.0):
+def make_desc(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau, sm_scale=0.0,
+              q_per_kv=1):
     """Build a loopkv_plan_desc; returns (desc, keepalive arrays)."""
     cap = np.ascontiguousarray(capacity, dtype=np.int32)
     kinds = np.ascontiguousarray(kinds, dtype=np.uint8)
@@ -178,12 +180,14 @@ def make_desc(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau, sm_
     d.kinds = kinds.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
     d.tau = float(tau)
     d.sm_scale = float(sm_scale)
+    d.q_per_kv = int(q_per_kv)
     return d, (cap, kinds)
 
 
-def query_sizes(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau=0.0):
+def query_sizes(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau=0.0, q_per_kv=1):
     """(table_bytes, cache_bytes) a plan needs; raises LoopKVError if invalid."""
-    d, keep = make_desc(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau)
+    d, keep = make_desc(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau,
+                        q_per_kv=q_per_kv)
     rc, sizes = loopkv_plan_query(d)
     _check(rc, "loopkv_plan_query")
     return int(sizes.table_bytes), int(sizes.cache_bytes)
@@ -193,7 +197,7 @@ class Plan:
     """A loaded LoopKV plan with its device table and cache (torch tensors)."""
 
     def __init__(self, n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau,
-                 sm_scale=0.0, device="cuda", stream=None):
+                 sm_scale=0.0, device="cuda", stream=None, q_per_kv=1):
         import torch
         self.n_loops, self.n_layers = n_loops, n_layers
         self.n_cells = n_loops * n_layers
@@ -202,8 +206,9 @@ class Plan:
         self.max_batch = int(self.capacity.size)
         self.kinds = np.ascontiguousarray(kinds, dtype=np.uint8)
         self.tau = float(tau)
+        self.q_per_kv = int(q_per_kv)
         d, keep = make_desc(n_loops, n_layers, n_kv_heads, head_dim, self.capacity, self.kinds,
-                            tau, sm_scale)
+                            tau, sm_scale, q_per_kv)
         rc, sizes = loopkv_plan_query(d)
         _check(rc, "loopkv_plan_query")
         self.table_bytes, self.cache_bytes = int(sizes.table_bytes), int(sizes.cache_bytes)
@@ -246,11 +251,18 @@ class Plan:
         _check(rc, "loopkv_append")
 
     def decode(self, cells, q, out=None, lse=None, mask=None, nsel=None, stream=None):
-        """q: bf16 [n_cells, batch, H, D] on the device; returns out (fp32, same shape)."""
+        """q: bf16 [n_cells, batch, H, D] on the device, or [n_cells, batch, H,
+        q_per_kv, D] for a plan with several query heads per KV head; returns
+        out (fp32, same shape).  lse: [n_cells, batch, H(, q_per_kv)]; mask
+        and nsel are per KV head."""
         import torch
         cells = np.ascontiguousarray(cells, dtype=np.int32)
         assert q.dtype == torch.bfloat16 and q.is_contiguous()
-        nc, batch, H, D = q.shape
+        if q.dim() == 5:
+            nc, batch, H, g, D = q.shape
+        else:
+            (nc, batch, H, D), g = q.shape, 1
+        assert g == self.q_per_kv
         assert nc == cells.size and H == self.n_heads and D == self.head_dim
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float32, device=q.device)

@@ -98,9 +98,11 @@ def raw_values(wl, cell, b, h, t0, t1):
     return px.float_to_bf16_bits(px.normal_from_bits(*u))
 
 
-def query_positions(wl, cell, b, h, n):
-    """Attended positions the query of a unit of length n is built from."""
-    u = px.philox4x32(np.uint32(n), np.uint32(0), _unit_word(wl, b, h), np.uint32(cell),
+def query_positions(wl, cell, b, h, n, rep=0):
+    """Attended positions the query of a unit of length n is built from.
+
+    rep: query head of the KV head's group (0 for one query per KV head)."""
+    u = px.philox4x32(np.uint32(n), np.uint32(rep << 16), _unit_word(wl, b, h), np.uint32(cell),
                       wl.seed, STREAM_QPOS)
     u = [int(x) for x in u]
     want = 3 if wl.query_mode == "sum3" else 1
@@ -115,15 +117,17 @@ def query_positions(wl, cell, b, h, n):
     return picks
 
 
-def query(wl, cell, b, h, n):
-    """bf16 bits [D] of the query of unit (cell, b, h) when it holds n tokens."""
+def query(wl, cell, b, h, n, rep=0):
+    """bf16 bits [D] of the query of unit (cell, b, h) when it holds n tokens.
+
+    rep: query head of the KV head's group; rep 0 is the one-query stream."""
     D = wl.head_dim
     share = wl.kinds[cell] == SHARE
     keys = []
-    for p in query_positions(wl, cell, b, h, n):
+    for p in query_positions(wl, cell, b, h, n, rep):
         src = wl.source_cell(cell) if (share and p < n - 1) else cell
         keys.append(px.bf16_bits_to_float(raw_keys(wl, src, b, h, p, p + 1)[0]))
-    d = np.arange(D, dtype=np.uint32)
+    d = np.arange(D, dtype=np.uint32) + np.uint32(rep << 16)
     u = px.philox4x32(np.uint32(n), d, _unit_word(wl, b, h), np.uint32(cell), wl.seed,
                       STREAM_QNOISE)
     z = px.normal_from_bits(*u)
@@ -135,6 +139,11 @@ def query(wl, cell, b, h, n):
     else:
         x = ((np.float32(2.0) * keys[0]).astype(np.float32) + z).astype(np.float32)
     return px.float_to_bf16_bits(x)
+
+
+def query_group(wl, cell, b, h, n, g):
+    """bf16 bits [g][D]: the queries of the g query heads sharing KV head h."""
+    return np.stack([query(wl, cell, b, h, n, rep=r) for r in range(g)])
 
 
 # ------------------------------------------------------------------ tables

@@ -29,6 +29,42 @@ def workload(config):
     return W.make(config)
 
 
+def _oracle_units(orc, wl, cell, b, n_own, n_src, h):
+    """The oracle's unit (and SHARE source) for (cell, b, h), built from the
+    host generator's raw keys and values."""
+    kind = int(wl.kinds[cell])
+    cap = int(wl.capacity[b])
+    own = orc.OracleUnit(kind, wl.head_dim, cap)
+    if kind == W.SHARE:
+        k = np.zeros((n_own, wl.head_dim), np.uint16)
+        v = np.zeros((n_own, wl.head_dim), np.uint16)
+        k[-1] = W.raw_keys(wl, cell, b, h, n_own - 1, n_own)[0]
+        v[-1] = W.raw_values(wl, cell, b, h, n_own - 1, n_own)[0]
+        own.append(k, v)
+        src_cell = wl.source_cell(cell)
+        src = orc.OracleUnit(int(wl.kinds[src_cell]), wl.head_dim, cap)
+        src.append(W.raw_keys(wl, src_cell, b, h, 0, n_src), W.raw_values(wl, src_cell, b, h, 0, n_src))
+    else:
+        own.append(W.raw_keys(wl, cell, b, h, 0, n_own), W.raw_values(wl, cell, b, h, 0, n_own))
+        src = None
+    return own, src
+
+
+def oracle_group_job(args):
+    """Oracle decode of one KV unit for its group of g query heads.
+
+    args = (config, cell, b, h, n_own, n_src, g).  Returns the host query
+    bits [g][D] and the oracle's per-head outputs, union mask and count."""
+    from oracle import oracle as orc
+    config, cell, b, h, n_own, n_src, g = args
+    wl = workload(config)
+    own, src = _oracle_units(orc, wl, cell, b, n_own, n_src, h)
+    q = W.query_group(wl, cell, b, h, n_own, g)
+    r = orc.decode_group(own, q, wl.tau, src=src, band=BAND)
+    return dict(q=q, out=r.out, lse=r.lse, mask=r.mask, nsel=r.nsel, slack=r.slack,
+                weights=r.weights, kind=int(wl.kinds[cell]))
+
+
 def oracle_unit_job(args):
     """Build the oracle state of one unit and decode it.
 

@@ -72,6 +72,19 @@ def test_plan_query_rejects_invalid_plans(lk):
     assert rc == 1
 
 
+def test_plan_query_checks_the_query_group(lk):
+    # query heads per KV head: 1, 2 or 4 (0 reads as 1); the cache does not
+    # depend on it (the group shares the KV head's storage)
+    base = _query(lk)[1].cache_bytes
+    for g in (0, 1, 2, 4):
+        d, keep = lk.make_desc(2, 2, 2, 64, [64, 96], [0, 2, 1, 0], 0.01, q_per_kv=g)
+        rc, sizes = lk.loopkv_plan_query(d)
+        assert rc == 0 and sizes.cache_bytes == base, g
+    for g in (-1, 3, 5, 8):
+        d, keep = lk.make_desc(2, 2, 2, 64, [64, 96], [0, 2, 1, 0], 0.01, q_per_kv=g)
+        assert lk.loopkv_plan_query(d)[0] == 2, g
+
+
 def test_plan_load_checks_arguments_before_any_device_work(lk):
     d, keep = lk.make_desc(2, 2, 2, 64, [64, 96], [0, 2, 1, 0], 0.01)
     rc, h = lk.loopkv_plan_load(d, None, 0, None, 0, None)
