@@ -48,6 +48,9 @@ def parse():
                     help="CPU work budget of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--q-per-kv", type=int, default=1, choices=[1, 2, 4],
+                    help="query heads per KV head (grouped-query decode); 1 = one query "
+                         "per KV head, the workloads' own shape")
     ap.add_argument("--batch", type=int, default=0,
                     help="sequences per GPU (default: the workload's batch); smaller "
                          "batches are for profiling captures only")
@@ -74,12 +77,13 @@ def per_token_head_bytes(kind, D):
     return 4 * D               # bf16 key + value
 
 
-def decode_bytes(wl, cells, lens_own, lens_src, nsel_total):
+def decode_bytes(wl, cells, lens_own, lens_src, nsel_total, g=1):
     """Algorithmic HBM bytes of one decode launch over `cells`.
 
-    Per unit: each attended position at its storage's per-token bytes (bf16
-    residual and the SHARE current token at 4D bytes), the low-plane rows of
-    the selected positions (D/4 each), the query (2D) and the output (4D).
+    Per unit (KV head): each attended position at its storage's per-token
+    bytes (bf16 residual and the SHARE current token at 4D bytes), read once
+    for the g query heads of the group, the low-plane rows of the selected
+    positions (D/4 each), the queries (2D each) and the outputs (4D each).
     """
     D, H = wl.head_dim, wl.n_heads
     total = 0
@@ -97,7 +101,7 @@ def decode_bytes(wl, cells, lens_own, lens_src, nsel_total):
                 q = min(n_att, qtok)
                 r = n_att - q
             tok = q * per_token_head_bytes(dk, D) + r * 4 * D + (4 * D if share else 0)
-            total += H * (tok + 2 * D + 4 * D)
+            total += H * (tok + g * (2 * D + 4 * D))
     return int(total) + int(nsel_total) * (D // 4)
 
 
@@ -157,15 +161,18 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def workload_text(wl, B):
+def workload_text(wl, B, g=1):
     """One-line description of the benched workload."""
     k = wl.kinds
     plan = "plan %d Q4 / %d Q2 / %d SHARE / %d BF16 cells" % (
         (k == 0).sum(), (k == 1).sum(), (k == 2).sum(), (k == 3).sum())
     ctx = ("%d cached tokens" % int(wl.lengths[0]) if len(set(wl.lengths[:B].tolist())) == 1
            else "ragged %d-%d cached tokens" % (int(wl.lengths[:B].min()), int(wl.lengths[:B].max())))
-    return ("%s: %d loops x %d layers, %d KV heads, head dim %d, batch %d per GPU, %s + 1 "
-            "appended per step, %s, tau %g" % (wl.name, wl.n_loops, wl.n_layers, wl.n_heads,
+    heads = "%d KV heads" % wl.n_heads
+    if g > 1:
+        heads += " x %d query heads each (grouped-query)" % g
+    return ("%s: %d loops x %d layers, %s, head dim %d, batch %d per GPU, %s + 1 "
+            "appended per step, %s, tau %g" % (wl.name, wl.n_loops, wl.n_layers, heads,
                                               wl.head_dim, B, ctx, plan, wl.tau))
 
 
@@ -213,8 +220,9 @@ def ncu_traffic(kernel_src):
 
 # --------------------------------------------------------- oracle baseline
 
-def oracle_baseline(config, seconds, seqs_global):
-    """Time the CPU oracle on a fixed sample of the workload's units.
+def oracle_baseline(config, seconds, seqs_global, g=1):
+    """Time the CPU oracle on a fixed sample of the workload's units (each with
+    its g query heads).
 
     Returns (cell-steps/s, sample description, cores).  A cell-step is B x H
     unit decodes, so the rate is units/s divided by B * H.
@@ -246,24 +254,26 @@ def oracle_baseline(config, seconds, seqs_global):
             sc = wl.source_cell(c)
             src = orc.OracleUnit(int(wl.kinds[sc]), wl.head_dim, cap)
             src.append(W.raw_keys(wl, sc, b, h, 0, n), W.raw_values(wl, sc, b, h, 0, n))
-            q = W.query(wl, c, b, h, n + 1)
+            q = W.query_group(wl, c, b, h, n + 1, g)
         else:
             own.append(W.raw_keys(wl, c, b, h, 0, n + 1), W.raw_values(wl, c, b, h, 0, n + 1))
-            q = W.query(wl, c, b, h, n + 1)
+            q = W.query_group(wl, c, b, h, n + 1, g)
         units.append((own, src, q))
     done = 0
     t0 = time.perf_counter()
     while True:
         for own, src, q in units:
-            orc.decode(own, q, wl.tau, src=src)
+            orc.decode_group(own, q, wl.tau, src=src)
             done += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
     rate_units = done / el
     desc = ("%d oracle decodes of %d sampled units (Q4, Q2, SHARE; %d tokens each, "
-            "%d-token contexts) in %.1f s on 1 core; cell-steps/s = units/s / (%d seqs x %d heads)"
-            % (done, len(units), n + 1, n + 1, el, wl.batch, wl.n_heads))
+            "%d-token contexts%s) in %.1f s on 1 core; cell-steps/s = units/s / (%d seqs x %d "
+            "heads)" % (done, len(units), n + 1, n + 1,
+                        ", %d query heads per unit" % g if g > 1 else "", el, wl.batch,
+                        wl.n_heads))
     return rate_units / (wl.batch * wl.n_heads), desc, 1
 
 
@@ -278,11 +288,11 @@ def run_reference(args, rank, world):
     vals = []
     desc = ""
     for _ in range(args.warmup):
-        oracle_baseline(args.config, 0.5, list(range(wl.batch)))
+        oracle_baseline(args.config, 0.5, list(range(wl.batch)), args.q_per_kv)
     t_all = time.perf_counter()
     for _ in range(args.steps):
         v, desc, cores = oracle_baseline(args.config, budget / max(1, args.steps) + 0.2,
-                                         list(range(wl.batch)))
+                                         list(range(wl.batch)), args.q_per_kv)
         vals.append(v)
     wall = time.perf_counter() - t_all
     value = float(np.mean(vals))
@@ -339,7 +349,8 @@ def main():
     total_steps = args.warmup + args.steps + (0 if args.no_e2e else args.warmup + args.steps)
     cap = np.full(B, int(n0.max()) + total_steps + 32, np.int32)
     cap = (cap + 31) // 32 * 32
-    plan = Plan(wl.n_loops, wl.n_layers, H, D, cap, wl.kinds, wl.tau, device=dev)
+    G = args.q_per_kv
+    plan = Plan(wl.n_loops, wl.n_layers, H, D, cap, wl.kinds, wl.tau, device=dev, q_per_kv=G)
     gen = DeviceGenerator(wl, dev)
 
     # build the cache: every token of every cell through the append kernel
@@ -363,12 +374,13 @@ def main():
             kk, vv = gen.kv(list(cells), seqs, n0 + s, 1)
             k.append(kk)
             v.append(vv)
-            q.append(gen.queries(list(cells), seqs, np.tile(n0 + s + 1, (len(cells), 1))))
+            q.append(gen.queries(list(cells), seqs, np.tile(n0 + s + 1, (len(cells), 1)), g=G))
         return q, k, v
 
     n_dev_steps = args.warmup + args.steps
     inputs = [step_inputs(s) for s in range(n_dev_steps)]
-    outs = [torch.empty((len(c), B, H, D), dtype=torch.float32, device=dev) for c in phase]
+    oshape = (B, H, G, D) if G > 1 else (B, H, D)
+    outs = [torch.empty((len(c),) + oshape, dtype=torch.float32, device=dev) for c in phase]
     nsels = [[torch.zeros((len(c), B, H), dtype=torch.int32, device=dev) for c in phase]
              for _ in range(args.steps)]
     stream = torch.cuda.current_stream()
@@ -408,7 +420,7 @@ def main():
             lens_own = n0 + s + 1
             # non-final loops decode before the final loop's append of this step
             lens_src = n0 + s if pi == 0 else n0 + s + 1
-            dec_bytes += decode_bytes(wl, cells, lens_own, lens_src, int(nsels[i][pi].sum()))
+            dec_bytes += decode_bytes(wl, cells, lens_own, lens_src, int(nsels[i][pi].sum()), G)
 
     elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], world, dev)
     ms_per_step = elapsed_ms / args.steps
@@ -465,7 +477,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, cores = oracle_baseline(args.config, args.cpu_seconds, seqs)
+        v, desc, cores = oracle_baseline(args.config, args.cpu_seconds, seqs, G)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
 
     if rank == 0:
@@ -474,10 +486,11 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "u2/u4 codes, fp32 accumulate", "data": "synthetic",
-            "config": {"workload": workload_text(wl, B),
+            "config": {"workload": workload_text(wl, B, G),
                        "step": "append 1 token + decode, every cell, serving order",
                        "global_batch": B * world, "seq_len": int(n0[0]),
                        "parallelism": "dp%d (independent sequences)" % world,
+                       "q_per_kv": G,
                        "l2": "inputs larger than L2 (KV cache %.1f GB)" % (plan.cache_bytes / 1e9),
                        "build_s": build_s},
             "roofline": roofline,

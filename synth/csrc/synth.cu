@@ -88,22 +88,27 @@ __global__ void gen_kv_kernel(uint16_t* __restrict__ k, uint16_t* __restrict__ v
 // One warp per (c, b, h) query; lanes over channels.
 // mode 0: sum of raw keys at 3 distinct attended positions + 0.5 * N(0,1)
 // mode 1: 2 * raw key at one attended position + N(0,1)
+// One warp per query: [n_cells][batch][H][g][D], query head rep < g of KV
+// head h (rep 0 is the one-query stream; rep r offsets the stream words by
+// r << 16, as the host generator does).
 __global__ void gen_q_kernel(uint16_t* __restrict__ q, const int32_t* __restrict__ cells,
                              const int32_t* __restrict__ srcs, const int32_t* __restrict__ seqs,
-                             const int32_t* __restrict__ lens, int n_cells, int batch, int H, int D,
-                             int mode, int table_cells, const float* __restrict__ chscale,
+                             const int32_t* __restrict__ lens, int n_cells, int batch, int H, int g,
+                             int D, int mode, int table_cells, const float* __restrict__ chscale,
                              uint32_t seed, float nscale) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= n_cells * batch * H) return;
-  const int h = warp % H;
-  const int bl = (warp / H) % batch;
-  const int c = warp / (H * batch);
+  if (warp >= (long long)n_cells * batch * H * g) return;
+  const int rep = (int)(warp % g);
+  const int h = (int)((warp / g) % H);
+  const int bl = (int)((warp / ((long long)g * H)) % batch);
+  const int c = (int)(warp / ((long long)g * H * batch));
   const int cell = cells[c], src = srcs[c], b = seqs[bl];
   const int n = lens[c * batch + bl];
   if (cell < 0 || cell >= table_cells || src < 0 || src >= table_cells) return;
   const bool share = src != cell;
-  const U4 u = philox((uint32_t)n, 0u, (uint32_t)(h + H * b), (uint32_t)cell, seed, kStreamQPos);
+  const uint32_t rw = (uint32_t)rep << 16;
+  const U4 u = philox((uint32_t)n, rw, (uint32_t)(h + H * b), (uint32_t)cell, seed, kStreamQPos);
   const uint32_t uu[3] = {u.x, u.y, u.z};
   const int want = mode == 0 ? 3 : 1;
   const int kcount = n < want ? n : want;
@@ -124,7 +129,7 @@ __global__ void gen_q_kernel(uint16_t* __restrict__ q, const int32_t* __restrict
       const int kc = (share && p < n - 1) ? src : cell;
       key[i] = from_bf16_bits(key_bits(kc, b, h, (uint32_t)p, d, H, D, chscale, seed, nscale));
     }
-    const U4 un = philox((uint32_t)n, (uint32_t)d, (uint32_t)(h + H * b), (uint32_t)cell, seed,
+    const U4 un = philox((uint32_t)n, (uint32_t)d + rw, (uint32_t)(h + H * b), (uint32_t)cell, seed,
                          kStreamQNoise);
     const float z = normal_from(un, nscale);
     float x;
@@ -158,16 +163,16 @@ int synth_gen_kv(uint16_t* k, uint16_t* v, const int32_t* d_cells, const int32_t
 }
 
 int synth_gen_q(uint16_t* q, const int32_t* d_cells, const int32_t* d_srcs, const int32_t* d_seqs,
-                const int32_t* d_lens, int n_cells, int batch, int H, int D, int mode,
+                const int32_t* d_lens, int n_cells, int batch, int H, int g, int D, int mode,
                 int table_cells, const float* d_chscale, uint32_t seed, float nscale,
                 void* stream) {
-  const long long warps = (long long)n_cells * batch * H;
+  const long long warps = (long long)n_cells * batch * H * g;
   if (warps == 0) return 0;
   const int threads = 256;
   const long long blocks = (warps * 32 + threads - 1) / threads;
   gen_q_kernel<<<(unsigned)blocks, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      q, d_cells, d_srcs, d_seqs, d_lens, n_cells, batch, H, D, mode, table_cells, d_chscale, seed,
-      nscale);
+      q, d_cells, d_srcs, d_seqs, d_lens, n_cells, batch, H, g, D, mode, table_cells, d_chscale,
+      seed, nscale);
   return (int)cudaGetLastError();
 }
 

@@ -27,7 +27,7 @@ def _load():
         lib.synth_gen_kv.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, ctypes.c_uint32,
                                      ctypes.c_float, P]
         lib.synth_gen_kv.restype = I
-        lib.synth_gen_q.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, ctypes.c_uint32,
+        lib.synth_gen_q.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, ctypes.c_uint32,
                                     ctypes.c_float, P]
         lib.synth_gen_q.restype = I
         _lib = lib
@@ -74,12 +74,13 @@ class DeviceGenerator:
         assert rc == 0, rc
         return k, v
 
-    def queries(self, cells, seqs, lens, out=None, stream=None):
-        """bf16 [n_cells, len(seqs), H, D]; lens [n_cells, len(seqs)] = unit lengths."""
+    def queries(self, cells, seqs, lens, out=None, stream=None, g=1):
+        """bf16 [n_cells, len(seqs), H, D] (g = 1) or [n_cells, len(seqs), H, g, D]
+        (g query heads per KV head); lens [n_cells, len(seqs)] = unit lengths."""
         import torch
         wl = self.wl
         srcs = [wl.data_cell(c) for c in cells]
-        shape = (len(cells), len(seqs), wl.n_heads, wl.head_dim)
+        shape = (len(cells), len(seqs), wl.n_heads) + ((g,) if g > 1 else ()) + (wl.head_dim,)
         if out is None:
             out = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
         mode = 0 if wl.query_mode == "sum3" else 1
@@ -87,7 +88,7 @@ class DeviceGenerator:
         d_cells, d_srcs, d_seqs = self._i32(cells), self._i32(srcs), self._i32(seqs)
         d_lens = self._i32(np.asarray(lens).reshape(-1))
         rc = _load().synth_gen_q(_p(out), _p(d_cells), _p(d_srcs), _p(d_seqs), _p(d_lens),
-                                 len(cells), len(seqs), wl.n_heads, wl.head_dim, mode,
+                                 len(cells), len(seqs), wl.n_heads, g, wl.head_dim, mode,
                                  wl.n_cells, _p(self.chscale), wl.seed, self.nscale,
                                  ctypes.c_void_p(s.cuda_stream))
         s.synchronize()

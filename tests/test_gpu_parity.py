@@ -56,6 +56,13 @@ def test_device_generator_matches_host(dev):
             for bl, b in enumerate(seqs):
                 for h in (0, wl.n_heads - 1):
                     assert (q[ci, bl, h] == W.query(wl, c, b, h, int(lens[ci, bl]))).all()
+        # query heads of a KV head's group (grouped-query decode)
+        qg = gen.queries(cells, seqs, lens, g=3).view(torch.int16).cpu().numpy().view(np.uint16)
+        for ci, c in enumerate(cells):
+            for bl, b in enumerate(seqs):
+                for h in (0, wl.n_heads - 1):
+                    ref = W.query_group(wl, c, b, h, int(lens[ci, bl]), 3)
+                    assert (qg[ci, bl, h] == ref).all() and (ref[0] == q[ci, bl, h]).all()
 
 
 def _run_decode_only(config, pool, dev, cells=None, seqs=None, n_sample=16, split=None,
