@@ -243,12 +243,14 @@ __device__ __forceinline__ void dot_bf16(const uint8_t* row, const float* q_s, f
 template <int D, bool Q4, int G>
 __device__ __forceinline__ void dot_codes(const uint4 (&h)[D / 64], const uint4 (&l)[D / 64],
                                           const float2* qs2, float (&dot)[G]) {
-  // four independent accumulators per query keep the fma chains short
-  float2 acc[G][4];
+  // independent accumulators keep the fma chains short: four per query for
+  // one query, fewer when the queries themselves give independent chains
+  constexpr int NA = G >= 4 ? 1 : 4 / G;
+  float2 acc[G][NA];
 #pragma unroll
   for (int r = 0; r < G; ++r)
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[r][k] = make_float2(0.f, 0.f);
+    for (int k = 0; k < NA; ++k) acc[r][k] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < D / 64; ++c) {
     const uint32_t hw[4] = {h[c].x, h[c].y, h[c].z, h[c].w};
@@ -264,17 +266,24 @@ __device__ __forceinline__ void dot_codes(const uint4 (&h)[D / 64], const uint4 
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float4 qq = q4p[i];
-          acc[r][(2 * i) & 3] = fma2(make_float2(qq.x, qq.y), v[2 * i], acc[r][(2 * i) & 3]);
-          acc[r][(2 * i + 1) & 3] =
-              fma2(make_float2(qq.z, qq.w), v[2 * i + 1], acc[r][(2 * i + 1) & 3]);
+          acc[r][(2 * i) % NA] = fma2(make_float2(qq.x, qq.y), v[2 * i], acc[r][(2 * i) % NA]);
+          acc[r][(2 * i + 1) % NA] =
+              fma2(make_float2(qq.z, qq.w), v[2 * i + 1], acc[r][(2 * i + 1) % NA]);
         }
       }
     }
   }
 #pragma unroll
   for (int r = 0; r < G; ++r) {
-    const float2 a = add2(acc[r][0], acc[r][1]), b = add2(acc[r][2], acc[r][3]);
-    dot[r] = (a.x + b.x) + (a.y + b.y);
+    if constexpr (NA == 4) {
+      const float2 a = add2(acc[r][0], acc[r][1]), b = add2(acc[r][2], acc[r][3]);
+      dot[r] = (a.x + b.x) + (a.y + b.y);
+    } else if constexpr (NA == 2) {
+      const float2 a = add2(acc[r][0], acc[r][1]);
+      dot[r] = a.x + a.y;
+    } else {
+      dot[r] = acc[r][0].x + acc[r][0].y;
+    }
   }
 }
 
@@ -311,10 +320,12 @@ __device__ __forceinline__ void load_kgroup(KGroup<D>& g, const uint8_t* kh, siz
 
 // Score one group held in registers for the G queries; s[r] = the lane's
 // score for query r (or -inf past qlim).
+// qf[i]: 2^(kSub - o) of the lane's channel i (o: the bit offset its code
+// keeps after conversion); q_s: the group's queries [G][D].
 template <int D, bool Q4, int G>
-__device__ __forceinline__ void key_group(const KGroup<D>& g, const float (&qv)[G][D / 32],
-                                          const float (&qz)[G][D / 32], float* qs, int pos,
-                                          int qlim, float sscale, int lane, float (&s)[G]) {
+__device__ __forceinline__ void key_group(const KGroup<D>& g, const float (&qf)[D / 32],
+                                          const float* q_s, float* qs, int pos, int qlim,
+                                          float sscale, int lane, float (&s)[G]) {
   constexpr int CPL = D / 32;
   // fold each query into the group's key scale / zero point
   float cpart[G];
@@ -323,8 +334,9 @@ __device__ __forceinline__ void key_group(const KGroup<D>& g, const float (&qv)[
     cpart[r] = 0.f;
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
-      qs[r * D + CPL * lane + i] = qv[r][i] * g.sc[i];
-      cpart[r] = fmaf(qz[r][i], g.zr[i], cpart[r]);
+      const float qz = q_s[r * D + CPL * lane + i];
+      qs[r * D + CPL * lane + i] = (qz * qf[i]) * g.sc[i];
+      cpart[r] = fmaf(qz, g.zr[i], cpart[r]);
     }
   }
 #pragma unroll
@@ -369,17 +381,14 @@ __device__ __forceinline__ void key_pass(const Unit& u, int b_begin, int b_end, 
   constexpr int CPL = D / 32;  // channels per lane for the q fold
   const int first = b_begin + warp;
   if (first >= b_end) return;
-  // q of the lane's channels, times 2^(kSub - o): o is the bit offset the
-  // channel's code keeps after conversion (see codes4_to_pairs / codes2_to_pairs)
-  float qv[G][CPL], qz[G][CPL];
+  // 2^(kSub - o) for the lane's channels: o is the bit offset the channel's
+  // code keeps after conversion (see codes4_to_pairs / codes2_to_pairs)
+  float qf[CPL];
 #pragma unroll
-  for (int r = 0; r < G; ++r)
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      const int j = (CPL * lane + i) & 15;
-      qz[r][i] = q_s[r * D + CPL * lane + i];
-      qv[r][i] = qz[r][i] * pow2(kSub - (Q4 ? code4_off(j >> 1) : code2_off(j)));
-    }
+  for (int i = 0; i < CPL; ++i) {
+    const int j = (CPL * lane + i) & 15;
+    qf[i] = pow2(kSub - (Q4 ? code4_off(j >> 1) : code2_off(j)));
+  }
   const int qlim = min(p1, u.nq);
   constexpr size_t GB = 8 * D;                      // bytes of one group in each block
   constexpr size_t STEP = (size_t)kWarps * GB;      // a warp's stride between its groups
@@ -397,7 +406,7 @@ __device__ __forceinline__ void key_pass(const Unit& u, int b_begin, int b_end, 
     if (hasb) load_kgroup<D, Q4>(b, kh + STEP, lo_off, km + STEP / 4);
     if (kAheadK > 0 && pon && hasb)
       prefetch_kgroup<D, Q4>(kh + kAheadK * STEP, lo_off, km + kAheadK * STEP / 4);
-    key_group<D, Q4, G>(a, qv, qz, qs, bk * 32 + lane, qlim, sscale, lane, s);
+    key_group<D, Q4, G>(a, qf, q_s, qs, bk * 32 + lane, qlim, sscale, lane, s);
     if (bk * 32 + lane < qlim) {
 #pragma unroll
       for (int r = 0; r < G; ++r) {
@@ -413,7 +422,7 @@ __device__ __forceinline__ void key_pass(const Unit& u, int b_begin, int b_end, 
     if (hasa) load_kgroup<D, Q4>(a, kh + STEP, lo_off, km + STEP / 4);
     if (kAheadK > 0 && pon && hasa)
       prefetch_kgroup<D, Q4>(kh + kAheadK * STEP, lo_off, km + kAheadK * STEP / 4);
-    key_group<D, Q4, G>(b, qv, qz, qs, bk * 32 + lane, qlim, sscale, lane, s);
+    key_group<D, Q4, G>(b, qf, q_s, qs, bk * 32 + lane, qlim, sscale, lane, s);
     if (bk * 32 + lane < qlim) {
 #pragma unroll
       for (int r = 0; r < G; ++r) {
@@ -635,11 +644,17 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   const uint8_t* vm = u.data + u.Ld.v_meta + trow + (hf * VS::CH / 32) * 8;
   constexpr size_t VSTEP = (size_t)kWarps * 32 * (D / 4);
   auto full_block = [&](int bk) { return (bk + 1) * 32 <= qlim; };
-  uint32_t nh[LPT][VS::NW];
-  float nm[LPT][2 * VS::NGRP];
-  if (blk0 + warp < blk1 && full_block(blk0 + warp)) {
+  // Up to two queries per KV head: the next block's rows wait in registers.
+  // Four keep no registers for them: rows are loaded as they are used, with
+  // the next block's lines requested into L2 one block ahead (measured
+  // faster for four, slower for two).
+  constexpr bool kRegNext = G <= 2;
+  constexpr int NB = kRegNext ? LPT : 1;
+  uint32_t nh[NB][VS::NW];
+  float nm[NB][2 * VS::NGRP];
+  if (kRegNext && blk0 + warp < blk1 && full_block(blk0 + warp)) {
 #pragma unroll
-    for (int it = 0; it < LPT; ++it) {
+    for (int it = 0; it < NB; ++it) {
       load_words<VS::NW>(nh[it], vh + it * TPI * vrow);
       load_meta<VS::NGRP>(nm[it], vm + it * TPI * vrow);
     }
@@ -784,12 +799,12 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       mask_s[bk - blk0] = ballot;
       if (p.mask != nullptr && q4 && bk < nqb) p.mask[uidx * p.mask_words + bk] = ballot;
     }
-    if (full_block(bk)) {
+    if (kRegNext && full_block(bk)) {
       // a full quantized block: rows arrived with the previous iteration
       uint32_t hw[LPT][VS::NW];
       float mt[LPT][2 * VS::NGRP];
 #pragma unroll
-      for (int it = 0; it < LPT; ++it) {
+      for (int it = 0; it < NB; ++it) {
 #pragma unroll
         for (int k = 0; k < VS::NW; ++k) hw[it][k] = nh[it][k];
 #pragma unroll
@@ -797,7 +812,7 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       }
       if (bk + kWarps < blk1 && full_block(bk + kWarps)) {
 #pragma unroll
-        for (int it = 0; it < LPT; ++it) {
+        for (int it = 0; it < NB; ++it) {
           load_words<VS::NW>(nh[it], vh + VSTEP + it * TPI * vrow);
           load_meta<VS::NGRP>(nm[it], vm + VSTEP + it * TPI * vrow);
         }
@@ -819,6 +834,26 @@ decode_kernel(const DecodeParams p, const CellList cl) {
         for (int r = 0; r < G; ++r) pt[r] = __shfl_sync(0xffffffffu, pw[r], tk);
         const float mid = ((ballot >> tk) & 1u) ? 0.f : mid_unsel;
         token_share(hw[it], mt[it], pt, mid, vh + lo_off + it * TPI * vrow);
+      }
+    } else if (!kRegNext && full_block(bk)) {
+      // a full quantized block, rows loaded as used; the next block's lines
+      // (V_hi rows, then V_meta rows, D / 16 lines each) go to L2 first
+      if (bk + kWarps < qend && lane < 2 * (D / 16)) {
+        const size_t blk = (size_t)(bk + kWarps) * 32 * vrow + (lane % (D / 16)) * 128;
+        prefetch_l2(u.data + (lane < D / 16 ? u.Ld.v_hi : u.Ld.v_meta) + blk);
+      }
+#pragma unroll
+      for (int it = 0; it < LPT; ++it) {
+        const int tk = it * TPI + lane / LPT;
+        float pt[G];
+#pragma unroll
+        for (int r = 0; r < G; ++r) pt[r] = __shfl_sync(0xffffffffu, pw[r], tk);
+        uint32_t hwv[VS::NW];
+        float mtv[2 * VS::NGRP];
+        load_words<VS::NW>(hwv, vh + it * TPI * vrow);
+        load_meta<VS::NGRP>(mtv, vm + it * TPI * vrow);
+        const float mid = ((ballot >> tk) & 1u) ? 0.f : mid_unsel;
+        token_share(hwv, mtv, pt, mid, vh + lo_off + it * TPI * vrow);
       }
     } else {
       // partial block: quantized tokens below qlim, bf16 ones up to p1
