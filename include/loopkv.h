@@ -214,6 +214,55 @@ loopkv_status loopkv_check(loopkv_plan* plan, void* stream);
 /* Static description of a status code. */
 const char* loopkv_status_string(loopkv_status status);
 
+/* ---- Planner ------------------------------------------------------------
+ * "LoopKV: Loop-Aware KV Cache Compression for Serving Looped Transformers",
+ * section 概要: a one-time offline profile gives every (loop, layer) cell a
+ * predicted damage for 4-bit storage, 2-bit storage and reuse of the final
+ * loop's KV (SHARE); damages add over cells; the planner minimizes reads
+ * under budgets for predicted damage and storage.  The pages fix nothing
+ * else; this library reads it as follows.  Per cached token and KV head:
+ *   Q4    stores 6 blocks of D/4 bytes (K hi/lo/meta, V hi/lo/meta) and reads
+ *         5 of them plus a low-plane row for a fraction sel_fraction of its
+ *         tokens;
+ *   Q2    stores and reads 4 blocks;
+ *   SHARE stores nothing per token and reads what the final-loop cell of its
+ *         layer reads (its own read of that KV); not allowed in the final loop.
+ * Among the plans within both budgets the one with the fewest reads wins,
+ * then the least damage, then the least storage (ties beyond that: any).
+ * Exact: a dynamic program over layers whose options are the 2 * 3^(L-1)
+ * assignments of a layer's cells, over (damage, storage) states. */
+typedef struct {
+  int32_t n_loops;         /* 1 .. 6 */
+  int32_t n_layers;        /* >= 1; n_loops * n_layers <= 4096 */
+  int32_t head_dim;        /* 64 or 128 */
+  const int32_t* damage;   /* host [n_loops * n_layers][3], loop-major cells:
+                              predicted damage of Q4, Q2 and SHARE in integer
+                              profile units, >= 0 (SHARE ignored in the final
+                              loop) */
+  int64_t damage_budget;   /* >= 0: total damage allowed */
+  int64_t storage_budget;  /* >= 0: bytes per cached token and KV head,
+                              summed over the cells */
+  float sel_fraction;      /* [0, 1]: expected fraction of 4-bit tokens whose
+                              low plane is read; counted in thousandths */
+} loopkv_planner_desc;
+
+typedef struct {
+  double reads;            /* bytes read per decode step per cached token and
+                              KV head, summed over the cells */
+  int64_t damage;          /* total predicted damage */
+  int64_t storage;         /* bytes per cached token and KV head */
+} loopkv_plan_cost;
+
+/* Choose every cell's storage (kinds_out: host [n_loops * n_layers],
+ * loop-major loopkv_kind values, ready for loopkv_plan_desc.kinds) and
+ * report the plan's cost (cost may be NULL).  Host only; no device work.
+ * Errors: LOOPKV_ERR_INVALID_ARG (null pointers, negative values, sizes out
+ * of range), LOOPKV_ERR_PLAN (no plan fits the budgets; kinds_out untouched),
+ * LOOPKV_ERR_UNSUPPORTED (more than 2^20 (damage, storage) states after the
+ * budgets are capped at what the cells can use). */
+loopkv_status loopkv_plan_optimize(const loopkv_planner_desc* desc, uint8_t* kinds_out,
+                                   loopkv_plan_cost* cost);
+
 #ifdef __cplusplus
 }
 #endif

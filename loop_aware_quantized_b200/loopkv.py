@@ -56,6 +56,22 @@ class loopkv_plan_desc(ctypes.Structure):
     ]
 
 
+class loopkv_planner_desc(ctypes.Structure):
+    _fields_ = [
+        ("n_loops", ctypes.c_int32),
+        ("n_layers", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("damage", ctypes.POINTER(ctypes.c_int32)),
+        ("damage_budget", ctypes.c_int64),
+        ("storage_budget", ctypes.c_int64),
+        ("sel_fraction", ctypes.c_float),
+    ]
+
+
+class loopkv_plan_cost(ctypes.Structure):
+    _fields_ = [("reads", ctypes.c_double), ("damage", ctypes.c_int64), ("storage", ctypes.c_int64)]
+
+
 class loopkv_sizes(ctypes.Structure):
     _fields_ = [("table_bytes", ctypes.c_size_t), ("cache_bytes", ctypes.c_size_t)]
 
@@ -82,6 +98,8 @@ def _load():
                                     ctypes.POINTER(ctypes.c_uint64)]),
         "loopkv_check": (st, [P, P]),
         "loopkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "loopkv_plan_optimize": (st, [ctypes.POINTER(loopkv_planner_desc), P,
+                                      ctypes.POINTER(loopkv_plan_cost)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -125,6 +143,12 @@ def loopkv_decode(handle, h_cells, n_cells, batch, d_q, d_out, d_lse, d_mask, ma
                   d_nsel, stream):
     return _lib.loopkv_decode(handle, h_cells, n_cells, batch, d_q, d_out, d_lse, d_mask,
                               mask_words, d_nsel, stream)
+
+
+def loopkv_plan_optimize(desc, kinds_out):
+    cost = loopkv_plan_cost()
+    ref = None if desc is None else ctypes.byref(desc)
+    return _lib.loopkv_plan_optimize(ref, kinds_out, ctypes.byref(cost)), cost
 
 
 def loopkv_set_lengths(handle, h_cells, n_cells, batch, h_len, stream):
@@ -298,3 +322,22 @@ class Plan:
 
     def check(self, stream=None):
         _check(loopkv_check(self._handle, _stream_handle(stream)), "loopkv_check")
+
+
+def plan_optimize(n_loops, n_layers, head_dim, damage, damage_budget, storage_budget,
+                  sel_fraction=0.0):
+    """Plan every cell (loop-major kinds) to minimize reads within a damage and
+    a storage budget.  damage: int [n_loops * n_layers, 3] (Q4, Q2, SHARE);
+    storage_budget: bytes per cached token and KV head.  Returns (kinds,
+    {"reads", "damage", "storage"}); raises LoopKVError when nothing fits."""
+    dmg = np.ascontiguousarray(damage, dtype=np.int32).reshape(-1, 3)
+    assert dmg.shape[0] == n_loops * n_layers
+    d = loopkv_planner_desc()
+    d.n_loops, d.n_layers, d.head_dim = n_loops, n_layers, head_dim
+    d.damage = dmg.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    d.damage_budget, d.storage_budget = int(damage_budget), int(storage_budget)
+    d.sel_fraction = float(sel_fraction)
+    kinds = np.zeros(n_loops * n_layers, np.uint8)
+    rc, cost = loopkv_plan_optimize(d, _np_ptr(kinds))
+    _check(rc, "loopkv_plan_optimize")
+    return kinds, {"reads": cost.reads, "damage": int(cost.damage), "storage": int(cost.storage)}

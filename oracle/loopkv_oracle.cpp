@@ -470,4 +470,67 @@ int orc_decode(const void* own_p, const void* src_p, const uint16_t* q,
                           n_mask_words, nsel, slack, weights);
 }
 
+// ---- planner ---------------------------------------------------------------
+// The plan that minimizes reads under a damage budget and a storage budget,
+// by trying every assignment (small instances only).  "LoopKV: Loop-Aware KV
+// Cache Compression for Serving Looped Transformers", section 概要: an offline
+// profile gives each (loop, layer) cell a predicted damage for 4-bit storage,
+// 2-bit storage and reuse of the final loop's KV (damages add); the planner
+// minimizes reads under budgets for predicted damage and storage.  Readings:
+//   P1 per cached token and KV head, a 4-bit cell stores its six blocks
+//      (K hi/lo/meta, V hi/lo/meta: 6 x D/4 bytes) and reads five of them plus
+//      the low-plane row of a selected fraction sel of its tokens
+//      (5 + sel quarters of D bytes); a 2-bit cell stores and reads four
+//      blocks; a SHARE cell stores nothing per token and reads what its
+//      layer's final-loop cell reads (its own separate read of that KV);
+//   P2 damages are integers (the profile's units) and add over cells;
+//   P3 among the assignments within both budgets the lowest total reads
+//      wins, then the lowest damage, then the lowest storage.
+// Units: storage in quarters of D bytes; reads in thousandths of a quarter
+// of D bytes, sel_milli = round(1000 sel).  damage: [cells][3] (Q4, Q2,
+// SHARE), loop-major cells.  kinds_out: loop-major, 0 = Q4, 1 = Q2,
+// 2 = SHARE.  Returns 0, or -1 when no assignment fits (or bad input).
+int orc_plan_brute(int n_loops, int n_layers, const int32_t* damage, int64_t damage_budget,
+                   int64_t storage_budget_q, int sel_milli, uint8_t* kinds_out,
+                   int64_t* best_reads, int64_t* best_damage, int64_t* best_storage) {
+  const int L = n_loops, N = n_layers, cells = L * N;
+  if (L < 1 || N < 1 || cells > 16) return -1;
+  auto options = [&](int c) { return (c / N == L - 1) ? 2 : 3; };  // no SHARE in the final loop
+  std::vector<int> choice(cells, 0);
+  bool found = false;
+  int64_t br = 0, bd = 0, bs = 0;
+  std::vector<uint8_t> best(cells, 0);
+  for (;;) {
+    int64_t rd = 0, dm = 0, st = 0;
+    for (int c = 0; c < cells; ++c) {
+      const int k = choice[c];
+      dm += damage[c * 3 + k];
+      if (k == 0) { st += 6; rd += 5000 + sel_milli; }
+      else if (k == 1) { st += 4; rd += 4000; }
+      else {
+        const int fk = choice[(L - 1) * N + c % N];  // the layer's final-loop cell
+        rd += fk == 0 ? 5000 + sel_milli : 4000;
+      }
+    }
+    if (dm <= damage_budget && st <= storage_budget_q) {
+      bool better = !found || rd < br || (rd == br && (dm < bd || (dm == bd && st < bs)));
+      if (better) {
+        found = true; br = rd; bd = dm; bs = st;
+        for (int c = 0; c < cells; ++c) best[c] = static_cast<uint8_t>(choice[c]);
+      }
+    }
+    int c = 0;
+    while (c < cells) {
+      if (++choice[c] < options(c)) break;
+      choice[c] = 0;
+      ++c;
+    }
+    if (c == cells) break;
+  }
+  if (!found) return -1;
+  for (int c = 0; c < cells; ++c) kinds_out[c] = best[c];
+  *best_reads = br; *best_damage = bd; *best_storage = bs;
+  return 0;
+}
+
 }  // extern "C"

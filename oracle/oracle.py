@@ -46,6 +46,9 @@ def _load():
     lib.orc_decode_group.argtypes = [P, P, P, ctypes.c_int, ctypes.c_double, ctypes.c_double,
                                      ctypes.c_double, P, P, P, P, P, P, P]
     lib.orc_decode_group.restype = ctypes.c_int
+    lib.orc_plan_brute.argtypes = [ctypes.c_int, ctypes.c_int, P, ctypes.c_int64, ctypes.c_int64,
+                                   ctypes.c_int, P, P, P, P]
+    lib.orc_plan_brute.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -196,3 +199,19 @@ def decode_group(unit, q_bits, tau, src=None, sm_scale=0.0, band=1e-6):
         raise ValueError("oracle decode rejected its input")
     return GroupDecodeResult(out=out, lse=lse, mask=mask[: nw[0]].copy(), nsel=int(nsel[0]),
                              slack=slack, weights=weights[: g * npos].reshape(g, npos).copy())
+
+
+def plan_brute(n_loops, n_layers, damage, damage_budget, storage_budget_q, sel_milli):
+    """Best plan by exhaustive search (cells <= 16): (kinds, reads, damage, storage)
+    in the oracle's units, or None when nothing fits the budgets."""
+    dmg = np.ascontiguousarray(damage, dtype=np.int32).reshape(-1, 3)
+    kinds = np.zeros(n_loops * n_layers, np.uint8)
+    r = np.zeros(1, np.int64)
+    d = np.zeros(1, np.int64)
+    s = np.zeros(1, np.int64)
+    rc = _load().orc_plan_brute(n_loops, n_layers, _ptr(dmg), int(damage_budget),
+                                int(storage_budget_q), int(sel_milli), _ptr(kinds), _ptr(r),
+                                _ptr(d), _ptr(s))
+    if rc != 0:
+        return None
+    return kinds, int(r[0]), int(d[0]), int(s[0])

@@ -373,6 +373,43 @@ def pin_group_query_heads():
         assert np.array_equal(rs.weights[h], orc.decode(own, q[h], tau, src=u).weights)
 
 
+def pin_planner_worked_example():
+    # Two loops x two layers, D-quarter units.  Damage [Q4, Q2, SHARE] per
+    # cell (loop-major): c0 [1,5,3], c1 [2,6,4], c2 [0,3,0], c3 [1,2,0] (the
+    # final loop may not SHARE however cheap it looks).  Reads per cell: Q4
+    # 5000, Q2 4000, SHARE = its layer's final cell's; storage Q4 6, Q2 4,
+    # SHARE 0.
+    dm = np.array([[1, 5, 3], [2, 6, 4], [0, 3, 0], [1, 2, 0]])
+    # unlimited: final cells 2-bit (4000 each), c0 and c1 SHARE them (4000
+    # each, damage 3 and 4 < their own 2-bit 5 and 6): reads 16000, damage
+    # 3 + 4 + 3 + 2 = 12, storage 8
+    k, r, d, s = orc.plan_brute(2, 2, dm, 100, 100, 0)
+    assert list(k) == [2, 2, 1, 1] and (r, d, s) == (16000, 12, 8)
+    # damage budget 4: only all-4-bit fits (damage 1 + 2 + 0 + 1)
+    k, r, d, s = orc.plan_brute(2, 2, dm, 4, 100, 0)
+    assert list(k) == [0, 0, 0, 0] and (r, d, s) == (20000, 4, 24)
+    # a selected fraction of 0.25 adds 250 per 4-bit cell, also to a SHARE
+    # cell whose final cell is 4-bit
+    k, r, d, s = orc.plan_brute(2, 2, dm, 4, 100, 250)
+    assert r == 4 * 5250
+    # damage budget 9, storage 14: both layers at 8000 reads (final 2-bit +
+    # SHARE) cost damage 12; layer 1 can keep that (damage 2 + 4 = 6) if
+    # layer 0 stays within 3: its final cell 4-bit + c0 SHARE (0 + 3, reads
+    # 10000, storage 6).  The alternative (layer 0 at 8000, layer 1 all
+    # 4-bit, damage 6 + 3) needs storage 4 + 12 = 16.  So reads 18000,
+    # damage 9, storage 10.
+    k, r, d, s = orc.plan_brute(2, 2, dm, 9, 14, 0)
+    assert list(k) == [2, 2, 0, 1] and (r, d, s) == (18000, 9, 10)
+    # nothing has zero damage in c0
+    assert orc.plan_brute(2, 2, dm, 0, 100, 0) is None
+    # equal reads are settled by damage before storage: with c1's SHARE at
+    # damage 9, c1 keeps its own 2-bit (6) although SHARE would store nothing
+    dm2 = dm.copy()
+    dm2[1, 2] = 9
+    k, r, d, s = orc.plan_brute(2, 2, dm2, 100, 100, 0)
+    assert list(k) == [2, 1, 1, 1] and (r, d, s) == (16000, 3 + 6 + 3 + 2, 12)
+
+
 def pin_high_plane_worked_example():
     # 32 tokens with equal keys (key scale 0, so every weight is 1/32).  Each
     # value token is 0 on channel 0, 15 on channel 1, 13 on channel 2 and 0
@@ -439,4 +476,5 @@ ALL_PINS = [
     pin_high_plane_worked_example,
     pin_mask_properties,
     pin_group_query_heads,
+    pin_planner_worked_example,
 ]

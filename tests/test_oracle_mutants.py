@@ -43,6 +43,11 @@ MUTANTS = [
      "const double* qh = &qd[0];"),
     ("sign of zero point", "static_cast<double>(data->kz[gr * D + d]);",
      "-static_cast<double>(data->kz[gr * D + d]);"),
+    ("planner: SHARE in the final loop", "return (c / N == L - 1) ? 2 : 3;",
+     "return 3;"),
+    ("planner: SHARE reads nothing", "rd += fk == 0 ? 5000 + sel_milli : 4000;", "rd += 0;"),
+    ("planner: damage tie-break dropped", "(rd == br && (dm < bd || (dm == bd && st < bs)))",
+     "(rd == br && st < bs)"),
 ]
 
 
