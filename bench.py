@@ -434,31 +434,58 @@ def main():
         for s in range(args.steps):
             q, k, v = step_inputs(n_dev_steps + s)
             host_in.append([[x.cpu().pin_memory() for x in grp] for grp in (q, k, v)])
-        dq = [torch.empty_like(x) for x in inputs[0][0]]
-        dk = [torch.empty_like(x) for x in inputs[0][1]]
-        dv = [torch.empty_like(x) for x in inputs[0][2]]
-        host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        # Double-buffered serving loop: step s+1's inputs go to the device
+        # (and step s's outputs come back) on a copy stream while step s
+        # decodes; the events order every buffer reuse.
+        copy = torch.cuda.Stream(device=dev)
+        dbuf = [[[torch.empty_like(x) for x in grp] for grp in inputs[0]] for _ in range(2)]
+        obuf = [[torch.empty_like(o) for o in outs] for _ in range(2)]
+        host_out = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+                    for _ in range(2)]
         h2d = sum(x.numel() * x.element_size() for grp in host_in[0] for x in grp)
         d2h = sum(o.numel() * o.element_size() for o in outs)
+        ev_in = [torch.cuda.Event() for _ in range(args.steps)]
+        ev_done = [torch.cuda.Event() for _ in range(args.steps)]
+        ev_out = [torch.cuda.Event() for _ in range(args.steps)]
+
+        def upload(s):
+            with torch.cuda.stream(copy):
+                if s >= 2:
+                    copy.wait_event(ev_done[s - 2])      # step s-2 has read this buffer
+                for dst, src in zip(sum(dbuf[s % 2], []), sum(host_in[s], [])):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[s].record(copy)
+
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        copy.wait_event(e0)
+        upload(0)
         for s in range(args.steps):
-            hq, hk, hv = host_in[s]
-            for dst, src in zip(dq + dk + dv, hq + hk + hv):
-                dst.copy_(src, non_blocking=True)
-            steps.decode_step(plan, phase, dq, dk, dv, outs)
-            for dst, src in zip(host_out, outs):
-                dst.copy_(src, non_blocking=True)
+            stream.wait_event(ev_in[s])
+            if s >= 2:
+                stream.wait_event(ev_out[s - 2])         # step s-2's outputs are read back
+            dq, dk, dv = dbuf[s % 2]
+            steps.decode_step(plan, phase, dq, dk, dv, obuf[s % 2])
+            ev_done[s].record(stream)
+            if s + 1 < args.steps:
+                upload(s + 1)
+            with torch.cuda.stream(copy):
+                copy.wait_event(ev_done[s])
+                for dst, src in zip(host_out[s % 2], obuf[s % 2]):
+                    dst.copy_(src, non_blocking=True)
+                ev_out[s].record(copy)
+        stream.wait_event(ev_out[args.steps - 1])
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0] / args.steps
         e2e = {"value": wl.n_cells * world / (e2e_ms / 1000.0), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e2e_ms}
+               "ms_per_step": e2e_ms,
+               "overlap": "double-buffered: a step's copies overlap the neighbouring decodes"}
         plan.check()
 
     peak, peak_kind = measured_peaks()

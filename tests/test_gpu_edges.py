@@ -159,3 +159,13 @@ def test_argument_errors(cuda_device):
     plan.append([0], k, v, n_new=np.zeros(2, np.int32))
     assert (plan.lengths()[0, :2] == 40).all()
     plan.check()
+
+
+def test_planner_plan_drives_the_cache(pool, cuda_device):
+    # a plan chosen by loopkv_plan_optimize (host) is loaded, filled and
+    # decoded like any other, unit by unit against the oracle
+    from loop_aware_quantized_b200 import plan_optimize
+    damage = np.array([[1, 5, 3], [2, 6, 4], [0, 3, 9], [1, 2, 9]])
+    kinds, cost = plan_optimize(2, 2, 64, damage, 9, 14 * 16, 0.0)
+    assert sorted(set(int(k) for k in kinds)) == [Q4, Q2, SH], kinds
+    _check_spec(_spec(64, tuple(int(k) for k in kinds), (33, 97, 300), 0.02), pool, cuda_device)
