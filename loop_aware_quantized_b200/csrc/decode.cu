@@ -6,28 +6,33 @@
 // precision; one fused kernel runs the per-cell plan.
 //
 // One CTA (8 warps) handles a contiguous, 32-aligned range of one unit's
-// attended positions; when a unit is split over several CTAs they form a
+// attended positions for the G query heads that share the unit's KV head
+// (G = 1, 2 or 4); when a unit is split over several CTAs they form a
 // thread-block cluster and exchange their partial softmax statistics and
 // partial outputs through distributed shared memory, so no global
 // workspace is needed.  The scores of the CTA's range stay in shared memory
 // between the two passes:
-//   pass 1  keys: per 32-token group, q is folded with the group's per-channel
-//           key scales (qs_d = q_d * scale_d) and zero points
-//           (c = sum_d q_d * zero_d), then each lane (one token) forms
-//           sum_d qs_d * code_d + c from its packed planes.  Scores are kept
-//           in log2 units.
-//   softmax the CTA's max and sum of exponentials, merged across the cluster
-//           into the unit's logsumexp.
-//   pass 2  values: lane = position computes p and the selection p >= tau
-//           (a warp ballot gives the mask word of the group); lanes then
-//           work per token (64 channels per lane) accumulating
-//           p * scale * code in fp32 and the per-group constant
+//   pass 1  keys: per 32-token group, each query is folded with the group's
+//           per-channel key scales (qs_d = q_d * scale_d) and zero points
+//           (c = sum_d q_d * zero_d), then each lane (one token) unpacks its
+//           packed planes once and forms sum_d qs_d * code_d + c for every
+//           query.  Scores are kept in log2 units.
+//   softmax per query: the CTA's max and sum of exponentials, merged across
+//           the cluster into the unit's logsumexp.
+//   pass 2  values: lane = position computes p for every query and the
+//           selection (some query has p >= tau; a warp ballot gives the
+//           mask word of the group); lanes then work per token ((D / 64) G
+//           lanes of 64 / G channels) accumulating p * scale * code in fp32
+//           for every query and the per-group constant
 //           p * (zero [+ 1.5 * scale]) separately; the low plane row of a
 //           token is loaded only when the token is selected.
 //   combine warp shuffles reduce the per-token partial outputs, shared
 //           memory reduces across warps, DSMEM across the cluster.
-// No tensor cores: one query per KV head makes this a stream over the
-// cache, bound by HBM bandwidth.
+// Each pass loads a warp's next group into registers while the current one
+// is processed and requests its lines into L2 at the same time.
+// No tensor cores: single-query decode is not a dense contraction; the
+// kernel streams the cache once, and the ALU pipe (one logic op per code)
+// is what bounds it in practice.
 
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
