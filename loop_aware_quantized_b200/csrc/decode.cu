@@ -464,6 +464,32 @@ __device__ __forceinline__ uint32_t ld_stream1(const void* p) {
   return r;
 }
 
+// Asynchronous 16-byte copies global -> shared (L1 bypassed), in groups
+// that a thread waits for; the warp then syncs before reading them.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+               ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// One 32-token value block into a warp's staging buffer: the block's V_hi
+// rows ([32][D / 4] bytes), then its V_meta rows (the same size).  Both are
+// contiguous in the cache and 16-byte aligned.
+template <int D>
+__device__ __forceinline__ void stage_vblock(uint8_t* st, const Unit& u, int bk, int lane) {
+  constexpr int BB = 8 * D;  // bytes of one block of a value plane / of value meta
+  const uint8_t* hi = u.data + u.Ld.v_hi + (size_t)bk * BB;
+  const uint8_t* me = u.data + u.Ld.v_meta + (size_t)bk * BB;
+#pragma unroll
+  for (int i = lane; i < BB / 16; i += 32) {
+    cp_async16(st + 16 * i, hi + 16 * i);
+    cp_async16(st + BB + 16 * i, me + 16 * i);
+  }
+}
+
 // NW plane words of a value row (16 NW bytes, 16-byte aligned for NW = 4).
 template <int NW>
 __device__ __forceinline__ void load_words(uint32_t (&w)[NW], const uint8_t* p) {
@@ -486,6 +512,30 @@ __device__ __forceinline__ void load_meta(float (&m)[2 * NGRP], const uint8_t* p
     m[0] = x.x; m[1] = x.y; m[2] = x.z; m[3] = x.w;
   } else {
     const float2 x = __ldg(reinterpret_cast<const float2*>(p));
+    m[0] = x.x; m[1] = x.y;
+  }
+}
+
+// The same words and (scale, zero) pairs from a staged block in shared memory.
+template <int NW>
+__device__ __forceinline__ void lds_words(uint32_t (&w)[NW], const uint8_t* p) {
+  if constexpr (NW == 4) {
+    const uint4 x = *reinterpret_cast<const uint4*>(p);
+    w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+  } else if constexpr (NW == 2) {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    w[0] = x.x; w[1] = x.y;
+  } else {
+    w[0] = *reinterpret_cast<const uint32_t*>(p);
+  }
+}
+template <int NGRP>
+__device__ __forceinline__ void lds_meta(float (&m)[2 * NGRP], const uint8_t* p) {
+  if constexpr (NGRP == 2) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    m[0] = x.x; m[1] = x.y; m[2] = x.z; m[3] = x.w;
+  } else {
+    const float2 x = *reinterpret_cast<const float2*>(p);
     m[0] = x.x; m[1] = x.y;
   }
 }
@@ -664,6 +714,18 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       load_meta<VS::NGRP>(nm[it], vm + it * TPI * vrow);
     }
   }
+  // Four queries per KV head: full blocks go through two staging buffers
+  // in shared memory, the next block's copy in flight while the current one
+  // is used.  The buffers are the warp's own q * scale rows (free after
+  // pass 1) and its rows of the final reduction (unused until then).
+  uint8_t* const stg0 = reinterpret_cast<uint8_t*>(qs);
+  uint8_t* const stg1 = reinterpret_cast<uint8_t*>(red + warp * G * D);
+  static_assert(kRegNext || 16 * D <= 4 * G * D, "a staged value block must fit a warp's rows");
+  int sti = 0;
+  if (!kRegNext) {
+    if (blk0 + warp < blk1 && full_block(blk0 + warp)) stage_vblock<D>(stg0, u, blk0 + warp, lane);
+    cp_async_commit();
+  }
   // bf16 positions: residual, raw cells, the SHARE current token
   for (int pos = max(p0, u.nq) + 32 * warp + lane; pos < p1; pos += 32 * kWarps) {
     float s[G];
@@ -841,12 +903,14 @@ decode_kernel(const DecodeParams p, const CellList cl) {
         token_share(hw[it], mt[it], pt, mid, vh + lo_off + it * TPI * vrow);
       }
     } else if (!kRegNext && full_block(bk)) {
-      // a full quantized block, rows loaded as used; the next block's lines
-      // (V_hi rows, then V_meta rows, D / 16 lines each) go to L2 first
-      if (bk + kWarps < qend && lane < 2 * (D / 16)) {
-        const size_t blk = (size_t)(bk + kWarps) * 32 * vrow + (lane % (D / 16)) * 128;
-        prefetch_l2(u.data + (lane < D / 16 ? u.Ld.v_hi : u.Ld.v_meta) + blk);
-      }
+      // a full quantized block from its staging buffer; the next full block
+      // is copied into the other one meanwhile
+      const uint8_t* cur = sti ? stg1 : stg0;
+      if (bk + kWarps < blk1 && full_block(bk + kWarps))
+        stage_vblock<D>(sti ? stg0 : stg1, u, bk + kWarps, lane);
+      cp_async_commit();
+      cp_async_wait<1>();
+      __syncwarp();
 #pragma unroll
       for (int it = 0; it < LPT; ++it) {
         const int tk = it * TPI + lane / LPT;
@@ -855,11 +919,13 @@ decode_kernel(const DecodeParams p, const CellList cl) {
         for (int r = 0; r < G; ++r) pt[r] = __shfl_sync(0xffffffffu, pw[r], tk);
         uint32_t hwv[VS::NW];
         float mtv[2 * VS::NGRP];
-        load_words<VS::NW>(hwv, vh + it * TPI * vrow);
-        load_meta<VS::NGRP>(mtv, vm + it * TPI * vrow);
+        lds_words<VS::NW>(hwv, cur + tk * vrow + hf * (VS::CH / 4));
+        lds_meta<VS::NGRP>(mtv, cur + 8 * D + tk * vrow + (hf * VS::CH / 32) * 8);
         const float mid = ((ballot >> tk) & 1u) ? 0.f : mid_unsel;
         token_share(hwv, mtv, pt, mid, vh + lo_off + it * TPI * vrow);
       }
+      __syncwarp();  // the buffer is refilled two blocks on
+      sti ^= 1;
     } else {
       // partial block: quantized tokens below qlim, bf16 ones up to p1
 #pragma unroll
@@ -882,6 +948,7 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       }
     }
   }
+  if (!kRegNext) cp_async_wait<0>();  // nothing stays in flight into the reduction rows
   // low planes of the selected tokens: acc += p * scale * lo.  The warp
   // gathers its selected positions into a list and processes them TPI at a
   // time, so the cost follows the number of selected tokens.

@@ -86,15 +86,17 @@ def test_group_decode_matches_oracle(pool, cuda_device, g, D):
         _run(_spec(D, kinds, lengths, 0.02), g, pool, cuda_device)
 
 
+@pytest.mark.parametrize("g", [2, 4])
 @pytest.mark.parametrize("tau", [0.0, 2.0])
-def test_group_tau_extremes(pool, cuda_device, tau):
-    _run(_spec(128, (Q4, SH, Q2, Q4), (40, 300, 1000), tau), 2, pool, cuda_device)
+def test_group_tau_extremes(pool, cuda_device, tau, g):
+    _run(_spec(128, (Q4, SH, Q2, Q4), (40, 300, 1000), tau), g, pool, cuda_device)
 
 
+@pytest.mark.parametrize("g", [2, 4])
 @pytest.mark.parametrize("split", [2, 4])
-def test_group_cluster_split(pool, cuda_device, split, monkeypatch):
+def test_group_cluster_split(pool, cuda_device, split, g, monkeypatch):
     monkeypatch.setenv("LOOPKV_DECODE_SPLIT", str(split))
-    _run(_spec(128, (Q4, SH, Q2, Q4), (65, 700, 1500), 0.01), 2, pool, cuda_device)
+    _run(_spec(128, (Q4, SH, Q2, Q4), (65, 700, 1500), 0.01), g, pool, cuda_device)
 
 
 def test_group_long_units_split_automatically(pool, cuda_device):
