@@ -12,6 +12,7 @@ from .oracle import (  # noqa: F401
     KIND_BF16,
     KIND_Q2,
     KIND_Q4,
+    KIND_RES2,
     KIND_SHARE,
     DecodeResult,
     OracleUnit,

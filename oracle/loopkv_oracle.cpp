@@ -33,6 +33,26 @@
 //      plane is fetched for the group when any head's weight reaches tau,
 //      and every head of the group reconstructs that token with it (the
 //      selection is the union over the group's heads).
+// "ResidualQuant: KV Cache Quantization for Looped Transformers with 2-Bit
+// Residuals", section 概要 (the abstract): the final loop's KV state is the
+// reference and the other loops keep low-precision residuals against it.
+// Readings for that cell kind (RES2):
+//   R9  a RES2 cell sits in a non-final loop; its reference is the final
+//       loop's cell of the same layer, sequence and head, stored as 4-bit,
+//       2-bit or bf16.  For a position t the residual is d = x - r, where x
+//       is the cell's own bf16 input and r the reference's stored value at t
+//       dequantized in fp32 (r = fl(fl(scale * q) + zero) with the full code
+//       q, no fused multiply-add; the raw value for a bf16 reference), and d
+//       = fl(x - r).  Residuals are quantized like a 2-bit cell (R1, R2);
+//   R10 a residual group is quantized once the cell holds the 32 tokens
+//       after it too (32 (g + 2) tokens for group g), so that the reference,
+//       appended later in a decode step, holds the group by then; the cell
+//       keeps its last 32..63 tokens (all of them below 32) in bf16;
+//   R11 a quantized position reads r^ + d^: r^ the reference's reading as
+//       the cell's own decode takes it (keys at stored precision; a 4-bit
+//       reference's values through the tau rule of R4 with the cell's own
+//       weights), d^ = scale * code + zero of the residual; bf16 positions
+//       read the cell's own token.
 // All attention arithmetic is fp64 (dequantized values, scores, softmax,
 // weighted sum).  Quantization is fp32 because the codes are defined by it.
 //
@@ -49,7 +69,9 @@ namespace {
 
 constexpr int kG = 32;  // group size (R1)
 
-enum Kind { KIND_Q4 = 0, KIND_Q2 = 1, KIND_SHARE = 2, KIND_BF16 = 3 };
+enum Kind { KIND_Q4 = 0, KIND_Q2 = 1, KIND_SHARE = 2, KIND_BF16 = 3, KIND_RES2 = 4 };
+
+constexpr int kResWindow = 64;  // bf16 token slots of a RES2 cell (R10)
 
 float bf16_to_float(uint16_t b) {
   uint32_t u = static_cast<uint32_t>(b) << 16;
@@ -94,12 +116,16 @@ struct Unit {
   std::vector<uint8_t> vq;   // [qtok][D] value codes
   std::vector<float> vs, vz; // [qtok][D/32] per-token value scale, zero
   std::vector<uint16_t> rk, rv;  // residual [R][D] bf16 bits
-  // KIND_BF16: every token raw.
+  // KIND_BF16 and KIND_RES2: every token raw (RES2 derives its residual
+  // codes from these and its reference, R9).
   std::vector<uint16_t> bk, bv;  // [n][D]
   // KIND_SHARE: the current token only.
   std::vector<uint16_t> ck, cv;  // [D]
 
-  int qtok() const { return (kind == KIND_Q4 || kind == KIND_Q2) ? n - residual() : 0; }
+  int qtok() const {
+    if (kind == KIND_RES2) return n / kG >= 2 ? (n / kG - 1) * kG : 0;  // R10
+    return (kind == KIND_Q4 || kind == KIND_Q2) ? n - residual() : 0;
+  }
   int residual() const { return static_cast<int>(rk.size()) / D; }
   int bits() const { return kind == KIND_Q4 ? 4 : 2; }
 
@@ -138,7 +164,7 @@ struct Unit {
     if (kind == KIND_SHARE) {
       ck.assign(k, k + D);
       cv.assign(v, v + D);
-    } else if (kind == KIND_BF16) {
+    } else if (kind == KIND_BF16 || kind == KIND_RES2) {
       bk.insert(bk.end(), k, k + D);
       bv.insert(bv.end(), v, v + D);
     } else {
@@ -149,6 +175,80 @@ struct Unit {
     ++n;
   }
 };
+
+// Quantized residual state of a RES2 unit against its reference (R9, R10):
+// the same arrays a 2-bit cell keeps, for the positions below own.qtok().
+struct ResState {
+  int qtok = 0;
+  std::vector<uint8_t> kq, vq;
+  std::vector<float> ks, kz, vs, vz;
+};
+
+bool reference_ok(const Unit& own, const Unit* ref) {
+  if (ref == nullptr || ref->D != own.D) return false;
+  if (ref->kind == KIND_Q4 || ref->kind == KIND_Q2) return ref->qtok() >= own.qtok();
+  if (ref->kind == KIND_BF16) return ref->n >= own.qtok();
+  return false;
+}
+
+// The reference's stored key / value at (pos, d) in fp32 (R9).
+float ref_key32(const Unit& ref, int pos, int d) {
+  const int D = ref.D;
+  if (ref.kind == KIND_BF16) return bf16_to_float(ref.bk[static_cast<size_t>(pos) * D + d]);
+  const int gr = pos / kG;
+  const float q = static_cast<float>(ref.kq[static_cast<size_t>(pos) * D + d]);
+  const float prod = ref.ks[gr * D + d] * q;
+  return prod + ref.kz[gr * D + d];
+}
+float ref_value32(const Unit& ref, int pos, int d) {
+  const int D = ref.D;
+  if (ref.kind == KIND_BF16) return bf16_to_float(ref.bv[static_cast<size_t>(pos) * D + d]);
+  const size_t j = static_cast<size_t>(pos) * (D / kG) + d / kG;
+  const float q = static_cast<float>(ref.vq[static_cast<size_t>(pos) * D + d]);
+  const float prod = ref.vs[j] * q;
+  return prod + ref.vz[j];
+}
+
+ResState residual_state(const Unit& own, const Unit& ref) {
+  const int D = own.D;
+  ResState st;
+  st.qtok = own.qtok();
+  const int ng = st.qtok / kG;
+  st.kq.resize(static_cast<size_t>(st.qtok) * D);
+  st.vq.resize(static_cast<size_t>(st.qtok) * D);
+  st.ks.resize(static_cast<size_t>(ng) * D);
+  st.kz.resize(static_cast<size_t>(ng) * D);
+  st.vs.resize(static_cast<size_t>(st.qtok) * (D / kG));
+  st.vz.resize(static_cast<size_t>(st.qtok) * (D / kG));
+  float x[kG];
+  uint8_t c[kG];
+  for (int g = 0; g < ng; ++g) {
+    // keys: per channel over the group's 32 tokens
+    for (int d = 0; d < D; ++d) {
+      for (int i = 0; i < kG; ++i) {
+        const int pos = g * kG + i;
+        const float xi = bf16_to_float(own.bk[static_cast<size_t>(pos) * D + d]);
+        x[i] = xi - ref_key32(ref, pos, d);
+      }
+      quantize_group(x, 2, c, &st.ks[g * D + d], &st.kz[g * D + d]);
+      for (int i = 0; i < kG; ++i) st.kq[static_cast<size_t>(g * kG + i) * D + d] = c[i];
+    }
+  }
+  // values: per token over groups of 32 channels
+  for (int pos = 0; pos < st.qtok; ++pos) {
+    for (int j = 0; j < D / kG; ++j) {
+      for (int e = 0; e < kG; ++e) {
+        const int d = j * kG + e;
+        const float xi = bf16_to_float(own.bv[static_cast<size_t>(pos) * D + d]);
+        x[e] = xi - ref_value32(ref, pos, d);
+      }
+      const size_t t = static_cast<size_t>(pos) * (D / kG) + j;
+      quantize_group(x, 2, c, &st.vs[t], &st.vz[t]);
+      for (int e = 0; e < kG; ++e) st.vq[static_cast<size_t>(pos) * D + j * kG + e] = c[e];
+    }
+  }
+  return st;
+}
 
 size_t round128(size_t x) { return (x + 127) / 128 * 128; }
 
@@ -167,15 +267,16 @@ Layout make_layout(int kind, int D, int cap) {
   const size_t vblock = ng * kG * (D / 4);    // one value plane or value meta
   const size_t rblock = static_cast<size_t>(kG) * D * 2;
   size_t off = 0;
-  if (kind == KIND_Q4 || kind == KIND_Q2) {
+  if (kind == KIND_Q4 || kind == KIND_Q2 || kind == KIND_RES2) {
     L.k_hi = off; off += round128(kblock);
     if (kind == KIND_Q4) { L.k_lo = off; off += round128(kblock); }
     L.k_meta = off; off += round128(kblock);
     L.v_hi = off; off += round128(vblock);
     if (kind == KIND_Q4) { L.v_lo = off; off += round128(vblock); }
     L.v_meta = off; off += round128(vblock);
-    L.res_k = off; off += rblock;
-    L.res_v = off; off += rblock;
+    const size_t window = (kind == KIND_RES2) ? rblock * (kResWindow / kG) : rblock;
+    L.res_k = off; off += window;
+    L.res_v = off; off += window;
   } else if (kind == KIND_SHARE) {
     L.cur_k = off; off += round128(static_cast<size_t>(D) * 2);
     L.cur_v = off; off += round128(static_cast<size_t>(D) * 2);
@@ -204,7 +305,7 @@ void orc_quantize_group(const float* x, int bits, uint8_t* code, float* scale,
 
 // ---- unit state ------------------------------------------------------------
 void* orc_unit_new(int kind, int D, int cap) {
-  if (kind < 0 || kind > 3 || (D != 64 && D != 128) || cap < 0) return nullptr;
+  if (kind < 0 || kind > 4 || (D != 64 && D != 128) || cap < 0) return nullptr;
   Unit* u = new Unit();
   u->kind = kind;
   u->D = D;
@@ -229,16 +330,31 @@ int orc_unit_append(void* p, const uint16_t* k, const uint16_t* v, int n_new) {
 
 // Quantized state, for tests: key codes [qtok][D], key scale/zero [qtok/32][D],
 // value codes [qtok][D], value scale/zero [qtok][D/32].  Any pointer may be
-// null.  Returns qtok.
-int orc_unit_export(const void* p, uint8_t* kq, float* ks, float* kz, uint8_t* vq,
-                    float* vs, float* vz) {
+// null.  src: the reference unit of a RES2 unit (else ignored); the codes of
+// a RES2 unit are its residual codes.  Returns qtok, or -1 when a RES2 unit's
+// reference is missing or does not hold its quantized positions.
+int orc_unit_export(const void* p, const void* src, uint8_t* kq, float* ks, float* kz,
+                    uint8_t* vq, float* vs, float* vz) {
   const Unit* u = static_cast<const Unit*>(p);
-  if (kq) std::copy(u->kq.begin(), u->kq.end(), kq);
-  if (ks) std::copy(u->ks.begin(), u->ks.end(), ks);
-  if (kz) std::copy(u->kz.begin(), u->kz.end(), kz);
-  if (vq) std::copy(u->vq.begin(), u->vq.end(), vq);
-  if (vs) std::copy(u->vs.begin(), u->vs.end(), vs);
-  if (vz) std::copy(u->vz.begin(), u->vz.end(), vz);
+  ResState rs;
+  const ResState* st = nullptr;
+  if (u->kind == KIND_RES2) {
+    if (!reference_ok(*u, static_cast<const Unit*>(src))) return -1;
+    rs = residual_state(*u, *static_cast<const Unit*>(src));
+    st = &rs;
+  }
+  const std::vector<uint8_t>& ukq = st ? st->kq : u->kq;
+  const std::vector<float>& uks = st ? st->ks : u->ks;
+  const std::vector<float>& ukz = st ? st->kz : u->kz;
+  const std::vector<uint8_t>& uvq = st ? st->vq : u->vq;
+  const std::vector<float>& uvs = st ? st->vs : u->vs;
+  const std::vector<float>& uvz = st ? st->vz : u->vz;
+  if (kq) std::copy(ukq.begin(), ukq.end(), kq);
+  if (ks) std::copy(uks.begin(), uks.end(), ks);
+  if (kz) std::copy(ukz.begin(), ukz.end(), kz);
+  if (vq) std::copy(uvq.begin(), uvq.end(), vq);
+  if (vs) std::copy(uvs.begin(), uvs.end(), vs);
+  if (vz) std::copy(uvz.begin(), uvz.end(), vz);
   return u->qtok();
 }
 
@@ -246,12 +362,15 @@ size_t orc_region_bytes(int kind, int D, int cap) { return make_layout(kind, D, 
 
 // Write the unit's bytes in the canonical layout; valid[i] = 1 for every byte
 // the layout defines at the unit's current length (unused groups and residual
-// slots stay 0 in both arrays).  Returns 0, or -1 on a size mismatch.
-int orc_unit_serialize(const void* p, uint8_t* out, uint8_t* valid, size_t bytes) {
+// slots stay 0 in both arrays).  src: a RES2 unit's reference (else ignored).
+// Returns 0, or -1 on a size mismatch or a missing / short reference.
+int orc_unit_serialize(const void* p, const void* src, uint8_t* out, uint8_t* valid,
+                       size_t bytes) {
   const Unit* u = static_cast<const Unit*>(p);
   const int D = u->D;
   const Layout L = make_layout(u->kind, D, u->cap);
   if (bytes != L.total) return -1;
+  if (u->kind == KIND_RES2 && !reference_ok(*u, static_cast<const Unit*>(src))) return -1;
   std::memset(out, 0, bytes);
   std::memset(valid, 0, bytes);
   if (u->kind == KIND_SHARE) {
@@ -267,6 +386,15 @@ int orc_unit_serialize(const void* p, uint8_t* out, uint8_t* valid, size_t bytes
     return 0;
   }
   const bool q4 = u->kind == KIND_Q4;
+  const bool res2 = u->kind == KIND_RES2;
+  ResState rs;
+  if (res2) rs = residual_state(*u, *static_cast<const Unit*>(src));
+  const std::vector<uint8_t>& ukq = res2 ? rs.kq : u->kq;
+  const std::vector<float>& uks = res2 ? rs.ks : u->ks;
+  const std::vector<float>& ukz = res2 ? rs.kz : u->kz;
+  const std::vector<uint8_t>& uvq = res2 ? rs.vq : u->vq;
+  const std::vector<float>& uvs = res2 ? rs.vs : u->vs;
+  const std::vector<float>& uvz = res2 ? rs.vz : u->vz;
   const int ngq = u->qtok() / kG;
   for (int g = 0; g < ngq; ++g) {
     // key planes: [g][chunk of 64 channels][token][4 words of 16 codes]
@@ -276,7 +404,7 @@ int orc_unit_serialize(const void* p, uint8_t* out, uint8_t* valid, size_t bytes
           uint32_t hi = 0, lo = 0;
           for (int j = 0; j < 16; ++j) {
             const int d = 64 * c + 16 * w + j;
-            const uint32_t q = u->kq[static_cast<size_t>(g * kG + t) * D + d];
+            const uint32_t q = ukq[static_cast<size_t>(g * kG + t) * D + d];
             const uint32_t plane_hi = q4 ? (q >> 2) : q;
             hi |= (plane_hi & 3u) << (2 * j);
             lo |= (q & 3u) << (2 * j);
@@ -288,15 +416,15 @@ int orc_unit_serialize(const void* p, uint8_t* out, uint8_t* valid, size_t bytes
       }
     }
     // key meta: scale[D] then zero[D]
-    put_bytes(out, valid, L.k_meta + static_cast<size_t>(g) * 8 * D, &u->ks[g * D], 4 * D);
-    put_bytes(out, valid, L.k_meta + static_cast<size_t>(g) * 8 * D + 4 * D, &u->kz[g * D], 4 * D);
+    put_bytes(out, valid, L.k_meta + static_cast<size_t>(g) * 8 * D, &uks[g * D], 4 * D);
+    put_bytes(out, valid, L.k_meta + static_cast<size_t>(g) * 8 * D + 4 * D, &ukz[g * D], 4 * D);
   }
   for (int t = 0; t < u->qtok(); ++t) {
     // value planes: [token][D/16 words]
     for (int w = 0; w < D / 16; ++w) {
       uint32_t hi = 0, lo = 0;
       for (int j = 0; j < 16; ++j) {
-        const uint32_t q = u->vq[static_cast<size_t>(t) * D + 16 * w + j];
+        const uint32_t q = uvq[static_cast<size_t>(t) * D + 16 * w + j];
         const uint32_t plane_hi = q4 ? (q >> 2) : q;
         hi |= (plane_hi & 3u) << (2 * j);
         lo |= (q & 3u) << (2 * j);
@@ -308,9 +436,18 @@ int orc_unit_serialize(const void* p, uint8_t* out, uint8_t* valid, size_t bytes
     // value meta: (scale_j, zero_j) pairs
     for (int j = 0; j < D / kG; ++j) {
       const size_t off = static_cast<size_t>(t) * (D / 4) + j * 8;
-      put_bytes(out, valid, L.v_meta + off, &u->vs[t * (D / kG) + j], 4);
-      put_bytes(out, valid, L.v_meta + off + 4, &u->vz[t * (D / kG) + j], 4);
+      put_bytes(out, valid, L.v_meta + off, &uvs[t * (D / kG) + j], 4);
+      put_bytes(out, valid, L.v_meta + off + 4, &uvz[t * (D / kG) + j], 4);
     }
+  }
+  if (res2) {
+    // bf16 window: position t in slot t mod 64 (R10)
+    for (int t = u->qtok(); t < u->n; ++t) {
+      const size_t slot = static_cast<size_t>(t % kResWindow) * D * 2;
+      put_bytes(out, valid, L.res_k + slot, &u->bk[static_cast<size_t>(t) * D], D * 2);
+      put_bytes(out, valid, L.res_v + slot, &u->bv[static_cast<size_t>(t) * D], D * 2);
+    }
+    return 0;
   }
   for (int r = 0; r < u->residual(); ++r) {
     put_bytes(out, valid, L.res_k + static_cast<size_t>(r) * D * 2, &u->rk[r * D], D * 2);
@@ -346,6 +483,14 @@ int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, in
   const Unit* data = own;
   int n_att = own->n;
   const bool share = own->kind == KIND_SHARE;
+  const bool res2 = own->kind == KIND_RES2;
+  ResState rs;
+  if (res2) {
+    // the reference's reading plus the residual below qtok (R11)
+    if (!reference_ok(*own, src)) return -1;
+    rs = residual_state(*own, *src);
+    data = src;
+  }
   if (share) {
     if (src == nullptr || src->kind == KIND_SHARE || src->D != D) return -1;
     data = src;
@@ -359,12 +504,17 @@ int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, in
   for (int i = 0; i < g * D; ++i) qd[i] = static_cast<double>(bf16_to_float(q[i]));
 
   const bool quant = data->kind == KIND_Q4 || data->kind == KIND_Q2;
-  const int qtok = quant ? data->qtok() : 0;
+  // quantized positions of the data cell; for RES2 those that carry a residual
+  const int qtok = res2 ? rs.qtok : (quant ? data->qtok() : 0);
   const int npos = n_att + (share ? 1 : 0);
 
   // dequantized key of a position (fp64)
   std::vector<double> khat(D);
   auto key_of = [&](int pos) {
+    if (res2 && pos >= qtok) {
+      for (int d = 0; d < D; ++d) khat[d] = bf16_to_float(own->bk[static_cast<size_t>(pos) * D + d]);
+      return;
+    }
     if (share && pos == n_att) {
       for (int d = 0; d < D; ++d) khat[d] = bf16_to_float(own->ck[d]);
     } else if (data->kind == KIND_BF16) {
@@ -378,6 +528,12 @@ int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, in
     } else {
       const int r = pos - qtok;
       for (int d = 0; d < D; ++d) khat[d] = bf16_to_float(data->rk[static_cast<size_t>(r) * D + d]);
+    }
+    if (res2) {
+      const int gr = pos / kG;
+      for (int d = 0; d < D; ++d)
+        khat[d] += static_cast<double>(rs.ks[gr * D + d]) * rs.kq[static_cast<size_t>(pos) * D + d] +
+                   static_cast<double>(rs.kz[gr * D + d]);
     }
   };
 
@@ -430,7 +586,9 @@ int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, in
     for (int d = 0; d < D; ++d) {
       double v;
       double dev = 0.0;  // |lo - 1.5| * scale: the most the selection moves v
-      if (share && pos == n_att) {
+      if (res2 && pos >= qtok) {
+        v = bf16_to_float(own->bv[static_cast<size_t>(pos) * D + d]);
+      } else if (share && pos == n_att) {
         v = bf16_to_float(own->cv[d]);
       } else if (data->kind == KIND_BF16) {
         v = bf16_to_float(data->bv[static_cast<size_t>(pos) * D + d]);
@@ -449,6 +607,11 @@ int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, in
         }
       } else {
         v = bf16_to_float(data->rv[static_cast<size_t>(pos - qtok) * D + d]);
+      }
+      if (res2 && pos < qtok) {
+        const size_t j = static_cast<size_t>(pos) * (D / kG) + d / kG;
+        v += static_cast<double>(rs.vs[j]) * rs.vq[static_cast<size_t>(pos) * D + d] +
+             static_cast<double>(rs.vz[j]);
       }
       for (int h = 0; h < g; ++h) {
         const double ph = p[static_cast<size_t>(h) * npos + pos];

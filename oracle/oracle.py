@@ -12,7 +12,7 @@ import numpy as np
 
 from . import build as _build
 
-KIND_Q4, KIND_Q2, KIND_SHARE, KIND_BF16 = 0, 1, 2, 3
+KIND_Q4, KIND_Q2, KIND_SHARE, KIND_BF16, KIND_RES2 = 0, 1, 2, 3, 4
 G = 32
 
 _lib = None
@@ -34,11 +34,11 @@ def _load():
     lib.orc_unit_len.restype = ctypes.c_int
     lib.orc_unit_append.argtypes = [P, P, P, ctypes.c_int]
     lib.orc_unit_append.restype = ctypes.c_int
-    lib.orc_unit_export.argtypes = [P, P, P, P, P, P, P]
+    lib.orc_unit_export.argtypes = [P, P, P, P, P, P, P, P]
     lib.orc_unit_export.restype = ctypes.c_int
     lib.orc_region_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.orc_region_bytes.restype = ctypes.c_size_t
-    lib.orc_unit_serialize.argtypes = [P, P, P, ctypes.c_size_t]
+    lib.orc_unit_serialize.argtypes = [P, P, P, P, ctypes.c_size_t]
     lib.orc_unit_serialize.restype = ctypes.c_int
     lib.orc_decode.argtypes = [P, P, P, ctypes.c_double, ctypes.c_double,
                                ctypes.c_double, P, P, P, P, P, P, P]
@@ -104,9 +104,16 @@ class OracleUnit:
         if rc != 0:
             raise ValueError("oracle append rejected (capacity)")
 
-    def export(self):
-        """Quantized state: dict of key/value codes, scales and zero points."""
-        qtok = self._lib.orc_unit_export(self._h, None, None, None, None, None, None)
+    def export(self, src=None):
+        """Quantized state: dict of key/value codes, scales and zero points.
+
+        ``src``: the reference unit of a residual (RES2) unit, whose codes are
+        its residual codes against that reference.
+        """
+        sh = None if src is None else src._h
+        qtok = self._lib.orc_unit_export(self._h, sh, None, None, None, None, None, None)
+        if qtok < 0:
+            raise ValueError("residual unit without a reference holding its positions")
         D = self.D
         kq = np.zeros((qtok, D), np.uint8)
         ks = np.zeros((qtok // G, D), np.float32)
@@ -114,17 +121,20 @@ class OracleUnit:
         vq = np.zeros((qtok, D), np.uint8)
         vs = np.zeros((qtok, D // G), np.float32)
         vz = np.zeros((qtok, D // G), np.float32)
-        self._lib.orc_unit_export(self._h, _ptr(kq), _ptr(ks), _ptr(kz), _ptr(vq),
-                             _ptr(vs), _ptr(vz))
+        self._lib.orc_unit_export(self._h, sh, _ptr(kq), _ptr(ks), _ptr(kz), _ptr(vq),
+                                  _ptr(vs), _ptr(vz))
         return dict(qtok=qtok, kq=kq, ks=ks, kz=kz, vq=vq, vs=vs, vz=vz)
 
-    def serialize(self):
-        """(bytes u8[R], valid u8[R]) of the unit in the canonical layout."""
+    def serialize(self, src=None):
+        """(bytes u8[R], valid u8[R]) of the unit in the canonical layout
+        (``src``: a residual unit's reference)."""
         nbytes = region_bytes(self.kind, self.D, self.cap)
         out = np.zeros(nbytes, np.uint8)
         valid = np.zeros(nbytes, np.uint8)
-        rc = self._lib.orc_unit_serialize(self._h, _ptr(out), _ptr(valid), nbytes)
-        assert rc == 0
+        rc = self._lib.orc_unit_serialize(self._h, None if src is None else src._h, _ptr(out),
+                                          _ptr(valid), nbytes)
+        if rc != 0:
+            raise ValueError("oracle serialize rejected its input")
         return out, valid
 
 
@@ -142,7 +152,7 @@ def decode(unit, q_bits, tau, src=None, sm_scale=0.0, band=1e-6):
     """Decode one unit for the query ``q_bits`` (bf16 bits [D]).
 
     ``src`` is the final loop's unit of the same layer, sequence and head when
-    ``unit`` is a SHARE unit.
+    ``unit`` is a SHARE unit or a residual (RES2) unit.
     """
     D = unit.D
     q = np.ascontiguousarray(q_bits, dtype=np.uint16).reshape(D)

@@ -459,6 +459,156 @@ def pin_mask_properties():
     assert (r2.mask[0] >> 5) & 1 == 1
 
 
+# --------------------------------------------------------- residual (RES2) pins
+# "ResidualQuant: KV Cache Quantization for Looped Transformers with 2-Bit
+# Residuals", section 概要: the final loop's KV is the reference and the
+# other loops store 2-bit residuals against it.
+
+def pin_residual_deferred_window():
+    # A residual group is quantized once the 32 tokens after it are in, so
+    # the bf16 window keeps 32..63 tokens (all of them below 32):
+    # qtok(n) = 32 * max(0, floor(n / 32) - 1).
+    D = 64
+    ref, _, _ = _unit(orc.KIND_BF16, D, 200, 300)
+    k = rng_bits(301, (200, D))
+    v = rng_bits(302, (200, D))
+    a = orc.OracleUnit(orc.KIND_RES2, D, 256)
+    for t in range(200):
+        a.append(k[t:t + 1], v[t:t + 1])
+        n = t + 1
+        assert a.export(src=ref)["qtok"] == max(0, n // G - 1) * G, n
+    b = orc.OracleUnit(orc.KIND_RES2, D, 256)
+    b.append(k[:77], v[:77])
+    b.append(k[77:], v[77:])
+    oa, va = a.serialize(src=ref)
+    ob, vb = b.serialize(src=ref)
+    assert (oa == ob).all() and (va == vb).all()
+
+
+def pin_residual_worked_example():
+    # bf16 reference r = 1 everywhere; the cell's token t < 32 is r + (t mod 4)
+    # on every channel, so every residual is t mod 4: key channels span [0, 3]
+    # over a group (scale 1, zero 0, codes t mod 4), each value group of
+    # token t is constant (scale 0, zero t mod 4, codes 0).  Layout as a
+    # 2-bit cell plus a 64-slot bf16 window (position t in slot t mod 64).
+    D = 64
+    n = 70
+    ones = np.ones((n, D), np.float32)
+    ref = orc.OracleUnit(orc.KIND_BF16, D, 128)
+    ref.append(bf16(ones), bf16(ones))
+    x = 1.0 + (np.arange(n) % 4)[:, None] * np.ones((1, D), np.float32)
+    x[32:] = np.arange(32, n)[:, None]  # window tokens: distinct rows
+    u = orc.OracleUnit(orc.KIND_RES2, D, 128)
+    u.append(bf16(x), bf16(x))
+    st = u.export(src=ref)
+    assert st["qtok"] == 32
+    assert (st["ks"] == 1.0).all() and (st["kz"] == 0.0).all()
+    assert (st["kq"] == (np.arange(32) % 4)[:, None]).all()
+    assert (st["vs"] == 0.0).all() and (st["vq"] == 0).all()
+    assert (st["vz"][:, 0] == np.arange(32) % 4).all()
+    out, valid = u.serialize(src=ref)
+    words = out.view(np.uint32)
+    kblock = (128 // G) * 8 * D
+    vblock = (128 // G) * G * (D // 4)
+    # key plane, group 0, chunk 0: token t's word 0 is (t mod 4) * 0x55555555
+    for t in range(4):
+        assert words[t * 4] == (t % 4) * 0x55555555, (t, hex(words[t * 4]))
+    # window: K rows after k_hi, k_meta, v_hi, v_meta; position 64 -> slot 0,
+    # position 33 -> slot 33
+    res_k = 2 * kblock + 2 * vblock
+    row = out[res_k: res_k + 2 * D].view(np.uint16)
+    assert (row == bf16(x[64])).all()
+    row = out[res_k + 33 * 2 * D: res_k + 34 * 2 * D].view(np.uint16)
+    assert (row == bf16(x[33])).all()
+    # defined bytes: one group of K (plane + meta), 32 V rows (plane + meta),
+    # 38 window tokens of K and V
+    assert valid.sum() == 2 * 8 * D + 2 * G * (D // 4) + 2 * 38 * 2 * D
+    # the zero residual of an identical cell reads back the reference exactly
+    same = orc.OracleUnit(orc.KIND_RES2, D, 128)
+    same.append(bf16(ones), bf16(ones))
+    z = same.export(src=ref)
+    assert (z["ks"] == 0).all() and (z["kz"] == 0).all() and (z["vz"] == 0).all()
+
+
+def _ref32(st, pos, keys):
+    """The reference's stored value in fp32: fl(fl(scale * code) + zero)."""
+    g = pos // G
+    if keys:
+        return (st["ks"][g] * st["kq"][pos].astype(np.float32)) + st["kz"][g]
+    s = np.repeat(st["vs"][pos], G)
+    z = np.repeat(st["vz"][pos], G)
+    return (s * st["vq"][pos].astype(np.float32)) + z
+
+
+def pin_residual_reconstructs():
+    # Against a 4-bit reference: (a) every quantized position reconstructs
+    # its own input within half a residual step, (b) decode is textbook
+    # attention over r^ + d^ (reference keys at stored precision, reference
+    # values through the tau rule) and the cell's own bf16 window tokens.
+    D = 64
+    n = 3 * G + 13
+    ref, _, _ = _unit(orc.KIND_Q4, D, n + 5, 310)
+    k = rng_bits(311, (n, D), 1.0)
+    v = rng_bits(312, (n, D))
+    u = orc.OracleUnit(orc.KIND_RES2, D, 160)
+    u.append(k, v)
+    rs = ref.export()
+    st = u.export(src=ref)
+    qtok = st["qtok"]
+    assert qtok == 2 * G
+    kx = f32(k).astype(np.float32)
+    vx = f32(v).astype(np.float32)
+    for pos in range(qtok):
+        g = pos // G
+        kr = _ref32(rs, pos, True).astype(np.float64)
+        kh = kr + st["ks"][g].astype(np.float64) * st["kq"][pos] + st["kz"][g]
+        assert (np.abs(kx[pos] - kh) <= st["ks"][g] * 0.5000005 + 1e-6).all(), pos
+        vr = _ref32(rs, pos, False).astype(np.float64)
+        vs = np.repeat(st["vs"][pos], G).astype(np.float64)
+        vh = vr + vs * st["vq"][pos] + np.repeat(st["vz"][pos], G)
+        assert (np.abs(vx[pos] - vh) <= vs * 0.5000005 + 1e-6).all(), pos
+    gi = np.arange(qtok) // G
+    kref = rs["ks"][gi].astype(np.float64) * rs["kq"][:qtok] + rs["kz"][gi]
+    kres = st["ks"][gi].astype(np.float64) * st["kq"] + st["kz"][gi]
+    keys = np.concatenate([kref + kres, kx[qtok:].astype(np.float64)])
+    vs = np.repeat(st["vs"].astype(np.float64), G, axis=1)
+    vres = vs * st["vq"] + np.repeat(st["vz"].astype(np.float64), G, axis=1)
+    rvs = np.repeat(rs["vs"][:qtok].astype(np.float64), G, axis=1)
+    rvz = np.repeat(rs["vz"][:qtok].astype(np.float64), G, axis=1)
+    q = rng_bits(313, (D,), 2.0)
+    for tau, mode in ((0.0, "full"), (1.5, "hi")):
+        c = rs["vq"][:qtok].astype(np.float64)
+        if mode == "hi":
+            c = 4.0 * (rs["vq"][:qtok] >> 2) + 1.5
+        vals = np.concatenate([rvs * c + rvz + vres, vx[qtok:].astype(np.float64)])
+        r = orc.decode(u, q, tau=tau, src=ref)
+        want = sdpa(f32(q), keys, vals, 1 / np.sqrt(D))
+        assert np.abs(r.out - want).max() < 1e-12, (tau, np.abs(r.out - want).max())
+        assert r.nsel == (qtok if tau == 0.0 else 0)
+
+
+def pin_residual_reference_checks():
+    # No reference, a reference that does not yet hold the quantized
+    # positions, and a SHARE reference are all rejected.
+    D = 64
+    u = orc.OracleUnit(orc.KIND_RES2, D, 128)
+    u.append(rng_bits(320, (70, D)), rng_bits(321, (70, D)))
+    q = rng_bits(322, (D,))
+    short, _, _ = _unit(orc.KIND_Q4, D, 40, 323)   # holds one group; u needs 32 quantized
+    ok, _, _ = _unit(orc.KIND_Q4, D, 64, 324)
+    sh = orc.OracleUnit(orc.KIND_SHARE, D, 0)
+    sh.append(rng_bits(325, (3, D)), rng_bits(326, (3, D)))
+    orc.decode(u, q, tau=0.01, src=ok)
+    orc.decode(u, q, tau=0.01, src=short)   # 32 quantized reference positions suffice
+    tiny, _, _ = _unit(orc.KIND_Q4, D, 31, 327)
+    for bad in (None, tiny, sh):
+        try:
+            orc.decode(u, q, tau=0.01, src=bad)
+        except ValueError:
+            continue
+        raise AssertionError("residual unit accepted a bad reference")
+
+
 ALL_PINS = [
     pin_quantize_q2_ties,
     pin_quantize_q4_ties,
@@ -477,4 +627,8 @@ ALL_PINS = [
     pin_mask_properties,
     pin_group_query_heads,
     pin_planner_worked_example,
+    pin_residual_deferred_window,
+    pin_residual_worked_example,
+    pin_residual_reconstructs,
+    pin_residual_reference_checks,
 ]

@@ -48,6 +48,22 @@ MUTANTS = [
     ("planner: SHARE reads nothing", "rd += fk == 0 ? 5000 + sel_milli : 4000;", "rd += 0;"),
     ("planner: damage tie-break dropped", "(rd == br && (dm < bd || (dm == bd && st < bs)))",
      "(rd == br && st < bs)"),
+    ("residual against the reference's high plane",
+     "const float q = static_cast<float>(ref.kq[static_cast<size_t>(pos) * D + d]);",
+     "const float q = static_cast<float>(ref.kq[static_cast<size_t>(pos) * D + d] & 12);"),
+    ("value residual against the reference's high plane",
+     "const float q = static_cast<float>(ref.vq[static_cast<size_t>(pos) * D + d]);",
+     "const float q = static_cast<float>(ref.vq[static_cast<size_t>(pos) * D + d] & 12);"),
+    ("residual window not deferred",
+     "if (kind == KIND_RES2) return n / kG >= 2 ? (n / kG - 1) * kG : 0;",
+     "if (kind == KIND_RES2) return n / kG * kG;"),
+    ("key residual codes dropped", "khat[d] += static_cast<double>(rs.ks[gr * D + d])",
+     "khat[d] += 0.0 * static_cast<double>(rs.ks[gr * D + d])"),
+    ("value residual codes dropped", "v += static_cast<double>(rs.vs[j])",
+     "v += 0.0 * static_cast<double>(rs.vs[j])"),
+    ("residual window slot not modulo 64",
+     "const size_t slot = static_cast<size_t>(t % kResWindow) * D * 2;",
+     "const size_t slot = static_cast<size_t>(t - u->qtok()) * D * 2;"),
 ]
 
 
