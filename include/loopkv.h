@@ -26,6 +26,24 @@
  *   - softmax scale 1/sqrt(head_dim) unless given; one query per KV head.
  * LOOPKV_BF16 (raw bf16 cells) exists for ablations and checks.
  *
+ * Residual cells.  "ResidualQuant: KV Cache Quantization for Looped
+ * Transformers with 2-Bit Residuals", section 概要 (abstract): the final
+ * loop's KV is a reference and the other loops keep low-precision residuals
+ * against it.  A LOOPKV_RES2 cell (non-final loops only) stores, for each
+ * position t, d = fl32(x - r) quantized like a LOOPKV_Q2 cell, where x is
+ * its own bf16 input and r the reference's stored value at t in fp32:
+ * fl32(fl32(scale * q) + zero) with the full code q of a 4-bit or 2-bit
+ * reference, the raw value of a bf16 one.  The reference is the final loop's
+ * cell of the same layer, sequence and head (LOOPKV_Q4, LOOPKV_Q2 or
+ * LOOPKV_BF16).  A residual group g is quantized when the cell reaches
+ * 32 (g + 2) tokens, so the reference, appended after it in a decode step,
+ * already holds the group; the cell keeps its other tokens, 32..63 of them
+ * once it has 32 (all of them before), in bf16.  Decode reads a quantized
+ * position as the reference's reading (keys at stored precision, values of
+ * a 4-bit reference through the tau rule with the cell's own weights) plus
+ * scale * code + zero of the residual, and a bf16 position as the cell's own
+ * token.
+ *
  * Terms.  cells = n_loops * n_layers, indexed loop-major (cell = loop *
  * n_layers + layer).  A unit is one (cell, sequence, head).  Tokens of a
  * unit are positions 0..n-1.
@@ -63,7 +81,9 @@
  *   res_K [32][D], res_V [32][D]            bf16 residual; slot r holds
  *                                           position 32*floor(n/32) + r
  * LOOPKV_Q2 has the same blocks without K_lo and V_lo; its "hi" planes hold
- * the 2-bit codes.  LOOPKV_SHARE holds cur_K[D], cur_V[D] (bf16, each block
+ * the 2-bit codes.  LOOPKV_RES2 has the LOOPKV_Q2 blocks holding residual
+ * codes, with res_K [64][D], res_V [64][D] instead: position t of its bf16
+ * window in slot t mod 64.  LOOPKV_SHARE holds cur_K[D], cur_V[D] (bf16, each block
  * rounded up to 128 bytes).  LOOPKV_BF16 holds K[C][D] then V[C][D] (bf16,
  * each rounded up to 128 bytes).
  */
@@ -91,7 +111,8 @@ typedef enum {
   LOOPKV_Q4 = 0,    /* 4-bit codes kept as hi and lo 2-bit planes */
   LOOPKV_Q2 = 1,    /* 2-bit codes */
   LOOPKV_SHARE = 2, /* reuse the final loop's KV; keeps its current token */
-  LOOPKV_BF16 = 3   /* raw bf16 (ablation / checks) */
+  LOOPKV_BF16 = 3,  /* raw bf16 (ablation / checks) */
+  LOOPKV_RES2 = 4   /* 2-bit residuals against the final loop's KV */
 } loopkv_kind;
 
 /* Largest number of cells one loopkv_append / loopkv_decode call may name. */
@@ -108,8 +129,8 @@ typedef struct {
   const int32_t* capacity;/* host [max_batch]: tokens each unit of sequence b
                              can hold, 0 .. 2^20 */
   const uint8_t* kinds;   /* host [n_loops * n_layers], loop-major,
-                             loopkv_kind values; LOOPKV_SHARE only in loops
-                             < n_loops - 1 */
+                             loopkv_kind values; LOOPKV_SHARE and
+                             LOOPKV_RES2 only in loops < n_loops - 1 */
   float tau;              /* low-plane threshold on the softmax weight, >= 0 */
   float sm_scale;         /* softmax scale; <= 0 means 1/sqrt(head_dim) */
   int32_t q_per_kv;       /* query heads per KV head (grouped-query
@@ -152,9 +173,14 @@ void loopkv_plan_free(loopkv_plan* plan);
  * tokens they are quantized as one group (keys per channel, values per token
  * per 32 channels) into the planes.  SHARE cells keep only the last appended
  * token as their current key and value.  BF16 cells store tokens raw.
- * Lengths grow by h_n_new[b].  h_cells: distinct cell indices; h_n_new: host
- * [batch], each 0 .. n_new_max.
- * Errors (nothing launched): LOOPKV_ERR_INVALID_ARG, LOOPKV_ERR_CAPACITY
+ * RES2 cells keep tokens in their bf16 window and quantize residual group g
+ * once they hold 32 (g + 2) tokens, reading the reference's group g; the
+ * reference must hold that group before the call (its length before the
+ * call is what counts, so a call may append a RES2 cell and its reference
+ * together).  Lengths grow by h_n_new[b].  h_cells: distinct cell indices;
+ * h_n_new: host [batch], each 0 .. n_new_max.
+ * Errors (nothing launched): LOOPKV_ERR_INVALID_ARG (also: a RES2 append
+ * whose reference does not yet hold a group it needs), LOOPKV_ERR_CAPACITY
  * (len + n_new > capacity for a non-SHARE unit). */
 loopkv_status loopkv_append(loopkv_plan* plan, const int32_t* h_cells, int32_t n_cells,
                             int32_t batch, const int32_t* h_n_new, int32_t n_new_max,
@@ -166,7 +192,8 @@ loopkv_status loopkv_append(loopkv_plan* plan, const int32_t* h_cells, int32_t n
  *     d_q: bf16 [n_cells][batch][n_kv_heads][g][head_dim]
  * computes over the unit's attended positions (its own n tokens; for a SHARE
  * unit of length n, the final loop's stored positions [0, n-1) and its own
- * current token) the scores sm_scale * <q_r, k>, with keys dequantized at
+ * current token; for a RES2 unit its n tokens, the residual-coded ones read
+ * through the reference) the scores sm_scale * <q_r, k>, with keys dequantized at
  * their stored precision, each query's softmax p_r, the selection of the
  * 4-bit quantized positions where some query of the group has p_r >= tau
  * (one query: p >= tau; the KV head's low plane is read once for the whole
@@ -180,8 +207,10 @@ loopkv_status loopkv_append(loopkv_plan* plan, const int32_t* h_cells, int32_t n
  *             0 .. ceil(nq/32)-1 are written, nq = 4-bit positions attended
  *     d_nsel: int32 [n_cells][batch][n_kv_heads], number of selected positions
  * Every unit must hold n >= 1 tokens; a SHARE unit needs its source to hold
- * at least n-1.  SHARE units read the source as it is stored when the kernel
+ * at least n-1; a RES2 unit needs its reference to hold its residual-coded
+ * positions.  SHARE units read the source as it is stored when the kernel
  * runs (decode a loop before appending to the final loop for serving order).
+ * RES2 cells run in a second launch on the same stream.
  * Errors (nothing launched): LOOPKV_ERR_INVALID_ARG, LOOPKV_ERR_UNSUPPORTED
  * (a unit longer than the kernel's limit). */
 loopkv_status loopkv_decode(loopkv_plan* plan, const int32_t* h_cells, int32_t n_cells,
@@ -194,8 +223,10 @@ loopkv_status loopkv_decode(loopkv_plan* plan, const int32_t* h_cells, int32_t n
  * keeps every stored position valid: new <= old and, for Q4/Q2 cells,
  * new >= 32*floor(old/32) (drop residual tokens only) or new a multiple of
  * 32 (drop whole groups); SHARE cells: new == old (only the current
- * token is kept, so a SHARE unit can only be reset).  For rollback and reuse
- * of sequence slots.  Errors: LOOPKV_ERR_INVALID_ARG. */
+ * token is kept, so a SHARE unit can only be reset); RES2 cells: new keeps
+ * the same residual-coded count 32 * max(0, floor(n/32) - 1) (drop window
+ * tokens only).  For rollback and reuse of sequence slots.
+ * Errors: LOOPKV_ERR_INVALID_ARG. */
 loopkv_status loopkv_set_lengths(loopkv_plan* plan, const int32_t* h_cells, int32_t n_cells,
                                  int32_t batch, const int32_t* h_len, void* stream);
 

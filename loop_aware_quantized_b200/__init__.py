@@ -7,7 +7,7 @@ imported on first use of a name below, and that import fails if the library
 has not been built: there is no other code path.
 """
 
-_EXPORTS = ("LOOPKV_BF16", "LOOPKV_Q2", "LOOPKV_Q4", "LOOPKV_SHARE", "LoopKVError", "Plan",
+_EXPORTS = ("LOOPKV_BF16", "LOOPKV_Q2", "LOOPKV_Q4", "LOOPKV_RES2", "LOOPKV_SHARE", "LoopKVError", "Plan",
             "plan_optimize", "query_sizes")
 
 

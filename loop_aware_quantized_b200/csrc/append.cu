@@ -80,7 +80,7 @@ append_kernel(const AppendParams p, const CellList cl) {
   }
   uint8_t* base = p.cache + s.offset + (size_t)h * s.stride;
   const UnitLayout L = unit_layout(kind, D, s.cap);
-  const size_t in_off = (((size_t)ci * p.batch + b) * H + h) * (size_t)p.n_new_max * D;
+  const size_t in_off = (((size_t)cl.out[ci] * p.batch + b) * H + h) * (size_t)p.n_new_max * D;
   const uint16_t* kin = p.k + in_off;
   const uint16_t* vin = p.v + in_off;
 
@@ -246,6 +246,188 @@ append_kernel(const AppendParams p, const CellList cl) {
   }
 }
 
+// The reference's stored key / value at (pos, d) dequantized in fp32, the
+// way a residual is taken against it: fl(fl(scale * q) + zero) with the full
+// code q of a 4-bit or 2-bit reference, the raw value of a bf16 one.
+__device__ float ref_key32(const uint8_t* rb, const UnitLayout& RL, int rkind, int pos, int d,
+                           int D) {
+  if (rkind == LOOPKV_BF16)
+    return bf16f(*reinterpret_cast<const uint16_t*>(rb + RL.raw_k + ((size_t)pos * D + d) * 2));
+  const int g = pos / kGroup, t = pos % kGroup, c = d / 64, w = (d % 64) / 16, j = d % 16;
+  const size_t off = (size_t)g * 8 * D + c * 512 + t * 16 + w * 4;
+  uint32_t q = (*reinterpret_cast<const uint32_t*>(rb + RL.k_hi + off) >> (2 * j)) & 3u;
+  if (rkind == LOOPKV_Q4)
+    q = 4u * q + ((*reinterpret_cast<const uint32_t*>(rb + RL.k_lo + off) >> (2 * j)) & 3u);
+  const float* meta = reinterpret_cast<const float*>(rb + RL.k_meta + (size_t)g * 8 * D);
+  return __fadd_rn(__fmul_rn(meta[d], (float)q), meta[D + d]);
+}
+
+__device__ float ref_value32(const uint8_t* rb, const UnitLayout& RL, int rkind, int pos, int d,
+                             int D) {
+  if (rkind == LOOPKV_BF16)
+    return bf16f(*reinterpret_cast<const uint16_t*>(rb + RL.raw_v + ((size_t)pos * D + d) * 2));
+  const size_t row = (size_t)pos * (D / 4);
+  const int w = d / 16, j = d % 16;
+  uint32_t q = (*reinterpret_cast<const uint32_t*>(rb + RL.v_hi + row + w * 4) >> (2 * j)) & 3u;
+  if (rkind == LOOPKV_Q4)
+    q = 4u * q + ((*reinterpret_cast<const uint32_t*>(rb + RL.v_lo + row + w * 4) >> (2 * j)) & 3u);
+  const float* m = reinterpret_cast<const float*>(rb + RL.v_meta + row + (d / kGroup) * 8);
+  return __fadd_rn(__fmul_rn(m[0], (float)q), m[1]);
+}
+
+// Append to RES2 units ("ResidualQuant: KV Cache Quantization for Looped
+// Transformers with 2-Bit Residuals", section 概要: 2-bit residuals against
+// the final loop's KV).  One CTA per unit.  Tokens live in a 64-slot bf16
+// window (position t in slot t mod 64); residual group g is quantized when
+// the unit reaches 32 (g + 2) tokens: each warp takes a group, forms the
+// residuals x - r in an fp32 tile (r: the reference's stored value, read
+// from its planes) and quantizes them at 2 bits exactly as a Q2 cell's
+// tokens (keys per channel, values per token per 32 channels).  Window
+// slots are written after every group has read them.
+template <int D>
+__global__ void __launch_bounds__(kAppendThreads)
+append_res2_kernel(const AppendParams p, const CellList cl) {
+  constexpr int XROW = D + 1;     // fp32 per padded tile row
+  constexpr int CROW = D + 16;    // bytes per padded code row
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* xk = reinterpret_cast<float*>(sm) + warp * (2 * 32 * XROW);
+  float* xv = xk + 32 * XROW;
+  uint8_t* codes = sm + (size_t)kAppendWarps * (2 * 32 * XROW) * 4 + warp * (32 * CROW);
+
+  const int H = p.n_heads;
+  const int h = blockIdx.x % H;
+  const int b = (blockIdx.x / H) % p.batch;
+  const int ci = blockIdx.x / (H * p.batch);
+  const int cell = cl.cell[ci];
+  const int n_new = p.n_new[b];
+  if (n_new <= 0) return;
+
+  const TableHeader* hdr = reinterpret_cast<const TableHeader*>(p.table);
+  const DevCell* cells = reinterpret_cast<const DevCell*>(p.table + table_cells_offset());
+  const DevSeq* seqs = reinterpret_cast<const DevSeq*>(p.table + table_seqs_offset(hdr->n_cells));
+  const DevCell c = cells[cell];
+  const DevSeq s = seqs[(size_t)cell * hdr->max_batch + b];
+  const DevCell rc = cells[c.src];
+  const DevSeq rs = seqs[(size_t)c.src * hdr->max_batch + b];
+  const int rkind = rc.kind;
+  const int n_old = s.len;
+  const int n1 = n_old + n_new;
+  const int q0 = res2_qtok(n_old), q1 = res2_qtok(n1);
+  const int ref_pos = rkind == LOOPKV_BF16 ? rs.len : rs.len / kGroup * kGroup;
+  const bool ref_ok = rkind == LOOPKV_Q4 || rkind == LOOPKV_Q2 || rkind == LOOPKV_BF16;
+  if (c.kind != LOOPKV_RES2 || !ref_ok || n_old < 0 || n1 > s.cap || q1 > ref_pos) {
+    // host checks make this unreachable; flag it and leave the unit alone
+    if (threadIdx.x == 0) atomicOr(reinterpret_cast<uint32_t*>(p.table), kStatusLength);
+    return;
+  }
+  uint8_t* base = p.cache + s.offset + (size_t)h * s.stride;
+  const uint8_t* rbase = p.cache + rs.offset + (size_t)h * rs.stride;
+  const UnitLayout L = unit_layout(LOOPKV_RES2, D, s.cap);
+  const UnitLayout RL = unit_layout(rkind, D, rs.cap);
+  const size_t in_off = (((size_t)cl.out[ci] * p.batch + b) * H + h) * (size_t)p.n_new_max * D;
+  const uint16_t* kin = p.k + in_off;
+  const uint16_t* vin = p.v + in_off;
+  const uint16_t* wk = reinterpret_cast<const uint16_t*>(base + L.res_k);
+  const uint16_t* wv = reinterpret_cast<const uint16_t*>(base + L.res_v);
+
+  for (int g = q0 / kGroup + warp; g < q1 / kGroup; g += kAppendWarps) {
+    // residuals of the group's 32 tokens (window slots or new tokens)
+    for (int i = lane; i < 32 * D; i += 32) {
+      const int t = i / D, d = i % D;
+      const int pos = g * kGroup + t;
+      const uint16_t kx = pos < n_old ? wk[(size_t)(pos % kResWindow) * D + d]
+                                      : kin[(size_t)(pos - n_old) * D + d];
+      const uint16_t vx = pos < n_old ? wv[(size_t)(pos % kResWindow) * D + d]
+                                      : vin[(size_t)(pos - n_old) * D + d];
+      xk[t * XROW + d] = __fsub_rn(bf16f(kx), ref_key32(rbase, RL, rkind, pos, d, D));
+      xv[t * XROW + d] = __fsub_rn(bf16f(vx), ref_value32(rbase, RL, rkind, pos, d, D));
+    }
+    __syncwarp();
+
+    // keys: per channel over the 32 tokens
+    float* kmeta = reinterpret_cast<float*>(base + L.k_meta + (size_t)g * 8 * D);
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const int d = lane + 32 * i;
+      float mn = xk[d], mx = mn;
+      for (int t = 1; t < 32; ++t) {
+        mn = fminf(mn, xk[t * XROW + d]);
+        mx = fmaxf(mx, xk[t * XROW + d]);
+      }
+      const float sc = group_scale(mn, mx, 3);
+      for (int t = 0; t < 32; ++t) codes[t * CROW + d] = (uint8_t)quant_code(xk[t * XROW + d], mn, sc, 3);
+      kmeta[d] = sc;
+      kmeta[D + d] = canon_zero(mn);
+    }
+    __syncwarp();
+    // pack: lane = token; chunk c of 64 channels -> 4 words
+#pragma unroll
+    for (int cc = 0; cc < D / 64; ++cc) {
+      uint32_t hiw[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t hv = 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) hv |= ((uint32_t)codes[lane * CROW + 64 * cc + 16 * w + j] & 3u) << (2 * j);
+        hiw[w] = hv;
+      }
+      const size_t off = (size_t)g * 8 * D + cc * 512 + lane * 16;
+      *reinterpret_cast<uint4*>(base + L.k_hi + off) = make_uint4(hiw[0], hiw[1], hiw[2], hiw[3]);
+    }
+
+    // values: lane = token, per group of 32 channels
+    {
+      const int t = lane;
+      const size_t tpos = (size_t)g * kGroup + t;
+      const float* row = xv + t * XROW;
+      uint32_t hiw[D / 16];
+      float meta[D / 16];
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        float mn = row[32 * j], mx = mn;
+        for (int e = 1; e < 32; ++e) {
+          mn = fminf(mn, row[32 * j + e]);
+          mx = fmaxf(mx, row[32 * j + e]);
+        }
+        const float sc = group_scale(mn, mx, 3);
+        uint32_t w0 = 0, w1 = 0;
+        for (int e = 0; e < 16; ++e) {
+          w0 |= quant_code(row[32 * j + e], mn, sc, 3) << (2 * e);
+          w1 |= quant_code(row[32 * j + 16 + e], mn, sc, 3) << (2 * e);
+        }
+        hiw[2 * j] = w0;
+        hiw[2 * j + 1] = w1;
+        meta[2 * j] = sc;
+        meta[2 * j + 1] = canon_zero(mn);
+      }
+      uint4* vh = reinterpret_cast<uint4*>(base + L.v_hi + tpos * (D / 4));
+      float4* vm = reinterpret_cast<float4*>(base + L.v_meta + tpos * (D / 4));
+#pragma unroll
+      for (int i = 0; i < D / 64; ++i) {
+        vh[i] = make_uint4(hiw[4 * i], hiw[4 * i + 1], hiw[4 * i + 2], hiw[4 * i + 3]);
+        vm[i] = make_float4(meta[4 * i], meta[4 * i + 1], meta[4 * i + 2], meta[4 * i + 3]);
+      }
+    }
+    __syncwarp();
+  }
+  __syncthreads();  // every group has read its window slots
+
+  // new tokens past the residual-coded range go to their window slots
+  const int first = n_old > q1 ? n_old : q1;
+  uint8_t* rk = base + L.res_k;
+  uint8_t* rv = base + L.res_v;
+  for (int i = threadIdx.x; i < (n1 - first) * (D / 8); i += kAppendThreads) {
+    const int t = i / (D / 8), cc = i % (D / 8);
+    const int pos = first + t;
+    const size_t slot = (size_t)(pos % kResWindow) * D * 2;
+    reinterpret_cast<uint4*>(rk + slot)[cc] =
+        reinterpret_cast<const uint4*>(kin + (size_t)(pos - n_old) * D)[cc];
+    reinterpret_cast<uint4*>(rv + slot)[cc] =
+        reinterpret_cast<const uint4*>(vin + (size_t)(pos - n_old) * D)[cc];
+  }
+}
+
 __global__ void commit_lengths_kernel(uint8_t* table, const CellList cl, int n_cells, int batch,
                                       const AppendParams p) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -260,24 +442,29 @@ template <int D>
 size_t append_smem() {
   return (size_t)kAppendWarps * (2 * 32 * (D + 2) * 2 + 32 * (D + 16));
 }
+template <int D>
+size_t append_res2_smem() {
+  return (size_t)kAppendWarps * (2 * 32 * (D + 1) * 4 + 32 * (D + 16));
+}
 
 template <int D>
-int launch_append_t(const AppendParams& p, const CellList& cells, cudaStream_t stream) {
-  const size_t smem = append_smem<D>();
-  cudaError_t e = cudaFuncSetAttribute(append_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+int launch_append_t(const AppendParams& p, const CellList& cells, cudaStream_t stream, bool res2) {
+  const size_t smem = res2 ? append_res2_smem<D>() : append_smem<D>();
+  auto kern = res2 ? append_res2_kernel<D> : append_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_cells * p.batch * p.n_heads;
-  append_kernel<D><<<(unsigned)units, kAppendThreads, smem, stream>>>(p, cells);
+  kern<<<(unsigned)units, kAppendThreads, smem, stream>>>(p, cells);
   return (int)cudaGetLastError();
 }
 
 }  // namespace
 
-int launch_append(const AppendParams& p, const CellList& cells, void* stream, int head_dim) {
+int launch_append(const AppendParams& p, const CellList& cells, void* stream, int head_dim,
+                  bool res2) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (head_dim == 64) return launch_append_t<64>(p, cells, s);
-  return launch_append_t<128>(p, cells, s);
+  if (head_dim == 64) return launch_append_t<64>(p, cells, s, res2);
+  return launch_append_t<128>(p, cells, s, res2);
 }
 
 int launch_commit_lengths(uint8_t* table, const CellList& cells, int n_cells, int batch,

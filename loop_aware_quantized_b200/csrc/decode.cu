@@ -166,10 +166,14 @@ struct Unit {
   int nq;               // leading quantized positions among them
   int qtok;             // quantized tokens stored in the data unit
   int npos;             // n_att + has_cur
+  int rtok;             // RES2: positions that carry a residual (read through data)
   bool has_cur;
   bool ok;
 };
 
+// RES2: the unit's own region holds residual codes and its bf16 window,
+// data is its reference (the final loop's cell of the layer).
+template <bool RES2>
 __device__ Unit resolve(const DecodeParams& p, int cell, int b, int h, int D) {
   Unit u{};
   const TableHeader* hdr = reinterpret_cast<const TableHeader*>(p.table);
@@ -178,6 +182,27 @@ __device__ Unit resolve(const DecodeParams& p, int cell, int b, int h, int D) {
   const int B = hdr->max_batch;
   const DevCell oc = cells[cell];
   const DevSeq os = seqs[(size_t)cell * B + b];
+  if constexpr (RES2) {
+    const DevCell dc = cells[oc.src];
+    const DevSeq ds = seqs[(size_t)oc.src * B + b];
+    u.own_kind = oc.kind;
+    u.own = p.cache + os.offset + (size_t)h * os.stride;
+    u.Lo = unit_layout(LOOPKV_RES2, D, os.cap);
+    u.data_kind = dc.kind;
+    u.data = p.cache + ds.offset + (size_t)h * ds.stride;
+    u.Ld = unit_layout(dc.kind, D, ds.cap);
+    u.n_att = os.len;
+    u.has_cur = false;
+    u.rtok = res2_qtok(os.len);
+    const bool quant = dc.kind == LOOPKV_Q4 || dc.kind == LOOPKV_Q2;
+    const int ref_pos = quant ? ds.len / kGroup * kGroup : ds.len;
+    u.ok = oc.kind == LOOPKV_RES2 && os.len >= 1 && os.len <= os.cap && ds.len <= ds.cap &&
+           (quant || dc.kind == LOOPKV_BF16) && u.rtok <= ref_pos;
+    u.qtok = quant ? u.rtok : 0;
+    u.nq = u.qtok;
+    u.npos = u.n_att;
+    return u;
+  }
   u.own_kind = oc.kind;
   u.own = p.cache + os.offset + (size_t)h * os.stride;
   u.Lo = unit_layout(oc.kind, D, os.cap);
@@ -205,8 +230,14 @@ __device__ Unit resolve(const DecodeParams& p, int cell, int b, int h, int D) {
   return u;
 }
 
-// Pointer to the bf16 key (or value) row of a raw position.
+// Pointer to the bf16 key (or value) row of a raw position (RES2: positions
+// past the residual-coded ones are in the unit's own window, slot pos mod 64).
+template <bool RES2>
 __device__ __forceinline__ const uint8_t* raw_row(const Unit& u, int pos, int D, bool value) {
+  if constexpr (RES2) {
+    if (pos >= u.rtok)
+      return u.own + (value ? u.Lo.res_v : u.Lo.res_k) + (size_t)(pos % kResWindow) * D * 2;
+  }
   if (u.has_cur && pos == u.n_att) return u.own + (value ? u.Lo.cur_v : u.Lo.cur_k);
   if (u.data_kind == LOOPKV_BF16)
     return u.data + (value ? u.Ld.raw_v : u.Ld.raw_k) + (size_t)pos * D * 2;
@@ -379,7 +410,9 @@ __device__ __forceinline__ void prefetch_kgroup(const uint8_t* kh, size_t lo_off
 // Two register buffers alternate, so the next group's loads are in flight
 // while the current one is scored, without copies between them.  Scores of
 // query r go to sc[r * S + pos - p0]; lmax[r] is raised to their maximum.
-template <int D, bool Q4, int G>
+// ADD: the scores are added to what sc holds (a RES2 unit's residual keys
+// on top of its reference's); lmax is then left alone.
+template <int D, bool Q4, int G, bool ADD = false>
 __device__ __forceinline__ void key_pass(const Unit& u, int b_begin, int b_end, int p0, int p1,
                                          const float* q_s, float* qs, float* sc, int S,
                                          float sscale, int warp, int lane, float (&lmax)[G]) {
@@ -415,8 +448,12 @@ __device__ __forceinline__ void key_pass(const Unit& u, int b_begin, int b_end, 
     if (bk * 32 + lane < qlim) {
 #pragma unroll
       for (int r = 0; r < G; ++r) {
-        sc[r * S + bk * 32 + lane - p0] = s[r];
-        lmax[r] = fmaxf(lmax[r], s[r]);
+        if (ADD) {
+          sc[r * S + bk * 32 + lane - p0] += s[r];
+        } else {
+          sc[r * S + bk * 32 + lane - p0] = s[r];
+          lmax[r] = fmaxf(lmax[r], s[r]);
+        }
       }
     }
     if (!hasb) break;
@@ -431,8 +468,12 @@ __device__ __forceinline__ void key_pass(const Unit& u, int b_begin, int b_end, 
     if (bk * 32 + lane < qlim) {
 #pragma unroll
       for (int r = 0; r < G; ++r) {
-        sc[r * S + bk * 32 + lane - p0] = s[r];
-        lmax[r] = fmaxf(lmax[r], s[r]);
+        if (ADD) {
+          sc[r * S + bk * 32 + lane - p0] += s[r];
+        } else {
+          sc[r * S + bk * 32 + lane - p0] = s[r];
+          lmax[r] = fmaxf(lmax[r], s[r]);
+        }
       }
     }
     if (!hasa) break;
@@ -625,7 +666,7 @@ __device__ __forceinline__ void low_planes(float2 (&acc)[G][32 / G], const Unit&
 // KV head.  DENSE_LO: tau <= 0, every 4-bit token takes its low plane (read
 // densely in the value loop); otherwise low planes come from the
 // selected-position list.
-template <int D, int G, bool DENSE_LO>
+template <int D, int G, bool DENSE_LO, bool RES2>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p, const CellList cl) {
   using VS = VShare<G>;
@@ -649,9 +690,10 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   const int ci = unit_id / (H * p.batch);
   const int cell = cl.cell[ci];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const size_t uidx = ((size_t)ci * p.batch + b) * H + h;
+  // outputs (and queries) sit at the cell's index in the caller's list
+  const size_t uidx = ((size_t)cl.out[ci] * p.batch + b) * H + h;
 
-  const Unit u = resolve(p, cell, b, h, D);
+  const Unit u = resolve<RES2>(p, cell, b, h, D);
   if (!u.ok) {
     // Host checks make this unreachable; flag it and leave the outputs alone.
     // Every CTA of the cluster takes this branch together (same unit).
@@ -722,19 +764,42 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   uint8_t* const stg1 = reinterpret_cast<uint8_t*>(red + warp * G * D);
   static_assert(kRegNext || 16 * D <= 4 * G * D, "a staged value block must fit a warp's rows");
   int sti = 0;
-  if (!kRegNext) {
-    if (blk0 + warp < blk1 && full_block(blk0 + warp)) stage_vblock<D>(stg0, u, blk0 + warp, lane);
-    cp_async_commit();
-  }
-  // bf16 positions: residual, raw cells, the SHARE current token
+  auto stage_first = [&]() {
+    if (!kRegNext) {
+      if (blk0 + warp < blk1 && full_block(blk0 + warp)) stage_vblock<D>(stg0, u, blk0 + warp, lane);
+      cp_async_commit();
+    }
+  };
+  if constexpr (!RES2) stage_first();
+  // bf16 positions: residual, raw cells, the SHARE current token, a RES2
+  // unit's window (and its bf16 reference's positions)
   for (int pos = max(p0, u.nq) + 32 * warp + lane; pos < p1; pos += 32 * kWarps) {
     float s[G];
-    dot_bf16<D, G>(raw_row(u, pos, D, false), q_s, s);
+    dot_bf16<D, G>(raw_row<RES2>(u, pos, D, false), q_s, s);
 #pragma unroll
     for (int r = 0; r < G; ++r) {
       sc[r * S + pos - p0] = s[r] * sscale;
       lmax[r] = fmaxf(lmax[r], s[r] * sscale);
     }
+  }
+  if constexpr (RES2) {
+    // residual keys: sc += sm_scale * <q, d^> over the residual-coded
+    // positions (written above by the same threads: the same warp-strided
+    // blocks, lane = token), then the maximum over the finished scores
+    Unit ur = u;
+    ur.data = u.own;
+    ur.Ld = u.Lo;
+    ur.data_kind = LOOPKV_Q2;
+    ur.nq = u.rtok;
+    key_pass<D, false, G, true>(ur, blk0, min(blk1, u.rtok / 32), p0, p1, q_s, qs, sc, S, sscale,
+                                warp, lane, lmax);
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      lmax[r] = -INFINITY;
+      for (int i = tid; i < p1 - p0; i += kThreads) lmax[r] = fmaxf(lmax[r], sc[r * S + i]);
+    }
+    stage_first();  // the staging buffer is the q * scale rows the residual pass used
   }
 #pragma unroll
   for (int r = 0; r < G; ++r) {
@@ -943,12 +1008,45 @@ decode_kernel(const DecodeParams p, const CellList cl) {
           const float mid = ((ballot >> tk) & 1u) ? 0.f : mid_unsel;
           token_share(hwv, mtv, pt, mid, vh + lo_off + it * TPI * vrow);
         } else if (tpos < p1) {
-          value_raw<G>(acc, raw_row(u, tpos, D, true) + hf * VS::CH * 2, pt);
+          value_raw<G>(acc, raw_row<RES2>(u, tpos, D, true) + hf * VS::CH * 2, pt);
         }
       }
     }
   }
   if (!kRegNext) cp_async_wait<0>();  // nothing stays in flight into the reduction rows
+  if constexpr (RES2) {
+    // residual values: acc += p * (scale * code + zero) of the unit's own
+    // 2-bit residual rows, every residual-coded position (full blocks)
+    const uint8_t* rvh = u.own + u.Lo.v_hi;
+    const uint8_t* rvm = u.own + u.Lo.v_meta;
+    const float rmul = pow2(kSub);
+    for (int bk = blk0 + warp; bk < min(blk1, u.rtok / 32); bk += kWarps) {
+      float pw[G];
+#pragma unroll
+      for (int r = 0; r < G; ++r) pw[r] = sc[r * S + bk * 32 + lane - p0] * f[r];
+#pragma unroll
+      for (int it = 0; it < LPT; ++it) {
+        const int tk = it * TPI + lane / LPT;
+        float pt[G];
+#pragma unroll
+        for (int r = 0; r < G; ++r) pt[r] = __shfl_sync(0xffffffffu, pw[r], tk);
+        const size_t row = (size_t)(bk * 32 + tk) * vrow;
+        uint32_t hw[VS::NW];
+        float mt[2 * VS::NGRP];
+        load_words<VS::NW>(hw, rvh + row + hf * (VS::CH / 4));
+        load_meta<VS::NGRP>(mt, rvm + row + (hf * VS::CH / 32) * 8);
+        float a[G][VS::NGRP];
+#pragma unroll
+        for (int r = 0; r < G; ++r)
+#pragma unroll
+          for (int gi = 0; gi < VS::NGRP; ++gi) {
+            a[r][gi] = (rmul * pt[r]) * mt[2 * gi];
+            gc[r][gi] = fmaf(pt[r], mt[2 * gi + 1], gc[r][gi]);
+          }
+        value_codes<G>(acc, hw, a);
+      }
+    }
+  }
   // low planes of the selected tokens: acc += p * scale * lo.  The warp
   // gathers its selected positions into a list and processes them TPI at a
   // time, so the cost follows the number of selected tokens.
@@ -1052,10 +1150,10 @@ constexpr size_t decode_smem(int S) {
                           (size_t)G * S);
 }
 
-template <int D, int G, bool DENSE_LO>
+template <int D, int G, bool DENSE_LO, bool RES2>
 int launch_decode_t(const DecodeParams& p, const CellList& cells, cudaStream_t stream) {
   const size_t smem = decode_smem<D, G>(p.slots);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, DENSE_LO>,
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, DENSE_LO, RES2>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_cells * p.batch * p.n_heads;
@@ -1075,21 +1173,22 @@ int launch_decode_t(const DecodeParams& p, const CellList& cells, cudaStream_t s
   }
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, G, DENSE_LO>, p, cells);
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, G, DENSE_LO, RES2>, p, cells);
   return (int)e;
 }
 
-template <int D, int G>
+template <int D, int G, bool RES2>
 int launch_decode_g(const DecodeParams& p, const CellList& cells, cudaStream_t s) {
   const bool dense = !(p.tau > 0.f);
-  return dense ? launch_decode_t<D, G, true>(p, cells, s) : launch_decode_t<D, G, false>(p, cells, s);
+  return dense ? launch_decode_t<D, G, true, RES2>(p, cells, s)
+               : launch_decode_t<D, G, false, RES2>(p, cells, s);
 }
 
-template <int D>
+template <int D, bool RES2>
 int launch_decode_d(const DecodeParams& p, const CellList& cells, cudaStream_t s) {
-  if (p.group == 2) return launch_decode_g<D, 2>(p, cells, s);
-  if (p.group == 4) return launch_decode_g<D, 4>(p, cells, s);
-  return launch_decode_g<D, 1>(p, cells, s);
+  if (p.group == 2) return launch_decode_g<D, 2, RES2>(p, cells, s);
+  if (p.group == 4) return launch_decode_g<D, 4, RES2>(p, cells, s);
+  return launch_decode_g<D, 1, RES2>(p, cells, s);
 }
 
 // Largest score slots per query that keep two CTAs on an SM (at most
@@ -1112,10 +1211,11 @@ int decode_max_slots(int head_dim, int group) {
 }
 int decode_max_split() { return kMaxSplit; }
 
-int launch_decode(const DecodeParams& p, const CellList& cells, void* stream, int head_dim) {
+int launch_decode(const DecodeParams& p, const CellList& cells, void* stream, int head_dim,
+                  bool res2) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (head_dim == 64) return launch_decode_d<64>(p, cells, s);
-  return launch_decode_d<128>(p, cells, s);
+  if (head_dim == 64) return res2 ? launch_decode_d<64, true>(p, cells, s) : launch_decode_d<64, false>(p, cells, s);
+  return res2 ? launch_decode_d<128, true>(p, cells, s) : launch_decode_d<128, false>(p, cells, s);
 }
 
 }  // namespace loopkv

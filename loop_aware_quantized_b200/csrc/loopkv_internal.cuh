@@ -12,6 +12,11 @@
 namespace loopkv {
 
 constexpr int kGroup = 32;  // tokens per key group, channels per value group
+constexpr int kResWindow = 64;  // bf16 window slots of a RES2 unit
+
+// Residual-coded positions of a RES2 unit of n tokens: group g is quantized
+// once the unit holds 32 (g + 2) tokens.
+inline __host__ __device__ int res2_qtok(int n) { return n >= 2 * kGroup ? (n / kGroup - 1) * kGroup : 0; }
 
 // Status bits a kernel may set in the table's status word.
 constexpr uint32_t kStatusLength = 1u;     // a length outside [0, capacity]
@@ -28,7 +33,7 @@ static_assert(sizeof(TableHeader) == 256, "header size");
 
 struct DevCell {               // 16 bytes per cell
   int32_t kind;                // loopkv_kind
-  int32_t src;                 // SHARE: the final-loop cell of the same layer; else itself
+  int32_t src;                 // SHARE, RES2: the final-loop cell of the same layer; else itself
   int32_t pad[2];
 };
 
@@ -65,16 +70,17 @@ inline __host__ __device__ UnitLayout unit_layout(int kind, int D, int cap) {
   const size_t block = ng * 8 * (size_t)D;  // a key plane, key meta, value plane or value meta
   const size_t res = (size_t)kGroup * D * 2;
   size_t off = 0;
-  if (kind == LOOPKV_Q4 || kind == LOOPKV_Q2) {
+  if (kind == LOOPKV_Q4 || kind == LOOPKV_Q2 || kind == LOOPKV_RES2) {
     const bool q4 = kind == LOOPKV_Q4;
+    const size_t window = kind == LOOPKV_RES2 ? res * (kResWindow / kGroup) : res;
     L.k_hi = off;   off += block;
     L.k_lo = off;   off += q4 ? block : 0;
     L.k_meta = off; off += block;
     L.v_hi = off;   off += block;
     L.v_lo = off;   off += q4 ? block : 0;
     L.v_meta = off; off += block;
-    L.res_k = off;  off += res;
-    L.res_v = off;  off += res;
+    L.res_k = off;  off += window;
+    L.res_v = off;  off += window;
   } else if (kind == LOOPKV_SHARE) {
     L.cur_k = off;  off += round_up((size_t)D * 2, 128);
     L.cur_v = off;  off += round_up((size_t)D * 2, 128);
@@ -90,6 +96,7 @@ inline __host__ __device__ UnitLayout unit_layout(int kind, int D, int cap) {
 
 struct CellList {
   int32_t cell[LOOPKV_MAX_CELLS_PER_CALL];
+  int32_t out[LOOPKV_MAX_CELLS_PER_CALL];  // the cell's index in the caller's list (its input / output slot)
 };
 
 struct AppendParams {
@@ -119,10 +126,14 @@ struct DecodeParams {
 };
 
 // Launchers (decode.cu / append.cu).  Return cudaGetLastError() as int.
-int launch_append(const AppendParams& p, const CellList& cells, void* stream, int head_dim);
+// res2: the cells are all RES2 (their own kernel); else none is.  cells.out[i]
+// is cell i's index in the caller's list (its slot of the inputs / outputs).
+int launch_append(const AppendParams& p, const CellList& cells, void* stream, int head_dim,
+                  bool res2);
 int launch_commit_lengths(uint8_t* table, const CellList& cells, int n_cells, int batch,
                           const int32_t* n_new, void* stream);
-int launch_decode(const DecodeParams& p, const CellList& cells, void* stream, int head_dim);
+int launch_decode(const DecodeParams& p, const CellList& cells, void* stream, int head_dim,
+                  bool res2);
 int decode_max_slots(int head_dim, int group);  // largest per-query score slots per CTA
 int decode_max_split();                 // largest cluster size used
 

@@ -28,6 +28,12 @@ struct loopkv_plan {
   size_t cache_bytes = 0;
 
   int src(int cell) const { return (n_loops - 1) * n_layers + cell % n_layers; }
+  // positions of a unit's reference that a RES2 unit may read: the
+  // quantized ones of a Q4/Q2 reference, every one of a BF16 reference
+  int ref_positions(int cell, int b) const {
+    const int r = src(cell);
+    return kinds[r] == LOOPKV_BF16 ? L(r, b) : L(r, b) / kGroup * kGroup;
+  }
   int32_t& L(int cell, int b) { return len[(size_t)cell * max_batch + b]; }
   int32_t L(int cell, int b) const { return len[(size_t)cell * max_batch + b]; }
 };
@@ -56,8 +62,11 @@ loopkv_status validate_desc(const loopkv_plan_desc* d) {
   const int cells = d->n_loops * d->n_layers;
   for (int c = 0; c < cells; ++c) {
     const int k = d->kinds[c];
-    if (k > LOOPKV_BF16) return LOOPKV_ERR_PLAN;
-    if (k == LOOPKV_SHARE && c / d->n_layers == d->n_loops - 1) return LOOPKV_ERR_PLAN;
+    if (k > LOOPKV_RES2) return LOOPKV_ERR_PLAN;
+    // SHARE and RES2 read the final loop's cell of their layer, so neither
+    // can sit in the final loop (whose cells are then Q4, Q2 or BF16)
+    if ((k == LOOPKV_SHARE || k == LOOPKV_RES2) && c / d->n_layers == d->n_loops - 1)
+      return LOOPKV_ERR_PLAN;
   }
   return LOOPKV_OK;
 }
@@ -82,11 +91,17 @@ loopkv_status check_cells(const loopkv_plan* p, const int32_t* h_cells, int32_t 
     if (c < 0 || c >= p->n_cells || seen[c]) return LOOPKV_ERR_INVALID_ARG;
     seen[c] = 1;
     out->cell[i] = c;
+    out->out[i] = i;
   }
   return LOOPKV_OK;
 }
 
 loopkv_status from_cuda(int e) { return e == 0 ? LOOPKV_OK : LOOPKV_ERR_CUDA; }
+
+loopkv_status decode_launch(loopkv_plan* p, const CellList& cl, int n_cells, int batch,
+                            int npos_max, bool res2, const uint16_t* d_q, float* d_out,
+                            float* d_lse, uint32_t* d_mask, int32_t mask_words, int32_t* d_nsel,
+                            void* stream);
 
 int env_int(const char* name, int dflt) {
   const char* v = std::getenv(name);
@@ -151,7 +166,7 @@ loopkv_status loopkv_plan_load(const loopkv_plan_desc* desc, void* d_table, size
   size_t off = 0;
   for (int c = 0; c < p->n_cells; ++c) {
     cells[c].kind = p->kinds[c];
-    cells[c].src = p->kinds[c] == LOOPKV_SHARE ? p->src(c) : c;
+    cells[c].src = (p->kinds[c] == LOOPKV_SHARE || p->kinds[c] == LOOPKV_RES2) ? p->src(c) : c;
     for (int b = 0; b < p->max_batch; ++b) {
       const size_t stride = unit_layout(p->kinds[c], p->D, p->cap[b]).total;
       DevSeq& s = seqs[(size_t)c * p->max_batch + b];
@@ -198,6 +213,26 @@ loopkv_status loopkv_append(loopkv_plan* p, const int32_t* h_cells, int32_t n_ce
     for (int b = 0; b < batch; ++b)
       if ((long long)p->L(c, b) + h_n_new[b] > p->cap[b]) return LOOPKV_ERR_CAPACITY;
   }
+  for (int i = 0; i < n_cells; ++i) {
+    const int c = cl.cell[i];
+    if (p->kinds[c] != LOOPKV_RES2) continue;
+    // the reference's groups this append quantizes against must be there
+    // already (its length before this call: the kernels run side by side)
+    for (int b = 0; b < batch; ++b)
+      if (h_n_new[b] > 0 && res2_qtok(p->L(c, b) + h_n_new[b]) > p->ref_positions(c, b))
+        return LOOPKV_ERR_INVALID_ARG;
+  }
+  // RES2 cells go to their own kernel: split the list, keeping each
+  // cell's index in the caller's list (its input slot)
+  CellList plain{}, res{};
+  int n_plain = 0, n_res = 0;
+  for (int i = 0; i < n_cells; ++i) {
+    CellList& dst = p->kinds[cl.cell[i]] == LOOPKV_RES2 ? res : plain;
+    int& k = p->kinds[cl.cell[i]] == LOOPKV_RES2 ? n_res : n_plain;
+    dst.cell[k] = cl.cell[i];
+    dst.out[k] = i;
+    ++k;
+  }
   AppendParams ap{};
   ap.table = p->d_table;
   ap.cache = p->d_cache;
@@ -208,7 +243,15 @@ loopkv_status loopkv_append(loopkv_plan* p, const int32_t* h_cells, int32_t n_ce
   ap.n_heads = p->H;
   ap.n_new_max = n_new_max;
   for (int b = 0; b < batch; ++b) ap.n_new[b] = h_n_new[b];
-  int e = launch_append(ap, cl, stream, p->D);
+  int e = 0;
+  if (n_plain > 0) {
+    ap.n_cells = n_plain;
+    e = launch_append(ap, plain, stream, p->D, false);
+  }
+  if (e == 0 && n_res > 0) {
+    ap.n_cells = n_res;
+    e = launch_append(ap, res, stream, p->D, true);
+  }
   if (e == 0) e = launch_commit_lengths(p->d_table, cl, n_cells, batch, h_n_new, stream);
   if (e != 0) return LOOPKV_ERR_CUDA;
   for (int i = 0; i < n_cells; ++i)
@@ -224,11 +267,14 @@ loopkv_status loopkv_decode(loopkv_plan* p, const int32_t* h_cells, int32_t n_ce
   if (st != LOOPKV_OK) return st;
   if (d_q == nullptr || d_out == nullptr || !aligned16(d_q) || !aligned16(d_out))
     return LOOPKV_ERR_INVALID_ARG;
-  int npos_max = 0;
+  int npos_max[2] = {0, 0};  // plain cells, RES2 cells
+  CellList lists[2]{};
+  int counts[2] = {0, 0};
   for (int i = 0; i < n_cells; ++i) {
     const int c = cl.cell[i];
     const bool share = p->kinds[c] == LOOPKV_SHARE;
-    const int dkind = share ? p->kinds[p->src(c)] : p->kinds[c];
+    const bool res2 = p->kinds[c] == LOOPKV_RES2;
+    const int dkind = (share || res2) ? p->kinds[p->src(c)] : p->kinds[c];
     for (int b = 0; b < batch; ++b) {
       const int n = p->L(c, b);
       if (n < 1) return LOOPKV_ERR_INVALID_ARG;
@@ -238,15 +284,39 @@ loopkv_status loopkv_decode(loopkv_plan* p, const int32_t* h_cells, int32_t n_ce
         nd = p->L(p->src(c), b);
         if (n_att > nd) return LOOPKV_ERR_INVALID_ARG;
       }
-      if (d_mask != nullptr && dkind == LOOPKV_Q4) {
-        const int nq = std::min(n_att, nd / kGroup * kGroup);
-        if ((nq + kGroup - 1) / kGroup > mask_words) return LOOPKV_ERR_INVALID_ARG;
+      int nq = std::min(n_att, nd / kGroup * kGroup);
+      if (res2) {
+        nq = res2_qtok(n);
+        if (nq > p->ref_positions(c, b)) return LOOPKV_ERR_INVALID_ARG;
       }
-      npos_max = std::max(npos_max, n);
+      if (d_mask != nullptr && dkind == LOOPKV_Q4 && (nq + kGroup - 1) / kGroup > mask_words)
+        return LOOPKV_ERR_INVALID_ARG;
+      npos_max[res2] = std::max(npos_max[res2], n);
     }
+    lists[res2].cell[counts[res2]] = c;
+    lists[res2].out[counts[res2]] = i;
+    ++counts[res2];
   }
   if (d_mask != nullptr && (mask_words < 0 || !aligned16(d_mask))) return LOOPKV_ERR_INVALID_ARG;
+  for (int k = 0; k < 2; ++k) {
+    if (counts[k] == 0) continue;
+    st = decode_launch(p, lists[k], counts[k], batch, npos_max[k], k == 1, d_q, d_out, d_lse,
+                       d_mask, mask_words, d_nsel, stream);
+    if (st != LOOPKV_OK) return st;
+  }
+  return LOOPKV_OK;
+}
 
+}  // extern "C"
+
+namespace {
+
+// One decode launch over cells of one sort (all RES2 or none): choose the
+// cluster split and the score slots, fill the parameter block, launch.
+loopkv_status decode_launch(loopkv_plan* p, const CellList& cl, int n_cells, int batch,
+                            int npos_max, bool res2, const uint16_t* d_q, float* d_out,
+                            float* d_lse, uint32_t* d_mask, int32_t mask_words, int32_t* d_nsel,
+                            void* stream) {
   // Split a unit over a cluster of CTAs when its positions do not fit one
   // CTA's score slots (per query of the group), or when there are too few
   // units to fill the GPU.
@@ -281,8 +351,12 @@ loopkv_status loopkv_decode(loopkv_plan* p, const int32_t* h_cells, int32_t n_ce
   dp.slots = slots_for(split);
   dp.tau = p->tau;
   dp.score_scale = p->sm_scale * 1.4426950408889634f;
-  return from_cuda(launch_decode(dp, cl, stream, p->D));
+  return from_cuda(launch_decode(dp, cl, stream, p->D, res2));
 }
+
+}  // namespace
+
+extern "C" {
 
 loopkv_status loopkv_set_lengths(loopkv_plan* p, const int32_t* h_cells, int32_t n_cells,
                                  int32_t batch, const int32_t* h_len, void* stream) {
@@ -300,6 +374,8 @@ loopkv_status loopkv_set_lengths(loopkv_plan* p, const int32_t* h_cells, int32_t
       if ((k == LOOPKV_Q4 || k == LOOPKV_Q2) && nw < old / kGroup * kGroup && nw % kGroup != 0)
         return LOOPKV_ERR_INVALID_ARG;
       if (k == LOOPKV_SHARE && nw != old) return LOOPKV_ERR_INVALID_ARG;  // current token is gone
+      // RES2: the residual-coded count must stay (its bf16 window is gone)
+      if (k == LOOPKV_RES2 && res2_qtok(nw) != res2_qtok(old)) return LOOPKV_ERR_INVALID_ARG;
     }
   }
   // Residual slots of a Q4/Q2 unit cut back to a group boundary hold tokens

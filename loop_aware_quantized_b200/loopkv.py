@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 # LOOPKV_LIBRARY may name another build of the same library (same ABI).
 LIB_PATH = os.environ.get("LOOPKV_LIBRARY") or os.path.join(_HERE, "libloopkv.so")
 
-LOOPKV_Q4, LOOPKV_Q2, LOOPKV_SHARE, LOOPKV_BF16 = 0, 1, 2, 3
+LOOPKV_Q4, LOOPKV_Q2, LOOPKV_SHARE, LOOPKV_BF16, LOOPKV_RES2 = 0, 1, 2, 3, 4
 LOOPKV_MAX_CELLS_PER_CALL = 256
 LOOPKV_MAX_BATCH = 256
 

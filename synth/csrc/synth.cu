@@ -57,12 +57,41 @@ __device__ __forceinline__ uint16_t key_bits(int cell, int b, int h, uint32_t t,
   return to_bf16_bits(__fmul_rn(z, chscale[((size_t)cell * H + h) * D + d]));
 }
 
+__device__ __forceinline__ uint16_t value_bits(int cell, int b, int h, uint32_t t, int d, int H,
+                                               uint32_t seed, float nscale) {
+  const U4 u = philox(t, (uint32_t)d, (uint32_t)(h + H * b), (uint32_t)cell, seed, kStreamV);
+  return to_bf16_bits(normal_from(u, nscale));
+}
+
+// Keys / values of a cell that follows a reference cell (refs[cell] >= 0):
+// the reference's raw token plus 0.25 * N(0,1) of the cell's own stream
+// (keys: times the cell's channel scale).
+__device__ __forceinline__ uint16_t key_of(int cell, const int32_t* refs, int b, int h, uint32_t t,
+                                           int d, int H, int D, const float* chscale,
+                                           uint32_t seed, float nscale) {
+  const int ref = refs[cell];
+  if (ref < 0) return key_bits(cell, b, h, t, d, H, D, chscale, seed, nscale);
+  const float kr = from_bf16_bits(key_bits(ref, b, h, t, d, H, D, chscale, seed, nscale));
+  const U4 u = philox(t, (uint32_t)d, (uint32_t)(h + H * b), (uint32_t)cell, seed, kStreamK);
+  const float z = __fmul_rn(__fmul_rn(normal_from(u, nscale), 0.25f),
+                            chscale[((size_t)cell * H + h) * D + d]);
+  return to_bf16_bits(__fadd_rn(kr, z));
+}
+__device__ __forceinline__ uint16_t value_of(int cell, const int32_t* refs, int b, int h,
+                                             uint32_t t, int d, int H, uint32_t seed, float nscale) {
+  const int ref = refs[cell];
+  if (ref < 0) return value_bits(cell, b, h, t, d, H, seed, nscale);
+  const float vr = from_bf16_bits(value_bits(ref, b, h, t, d, H, seed, nscale));
+  const U4 u = philox(t, (uint32_t)d, (uint32_t)(h + H * b), (uint32_t)cell, seed, kStreamV);
+  return to_bf16_bits(__fadd_rn(vr, __fmul_rn(normal_from(u, nscale), 0.25f)));
+}
+
 // out[c][b][h][i][d] for positions t0[b] + i, i < T.
 __global__ void gen_kv_kernel(uint16_t* __restrict__ k, uint16_t* __restrict__ v,
                               const int32_t* __restrict__ cells, const int32_t* __restrict__ seqs,
                               const int32_t* __restrict__ t0, int n_cells, int batch, int H, int D,
                               int T, int table_cells, const float* __restrict__ chscale,
-                              uint32_t seed, float nscale) {
+                              const int32_t* __restrict__ refs, uint32_t seed, float nscale) {
   const size_t total = (size_t)n_cells * batch * H * T * D;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -77,11 +106,8 @@ __global__ void gen_kv_kernel(uint16_t* __restrict__ k, uint16_t* __restrict__ v
     const int cell = cells[c], b = seqs[bl];
     if (cell < 0 || cell >= table_cells) continue;  // host passes valid ids; never index past the table
     const uint32_t t = (uint32_t)(t0[bl] + ti);
-    if (k) k[i] = key_bits(cell, b, h, t, d, H, D, chscale, seed, nscale);
-    if (v) {
-      const U4 u = philox(t, (uint32_t)d, (uint32_t)(h + H * b), (uint32_t)cell, seed, kStreamV);
-      v[i] = to_bf16_bits(normal_from(u, nscale));
-    }
+    if (k) k[i] = key_of(cell, refs, b, h, t, d, H, D, chscale, seed, nscale);
+    if (v) v[i] = value_of(cell, refs, b, h, t, d, H, seed, nscale);
   }
 }
 
@@ -95,7 +121,7 @@ __global__ void gen_q_kernel(uint16_t* __restrict__ q, const int32_t* __restrict
                              const int32_t* __restrict__ srcs, const int32_t* __restrict__ seqs,
                              const int32_t* __restrict__ lens, int n_cells, int batch, int H, int g,
                              int D, int mode, int table_cells, const float* __restrict__ chscale,
-                             uint32_t seed, float nscale) {
+                             const int32_t* __restrict__ refs, uint32_t seed, float nscale) {
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= (long long)n_cells * batch * H * g) return;
@@ -127,7 +153,7 @@ __global__ void gen_q_kernel(uint16_t* __restrict__ q, const int32_t* __restrict
     for (int i = 0; i < kcount; ++i) {
       const int p = picks[i];
       const int kc = (share && p < n - 1) ? src : cell;
-      key[i] = from_bf16_bits(key_bits(kc, b, h, (uint32_t)p, d, H, D, chscale, seed, nscale));
+      key[i] = from_bf16_bits(key_of(kc, refs, b, h, (uint32_t)p, d, H, D, chscale, seed, nscale));
     }
     const U4 un = philox((uint32_t)n, (uint32_t)d + rw, (uint32_t)(h + H * b), (uint32_t)cell, seed,
                          kStreamQNoise);
@@ -150,29 +176,30 @@ extern "C" {
 
 int synth_gen_kv(uint16_t* k, uint16_t* v, const int32_t* d_cells, const int32_t* d_seqs,
                  const int32_t* d_t0, int n_cells, int batch, int H, int D, int T,
-                 int table_cells, const float* d_chscale, uint32_t seed, float nscale,
-                 void* stream) {
+                 int table_cells, const float* d_chscale, const int32_t* d_refs, uint32_t seed,
+                 float nscale, void* stream) {
   const size_t total = (size_t)n_cells * batch * H * T * D;
   if (total == 0) return 0;
   const int threads = 256;
   size_t blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 64) blocks = 148 * 64;
   gen_kv_kernel<<<(unsigned)blocks, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      k, v, d_cells, d_seqs, d_t0, n_cells, batch, H, D, T, table_cells, d_chscale, seed, nscale);
+      k, v, d_cells, d_seqs, d_t0, n_cells, batch, H, D, T, table_cells, d_chscale, d_refs, seed,
+      nscale);
   return (int)cudaGetLastError();
 }
 
 int synth_gen_q(uint16_t* q, const int32_t* d_cells, const int32_t* d_srcs, const int32_t* d_seqs,
                 const int32_t* d_lens, int n_cells, int batch, int H, int g, int D, int mode,
-                int table_cells, const float* d_chscale, uint32_t seed, float nscale,
-                void* stream) {
+                int table_cells, const float* d_chscale, const int32_t* d_refs, uint32_t seed,
+                float nscale, void* stream) {
   const long long warps = (long long)n_cells * batch * H * g;
   if (warps == 0) return 0;
   const int threads = 256;
   const long long blocks = (warps * 32 + threads - 1) / threads;
   gen_q_kernel<<<(unsigned)blocks, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       q, d_cells, d_srcs, d_seqs, d_lens, n_cells, batch, H, g, D, mode, table_cells, d_chscale,
-      seed, nscale);
+      d_refs, seed, nscale);
   return (int)cudaGetLastError();
 }
 

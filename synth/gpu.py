@@ -24,10 +24,10 @@ def _load():
             raise ImportError("libloopkv_synth.so is missing; run `python synth/build.py`")
         lib = ctypes.CDLL(LIB_PATH)
         P, I = ctypes.c_void_p, ctypes.c_int
-        lib.synth_gen_kv.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, ctypes.c_uint32,
+        lib.synth_gen_kv.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, ctypes.c_uint32,
                                      ctypes.c_float, P]
         lib.synth_gen_kv.restype = I
-        lib.synth_gen_q.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, ctypes.c_uint32,
+        lib.synth_gen_q.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, ctypes.c_uint32,
                                     ctypes.c_float, P]
         lib.synth_gen_q.restype = I
         _lib = lib
@@ -46,6 +46,8 @@ class DeviceGenerator:
         self.wl = wl
         self.device = torch.device(device)
         self.chscale = torch.from_numpy(np.ascontiguousarray(wl.chscale)).to(self.device)
+        # per cell: the reference cell a residual cell's tokens follow, else -1
+        self.refs = self._i32([wl.token_ref(c) for c in range(wl.n_cells)])
         self.nscale = float(px.NORMAL_SCALE)
 
     def _i32(self, a):
@@ -67,7 +69,7 @@ class DeviceGenerator:
         d_cells, d_seqs, d_t0 = self._i32(cells), self._i32(seqs), self._i32(t0)
         rc = _load().synth_gen_kv(_p(k), _p(v), _p(d_cells), _p(d_seqs), _p(d_t0), len(cells),
                                   len(seqs), wl.n_heads, wl.head_dim, T, wl.n_cells,
-                                  _p(self.chscale),
+                                  _p(self.chscale), _p(self.refs),
                                   wl.seed, self.nscale, ctypes.c_void_p(s.cuda_stream))
         s.synchronize()
         del d_cells, d_seqs, d_t0
@@ -89,7 +91,7 @@ class DeviceGenerator:
         d_lens = self._i32(np.asarray(lens).reshape(-1))
         rc = _load().synth_gen_q(_p(out), _p(d_cells), _p(d_srcs), _p(d_seqs), _p(d_lens),
                                  len(cells), len(seqs), wl.n_heads, g, wl.head_dim, mode,
-                                 wl.n_cells, _p(self.chscale), wl.seed, self.nscale,
+                                 wl.n_cells, _p(self.chscale), _p(self.refs), wl.seed, self.nscale,
                                  ctypes.c_void_p(s.cuda_stream))
         s.synchronize()
         del d_cells, d_srcs, d_seqs, d_lens

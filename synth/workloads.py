@@ -16,6 +16,10 @@ Recipes (the shapes follow a 1.4B-parameter looped model at 4K-16K context):
           exp(N(0,1)); "outlier": N(0,1), with 4 channels per (cell, head)
           scaled by 10.
   values  N(0,1).
+  Cells stored as 2-bit residuals against the final loop (RES2) follow their
+  reference: each raw key is the reference cell's raw key plus 0.25 * N(0,1)
+  times the cell's own channel factor, each raw value the reference's value
+  plus 0.25 * N(0,1) (the loops of a looped model keep close KV states).
   queries "sum3": the sum of the raw keys at 3 distinct random attended
           positions plus 0.5 * N(0,1); "peaked": 2 * the raw key at one random
           attended position plus N(0,1).  Attended positions of a SHARE unit
@@ -31,8 +35,8 @@ import numpy as np
 
 from . import philox as px
 
-Q4, Q2, SHARE, BF16 = 0, 1, 2, 3
-KIND_NAMES = {Q4: "Q4", Q2: "Q2", SHARE: "SHARE", BF16: "BF16"}
+Q4, Q2, SHARE, BF16, RES2 = 0, 1, 2, 3, 4
+KIND_NAMES = {Q4: "Q4", Q2: "Q2", SHARE: "SHARE", BF16: "BF16", RES2: "RES2"}
 
 # Philox key word 1 selects the stream; key word 0 is the workload seed.
 STREAM_K, STREAM_V, STREAM_QNOISE, STREAM_QPOS = 1, 2, 3, 4
@@ -68,6 +72,10 @@ class Workload:
     def data_cell(self, cell):
         return self.source_cell(cell) if self.kinds[cell] == SHARE else cell
 
+    def token_ref(self, cell):
+        """Cell whose raw tokens a residual cell's tokens follow, else -1."""
+        return self.source_cell(cell) if self.kinds[cell] == RES2 else -1
+
     def cells_of_loop(self, loop):
         return list(range(loop * self.n_layers, (loop + 1) * self.n_layers))
 
@@ -85,6 +93,11 @@ def raw_keys(wl, cell, b, h, t0, t1):
     d = np.arange(D, dtype=np.uint32)[None, :]
     u = px.philox4x32(t, d, _unit_word(wl, b, h), np.uint32(cell), wl.seed, STREAM_K)
     z = px.normal_from_bits(*u)
+    ref = wl.token_ref(cell)
+    if ref >= 0:
+        kr = px.bf16_bits_to_float(raw_keys(wl, ref, b, h, t0, t1))
+        noise = ((z * np.float32(0.25)).astype(np.float32) * wl.chscale[cell, h][None, :])
+        return px.float_to_bf16_bits((kr + noise.astype(np.float32)).astype(np.float32))
     x = (z * wl.chscale[cell, h][None, :]).astype(np.float32)
     return px.float_to_bf16_bits(x)
 
@@ -95,7 +108,12 @@ def raw_values(wl, cell, b, h, t0, t1):
     t = np.arange(t0, t1, dtype=np.uint32)[:, None]
     d = np.arange(D, dtype=np.uint32)[None, :]
     u = px.philox4x32(t, d, _unit_word(wl, b, h), np.uint32(cell), wl.seed, STREAM_V)
-    return px.float_to_bf16_bits(px.normal_from_bits(*u))
+    z = px.normal_from_bits(*u)
+    ref = wl.token_ref(cell)
+    if ref >= 0:
+        vr = px.bf16_bits_to_float(raw_values(wl, ref, b, h, t0, t1))
+        return px.float_to_bf16_bits((vr + (z * np.float32(0.25)).astype(np.float32)).astype(np.float32))
+    return px.float_to_bf16_bits(z)
 
 
 def query_positions(wl, cell, b, h, n, rep=0):
@@ -208,7 +226,7 @@ def round_up(x, m):
 # --------------------------------------------------------------- the configs
 
 def make(config, **over):
-    """Workload for config 0, 1, 2, "3a".."3d" or 4; keyword args override fields."""
+    """Workload for config 0, 1, 2, "2r", "3a".."3d" or 4; keyword args override fields."""
     config = str(config)
     if config == "0":
         # plan given as [[Q4, Q2], [SHARE, Q4]] indexed [layer][loop]
@@ -223,10 +241,14 @@ def make(config, **over):
                       np.array([4096 + 17], np.int32), round_up([4096 + 17 + 64], 32).astype(np.int32),
                       "lognormal", "sum3", lognormal_chscale(1, 96, 16, 128),
                       "4x24 cells, 16 heads, D 128, batch 1, 4096 + 17 tokens")
-    elif config == "2" or config.startswith("3"):
+    elif config in ("2", "2r") or config.startswith("3"):
         kinds = percent_plan(2, 4, 24, 0.35, 0.30, final_all_q4=True)
         tau = 0.002
         name = "batched-16k"
+        if config == "2r":
+            # the SHARE cells of the plan stored as 2-bit residuals instead
+            kinds = np.where(kinds == SHARE, RES2, kinds).astype(np.uint8)
+            name = "batched-16k-residual"
         if config.startswith("3"):
             sub = config[1:]
             if sub == "a":

@@ -15,8 +15,12 @@ def make_plan(wl, seqs):
 
 
 def build_cache(wl, plan, gen, seqs, lengths, cells=None, chunk_tokens=None):
-    """Append every token of [0, lengths[b]) to each cell (one call per cell)."""
+    """Append every token of [0, lengths[b]) to each cell (one call per cell).
+
+    The final loop's cells go first: a RES2 cell quantizes its residuals
+    against them, so they must hold the tokens before it does."""
     cells = list(range(wl.n_cells)) if cells is None else list(cells)
+    cells.sort(key=lambda c: c // wl.n_layers != wl.n_loops - 1)
     T = int(max(lengths))
     kbuf = vbuf = None
     for c in cells:

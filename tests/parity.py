@@ -30,12 +30,15 @@ def workload(config):
 
 
 def _oracle_units(orc, wl, cell, b, n_own, n_src, h):
-    """The oracle's unit (and SHARE source) for (cell, b, h), built from the
-    host generator's raw keys and values."""
+    """The oracle's unit (and the SHARE source or RES2 reference: the final
+    loop's unit, n_src tokens) for (cell, b, h), built from the host
+    generator's raw keys and values."""
     kind = int(wl.kinds[cell])
     cap = int(wl.capacity[b])
     own = orc.OracleUnit(kind, wl.head_dim, cap)
     if kind == W.SHARE:
+        # A SHARE unit keeps only its current token; earlier tokens only add
+        # to its length, so they are appended as zeros.
         k = np.zeros((n_own, wl.head_dim), np.uint16)
         v = np.zeros((n_own, wl.head_dim), np.uint16)
         k[-1] = W.raw_keys(wl, cell, b, h, n_own - 1, n_own)[0]
@@ -47,6 +50,11 @@ def _oracle_units(orc, wl, cell, b, n_own, n_src, h):
     else:
         own.append(W.raw_keys(wl, cell, b, h, 0, n_own), W.raw_values(wl, cell, b, h, 0, n_own))
         src = None
+        if kind == W.RES2:
+            src_cell = wl.source_cell(cell)
+            src = orc.OracleUnit(int(wl.kinds[src_cell]), wl.head_dim, cap)
+            src.append(W.raw_keys(wl, src_cell, b, h, 0, n_src),
+                       W.raw_values(wl, src_cell, b, h, 0, n_src))
     return own, src
 
 
@@ -69,7 +77,8 @@ def oracle_unit_job(args):
     """Build the oracle state of one unit and decode it.
 
     args = (config, cell, b, h, n_own, n_src, want_bytes): n_own tokens in the
-    unit, n_src tokens in its SHARE source (ignored otherwise).
+    unit, n_src tokens in its SHARE source or RES2 reference (ignored
+    otherwise).
     Returns a dict with the host query bits, the oracle result and, if asked,
     the unit's canonical bytes.
     """
@@ -77,28 +86,13 @@ def oracle_unit_job(args):
     config, cell, b, h, n_own, n_src, want_bytes = args
     wl = workload(config)
     kind = int(wl.kinds[cell])
-    cap = int(wl.capacity[b])
-    own = orc.OracleUnit(kind, wl.head_dim, cap)
-    if kind == W.SHARE:
-        # A SHARE unit keeps only its current token; earlier tokens only add
-        # to its length, so they are appended as zeros.
-        k = np.zeros((n_own, wl.head_dim), np.uint16)
-        v = np.zeros((n_own, wl.head_dim), np.uint16)
-        k[-1] = W.raw_keys(wl, cell, b, h, n_own - 1, n_own)[0]
-        v[-1] = W.raw_values(wl, cell, b, h, n_own - 1, n_own)[0]
-        own.append(k, v)
-        src_cell = wl.source_cell(cell)
-        src = orc.OracleUnit(int(wl.kinds[src_cell]), wl.head_dim, cap)
-        src.append(W.raw_keys(wl, src_cell, b, h, 0, n_src), W.raw_values(wl, src_cell, b, h, 0, n_src))
-    else:
-        own.append(W.raw_keys(wl, cell, b, h, 0, n_own), W.raw_values(wl, cell, b, h, 0, n_own))
-        src = None
+    own, src = _oracle_units(orc, wl, cell, b, n_own, n_src, h)
     q = W.query(wl, cell, b, h, n_own)
     r = orc.decode(own, q, wl.tau, src=src, band=BAND)
     out = dict(q=q, out=r.out, lse=r.lse, mask=r.mask, nsel=r.nsel, slack=r.slack,
                weights=r.weights, kind=kind)
     if want_bytes:
-        out["bytes"], out["valid"] = own.serialize()
+        out["bytes"], out["valid"] = own.serialize(src=src if kind == W.RES2 else None)
     return out
 
 

@@ -61,7 +61,10 @@ def test_plan_query_rejects_invalid_plans(lk):
     assert _query(lk)[0] == 0
     assert _query(lk, kinds=[0, 0, 2, 0])[0] == 2          # SHARE in the final loop
     assert _query(lk, n_loops=1, n_layers=4, kinds=[0, 2, 0, 0])[0] == 2
-    assert _query(lk, kinds=[0, 4, 1, 0])[0] == 2          # unknown kind
+    assert _query(lk, kinds=[0, 5, 1, 0])[0] == 2          # unknown kind
+    assert _query(lk, kinds=[0, 0, 4, 0])[0] == 2          # RES2 in the final loop
+    assert _query(lk, kinds=[0, 4, 1, 0])[0] == 0          # RES2 in a non-final loop
+    assert _query(lk, kinds=[4, 4, 3, 1])[0] == 0          # bf16 and 2-bit references
     assert _query(lk, head_dim=96)[0] == 2
     assert _query(lk, tau=-1.0)[0] == 2
     assert _query(lk, tau=float("nan"))[0] == 2
@@ -113,7 +116,7 @@ def test_cache_size_matches_the_oracle_layout(lk):
     unit's region size (library plan_query vs oracle region_bytes)."""
     from oracle import oracle as orc
     from synth import workloads as W
-    for config in ("0", "1", "2", "4"):
+    for config in ("0", "1", "2", "2r", "4"):
         wl = W.make(config)
         rc, sizes = _query(lk, n_loops=wl.n_loops, n_layers=wl.n_layers, n_kv_heads=wl.n_heads,
                            head_dim=wl.head_dim, capacity=wl.capacity, kinds=wl.kinds,

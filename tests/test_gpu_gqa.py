@@ -87,6 +87,14 @@ def test_group_decode_matches_oracle(pool, cuda_device, g, D):
 
 
 @pytest.mark.parametrize("g", [2, 4])
+def test_group_residual_cells(pool, cuda_device, g):
+    RS = W.RES2
+    lengths = (1, 33, 97, 300)
+    for kinds in ((RS, RS, Q4, Q2), (RS, SH, BF, Q4)):
+        _run(_spec(128, kinds, lengths, 0.02), g, pool, cuda_device)
+
+
+@pytest.mark.parametrize("g", [2, 4])
 @pytest.mark.parametrize("tau", [0.0, 2.0])
 def test_group_tau_extremes(pool, cuda_device, tau, g):
     _run(_spec(128, (Q4, SH, Q2, Q4), (40, 300, 1000), tau), g, pool, cuda_device)

@@ -35,12 +35,14 @@ def _gen(wl, dev):
 
 def test_device_generator_matches_host(dev):
     import torch
-    for config in ("0", "2", "4"):
+    for config in ("0", "2", "2r", "4"):
         wl = W.make(config)
         gen = _gen(wl, dev)
         seqs = [0, wl.batch - 1]
         t0 = np.array([5, 1000], np.int32)
         cells = [0, wl.n_cells - 1]
+        if config == "2r":  # a residual cell: its tokens follow its reference's
+            cells[0] = int(np.nonzero(wl.kinds == W.RES2)[0][0])
         k, v = gen.kv(cells, seqs, t0, 40)
         kh = k.view(torch.int16).cpu().numpy().view(np.uint16)
         vh = v.view(torch.int16).cpu().numpy().view(np.uint16)
@@ -70,8 +72,9 @@ def _run_decode_only(config, pool, dev, cells=None, seqs=None, n_sample=16, spli
     wl = W.make(config)
     seqs = list(range(wl.batch)) if seqs is None else list(seqs)
     cells = list(range(wl.n_cells)) if cells is None else list(cells)
-    # SHARE cells need their source built as well
-    need = sorted(set(cells) | {wl.data_cell(c) for c in cells})
+    # SHARE and RES2 cells need the final loop's cell of their layer as well
+    need = sorted(set(cells) | {wl.source_cell(c) for c in cells
+                                if wl.kinds[c] in (W.SHARE, W.RES2)})
     lengths = wl.lengths[seqs]
     plan = GH.make_plan(wl, seqs)
     gen = _gen(wl, dev)
@@ -111,6 +114,12 @@ def test_config1_single_sequence(pool, dev):
 
 def test_config2_batched_16k(pool, dev):
     stats = _run_decode_only("2", pool, dev, n_sample=24)
+    assert max(s["max_abs"] for s in stats) < P.OUT_ABS_TOL
+
+
+def test_config2r_residual_cells_16k(pool, dev):
+    # the config-2 plan with its SHARE cells stored as 2-bit residuals
+    stats = _run_decode_only("2r", pool, dev, n_sample=24)
     assert max(s["max_abs"] for s in stats) < P.OUT_ABS_TOL
 
 

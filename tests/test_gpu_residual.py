@@ -1,0 +1,87 @@
+"""RES2 cells (2-bit residuals against the final loop's KV) on the CUDA path
+against the CPU oracle (needs a B200): cache bytes, outputs, masks and
+counts over every reference kind, group and window boundaries, serving-order
+appends, cluster splits, and the host checks on the reference."""
+
+import numpy as np
+import pytest
+
+from synth import workloads as W
+from tests import gpu_harness as GH
+from tests.test_gpu_edges import _check_spec, _spec
+
+pytestmark = pytest.mark.gpu
+
+Q4, Q2, SH, BF, RS = W.Q4, W.Q2, W.SHARE, W.BF16, W.RES2
+
+
+@pytest.fixture(scope="module")
+def pool():
+    from tests import parity as P
+    p = P.make_pool(8)
+    yield p
+    p.terminate()
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_residual_cells_match_oracle(pool, cuda_device, D):
+    # window edges: 63 / 64 / 65 tokens move the residual-coded count 0 -> 32
+    lengths = (1, 31, 63, 64, 65, 97, 200)
+    for kinds in ((RS, RS, Q4, Q2), (RS, Q4, BF, Q4), (RS, SH, Q4, Q2)):
+        _check_spec(_spec(D, kinds, lengths, 0.01), pool, cuda_device)
+
+
+@pytest.mark.parametrize("tau", [0.0, 2.0])
+def test_residual_tau_extremes(pool, cuda_device, tau):
+    _check_spec(_spec(128, (RS, RS, Q4, Q2), (40, 300, 1000), tau), pool, cuda_device)
+
+
+def test_residual_serving_order_appends(pool, cuda_device):
+    # one token per step for every cell, loop-major: each residual group is
+    # quantized one step after the reference holds it
+    _check_spec(_spec(64, (RS, RS, Q4, BF), (1, 31, 64, 70, 130), 0.02), pool, cuda_device,
+                token_by_token=True)
+
+
+@pytest.mark.parametrize("split", [2, 4])
+def test_residual_cluster_split(pool, cuda_device, split, monkeypatch):
+    monkeypatch.setenv("LOOPKV_DECODE_SPLIT", str(split))
+    _check_spec(_spec(128, (RS, Q2, Q4, Q4), (65, 700, 1500), 0.01), pool, cuda_device)
+
+
+def test_residual_append_needs_its_reference(cuda_device):
+    import torch
+    from loop_aware_quantized_b200 import LoopKVError, Plan
+    from synth.gpu import DeviceGenerator
+    wl = W.custom(2, 1, 2, 64, (RS, Q4), (300,), (320,), 0.01)
+    plan = Plan(2, 1, 2, 64, wl.capacity, wl.kinds, wl.tau)
+    gen = DeviceGenerator(wl, cuda_device)
+
+    def append(cell, t0, n):
+        k, v = gen.kv([cell], [0], np.array([t0], np.int32), n)
+        plan.append([cell], k, v)
+
+    with pytest.raises(LoopKVError):
+        append(0, 0, 100)           # the reference holds nothing yet
+    assert plan.lengths()[0, 0] == 0
+    append(0, 0, 63)                # nothing to quantize below 64 tokens
+    append(1, 0, 100)               # reference: 96 quantized positions
+    append(0, 63, 77)               # 140 tokens: 96 residual-coded
+    with pytest.raises(LoopKVError):
+        append(0, 140, 40)          # 180 tokens would need 160
+    assert plan.lengths()[0, 0] == 140
+    plan.check()
+    torch.cuda.synchronize()
+
+
+def test_residual_rollback_keeps_the_coded_range(pool, cuda_device):
+    import torch
+    from loop_aware_quantized_b200 import LoopKVError
+    spec = _spec(64, (RS, RS, Q4, Q2), (130, 150), 0.02)
+    plan = _check_spec(spec, pool, cuda_device)
+    # 130 and 150 tokens: 96 residual-coded; 129 keeps 96, 127 would drop to 64
+    with pytest.raises(LoopKVError):
+        plan.set_lengths([0], np.array([[127, 150]], np.int32))
+    plan.set_lengths([0], np.array([[129, 140]], np.int32))
+    assert list(plan.lengths()[0, :2]) == [129, 140]
+    torch.cuda.synchronize()
