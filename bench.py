@@ -84,11 +84,23 @@ def decode_bytes(wl, cells, lens_own, lens_src, nsel_total, g=1):
     bytes (bf16 residual and the SHARE current token at 4D bytes), read once
     for the g query heads of the group, the low-plane rows of the selected
     positions (D/4 each), the queries (2D each) and the outputs (4D each).
+    A RES2 unit reads its residual-coded positions twice over: the
+    reference's bytes plus its own 2-bit residual rows (D per token), and
+    its bf16 window at 4D per token.
     """
     D, H = wl.head_dim, wl.n_heads
     total = 0
     for c in cells:
         share = wl.kinds[c] == 2
+        if wl.kinds[c] == 4:
+            rk = int(wl.kinds[wl.source_cell(c)])
+            for n in lens_own:
+                n = int(n)
+                rt = (n // 32 - 1) * 32 if n >= 64 else 0
+                ref = rt * (4 * D if rk == 3 else per_token_head_bytes(rk, D))
+                tok = ref + rt * per_token_head_bytes(1, D) + (n - rt) * 4 * D
+                total += H * (tok + g * (2 * D + 4 * D))
+            continue
         dk = int(wl.kinds[wl.data_cell(c)])
         for b, n in enumerate(lens_own):
             n = int(n)
@@ -166,6 +178,8 @@ def workload_text(wl, B, g=1):
     k = wl.kinds
     plan = "plan %d Q4 / %d Q2 / %d SHARE / %d BF16 cells" % (
         (k == 0).sum(), (k == 1).sum(), (k == 2).sum(), (k == 3).sum())
+    if (k == 4).any():
+        plan += " / %d RES2 (2-bit residuals against the final loop)" % (k == 4).sum()
     ctx = ("%d cached tokens" % int(wl.lengths[0]) if len(set(wl.lengths[:B].tolist())) == 1
            else "ragged %d-%d cached tokens" % (int(wl.lengths[:B].min()), int(wl.lengths[:B].max())))
     heads = "%d KV heads" % wl.n_heads
@@ -233,7 +247,7 @@ def oracle_baseline(config, seconds, seqs_global, g=1):
     n = int(wl.lengths[0])
     rng = np.random.default_rng(0)
     picks = []
-    for kind in (0, 1, 2):
+    for kind in (0, 1, 2, 4):
         cs = [c for c in range(wl.n_cells) if wl.kinds[c] == kind]
         if cs:
             picks.append((int(rng.choice(cs)), int(rng.integers(wl.batch)),
@@ -257,6 +271,10 @@ def oracle_baseline(config, seconds, seqs_global, g=1):
             q = W.query_group(wl, c, b, h, n + 1, g)
         else:
             own.append(W.raw_keys(wl, c, b, h, 0, n + 1), W.raw_values(wl, c, b, h, 0, n + 1))
+            if kind == 4:  # the reference, one token behind in serving order
+                sc = wl.source_cell(c)
+                src = orc.OracleUnit(int(wl.kinds[sc]), wl.head_dim, cap)
+                src.append(W.raw_keys(wl, sc, b, h, 0, n), W.raw_values(wl, sc, b, h, 0, n))
             q = W.query_group(wl, c, b, h, n + 1, g)
         units.append((own, src, q))
     done = 0
@@ -269,7 +287,7 @@ def oracle_baseline(config, seconds, seqs_global, g=1):
         if el >= seconds:
             break
     rate_units = done / el
-    desc = ("%d oracle decodes of %d sampled units (Q4, Q2, SHARE; %d tokens each, "
+    desc = ("%d oracle decodes of %d sampled units (one per kind of the plan; %d tokens each, "
             "%d-token contexts%s) in %.1f s on 1 core; cell-steps/s = units/s / (%d seqs x %d "
             "heads)" % (done, len(units), n + 1, n + 1,
                         ", %d query heads per unit" % g if g > 1 else "", el, wl.batch,
@@ -354,9 +372,11 @@ def main():
     gen = DeviceGenerator(wl, dev)
 
     # build the cache: every token of every cell through the append kernel
+    # (the final loop first: RES2 cells quantize against it)
     t_build = time.perf_counter()
     kbuf = vbuf = None
-    for c in range(wl.n_cells):
+    final = list(range((wl.n_loops - 1) * wl.n_layers, wl.n_cells))
+    for c in final + [c for c in range(wl.n_cells) if c not in final]:
         kbuf, vbuf = gen.kv([c], seqs, np.zeros(B, np.int32), int(n0.max()), k=kbuf, v=vbuf)
         plan.append([c], kbuf, vbuf, n_new=n0)
     del kbuf, vbuf
@@ -425,7 +445,11 @@ def main():
     elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], world, dev)
     ms_per_step = elapsed_ms / args.steps
     value = wl.n_cells * world / (ms_per_step / 1000.0)
-    launches_per_step = 3 * len(phase)   # append + length commit + decode per phase
+    # per phase: an append and a decode launch for the plain cells and one
+    # each for RES2 cells (when the phase has them), and the length commit
+    launches_per_step = sum(1 + 2 * (int(any(wl.kinds[c] != 4 for c in cells)) +
+                                     int(any(wl.kinds[c] == 4 for c in cells)))
+                            for cells in phase)
 
     # ---- end to end through the API: pinned host inputs in, outputs out
     e2e = None
