@@ -27,9 +27,10 @@
  * LOOPKV_BF16 (raw bf16 cells) exists for ablations and checks.
  *
  * Residual cells.  "ResidualQuant: KV Cache Quantization for Looped
- * Transformers with 2-Bit Residuals", section 概要 (abstract): the final
- * loop's KV is a reference and the other loops keep low-precision residuals
- * against it.  A LOOPKV_RES2 cell (non-final loops only) stores, for each
+ * Transformers with 2-Bit Residuals", as summarised in the related-paper list
+ * (関連論文リスト) of the page "LoopVQ: Sub 1-bit KV Cache Quantization for
+ * Looped Transformers": the final loop's KV is a reference and the other
+ * loops keep low-precision residuals against it.  A LOOPKV_RES2 cell (non-final loops only) stores, for each
  * position t, d = fl32(x - r) quantized like a LOOPKV_Q2 cell, where x is
  * its own bf16 input and r the reference's stored value at t in fp32:
  * fl32(fl32(scale * q) + zero) with the full code q of a 4-bit or 2-bit

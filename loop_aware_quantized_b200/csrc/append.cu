@@ -275,10 +275,12 @@ __device__ float ref_value32(const uint8_t* rb, const UnitLayout& RL, int rkind,
   return __fadd_rn(__fmul_rn(m[0], (float)q), m[1]);
 }
 
-// Append to RES2 units ("ResidualQuant: KV Cache Quantization for Looped
-// Transformers with 2-Bit Residuals", section 概要: 2-bit residuals against
-// the final loop's KV).  One CTA per unit.  Tokens live in a 64-slot bf16
-// window (position t in slot t mod 64); residual group g is quantized when
+// Append to RES2 units (2-bit residuals against the final loop's KV:
+// "ResidualQuant: KV Cache Quantization for Looped Transformers with 2-Bit
+// Residuals", as summarised in the related-paper list (関連論文リスト) of the
+// page "LoopVQ: Sub 1-bit KV Cache Quantization for Looped Transformers").
+// One CTA per unit.  Tokens live in a 64-slot bf16 window (position t in
+// slot t mod 64); residual group g is quantized when
 // the unit reaches 32 (g + 2) tokens: each warp takes a group, forms the
 // residuals x - r in an fp32 tile (r: the reference's stored value, read
 // from its planes) and quantizes them at 2 bits exactly as a Q2 cell's

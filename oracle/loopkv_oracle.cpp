@@ -34,8 +34,10 @@
 //      and every head of the group reconstructs that token with it (the
 //      selection is the union over the group's heads).
 // "ResidualQuant: KV Cache Quantization for Looped Transformers with 2-Bit
-// Residuals", section 概要 (the abstract): the final loop's KV state is the
-// reference and the other loops keep low-precision residuals against it.
+// Residuals", as summarised in the related-paper list (関連論文リスト) of the
+// page "LoopVQ: Sub 1-bit KV Cache Quantization for Looped Transformers":
+// the final loop's KV state is the reference and the other loops keep
+// low-precision residuals against it.
 // Readings for that cell kind (RES2):
 //   R9  a RES2 cell sits in a non-final loop; its reference is the final
 //       loop's cell of the same layer, sequence and head, stored as 4-bit,

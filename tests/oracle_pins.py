@@ -461,8 +461,10 @@ def pin_mask_properties():
 
 # --------------------------------------------------------- residual (RES2) pins
 # "ResidualQuant: KV Cache Quantization for Looped Transformers with 2-Bit
-# Residuals", section 概要: the final loop's KV is the reference and the
-# other loops store 2-bit residuals against it.
+# Residuals", as summarised in the related-paper list (関連論文リスト) of the
+# page "LoopVQ: Sub 1-bit KV Cache Quantization for Looped Transformers": the
+# final loop's KV is the reference and the other loops store 2-bit
+# residuals against it.
 
 def pin_residual_deferred_window():
     # A residual group is quantized once the 32 tokens after it are in, so
