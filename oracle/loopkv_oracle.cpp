@@ -55,6 +55,20 @@
 //       reference's values through the tau rule of R4 with the cell's own
 //       weights), d^ = scale * code + zero of the residual; bf16 positions
 //       read the cell's own token.
+// "LoopVQ: Sub 1-bit KV Cache Quantization for Looped Transformers",
+// section 概要 (the abstract): a vector quantizer codes channels of several
+// loop steps jointly, at 0.5 bits per element, with codebooks fine-tuned
+// offline.  Readings for its decode (the codebooks are inputs here):
+//   V1  a sub-vector is c consecutive channels of one token (channels
+//       c*j .. c*j+c-1, group j) across the L loops of its layer, loop-major
+//       (element (l, i) at l*c + i); one byte indexes a 256-entry codebook,
+//       so L*c = 16 elements per byte is 0.5 bits per element at L = 4, c = 4;
+//   V2  one codebook per (layer, KV head) for keys and one for values,
+//       shared by the sequences and the channel groups, fp32 entries;
+//   V3  decoding loop l reads slice [l*c, l*c + c) of each indexed entry as
+//       the token's channels of group j; softmax attention as in R7;
+//   V4  every position of a unit is coded (the op attends over coded
+//       tokens only).
 // All attention arithmetic is fp64 (dequantized values, scores, softmax,
 // weighted sum).  Quantization is fp32 because the codes are defined by it.
 //
@@ -633,6 +647,48 @@ int orc_decode(const void* own_p, const void* src_p, const uint16_t* q,
                double* slack, double* weights) {
   return orc_decode_group(own_p, src_p, q, 1, tau, sm_scale, band, out, lse, mask,
                           n_mask_words, nsel, slack, weights);
+}
+
+// ---- LoopVQ decode ----------------------------------------------------------
+// One unit, one loop (V1-V4).  idx_k, idx_v: [n][D/c] codebook indices;
+// cb_k, cb_v: [256][L*c] entries; q: bf16 bits [D]; sm_scale <= 0 means
+// 1/sqrt(D).  out[D] (fp64) and *lse (natural log).  Returns 0, or -1 on
+// invalid sizes (n < 1, loop outside [0, L), c not dividing D).
+int orc_vq_decode(int n_loops, int D, int c, int n, int loop, const uint8_t* idx_k,
+                  const uint8_t* idx_v, const float* cb_k, const float* cb_v, const uint16_t* q,
+                  double sm_scale, double* out, double* lse) {
+  if (n < 1 || n_loops < 1 || loop < 0 || loop >= n_loops || c < 1 || D % c != 0) return -1;
+  if (sm_scale <= 0.0) sm_scale = 1.0 / std::sqrt(static_cast<double>(D));
+  const int groups = D / c, width = n_loops * c;
+  // the loop's channels of an indexed entry (V1, V3)
+  auto entry = [&](const float* cb, int e, int d) {
+    const int i = d % c;
+    return static_cast<double>(cb[static_cast<size_t>(e) * width + loop * c + i]);
+  };
+  std::vector<double> s(n);
+  double smax = -INFINITY;
+  for (int t = 0; t < n; ++t) {
+    double acc = 0.0;
+    for (int d = 0; d < D; ++d) {
+      const int e = idx_k[static_cast<size_t>(t) * groups + d / c];
+      acc += static_cast<double>(bf16_to_float(q[d])) * entry(cb_k, e, d);
+    }
+    s[t] = sm_scale * acc;
+    smax = std::max(smax, s[t]);
+  }
+  double sum = 0.0;
+  for (int t = 0; t < n; ++t) sum += std::exp(s[t] - smax);
+  const double l = smax + std::log(sum);
+  *lse = l;
+  for (int d = 0; d < D; ++d) out[d] = 0.0;
+  for (int t = 0; t < n; ++t) {
+    const double p = std::exp(s[t] - l);
+    for (int d = 0; d < D; ++d) {
+      const int e = idx_v[static_cast<size_t>(t) * groups + d / c];
+      out[d] += p * entry(cb_v, e, d);
+    }
+  }
+  return 0;
 }
 
 // ---- planner ---------------------------------------------------------------

@@ -46,6 +46,9 @@ def _load():
     lib.orc_decode_group.argtypes = [P, P, P, ctypes.c_int, ctypes.c_double, ctypes.c_double,
                                      ctypes.c_double, P, P, P, P, P, P, P]
     lib.orc_decode_group.restype = ctypes.c_int
+    lib.orc_vq_decode.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_int, P, P, P, P, P, ctypes.c_double, P, P]
+    lib.orc_vq_decode.restype = ctypes.c_int
     lib.orc_plan_brute.argtypes = [ctypes.c_int, ctypes.c_int, P, ctypes.c_int64, ctypes.c_int64,
                                    ctypes.c_int, P, P, P, P]
     lib.orc_plan_brute.restype = ctypes.c_int
@@ -225,3 +228,24 @@ def plan_brute(n_loops, n_layers, damage, damage_budget, storage_budget_q, sel_m
     if rc != 0:
         return None
     return kinds, int(r[0]), int(d[0]), int(s[0])
+
+
+def vq_decode(idx_k, idx_v, cb_k, cb_v, q_bits, loop, n_loops, sm_scale=0.0):
+    """LoopVQ decode of one unit for one loop: idx_k / idx_v u8 [n, D/c],
+    cb_k / cb_v fp32 [256, n_loops * c], q bf16 bits [D] -> (out fp64 [D], lse)."""
+    idx_k = np.ascontiguousarray(idx_k, dtype=np.uint8)
+    idx_v = np.ascontiguousarray(idx_v, dtype=np.uint8)
+    cb_k = np.ascontiguousarray(cb_k, dtype=np.float32)
+    cb_v = np.ascontiguousarray(cb_v, dtype=np.float32)
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16).reshape(-1)
+    n, groups = idx_k.shape
+    D = q.size
+    c = D // groups
+    assert idx_v.shape == idx_k.shape and cb_k.shape == (256, n_loops * c) == cb_v.shape
+    out = np.zeros(D, np.float64)
+    lse = np.zeros(1, np.float64)
+    rc = _load().orc_vq_decode(n_loops, D, c, n, int(loop), _ptr(idx_k), _ptr(idx_v), _ptr(cb_k),
+                               _ptr(cb_v), _ptr(q), float(sm_scale), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle vq decode rejected its input")
+    return out, float(lse[0])

@@ -611,6 +611,65 @@ def pin_residual_reference_checks():
         raise AssertionError("residual unit accepted a bad reference")
 
 
+# ------------------------------------------------------------ LoopVQ pins
+# "LoopVQ: Sub 1-bit KV Cache Quantization for Looped Transformers", section
+# 概要: channels of several loop steps are coded jointly by a codebook.
+
+def _vq_exact(D, L, c, n, seed):
+    """A codebook that holds every (token, group) sub-vector of raw per-loop
+    keys and values exactly, and the indices that pick them."""
+    groups = D // c
+    assert n * groups == 256
+    K = f32(rng_bits(seed, (L, n, D)))
+    V = f32(rng_bits(seed + 1, (L, n, D)))
+    perm = np.argsort(f32(rng_bits(seed + 2, (256,))), kind="stable")  # a shuffle of the entries
+    cb_k = np.zeros((256, L * c), np.float32)
+    cb_v = np.zeros((256, L * c), np.float32)
+    idx_k = np.zeros((n, groups), np.uint8)
+    idx_v = np.zeros((n, groups), np.uint8)
+    for t in range(n):
+        for j in range(groups):
+            e, ev = t * groups + j, int(perm[t * groups + j])
+            idx_k[t, j], idx_v[t, j] = e, ev
+            for l in range(L):
+                cb_k[e, l * c:(l + 1) * c] = K[l, t, j * c:(j + 1) * c]
+                cb_v[ev, l * c:(l + 1) * c] = V[l, t, j * c:(j + 1) * c]
+    return K, V, cb_k, cb_v, idx_k, idx_v
+
+
+def pin_vq_exact_codebook():
+    # With a codebook that holds each sub-vector exactly, decoding loop l is
+    # textbook attention over loop l's raw keys and values (every loop, two
+    # head dims, values indexed through a shuffled codebook).
+    for D, L, c, n in ((64, 4, 4, 16), (128, 2, 8, 16)):
+        K, V, cb_k, cb_v, idx_k, idx_v = _vq_exact(D, L, c, n, 400 + D)
+        q = rng_bits(401 + D, (D,), 2.0)
+        for loop in range(L):
+            out, lse = orc.vq_decode(idx_k, idx_v, cb_k, cb_v, q, loop, L)
+            want = sdpa(f32(q), K[loop].astype(np.float64), V[loop].astype(np.float64),
+                        1 / np.sqrt(D))
+            assert np.abs(out - want).max() < 1e-12, (D, loop, np.abs(out - want).max())
+
+
+def pin_vq_uniform_keys():
+    # Every key entry reads the same vector at loop 2: all scores equal, so
+    # lse = s + ln n and the output is the plain mean of the value slices.
+    D, L, c, n = 64, 4, 4, 40
+    rng = np.random.default_rng(5)
+    cb_k = rng.standard_normal((256, L * c)).astype(np.float32)
+    kvec = rng.standard_normal(c).astype(np.float32)
+    cb_k[:, 2 * c:3 * c] = kvec
+    cb_v = rng.standard_normal((256, L * c)).astype(np.float32)
+    idx_k = rng.integers(0, 256, (n, D // c)).astype(np.uint8)
+    idx_v = rng.integers(0, 256, (n, D // c)).astype(np.uint8)
+    q = rng_bits(410, (D,), 1.0)
+    out, lse = orc.vq_decode(idx_k, idx_v, cb_k, cb_v, q, 2, L)
+    s = float(np.dot(f32(q).astype(np.float64), np.tile(kvec.astype(np.float64), D // c))) / np.sqrt(D)
+    assert abs(lse - (s + np.log(n))) < 1e-12
+    vals = cb_v[idx_v][:, :, 2 * c:3 * c].reshape(n, D).astype(np.float64)
+    assert np.abs(out - vals.mean(axis=0)).max() < 1e-12
+
+
 ALL_PINS = [
     pin_quantize_q2_ties,
     pin_quantize_q4_ties,
@@ -633,4 +692,6 @@ ALL_PINS = [
     pin_residual_worked_example,
     pin_residual_reconstructs,
     pin_residual_reference_checks,
+    pin_vq_exact_codebook,
+    pin_vq_uniform_keys,
 ]

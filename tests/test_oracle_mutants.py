@@ -61,6 +61,12 @@ MUTANTS = [
      "khat[d] += 0.0 * static_cast<double>(rs.ks[gr * D + d])"),
     ("value residual codes dropped", "v += static_cast<double>(rs.vs[j])",
      "v += 0.0 * static_cast<double>(rs.vs[j])"),
+    ("vq loop slice interleaved", "cb[static_cast<size_t>(e) * width + loop * c + i]",
+     "cb[static_cast<size_t>(e) * width + i * n_loops + loop]"),
+    ("vq values read the key indices", "const int e = idx_v[static_cast<size_t>(t) * groups + d / c];",
+     "const int e = idx_k[static_cast<size_t>(t) * groups + d / c];"),
+    ("vq group of a channel", "const int e = idx_k[static_cast<size_t>(t) * groups + d / c];",
+     "const int e = idx_k[static_cast<size_t>(t) * groups + d % groups];"),
     ("residual window slot not modulo 64",
      "const size_t slot = static_cast<size_t>(t % kResWindow) * D * 2;",
      "const size_t slot = static_cast<size_t>(t - u->qtok()) * D * 2;"),
