@@ -295,6 +295,49 @@ typedef struct {
 loopkv_status loopkv_plan_optimize(const loopkv_planner_desc* desc, uint8_t* kinds_out,
                                    loopkv_plan_cost* cost);
 
+/* ---- LoopVQ decode --------------------------------------------------------
+ * "LoopVQ: Sub 1-bit KV Cache Quantization for Looped Transformers", section
+ * 概要 (abstract): a vector quantizer codes channels of several loop steps
+ * jointly (0.5 bits per element), with codebooks fine-tuned offline.  The
+ * abstract fixes no format; this library reads it as follows (the CPU
+ * oracle takes the same readings):
+ *   - a sub-vector is 4 consecutive channels of one token (group j: channels
+ *     4j .. 4j+3) across the n_loops loops of its layer, loop-major (element
+ *     (l, i) at 4l + i); one byte indexes a 256-entry codebook, so one byte
+ *     codes 4 * n_loops elements (0.5 bits per element at 4 loops);
+ *   - one key codebook and one value codebook per (layer, KV head), fp32
+ *     entries [256][4 * n_loops], shared by sequences and channel groups
+ *     (trained offline: inputs here);
+ *   - decoding loop l reads slice [4l, 4l + 4) of each indexed entry as the
+ *     token's channels of group j; scores sm_scale * <q, k>, softmax, and
+ *     out = sum_t p_t v_t in fp32;
+ *   - every position [0, len[b]) of a unit is coded.
+ * Shapes: idx_k, idx_v uint8 [n_layers][batch][n_kv_heads][capacity][D/4]
+ * (a token's D/4 indices contiguous); cb_k, cb_v fp32
+ * [n_layers][n_kv_heads][256][4 * n_loops]; q bf16 [n_layers][batch]
+ * [n_kv_heads][D]; out fp32, same shape; lse fp32 [n_layers][batch]
+ * [n_kv_heads] (natural log) or NULL.  All device pointers 16-byte aligned;
+ * the caller owns them. */
+typedef struct {
+  int32_t n_loops;     /* loops coded jointly, 1 .. 8 */
+  int32_t n_layers;    /* layers decoded by one call, >= 1 */
+  int32_t n_kv_heads;  /* >= 1 */
+  int32_t head_dim;    /* 64 or 128 */
+  int32_t batch;       /* sequences, 1 .. LOOPKV_MAX_BATCH */
+  int32_t capacity;    /* token stride of the index arrays, 1 .. 2^20 */
+  float sm_scale;      /* <= 0 means 1/sqrt(head_dim) */
+} loopkv_vq_desc;
+
+/* Decode loop `loop` (0 .. n_loops-1) of every (layer, sequence, KV head)
+ * over positions [0, h_len[b]) (host [batch], each 1 .. capacity).  Enqueued
+ * on `stream`.  Errors (nothing launched): LOOPKV_ERR_INVALID_ARG (null or
+ * misaligned pointers, sizes out of range), LOOPKV_ERR_UNSUPPORTED (a
+ * sequence longer than 8 CTAs of score slots), LOOPKV_ERR_CUDA. */
+loopkv_status loopkv_vq_decode(const loopkv_vq_desc* desc, int32_t loop, const int32_t* h_len,
+                               const uint8_t* d_idx_k, const uint8_t* d_idx_v,
+                               const float* d_cb_k, const float* d_cb_v, const uint16_t* d_q,
+                               float* d_out, float* d_lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,327 @@
+// LoopVQ decode for sm_100a: attention over a KV cache coded by cross-loop
+// codebooks.
+//
+// "LoopVQ: Sub 1-bit KV Cache Quantization for Looped Transformers",
+// section 概要: a vector quantizer codes channels of several loop steps
+// jointly at 0.5 bits per element.  Here one byte indexes a 256-entry
+// codebook whose entries hold 4 channels of a token across the L loops of
+// its layer (loop-major); decoding loop l reads slice [4l, 4l + 4) of each
+// indexed entry (the format is spelled out in include/loopkv.h).
+//
+// One CTA (8 warps) per (layer, sequence, KV head, split); splits of a long
+// sequence form a thread-block cluster and merge through DSMEM.
+//   table   per channel group j and entry e, LUT[j][e] = <q_j, entry_e's
+//           loop slice> (the query is folded into the codebook once, so a
+//           token's score is D/4 shared-memory lookups and adds);
+//   pass 1  lane = token: its D/4 key indices (one 16-byte load per 16
+//           groups), score = sum_j LUT[j][idx_j], kept in shared memory
+//           (log2 units);
+//   softmax the CTA's max and sum of exponentials, merged over the cluster;
+//   pass 2  lane = token: p_t added into W[j][idx_v_j] (a weight histogram
+//           over the value codebook, shared-memory atomics);
+//   output  out[4j + i] = sum_e W[j][e] * entry_e[4l + i].
+// The index streams are read once (D/2 bytes per token at D = 128: 32 key
+// and 32 value bytes); the work per token is D/2 random shared-memory
+// accesses, so the kernel is bound by shared-memory bank conflicts of those
+// lookups rather than by HBM.
+
+#include <cooperative_groups.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "loopkv_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace loopkv {
+namespace {
+
+constexpr int kVqThreads = 256;
+constexpr int kVqWarps = kVqThreads / 32;
+constexpr int kVqSub = 4;        // channels per sub-vector
+constexpr int kEntries = 256;    // codebook entries (one byte)
+constexpr int kRow = kEntries + 1;  // padded table row: group j's row starts in bank j
+constexpr int kVqSlots = 8192;   // score slots per CTA (two CTAs per SM)
+constexpr int kVqMaxSplit = 8;   // portable cluster size
+
+struct VqParams {
+  const uint8_t* idx_k;
+  const uint8_t* idx_v;
+  const float* cb_k;
+  const float* cb_v;
+  const uint16_t* q;
+  float* out;
+  float* lse;
+  int32_t batch, H, L, cap, loop, split;
+  float score_scale;  // sm_scale * log2(e)
+  int32_t len[LOOPKV_MAX_BATCH];
+};
+
+__device__ __forceinline__ uint4 ld_idx(const uint8_t* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// The D/4 indices of a token as D/16 words (index 4k + m in byte m of word k).
+template <int D>
+__device__ __forceinline__ void load_indices(uint32_t (&w)[D / 16], const uint8_t* row) {
+#pragma unroll
+  for (int k = 0; k < D / 64; ++k) {
+    const uint4 x = ld_idx(row + 16 * k);
+    w[4 * k] = x.x;
+    w[4 * k + 1] = x.y;
+    w[4 * k + 2] = x.z;
+    w[4 * k + 3] = x.w;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kVqThreads, 2)
+vq_decode_kernel(const VqParams p) {
+  constexpr int GR = D / kVqSub;  // channel groups
+  extern __shared__ __align__(16) float sm[];
+  float* lut = sm;                 // [GR][kRow]
+  float* wv = lut + GR * kRow;     // [GR][kRow]
+  float* q_s = wv + GR * kRow;     // [D]
+  float* misc = q_s + D;           // [64]
+  float* sc = misc + 64;           // [kVqSlots]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = p.split;
+  const int rank = blockIdx.x % split;
+  const int unit = blockIdx.x / split;
+  const int h = unit % p.H;
+  const int b = (unit / p.H) % p.batch;
+  const int layer = unit / (p.H * p.batch);
+  const int n = p.len[b];
+  const int chunk = ((n + split - 1) / split + 31) / 32 * 32;  // <= kVqSlots (host check)
+  const int p0 = rank * chunk;
+  const int p1 = min(n, p0 + chunk);
+  const size_t uidx = ((size_t)layer * p.batch + b) * p.H + h;
+  const int W = p.L * kVqSub;  // floats per codebook entry
+  const size_t cbo = ((size_t)layer * p.H + h) * kEntries * W + (size_t)p.loop * kVqSub;
+  const float* cbk = p.cb_k + cbo;
+  const float* cbv = p.cb_v + cbo;
+
+  for (int d = tid; d < D; d += kVqThreads) q_s[d] = __uint_as_float((uint32_t)p.q[uidx * D + d] << 16);
+  for (int i = tid; i < GR * kRow; i += kVqThreads) wv[i] = 0.f;
+  __syncthreads();
+  // LUT[j][e] = sum_i q[4j + i] * entry_e[4 loop + i] (thread = entry)
+  for (int i = tid; i < GR * kEntries; i += kVqThreads) {
+    const int j = i / kEntries, e = i % kEntries;
+    const float4 c4 = __ldg(reinterpret_cast<const float4*>(cbk + (size_t)e * W));
+    const float* qq = q_s + kVqSub * j;
+    float a = qq[0] * c4.x;
+    a = fmaf(qq[1], c4.y, a);
+    a = fmaf(qq[2], c4.z, a);
+    a = fmaf(qq[3], c4.w, a);
+    lut[j * kRow + e] = a;
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- pass 1
+  const uint8_t* ik = p.idx_k + uidx * (size_t)p.cap * GR;
+  float lmax = -INFINITY;
+  for (int base = p0 + 32 * warp; base < p1; base += 32 * kVqWarps) {
+    const int t = base + lane;
+    if (t < p1) {
+      uint32_t w[D / 16];
+      load_indices<D>(w, ik + (size_t)t * GR);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t x = w[k];
+        a0 += lut[(4 * k) * kRow + (x & 255u)];
+        a1 += lut[(4 * k + 1) * kRow + ((x >> 8) & 255u)];
+        a2 += lut[(4 * k + 2) * kRow + ((x >> 16) & 255u)];
+        a3 += lut[(4 * k + 3) * kRow + (x >> 24)];
+      }
+      const float s = ((a0 + a1) + (a2 + a3)) * p.score_scale;
+      sc[t - p0] = s;
+      lmax = fmaxf(lmax, s);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+  if (lane == 0) misc[warp] = lmax;
+  __syncthreads();
+  float m = misc[0];
+#pragma unroll
+  for (int k = 1; k < kVqWarps; ++k) m = fmaxf(m, misc[k]);
+  float ls = 0.f;
+  for (int i = tid; i < p1 - p0; i += kVqThreads) ls += exp2f(sc[i] - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  if (lane == 0) misc[8 + warp] = ls;
+  __syncthreads();
+  float l = 0.f;
+#pragma unroll
+  for (int k = 0; k < kVqWarps; ++k) l += misc[8 + k];
+  if (p1 <= p0) {
+    m = -INFINITY;
+    l = 0.f;
+  }
+  float M = m, Lt = l;
+  if (split > 1) {
+    cg::cluster_group cluster = cg::this_cluster();
+    if (tid == 0) {
+      misc[32] = m;
+      misc[33] = l;
+    }
+    cluster.sync();
+    M = -INFINITY;
+    for (int k = 0; k < split; ++k) M = fmaxf(M, cluster.map_shared_rank(misc, k)[32]);
+    Lt = 0.f;
+    for (int k = 0; k < split; ++k) {
+      const float* rm = cluster.map_shared_rank(misc, k);
+      if (rm[33] > 0.f) Lt += rm[33] * exp2f(rm[32] - M);
+    }
+  }
+  const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+
+  // ---------------------------------------------------------------- pass 2
+  const uint8_t* iv = p.idx_v + uidx * (size_t)p.cap * GR;
+  for (int base = p0 + 32 * warp; base < p1; base += 32 * kVqWarps) {
+    const int t = base + lane;
+    if (t < p1) {
+      const float pw = exp2f(sc[t - p0] - M) * inv;
+      uint32_t w[D / 16];
+      load_indices<D>(w, iv + (size_t)t * GR);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t x = w[k];
+        atomicAdd(&wv[(4 * k) * kRow + (x & 255u)], pw);
+        atomicAdd(&wv[(4 * k + 1) * kRow + ((x >> 8) & 255u)], pw);
+        atomicAdd(&wv[(4 * k + 2) * kRow + ((x >> 16) & 255u)], pw);
+        atomicAdd(&wv[(4 * k + 3) * kRow + (x >> 24)], pw);
+      }
+    }
+  }
+  __syncthreads();
+  // out[4j + i] = sum_e W[j][e] * entry_e[4 loop + i]: PARTS threads per
+  // channel split the entries; the table's rows are free now
+  constexpr int PARTS = kVqThreads / D;
+  {
+    const int d = tid % D, part = tid / D, j = d / kVqSub, i = d % kVqSub;
+    float o = 0.f;
+    for (int e = part; e < kEntries; e += PARTS) o = fmaf(wv[j * kRow + e], __ldg(cbv + (size_t)e * W + i), o);
+    lut[tid] = o;
+  }
+  __syncthreads();
+  if (tid < D) {
+    float o = 0.f;
+#pragma unroll
+    for (int k = 0; k < PARTS; ++k) o += lut[k * D + tid];
+    q_s[tid] = o;  // the query is no longer needed
+  }
+  __syncthreads();
+
+  if (split > 1) {
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    if (rank == 0) {
+      for (int d = tid; d < D; d += kVqThreads) {
+        float o = 0.f;
+        for (int k = 0; k < split; ++k) o += cluster.map_shared_rank(q_s, k)[d];
+        p.out[uidx * D + d] = o;
+      }
+      if (tid == 0 && p.lse) p.lse[uidx] = (M + log2f(Lt)) * 0.69314718055994531f;
+    }
+    cluster.sync();  // every CTA's shared memory stays alive until rank 0 has read it
+  } else {
+    for (int d = tid; d < D; d += kVqThreads) p.out[uidx * D + d] = q_s[d];
+    if (tid == 0 && p.lse) p.lse[uidx] = (M + log2f(Lt)) * 0.69314718055994531f;
+  }
+}
+
+template <int D>
+constexpr size_t vq_smem() {
+  return sizeof(float) * ((size_t)2 * (D / kVqSub) * kRow + D + 64 + kVqSlots);
+}
+
+template <int D>
+int launch_vq_t(const VqParams& p, long long units, cudaStream_t stream) {
+  const size_t smem = vq_smem<D>();
+  cudaError_t e = cudaFuncSetAttribute(vq_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return (int)e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(units * p.split), 1, 1);
+  cfg.blockDim = dim3(kVqThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  int nattr = 0;
+  if (p.split > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    nattr = 1;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = nattr;
+  return (int)cudaLaunchKernelEx(&cfg, vq_decode_kernel<D>, p);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace loopkv
+
+using namespace loopkv;
+
+extern "C" loopkv_status loopkv_vq_decode(const loopkv_vq_desc* d, int32_t loop, const int32_t* h_len,
+                                          const uint8_t* d_idx_k, const uint8_t* d_idx_v,
+                                          const float* d_cb_k, const float* d_cb_v,
+                                          const uint16_t* d_q, float* d_out, float* d_lse,
+                                          void* stream) {
+  if (d == nullptr || h_len == nullptr) return LOOPKV_ERR_INVALID_ARG;
+  if (d->n_loops < 1 || d->n_loops > 8 || d->n_layers < 1 || d->n_kv_heads < 1 ||
+      d->n_kv_heads > (1 << 16) || (d->head_dim != 64 && d->head_dim != 128) || d->batch < 1 ||
+      d->batch > LOOPKV_MAX_BATCH || d->capacity < 1 || d->capacity > (1 << 20) ||
+      !std::isfinite(d->sm_scale))
+    return LOOPKV_ERR_INVALID_ARG;
+  if (loop < 0 || loop >= d->n_loops) return LOOPKV_ERR_INVALID_ARG;
+  const void* ptrs[7] = {d_idx_k, d_idx_v, d_cb_k, d_cb_v, d_q, d_out, nullptr};
+  for (int i = 0; i < 6; ++i)
+    if (ptrs[i] == nullptr || !aligned16(ptrs[i])) return LOOPKV_ERR_INVALID_ARG;
+  if (d_lse != nullptr && (reinterpret_cast<uintptr_t>(d_lse) & 3u) != 0) return LOOPKV_ERR_INVALID_ARG;
+  VqParams p{};
+  int nmax = 0;
+  for (int b = 0; b < d->batch; ++b) {
+    if (h_len[b] < 1 || h_len[b] > d->capacity) return LOOPKV_ERR_INVALID_ARG;
+    p.len[b] = h_len[b];
+    nmax = h_len[b] > nmax ? h_len[b] : nmax;
+  }
+  const long long units = (long long)d->n_layers * d->batch * d->n_kv_heads;
+  auto slots_for = [&](int s) { return ((nmax + s - 1) / s + 31) / 32 * 32; };
+  int split = 1;
+  while (slots_for(split) > kVqSlots && split < kVqMaxSplit) split *= 2;
+  if (slots_for(split) > kVqSlots) return LOOPKV_ERR_UNSUPPORTED;
+  while (units * split < 148 * 4 && split < kVqMaxSplit && nmax / (2 * split) >= 512) split *= 2;
+  if (units * split >= (1LL << 31)) return LOOPKV_ERR_UNSUPPORTED;
+  p.idx_k = d_idx_k;
+  p.idx_v = d_idx_v;
+  p.cb_k = d_cb_k;
+  p.cb_v = d_cb_v;
+  p.q = d_q;
+  p.out = d_out;
+  p.lse = d_lse;
+  p.batch = d->batch;
+  p.H = d->n_kv_heads;
+  p.L = d->n_loops;
+  p.cap = d->capacity;
+  p.loop = loop;
+  p.split = split;
+  const float sm_scale = d->sm_scale > 0.f ? d->sm_scale : 1.0f / std::sqrt((float)d->head_dim);
+  p.score_scale = sm_scale * 1.4426950408889634f;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int e = d->head_dim == 64 ? launch_vq_t<64>(p, units, s) : launch_vq_t<128>(p, units, s);
+  return e == 0 ? LOOPKV_OK : LOOPKV_ERR_CUDA;
+}

@@ -72,6 +72,18 @@ class loopkv_plan_cost(ctypes.Structure):
     _fields_ = [("reads", ctypes.c_double), ("damage", ctypes.c_int64), ("storage", ctypes.c_int64)]
 
 
+class loopkv_vq_desc(ctypes.Structure):
+    _fields_ = [
+        ("n_loops", ctypes.c_int32),
+        ("n_layers", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("batch", ctypes.c_int32),
+        ("capacity", ctypes.c_int32),
+        ("sm_scale", ctypes.c_float),
+    ]
+
+
 class loopkv_sizes(ctypes.Structure):
     _fields_ = [("table_bytes", ctypes.c_size_t), ("cache_bytes", ctypes.c_size_t)]
 
@@ -100,6 +112,8 @@ def _load():
         "loopkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "loopkv_plan_optimize": (st, [ctypes.POINTER(loopkv_planner_desc), P,
                                       ctypes.POINTER(loopkv_plan_cost)]),
+        "loopkv_vq_decode": (st, [ctypes.POINTER(loopkv_vq_desc), I32, P, P, P, P, P, P, P, P,
+                                  P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -143,6 +157,13 @@ def loopkv_decode(handle, h_cells, n_cells, batch, d_q, d_out, d_lse, d_mask, ma
                   d_nsel, stream):
     return _lib.loopkv_decode(handle, h_cells, n_cells, batch, d_q, d_out, d_lse, d_mask,
                               mask_words, d_nsel, stream)
+
+
+def loopkv_vq_decode(desc, loop, h_len, d_idx_k, d_idx_v, d_cb_k, d_cb_v, d_q, d_out, d_lse,
+                     stream):
+    ref = None if desc is None else ctypes.byref(desc)
+    return _lib.loopkv_vq_decode(ref, loop, h_len, d_idx_k, d_idx_v, d_cb_k, d_cb_v, d_q, d_out,
+                                 d_lse, stream)
 
 
 def loopkv_plan_optimize(desc, kinds_out):
@@ -341,3 +362,31 @@ def plan_optimize(n_loops, n_layers, head_dim, damage, damage_budget, storage_bu
     rc, cost = loopkv_plan_optimize(d, _np_ptr(kinds))
     _check(rc, "loopkv_plan_optimize")
     return kinds, {"reads": cost.reads, "damage": int(cost.damage), "storage": int(cost.storage)}
+
+
+def vq_decode(loop, lengths, idx_k, idx_v, cb_k, cb_v, q, out=None, lse=None, sm_scale=0.0,
+              stream=None):
+    """LoopVQ decode of loop ``loop`` for every (layer, sequence, KV head).
+
+    idx_k / idx_v: uint8 [n_layers, batch, H, capacity, D/4]; cb_k / cb_v:
+    fp32 [n_layers, H, 256, 4 * n_loops]; q: bf16 [n_layers, batch, H, D];
+    lengths: host [batch] coded tokens.  Returns out (fp32, q's shape)."""
+    import torch
+    assert idx_k.dtype == torch.uint8 and idx_v.shape == idx_k.shape
+    assert cb_k.dtype == torch.float32 and cb_v.shape == cb_k.shape
+    assert q.dtype == torch.bfloat16
+    for t in (idx_k, idx_v, cb_k, cb_v, q):
+        assert t.is_contiguous()
+    n_layers, batch, H, cap, groups = idx_k.shape
+    D = q.shape[-1]
+    assert groups * 4 == D and q.shape == (n_layers, batch, H, D)
+    assert cb_k.shape[:3] == (n_layers, H, 256) and cb_k.shape[3] % 4 == 0
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    d = loopkv_vq_desc(cb_k.shape[3] // 4, n_layers, H, D, batch, cap, float(sm_scale))
+    lengths = np.ascontiguousarray(lengths, dtype=np.int32)
+    assert lengths.size == batch
+    rc = loopkv_vq_decode(d, int(loop), _np_ptr(lengths), _ptr(idx_k), _ptr(idx_v), _ptr(cb_k),
+                          _ptr(cb_v), _ptr(q), _ptr(out), _ptr(lse), _stream_handle(stream))
+    _check(rc, "loopkv_vq_decode")
+    return out

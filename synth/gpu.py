@@ -30,6 +30,10 @@ def _load():
         lib.synth_gen_q.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, ctypes.c_uint32,
                                     ctypes.c_float, P]
         lib.synth_gen_q.restype = I
+        lib.synth_gen_vq_idx.argtypes = [P, I, I, I, I, I, I, I, ctypes.c_uint32, P]
+        lib.synth_gen_vq_idx.restype = I
+        lib.synth_gen_vq_q.argtypes = [P, I, I, I, I, I, ctypes.c_uint32, ctypes.c_float, P]
+        lib.synth_gen_vq_q.restype = I
         _lib = lib
     return _lib
 
@@ -102,3 +106,51 @@ class DeviceGenerator:
 def host_kv(wl, cell, b, h, t0, t1):
     """Host twin: (keys, values) bf16 bits [t1 - t0, D]."""
     return W.raw_keys(wl, cell, b, h, t0, t1), W.raw_values(wl, cell, b, h, t0, t1)
+
+
+class VqDeviceGenerator:
+    """LoopVQ inputs on a CUDA device (same bits as the host generator)."""
+
+    def __init__(self, wl, device="cuda"):
+        import torch
+        self.wl = wl
+        self.device = torch.device(device)
+        self.nscale = float(px.NORMAL_SCALE)
+
+    def indices(self, which, T=None, out=None):
+        """uint8 [n_layers, batch, H, capacity, D/4]; tokens < T filled."""
+        import torch
+        wl = self.wl
+        T = wl.capacity if T is None else T
+        shape = (wl.n_layers, wl.batch, wl.n_heads, wl.capacity, wl.head_dim // 4)
+        if out is None:
+            out = torch.zeros(shape, dtype=torch.uint8, device=self.device)
+        s = torch.cuda.current_stream()
+        rc = _load().synth_gen_vq_idx(_p(out), wl.n_layers, wl.batch, wl.n_heads, wl.head_dim,
+                                      wl.capacity, int(T), int(which), wl.seed,
+                                      ctypes.c_void_p(s.cuda_stream))
+        s.synchronize()
+        assert rc == 0, rc
+        return out
+
+    def codebooks(self, which):
+        """fp32 [n_layers, H, 256, 4 * n_loops] from the host generator (small)."""
+        import torch
+        wl = self.wl
+        cb = np.stack([np.stack([W.vq_codebook(wl, which, layer, h) for h in range(wl.n_heads)])
+                       for layer in range(wl.n_layers)])
+        return torch.from_numpy(np.ascontiguousarray(cb)).to(self.device)
+
+    def queries(self, loop, out=None):
+        """bf16 [n_layers, batch, H, D] of one loop."""
+        import torch
+        wl = self.wl
+        shape = (wl.n_layers, wl.batch, wl.n_heads, wl.head_dim)
+        if out is None:
+            out = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+        s = torch.cuda.current_stream()
+        rc = _load().synth_gen_vq_q(_p(out), wl.n_layers, wl.batch, wl.n_heads, wl.head_dim,
+                                    int(loop), wl.seed, self.nscale, ctypes.c_void_p(s.cuda_stream))
+        s.synchronize()
+        assert rc == 0, rc
+        return out

@@ -41,6 +41,7 @@ KIND_NAMES = {Q4: "Q4", Q2: "Q2", SHARE: "SHARE", BF16: "BF16", RES2: "RES2"}
 # Philox key word 1 selects the stream; key word 0 is the workload seed.
 STREAM_K, STREAM_V, STREAM_QNOISE, STREAM_QPOS = 1, 2, 3, 4
 STREAM_CHSCALE, STREAM_PLAN, STREAM_LEN, STREAM_OUTLIER = 5, 6, 7, 8
+STREAM_VQ_IDX, STREAM_VQ_CB, STREAM_VQ_Q = 9, 10, 11
 
 
 @dataclasses.dataclass
@@ -304,3 +305,70 @@ def custom(n_loops, n_layers, n_heads, head_dim, kinds, lengths, capacity, tau, 
     return Workload("custom", n_loops, n_layers, n_heads, head_dim, len(lengths), seed,
                     np.array(kinds, np.uint8), float(tau), np.array(lengths, np.int32),
                     np.array(capacity, np.int32), key_dist, query_mode, ch, "edge case")
+
+
+# ------------------------------------------------------- LoopVQ workloads
+# Codebook-coded caches for the LoopVQ decode ("LoopVQ: Sub 1-bit KV Cache
+# Quantization for Looped Transformers"): per (layer, sequence, KV head,
+# token) D/4 key and D/4 value indices, uniform over the 256 entries; per
+# (layer, KV head) a key and a value codebook of N(0,1) entries [256][4 L];
+# queries 2 * N(0,1).  which: 0 keys, 1 values.
+
+@dataclasses.dataclass
+class VqWorkload:
+    name: str
+    n_loops: int
+    n_layers: int
+    n_heads: int
+    head_dim: int
+    batch: int
+    seed: int
+    lengths: np.ndarray      # int32 [batch]: coded tokens per unit
+    capacity: int            # token stride of the index arrays
+    description: str = ""
+
+    @property
+    def n_cells(self):
+        return self.n_loops * self.n_layers
+
+
+def make_vq(config="vq16k", **over):
+    """LoopVQ workload: "vq16k" (the batched 16K shape) or "vqsmall"."""
+    if config == "vq16k":
+        wl = VqWorkload("vq-batched-16k", 4, 24, 16, 128, 32, 12, np.full(32, 16384, np.int32),
+                        16384, "4 loops x 24 layers, 16 KV heads, D 128, batch 32, 16384 coded tokens")
+    elif config == "vqsmall":
+        wl = VqWorkload("vq-small", 4, 2, 2, 128, 3, 13, np.array([1, 33, 700], np.int32), 704,
+                        "4 loops x 2 layers, 2 KV heads, D 128, batch 3, ragged")
+    else:
+        raise ValueError("unknown LoopVQ config %r" % config)
+    for k, v in over.items():
+        setattr(wl, k, v)
+    return wl
+
+
+def vq_indices(wl, which, layer, b, h, t0, t1):
+    """uint8 [t1 - t0, D/4]: codebook indices of tokens t0..t1-1 of a unit."""
+    groups = wl.head_dim // 4
+    t = np.arange(t0, t1, dtype=np.uint32)[:, None]
+    j = np.arange(groups, dtype=np.uint32)[None, :]
+    u = px.philox4x32(t, j, np.uint32(h + wl.n_heads * b), np.uint32(layer | (which << 16)),
+                      wl.seed, STREAM_VQ_IDX)
+    return (u[0] & np.uint32(255)).astype(np.uint8)
+
+
+def vq_codebook(wl, which, layer, h):
+    """fp32 [256, 4 * n_loops]: the key (which 0) or value (1) codebook."""
+    e = np.arange(256, dtype=np.uint32)[:, None]
+    k = np.arange(4 * wl.n_loops, dtype=np.uint32)[None, :]
+    u = px.philox4x32(e, k, np.uint32(h), np.uint32(layer | (which << 16)), wl.seed, STREAM_VQ_CB)
+    return px.normal_from_bits(*u)
+
+
+def vq_query(wl, loop, layer, b, h):
+    """bf16 bits [D]: the query of (loop, layer, sequence, KV head)."""
+    d = np.arange(wl.head_dim, dtype=np.uint32)
+    u = px.philox4x32(d, np.uint32(loop), np.uint32(h + wl.n_heads * b), np.uint32(layer), wl.seed,
+                      STREAM_VQ_Q)
+    z = px.normal_from_bits(*u)
+    return px.float_to_bf16_bits((np.float32(2.0) * z).astype(np.float32))

@@ -136,3 +136,24 @@ def test_config2_cache_fits_one_b200(lk):
     rc, sizes = _query(lk, n_loops=4, n_layers=24, n_kv_heads=16, head_dim=128,
                        capacity=wl.capacity, kinds=wl.kinds, tau=wl.tau)
     assert rc == 0 and sizes.cache_bytes < 120e9
+
+
+def test_vq_decode_checks_arguments_before_any_device_work(lk):
+    # every host check of the LoopVQ decode runs before a CUDA call, so it
+    # answers without a GPU
+    import ctypes
+    import numpy as np
+    assert lk.loopkv_vq_decode(None, 0, None, None, None, None, None, None, None, None, None) == 1
+    d = lk.loopkv_vq_desc(4, 2, 2, 128, 3, 704, 0.0)
+    lens = np.array([1, 33, 700], np.int32)
+    lp = lens.ctypes.data_as(ctypes.c_void_p)
+    fake = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced on these paths
+    args = [fake] * 6
+    assert lk.loopkv_vq_decode(d, 0, lp, None, *args[1:], None, None) == 1   # null index array
+    assert lk.loopkv_vq_decode(d, 4, lp, *args, None, None) == 1             # loop out of range
+    bad = np.array([1, 0, 3], np.int32)
+    assert lk.loopkv_vq_decode(d, 0, bad.ctypes.data_as(ctypes.c_void_p), *args, None, None) == 1
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert lk.loopkv_vq_decode(d, 0, lp, odd, *args[1:], None, None) == 1    # misaligned
+    d.head_dim = 96
+    assert lk.loopkv_vq_decode(d, 0, lp, *args, None, None) == 1
