@@ -214,14 +214,14 @@ def source_hash(paths):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_src):
-    """DRAM bytes / algorithmic bytes of the decode kernel from the committed ncu
-    capture (profiles/decode_traffic.json), when it was taken on the current
-    kernel source; else None.  Traffic grows with the units a launch
-    processes, so a full launch moves this ratio times its algorithmic bytes."""
-    rec_paths = ["loop_aware_quantized_b200/csrc/decode.cu",
-                 "loop_aware_quantized_b200/csrc/loopkv_internal.cuh"]
-    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+def ncu_traffic(kernel_src, record="decode_traffic.json",
+                rec_paths=("loop_aware_quantized_b200/csrc/decode.cu",
+                           "loop_aware_quantized_b200/csrc/loopkv_internal.cuh")):
+    """DRAM bytes / algorithmic bytes of a kernel from its committed ncu
+    capture (profiles/<record>), when it was taken on the current kernel
+    source; else None.  Traffic grows with the units a launch processes, so
+    a full launch moves this ratio times its algorithmic bytes."""
+    path = os.path.join(ROOT, "profiles", record)
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -295,11 +295,188 @@ def oracle_baseline(config, seconds, seqs_global, g=1):
     return rate_units / (wl.batch * wl.n_heads), desc, 1
 
 
+# --------------------------------------------------------------- LoopVQ leg
+
+VQ_CONFIGS = ("vq16k",)
+
+
+def vq_unit_bytes(n, D):
+    """Algorithmic bytes of one LoopVQ unit decode: n tokens' key and value
+    indices (D/4 bytes each), the two codebooks' loop slices (256 entries x
+    4 fp32 each), the query (2D) and the output (4D)."""
+    return n * (D // 2) + 2 * 256 * 4 * 4 + 2 * D + 4 * D
+
+
+def oracle_baseline_vq(config, seconds, loop=1):
+    """Time the CPU oracle's LoopVQ decode on sampled units: (cell-steps/s, sample, cores)."""
+    from oracle import oracle as orc
+    from synth import workloads as W
+    wl = W.make_vq(config)
+    n = int(wl.lengths[0])
+    units = []
+    for layer, b, h in ((3, 5, 7), (17, 30, 2)):
+        units.append((W.vq_indices(wl, 0, layer, b, h, 0, n), W.vq_indices(wl, 1, layer, b, h, 0, n),
+                      W.vq_codebook(wl, 0, layer, h), W.vq_codebook(wl, 1, layer, h),
+                      W.vq_query(wl, loop, layer, b, h)))
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        for ik, iv, ck, cv, q in units:
+            orc.vq_decode(ik, iv, ck, cv, q, loop, wl.n_loops)
+            done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    desc = ("%d oracle LoopVQ decodes of %d sampled units (%d coded tokens each) in %.1f s on 1 "
+            "core; cell-steps/s = units/s / (%d seqs x %d heads)" % (done, len(units), n, el,
+                                                                    wl.batch, wl.n_heads))
+    return done / el / (wl.batch * wl.n_heads), desc, 1
+
+
+def bench_vq(args, rank, world):
+    """The LoopVQ decode workload: every (loop, layer) cell per step, one
+    launch per loop (all layers, sequences and KV heads)."""
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from loop_aware_quantized_b200 import vq_decode
+    from synth import workloads as W
+    from synth.gpu import VqDeviceGenerator
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    wl = W.make_vq(args.config)
+    if args.batch:
+        wl.batch = args.batch
+        wl.lengths = wl.lengths[:args.batch]
+    B, H, D, L = wl.batch, wl.n_heads, wl.head_dim, wl.n_loops
+    gen = VqDeviceGenerator(wl, dev)
+    t_build = time.perf_counter()
+    ik, iv = gen.indices(0), gen.indices(1)
+    cbk, cbv = gen.codebooks(0), gen.codebooks(1)
+    torch.cuda.synchronize()
+    build_s = time.perf_counter() - t_build
+    n_steps = args.warmup + args.steps
+    # queries of step s, loop l: the generator's stream for "loop" l + 16 s
+    qs = [[gen.queries(l + 16 * s) for l in range(L)] for s in range(n_steps)]
+    outs = [torch.empty(qs[0][0].shape, dtype=torch.float32, device=dev) for _ in range(L)]
+    lens = wl.lengths[:B]
+    stream = torch.cuda.current_stream()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(L)] for _ in range(args.steps)]
+
+    def step(s, events=None, q=None):
+        for loop in range(L):
+            if events is not None:
+                events[loop][0].record(stream)
+            vq_decode(loop, lens, ik, iv, cbk, cbv, qs[s][loop] if q is None else q[loop],
+                      out=outs[loop])
+            if events is not None:
+                events[loop][1].record(stream)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, events=ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = sum(a.elapsed_time(b) for row in ev for (a, b) in row)
+    elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], world, dev)
+    ms_per_step = elapsed_ms / args.steps
+    value = wl.n_cells * world / (ms_per_step / 1000.0)
+    launch_bytes = wl.n_layers * H * sum(vq_unit_bytes(int(n), D) for n in lens)
+    n_launches = args.steps * L
+    achieved = launch_bytes * n_launches / (dec_ms / 1000.0) / 1e9
+    peak, peak_kind = measured_peaks()
+    tr = ncu_traffic(None, "vq_traffic.json", ("loop_aware_quantized_b200/csrc/vq.cu",
+                                                "loop_aware_quantized_b200/csrc/loopkv_internal.cuh"))
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None if tr is None else tr * launch_bytes,
+                "peak_kind": peak_kind + " copy bandwidth",
+                "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                "kernel": "loopkv LoopVQ decode", "bytes_per_launch": launch_bytes,
+                "ms_per_launch": dec_ms / n_launches,
+                "note": "the kernel's shared-memory table lookups bind it before HBM does"}
+
+    e2e = None
+    if not args.no_e2e:
+        host_q = [[gen.queries(l + 16 * (n_steps + s)).cpu().pin_memory() for l in range(L)]
+                  for s in range(args.steps)]
+        dq = [torch.empty_like(qs[0][0]) for _ in range(L)]
+        host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        h2d = sum(x.numel() * x.element_size() for x in host_q[0])
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(args.steps):
+            for dst, src in zip(dq, host_q[s]):
+                dst.copy_(src, non_blocking=True)
+            step(0, q=dq)
+            for dst, src in zip(host_out, outs):
+                dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0] / args.steps
+        e2e = {"value": wl.n_cells * world / (e2e_ms / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms, "overlap": "none: copy in, decode, copy out per step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, cores = oracle_baseline_vq(args.config, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u8 codebook indices, fp32 codebooks and accumulate", "data": "synthetic",
+            "config": {"workload": "%s: LoopVQ decode, %d loops x %d layers, %d KV heads, head "
+                                   "dim %d, batch %d per GPU, %d coded tokens, 1 byte per 4 "
+                                   "channels x %d loops (%.2f bits per element)" % (
+                                       wl.name, L, wl.n_layers, H, D, B, int(lens[0]), L,
+                                       8.0 / (4 * L)),
+                       "step": "decode every (loop, layer) cell: one launch per loop",
+                       "global_batch": B * world, "seq_len": int(lens[0]),
+                       "parallelism": "dp%d (independent sequences)" % world,
+                       "l2": "inputs larger than L2 (indices %.1f GB)" % (
+                           2 * ik.numel() / 1e9), "build_s": build_s},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": L * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 # -------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
+    if args.config in VQ_CONFIGS:
+        return run_reference_vq(args)
     from synth import workloads as W
     wl = W.make(args.config)
     budget = max(1.0, min(args.cpu_seconds, 6.0))
@@ -320,8 +497,8 @@ def run_reference(args, rank, world):
         "ms_per_step": 1000.0 * wl.n_cells / value if value > 0 else None,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": "batched-16k (4x24 cells, 16 KV heads, D128, batch 32, 16384 "
-                               "tokens, tau 0.002)", "impl": "CPU oracle (fp64 C++)"},
+        "config": {"workload": workload_text(wl, wl.batch, args.q_per_kv),
+                   "impl": "CPU oracle (fp64 C++)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -332,6 +509,35 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ main arm
 
+def run_reference_vq(args):
+    from synth import workloads as W
+    wl = W.make_vq(args.config)
+    budget = max(1.0, min(args.cpu_seconds, 6.0))
+    for _ in range(args.warmup):
+        oracle_baseline_vq(args.config, 0.3)
+    vals, desc = [], ""
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        v, desc, cores = oracle_baseline_vq(args.config, budget / max(1, args.steps) + 0.2)
+        vals.append(v)
+    wall = time.perf_counter() - t_all
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * wl.n_cells / value if value > 0 else None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "%s: LoopVQ decode (%s)" % (wl.name, wl.description),
+                   "impl": "CPU oracle (fp64 C++)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": wall,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -339,6 +545,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.config in VQ_CONFIGS:
+        bench_vq(args, rank, world)
         return
 
     import torch

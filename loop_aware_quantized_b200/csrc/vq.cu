@@ -18,8 +18,13 @@
 //           (log2 units);
 //   softmax the CTA's max and sum of exponentials, merged over the cluster;
 //   pass 2  lane = token: p_t added into W[j][idx_v_j] (a weight histogram
-//           over the value codebook, shared-memory atomics);
-//   output  out[4j + i] = sum_e W[j][e] * entry_e[4l + i].
+//           over the value codebook): p_t as a fixed-point integer
+//           (units of 2^-31) with integer shared-memory atomics, which are
+//           native, order-independent and exact; every bin holds at most
+//           the sum of all weights (1), and each token's rounding (<= 2^-32)
+//           lands in one bin, so an output moves by at most n 2^-32 times
+//           the largest codebook magnitude;
+//   output  out[4j + i] = 2^-31 sum_e W[j][e] * entry_e[4l + i].
 // The index streams are read once (D/2 bytes per token at D = 128: 32 key
 // and 32 value bytes); the work per token is D/2 random shared-memory
 // accesses, so the kernel is bound by shared-memory bank conflicts of those
@@ -86,8 +91,8 @@ vq_decode_kernel(const VqParams p) {
   constexpr int GR = D / kVqSub;  // channel groups
   extern __shared__ __align__(16) float sm[];
   float* lut = sm;                 // [GR][kRow]
-  float* wv = lut + GR * kRow;     // [GR][kRow]
-  float* q_s = wv + GR * kRow;     // [D]
+  uint32_t* wv = reinterpret_cast<uint32_t*>(lut + GR * kRow);  // [GR][kRow] fixed point
+  float* q_s = lut + 2 * GR * kRow;  // [D]
   float* misc = q_s + D;           // [64]
   float* sc = misc + 64;           // [kVqSlots]
 
@@ -109,7 +114,7 @@ vq_decode_kernel(const VqParams p) {
   const float* cbv = p.cb_v + cbo;
 
   for (int d = tid; d < D; d += kVqThreads) q_s[d] = __uint_as_float((uint32_t)p.q[uidx * D + d] << 16);
-  for (int i = tid; i < GR * kRow; i += kVqThreads) wv[i] = 0.f;
+  for (int i = tid; i < GR * kRow; i += kVqThreads) wv[i] = 0u;
   __syncthreads();
   // LUT[j][e] = sum_i q[4j + i] * entry_e[4 loop + i] (thread = entry)
   for (int i = tid; i < GR * kEntries; i += kVqThreads) {
@@ -125,24 +130,47 @@ vq_decode_kernel(const VqParams p) {
   __syncthreads();
 
   // ---------------------------------------------------------------- pass 1
+  // two tokens per lane and iteration (t and t + 32): twice the independent
+  // table lookups in flight per warp
   const uint8_t* ik = p.idx_k + uidx * (size_t)p.cap * GR;
   float lmax = -INFINITY;
-  for (int base = p0 + 32 * warp; base < p1; base += 32 * kVqWarps) {
-    const int t = base + lane;
-    if (t < p1) {
-      uint32_t w[D / 16];
-      load_indices<D>(w, ik + (size_t)t * GR);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  for (int base = p0 + 64 * warp; base < p1; base += 64 * kVqWarps) {
+    const int t0 = base + lane, t1 = t0 + 32;
+    uint32_t w0[D / 16], w1[D / 16];
+    if (t0 < p1) load_indices<D>(w0, ik + (size_t)t0 * GR);
+    if (t1 < p1) load_indices<D>(w1, ik + (size_t)t1 * GR);
+    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+    if (t1 < p1) {
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
-        const uint32_t x = w[k];
+        const uint32_t x = w0[k], y = w1[k];
+        a0 += lut[(4 * k) * kRow + (x & 255u)];
+        b0 += lut[(4 * k) * kRow + (y & 255u)];
+        a1 += lut[(4 * k + 1) * kRow + ((x >> 8) & 255u)];
+        b1 += lut[(4 * k + 1) * kRow + ((y >> 8) & 255u)];
+        a0 += lut[(4 * k + 2) * kRow + ((x >> 16) & 255u)];
+        b0 += lut[(4 * k + 2) * kRow + ((y >> 16) & 255u)];
+        a1 += lut[(4 * k + 3) * kRow + (x >> 24)];
+        b1 += lut[(4 * k + 3) * kRow + (y >> 24)];
+      }
+    } else if (t0 < p1) {
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t x = w0[k];
         a0 += lut[(4 * k) * kRow + (x & 255u)];
         a1 += lut[(4 * k + 1) * kRow + ((x >> 8) & 255u)];
-        a2 += lut[(4 * k + 2) * kRow + ((x >> 16) & 255u)];
-        a3 += lut[(4 * k + 3) * kRow + (x >> 24)];
+        a0 += lut[(4 * k + 2) * kRow + ((x >> 16) & 255u)];
+        a1 += lut[(4 * k + 3) * kRow + (x >> 24)];
       }
-      const float s = ((a0 + a1) + (a2 + a3)) * p.score_scale;
-      sc[t - p0] = s;
+    }
+    if (t0 < p1) {
+      const float s = (a0 + a1) * p.score_scale;
+      sc[t0 - p0] = s;
+      lmax = fmaxf(lmax, s);
+    }
+    if (t1 < p1) {
+      const float s = (b0 + b1) * p.score_scale;
+      sc[t1 - p0] = s;
       lmax = fmaxf(lmax, s);
     }
   }
@@ -186,15 +214,27 @@ vq_decode_kernel(const VqParams p) {
 
   // ---------------------------------------------------------------- pass 2
   const uint8_t* iv = p.idx_v + uidx * (size_t)p.cap * GR;
-  for (int base = p0 + 32 * warp; base < p1; base += 32 * kVqWarps) {
-    const int t = base + lane;
-    if (t < p1) {
-      const float pw = exp2f(sc[t - p0] - M) * inv;
-      uint32_t w[D / 16];
-      load_indices<D>(w, iv + (size_t)t * GR);
+  for (int base = p0 + 64 * warp; base < p1; base += 64 * kVqWarps) {
+    const int t0 = base + lane, t1 = t0 + 32;
+    uint32_t w0[D / 16], w1[D / 16];
+    if (t0 < p1) load_indices<D>(w0, iv + (size_t)t0 * GR);
+    if (t1 < p1) load_indices<D>(w1, iv + (size_t)t1 * GR);
+    if (t0 < p1) {
+      const uint32_t pw = __float2uint_rn(exp2f(sc[t0 - p0] - M) * inv * 2147483648.0f);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
-        const uint32_t x = w[k];
+        const uint32_t x = w0[k];
+        atomicAdd(&wv[(4 * k) * kRow + (x & 255u)], pw);
+        atomicAdd(&wv[(4 * k + 1) * kRow + ((x >> 8) & 255u)], pw);
+        atomicAdd(&wv[(4 * k + 2) * kRow + ((x >> 16) & 255u)], pw);
+        atomicAdd(&wv[(4 * k + 3) * kRow + (x >> 24)], pw);
+      }
+    }
+    if (t1 < p1) {
+      const uint32_t pw = __float2uint_rn(exp2f(sc[t1 - p0] - M) * inv * 2147483648.0f);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t x = w1[k];
         atomicAdd(&wv[(4 * k) * kRow + (x & 255u)], pw);
         atomicAdd(&wv[(4 * k + 1) * kRow + ((x >> 8) & 255u)], pw);
         atomicAdd(&wv[(4 * k + 2) * kRow + ((x >> 16) & 255u)], pw);
@@ -209,8 +249,9 @@ vq_decode_kernel(const VqParams p) {
   {
     const int d = tid % D, part = tid / D, j = d / kVqSub, i = d % kVqSub;
     float o = 0.f;
-    for (int e = part; e < kEntries; e += PARTS) o = fmaf(wv[j * kRow + e], __ldg(cbv + (size_t)e * W + i), o);
-    lut[tid] = o;
+    for (int e = part; e < kEntries; e += PARTS)
+      o = fmaf((float)wv[j * kRow + e], __ldg(cbv + (size_t)e * W + i), o);
+    lut[tid] = o * 4.656612873077393e-10f;  // 2^-31
   }
   __syncthreads();
   if (tid < D) {
