@@ -131,14 +131,25 @@ vq_decode_kernel(const VqParams p) {
 
   // ---------------------------------------------------------------- pass 1
   // two tokens per lane and iteration (t and t + 32): twice the independent
-  // table lookups in flight per warp
+  // table lookups in flight per warp; the next iteration's indices are
+  // loaded into registers while the current ones are used
   const uint8_t* ik = p.idx_k + uidx * (size_t)p.cap * GR;
+  constexpr int STRIDE = 64 * kVqWarps;
   float lmax = -INFINITY;
-  for (int base = p0 + 64 * warp; base < p1; base += 64 * kVqWarps) {
+  uint32_t n0[D / 16], n1[D / 16];
+  if (p0 + 64 * warp + lane < p1) load_indices<D>(n0, ik + (size_t)(p0 + 64 * warp + lane) * GR);
+  if (p0 + 64 * warp + lane + 32 < p1)
+    load_indices<D>(n1, ik + (size_t)(p0 + 64 * warp + lane + 32) * GR);
+  for (int base = p0 + 64 * warp; base < p1; base += STRIDE) {
     const int t0 = base + lane, t1 = t0 + 32;
     uint32_t w0[D / 16], w1[D / 16];
-    if (t0 < p1) load_indices<D>(w0, ik + (size_t)t0 * GR);
-    if (t1 < p1) load_indices<D>(w1, ik + (size_t)t1 * GR);
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+      w0[k] = n0[k];
+      w1[k] = n1[k];
+    }
+    if (t0 + STRIDE < p1) load_indices<D>(n0, ik + (size_t)(t0 + STRIDE) * GR);
+    if (t1 + STRIDE < p1) load_indices<D>(n1, ik + (size_t)(t1 + STRIDE) * GR);
     float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
     if (t1 < p1) {
 #pragma unroll
@@ -214,11 +225,19 @@ vq_decode_kernel(const VqParams p) {
 
   // ---------------------------------------------------------------- pass 2
   const uint8_t* iv = p.idx_v + uidx * (size_t)p.cap * GR;
-  for (int base = p0 + 64 * warp; base < p1; base += 64 * kVqWarps) {
+  if (p0 + 64 * warp + lane < p1) load_indices<D>(n0, iv + (size_t)(p0 + 64 * warp + lane) * GR);
+  if (p0 + 64 * warp + lane + 32 < p1)
+    load_indices<D>(n1, iv + (size_t)(p0 + 64 * warp + lane + 32) * GR);
+  for (int base = p0 + 64 * warp; base < p1; base += STRIDE) {
     const int t0 = base + lane, t1 = t0 + 32;
     uint32_t w0[D / 16], w1[D / 16];
-    if (t0 < p1) load_indices<D>(w0, iv + (size_t)t0 * GR);
-    if (t1 < p1) load_indices<D>(w1, iv + (size_t)t1 * GR);
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+      w0[k] = n0[k];
+      w1[k] = n1[k];
+    }
+    if (t0 + STRIDE < p1) load_indices<D>(n0, iv + (size_t)(t0 + STRIDE) * GR);
+    if (t1 + STRIDE < p1) load_indices<D>(n1, iv + (size_t)(t1 + STRIDE) * GR);
     if (t0 < p1) {
       const uint32_t pw = __float2uint_rn(exp2f(sc[t0 - p0] - M) * inv * 2147483648.0f);
 #pragma unroll
