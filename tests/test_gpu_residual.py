@@ -85,3 +85,31 @@ def test_residual_rollback_keeps_the_coded_range(pool, cuda_device):
     plan.set_lengths([0], np.array([[129, 140]], np.int32))
     assert list(plan.lengths()[0, :2]) == [129, 140]
     torch.cuda.synchronize()
+
+
+def test_residual_rollback_then_append(pool, cuda_device):
+    """Window tokens dropped by set_lengths (or the whole unit reset) and
+    appended again give the bytes and outputs of a fresh build."""
+    import torch
+    from synth.gpu import DeviceGenerator
+    spec = _spec(64, (RS, Q2, Q4, Q4), (100, 150, 200), 0.02)
+    wl = W.custom(*spec)
+    seqs = [0, 1, 2]
+    plan = GH.make_plan(wl, seqs)
+    gen = DeviceGenerator(wl, cuda_device)
+    cells = list(range(wl.n_cells))
+    GH.build_cache(wl, plan, gen, seqs, wl.lengths)
+    # residual-coded counts 64 / 96 / 160 stay; sequence 2 is reset
+    back = np.array([97, 130, 0], np.int32)
+    plan.set_lengths([0], back[None, :])
+    assert (plan.lengths()[0, :3] == back).all()
+    T = int((wl.lengths - back).max())
+    k, v = gen.kv([0], seqs, back, T)
+    plan.append([0], k, v, n_new=(wl.lengths - back).astype(np.int32))
+    lens = np.tile(wl.lengths, (wl.n_cells, 1)).astype(np.int32)
+    res = GH.decode_all(wl, plan, gen, seqs, cells, lens, cuda_device)
+    plan.check()
+    units = [(c, b, h) for c in cells for b in seqs for h in range(wl.n_heads)]
+    n_of = lambda c, b: int(wl.lengths[b])  # noqa: E731
+    GH.compare(spec, wl, plan, res, cells, seqs, units, n_of, n_of, pool)
+    torch.cuda.synchronize()
