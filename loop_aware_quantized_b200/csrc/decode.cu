@@ -375,10 +375,31 @@ __device__ __forceinline__ void key_group(const KGroup<D>& g, const float (&qf)[
       cpart[r] = fmaf(qz, g.zr[i], cpart[r]);
     }
   }
+  if constexpr (G == 1) {
 #pragma unroll
-  for (int r = 0; r < G; ++r)
+    for (int o = 16; o > 0; o >>= 1) cpart[0] += __shfl_xor_sync(0xffffffffu, cpart[0], o);
+  } else {
+    // transposed butterfly: the first steps halve the queries a lane keeps
+    // (lane bit 4, then bit 3), the rest sum one query over the warp; the
+    // G totals are then read from the lanes that hold them
+    const bool b4 = (lane & 16) != 0;
+    float k;
+    if constexpr (G == 2) {
+      k = (b4 ? cpart[1] : cpart[0]) + __shfl_xor_sync(0xffffffffu, b4 ? cpart[0] : cpart[1], 16);
+    } else {
+      const float r0 = __shfl_xor_sync(0xffffffffu, b4 ? cpart[0] : cpart[2], 16);
+      const float r1 = __shfl_xor_sync(0xffffffffu, b4 ? cpart[1] : cpart[3], 16);
+      const float k0 = (b4 ? cpart[2] : cpart[0]) + r0;
+      const float k1 = (b4 ? cpart[3] : cpart[1]) + r1;
+      const bool b3 = (lane & 8) != 0;
+      k = (b3 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, b3 ? k0 : k1, 8);
+    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cpart[r] += __shfl_xor_sync(0xffffffffu, cpart[r], o);
+    for (int o = (G == 2 ? 8 : 4); o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+#pragma unroll
+    for (int r = 0; r < G; ++r)
+      cpart[r] = __shfl_sync(0xffffffffu, k, G == 2 ? 16 * r : 16 * (r >> 1) + 8 * (r & 1));
+  }
   __syncwarp();
 #pragma unroll
   for (int r = 0; r < G; ++r) s[r] = -INFINITY;
@@ -896,13 +917,27 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   auto token_share = [&](const uint32_t (&hw)[VS::NW], const float (&mt)[2 * VS::NGRP],
                          const float (&pt)[G], float mid, const uint8_t* lo_row) {
     float a[G][VS::NGRP];
-#pragma unroll
-    for (int r = 0; r < G; ++r)
+    if constexpr (G == 1) {
 #pragma unroll
       for (int gi = 0; gi < VS::NGRP; ++gi) {
-        a[r][gi] = (hmul * pt[r]) * mt[2 * gi];
-        gc[r][gi] = fmaf(mid, a[r][gi], fmaf(pt[r], mt[2 * gi + 1], gc[r][gi]));
+        a[0][gi] = (hmul * pt[0]) * mt[2 * gi];
+        gc[0][gi] = fmaf(mid, a[0][gi], fmaf(pt[0], mt[2 * gi + 1], gc[0][gi]));
       }
+    } else {
+      // the group's weight scale and constant, once for every query:
+      // a_r = p_r * (hmul * scale) (hmul a power of two: the same product),
+      // constant p_r * (zero + mid * hmul * scale)
+#pragma unroll
+      for (int gi = 0; gi < VS::NGRP; ++gi) {
+        const float hs = hmul * mt[2 * gi];
+        const float zc = fmaf(mid * hmul, mt[2 * gi], mt[2 * gi + 1]);
+#pragma unroll
+        for (int r = 0; r < G; ++r) {
+          a[r][gi] = pt[r] * hs;
+          gc[r][gi] = fmaf(pt[r], zc, gc[r][gi]);
+        }
+      }
+    }
     value_codes<G>(acc, hw, a);
     if (dense_lo) {
       uint32_t lw[VS::NW];
