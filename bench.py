@@ -214,7 +214,7 @@ def source_hash(paths):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_src, record="decode_traffic.json",
+def ncu_traffic(record="decode_traffic.json",
                 rec_paths=("loop_aware_quantized_b200/csrc/decode.cu",
                            "loop_aware_quantized_b200/csrc/loopkv_internal.cuh")):
     """DRAM bytes / algorithmic bytes of a kernel from its committed ncu
@@ -405,8 +405,8 @@ def bench_vq(args, rank, world):
     n_launches = args.steps * L
     achieved = launch_bytes * n_launches / (dec_ms / 1000.0) / 1e9
     peak, peak_kind = measured_peaks()
-    tr = ncu_traffic(None, "vq_traffic.json", ("loop_aware_quantized_b200/csrc/vq.cu",
-                                                "loop_aware_quantized_b200/csrc/loopkv_internal.cuh"))
+    tr = ncu_traffic("vq_traffic.json", ("loop_aware_quantized_b200/csrc/vq.cu",
+                                         "loop_aware_quantized_b200/csrc/loopkv_internal.cuh"))
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": None if tr is None else tr * launch_bytes,
                 "peak_kind": peak_kind + " copy bandwidth",
@@ -724,9 +724,7 @@ def main():
     peak, peak_kind = measured_peaks()
     achieved = dec_bytes / (dec_ms / 1000.0) / 1e9 if dec_ms > 0 else 0.0
     n_dec_launches = args.steps * len(phase)
-    kernel_src = [os.path.join(ROOT, "loop_aware_quantized_b200", "csrc", f)
-                  for f in ("decode.cu", "loopkv_internal.cuh")]
-    tr = ncu_traffic(kernel_src)
+    tr = ncu_traffic()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak,
                 "traffic": None if tr is None else tr * dec_bytes / n_dec_launches,

@@ -348,9 +348,9 @@ extern "C" loopkv_status loopkv_vq_decode(const loopkv_vq_desc* d, int32_t loop,
       !std::isfinite(d->sm_scale))
     return LOOPKV_ERR_INVALID_ARG;
   if (loop < 0 || loop >= d->n_loops) return LOOPKV_ERR_INVALID_ARG;
-  const void* ptrs[7] = {d_idx_k, d_idx_v, d_cb_k, d_cb_v, d_q, d_out, nullptr};
-  for (int i = 0; i < 6; ++i)
-    if (ptrs[i] == nullptr || !aligned16(ptrs[i])) return LOOPKV_ERR_INVALID_ARG;
+  const void* ptrs[6] = {d_idx_k, d_idx_v, d_cb_k, d_cb_v, d_q, d_out};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return LOOPKV_ERR_INVALID_ARG;
   if (d_lse != nullptr && (reinterpret_cast<uintptr_t>(d_lse) & 3u) != 0) return LOOPKV_ERR_INVALID_ARG;
   VqParams p{};
   int nmax = 0;
