@@ -68,7 +68,11 @@
 //   V3  decoding loop l reads slice [l*c, l*c + c) of each indexed entry as
 //       the token's channels of group j; softmax attention as in R7;
 //   V4  every position of a unit is coded (the op attends over coded
-//       tokens only).
+//       tokens only);
+//   V5  encoding a token picks, per group, the entry nearest to its
+//       sub-vector in squared Euclidean distance, computed in fp32 as
+//       sum over m = 0 .. 4L-1 (in that order) of fl(fl(x_m - c_m)^2), no
+//       fused multiply-add; ties go to the lowest index.
 // All attention arithmetic is fp64 (dequantized values, scores, softmax,
 // weighted sum).  Quantization is fp32 because the codes are defined by it.
 //
@@ -687,6 +691,37 @@ int orc_vq_decode(int n_loops, int D, int c, int n, int loop, const uint8_t* idx
       const int e = idx_v[static_cast<size_t>(t) * groups + d / c];
       out[d] += p * entry(cb_v, e, d);
     }
+  }
+  return 0;
+}
+
+// One token's codebook indices (V1, V5).  x: bf16 bits [n_loops][D], the
+// token's keys (or values) in every loop of its layer; cb: [256][L*c];
+// idx_out: [D/c].  Returns 0, or -1 on invalid sizes.
+int orc_vq_encode(int n_loops, int D, int c, const uint16_t* x, const float* cb,
+                  uint8_t* idx_out) {
+  if (n_loops < 1 || c < 1 || D % c != 0) return -1;
+  const int width = n_loops * c;
+  std::vector<float> sub(width);
+  for (int j = 0; j < D / c; ++j) {
+    for (int l = 0; l < n_loops; ++l)
+      for (int i = 0; i < c; ++i)
+        sub[l * c + i] = bf16_to_float(x[static_cast<size_t>(l) * D + j * c + i]);
+    int best = 0;
+    float best_d = INFINITY;
+    for (int e = 0; e < 256; ++e) {
+      float dist = 0.0f;
+      for (int m = 0; m < width; ++m) {
+        const float diff = sub[m] - cb[static_cast<size_t>(e) * width + m];
+        const float sq = diff * diff;
+        dist = dist + sq;
+      }
+      if (dist < best_d) {
+        best_d = dist;
+        best = e;
+      }
+    }
+    idx_out[j] = static_cast<uint8_t>(best);
   }
   return 0;
 }

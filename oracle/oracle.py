@@ -49,6 +49,8 @@ def _load():
     lib.orc_vq_decode.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_int, P, P, P, P, P, ctypes.c_double, P, P]
     lib.orc_vq_decode.restype = ctypes.c_int
+    lib.orc_vq_encode.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
+    lib.orc_vq_encode.restype = ctypes.c_int
     lib.orc_plan_brute.argtypes = [ctypes.c_int, ctypes.c_int, P, ctypes.c_int64, ctypes.c_int64,
                                    ctypes.c_int, P, P, P, P]
     lib.orc_plan_brute.restype = ctypes.c_int
@@ -249,3 +251,17 @@ def vq_decode(idx_k, idx_v, cb_k, cb_v, q_bits, loop, n_loops, sm_scale=0.0):
     if rc != 0:
         raise ValueError("oracle vq decode rejected its input")
     return out, float(lse[0])
+
+
+def vq_encode(x_bits, cb, c=4):
+    """Codebook indices of one token: x_bits bf16 bits [n_loops, D] (the
+    token in every loop of its layer), cb fp32 [256, n_loops * c] -> u8 [D/c]."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    L, D = x.shape
+    cb = np.ascontiguousarray(cb, dtype=np.float32)
+    assert cb.shape == (256, L * c)
+    out = np.zeros(D // c, np.uint8)
+    rc = _load().orc_vq_encode(L, D, c, _ptr(x), _ptr(cb), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle vq encode rejected its input")
+    return out

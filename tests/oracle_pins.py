@@ -670,6 +670,37 @@ def pin_vq_uniform_keys():
     assert np.abs(out - vals.mean(axis=0)).max() < 1e-12
 
 
+def pin_vq_encode_nearest():
+    # (a) a codebook holding every sub-vector exactly gives back their indices
+    # (distance 0); (b) on random data the chosen entry's distance, in fp64,
+    # is the brute-force minimum up to fp32 rounding; (c) equal entries: the
+    # lowest index wins.
+    D, L, c, n = 64, 4, 4, 16
+    K, V, cb_k, cb_v, idx_k, idx_v = _vq_exact(D, L, c, n, 420)
+    for t in range(n):
+        x = bf16(K[:, t, :])
+        assert (orc.vq_encode(x, cb_k) == idx_k[t]).all(), t
+    rng = np.random.default_rng(11)
+    cb = rng.standard_normal((256, L * c)).astype(np.float32)
+    for t in range(8):
+        x = rng_bits(430 + t, (L, 128))
+        idx = orc.vq_encode(x, cb)
+        xf = f32(x).astype(np.float64)
+        for j in range(32):
+            sub = xf[:, 4 * j:4 * j + 4].reshape(-1)
+            dist = ((cb.astype(np.float64) - sub[None, :]) ** 2).sum(axis=1)
+            assert dist[idx[j]] <= dist.min() * (1 + 1e-5) + 1e-9, (t, j)
+    x = rng_bits(440, (L, 64))
+    first = int(orc.vq_encode(x, cb)[0])
+    assert 0 < first < 255, first      # (this seed's pick leaves room on both sides)
+    cb2 = cb.copy()
+    cb2[255] = cb2[first]              # a later duplicate of the chosen entry
+    assert orc.vq_encode(x, cb2)[0] == first
+    cb3 = cb.copy()
+    cb3[0] = cb3[first]                # an earlier duplicate wins
+    assert orc.vq_encode(x, cb3)[0] == 0
+
+
 ALL_PINS = [
     pin_quantize_q2_ties,
     pin_quantize_q4_ties,
@@ -694,4 +725,5 @@ ALL_PINS = [
     pin_residual_reference_checks,
     pin_vq_exact_codebook,
     pin_vq_uniform_keys,
+    pin_vq_encode_nearest,
 ]

@@ -67,6 +67,10 @@ MUTANTS = [
      "const int e = idx_k[static_cast<size_t>(t) * groups + d / c];"),
     ("vq group of a channel", "const int e = idx_k[static_cast<size_t>(t) * groups + d / c];",
      "const int e = idx_k[static_cast<size_t>(t) * groups + d % groups];"),
+    ("vq encode keeps the farthest entry", "if (dist < best_d) {", "if (dist > best_d || e == 0) {"),
+    ("vq encode ties to the highest index", "if (dist < best_d) {", "if (dist <= best_d) {"),
+    ("vq encode reads one loop only", "sub[l * c + i] = bf16_to_float(x[static_cast<size_t>(l) * D + j * c + i]);",
+     "sub[l * c + i] = bf16_to_float(x[j * c + i]);"),
     ("residual window slot not modulo 64",
      "const size_t slot = static_cast<size_t>(t % kResWindow) * D * 2;",
      "const size_t slot = static_cast<size_t>(t - u->qtok()) * D * 2;"),
