@@ -338,6 +338,22 @@ loopkv_status loopkv_vq_decode(const loopkv_vq_desc* desc, int32_t loop, const i
                                const float* d_cb_k, const float* d_cb_v, const uint16_t* d_q,
                                float* d_out, float* d_lse, void* stream);
 
+/* Encode n_new tokens of every (layer, sequence, KV head) once every loop
+ * has produced them: d_x bf16 [n_loops][n_layers][batch][n_kv_heads][n_new]
+ * [head_dim] holds each token's keys (or values) in every loop; its D/4
+ * codebook indices go to positions h_pos[b] .. h_pos[b] + n_new - 1 of
+ * d_idx [n_layers][batch][n_kv_heads][capacity][D/4], using d_cb (the key
+ * or the value codebooks, shapes as for loopkv_vq_decode).  Per group: the
+ * entry nearest to the sub-vector in squared Euclidean distance, computed
+ * in fp32 as sum over m = 0 .. 4 n_loops - 1 (in that order) of
+ * fl(fl(x_m - c_m)^2) without fused multiply-add; ties go to the lowest
+ * index.  Call once for keys and once for values.  Errors (nothing
+ * launched): LOOPKV_ERR_INVALID_ARG (null or misaligned pointers, sizes,
+ * positions outside the capacity). */
+loopkv_status loopkv_vq_encode(const loopkv_vq_desc* desc, const int32_t* h_pos, int32_t n_new,
+                               const uint16_t* d_x, const float* d_cb, uint8_t* d_idx,
+                               void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,7 +8,7 @@ has not been built: there is no other code path.
 """
 
 _EXPORTS = ("LOOPKV_BF16", "LOOPKV_Q2", "LOOPKV_Q4", "LOOPKV_RES2", "LOOPKV_SHARE", "LoopKVError", "Plan",
-            "plan_optimize", "query_sizes", "vq_decode")
+            "plan_optimize", "query_sizes", "vq_decode", "vq_encode")
 
 
 def __getattr__(name):

@@ -299,6 +299,72 @@ vq_decode_kernel(const VqParams p) {
   }
 }
 
+// Encoder: one CTA per new token of a (layer, sequence, KV head); thread e
+// holds codebook entry e and computes its squared distance to the token's
+// D/4 sub-vectors in the fixed fp32 order (no fused multiply-add); the
+// smallest (distance, index) pair per group wins, so ties go to the lowest
+// index.
+struct VqEncodeParams {
+  const uint16_t* x;   // [L][n_layers][batch][H][n_new][D]
+  const float* cb;     // [n_layers][H][256][4 L]
+  uint8_t* idx;        // [n_layers][batch][H][cap][D/4]
+  int32_t n_layers, batch, H, L, cap, n_new;
+  int32_t pos[LOOPKV_MAX_BATCH];
+};
+
+template <int D>
+__global__ void __launch_bounds__(kEntries)
+vq_encode_kernel(const VqEncodeParams p) {
+  constexpr int GR = D / kVqSub;
+  __shared__ float x_s[GR][8 * kVqSub];                 // sub-vectors, loop-major
+  __shared__ unsigned long long best[kEntries / 32][GR];
+  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  const int i = blockIdx.x % p.n_new;
+  const int unit = blockIdx.x / p.n_new;
+  const int h = unit % p.H;
+  const int b = (unit / p.H) % p.batch;
+  const int layer = unit / (p.H * p.batch);
+  const int W = p.L * kVqSub;
+  const size_t loop_stride = (size_t)p.n_layers * p.batch * p.H * p.n_new * D;
+  const size_t tok = ((((size_t)layer * p.batch + b) * p.H + h) * p.n_new + i) * D;
+  for (int k = e; k < p.L * D; k += kEntries) {
+    const int l = k / D, d = k % D;
+    x_s[d / kVqSub][l * kVqSub + d % kVqSub] =
+        __uint_as_float((uint32_t)p.x[l * loop_stride + tok + d] << 16);
+  }
+  float c[8 * kVqSub];
+  const float* ce = p.cb + (((size_t)layer * p.H + h) * kEntries + e) * W;
+#pragma unroll
+  for (int m = 0; m < 8 * kVqSub; ++m) c[m] = m < W ? __ldg(ce + m) : 0.f;
+  __syncthreads();
+  for (int j = 0; j < GR; ++j) {
+    float dist = 0.f;
+#pragma unroll
+    for (int m = 0; m < 8 * kVqSub; ++m) {
+      if (m < W) {
+        const float diff = __fsub_rn(x_s[j][m], c[m]);
+        dist = __fadd_rn(dist, __fmul_rn(diff, diff));
+      }
+    }
+    // distances are >= 0, so their bit patterns order like the values
+    unsigned long long key = ((unsigned long long)__float_as_uint(dist) << 32) | (unsigned)e;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
+      key = other < key ? other : key;
+    }
+    if (lane == 0) best[warp][j] = key;
+  }
+  __syncthreads();
+  if (e < GR) {
+    unsigned long long key = best[0][e];
+#pragma unroll
+    for (int w = 1; w < kEntries / 32; ++w) key = best[w][e] < key ? best[w][e] : key;
+    const size_t row = (((size_t)layer * p.batch + b) * p.H + h) * p.cap + p.pos[b] + i;
+    p.idx[row * GR + e] = (uint8_t)(key & 0xFFu);
+  }
+}
+
 template <int D>
 constexpr size_t vq_smem() {
   return sizeof(float) * ((size_t)2 * (D / kVqSub) * kRow + D + 64 + kVqSlots);
@@ -331,6 +397,14 @@ int launch_vq_t(const VqParams& p, long long units, cudaStream_t stream) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+bool vq_desc_ok(const loopkv_vq_desc* d) {
+  return d != nullptr && d->n_loops >= 1 && d->n_loops <= 8 && d->n_layers >= 1 &&
+         d->n_kv_heads >= 1 && d->n_kv_heads <= (1 << 16) &&
+         (d->head_dim == 64 || d->head_dim == 128) && d->batch >= 1 &&
+         d->batch <= LOOPKV_MAX_BATCH && d->capacity >= 1 && d->capacity <= (1 << 20) &&
+         std::isfinite(d->sm_scale);
+}
+
 }  // namespace
 }  // namespace loopkv
 
@@ -341,12 +415,7 @@ extern "C" loopkv_status loopkv_vq_decode(const loopkv_vq_desc* d, int32_t loop,
                                           const float* d_cb_k, const float* d_cb_v,
                                           const uint16_t* d_q, float* d_out, float* d_lse,
                                           void* stream) {
-  if (d == nullptr || h_len == nullptr) return LOOPKV_ERR_INVALID_ARG;
-  if (d->n_loops < 1 || d->n_loops > 8 || d->n_layers < 1 || d->n_kv_heads < 1 ||
-      d->n_kv_heads > (1 << 16) || (d->head_dim != 64 && d->head_dim != 128) || d->batch < 1 ||
-      d->batch > LOOPKV_MAX_BATCH || d->capacity < 1 || d->capacity > (1 << 20) ||
-      !std::isfinite(d->sm_scale))
-    return LOOPKV_ERR_INVALID_ARG;
+  if (h_len == nullptr || !vq_desc_ok(d)) return LOOPKV_ERR_INVALID_ARG;
   if (loop < 0 || loop >= d->n_loops) return LOOPKV_ERR_INVALID_ARG;
   const void* ptrs[6] = {d_idx_k, d_idx_v, d_cb_k, d_cb_v, d_q, d_out};
   for (const void* ptr : ptrs)
@@ -384,4 +453,36 @@ extern "C" loopkv_status loopkv_vq_decode(const loopkv_vq_desc* d, int32_t loop,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int e = d->head_dim == 64 ? launch_vq_t<64>(p, units, s) : launch_vq_t<128>(p, units, s);
   return e == 0 ? LOOPKV_OK : LOOPKV_ERR_CUDA;
+}
+
+extern "C" loopkv_status loopkv_vq_encode(const loopkv_vq_desc* d, const int32_t* h_pos,
+                                          int32_t n_new, const uint16_t* d_x, const float* d_cb,
+                                          uint8_t* d_idx, void* stream) {
+  if (h_pos == nullptr || !vq_desc_ok(d) || n_new < 0) return LOOPKV_ERR_INVALID_ARG;
+  if (n_new == 0) return LOOPKV_OK;
+  const void* ptrs[3] = {d_x, d_cb, d_idx};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return LOOPKV_ERR_INVALID_ARG;
+  VqEncodeParams p{};
+  for (int b = 0; b < d->batch; ++b) {
+    if (h_pos[b] < 0 || (long long)h_pos[b] + n_new > d->capacity) return LOOPKV_ERR_INVALID_ARG;
+    p.pos[b] = h_pos[b];
+  }
+  const long long blocks = (long long)d->n_layers * d->batch * d->n_kv_heads * n_new;
+  if (blocks >= (1LL << 31)) return LOOPKV_ERR_UNSUPPORTED;
+  p.x = d_x;
+  p.cb = d_cb;
+  p.idx = d_idx;
+  p.n_layers = d->n_layers;
+  p.batch = d->batch;
+  p.H = d->n_kv_heads;
+  p.L = d->n_loops;
+  p.cap = d->capacity;
+  p.n_new = n_new;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d->head_dim == 64)
+    vq_encode_kernel<64><<<(unsigned)blocks, kEntries, 0, s>>>(p);
+  else
+    vq_encode_kernel<128><<<(unsigned)blocks, kEntries, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LOOPKV_OK : LOOPKV_ERR_CUDA;
 }

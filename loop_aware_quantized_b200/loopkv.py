@@ -114,6 +114,7 @@ def _load():
                                       ctypes.POINTER(loopkv_plan_cost)]),
         "loopkv_vq_decode": (st, [ctypes.POINTER(loopkv_vq_desc), I32, P, P, P, P, P, P, P, P,
                                   P]),
+        "loopkv_vq_encode": (st, [ctypes.POINTER(loopkv_vq_desc), P, I32, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -164,6 +165,11 @@ def loopkv_vq_decode(desc, loop, h_len, d_idx_k, d_idx_v, d_cb_k, d_cb_v, d_q, d
     ref = None if desc is None else ctypes.byref(desc)
     return _lib.loopkv_vq_decode(ref, loop, h_len, d_idx_k, d_idx_v, d_cb_k, d_cb_v, d_q, d_out,
                                  d_lse, stream)
+
+
+def loopkv_vq_encode(desc, h_pos, n_new, d_x, d_cb, d_idx, stream):
+    ref = None if desc is None else ctypes.byref(desc)
+    return _lib.loopkv_vq_encode(ref, h_pos, n_new, d_x, d_cb, d_idx, stream)
 
 
 def loopkv_plan_optimize(desc, kinds_out):
@@ -390,3 +396,24 @@ def vq_decode(loop, lengths, idx_k, idx_v, cb_k, cb_v, q, out=None, lse=None, sm
                           _ptr(cb_v), _ptr(q), _ptr(out), _ptr(lse), _stream_handle(stream))
     _check(rc, "loopkv_vq_decode")
     return out
+
+
+def vq_encode(positions, x, cb, idx, stream=None):
+    """LoopVQ encoder: x bf16 [n_loops, n_layers, batch, H, n_new, D] (each
+    token in every loop of its layer) -> codebook indices written into idx
+    (uint8 [n_layers, batch, H, capacity, D/4]) at positions[b] + i, using cb
+    (fp32 [n_layers, H, 256, 4 * n_loops]).  Returns idx."""
+    import torch
+    assert x.dtype == torch.bfloat16 and cb.dtype == torch.float32 and idx.dtype == torch.uint8
+    for t in (x, cb, idx):
+        assert t.is_contiguous()
+    L, n_layers, batch, H, n_new, D = x.shape
+    assert idx.shape == (n_layers, batch, H, idx.shape[3], D // 4)
+    assert cb.shape == (n_layers, H, 256, 4 * L)
+    d = loopkv_vq_desc(L, n_layers, H, D, batch, idx.shape[3], 0.0)
+    positions = np.ascontiguousarray(positions, dtype=np.int32)
+    assert positions.size == batch
+    rc = loopkv_vq_encode(d, _np_ptr(positions), int(n_new), _ptr(x), _ptr(cb), _ptr(idx),
+                          _stream_handle(stream))
+    _check(rc, "loopkv_vq_encode")
+    return idx

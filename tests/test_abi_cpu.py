@@ -157,3 +157,18 @@ def test_vq_decode_checks_arguments_before_any_device_work(lk):
     assert lk.loopkv_vq_decode(d, 0, lp, odd, *args[1:], None, None) == 1    # misaligned
     d.head_dim = 96
     assert lk.loopkv_vq_decode(d, 0, lp, *args, None, None) == 1
+
+
+def test_vq_encode_checks_arguments_before_any_device_work(lk):
+    import ctypes
+    import numpy as np
+    d = lk.loopkv_vq_desc(4, 2, 2, 128, 2, 16, 0.0)
+    pos = np.array([3, 0], np.int32)
+    pp = pos.ctypes.data_as(ctypes.c_void_p)
+    fake = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced on these paths
+    assert lk.loopkv_vq_encode(None, pp, 5, fake, fake, fake, None) == 1
+    assert lk.loopkv_vq_encode(d, pp, 0, None, None, None, None) == 0      # nothing to do
+    assert lk.loopkv_vq_encode(d, pp, -1, fake, fake, fake, None) == 1
+    assert lk.loopkv_vq_encode(d, pp, 14, fake, fake, fake, None) == 1     # 3 + 14 > 16
+    assert lk.loopkv_vq_encode(d, pp, 5, None, fake, fake, None) == 1
+    assert lk.loopkv_vq_encode(d, pp, 5, fake, ctypes.c_void_p((1 << 20) + 8), fake, None) == 1

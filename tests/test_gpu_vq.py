@@ -1,6 +1,7 @@
-"""LoopVQ decode on the CUDA path against the CPU oracle (needs a B200):
+"""LoopVQ decode and encoder on the CUDA path against the CPU oracle (needs a B200):
 ragged lengths, every loop, both head dims, cluster splits, the device input
-generator, the 16K shape on sampled units, and the host argument checks."""
+generator, the 16K shape on sampled units, the host argument checks, and
+bit-exact nearest-entry indices from the encoder."""
 
 import numpy as np
 import pytest
@@ -108,3 +109,36 @@ def test_vq_argument_checks(cuda_device):
         with pytest.raises(LoopKVError):
             vq_decode(loop, lens, ik, ik, cb, cb, q)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("D,L", [(128, 4), (64, 2), (128, 8)])
+def test_vq_encode_matches_oracle(cuda_device, D, L):
+    # nearest-entry indices, bit-exact: both sides compute the distances in
+    # the same fp32 order and break ties to the lowest index
+    import torch
+    from loop_aware_quantized_b200 import vq_encode
+    from oracle import oracle as orc
+    from synth import philox as px
+    wl = W.make_vq("vqsmall", head_dim=D, n_loops=L, batch=2, lengths=np.array([9, 9], np.int32),
+                   capacity=16)
+    n_new, pos = 5, np.array([3, 0], np.int32)
+    shape = (L, wl.n_layers, wl.batch, wl.n_heads, n_new, D)
+    u = px.philox4x32(np.arange(int(np.prod(shape)), dtype=np.uint32), 0, 0, 0, 77, 99)
+    x = px.float_to_bf16_bits(px.normal_from_bits(*u).reshape(shape))
+    cb = np.stack([np.stack([W.vq_codebook(wl, 0, layer, h) for h in range(wl.n_heads)])
+                   for layer in range(wl.n_layers)])
+    dx = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(cuda_device)
+    dcb = torch.from_numpy(np.ascontiguousarray(cb)).to(cuda_device)
+    idx = torch.zeros((wl.n_layers, wl.batch, wl.n_heads, 16, D // 4), dtype=torch.uint8,
+                      device=cuda_device)
+    vq_encode(pos, dx, dcb, idx)
+    got = idx.cpu().numpy()
+    for layer in range(wl.n_layers):
+        for b in range(wl.batch):
+            for h in range(wl.n_heads):
+                for i in range(n_new):
+                    want = orc.vq_encode(x[:, layer, b, h, i, :], cb[layer, h])
+                    assert (got[layer, b, h, pos[b] + i] == want).all(), (layer, b, h, i)
+                # positions outside the written range stay untouched
+                untouched = [t for t in range(16) if not pos[b] <= t < pos[b] + n_new]
+                assert (got[layer, b, h, untouched] == 0).all()
