@@ -334,13 +334,15 @@ def oracle_baseline_vq(config, seconds, loop=1):
 
 
 def bench_vq(args, rank, world):
-    """The LoopVQ decode workload: every (loop, layer) cell per step, one
-    launch per loop (all layers, sequences and KV heads)."""
+    """The LoopVQ workload: per step, the new token of every (layer,
+    sequence, KV head) is encoded (keys, values: one launch each, all loops
+    at once) and every (loop, layer) cell is decoded (one launch per loop,
+    all layers, sequences and KV heads)."""
     import torch
     import torch.distributed as dist
     from datetime import timedelta
 
-    from loop_aware_quantized_b200 import vq_decode
+    from loop_aware_quantized_b200 import vq_decode, vq_encode
     from synth import workloads as W
     from synth.gpu import VqDeviceGenerator
 
@@ -354,32 +356,46 @@ def bench_vq(args, rank, world):
         wl.batch = args.batch
         wl.lengths = wl.lengths[:args.batch]
     B, H, D, L = wl.batch, wl.n_heads, wl.head_dim, wl.n_loops
+    n0 = wl.lengths[:B].astype(np.int32)
+    n_steps = args.warmup + args.steps
+    total_steps = n_steps + (0 if args.no_e2e else args.steps)
+    wl.capacity = int(n0.max()) + total_steps   # room for one new token per step
     gen = VqDeviceGenerator(wl, dev)
     t_build = time.perf_counter()
-    ik, iv = gen.indices(0), gen.indices(1)
+    ik, iv = gen.indices(0, T=int(n0.max())), gen.indices(1, T=int(n0.max()))
     cbk, cbv = gen.codebooks(0), gen.codebooks(1)
     torch.cuda.synchronize()
     build_s = time.perf_counter() - t_build
-    n_steps = args.warmup + args.steps
-    # queries of step s, loop l: the generator's stream for "loop" l + 16 s
-    qs = [[gen.queries(l + 16 * s) for l in range(L)] for s in range(n_steps)]
-    outs = [torch.empty(qs[0][0].shape, dtype=torch.float32, device=dev) for _ in range(L)]
-    lens = wl.lengths[:B]
+
+    def inputs(s):
+        """Step s: queries per loop ("loop" stream l + 16 s) and the new
+        token's keys and values in every loop (streams 1000 + ..., 2000 + ...)."""
+        q = [gen.queries(l + 16 * s) for l in range(L)]
+        xk = torch.stack([gen.queries(1000 + l + 16 * s) for l in range(L)]).unsqueeze(4)
+        xv = torch.stack([gen.queries(2000 + l + 16 * s) for l in range(L)]).unsqueeze(4)
+        return q, xk.contiguous(), xv.contiguous()
+
+    ins = [inputs(s) for s in range(n_steps)]
+    outs = [torch.empty(ins[0][0][0].shape, dtype=torch.float32, device=dev) for _ in range(L)]
     stream = torch.cuda.current_stream()
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(L)] for _ in range(args.steps)]
 
-    def step(s, events=None, q=None):
+    def step(s, inp, events=None):
+        """Encode the token at position n0 + s, then decode over n0 + s + 1."""
+        q, xk, xv = inp
+        vq_encode(n0 + s, xk, cbk, ik)
+        vq_encode(n0 + s, xv, cbv, iv)
+        lens = n0 + s + 1
         for loop in range(L):
             if events is not None:
                 events[loop][0].record(stream)
-            vq_decode(loop, lens, ik, iv, cbk, cbv, qs[s][loop] if q is None else q[loop],
-                      out=outs[loop])
+            vq_decode(loop, lens, ik, iv, cbk, cbv, q[loop], out=outs[loop])
             if events is not None:
                 events[loop][1].record(stream)
 
     for s in range(args.warmup):
-        step(s)
+        step(s, ins[s])
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
     sampler.start()
@@ -390,7 +406,7 @@ def bench_vq(args, rank, world):
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(args.steps):
-        step(args.warmup + i, events=ev[i])
+        step(args.warmup + i, ins[args.warmup + i], events=ev[i])
     t_end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -401,9 +417,11 @@ def bench_vq(args, rank, world):
     elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], world, dev)
     ms_per_step = elapsed_ms / args.steps
     value = wl.n_cells * world / (ms_per_step / 1000.0)
-    launch_bytes = wl.n_layers * H * sum(vq_unit_bytes(int(n), D) for n in lens)
     n_launches = args.steps * L
-    achieved = launch_bytes * n_launches / (dec_ms / 1000.0) / 1e9
+    dec_bytes = sum(L * wl.n_layers * H * sum(vq_unit_bytes(int(n) + args.warmup + i + 1, D)
+                                              for n in n0) for i in range(args.steps))
+    launch_bytes = dec_bytes / n_launches
+    achieved = dec_bytes / (dec_ms / 1000.0) / 1e9
     peak, peak_kind = measured_peaks()
     tr = ncu_traffic("vq_traffic.json", ("loop_aware_quantized_b200/csrc/vq.cu",
                                          "loop_aware_quantized_b200/csrc/loopkv_internal.cuh"))
@@ -417,11 +435,15 @@ def bench_vq(args, rank, world):
 
     e2e = None
     if not args.no_e2e:
-        host_q = [[gen.queries(l + 16 * (n_steps + s)).cpu().pin_memory() for l in range(L)]
-                  for s in range(args.steps)]
-        dq = [torch.empty_like(qs[0][0]) for _ in range(L)]
+        host_in = []
+        for s in range(args.steps):
+            q, xk, xv = inputs(n_steps + s)
+            host_in.append(([x.cpu().pin_memory() for x in q], xk.cpu().pin_memory(),
+                            xv.cpu().pin_memory()))
+        dq = [torch.empty_like(x) for x in ins[0][0]]
+        dxk, dxv = torch.empty_like(ins[0][1]), torch.empty_like(ins[0][2])
         host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-        h2d = sum(x.numel() * x.element_size() for x in host_q[0])
+        h2d = sum(x.numel() * x.element_size() for x in host_in[0][0]) + 2 * dxk.numel() * 2
         d2h = sum(o.numel() * o.element_size() for o in outs)
         if world > 1:
             dist.barrier()
@@ -430,9 +452,12 @@ def bench_vq(args, rank, world):
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for s in range(args.steps):
-            for dst, src in zip(dq, host_q[s]):
+            hq, hxk, hxv = host_in[s]
+            for dst, src in zip(dq, hq):
                 dst.copy_(src, non_blocking=True)
-            step(0, q=dq)
+            dxk.copy_(hxk, non_blocking=True)
+            dxv.copy_(hxv, non_blocking=True)
+            step(n_steps + s, (dq, dxk, dxv))
             for dst, src in zip(host_out, outs):
                 dst.copy_(src, non_blocking=True)
         e1.record(stream)
@@ -440,7 +465,8 @@ def bench_vq(args, rank, world):
         e2e_ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0] / args.steps
         e2e = {"value": wl.n_cells * world / (e2e_ms / 1000.0), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e2e_ms, "overlap": "none: copy in, decode, copy out per step"}
+               "ms_per_step": e2e_ms,
+               "overlap": "none: copy in, encode + decode, copy out per step"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -452,18 +478,19 @@ def bench_vq(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "u8 codebook indices, fp32 codebooks and accumulate", "data": "synthetic",
-            "config": {"workload": "%s: LoopVQ decode, %d loops x %d layers, %d KV heads, head "
-                                   "dim %d, batch %d per GPU, %d coded tokens, 1 byte per 4 "
-                                   "channels x %d loops (%.2f bits per element)" % (
-                                       wl.name, L, wl.n_layers, H, D, B, int(lens[0]), L,
-                                       8.0 / (4 * L)),
-                       "step": "decode every (loop, layer) cell: one launch per loop",
-                       "global_batch": B * world, "seq_len": int(lens[0]),
+            "config": {"workload": "%s: LoopVQ, %d loops x %d layers, %d KV heads, head "
+                                   "dim %d, batch %d per GPU, %d coded tokens + 1 encoded per "
+                                   "step, 1 byte per 4 channels x %d loops (%.2f bits per "
+                                   "element)" % (wl.name, L, wl.n_layers, H, D, B, int(n0[0]), L,
+                                                 8.0 / (4 * L)),
+                       "step": "encode the new token (keys, values), then decode every "
+                               "(loop, layer) cell: one launch per loop",
+                       "global_batch": B * world, "seq_len": int(n0[0]),
                        "parallelism": "dp%d (independent sequences)" % world,
                        "l2": "inputs larger than L2 (indices %.1f GB)" % (
                            2 * ik.numel() / 1e9), "build_s": build_s},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": L * args.steps, "clocks": clocks,
+            "gpu_launches": (L + 2) * args.steps, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -48,7 +48,7 @@ constexpr int kVqWarps = kVqThreads / 32;
 constexpr int kVqSub = 4;        // channels per sub-vector
 constexpr int kEntries = 256;    // codebook entries (one byte)
 constexpr int kRow = kEntries + 1;  // padded table row: group j's row starts in bank j
-constexpr int kVqSlots = 8192;   // score slots per CTA (two CTAs per SM)
+constexpr int kVqSlots = 8448;   // score slots per CTA (two CTAs per SM; 16K + a few hundred tokens in two)
 constexpr int kVqMaxSplit = 8;   // portable cluster size
 
 struct VqParams {
