@@ -169,3 +169,21 @@ def test_planner_plan_drives_the_cache(pool, cuda_device):
     kinds, cost = plan_optimize(2, 2, 64, damage, 9, 14 * 16, 0.0)
     assert sorted(set(int(k) for k in kinds)) == [Q4, Q2, SH], kinds
     _check_spec(_spec(64, tuple(int(k) for k in kinds), (33, 97, 300), 0.02), pool, cuda_device)
+
+
+def test_longest_unit_then_refusal(pool, cuda_device):
+    """The longest unit a decode takes (8 CTAs of 24576 score slots: a
+    cluster of 8) matches the oracle; one past what 8 CTAs hold is refused
+    on the host with LOOPKV_ERR_UNSUPPORTED."""
+    import torch
+    from loop_aware_quantized_b200 import LoopKVError
+    spec = (1, 1, 1, 128, (Q4,), (196000,), (196032,), 0.002)
+    _check_spec(spec, pool, cuda_device)
+    from synth.gpu import DeviceGenerator
+    wl = W.custom(1, 1, 1, 128, (Q4,), (196700,), (196736,), 0.002)
+    plan = GH.make_plan(wl, [0])
+    GH.build_cache(wl, plan, DeviceGenerator(wl, cuda_device), [0], wl.lengths)
+    with pytest.raises(LoopKVError) as e:
+        plan.decode([0], torch.zeros((1, 1, 1, 128), dtype=torch.bfloat16, device=cuda_device))
+    assert e.value.status == 4
+    torch.cuda.synchronize()

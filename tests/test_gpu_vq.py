@@ -142,3 +142,20 @@ def test_vq_encode_matches_oracle(cuda_device, D, L):
                 # positions outside the written range stay untouched
                 untouched = [t for t in range(16) if not pos[b] <= t < pos[b] + n_new]
                 assert (got[layer, b, h, untouched] == 0).all()
+
+
+def test_vq_longest_unit_then_refusal(pool, cuda_device):
+    # 8 CTAs of 8448 score slots hold 67584 tokens; one more is refused
+    import torch
+    from loop_aware_quantized_b200 import LoopKVError, vq_decode
+    over = {"batch": 1, "lengths": np.array([67584], np.int32), "capacity": 67585, "n_layers": 1,
+            "n_heads": 1}
+    _run(("vqsmall", over), [2], pool, cuda_device)
+    wl = W.make_vq("vqsmall", **over)
+    ik = torch.zeros((1, 1, 1, 67585, 32), dtype=torch.uint8, device=cuda_device)
+    cb = torch.zeros((1, 1, 256, 16), dtype=torch.float32, device=cuda_device)
+    q = torch.zeros((1, 1, 1, 128), dtype=torch.bfloat16, device=cuda_device)
+    with pytest.raises(LoopKVError) as e:
+        vq_decode(0, np.array([67585], np.int32), ik, ik, cb, cb, q)
+    assert e.value.status == 4
+    torch.cuda.synchronize()
