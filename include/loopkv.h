@@ -65,8 +65,11 @@
  * the table, skips the affected unit, and is reported by loopkv_check().
  *
  * Asynchrony.  loopkv_append, loopkv_decode and loopkv_set_lengths only
- * enqueue work on the given stream and return.  A plan handle must not be
- * used from two host threads at once.
+ * enqueue work on the given stream and return.  A decode (and the LoopVQ
+ * calls) can be captured into a CUDA graph and replayed; an append or
+ * set_lengths updates the host copy of the lengths when it is called, so
+ * replaying one from a graph would leave that copy behind.  A plan handle
+ * must not be used from two host threads at once.
  *
  * Cache layout (canonical, part of the contract).  The cache is one buffer;
  * cell c, sequence b, head h owns a region at loopkv_unit_region().  With

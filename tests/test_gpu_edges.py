@@ -187,3 +187,32 @@ def test_longest_unit_then_refusal(pool, cuda_device):
         plan.decode([0], torch.zeros((1, 1, 1, 128), dtype=torch.bfloat16, device=cuda_device))
     assert e.value.status == 4
     torch.cuda.synchronize()
+
+
+def test_decode_replays_from_a_cuda_graph(cuda_device):
+    """loopkv_decode only enqueues work (no host synchronisation), so a
+    decode captured into a CUDA graph replays with the eager results, bit
+    for bit (the kernel's reductions have a fixed order)."""
+    import torch
+    from synth.gpu import DeviceGenerator
+    spec = _spec(128, (Q4, SH, Q2, Q4), (300, 1000), 0.01)
+    wl = W.custom(*spec)
+    seqs = [0, 1]
+    plan = GH.make_plan(wl, seqs)
+    gen = DeviceGenerator(wl, cuda_device)
+    GH.build_cache(wl, plan, gen, seqs, wl.lengths)
+    cells = list(range(wl.n_cells))
+    q = gen.queries(cells, seqs, np.tile(wl.lengths, (len(cells), 1)))
+    eager = plan.decode(cells, q).clone()
+    out = torch.zeros_like(eager)
+    s = torch.cuda.Stream(device=cuda_device)
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        plan.decode(cells, q, out=out, stream=s)
+    for _ in range(2):
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    plan.check()
