@@ -763,9 +763,8 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   constexpr size_t VSTEP = (size_t)kWarps * 32 * (D / 4);
   auto full_block = [&](int bk) { return (bk + 1) * 32 <= qlim; };
   // Up to two queries per KV head: the next block's rows wait in registers.
-  // Four keep no registers for them: rows are loaded as they are used, with
-  // the next block's lines requested into L2 one block ahead (measured
-  // faster for four, slower for two).
+  // Four have no registers to spare: their blocks go through shared-memory
+  // staging buffers (below).
   constexpr bool kRegNext = G <= 2;
   constexpr int NB = kRegNext ? LPT : 1;
   uint32_t nh[NB][VS::NW];
