@@ -248,7 +248,9 @@ class Plan:
     """A loaded LoopKV plan with its device table and cache (torch tensors)."""
 
     def __init__(self, n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau,
-                 sm_scale=0.0, device="cuda", stream=None, q_per_kv=1):
+                 sm_scale=0.0, device="cuda", stream=None, q_per_kv=1, cache_guard=0):
+        """cache_guard: extra bytes allocated after the cache (not given to the
+        library), so tests can check that nothing is written past its end."""
         import torch
         self.n_loops, self.n_layers = n_loops, n_layers
         self.n_cells = n_loops * n_layers
@@ -264,7 +266,8 @@ class Plan:
         _check(rc, "loopkv_plan_query")
         self.table_bytes, self.cache_bytes = int(sizes.table_bytes), int(sizes.cache_bytes)
         self.table = torch.empty(self.table_bytes, dtype=torch.uint8, device=device)
-        self.cache = torch.empty(max(self.cache_bytes, 256), dtype=torch.uint8, device=device)
+        self.cache = torch.empty(max(self.cache_bytes, 256) + int(cache_guard), dtype=torch.uint8,
+                                 device=device)
         self._handle = None
         rc, h = loopkv_plan_load(d, _ptr(self.table), self.table_bytes, _ptr(self.cache),
                                  self.cache_bytes, _stream_handle(stream))

@@ -216,3 +216,36 @@ def test_decode_replays_from_a_cuda_graph(cuda_device):
         torch.cuda.synchronize()
         assert torch.equal(out, eager)
     plan.check()
+
+
+def test_kernels_write_only_the_layout_bytes(pool, cuda_device):
+    """Guard check (stands in for a memory checker): the cache is filled with
+    a sentinel before a bulk build of every kind; afterwards every byte the
+    canonical layout does not define at the units' lengths still holds the
+    sentinel, and so do the guard bytes after the cache."""
+    import torch
+    from loop_aware_quantized_b200 import Plan
+    from synth.gpu import DeviceGenerator
+    RS = W.RES2
+    spec = _spec(64, (RS, SH, Q4, Q2, BF, Q4), (45, 96, 70), 0.02, n_loops=2, n_layers=3)
+    wl = W.custom(*spec)
+    seqs = [0, 1, 2]
+    guard = 1 << 16
+    plan = Plan(wl.n_loops, wl.n_layers, wl.n_heads, wl.head_dim, wl.capacity[seqs], wl.kinds,
+                wl.tau, cache_guard=guard)
+    plan.cache.fill_(0xA5)
+    gen = DeviceGenerator(wl, cuda_device)
+    GH.build_cache(wl, plan, gen, seqs, wl.lengths)
+    cells = list(range(wl.n_cells))
+    GH.decode_all(wl, plan, gen, seqs, cells, np.tile(wl.lengths, (wl.n_cells, 1)), cuda_device)
+    plan.check()
+    torch.cuda.synchronize()
+    assert (plan.cache[plan.cache_bytes:].cpu().numpy() == 0xA5).all(), "write past the cache"
+    jobs = [(spec, c, b, h, int(wl.lengths[b]), int(wl.lengths[b]), True)
+            for c in cells for b in seqs for h in range(wl.n_heads)]
+    for (c, b, h), ref in zip([(j[1], j[2], j[3]) for j in jobs], pool.map(P.oracle_unit_job, jobs)):
+        got = plan.unit_bytes(c, b, h).cpu().numpy()
+        outside = ref["valid"] == 0
+        bad = np.nonzero(outside & (got != 0xA5))[0]
+        assert bad.size == 0, "cell %d seq %d head %d: %d stray bytes, first at %d" % (
+            c, b, h, bad.size, bad[0])
