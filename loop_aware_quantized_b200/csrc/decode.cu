@@ -29,7 +29,11 @@
 //   combine warp shuffles reduce the per-token partial outputs, shared
 //           memory reduces across warps, DSMEM across the cluster.
 // Each pass loads a warp's next group into registers while the current one
-// is processed and requests its lines into L2 at the same time.
+// is processed and requests its lines into L2 at the same time; with four
+// queries per KV head the value blocks go through shared-memory staging
+// buffers filled by cp.async instead (no registers to spare).  A RES2 unit
+// (template flag, its own launch) runs both passes over its reference and
+// adds its own 2-bit residual planes.
 // No tensor cores: single-query decode is not a dense contraction; the
 // kernel streams the cache once, and the ALU pipe (one logic op per code)
 // is what bounds it in practice.
