@@ -172,3 +172,15 @@ def test_vq_encode_checks_arguments_before_any_device_work(lk):
     assert lk.loopkv_vq_encode(d, pp, 14, fake, fake, fake, None) == 1     # 3 + 14 > 16
     assert lk.loopkv_vq_encode(d, pp, 5, None, fake, fake, None) == 1
     assert lk.loopkv_vq_encode(d, pp, 5, fake, ctypes.c_void_p((1 << 20) + 8), fake, None) == 1
+
+
+def test_header_is_plain_c(tmp_path):
+    # the boundary is a C ABI: the header compiles as ISO C99 with no C++ or
+    # CUDA types, and every declared function is extern "C" for C++ callers
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "use.c"
+    src.write_text('#include "loopkv.h"\nint main(void) { return sizeof(loopkv_vq_desc) == 0; }\n')
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                           "-I", os.path.join(root, "include"), "-c", str(src),
+                           "-o", str(tmp_path / "use.o")])
