@@ -87,11 +87,18 @@ def test_group_decode_matches_oracle(pool, cuda_device, g, D):
 
 
 @pytest.mark.parametrize("g", [2, 4])
-def test_group_residual_cells(pool, cuda_device, g):
+@pytest.mark.parametrize("D", [64, 128])
+def test_group_residual_cells(pool, cuda_device, g, D):
     RS = W.RES2
     lengths = (1, 33, 97, 300)
     for kinds in ((RS, RS, Q4, Q2), (RS, SH, BF, Q4)):
-        _run(_spec(128, kinds, lengths, 0.02), g, pool, cuda_device)
+        _run(_spec(D, kinds, lengths, 0.02), g, pool, cuda_device)
+
+
+@pytest.mark.parametrize("g", [2, 4])
+def test_group_residual_cells_in_clusters(pool, cuda_device, g, monkeypatch):
+    monkeypatch.setenv("LOOPKV_DECODE_SPLIT", "2")
+    _run(_spec(128, (W.RES2, W.RES2, Q4, Q2), (65, 700, 1500), 0.01), g, pool, cuda_device)
 
 
 @pytest.mark.parametrize("g", [2, 4])
