@@ -491,6 +491,9 @@ def bench_vq(args, rank, world):
                            2 * ik.numel() / 1e9), "build_s": build_s},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": (L + 2) * args.steps, "clocks": clocks,
+            "token_head_cells_per_s": float(wl.n_cells * H * world *
+                                            np.sum(n0 + args.warmup + args.steps // 2 + 1)) /
+                                      (ms_per_step / 1000.0),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -782,6 +785,10 @@ def main():
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
+            # attended (position, KV head) pairs decoded per second, all cells
+            "token_head_cells_per_s": float(wl.n_cells * H * world *
+                                            np.sum(n0 + args.warmup + args.steps // 2 + 1)) /
+                                      (ms_per_step / 1000.0),
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
