@@ -250,7 +250,7 @@ def oracle_baseline(config, seconds, seqs_global, g=1):
     for kind in (0, 1, 2, 4):
         cs = [c for c in range(wl.n_cells) if wl.kinds[c] == kind]
         if cs:
-            picks.append((int(rng.choice(cs)), int(rng.integers(wl.batch)),
+            picks.append((int(rng.choice(cs)), int(rng.integers(len(seqs_global))),
                           int(rng.integers(wl.n_heads))))
     units = []
     for c, b, h in picks:
