@@ -48,11 +48,110 @@ __device__ __forceinline__ float canon_zero(float mn) { return mn == 0.0f ? 0.0f
 
 __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
+constexpr int kCodeRow = 16;  // padding bytes of a code-tile row (D + 16 bytes)
+
+// Keys of one 32-token group: per channel over the tokens (x(t, d), fp32),
+// the channel's scale and zero point into kmeta (scale[D] then zero[D]) and
+// its codes into the warp's code tile ([32][D + 16] bytes).  Lane d owns
+// channels d, d + 32, ...
+template <int D, typename X>
+__device__ __forceinline__ void quantize_key_group(X x, uint8_t* codes, float* kmeta, int qmax,
+                                                   int lane) {
+#pragma unroll
+  for (int i = 0; i < D / 32; ++i) {
+    const int d = lane + 32 * i;
+    float mn = x(0, d), mx = mn;
+    for (int t = 1; t < 32; ++t) {
+      mn = fminf(mn, x(t, d));
+      mx = fmaxf(mx, x(t, d));
+    }
+    const float sc = group_scale(mn, mx, qmax);
+    for (int t = 0; t < 32; ++t) codes[t * (D + kCodeRow) + d] = (uint8_t)quant_code(x(t, d), mn, sc, qmax);
+    kmeta[d] = sc;
+    kmeta[D + d] = canon_zero(mn);
+  }
+}
+
+// The code tile's row of token `lane` into the group's key planes: chunk c
+// of 64 channels -> 4 words per plane at hi + c * 512 + lane * 16 (lo: the
+// low plane, 4-bit only; a 2-bit code goes whole into hi).
+template <int D>
+__device__ __forceinline__ void pack_key_planes(const uint8_t* codes, uint8_t* hi, uint8_t* lo,
+                                                bool q4, int lane) {
+#pragma unroll
+  for (int cc = 0; cc < D / 64; ++cc) {
+    uint32_t hiw[4], low[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint4 cw = *reinterpret_cast<const uint4*>(codes + lane * (D + kCodeRow) + 64 * cc + 16 * w);
+      const uint32_t bytes[4] = {cw.x, cw.y, cw.z, cw.w};
+      uint32_t hv = 0, lv = 0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t q = (bytes[j / 4] >> (8 * (j % 4))) & 0xFFu;
+        hv |= ((q4 ? (q >> 2) : q) & 3u) << (2 * j);
+        lv |= (q & 3u) << (2 * j);
+      }
+      hiw[w] = hv;
+      low[w] = lv;
+    }
+    const size_t off = cc * 512 + lane * 16;
+    *reinterpret_cast<uint4*>(hi + off) = make_uint4(hiw[0], hiw[1], hiw[2], hiw[3]);
+    if (q4) *reinterpret_cast<uint4*>(lo + off) = make_uint4(low[0], low[1], low[2], low[3]);
+  }
+}
+
+// Values of one token: per group of 32 channels (v(c), fp32 of channel c)
+// the scale / zero pair and the codes, written as the token's V_hi (V_lo,
+// 4-bit) words and V_meta row (channel 16w + j of a row in bits 2j..2j+1
+// of word w).
+template <int D, typename V>
+__device__ __forceinline__ void quantize_value_row(V v, bool q4, int qmax, uint4* vh, uint4* vl,
+                                                   float4* vm) {
+  uint32_t hiw[D / 16], low[D / 16];
+  float meta[D / 16];
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j) {
+    float mn = v(32 * j), mx = mn;
+#pragma unroll
+    for (int e = 1; e < 32; ++e) {
+      mn = fminf(mn, v(32 * j + e));
+      mx = fmaxf(mx, v(32 * j + e));
+    }
+    const float sc = group_scale(mn, mx, qmax);
+    uint32_t hv0 = 0, lv0 = 0, hv1 = 0, lv1 = 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const uint32_t q = quant_code(v(32 * j + e), mn, sc, qmax);
+      const uint32_t h = (q4 ? (q >> 2) : q) & 3u, l = q & 3u;
+      if (e < 16) {
+        hv0 |= h << (2 * e);
+        lv0 |= l << (2 * e);
+      } else {
+        hv1 |= h << (2 * (e - 16));
+        lv1 |= l << (2 * (e - 16));
+      }
+    }
+    hiw[2 * j] = hv0;
+    hiw[2 * j + 1] = hv1;
+    low[2 * j] = lv0;
+    low[2 * j + 1] = lv1;
+    meta[2 * j] = sc;
+    meta[2 * j + 1] = canon_zero(mn);
+  }
+#pragma unroll
+  for (int i = 0; i < D / 64; ++i) {
+    vh[i] = make_uint4(hiw[4 * i], hiw[4 * i + 1], hiw[4 * i + 2], hiw[4 * i + 3]);
+    if (q4) vl[i] = make_uint4(low[4 * i], low[4 * i + 1], low[4 * i + 2], low[4 * i + 3]);
+    vm[i] = make_float4(meta[4 * i], meta[4 * i + 1], meta[4 * i + 2], meta[4 * i + 3]);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAppendThreads)
 append_kernel(const AppendParams p, const CellList cl) {
   constexpr int TROW = D + 2;     // bf16 per padded tile row
-  constexpr int CROW = D + 16;    // bytes per padded code row
+  constexpr int CROW = D + kCodeRow;  // bytes per padded code row
   extern __shared__ __align__(16) uint8_t sm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint16_t* tk = reinterpret_cast<uint16_t*>(sm) + warp * (2 * 32 * TROW);
@@ -134,97 +233,20 @@ append_kernel(const AppendParams p, const CellList cl) {
     __syncwarp();
 
     // keys: per channel over the 32 tokens
-    float* kmeta = reinterpret_cast<float*>(base + L.k_meta + (size_t)g * 8 * D);
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) {
-      const int d = lane + 32 * i;
-      float mn = bf16f(tk[d]), mx = mn;
-      for (int t = 1; t < 32; ++t) {
-        const float x = bf16f(tk[t * TROW + d]);
-        mn = fminf(mn, x);
-        mx = fmaxf(mx, x);
-      }
-      const float sc = group_scale(mn, mx, qmax);
-      for (int t = 0; t < 32; ++t)
-        codes[t * CROW + d] = (uint8_t)quant_code(bf16f(tk[t * TROW + d]), mn, sc, qmax);
-      kmeta[d] = sc;
-      kmeta[D + d] = canon_zero(mn);
-    }
+    quantize_key_group<D>([&](int t, int d) { return bf16f(tk[t * TROW + d]); }, codes,
+                          reinterpret_cast<float*>(base + L.k_meta + (size_t)g * 8 * D), qmax,
+                          lane);
     __syncwarp();
-    // pack: lane = token; chunk c of 64 channels -> 4 words per plane
-#pragma unroll
-    for (int cc = 0; cc < D / 64; ++cc) {
-      uint32_t hiw[4], low[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint4 cw = *reinterpret_cast<const uint4*>(codes + lane * CROW + 64 * cc + 16 * w);
-        const uint32_t bytes[4] = {cw.x, cw.y, cw.z, cw.w};
-        uint32_t hv = 0, lv = 0;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t q = (bytes[j / 4] >> (8 * (j % 4))) & 0xFFu;
-          hv |= ((q4 ? (q >> 2) : q) & 3u) << (2 * j);
-          lv |= (q & 3u) << (2 * j);
-        }
-        hiw[w] = hv;
-        low[w] = lv;
-      }
-      const size_t off = (size_t)g * 8 * D + cc * 512 + lane * 16;
-      *reinterpret_cast<uint4*>(base + L.k_hi + off) = make_uint4(hiw[0], hiw[1], hiw[2], hiw[3]);
-      if (q4) *reinterpret_cast<uint4*>(base + L.k_lo + off) = make_uint4(low[0], low[1], low[2], low[3]);
-    }
-
+    pack_key_planes<D>(codes, base + L.k_hi + (size_t)g * 8 * D, base + L.k_lo + (size_t)g * 8 * D,
+                       q4, lane);
     // values: lane = token, per group of 32 channels
     {
-      const int t = lane;
-      const size_t tpos = (size_t)g * kGroup + t;
-      uint32_t hiw[D / 16], low[D / 16];
-      float meta[D / 16];
-#pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
-        const uint32_t* row = reinterpret_cast<const uint32_t*>(tv + t * TROW + 32 * j);
-        float mn = bf16f(tv[t * TROW + 32 * j]), mx = mn;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const uint32_t w2 = row[e];
-          const float a = __uint_as_float(w2 << 16), bb = __uint_as_float(w2 & 0xFFFF0000u);
-          mn = fminf(mn, fminf(a, bb));
-          mx = fmaxf(mx, fmaxf(a, bb));
-        }
-        const float sc = group_scale(mn, mx, qmax);
-        uint32_t hv0 = 0, lv0 = 0, hv1 = 0, lv1 = 0;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const uint32_t w2 = row[e];
-          const uint32_t qa = quant_code(__uint_as_float(w2 << 16), mn, sc, qmax);
-          const uint32_t qb = quant_code(__uint_as_float(w2 & 0xFFFF0000u), mn, sc, qmax);
-          // channels 2e and 2e+1 of the group; word 0 holds channels 0..15
-          const int ja = (2 * e) % 16, jb = (2 * e + 1) % 16;
-          const uint32_t ha = (q4 ? (qa >> 2) : qa) & 3u, hb = (q4 ? (qb >> 2) : qb) & 3u;
-          if (e < 8) {
-            hv0 |= (ha << (2 * ja)) | (hb << (2 * jb));
-            lv0 |= ((qa & 3u) << (2 * ja)) | ((qb & 3u) << (2 * jb));
-          } else {
-            hv1 |= (ha << (2 * ja)) | (hb << (2 * jb));
-            lv1 |= ((qa & 3u) << (2 * ja)) | ((qb & 3u) << (2 * jb));
-          }
-        }
-        hiw[2 * j] = hv0;
-        hiw[2 * j + 1] = hv1;
-        low[2 * j] = lv0;
-        low[2 * j + 1] = lv1;
-        meta[2 * j] = sc;
-        meta[2 * j + 1] = canon_zero(mn);
-      }
-      uint4* vh = reinterpret_cast<uint4*>(base + L.v_hi + tpos * (D / 4));
-      uint4* vl = reinterpret_cast<uint4*>(base + L.v_lo + tpos * (D / 4));
-      float4* vm = reinterpret_cast<float4*>(base + L.v_meta + tpos * (D / 4));
-#pragma unroll
-      for (int i = 0; i < D / 64; ++i) {
-        vh[i] = make_uint4(hiw[4 * i], hiw[4 * i + 1], hiw[4 * i + 2], hiw[4 * i + 3]);
-        if (q4) vl[i] = make_uint4(low[4 * i], low[4 * i + 1], low[4 * i + 2], low[4 * i + 3]);
-        vm[i] = make_float4(meta[4 * i], meta[4 * i + 1], meta[4 * i + 2], meta[4 * i + 3]);
-      }
+      const size_t tpos = (size_t)g * kGroup + lane;
+      const uint16_t* row = tv + lane * TROW;
+      quantize_value_row<D>([&](int c) { return bf16f(row[c]); }, q4, qmax,
+                            reinterpret_cast<uint4*>(base + L.v_hi + tpos * (D / 4)),
+                            reinterpret_cast<uint4*>(base + L.v_lo + tpos * (D / 4)),
+                            reinterpret_cast<float4*>(base + L.v_meta + tpos * (D / 4)));
     }
     __syncwarp();
   }
@@ -290,7 +312,7 @@ template <int D>
 __global__ void __launch_bounds__(kAppendThreads)
 append_res2_kernel(const AppendParams p, const CellList cl) {
   constexpr int XROW = D + 1;     // fp32 per padded tile row
-  constexpr int CROW = D + 16;    // bytes per padded code row
+  constexpr int CROW = D + kCodeRow;  // bytes per padded code row
   extern __shared__ __align__(16) uint8_t sm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* xk = reinterpret_cast<float*>(sm) + warp * (2 * 32 * XROW);
@@ -347,69 +369,17 @@ append_res2_kernel(const AppendParams p, const CellList cl) {
     }
     __syncwarp();
 
-    // keys: per channel over the 32 tokens
-    float* kmeta = reinterpret_cast<float*>(base + L.k_meta + (size_t)g * 8 * D);
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) {
-      const int d = lane + 32 * i;
-      float mn = xk[d], mx = mn;
-      for (int t = 1; t < 32; ++t) {
-        mn = fminf(mn, xk[t * XROW + d]);
-        mx = fmaxf(mx, xk[t * XROW + d]);
-      }
-      const float sc = group_scale(mn, mx, 3);
-      for (int t = 0; t < 32; ++t) codes[t * CROW + d] = (uint8_t)quant_code(xk[t * XROW + d], mn, sc, 3);
-      kmeta[d] = sc;
-      kmeta[D + d] = canon_zero(mn);
-    }
+    // keys: per channel over the 32 tokens, then values per token, at 2 bits
+    quantize_key_group<D>([&](int t, int d) { return xk[t * XROW + d]; }, codes,
+                          reinterpret_cast<float*>(base + L.k_meta + (size_t)g * 8 * D), 3, lane);
     __syncwarp();
-    // pack: lane = token; chunk c of 64 channels -> 4 words
-#pragma unroll
-    for (int cc = 0; cc < D / 64; ++cc) {
-      uint32_t hiw[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint32_t hv = 0;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) hv |= ((uint32_t)codes[lane * CROW + 64 * cc + 16 * w + j] & 3u) << (2 * j);
-        hiw[w] = hv;
-      }
-      const size_t off = (size_t)g * 8 * D + cc * 512 + lane * 16;
-      *reinterpret_cast<uint4*>(base + L.k_hi + off) = make_uint4(hiw[0], hiw[1], hiw[2], hiw[3]);
-    }
-
-    // values: lane = token, per group of 32 channels
+    pack_key_planes<D>(codes, base + L.k_hi + (size_t)g * 8 * D, nullptr, false, lane);
     {
-      const int t = lane;
-      const size_t tpos = (size_t)g * kGroup + t;
-      const float* row = xv + t * XROW;
-      uint32_t hiw[D / 16];
-      float meta[D / 16];
-#pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
-        float mn = row[32 * j], mx = mn;
-        for (int e = 1; e < 32; ++e) {
-          mn = fminf(mn, row[32 * j + e]);
-          mx = fmaxf(mx, row[32 * j + e]);
-        }
-        const float sc = group_scale(mn, mx, 3);
-        uint32_t w0 = 0, w1 = 0;
-        for (int e = 0; e < 16; ++e) {
-          w0 |= quant_code(row[32 * j + e], mn, sc, 3) << (2 * e);
-          w1 |= quant_code(row[32 * j + 16 + e], mn, sc, 3) << (2 * e);
-        }
-        hiw[2 * j] = w0;
-        hiw[2 * j + 1] = w1;
-        meta[2 * j] = sc;
-        meta[2 * j + 1] = canon_zero(mn);
-      }
-      uint4* vh = reinterpret_cast<uint4*>(base + L.v_hi + tpos * (D / 4));
-      float4* vm = reinterpret_cast<float4*>(base + L.v_meta + tpos * (D / 4));
-#pragma unroll
-      for (int i = 0; i < D / 64; ++i) {
-        vh[i] = make_uint4(hiw[4 * i], hiw[4 * i + 1], hiw[4 * i + 2], hiw[4 * i + 3]);
-        vm[i] = make_float4(meta[4 * i], meta[4 * i + 1], meta[4 * i + 2], meta[4 * i + 3]);
-      }
+      const size_t tpos = (size_t)g * kGroup + lane;
+      const float* row = xv + lane * XROW;
+      quantize_value_row<D>([&](int c) { return row[c]; }, false, 3,
+                            reinterpret_cast<uint4*>(base + L.v_hi + tpos * (D / 4)), nullptr,
+                            reinterpret_cast<float4*>(base + L.v_meta + tpos * (D / 4)));
     }
     __syncwarp();
   }
