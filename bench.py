@@ -607,6 +607,13 @@ def main():
     cap = np.full(B, int(n0.max()) + total_steps + 32, np.int32)
     cap = (cap + 31) // 32 * 32
     G = args.q_per_kv
+    from loop_aware_quantized_b200 import query_sizes
+    _, need = query_sizes(wl.n_loops, wl.n_layers, H, D, cap, wl.kinds, wl.tau, q_per_kv=G)
+    free, _ = torch.cuda.mem_get_info(dev)
+    if need > 0.92 * free:
+        raise SystemExit("the KV cache of %d sequences needs %.1f GB, %.1f GB are free: pass a "
+                         "smaller --batch (the workload is decoded in sequence sub-batches)"
+                         % (B, need / 1e9, free / 1e9))
     plan = Plan(wl.n_loops, wl.n_layers, H, D, cap, wl.kinds, wl.tau, device=dev, q_per_kv=G)
     gen = DeviceGenerator(wl, dev)
 
