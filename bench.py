@@ -167,10 +167,25 @@ class ClockSampler:
             for name, val in zip(names, parts[4:8]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
+        note = None
         if not sm:
-            return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
-                "reasons": sorted(reasons), "samples": len(sm)}
+            # the timed region was shorter than the sampling interval: one
+            # reading right after it
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index),
+                                      "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits"],
+                                     capture_output=True, text=True, timeout=10).stdout
+                parts = [p.strip() for p in out.strip().split(",")]
+                sm, smax = [float(parts[0])], [float(parts[1])]
+                reasons = {n for n, v in zip(names, parts[4:8]) if v.lower().startswith("active")}
+                note = "timed region shorter than the 200 ms sampling interval: read right after it"
+            except Exception:
+                return None
+        rec = {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
+               "reasons": sorted(reasons), "samples": len(sm) if note is None else 0}
+        if note:
+            rec["note"] = note
+        return rec
 
 
 def workload_text(wl, B, g=1):
