@@ -23,7 +23,8 @@
  *   - a SHARE cell of length n attends over the final loop's stored
  *     positions [0, n-1) (same layer, sequence and head) plus its own
  *     current bf16 key and value;
- *   - softmax scale 1/sqrt(head_dim) unless given; one query per KV head.
+ *   - softmax scale 1/sqrt(head_dim) unless given; one query per KV head,
+ *     or a group of 2 or 4 sharing it (q_per_kv; see loopkv_decode).
  * LOOPKV_BF16 (raw bf16 cells) exists for ablations and checks.
  *
  * Residual cells.  "ResidualQuant: KV Cache Quantization for Looped
