@@ -375,7 +375,7 @@ def bench_vq(args, rank, world):
     n_steps = args.warmup + args.steps
     total_steps = n_steps + (0 if args.no_e2e else args.steps)
     wl.capacity = int(n0.max()) + total_steps   # room for one new token per step
-    gen = VqDeviceGenerator(wl, dev)
+    gen = VqDeviceGenerator(wl, dev, seq0=rank * B)   # weak scaling: disjoint sequences
     t_build = time.perf_counter()
     ik, iv = gen.indices(0, T=int(n0.max())), gen.indices(1, T=int(n0.max()))
     cbk, cbv = gen.codebooks(0), gen.codebooks(1)

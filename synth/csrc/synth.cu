@@ -174,9 +174,10 @@ __global__ void gen_q_kernel(uint16_t* __restrict__ q, const int32_t* __restrict
 constexpr uint32_t kStreamVqIdx = 9, kStreamVqQ = 11;
 
 // out [n_layers][batch][H][cap][D/4] indices of tokens < T (later token
-// slots untouched); which 0 keys, 1 values.
+// slots untouched) of sequences seq0 .. seq0 + batch - 1; which 0 keys, 1
+// values.
 __global__ void gen_vq_idx_kernel(uint8_t* __restrict__ out, int n_layers, int batch, int H, int D,
-                                  int cap, int T, int which, uint32_t seed) {
+                                  int cap, int T, int which, int seq0, uint32_t seed) {
   const int groups = D / 4;
   const size_t total = (size_t)n_layers * batch * H * T * groups;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
@@ -189,15 +190,15 @@ __global__ void gen_vq_idx_kernel(uint8_t* __restrict__ out, int n_layers, int b
     r /= H;
     const int b = (int)(r % batch);
     const int layer = (int)(r / batch);
-    const U4 u = philox((uint32_t)t, (uint32_t)j, (uint32_t)(h + H * b),
+    const U4 u = philox((uint32_t)t, (uint32_t)j, (uint32_t)(h + H * (b + seq0)),
                         (uint32_t)layer | ((uint32_t)which << 16), seed, kStreamVqIdx);
     out[((((size_t)layer * batch + b) * H + h) * cap + t) * groups + j] = (uint8_t)(u.x & 255u);
   }
 }
 
-// q [n_layers][batch][H][D] of one loop.
+// q [n_layers][batch][H][D] of one loop, sequences seq0 ...
 __global__ void gen_vq_q_kernel(uint16_t* __restrict__ q, int n_layers, int batch, int H, int D,
-                                int loop, uint32_t seed, float nscale) {
+                                int loop, int seq0, uint32_t seed, float nscale) {
   const size_t total = (size_t)n_layers * batch * H * D;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -207,8 +208,8 @@ __global__ void gen_vq_q_kernel(uint16_t* __restrict__ q, int n_layers, int batc
     r /= H;
     const int b = (int)(r % batch);
     const int layer = (int)(r / batch);
-    const U4 u = philox((uint32_t)d, (uint32_t)loop, (uint32_t)(h + H * b), (uint32_t)layer, seed,
-                        kStreamVqQ);
+    const U4 u = philox((uint32_t)d, (uint32_t)loop, (uint32_t)(h + H * (b + seq0)),
+                        (uint32_t)layer, seed, kStreamVqQ);
     q[i] = to_bf16_bits(__fmul_rn(2.0f, normal_from(u, nscale)));
   }
 }
@@ -218,25 +219,25 @@ __global__ void gen_vq_q_kernel(uint16_t* __restrict__ q, int n_layers, int batc
 extern "C" {
 
 int synth_gen_vq_idx(uint8_t* out, int n_layers, int batch, int H, int D, int cap, int T,
-                     int which, uint32_t seed, void* stream) {
+                     int which, int seq0, uint32_t seed, void* stream) {
   const size_t total = (size_t)n_layers * batch * H * T * (D / 4);
   if (total == 0) return 0;
   if (T > cap) return -1;
   size_t blocks = (total + 255) / 256;
   if (blocks > 148 * 64) blocks = 148 * 64;
   gen_vq_idx_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      out, n_layers, batch, H, D, cap, T, which, seed);
+      out, n_layers, batch, H, D, cap, T, which, seq0, seed);
   return (int)cudaGetLastError();
 }
 
-int synth_gen_vq_q(uint16_t* q, int n_layers, int batch, int H, int D, int loop, uint32_t seed,
-                   float nscale, void* stream) {
+int synth_gen_vq_q(uint16_t* q, int n_layers, int batch, int H, int D, int loop, int seq0,
+                   uint32_t seed, float nscale, void* stream) {
   const size_t total = (size_t)n_layers * batch * H * D;
   if (total == 0) return 0;
   size_t blocks = (total + 255) / 256;
   if (blocks > 148 * 64) blocks = 148 * 64;
   gen_vq_q_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      q, n_layers, batch, H, D, loop, seed, nscale);
+      q, n_layers, batch, H, D, loop, seq0, seed, nscale);
   return (int)cudaGetLastError();
 }
 

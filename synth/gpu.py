@@ -30,9 +30,9 @@ def _load():
         lib.synth_gen_q.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, ctypes.c_uint32,
                                     ctypes.c_float, P]
         lib.synth_gen_q.restype = I
-        lib.synth_gen_vq_idx.argtypes = [P, I, I, I, I, I, I, I, ctypes.c_uint32, P]
+        lib.synth_gen_vq_idx.argtypes = [P, I, I, I, I, I, I, I, I, ctypes.c_uint32, P]
         lib.synth_gen_vq_idx.restype = I
-        lib.synth_gen_vq_q.argtypes = [P, I, I, I, I, I, ctypes.c_uint32, ctypes.c_float, P]
+        lib.synth_gen_vq_q.argtypes = [P, I, I, I, I, I, I, ctypes.c_uint32, ctypes.c_float, P]
         lib.synth_gen_vq_q.restype = I
         _lib = lib
     return _lib
@@ -109,11 +109,15 @@ def host_kv(wl, cell, b, h, t0, t1):
 
 
 class VqDeviceGenerator:
-    """LoopVQ inputs on a CUDA device (same bits as the host generator)."""
+    """LoopVQ inputs on a CUDA device (same bits as the host generator).
 
-    def __init__(self, wl, device="cuda"):
+    seq0: global id of the first sequence (ranks of a multi-GPU run serve
+    disjoint sequences)."""
+
+    def __init__(self, wl, device="cuda", seq0=0):
         import torch
         self.wl = wl
+        self.seq0 = int(seq0)
         self.device = torch.device(device)
         self.nscale = float(px.NORMAL_SCALE)
 
@@ -127,7 +131,7 @@ class VqDeviceGenerator:
             out = torch.zeros(shape, dtype=torch.uint8, device=self.device)
         s = torch.cuda.current_stream()
         rc = _load().synth_gen_vq_idx(_p(out), wl.n_layers, wl.batch, wl.n_heads, wl.head_dim,
-                                      wl.capacity, int(T), int(which), wl.seed,
+                                      wl.capacity, int(T), int(which), self.seq0, wl.seed,
                                       ctypes.c_void_p(s.cuda_stream))
         s.synchronize()
         assert rc == 0, rc
@@ -150,7 +154,8 @@ class VqDeviceGenerator:
             out = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
         s = torch.cuda.current_stream()
         rc = _load().synth_gen_vq_q(_p(out), wl.n_layers, wl.batch, wl.n_heads, wl.head_dim,
-                                    int(loop), wl.seed, self.nscale, ctypes.c_void_p(s.cuda_stream))
+                                    int(loop), self.seq0, wl.seed, self.nscale,
+                                    ctypes.c_void_p(s.cuda_stream))
         s.synchronize()
         assert rc == 0, rc
         return out

@@ -87,6 +87,12 @@ def test_vq_device_generator_matches_host(cuda_device):
             assert (d[layer, b, h, :50] == W.vq_indices(wl, which, layer, b, h, 0, 50)).all()
     q = gen.queries(3).view(torch.int16).cpu().numpy().view(np.uint16)
     assert (q[1, 2, 1] == W.vq_query(wl, 3, 1, 2, 1)).all()
+    # a rank's generator starts at its first global sequence
+    g5 = VqDeviceGenerator(wl, cuda_device, seq0=5)
+    d = g5.indices(1).cpu().numpy()
+    assert (d[1, 2, 0, :40] == W.vq_indices(wl, 1, 1, 7, 0, 0, 40)).all()
+    q = g5.queries(2).view(torch.int16).cpu().numpy().view(np.uint16)
+    assert (q[0, 1, 1] == W.vq_query(wl, 2, 0, 6, 1)).all()
 
 
 def test_vq_16k_shape_sampled(pool, cuda_device):
