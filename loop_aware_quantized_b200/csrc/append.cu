@@ -159,9 +159,11 @@ append_kernel(const AppendParams p, const CellList cl) {
   uint8_t* codes = sm + kAppendWarps * (2 * 32 * TROW) * 2 + warp * (32 * CROW);
 
   const int H = p.n_heads;
-  const int h = blockIdx.x % H;
-  const int b = (blockIdx.x / H) % p.batch;
-  const int ci = blockIdx.x / (H * p.batch);
+  const int chunk = blockIdx.x % p.chunks;  // this CTA's share of the unit's groups / rows
+  const int unit = blockIdx.x / p.chunks;
+  const int h = unit % H;
+  const int b = (unit / H) % p.batch;
+  const int ci = unit / (H * p.batch);
   const int cell = cl.cell[ci];
   const int n_new = p.n_new[b];
   if (n_new <= 0) return;
@@ -174,7 +176,7 @@ append_kernel(const AppendParams p, const CellList cl) {
   const int kind = c.kind;
   const int n_old = s.len;
   if (n_old < 0 || (kind != LOOPKV_SHARE && n_old + n_new > s.cap)) {
-    if (threadIdx.x == 0) atomicOr(reinterpret_cast<uint32_t*>(p.table), kStatusLength);
+    if (threadIdx.x == 0 && chunk == 0) atomicOr(reinterpret_cast<uint32_t*>(p.table), kStatusLength);
     return;
   }
   uint8_t* base = p.cache + s.offset + (size_t)h * s.stride;
@@ -184,6 +186,7 @@ append_kernel(const AppendParams p, const CellList cl) {
   const uint16_t* vin = p.v + in_off;
 
   if (kind == LOOPKV_SHARE) {
+    if (chunk != 0) return;
     // keep only the last appended token as the current one
     const uint4* ks = reinterpret_cast<const uint4*>(kin + (size_t)(n_new - 1) * D);
     const uint4* vs = reinterpret_cast<const uint4*>(vin + (size_t)(n_new - 1) * D);
@@ -194,10 +197,13 @@ append_kernel(const AppendParams p, const CellList cl) {
     return;
   }
   if (kind == LOOPKV_BF16) {
-    const size_t n16 = (size_t)n_new * D / 8;
+    // rows split evenly over the unit's CTAs
+    const int per = (n_new + p.chunks - 1) / p.chunks;
+    const int t0 = chunk * per, t1 = min(n_new, t0 + per);
     uint4* kd = reinterpret_cast<uint4*>(base + L.raw_k + (size_t)n_old * D * 2);
     uint4* vd = reinterpret_cast<uint4*>(base + L.raw_v + (size_t)n_old * D * 2);
-    for (size_t i = threadIdx.x; i < n16; i += kAppendThreads) {
+    for (size_t i = (size_t)t0 * (D / 8) + threadIdx.x; i < (size_t)max(t1, t0) * (D / 8);
+         i += kAppendThreads) {
       const size_t t = i / (D / 8), cc = i % (D / 8);
       kd[i] = reinterpret_cast<const uint4*>(kin + t * D)[cc];
       vd[i] = reinterpret_cast<const uint4*>(vin + t * D)[cc];
@@ -212,8 +218,12 @@ append_kernel(const AppendParams p, const CellList cl) {
   const int qtok1 = n1 / kGroup * kGroup;
   const uint16_t* resk = reinterpret_cast<const uint16_t*>(base + L.res_k);
   const uint16_t* resv = reinterpret_cast<const uint16_t*>(base + L.res_v);
+  // this CTA's groups; only the first group reads the old residual, and it
+  // is in chunk 0, which also writes the new residual afterwards
+  const int gb = qtok0 / kGroup + chunk * kAppendGroupsPerCta;
+  const int ge = min(qtok1 / kGroup, gb + kAppendGroupsPerCta);
 
-  for (int g = qtok0 / kGroup + warp; g < qtok1 / kGroup; g += kAppendWarps) {
+  for (int g = gb + warp; g < ge; g += kAppendWarps) {
     // gather the group's 32 tokens: residual slots first, then new tokens
     for (int i = lane; i < 32 * (D / 2); i += 32) {
       const int t = i / (D / 2), cc = i % (D / 2);
@@ -251,6 +261,7 @@ append_kernel(const AppendParams p, const CellList cl) {
     __syncwarp();
   }
   __syncthreads();  // flushed groups have read the old residual
+  if (chunk != 0) return;
 
   // remaining tokens go to the residual
   const int r_first = (qtok1 > qtok0) ? qtok1 : n_old;  // first position to write
@@ -320,9 +331,11 @@ append_res2_kernel(const AppendParams p, const CellList cl) {
   uint8_t* codes = sm + (size_t)kAppendWarps * (2 * 32 * XROW) * 4 + warp * (32 * CROW);
 
   const int H = p.n_heads;
-  const int h = blockIdx.x % H;
-  const int b = (blockIdx.x / H) % p.batch;
-  const int ci = blockIdx.x / (H * p.batch);
+  const int chunk = blockIdx.x % p.chunks;  // this CTA's share of the unit's groups
+  const int unit = blockIdx.x / p.chunks;
+  const int h = unit % H;
+  const int b = (unit / H) % p.batch;
+  const int ci = unit / (H * p.batch);
   const int cell = cl.cell[ci];
   const int n_new = p.n_new[b];
   if (n_new <= 0) return;
@@ -342,7 +355,7 @@ append_res2_kernel(const AppendParams p, const CellList cl) {
   const bool ref_ok = rkind == LOOPKV_Q4 || rkind == LOOPKV_Q2 || rkind == LOOPKV_BF16;
   if (c.kind != LOOPKV_RES2 || !ref_ok || n_old < 0 || n1 > s.cap || q1 > ref_pos) {
     // host checks make this unreachable; flag it and leave the unit alone
-    if (threadIdx.x == 0) atomicOr(reinterpret_cast<uint32_t*>(p.table), kStatusLength);
+    if (threadIdx.x == 0 && chunk == 0) atomicOr(reinterpret_cast<uint32_t*>(p.table), kStatusLength);
     return;
   }
   uint8_t* base = p.cache + s.offset + (size_t)h * s.stride;
@@ -355,7 +368,11 @@ append_res2_kernel(const AppendParams p, const CellList cl) {
   const uint16_t* wk = reinterpret_cast<const uint16_t*>(base + L.res_k);
   const uint16_t* wv = reinterpret_cast<const uint16_t*>(base + L.res_v);
 
-  for (int g = q0 / kGroup + warp; g < q1 / kGroup; g += kAppendWarps) {
+  // this CTA's groups; the ones that read the old window (at most two) are
+  // in chunk 0, which also writes the window afterwards
+  const int gb = q0 / kGroup + chunk * kAppendGroupsPerCta;
+  const int ge = min(q1 / kGroup, gb + kAppendGroupsPerCta);
+  for (int g = gb + warp; g < ge; g += kAppendWarps) {
     // residuals of the group's 32 tokens (window slots or new tokens)
     for (int i = lane; i < 32 * D; i += 32) {
       const int t = i / D, d = i % D;
@@ -384,6 +401,7 @@ append_res2_kernel(const AppendParams p, const CellList cl) {
     __syncwarp();
   }
   __syncthreads();  // every group has read its window slots
+  if (chunk != 0) return;
 
   // new tokens past the residual-coded range go to their window slots
   const int first = n_old > q1 ? n_old : q1;
@@ -426,7 +444,7 @@ int launch_append_t(const AppendParams& p, const CellList& cells, cudaStream_t s
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_cells * p.batch * p.n_heads;
-  kern<<<(unsigned)units, kAppendThreads, smem, stream>>>(p, cells);
+  kern<<<(unsigned)(units * p.chunks), kAppendThreads, smem, stream>>>(p, cells);
   return (int)cudaGetLastError();
 }
 

@@ -105,8 +105,12 @@ struct AppendParams {
   const uint16_t* k;           // [n_cells][batch][H][n_new_max][D]
   const uint16_t* v;
   int32_t n_cells, batch, n_heads, n_new_max;
+  int32_t chunks;              // CTAs per unit: a bulk append splits its groups over them
   int32_t n_new[LOOPKV_MAX_BATCH];
 };
+
+// Groups one append CTA quantizes when an append brings many (bulk build).
+constexpr int kAppendGroupsPerCta = 16;
 
 struct DecodeParams {
   const uint8_t* table;

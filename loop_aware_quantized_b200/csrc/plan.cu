@@ -243,6 +243,11 @@ loopkv_status loopkv_append(loopkv_plan* p, const int32_t* h_cells, int32_t n_ce
   ap.n_heads = p->H;
   ap.n_new_max = n_new_max;
   for (int b = 0; b < batch; ++b) ap.n_new[b] = h_n_new[b];
+  // a bulk append (many groups per unit) spreads its groups over several
+  // CTAs per unit: at most ceil((n_new_max + 63) / 32) groups become due
+  const int groups_max = (n_new_max + 2 * kGroup - 1) / kGroup;
+  ap.chunks = (groups_max + kAppendGroupsPerCta - 1) / kAppendGroupsPerCta;
+  if (ap.chunks < 1) ap.chunks = 1;
   int e = 0;
   if (n_plain > 0) {
     ap.n_cells = n_plain;
