@@ -249,65 +249,87 @@ def ncu_traffic(record="decode_traffic.json",
 
 # --------------------------------------------------------- oracle baseline
 
-def oracle_baseline(config, seconds, seqs_global, g=1):
-    """Time the CPU oracle on a fixed sample of the workload's units (each with
-    its g query heads).
+class OracleSample:
+    """A fixed sample of a workload's units in the CPU oracle, built once;
+    rate(seconds) times the oracle's decodes of them on the calling core.
 
-    Returns (cell-steps/s, sample description, cores).  A cell-step is B x H
-    unit decodes, so the rate is units/s divided by B * H.
-    """
-    from oracle import oracle as orc
-    from synth import workloads as W
-    wl = W.make(config)
-    n = int(wl.lengths[0])
-    rng = np.random.default_rng(0)
-    picks = []
-    for kind in (0, 1, 2, 4):
-        cs = [c for c in range(wl.n_cells) if wl.kinds[c] == kind]
-        if cs:
-            picks.append((int(rng.choice(cs)), int(rng.integers(len(seqs_global))),
-                          int(rng.integers(wl.n_heads))))
-    units = []
-    for c, b, h in picks:
-        b = int(seqs_global[b])
-        kind = int(wl.kinds[c])
-        cap = int(wl.capacity[0])
-        own = orc.OracleUnit(kind, wl.head_dim, cap)
-        src = None
-        if kind == 2:
-            k = np.zeros((n + 1, wl.head_dim), np.uint16)
-            v = np.zeros_like(k)
-            k[-1] = W.raw_keys(wl, c, b, h, n, n + 1)[0]
-            v[-1] = W.raw_values(wl, c, b, h, n, n + 1)[0]
-            own.append(k, v)
-            sc = wl.source_cell(c)
-            src = orc.OracleUnit(int(wl.kinds[sc]), wl.head_dim, cap)
-            src.append(W.raw_keys(wl, sc, b, h, 0, n), W.raw_values(wl, sc, b, h, 0, n))
-            q = W.query_group(wl, c, b, h, n + 1, g)
-        else:
-            own.append(W.raw_keys(wl, c, b, h, 0, n + 1), W.raw_values(wl, c, b, h, 0, n + 1))
-            if kind == 4:  # the reference, one token behind in serving order
+    LoopKV workloads: one unit per cell kind of the plan, each with its g
+    query heads, at the workload's context (+1 token, as in a decode step).
+    LoopVQ workloads (vq=True): two units, decoding loop 1."""
+
+    def __init__(self, config, seqs_global, g=1, vq=False):
+        from oracle import oracle as orc
+        from synth import workloads as W
+        self.orc, self.vq, self.g = orc, vq, g
+        self.units = []
+        if vq:
+            wl = self.wl = W.make_vq(config)
+            n = self.n = int(wl.lengths[0])
+            for layer, b, h in ((3, 5, 7), (17, 30, 2)):
+                self.units.append((W.vq_indices(wl, 0, layer, b, h, 0, n),
+                                   W.vq_indices(wl, 1, layer, b, h, 0, n),
+                                   W.vq_codebook(wl, 0, layer, h), W.vq_codebook(wl, 1, layer, h),
+                                   W.vq_query(wl, 1, layer, b, h)))
+            return
+        wl = self.wl = W.make(config)
+        n = int(wl.lengths[0])
+        self.n = n + 1
+        rng = np.random.default_rng(0)
+        picks = []
+        for kind in (0, 1, 2, 4):
+            cs = [c for c in range(wl.n_cells) if wl.kinds[c] == kind]
+            if cs:
+                picks.append((int(rng.choice(cs)), int(rng.integers(len(seqs_global))),
+                              int(rng.integers(wl.n_heads))))
+        for c, b, h in picks:
+            b = int(seqs_global[b])
+            kind = int(wl.kinds[c])
+            cap = int(wl.capacity[0])
+            own = orc.OracleUnit(kind, wl.head_dim, cap)
+            src = None
+            if kind == 2:
+                k = np.zeros((n + 1, wl.head_dim), np.uint16)
+                v = np.zeros_like(k)
+                k[-1] = W.raw_keys(wl, c, b, h, n, n + 1)[0]
+                v[-1] = W.raw_values(wl, c, b, h, n, n + 1)[0]
+                own.append(k, v)
                 sc = wl.source_cell(c)
                 src = orc.OracleUnit(int(wl.kinds[sc]), wl.head_dim, cap)
                 src.append(W.raw_keys(wl, sc, b, h, 0, n), W.raw_values(wl, sc, b, h, 0, n))
-            q = W.query_group(wl, c, b, h, n + 1, g)
-        units.append((own, src, q))
-    done = 0
-    t0 = time.perf_counter()
-    while True:
-        for own, src, q in units:
-            orc.decode_group(own, q, wl.tau, src=src)
-            done += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    rate_units = done / el
-    desc = ("%d oracle decodes of %d sampled units (one per kind of the plan; %d tokens each, "
-            "%d-token contexts%s) in %.1f s on 1 core; cell-steps/s = units/s / (%d seqs x %d "
-            "heads)" % (done, len(units), n + 1, n + 1,
-                        ", %d query heads per unit" % g if g > 1 else "", el, wl.batch,
-                        wl.n_heads))
-    return rate_units / (wl.batch * wl.n_heads), desc, 1
+            else:
+                own.append(W.raw_keys(wl, c, b, h, 0, n + 1), W.raw_values(wl, c, b, h, 0, n + 1))
+                if kind == 4:  # the reference, one token behind in serving order
+                    sc = wl.source_cell(c)
+                    src = orc.OracleUnit(int(wl.kinds[sc]), wl.head_dim, cap)
+                    src.append(W.raw_keys(wl, sc, b, h, 0, n), W.raw_values(wl, sc, b, h, 0, n))
+            self.units.append((own, src, W.query_group(wl, c, b, h, n + 1, g)))
+
+    def rate(self, seconds):
+        """(cell-steps/s, sample description): a cell-step is B x H unit
+        decodes, so the rate is units/s divided by B * H."""
+        wl, orc = self.wl, self.orc
+        done = 0
+        t0 = time.perf_counter()
+        while True:
+            for u in self.units:
+                if self.vq:
+                    orc.vq_decode(*u, 1, wl.n_loops)
+                else:
+                    orc.decode_group(u[0], u[2], wl.tau, src=u[1])
+                done += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+        if self.vq:
+            desc = ("%d oracle LoopVQ decodes of %d sampled units (%d coded tokens each) in %.1f s "
+                    "on 1 core" % (done, len(self.units), self.n, el))
+        else:
+            desc = ("%d oracle decodes of %d sampled units (one per kind of the plan; %d tokens "
+                    "each%s) in %.1f s on 1 core" % (
+                        done, len(self.units), self.n,
+                        ", %d query heads per unit" % self.g if self.g > 1 else "", el))
+        desc += "; cell-steps/s = units/s / (%d seqs x %d heads)" % (wl.batch, wl.n_heads)
+        return done / el / (wl.batch * wl.n_heads), desc
 
 
 # --------------------------------------------------------------- LoopVQ leg
@@ -322,30 +344,14 @@ def vq_unit_bytes(n, D):
     return n * (D // 2) + 2 * 256 * 4 * 4 + 2 * D + 4 * D
 
 
-def oracle_baseline_vq(config, seconds, loop=1):
-    """Time the CPU oracle's LoopVQ decode on sampled units: (cell-steps/s, sample, cores)."""
-    from oracle import oracle as orc
-    from synth import workloads as W
-    wl = W.make_vq(config)
-    n = int(wl.lengths[0])
-    units = []
-    for layer, b, h in ((3, 5, 7), (17, 30, 2)):
-        units.append((W.vq_indices(wl, 0, layer, b, h, 0, n), W.vq_indices(wl, 1, layer, b, h, 0, n),
-                      W.vq_codebook(wl, 0, layer, h), W.vq_codebook(wl, 1, layer, h),
-                      W.vq_query(wl, loop, layer, b, h)))
-    done = 0
-    t0 = time.perf_counter()
-    while True:
-        for ik, iv, ck, cv, q in units:
-            orc.vq_decode(ik, iv, ck, cv, q, loop, wl.n_loops)
-            done += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    desc = ("%d oracle LoopVQ decodes of %d sampled units (%d coded tokens each) in %.1f s on 1 "
-            "core; cell-steps/s = units/s / (%d seqs x %d heads)" % (done, len(units), n, el,
-                                                                    wl.batch, wl.n_heads))
-    return done / el / (wl.batch * wl.n_heads), desc, 1
+def oracle_baseline(config, seconds, seqs_global, g=1):
+    """The oracle on one core: (cell-steps/s, sample description, cores)."""
+    return OracleSample(config, seqs_global, g).rate(seconds) + (1,)
+
+
+def oracle_baseline_vq(config, seconds):
+    """The oracle's LoopVQ decode on one core: (cell-steps/s, sample, cores)."""
+    return OracleSample(config, [], vq=True).rate(seconds) + (1,)
 
 
 def bench_vq(args, rank, world):
@@ -485,8 +491,11 @@ def bench_vq(args, rank, world):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, cores = oracle_baseline_vq(args.config, args.cpu_seconds)
-        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        v1, desc, _ = oracle_baseline_vq(args.config, args.cpu_seconds)
+        v, cores = oracle_all_cores(args.config, [], vq=True, cpu_seconds=2 * args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": "one process per host core, each timing its own sample like this one: "
+                         "%s; on one core alone: %.4g cell-steps/s" % (desc, v1)}
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -515,68 +524,89 @@ def bench_vq(args, rank, world):
         dist.destroy_process_group()
 
 
+# ------------------------------------------- the oracle on every host core
+
+_SAMPLE = None
+
+
+def _sample_init(config, seqs_global, g, vq):
+    global _SAMPLE
+    _SAMPLE = OracleSample(config, seqs_global, g, vq)
+
+
+def _sample_rate(seconds):
+    return _SAMPLE.rate(seconds)[0]
+
+
+class OracleAllCores:
+    """The oracle as it stands in one process per host core (spawned, so no
+    CUDA state is inherited), each with its own copy of the sample, built
+    once; rate(seconds) times them together and sums their cell-steps/s."""
+
+    def __init__(self, config, seqs_global, g=1, vq=False):
+        import multiprocessing as mp
+        self.cores = os.cpu_count() or 1
+        self.pool = mp.get_context("spawn").Pool(
+            self.cores, initializer=_sample_init, initargs=(config, list(seqs_global), g, vq))
+
+    def rate(self, seconds):
+        return float(sum(self.pool.map(_sample_rate, [seconds] * self.cores, chunksize=1)))
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def oracle_all_cores(config, seqs_global, g=1, vq=False, cpu_seconds=24.0):
+    """(summed cell-steps/s, cores) with each core timing its sample for
+    max(1 s, cpu_seconds / cores)."""
+    oc = OracleAllCores(config, seqs_global, g, vq)
+    try:
+        return oc.rate(max(1.0, cpu_seconds / oc.cores)), oc.cores
+    finally:
+        oc.close()
+
+
 # -------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle, one process per host core, timed on
+    bounded samples of the same workload (rank 0 only)."""
     if rank != 0:
         return
-    if args.config in VQ_CONFIGS:
-        return run_reference_vq(args)
     from synth import workloads as W
-    wl = W.make(args.config)
-    budget = max(1.0, min(args.cpu_seconds, 6.0))
-    vals = []
-    desc = ""
-    for _ in range(args.warmup):
-        oracle_baseline(args.config, 0.5, list(range(wl.batch)), args.q_per_kv)
+    vq = args.config in VQ_CONFIGS
+    if vq:
+        wl = W.make_vq(args.config)
+        text = "%s: LoopVQ decode (%s)" % (wl.name, wl.description)
+    else:
+        wl = W.make(args.config)
+        text = workload_text(wl, wl.batch, args.q_per_kv)
+    seqs = list(range(wl.batch))
+    one = OracleSample(args.config, seqs, args.q_per_kv, vq)
+    v1, desc = one.rate(max(1.0, min(args.cpu_seconds, 4.0)))
     t_all = time.perf_counter()
-    for _ in range(args.steps):
-        v, desc, cores = oracle_baseline(args.config, budget / max(1, args.steps) + 0.2,
-                                         list(range(wl.batch)), args.q_per_kv)
-        vals.append(v)
+    oc = OracleAllCores(args.config, seqs, args.q_per_kv, vq)
+    try:
+        per = max(1.0, min(args.cpu_seconds, 6.0) / max(1, args.steps))
+        for _ in range(args.warmup):
+            oc.rate(0.3)
+        vals = [oc.rate(per) for _ in range(args.steps)]
+    finally:
+        oc.close()
     wall = time.perf_counter() - t_all
     value = float(np.mean(vals))
+    sample = ("one process per host core (%d), each timing its own copy of this sample for "
+              "%.1f s per step: %s; on one core alone: %.4g cell-steps/s" % (oc.cores, per, desc, v1))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * wl.n_cells / value if value > 0 else None,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": workload_text(wl, wl.batch, args.q_per_kv),
-                   "impl": "CPU oracle (fp64 C++)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": desc},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        "wall_s": wall,
-    }
-    print(json.dumps(line), flush=True)
-
-
-# ------------------------------------------------------------------ main arm
-
-def run_reference_vq(args):
-    from synth import workloads as W
-    wl = W.make_vq(args.config)
-    budget = max(1.0, min(args.cpu_seconds, 6.0))
-    for _ in range(args.warmup):
-        oracle_baseline_vq(args.config, 0.3)
-    vals, desc = [], ""
-    t_all = time.perf_counter()
-    for _ in range(args.steps):
-        v, desc, cores = oracle_baseline_vq(args.config, budget / max(1, args.steps) + 0.2)
-        vals.append(v)
-    wall = time.perf_counter() - t_all
-    value = float(np.mean(vals))
-    line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * wl.n_cells / value if value > 0 else None,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic",
-        "config": {"workload": "%s: LoopVQ decode (%s)" % (wl.name, wl.description),
-                   "impl": "CPU oracle (fp64 C++)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": desc},
+        "config": {"workload": text, "impl": "CPU oracle (fp64 C++)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oc.cores, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": wall,
     }
@@ -787,8 +817,11 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, cores = oracle_baseline(args.config, args.cpu_seconds, seqs, G)
-        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        v1, desc, _ = oracle_baseline(args.config, args.cpu_seconds, seqs, G)
+        v, cores = oracle_all_cores(args.config, seqs, G, cpu_seconds=2 * args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": "one process per host core, each timing its own sample like this one: "
+                         "%s; on one core alone: %.4g cell-steps/s" % (desc, v1)}
 
     if rank == 0:
         line = {
