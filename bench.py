@@ -253,8 +253,9 @@ class OracleSample:
     """A fixed sample of a workload's units in the CPU oracle, built once;
     rate(seconds) times the oracle's decodes of them on the calling core.
 
-    LoopKV workloads: one unit per cell kind of the plan, each with its g
-    query heads, at the workload's context (+1 token, as in a decode step).
+    LoopKV workloads: one unit per cell kind the plan has (Q4, Q2, SHARE,
+    BF16, RES2), each with its g query heads, at the workload's context (+1
+    token, as in a decode step).
     LoopVQ workloads (vq=True): two units, decoding loop 1."""
 
     def __init__(self, config, seqs_global, g=1, vq=False):
@@ -276,11 +277,12 @@ class OracleSample:
         self.n = n + 1
         rng = np.random.default_rng(0)
         picks = []
-        for kind in (0, 1, 2, 4):
+        for kind in (0, 1, 2, 3, 4):
             cs = [c for c in range(wl.n_cells) if wl.kinds[c] == kind]
             if cs:
                 picks.append((int(rng.choice(cs)), int(rng.integers(len(seqs_global))),
                               int(rng.integers(wl.n_heads))))
+        self.cells = [c for c, _, _ in picks]
         for c, b, h in picks:
             b = int(seqs_global[b])
             kind = int(wl.kinds[c])
@@ -305,31 +307,44 @@ class OracleSample:
             self.units.append((own, src, W.query_group(wl, c, b, h, n + 1, g)))
 
     def rate(self, seconds):
-        """(cell-steps/s, sample description): a cell-step is B x H unit
-        decodes, so the rate is units/s divided by B * H."""
+        """(cell-steps/s, sample description), extrapolated from the sample: a
+        cell-step decodes B x H units of one cell, so a step of the workload
+        takes sum over its cells of B * H * (mean time of the sampled unit of
+        that cell's kind), and the rate is cells / that time."""
         wl, orc = self.wl, self.orc
         done = 0
+        spent = [0.0] * len(self.units)
+        calls = [0] * len(self.units)
         t0 = time.perf_counter()
         while True:
-            for u in self.units:
+            for i, u in enumerate(self.units):
+                t1 = time.perf_counter()
                 if self.vq:
                     orc.vq_decode(*u, 1, wl.n_loops)
                 else:
                     orc.decode_group(u[0], u[2], wl.tau, src=u[1])
+                spent[i] += time.perf_counter() - t1
+                calls[i] += 1
                 done += 1
             el = time.perf_counter() - t0
             if el >= seconds:
                 break
+        per_unit = [t / c for t, c in zip(spent, calls)]
         if self.vq:
+            unit_s = float(np.mean(per_unit))
+            step_s = wl.n_cells * wl.batch * wl.n_heads * unit_s
             desc = ("%d oracle LoopVQ decodes of %d sampled units (%d coded tokens each) in %.1f s "
                     "on 1 core" % (done, len(self.units), self.n, el))
         else:
+            by_kind = {int(self.wl.kinds[c]): t for c, t in zip(self.cells, per_unit)}
+            step_s = sum(by_kind[int(k)] for k in wl.kinds) * wl.batch * wl.n_heads
             desc = ("%d oracle decodes of %d sampled units (one per kind of the plan; %d tokens "
                     "each%s) in %.1f s on 1 core" % (
                         done, len(self.units), self.n,
                         ", %d query heads per unit" % self.g if self.g > 1 else "", el))
-        desc += "; cell-steps/s = units/s / (%d seqs x %d heads)" % (wl.batch, wl.n_heads)
-        return done / el / (wl.batch * wl.n_heads), desc
+        desc += ("; extrapolated: one step = %d cells x %d seqs x %d heads of units, each at its "
+                 "kind's sampled time" % (wl.n_cells, wl.batch, wl.n_heads))
+        return wl.n_cells / step_s, desc
 
 
 # --------------------------------------------------------------- LoopVQ leg
