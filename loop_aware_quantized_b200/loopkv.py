@@ -219,6 +219,52 @@ def _check(rc, where):
         raise LoopKVError(rc, where)
 
 
+def _invalid(where, what):
+    return LoopKVError(1, "%s: %s" % (where, what))
+
+
+def _need(t, where, name, dtypes, shape=None, ndim=None, device=None, optional=False):
+    """Check a tensor argument before its pointer reaches the library: a
+    contiguous CUDA tensor of one of ``dtypes``, with ``shape`` (or ``ndim``
+    dimensions) and on ``device`` when given.  The library sees only pointers,
+    so these are the checks it cannot make; a failure raises LoopKVError
+    with LOOPKV_ERR_INVALID_ARG and launches nothing."""
+    import torch
+    if t is None:
+        if optional:
+            return
+        raise _invalid(where, "%s is required" % name)
+    if not isinstance(t, torch.Tensor):
+        raise _invalid(where, "%s must be a torch tensor, not %s" % (name, type(t).__name__))
+    if not t.is_cuda:
+        raise _invalid(where, "%s must be on a CUDA device, not %s" % (name, t.device))
+    if device is not None and t.device != device:
+        raise _invalid(where, "%s is on %s, expected %s" % (name, t.device, device))
+    if t.dtype not in dtypes:
+        raise _invalid(where, "%s must be %s, not %s" % (
+            name, " or ".join(str(d) for d in dtypes), t.dtype))
+    if not t.is_contiguous():
+        raise _invalid(where, "%s must be contiguous" % name)
+    if ndim is not None and t.dim() != ndim:
+        raise _invalid(where, "%s must have %d dimensions, not %d" % (name, ndim, t.dim()))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise _invalid(where, "%s must have shape %s, not %s" % (
+            name, tuple(shape), tuple(t.shape)))
+
+
+def _host_ints(a, where, name, size):
+    a = np.ascontiguousarray(a, dtype=np.int32)
+    if a.size != size:
+        raise _invalid(where, "%s must hold %d values, not %d" % (name, size, a.size))
+    return a
+
+
+def _int_dtypes():
+    import torch
+    u32 = getattr(torch, "uint32", None)
+    return (torch.int32,) if u32 is None else (torch.int32, u32)
+
+
 def make_desc(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau, sm_scale=0.0,
               q_per_kv=1):
     """Build a loopkv_plan_desc; returns (desc, keepalive arrays)."""
@@ -292,14 +338,18 @@ class Plan:
     def append(self, cells, k, v, n_new=None, stream=None):
         """k, v: bf16 [n_cells, batch, H, n_new_max, D] on the device."""
         import torch
-        cells = np.ascontiguousarray(cells, dtype=np.int32)
-        assert k.dtype == torch.bfloat16 and v.dtype == torch.bfloat16
-        assert k.is_contiguous() and v.is_contiguous() and k.shape == v.shape
+        where = "Plan.append"
+        cells = np.ascontiguousarray(cells, dtype=np.int32).reshape(-1)
+        dev = self.cache.device
+        _need(k, where, "k", (torch.bfloat16,), ndim=5, device=dev)
         nc, batch, H, nmax, D = k.shape
-        assert nc == cells.size and H == self.n_heads and D == self.head_dim
+        if nc != cells.size or H != self.n_heads or D != self.head_dim:
+            raise _invalid(where, "k has shape %s; expected (%d cells, batch, %d heads, n_new_max, "
+                                  "%d)" % (tuple(k.shape), cells.size, self.n_heads, self.head_dim))
+        _need(v, where, "v", (torch.bfloat16,), shape=k.shape, device=dev)
         if n_new is None:
             n_new = np.full(batch, nmax, np.int32)
-        n_new = np.ascontiguousarray(n_new, dtype=np.int32)
+        n_new = _host_ints(n_new, where, "n_new", batch)
         rc = loopkv_append(self._handle, _np_ptr(cells), int(cells.size), int(batch),
                            _np_ptr(n_new), int(nmax), _ptr(k), _ptr(v), _stream_handle(stream))
         _check(rc, "loopkv_append")
@@ -310,16 +360,29 @@ class Plan:
         out (fp32, same shape).  lse: [n_cells, batch, H(, q_per_kv)]; mask
         and nsel are per KV head."""
         import torch
-        cells = np.ascontiguousarray(cells, dtype=np.int32)
-        assert q.dtype == torch.bfloat16 and q.is_contiguous()
-        if q.dim() == 5:
-            nc, batch, H, g, D = q.shape
-        else:
-            (nc, batch, H, D), g = q.shape, 1
-        assert g == self.q_per_kv
-        assert nc == cells.size and H == self.n_heads and D == self.head_dim
+        where = "Plan.decode"
+        cells = np.ascontiguousarray(cells, dtype=np.int32).reshape(-1)
+        dev = self.cache.device
+        _need(q, where, "q", (torch.bfloat16,), device=dev)
+        g = self.q_per_kv
+        batch = q.shape[1] if q.dim() > 1 else -1
+        want = (cells.size, batch, self.n_heads, g, self.head_dim)
+        if tuple(q.shape) != want and (g > 1 or tuple(q.shape) != want[:3] + want[4:]):
+            raise _invalid(where, "q has shape %s; expected (cells %d, batch, KV heads %d, "
+                                  "query heads %d, head dim %d)%s" % (
+                                      tuple(q.shape), cells.size, self.n_heads, g, self.head_dim,
+                                      ", the query-head axis optional" if g == 1 else ""))
+        nc, H = cells.size, self.n_heads
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        _need(out, where, "out", (torch.float32,), shape=q.shape, device=dev)
+        _need(lse, where, "lse", (torch.float32,), shape=q.shape[:-1], device=dev, optional=True)
+        _need(nsel, where, "nsel", (torch.int32,), shape=(nc, batch, H), device=dev,
+              optional=True)
+        _need(mask, where, "mask", _int_dtypes(), ndim=4, device=dev, optional=True)
+        if mask is not None and tuple(mask.shape[:3]) != (nc, batch, H):
+            raise _invalid(where, "mask has shape %s; expected (%d, %d, %d, words)" % (
+                tuple(mask.shape), nc, batch, H))
         mask_words = 0 if mask is None else int(mask.shape[-1])
         rc = loopkv_decode(self._handle, _np_ptr(cells), int(cells.size), int(batch), _ptr(q),
                            _ptr(out), _ptr(lse), _ptr(mask), mask_words, _ptr(nsel),
@@ -328,9 +391,12 @@ class Plan:
         return out
 
     def set_lengths(self, cells, lengths, stream=None):
-        cells = np.ascontiguousarray(cells, dtype=np.int32)
+        cells = np.ascontiguousarray(cells, dtype=np.int32).reshape(-1)
         lengths = np.ascontiguousarray(lengths, dtype=np.int32)
-        batch = lengths.shape[-1]
+        batch = lengths.shape[-1] if lengths.ndim else 0
+        if lengths.size != cells.size * batch:
+            raise _invalid("Plan.set_lengths", "lengths must be [cells][batch], got shape %s for "
+                                               "%d cells" % (lengths.shape, cells.size))
         rc = loopkv_set_lengths(self._handle, _np_ptr(cells), int(cells.size), int(batch),
                                 _np_ptr(lengths), _stream_handle(stream))
         _check(rc, "loopkv_set_lengths")
@@ -360,8 +426,11 @@ def plan_optimize(n_loops, n_layers, head_dim, damage, damage_budget, storage_bu
     a storage budget.  damage: int [n_loops * n_layers, 3] (Q4, Q2, SHARE);
     storage_budget: bytes per cached token and KV head.  Returns (kinds,
     {"reads", "damage", "storage"}); raises LoopKVError when nothing fits."""
-    dmg = np.ascontiguousarray(damage, dtype=np.int32).reshape(-1, 3)
-    assert dmg.shape[0] == n_loops * n_layers
+    dmg = np.ascontiguousarray(damage, dtype=np.int32)
+    if dmg.size != 3 * n_loops * n_layers:
+        raise _invalid("plan_optimize", "damage must be [%d cells][3], got shape %s" % (
+            n_loops * n_layers, dmg.shape))
+    dmg = dmg.reshape(-1, 3)
     d = loopkv_planner_desc()
     d.n_loops, d.n_layers, d.head_dim = n_loops, n_layers, head_dim
     d.damage = dmg.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
@@ -381,20 +450,27 @@ def vq_decode(loop, lengths, idx_k, idx_v, cb_k, cb_v, q, out=None, lse=None, sm
     fp32 [n_layers, H, 256, 4 * n_loops]; q: bf16 [n_layers, batch, H, D];
     lengths: host [batch] coded tokens.  Returns out (fp32, q's shape)."""
     import torch
-    assert idx_k.dtype == torch.uint8 and idx_v.shape == idx_k.shape
-    assert cb_k.dtype == torch.float32 and cb_v.shape == cb_k.shape
-    assert q.dtype == torch.bfloat16
-    for t in (idx_k, idx_v, cb_k, cb_v, q):
-        assert t.is_contiguous()
-    n_layers, batch, H, cap, groups = idx_k.shape
-    D = q.shape[-1]
-    assert groups * 4 == D and q.shape == (n_layers, batch, H, D)
-    assert cb_k.shape[:3] == (n_layers, H, 256) and cb_k.shape[3] % 4 == 0
+    where = "vq_decode"
+    _need(q, where, "q", (torch.bfloat16,), ndim=4)
+    dev = q.device
+    n_layers, batch, H, D = q.shape
+    _need(idx_k, where, "idx_k", (torch.uint8,), ndim=5, device=dev)
+    cap = idx_k.shape[3]
+    if tuple(idx_k.shape) != (n_layers, batch, H, cap, D // 4) or D % 4:
+        raise _invalid(where, "idx_k has shape %s; expected (%d, %d, %d, capacity, %d)" % (
+            tuple(idx_k.shape), n_layers, batch, H, D // 4))
+    _need(idx_v, where, "idx_v", (torch.uint8,), shape=idx_k.shape, device=dev)
+    _need(cb_k, where, "cb_k", (torch.float32,), ndim=4, device=dev)
+    if tuple(cb_k.shape[:3]) != (n_layers, H, 256) or cb_k.shape[3] % 4:
+        raise _invalid(where, "cb_k has shape %s; expected (%d, %d, 256, 4 * loops)" % (
+            tuple(cb_k.shape), n_layers, H))
+    _need(cb_v, where, "cb_v", (torch.float32,), shape=cb_k.shape, device=dev)
     if out is None:
-        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    _need(out, where, "out", (torch.float32,), shape=q.shape, device=dev)
+    _need(lse, where, "lse", (torch.float32,), shape=q.shape[:-1], device=dev, optional=True)
     d = loopkv_vq_desc(cb_k.shape[3] // 4, n_layers, H, D, batch, cap, float(sm_scale))
-    lengths = np.ascontiguousarray(lengths, dtype=np.int32)
-    assert lengths.size == batch
+    lengths = _host_ints(lengths, where, "lengths", batch)
     rc = loopkv_vq_decode(d, int(loop), _np_ptr(lengths), _ptr(idx_k), _ptr(idx_v), _ptr(cb_k),
                           _ptr(cb_v), _ptr(q), _ptr(out), _ptr(lse), _stream_handle(stream))
     _check(rc, "loopkv_vq_decode")
@@ -407,15 +483,17 @@ def vq_encode(positions, x, cb, idx, stream=None):
     (uint8 [n_layers, batch, H, capacity, D/4]) at positions[b] + i, using cb
     (fp32 [n_layers, H, 256, 4 * n_loops]).  Returns idx."""
     import torch
-    assert x.dtype == torch.bfloat16 and cb.dtype == torch.float32 and idx.dtype == torch.uint8
-    for t in (x, cb, idx):
-        assert t.is_contiguous()
+    where = "vq_encode"
+    _need(x, where, "x", (torch.bfloat16,), ndim=6)
+    dev = x.device
     L, n_layers, batch, H, n_new, D = x.shape
-    assert idx.shape == (n_layers, batch, H, idx.shape[3], D // 4)
-    assert cb.shape == (n_layers, H, 256, 4 * L)
+    _need(idx, where, "idx", (torch.uint8,), ndim=5, device=dev)
+    if tuple(idx.shape) != (n_layers, batch, H, idx.shape[3], D // 4) or D % 4:
+        raise _invalid(where, "idx has shape %s; expected (%d, %d, %d, capacity, %d)" % (
+            tuple(idx.shape), n_layers, batch, H, D // 4))
+    _need(cb, where, "cb", (torch.float32,), shape=(n_layers, H, 256, 4 * L), device=dev)
     d = loopkv_vq_desc(L, n_layers, H, D, batch, idx.shape[3], 0.0)
-    positions = np.ascontiguousarray(positions, dtype=np.int32)
-    assert positions.size == batch
+    positions = _host_ints(positions, where, "positions", batch)
     rc = loopkv_vq_encode(d, _np_ptr(positions), int(n_new), _ptr(x), _ptr(cb), _ptr(idx),
                           _stream_handle(stream))
     _check(rc, "loopkv_vq_encode")

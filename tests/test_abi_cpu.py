@@ -184,3 +184,38 @@ def test_header_is_plain_c(tmp_path):
     subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
                            "-I", os.path.join(root, "include"), "-c", str(src),
                            "-o", str(tmp_path / "use.o")])
+
+
+def test_binding_checks_tensors_before_passing_pointers(lk):
+    # the library sees only pointers: the binding refuses host tensors, wrong
+    # dtypes, layouts and shapes itself, with LOOPKV_ERR_INVALID_ARG and no
+    # call into the library (these inputs never reach a device)
+    import torch
+    where = "test"
+    host = torch.zeros((2, 3, 4), dtype=torch.float32)
+    with pytest.raises(lk.LoopKVError) as e:
+        lk._need(host, where, "out", (torch.float32,))
+    assert e.value.status == 1 and "CUDA" in str(e.value)
+    with pytest.raises(lk.LoopKVError) as e:
+        lk._need(np.zeros(3), where, "out", (torch.float32,))
+    assert e.value.status == 1 and "torch tensor" in str(e.value)
+    with pytest.raises(lk.LoopKVError):
+        lk._need(None, where, "q", (torch.bfloat16,))
+    lk._need(None, where, "lse", (torch.float32,), optional=True)
+    with pytest.raises(lk.LoopKVError) as e:
+        lk._host_ints([1, 2, 3], where, "lengths", 2)
+    assert "2 values" in str(e.value)
+    assert list(lk._host_ints((4, 5), where, "lengths", 2)) == [4, 5]
+    # the public LoopVQ calls run the same checks first
+    ik = torch.zeros((2, 3, 2, 16, 32), dtype=torch.uint8)
+    cb = torch.zeros((2, 2, 256, 16), dtype=torch.float32)
+    q = torch.zeros((2, 3, 2, 128), dtype=torch.bfloat16)
+    with pytest.raises(lk.LoopKVError) as e:
+        lk.vq_decode(0, np.array([1, 1, 1]), ik, ik, cb, cb, q)
+    assert e.value.status == 1
+    x = torch.zeros((4, 2, 3, 2, 1, 128), dtype=torch.bfloat16)
+    with pytest.raises(lk.LoopKVError) as e:
+        lk.vq_encode(np.zeros(3, np.int32), x, cb, ik)
+    assert e.value.status == 1
+    with pytest.raises(lk.LoopKVError):
+        lk.plan_optimize(2, 2, 64, np.zeros((3, 3)), 1, 1000)   # damage for 3 of 4 cells
