@@ -17,6 +17,13 @@ LIB_PATH = os.path.join(_HERE, "libloopkv_synth.so")
 _lib = None
 
 
+def _ok(rc):
+    """A generator call's status: 0, -1 for a range the output cannot hold, or
+    the CUDA error its launch returned."""
+    if rc != 0:
+        raise RuntimeError("synthetic input generator failed with status %d" % rc)
+
+
 def _load():
     global _lib
     if _lib is None:
@@ -77,7 +84,7 @@ class DeviceGenerator:
                                   wl.seed, self.nscale, ctypes.c_void_p(s.cuda_stream))
         s.synchronize()
         del d_cells, d_seqs, d_t0
-        assert rc == 0, rc
+        _ok(rc)
         return k, v
 
     def queries(self, cells, seqs, lens, out=None, stream=None, g=1):
@@ -99,7 +106,7 @@ class DeviceGenerator:
                                  ctypes.c_void_p(s.cuda_stream))
         s.synchronize()
         del d_cells, d_srcs, d_seqs, d_lens
-        assert rc == 0, rc
+        _ok(rc)
         return out
 
 
@@ -134,7 +141,7 @@ class VqDeviceGenerator:
                                       wl.capacity, int(T), int(which), self.seq0, wl.seed,
                                       ctypes.c_void_p(s.cuda_stream))
         s.synchronize()
-        assert rc == 0, rc
+        _ok(rc)
         return out
 
     def codebooks(self, which):
@@ -157,5 +164,5 @@ class VqDeviceGenerator:
                                     int(loop), self.seq0, wl.seed, self.nscale,
                                     ctypes.c_void_p(s.cuda_stream))
         s.synchronize()
-        assert rc == 0, rc
+        _ok(rc)
         return out
