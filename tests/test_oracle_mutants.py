@@ -74,6 +74,17 @@ MUTANTS = [
     ("residual window slot not modulo 64",
      "const size_t slot = static_cast<size_t>(t % kResWindow) * D * 2;",
      "const size_t slot = static_cast<size_t>(t - u->qtok()) * D * 2;"),
+    ("softmax scale 1/D", "sm_scale = 1.0 / std::sqrt(static_cast<double>(D));",
+     "sm_scale = 1.0 / static_cast<double>(D);"),
+    ("lse without the running max", "const double l = smax + std::log(sum);",
+     "const double l = std::log(sum);"),
+    ("bf16 residual keys read the values",
+     "khat[d] = bf16_to_float(data->rk[static_cast<size_t>(r) * D + d]);",
+     "khat[d] = bf16_to_float(data->rv[static_cast<size_t>(r) * D + d]);"),
+    ("SHARE current value read from its key", "v = bf16_to_float(own->cv[d]);",
+     "v = bf16_to_float(own->ck[d]);"),
+    ("mask bits in reverse order", "mask[pos / kG] |= 1u << (pos % kG);",
+     "mask[pos / kG] |= 1u << (kG - 1 - pos % kG);"),
 ]
 
 
