@@ -85,6 +85,15 @@ MUTANTS = [
      "v = bf16_to_float(own->ck[d]);"),
     ("mask bits in reverse order", "mask[pos / kG] |= 1u << (pos % kG);",
      "mask[pos / kG] |= 1u << (kG - 1 - pos % kG);"),
+    ("vq scores skip the softmax scale", "    s[t] = sm_scale * acc;", "    s[t] = acc;"),
+    ("vq value weights unnormalised", "const double p = std::exp(s[t] - l);",
+     "const double p = std::exp(s[t] - smax);"),
+    ("vq encode distance without the square", "const float sq = diff * diff;",
+     "const float sq = std::fabs(diff);"),
+    ("planner: storage budget ignored", "if (dm <= damage_budget && st <= storage_budget_q) {",
+     "if (dm <= damage_budget) {"),
+    ("planner: 2-bit reads priced as 4-bit", "else if (k == 1) { st += 4; rd += 4000; }",
+     "else if (k == 1) { st += 4; rd += 5000; }"),
 ]
 
 
