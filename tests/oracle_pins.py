@@ -82,6 +82,27 @@ def pin_quantize_fp32_scale():
     assert code[0] == 0 and code[1] == 15 and (code[2:] == 7).all(), code
 
 
+def pin_quantize_division_is_correctly_rounded():
+    # The ratio is one IEEE fp32 division (x - min) / scale, rounded once,
+    # then rounded half to even.  4 bits, group {0, 1.125, 0.5625, 0...}:
+    # scale = fl32(1.125 / 15) = 0.0750000030 (just above 0.075), and
+    # 0.5625 / 0.0750000030 = 7.49999970..., whose nearest fp32 is 7.49999952
+    # (7.5 is 2.98e-7 away, 7.49999952 only 1.79e-7), so the code is 7; a
+    # multiply by the rounded reciprocal lands on 7.5 and gives 8.
+    # 2 bits, group {0, 1.625, 0.8125, 0...}: scale = fl32(1.625 / 3) =
+    # 0.541666687, and 0.8125 / 0.541666687 = 1.49999995..., whose nearest
+    # fp32 is 1.5 (a tie, so code 2); the reciprocal path gives 1.49999988 -> 1.
+    x = np.zeros(G, np.float32)
+    x[1], x[2] = 1.125, 0.5625
+    code, s, z = orc.quantize_group(x, 4)
+    assert s == np.float32(1.125) / np.float32(15.0) and z == 0.0
+    assert code[0] == 0 and code[1] == 15 and code[2] == 7, code[:3]
+    x[1], x[2] = 1.625, 0.8125
+    code, s, z = orc.quantize_group(x, 2)
+    assert s == np.float32(1.625) / np.float32(3.0)
+    assert code[0] == 0 and code[1] == 3 and code[2] == 2, code[:3]
+
+
 def pin_quantize_degenerate():
     # constant group: scale 0, all codes 0, zero = the constant
     x = np.full(G, 3.25, np.float32)
@@ -705,6 +726,7 @@ ALL_PINS = [
     pin_quantize_q2_ties,
     pin_quantize_q4_ties,
     pin_quantize_fp32_scale,
+    pin_quantize_division_is_correctly_rounded,
     pin_quantize_degenerate,
     pin_quantize_brute_force,
     pin_pack_worked_example,

@@ -92,6 +92,10 @@ MUTANTS = [
      "const float sq = std::fabs(diff);"),
     ("planner: storage budget ignored", "if (dm <= damage_budget && st <= storage_budget_q) {",
      "if (dm <= damage_budget) {"),
+    ("division by the scale's reciprocal", "const float ratio = shifted / s;          // fp32",
+     "const float ratio = shifted * (1.0f / s);  // fp32"),
+    ("scale over 2^bits steps", "const float s = range / static_cast<float>(qmax);",
+     "const float s = range / static_cast<float>(qmax + 1);"),
     ("planner: 2-bit reads priced as 4-bit", "else if (k == 1) { st += 4; rd += 4000; }",
      "else if (k == 1) { st += 4; rd += 5000; }"),
 ]
