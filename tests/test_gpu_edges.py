@@ -249,3 +249,40 @@ def test_kernels_write_only_the_layout_bytes(pool, cuda_device):
         bad = np.nonzero(outside & (got != 0xA5))[0]
         assert bad.size == 0, "cell %d seq %d head %d: %d stray bytes, first at %d" % (
             c, b, h, bad.size, bad[0])
+
+
+def _division_case_tokens(D, hi, mid):
+    """32 tokens whose every key channel and every value group is {0, hi,
+    mid, 0, ...}: keys quantize per channel over the tokens, values per token
+    over 32-channel groups.  hi and mid are exact in bf16."""
+    k = np.zeros((32, D), np.float32)
+    k[1, :], k[2, :] = hi, mid
+    v = np.zeros((32, D), np.float32)
+    for j in range(0, D, 32):
+        v[:, j + 1], v[:, j + 2] = hi, mid
+    bits = lambda a: (a.view(np.uint32) >> 16).astype(np.uint16)  # noqa: E731  exact here
+    return bits(k), bits(v)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_quantizer_division_cases(cuda_device, D):
+    """Groups whose codes hang on the fp32 ratio being one correctly rounded
+    division (4 bits: scale fl32(1.125 / 15), 0.5625 -> code 7; 2 bits: scale
+    fl32(1.625 / 3), 0.8125 -> code 2; a multiply by the scale's rounded
+    reciprocal gives 8 and 1): the appended cache bytes equal the oracle's."""
+    from loop_aware_quantized_b200 import Plan
+    from oracle import oracle as orc
+    for kind, hi, mid in ((Q4, 1.125, 0.5625), (Q2, 1.625, 0.8125)):
+        kb, vb = _division_case_tokens(D, hi, mid)
+        plan = Plan(1, 1, 1, D, np.array([64], np.int32), np.array([kind], np.uint8), 0.01,
+                    device=cuda_device)
+        plan.append([0], P.bits_to_bf16_tensor(kb[None, None, None], cuda_device).contiguous(),
+                    P.bits_to_bf16_tensor(vb[None, None, None], cuda_device).contiguous())
+        got = plan.unit_bytes(0, 0, 0).cpu().numpy()
+        unit = orc.OracleUnit(kind, D, 64)
+        unit.append(kb, vb)
+        ref_bytes, valid = unit.serialize()
+        P.check_bytes("division case kind %d D %d" % (kind, D), dict(bytes=ref_bytes, valid=valid),
+                      got)
+        plan.check()
+        plan.close()
