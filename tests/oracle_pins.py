@@ -553,6 +553,33 @@ def pin_residual_worked_example():
     assert (z["ks"] == 0).all() and (z["kz"] == 0).all() and (z["vz"] == 0).all()
 
 
+def pin_residual_reference_rounding():
+    # r, the reference's stored value in fp32, is fl(fl(scale * code) + zero):
+    # the two roundings of a 4-bit dequantization.  Worked case: a reference
+    # key channel spanning [-2.71875, 2.953125] (both exact in bf16) has scale
+    # fl32(5.671875 / 15) = 0.378125012; its top code 15 gives
+    # fl(15 * 0.378125012) = 5.671875 (the product 5.67187518 lies 1.8e-7
+    # from it), and 5.671875 - 2.71875 = 2.953125 exactly, where one rounding
+    # of the exact 2.95312518 would give 2.95312524.  A residual cell whose
+    # keys are 0 on that channel stores d = -r, so its residual group's zero
+    # point (the group minimum) is -2.953125.
+    D = 64
+    n = 64   # the residual group 0 is quantized once the cell holds 64 tokens
+    zeros = np.zeros((n, D), np.float32)
+    kr = zeros.copy()
+    kr[0, 0], kr[1, 0] = -2.71875, 2.953125
+    ref = orc.OracleUnit(orc.KIND_Q4, D, 128)
+    ref.append(bf16(kr), bf16(zeros))
+    st_ref = ref.export()
+    assert st_ref["ks"][0, 0] == np.float32(5.671875) / np.float32(15.0)
+    assert st_ref["kz"][0, 0] == np.float32(-2.71875) and st_ref["kq"][1, 0] == 15
+    u = orc.OracleUnit(orc.KIND_RES2, D, 128)
+    u.append(bf16(zeros), bf16(zeros))
+    st = u.export(src=ref)
+    assert st["qtok"] == 32
+    assert st["kz"][0, 0] == np.float32(-2.953125), repr(st["kz"][0, 0])
+
+
 def _ref32(st, pos, keys):
     """The reference's stored value in fp32: fl(fl(scale * code) + zero)."""
     g = pos // G
@@ -743,6 +770,7 @@ ALL_PINS = [
     pin_planner_worked_example,
     pin_residual_deferred_window,
     pin_residual_worked_example,
+    pin_residual_reference_rounding,
     pin_residual_reconstructs,
     pin_residual_reference_checks,
     pin_vq_exact_codebook,

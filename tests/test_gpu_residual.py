@@ -113,3 +113,36 @@ def test_residual_rollback_then_append(pool, cuda_device):
     n_of = lambda c, b: int(wl.lengths[b])  # noqa: E731
     GH.compare(spec, wl, plan, res, cells, seqs, units, n_of, n_of, pool)
     torch.cuda.synchronize()
+
+
+def test_residual_reference_rounding_case(cuda_device):
+    """The worked case where the reference's value needs two roundings,
+    fl(fl(scale * code) + zero): a 4-bit reference key channel over
+    [-2.71875, 2.953125] and a residual cell of zero keys, whose residual
+    zero point is then -2.953125.  Both units' cache bytes equal the
+    oracle's."""
+    from loop_aware_quantized_b200 import Plan
+    from oracle import oracle as orc
+    from synth import philox as px
+    from tests import parity as P
+    D, n = 64, 64
+    zeros = np.zeros((n, D), np.float32)
+    kr = zeros.copy()
+    kr[0, 0], kr[1, 0] = -2.71875, 2.953125
+    bits = lambda a: px.float_to_bf16_bits(a)  # noqa: E731
+    plan = Plan(2, 1, 1, D, np.array([128], np.int32), np.array([RS, Q4], np.uint8), 0.01,
+                device=cuda_device)
+    dev = lambda a: P.bits_to_bf16_tensor(bits(a)[None, None, None], cuda_device).contiguous()  # noqa: E731
+    plan.append([1], dev(kr), dev(zeros))      # the final loop's cell: the reference
+    plan.append([0], dev(zeros), dev(zeros))   # the residual cell
+    ref = orc.OracleUnit(Q4, D, 128)
+    ref.append(bits(kr), bits(zeros))
+    own = orc.OracleUnit(RS, D, 128)
+    own.append(bits(zeros), bits(zeros))
+    assert own.export(src=ref)["kz"][0, 0] == np.float32(-2.953125)
+    for cell, unit, src in ((1, ref, None), (0, own, ref)):
+        want, valid = unit.serialize(src=src)
+        P.check_bytes("reference rounding case, cell %d" % cell, dict(bytes=want, valid=valid),
+                      plan.unit_bytes(cell, 0, 0).cpu().numpy())
+    plan.check()
+    plan.close()

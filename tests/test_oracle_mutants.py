@@ -96,6 +96,9 @@ MUTANTS = [
      "const float ratio = shifted * (1.0f / s);  // fp32"),
     ("scale over 2^bits steps", "const float s = range / static_cast<float>(qmax);",
      "const float s = range / static_cast<float>(qmax + 1);"),
+    ("residual reference dequantized with one rounding",
+     "  const float prod = ref.ks[gr * D + d] * q;\n  return prod + ref.kz[gr * D + d];",
+     "  return static_cast<float>(static_cast<double>(ref.ks[gr * D + d]) * q + ref.kz[gr * D + d]);"),
     ("planner: 2-bit reads priced as 4-bit", "else if (k == 1) { st += 4; rd += 4000; }",
      "else if (k == 1) { st += 4; rd += 5000; }"),
 ]
