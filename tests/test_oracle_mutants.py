@@ -99,6 +99,15 @@ MUTANTS = [
     ("residual reference dequantized with one rounding",
      "  const float prod = ref.ks[gr * D + d] * q;\n  return prod + ref.kz[gr * D + d];",
      "  return static_cast<float>(static_cast<double>(ref.ks[gr * D + d]) * q + ref.kz[gr * D + d]);"),
+    ("value meta pair stored zero first",
+     "      put_bytes(out, valid, L.v_meta + off, &uvs[t * (D / kG) + j], 4);\n"
+     "      put_bytes(out, valid, L.v_meta + off + 4, &uvz[t * (D / kG) + j], 4);",
+     "      put_bytes(out, valid, L.v_meta + off + 4, &uvs[t * (D / kG) + j], 4);\n"
+     "      put_bytes(out, valid, L.v_meta + off, &uvz[t * (D / kG) + j], 4);"),
+    ("key meta stored zeros first",
+     "put_bytes(out, valid, L.k_meta + static_cast<size_t>(g) * 8 * D, &uks[g * D], 4 * D);",
+     "put_bytes(out, valid, L.k_meta + static_cast<size_t>(g) * 8 * D + 4 * D, &uks[g * D], 4 * D);"),
+    ("key plane rows a word apart", "c * 512 + t * 16 + w * 4;", "c * 512 + t * 4 + w * 16;"),
     ("planner: 2-bit reads priced as 4-bit", "else if (k == 1) { st += 4; rd += 4000; }",
      "else if (k == 1) { st += 4; rd += 5000; }"),
 ]
