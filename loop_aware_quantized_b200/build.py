@@ -5,6 +5,7 @@ nvcc (``-gencode arch=compute_100a,code=sm_100a``).  Runs without a GPU.
 """
 
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -29,25 +30,43 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale(lib, deps):
-    if not os.path.exists(lib):
-        return True
-    t = os.path.getmtime(lib)
-    return any(os.path.getmtime(d) > t for d in deps)
+def _deps():
+    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [
+        os.path.join(ROOT, "include", "loopkv.h")]
+
+
+def _stamp(flags):
+    """Hash of what the library is built from: every source and header, the
+    flags and the compiler's version text."""
+    h = hashlib.sha256()
+    for d in _deps():
+        h.update(os.path.relpath(d, ROOT).encode())
+        with open(d, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(flags).encode())
+    h.update(subprocess.run([NVCC, "--version"], capture_output=True, check=True).stdout)
+    return h.hexdigest()
 
 
 def build(force=False, verbose=False, extra_flags=()):
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [
-        os.path.join(ROOT, "include", "loopkv.h")]
-    if not force and not _stale(LIB, deps):
-        return LIB
+    """Compile libloopkv.so unless it exists with a stamp matching the current
+    sources, flags and compiler (kept in libloopkv.so.stamp beside it)."""
+    flags = [*NVCC_FLAGS, *extra_flags]
+    stamp = _stamp(flags)
+    stamp_path = LIB + ".stamp"
+    if not force and os.path.exists(LIB) and os.path.exists(stamp_path):
+        with open(stamp_path) as f:
+            if f.read().strip() == stamp:
+                return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [NVCC, *NVCC_FLAGS, *extra_flags, "-shared", "-I", os.path.join(ROOT, "include"),
+    cmd = [NVCC, *flags, "-shared", "-I", os.path.join(ROOT, "include"),
            *sources(), "-o", tmp, "-cudart", "static"]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)
     os.replace(tmp, LIB)
+    with open(stamp_path, "w") as f:
+        f.write(stamp + "\n")
     return LIB
 
 

@@ -150,6 +150,7 @@ __device__ __forceinline__ void quantize_value_row(V v, bool q4, int qmax, uint4
 template <int D>
 __global__ void __launch_bounds__(kAppendThreads)
 append_kernel(const AppendParams p, const CellList cl) {
+  require_ieee_subnormals();
   constexpr int TROW = D + 2;     // bf16 per padded tile row
   constexpr int CROW = D + kCodeRow;  // bytes per padded code row
   extern __shared__ __align__(16) uint8_t sm[];
@@ -322,6 +323,7 @@ __device__ float ref_value32(const uint8_t* rb, const UnitLayout& RL, int rkind,
 template <int D>
 __global__ void __launch_bounds__(kAppendThreads)
 append_res2_kernel(const AppendParams p, const CellList cl) {
+  require_ieee_subnormals();
   constexpr int XROW = D + 1;     // fp32 per padded tile row
   constexpr int CROW = D + kCodeRow;  // bytes per padded code row
   extern __shared__ __align__(16) uint8_t sm[];

@@ -694,6 +694,7 @@ __device__ __forceinline__ void low_planes(float2 (&acc)[G][32 / G], const Unit&
 template <int D, int G, bool DENSE_LO, bool RES2>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p, const CellList cl) {
+  require_ieee_subnormals();
   using VS = VShare<G>;
   const int S = p.slots;  // score slots per query
   extern __shared__ __align__(16) float smem[];

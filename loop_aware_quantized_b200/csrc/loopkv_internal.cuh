@@ -48,6 +48,20 @@ static_assert(sizeof(DevSeq) == 32, "seq entry size");
 
 inline __host__ __device__ size_t round_up(size_t x, size_t m) { return (x + m - 1) / m * m; }
 
+// The kernels need IEEE fp32 with subnormals kept: the quantizer must give
+// the IEEE codes for subnormal inputs too, the decode turns codes into floats
+// as exact subnormals, and the LoopVQ encoder decides indices by fp32
+// distances.  A build that flushes subnormals to zero (-ftz=true, or
+// --use_fast_math) would change results without a sign, so it does not
+// build: there the compiler's __CUDA_FTZ reflection is 1, the call below
+// stays in the code, and ptxas stops on the undefined function it names.
+// In a correct build the branch is removed and costs nothing.
+extern "C" __device__ int __nvvm_reflect(const char*);
+extern "C" __device__ void loopkv_build_error_flush_to_zero_is_not_supported(void);
+__device__ __forceinline__ void require_ieee_subnormals() {
+  if (__nvvm_reflect("__CUDA_FTZ")) loopkv_build_error_flush_to_zero_is_not_supported();
+}
+
 inline __host__ __device__ size_t table_cells_offset() { return sizeof(TableHeader); }
 inline __host__ __device__ size_t table_seqs_offset(int n_cells) {
   return round_up(sizeof(TableHeader) + sizeof(DevCell) * (size_t)n_cells, 256);

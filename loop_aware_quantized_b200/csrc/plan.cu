@@ -17,6 +17,7 @@ using namespace loopkv;
 struct loopkv_plan {
   int n_loops = 0, n_layers = 0, n_cells = 0, H = 0, D = 0, max_batch = 0;
   int group = 1;                  // query heads per KV head
+  int min_split = 1;              // CTAs per decoded unit at least (the descriptor's decode_split)
   float tau = 0.f, sm_scale = 0.f;
   std::vector<uint8_t> kinds;     // [cells]
   std::vector<int32_t> cap;       // [max_batch]
@@ -56,6 +57,9 @@ loopkv_status validate_desc(const loopkv_plan_desc* d) {
   if (!(d->tau >= 0.f) || !std::isfinite(d->tau)) return LOOPKV_ERR_PLAN;
   if (!std::isfinite(d->sm_scale)) return LOOPKV_ERR_PLAN;
   if (d->q_per_kv != 0 && d->q_per_kv != 1 && d->q_per_kv != 2 && d->q_per_kv != 4)
+    return LOOPKV_ERR_PLAN;
+  if (d->decode_split < 0 || d->decode_split > decode_max_split() ||
+      (d->decode_split & (d->decode_split - 1)) != 0)
     return LOOPKV_ERR_PLAN;
   for (int b = 0; b < d->max_batch; ++b)
     if (d->capacity[b] < 0 || d->capacity[b] > kMaxCapacity) return LOOPKV_ERR_PLAN;
@@ -103,11 +107,6 @@ loopkv_status decode_launch(loopkv_plan* p, const CellList& cl, int n_cells, int
                             float* d_lse, uint32_t* d_mask, int32_t mask_words, int32_t* d_nsel,
                             void* stream);
 
-int env_int(const char* name, int dflt) {
-  const char* v = std::getenv(name);
-  return v ? std::atoi(v) : dflt;
-}
-
 }  // namespace
 
 extern "C" {
@@ -140,6 +139,7 @@ loopkv_status loopkv_plan_load(const loopkv_plan_desc* desc, void* d_table, size
   p->n_cells = desc->n_loops * desc->n_layers;
   p->H = desc->n_kv_heads;
   p->group = desc->q_per_kv > 1 ? desc->q_per_kv : 1;
+  p->min_split = desc->decode_split > 1 ? desc->decode_split : 1;
   p->D = desc->head_dim;
   p->max_batch = desc->max_batch;
   p->tau = desc->tau;
@@ -331,10 +331,8 @@ loopkv_status decode_launch(loopkv_plan* p, const CellList& cl, int n_cells, int
   auto slots_for = [&](int s) { return ((npos_max + s - 1) / s + 31) / 32 * 32; };
   while (slots_for(split) > max_slots && split < decode_max_split()) split *= 2;
   if (slots_for(split) > max_slots) return LOOPKV_ERR_UNSUPPORTED;
-  int want = env_int("LOOPKV_DECODE_SPLIT", 0);
-  if (want > 0) {
-    if (want > decode_max_split() || (want & (want - 1)) != 0) return LOOPKV_ERR_INVALID_ARG;
-    if (want > split) split = want;
+  if (p->min_split > 1) {
+    split = std::max(split, p->min_split);
   } else {
     while (units * split < 148 * 4 && split < decode_max_split() && npos_max / (2 * split) >= 512)
       split *= 2;

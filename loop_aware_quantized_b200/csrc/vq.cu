@@ -88,6 +88,7 @@ __device__ __forceinline__ void load_indices(uint32_t (&w)[D / 16], const uint8_
 template <int D>
 __global__ void __launch_bounds__(kVqThreads, 2)
 vq_decode_kernel(const VqParams p) {
+  require_ieee_subnormals();
   constexpr int GR = D / kVqSub;  // channel groups
   extern __shared__ __align__(16) float sm[];
   float* lut = sm;                 // [GR][kRow]
@@ -315,6 +316,7 @@ struct VqEncodeParams {
 template <int D>
 __global__ void __launch_bounds__(kEntries)
 vq_encode_kernel(const VqEncodeParams p) {
+  require_ieee_subnormals();
   constexpr int GR = D / kVqSub;
   __shared__ float x_s[GR][8 * kVqSub];                 // sub-vectors, loop-major
   __shared__ unsigned long long best[kEntries / 32][GR];

@@ -16,8 +16,7 @@ import os
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# LOOPKV_LIBRARY may name another build of the same library (same ABI).
-LIB_PATH = os.environ.get("LOOPKV_LIBRARY") or os.path.join(_HERE, "libloopkv.so")
+LIB_PATH = os.path.join(_HERE, "libloopkv.so")
 
 LOOPKV_Q4, LOOPKV_Q2, LOOPKV_SHARE, LOOPKV_BF16, LOOPKV_RES2 = 0, 1, 2, 3, 4
 LOOPKV_MAX_CELLS_PER_CALL = 256
@@ -53,6 +52,7 @@ class loopkv_plan_desc(ctypes.Structure):
         ("tau", ctypes.c_float),
         ("sm_scale", ctypes.c_float),
         ("q_per_kv", ctypes.c_int32),
+        ("decode_split", ctypes.c_int32),
     ]
 
 
@@ -266,7 +266,7 @@ def _int_dtypes():
 
 
 def make_desc(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau, sm_scale=0.0,
-              q_per_kv=1):
+              q_per_kv=1, decode_split=0):
     """Build a loopkv_plan_desc; returns (desc, keepalive arrays)."""
     cap = np.ascontiguousarray(capacity, dtype=np.int32)
     kinds = np.ascontiguousarray(kinds, dtype=np.uint8)
@@ -278,6 +278,7 @@ def make_desc(n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau, sm_
     d.tau = float(tau)
     d.sm_scale = float(sm_scale)
     d.q_per_kv = int(q_per_kv)
+    d.decode_split = int(decode_split)
     return d, (cap, kinds)
 
 
@@ -294,9 +295,11 @@ class Plan:
     """A loaded LoopKV plan with its device table and cache (torch tensors)."""
 
     def __init__(self, n_loops, n_layers, n_kv_heads, head_dim, capacity, kinds, tau,
-                 sm_scale=0.0, device="cuda", stream=None, q_per_kv=1, cache_guard=0):
+                 sm_scale=0.0, device="cuda", stream=None, q_per_kv=1, cache_guard=0,
+                 decode_split=0):
         """cache_guard: extra bytes allocated after the cache (not given to the
-        library), so tests can check that nothing is written past its end."""
+        library), so tests can check that nothing is written past its end.
+        decode_split: CTAs per decoded unit at least (0: the library chooses)."""
         import torch
         self.n_loops, self.n_layers = n_loops, n_layers
         self.n_cells = n_loops * n_layers
@@ -307,7 +310,7 @@ class Plan:
         self.tau = float(tau)
         self.q_per_kv = int(q_per_kv)
         d, keep = make_desc(n_loops, n_layers, n_kv_heads, head_dim, self.capacity, self.kinds,
-                            tau, sm_scale, q_per_kv)
+                            tau, sm_scale, q_per_kv, decode_split)
         rc, sizes = loopkv_plan_query(d)
         _check(rc, "loopkv_plan_query")
         self.table_bytes, self.cache_bytes = int(sizes.table_bytes), int(sizes.cache_bytes)

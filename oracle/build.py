@@ -4,6 +4,7 @@ Test infrastructure: plain g++, no fast-math and no floating-point contraction
 so that every fp32 step of the quantizer is the IEEE round-to-nearest one.
 """
 
+import hashlib
 import os
 import subprocess
 import sys
@@ -16,14 +17,30 @@ FLAGS = ["-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-Wall",
          "-shared", "-fPIC"]
 
 
+def _stamp():
+    """Hash of the source, the flags and the compiler's version text."""
+    h = hashlib.sha256()
+    with open(SRC, "rb") as f:
+        h.update(f.read())
+    h.update(" ".join(FLAGS).encode())
+    h.update(subprocess.run(["g++", "--version"], capture_output=True, check=True).stdout)
+    return h.hexdigest()
+
+
 def build(force: bool = False) -> str:
-    """Build the oracle library if missing or older than its source."""
-    if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= os.path.getmtime(SRC)):
-        return LIB
+    """Build the oracle library unless it exists with a stamp (liboracle.so.stamp)
+    matching the current source, flags and compiler."""
+    stamp = _stamp()
+    stamp_path = LIB + ".stamp"
+    if not force and os.path.exists(LIB) and os.path.exists(stamp_path):
+        with open(stamp_path) as f:
+            if f.read().strip() == stamp:
+                return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
     subprocess.check_call(["g++", *FLAGS, SRC, "-o", tmp])
     os.replace(tmp, LIB)
+    with open(stamp_path, "w") as f:
+        f.write(stamp + "\n")
     return LIB
 
 

@@ -484,18 +484,22 @@ int orc_unit_serialize(const void* p, const void* src, uint8_t* out, uint8_t* va
 // Outputs: out[g][D]; lse[g] (natural log); mask words, one per 32 positions
 // of the data cell's quantized range, bit j of word w = position 32w+j
 // selected by some head (only when the data cell is 4-bit); *nsel (selected
-// positions); slack[g][D] (nullable) = for head r, the sum over 4-bit
-// positions where some head's weight is within band of tau of
-// p_r * scale_v * |lo - 1.5|, the most a disagreement on those positions can
-// move each output.  *n_mask_words receives the number of mask words
-// written; weights[g][npos] (nullable) receives every head's softmax weight
-// of every attended position, own current last.
+// positions).  *n_mask_words receives the number of mask words written;
+// weights[g][npos] (nullable) receives every head's softmax weight of every
+// attended position, own current last.
+// sel_override (nullable; mask words in the layout of `mask`): a 4-bit
+// position where some head's weight lies within band of tau is selected
+// when its bit there is set and not selected otherwise, instead of by the
+// comparison p >= tau.  A kernel working in fp32 may decide such a position
+// either way; passing its choice gives the output that choice implies, so
+// the outputs can then be compared at the full tolerance.  Positions outside
+// the band are always decided by the comparison.
 // Returns 0, or -1 on invalid input (no positions, SHARE without a source,
 // SHARE longer than its source allows, g < 1).
 int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, int g,
                      double tau, double sm_scale, double band, double* out, double* lse,
-                     uint32_t* mask, int* n_mask_words, int* nsel, double* slack,
-                     double* weights) {
+                     uint32_t* mask, int* n_mask_words, int* nsel,
+                     const uint32_t* sel_override, double* weights) {
   const Unit* own = static_cast<const Unit*>(own_p);
   const Unit* src = static_cast<const Unit*>(src_p);
   const int D = own->D;
@@ -591,6 +595,7 @@ int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, in
       if (ph >= tau) sel[pos] = 1;
       if (std::fabs(ph - tau) <= band) near[pos] = 1;
     }
+    if (sel_override && near[pos]) sel[pos] = (sel_override[pos / kG] >> (pos % kG)) & 1u;
     if (sel[pos]) {
       mask[pos / kG] |= 1u << (pos % kG);
       ++count;
@@ -601,11 +606,9 @@ int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, in
 
   // weighted values, per head
   for (int i = 0; i < g * D; ++i) out[i] = 0.0;
-  if (slack) for (int i = 0; i < g * D; ++i) slack[i] = 0.0;
   for (int pos = 0; pos < npos; ++pos) {
     for (int d = 0; d < D; ++d) {
       double v;
-      double dev = 0.0;  // |lo - 1.5| * scale: the most the selection moves v
       if (res2 && pos >= qtok) {
         v = bf16_to_float(own->bv[static_cast<size_t>(pos) * D + d]);
       } else if (share && pos == n_att) {
@@ -621,7 +624,6 @@ int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, in
           const int hi = code >> 2, lo = code & 3;
           const double low_part = sel[pos] ? static_cast<double>(lo) : 1.5;  // R3
           v = sc * (4.0 * hi + low_part) + ze;
-          dev = sc * std::fabs(lo - 1.5);
         } else {
           v = sc * code + ze;
         }
@@ -636,21 +638,20 @@ int orc_decode_group(const void* own_p, const void* src_p, const uint16_t* q, in
       for (int h = 0; h < g; ++h) {
         const double ph = p[static_cast<size_t>(h) * npos + pos];
         out[static_cast<size_t>(h) * D + d] += ph * v;
-        if (slack && near[pos]) slack[static_cast<size_t>(h) * D + d] += ph * dev;
       }
     }
   }
   return 0;
 }
 
-// One query head (g = 1): q bf16 bits [D], out[D], *lse, slack[D] and
+// One query head (g = 1): q bf16 bits [D], out[D], *lse, sel_override and
 // weights[npos] as in orc_decode_group.
 int orc_decode(const void* own_p, const void* src_p, const uint16_t* q,
                double tau, double sm_scale, double band, double* out,
                double* lse, uint32_t* mask, int* n_mask_words, int* nsel,
-               double* slack, double* weights) {
+               const uint32_t* sel_override, double* weights) {
   return orc_decode_group(own_p, src_p, q, 1, tau, sm_scale, band, out, lse, mask,
-                          n_mask_words, nsel, slack, weights);
+                          n_mask_words, nsel, sel_override, weights);
 }
 
 // ---- LoopVQ decode ----------------------------------------------------------

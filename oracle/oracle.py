@@ -149,35 +149,46 @@ class DecodeResult:
     lse: float           # natural log
     mask: np.ndarray     # uint32 words over the 4-bit positions
     nsel: int
-    slack: np.ndarray    # fp64 [D]
     weights: np.ndarray  # fp64 softmax weight per attended position
 
 
-def decode(unit, q_bits, tau, src=None, sm_scale=0.0, band=1e-6):
+def _override_words(sel_override, npos):
+    """Selection override as uint32 words covering npos positions (or None)."""
+    if sel_override is None:
+        return None
+    words = np.zeros(max(npos // G + 2, 1), np.uint32)
+    given = np.ascontiguousarray(sel_override, dtype=np.uint32).reshape(-1)
+    words[: min(given.size, words.size)] = given[: words.size]
+    return words
+
+
+def decode(unit, q_bits, tau, src=None, sm_scale=0.0, band=1e-6, sel_override=None):
     """Decode one unit for the query ``q_bits`` (bf16 bits [D]).
 
     ``src`` is the final loop's unit of the same layer, sequence and head when
-    ``unit`` is a SHARE unit or a residual (RES2) unit.
+    ``unit`` is a SHARE unit or a residual (RES2) unit.  ``sel_override``
+    (mask words): the selection of positions whose weight is within ``band``
+    of ``tau`` (see ``orc_decode_group``).
     """
     D = unit.D
     q = np.ascontiguousarray(q_bits, dtype=np.uint16).reshape(D)
     npos = unit.n
     out = np.zeros(D, np.float64)
-    slack = np.zeros(D, np.float64)
-    # slack beyond npos: a planted mistake in a test copy may write more
+    # room beyond npos: a planted mistake in a test copy may write more
     weights = np.zeros(npos + 2, np.float64)
     lse = np.zeros(1, np.float64)
     mask = np.zeros(max(npos // G + 2, 1), np.uint32)
     nw = np.zeros(1, np.int32)
     nsel = np.zeros(1, np.int32)
+    ov = _override_words(sel_override, npos)
     rc = unit._lib.orc_decode(unit._h, None if src is None else src._h, _ptr(q),
                          float(tau), float(sm_scale), float(band), _ptr(out),
                          _ptr(lse), _ptr(mask), _ptr(nw), _ptr(nsel),
-                         _ptr(slack), _ptr(weights))
+                         _ptr(ov), _ptr(weights))
     if rc != 0:
         raise ValueError("oracle decode rejected its input")
     return DecodeResult(out=out, lse=float(lse[0]), mask=mask[: nw[0]].copy(),
-                        nsel=int(nsel[0]), slack=slack, weights=weights[:npos])
+                        nsel=int(nsel[0]), weights=weights[:npos])
 
 
 @dataclasses.dataclass
@@ -186,34 +197,34 @@ class GroupDecodeResult:
     lse: np.ndarray      # fp64 [g], natural log
     mask: np.ndarray     # uint32 words over the 4-bit positions (union over heads)
     nsel: int
-    slack: np.ndarray    # fp64 [g][D]
     weights: np.ndarray  # fp64 [g][npos]
 
 
-def decode_group(unit, q_bits, tau, src=None, sm_scale=0.0, band=1e-6):
+def decode_group(unit, q_bits, tau, src=None, sm_scale=0.0, band=1e-6, sel_override=None):
     """Decode one unit for a group of query heads sharing its keys and values.
 
-    ``q_bits``: bf16 bits [g][D].  The selection is the union over the heads.
+    ``q_bits``: bf16 bits [g][D].  The selection is the union over the heads;
+    ``sel_override`` as in ``decode``.
     """
     D = unit.D
     q = np.ascontiguousarray(q_bits, dtype=np.uint16).reshape(-1, D)
     g = q.shape[0]
     npos = unit.n
     out = np.zeros((g, D), np.float64)
-    slack = np.zeros((g, D), np.float64)
-    weights = np.zeros(g * (npos + 2), np.float64)  # slack as in decode()
+    weights = np.zeros(g * (npos + 2), np.float64)  # room as in decode()
     lse = np.zeros(g, np.float64)
     mask = np.zeros(max(npos // G + 2, 1), np.uint32)
     nw = np.zeros(1, np.int32)
     nsel = np.zeros(1, np.int32)
+    ov = _override_words(sel_override, npos)
     rc = unit._lib.orc_decode_group(unit._h, None if src is None else src._h, _ptr(q), g,
                                     float(tau), float(sm_scale), float(band), _ptr(out),
                                     _ptr(lse), _ptr(mask), _ptr(nw), _ptr(nsel),
-                                    _ptr(slack), _ptr(weights))
+                                    _ptr(ov), _ptr(weights))
     if rc != 0:
         raise ValueError("oracle decode rejected its input")
     return GroupDecodeResult(out=out, lse=lse, mask=mask[: nw[0]].copy(), nsel=int(nsel[0]),
-                             slack=slack, weights=weights[: g * npos].reshape(g, npos).copy())
+                             weights=weights[: g * npos].reshape(g, npos).copy())
 
 
 def plan_brute(n_loops, n_layers, damage, damage_budget, storage_budget_q, sel_milli):

@@ -1,5 +1,6 @@
 """Build the GPU input generator ``synth/libloopkv_synth.so`` (sm_100a)."""
 
+import hashlib
 import os
 import subprocess
 import sys
@@ -10,13 +11,34 @@ LIB = os.path.join(HERE, "libloopkv_synth.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 
+FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-Xcompiler", "-fPIC",
+         "-shared"]
+
+
+def _stamp():
+    """Hash of the source, the flags and the compiler's version text."""
+    h = hashlib.sha256()
+    with open(SRC, "rb") as f:
+        h.update(f.read())
+    h.update(" ".join(FLAGS).encode())
+    h.update(subprocess.run([NVCC, "--version"], capture_output=True, check=True).stdout)
+    return h.hexdigest()
+
+
 def build(force=False):
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
-        return LIB
+    """Build unless the library exists with a stamp (libloopkv_synth.so.stamp)
+    matching the current source, flags and compiler."""
+    stamp = _stamp()
+    stamp_path = LIB + ".stamp"
+    if not force and os.path.exists(LIB) and os.path.exists(stamp_path):
+        with open(stamp_path) as f:
+            if f.read().strip() == stamp:
+                return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
-    subprocess.check_call([NVCC, "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
-                           "-Xcompiler", "-fPIC", "-shared", SRC, "-o", tmp, "-cudart", "static"])
+    subprocess.check_call([NVCC, *FLAGS, SRC, "-o", tmp, "-cudart", "static"])
     os.replace(tmp, LIB)
+    with open(stamp_path, "w") as f:
+        f.write(stamp + "\n")
     return LIB
 
 

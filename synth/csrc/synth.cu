@@ -214,9 +214,29 @@ __global__ void gen_vq_q_kernel(uint16_t* __restrict__ q, int n_layers, int batc
   }
 }
 
+// Philox4x32-10 of n (counter, key) rows: in [n][6] = c0..c3, k0, k1; out [n][4].
+__global__ void philox_rows_kernel(const uint32_t* __restrict__ in, uint32_t* __restrict__ out,
+                                   int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const uint32_t* r = in + (size_t)i * 6;
+  const U4 u = philox(r[0], r[1], r[2], r[3], r[4], r[5]);
+  uint32_t* o = out + (size_t)i * 4;
+  o[0] = u.x; o[1] = u.y; o[2] = u.z; o[3] = u.w;
+}
+
 }  // namespace
 
 extern "C" {
+
+// The generator's Philox4x32-10 on explicit (counter, key) rows, so it can be
+// checked against the published known-answer vectors.
+int synth_philox(const uint32_t* d_in, uint32_t* d_out, int n, void* stream) {
+  if (n <= 0) return 0;
+  philox_rows_kernel<<<(unsigned)((n + 127) / 128), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      d_in, d_out, n);
+  return (int)cudaGetLastError();
+}
 
 int synth_gen_vq_idx(uint8_t* out, int n_layers, int batch, int H, int D, int cap, int T,
                      int which, int seq0, uint32_t seed, void* stream) {

@@ -41,12 +41,26 @@ def _load():
         lib.synth_gen_vq_idx.restype = I
         lib.synth_gen_vq_q.argtypes = [P, I, I, I, I, I, I, ctypes.c_uint32, ctypes.c_float, P]
         lib.synth_gen_vq_q.restype = I
+        lib.synth_philox.argtypes = [P, P, I, P]
+        lib.synth_philox.restype = I
         _lib = lib
     return _lib
 
 
 def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def philox_rows(rows, device="cuda"):
+    """The device generator's Philox4x32-10 of (c0, c1, c2, c3, k0, k1) rows ->
+    uint32 [n][4] (host array)."""
+    import torch
+    a = np.ascontiguousarray(rows, dtype=np.uint32).reshape(-1, 6)
+    d_in = torch.from_numpy(a.view(np.int32)).to(device)
+    d_out = torch.empty((a.shape[0], 4), dtype=torch.int32, device=device)
+    _ok(_load().synth_philox(_p(d_in), _p(d_out), a.shape[0], None))
+    torch.cuda.synchronize()
+    return d_out.cpu().numpy().view(np.uint32)
 
 
 class DeviceGenerator:

@@ -8,10 +8,10 @@ from tests import parity as P
 from synth import workloads as W
 
 
-def make_plan(wl, seqs):
+def make_plan(wl, seqs, decode_split=0):
     from loop_aware_quantized_b200 import Plan
     return Plan(wl.n_loops, wl.n_layers, wl.n_heads, wl.head_dim, wl.capacity[seqs], wl.kinds,
-                wl.tau)
+                wl.tau, decode_split=decode_split)
 
 
 def build_cache(wl, plan, gen, seqs, lengths, cells=None, chunk_tokens=None):

@@ -385,13 +385,50 @@ def pin_group_query_heads():
     # a group of one head is the one-query decode
     r1, o1 = orc.decode_group(u, q[:1], tau), orc.decode(u, q[0], tau)
     assert np.array_equal(r1.out[0], o1.out) and np.array_equal(r1.mask, o1.mask)
-    assert r1.nsel == o1.nsel and np.array_equal(r1.slack[0], o1.slack)
+    assert r1.nsel == o1.nsel and np.array_equal(r1.weights[0], o1.weights)
     # SHARE units group the same way over the final loop's positions
     own = orc.OracleUnit(orc.KIND_SHARE, D, 0)
     own.append(rng_bits(95, (120, D)), rng_bits(96, (120, D)))
     rs = orc.decode_group(own, q, tau, src=u)
     for h in range(q.shape[0]):
         assert np.array_equal(rs.weights[h], orc.decode(own, q[h], tau, src=u).weights)
+
+
+def pin_selection_override():
+    # A position whose weight is within the band of tau takes the selection
+    # the caller passes; with tau set to one position's own weight, turning
+    # that position off moves each output channel by exactly
+    # p * scale * (1.5 - lo) (its value falls back to the high-plane
+    # midpoint), clears its mask bit and lowers the count by one.  Bits of
+    # positions outside the band are ignored.
+    D = 64
+    u, k, v = _unit(orc.KIND_Q4, D, 150, 90)
+    kf = f32(k)
+    q = bf16(2.0 * kf[37])
+    base = orc.decode(u, q, 0.5)
+    t = int(np.argsort(base.weights[:128])[-3])       # a quantized position, not the peak
+    tau = float(base.weights[t])
+    r = orc.decode(u, q, tau)
+    sel = _mask_bits(r.mask, 128)
+    assert sel[t] and r.nsel == int(sel.sum())
+    ov = r.mask.copy()
+    ov[t // G] &= ~np.uint32(1 << (t % G))
+    far = int(np.nonzero(sel & (np.abs(r.weights[:128] - tau) > 1e-6))[0][0])   # selected, outside the band
+    ov[far // G] &= ~np.uint32(1 << (far % G))
+    o = orc.decode(u, q, tau, sel_override=ov)
+    st = u.export()
+    lo = (st["vq"][t].astype(np.int64) & 3).astype(np.float64)
+    sc = np.repeat(st["vs"][t].astype(np.float64), G)
+    expect = r.out + r.weights[t] * sc * (1.5 - lo)
+    assert np.abs(o.out - expect).max() < 1e-12
+    assert o.nsel == r.nsel - 1 and np.array_equal(o.weights, r.weights)
+    want = r.mask.copy()
+    want[t // G] &= ~np.uint32(1 << (t % G))
+    assert np.array_equal(o.mask, want)
+    # the same through a group of one head, and no override changes nothing
+    g = orc.decode_group(u, q[None], tau, sel_override=ov)
+    assert np.array_equal(g.out[0], o.out) and np.array_equal(g.mask, o.mask)
+    assert np.array_equal(orc.decode(u, q, tau, sel_override=r.mask).out, r.out)
 
 
 def pin_planner_worked_example():
@@ -767,6 +804,7 @@ ALL_PINS = [
     pin_high_plane_worked_example,
     pin_mask_properties,
     pin_group_query_heads,
+    pin_selection_override,
     pin_planner_worked_example,
     pin_residual_deferred_window,
     pin_residual_worked_example,

@@ -88,6 +88,28 @@ def test_plan_query_checks_the_query_group(lk):
         assert lk.loopkv_plan_query(d)[0] == 2, g
 
 
+def test_plan_query_checks_the_decode_split(lk):
+    # CTAs per decoded unit: 0 (the library chooses), 1, 2, 4 or 8
+    for sp in (0, 1, 2, 4, 8):
+        d, keep = lk.make_desc(2, 2, 2, 64, [64, 96], [0, 2, 1, 0], 0.01, decode_split=sp)
+        assert lk.loopkv_plan_query(d)[0] == 0, sp
+    for sp in (-1, 3, 6, 16):
+        d, keep = lk.make_desc(2, 2, 2, 64, [64, 96], [0, 2, 1, 0], 0.01, decode_split=sp)
+        assert lk.loopkv_plan_query(d)[0] == 2, sp
+
+
+def test_binding_loads_only_the_in_tree_library():
+    # no environment variable can point the binding at another build
+    import subprocess
+    import sys
+    env = dict(os.environ, LOOPKV_LIBRARY="/nonexistent/libloopkv.so")
+    code = ("import sys; sys.path.insert(0, %r); from loop_aware_quantized_b200 import loopkv; "
+            "print(loopkv.LIB_PATH)" % ROOT)
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                         check=True).stdout.strip()
+    assert out == os.path.join(ROOT, "loop_aware_quantized_b200", "libloopkv.so")
+
+
 def test_plan_load_checks_arguments_before_any_device_work(lk):
     d, keep = lk.make_desc(2, 2, 2, 64, [64, 96], [0, 2, 1, 0], 0.01)
     rc, h = lk.loopkv_plan_load(d, None, 0, None, 0, None)

@@ -26,13 +26,14 @@ def _spec(D, kinds, lengths, tau, n_loops=2, n_layers=2, H=2, extra=64):
     return (n_loops, n_layers, H, D, tuple(kinds), tuple(lengths), cap, tau)
 
 
-def _check_spec(spec, pool, dev, token_by_token=False, src_lengths=None):
-    """Build all cells of a custom workload, decode every unit, oracle-check all."""
+def _check_spec(spec, pool, dev, token_by_token=False, src_lengths=None, split=0):
+    """Build all cells of a custom workload, decode every unit, oracle-check all
+    (split: CTAs per decoded unit at least; 0 lets the library choose)."""
     import torch
     from synth.gpu import DeviceGenerator
     wl = W.custom(*spec)
     seqs = list(range(wl.batch))
-    plan = GH.make_plan(wl, seqs)
+    plan = GH.make_plan(wl, seqs, decode_split=split)
     gen = DeviceGenerator(wl, dev)
     cells = list(range(wl.n_cells))
     if token_by_token:

@@ -67,8 +67,7 @@ def test_device_generator_matches_host(dev):
                     assert (qg[ci, bl, h] == ref).all() and (ref[0] == q[ci, bl, h]).all()
 
 
-def _run_decode_only(config, pool, dev, cells=None, seqs=None, n_sample=16, split=None,
-                     monkeypatch=None):
+def _run_decode_only(config, pool, dev, cells=None, seqs=None, n_sample=16, split=0):
     wl = W.make(config)
     seqs = list(range(wl.batch)) if seqs is None else list(seqs)
     cells = list(range(wl.n_cells)) if cells is None else list(cells)
@@ -76,12 +75,10 @@ def _run_decode_only(config, pool, dev, cells=None, seqs=None, n_sample=16, spli
     need = sorted(set(cells) | {wl.source_cell(c) for c in cells
                                 if wl.kinds[c] in (W.SHARE, W.RES2)})
     lengths = wl.lengths[seqs]
-    plan = GH.make_plan(wl, seqs)
+    plan = GH.make_plan(wl, seqs, decode_split=split)
     gen = _gen(wl, dev)
     GH.build_cache(wl, plan, gen, seqs, lengths, cells=need)
     lens = np.array([[wl.lengths[b] for b in seqs] for _ in cells], np.int32)
-    if split is not None:
-        monkeypatch.setenv("LOOPKV_DECODE_SPLIT", str(split))
     res = GH.decode_all(wl, plan, gen, seqs, cells, lens, dev)
     plan.check()
     units = GH.sample_units(wl, cells, seqs, n_sample, seed=int(config[0]) + 7)
@@ -104,8 +101,8 @@ def test_config0_tiny_all_units(pool, dev):
 
 
 @pytest.mark.parametrize("split", [2, 4, 8])
-def test_config0_cluster_split(pool, dev, split, monkeypatch):
-    _run_decode_only("0", pool, dev, n_sample=8, split=split, monkeypatch=monkeypatch)
+def test_config0_cluster_split(pool, dev, split):
+    _run_decode_only("0", pool, dev, n_sample=8, split=split)
 
 
 def test_config1_single_sequence(pool, dev):

@@ -44,9 +44,9 @@ def test_residual_serving_order_appends(pool, cuda_device):
 
 
 @pytest.mark.parametrize("split", [2, 4])
-def test_residual_cluster_split(pool, cuda_device, split, monkeypatch):
-    monkeypatch.setenv("LOOPKV_DECODE_SPLIT", str(split))
-    _check_spec(_spec(128, (RS, Q2, Q4, Q4), (65, 700, 1500), 0.01), pool, cuda_device)
+def test_residual_cluster_split(pool, cuda_device, split):
+    _check_spec(_spec(128, (RS, Q2, Q4, Q4), (65, 700, 1500), 0.01), pool, cuda_device,
+                split=split)
 
 
 def test_residual_append_needs_its_reference(cuda_device):

@@ -55,7 +55,7 @@ def _run(wl_args, loops, pool, dev, units=None):
         for (layer, b, h), ref in zip(units, pool.map(_oracle_vq_job, jobs)):
             tag = "%s loop %d layer %d b %d h %d" % (wl.name, loop, layer, b, h)
             assert (qh[layer, b, h] == ref["q"]).all(), tag + ": device query differs from host"
-            P.check_unit(tag, dict(out=ref["out"], slack=np.zeros_like(ref["out"]), lse=ref["lse"]),
+            P.check_unit(tag, dict(out=ref["out"], lse=ref["lse"]),
                          out[layer, b, h], lse=lse[layer, b, h])
 
 

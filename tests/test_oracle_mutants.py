@@ -37,6 +37,10 @@ MUTANTS = [
      "sel[pos] ? static_cast<double>(lo) : 2.0"),
     ("zero point dropped", "v = sc * code + ze;", "v = sc * code;"),
     ("tie not selected", "if (ph >= tau) sel[pos] = 1;", "if (ph > tau) sel[pos] = 1;"),
+    ("override outside the band", "if (sel_override && near[pos]) sel[pos]",
+     "if (sel_override) sel[pos]"),
+    ("override ignored", "if (sel_override && near[pos]) sel[pos]",
+     "if (sel_override && near[pos] && false) sel[pos]"),
     ("selection from one head only", "if (ph >= tau) sel[pos] = 1;",
      "if (ph >= tau && h == 0) sel[pos] = 1;"),
     ("query heads share one query", "const double* qh = &qd[static_cast<size_t>(h) * D];",
