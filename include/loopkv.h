@@ -4,10 +4,10 @@
  * What it computes.  "LoopKV: Loop-Aware KV Cache Compression for Serving
  * Looped Transformers", section 概要 (abstract): a looped transformer keeps
  * one KV cache per (loop, layer) cell; a plan gives every cell 4-bit storage,
- * 2-bit storage, or reuse of the final loop's KV (SHARE); during decoding
- * each loop reads the high 2 bits of every 4-bit value and fetches the low
- * 2 bits only where its own attention weights need 4-bit precision; one
- * fused kernel runs the plan.  The abstract fixes no arithmetic; this
+ * 2-bit storage, or reuse of the final loop's KV (SHARE); a 4-bit value is
+ * held as two 2-bit planes, every loop streams the upper plane, and the
+ * lower plane is gathered only for the tokens that loop's softmax weights
+ * mark as needing full precision; a single fused kernel executes the plan.  The abstract fixes no arithmetic; this
  * library takes these readings (the CPU oracle under oracle/ takes the same):
  *   - asymmetric min/max quantization as in "KIVI: A Tuning-Free Asymmetric
  *     2bit Quantization for KV Cache": keys per channel over groups of 32
@@ -260,8 +260,9 @@ const char* loopkv_status_string(loopkv_status status);
  * "LoopKV: Loop-Aware KV Cache Compression for Serving Looped Transformers",
  * section 概要: a one-time offline profile gives every (loop, layer) cell a
  * predicted damage for 4-bit storage, 2-bit storage and reuse of the final
- * loop's KV (SHARE); damages add over cells; the planner minimizes reads
- * under budgets for predicted damage and storage.  The pages fix nothing
+ * loop's KV (SHARE); damages add over cells; the planner looks for the plan
+ * with the least data read whose predicted damage and storage each stay
+ * within a budget.  The pages fix nothing
  * else; this library reads it as follows.  Per cached token and KV head:
  *   Q4    stores 6 blocks of D/4 bytes (K hi/lo/meta, V hi/lo/meta) and reads
  *         5 of them plus a low-plane row for a fraction sel_fraction of its

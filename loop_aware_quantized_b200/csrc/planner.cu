@@ -1,11 +1,11 @@
-// LoopKV planner (host code): the plan that minimizes reads under a damage
+// LoopKV planner (host code): the plan with the fewest reads within a damage
 // budget and a storage budget.
 //
 // "LoopKV: Loop-Aware KV Cache Compression for Serving Looped Transformers",
 // section 概要: a one-time offline profile gives each (loop, layer) cell a
 // predicted damage for 4-bit storage, 2-bit storage or reuse of the final
-// loop's KV; damages add over cells; the planner minimizes reads under
-// budgets for predicted damage and storage.  The costs per cached token and
+// loop's KV; damages add over cells; the planner looks for the least data
+// read while predicted damage and storage each stay within a budget.  The costs per cached token and
 // KV head, in quarters of head_dim bytes, are read as: Q4 stores 6 blocks
 // and reads 5 plus a low-plane row for a fraction of its tokens; Q2 stores
 // and reads 4; SHARE stores nothing and reads what its layer's final-loop

@@ -10,25 +10,31 @@
 //
 // One CTA (8 warps) per (layer, sequence, KV head, split); splits of a long
 // sequence form a thread-block cluster and merge through DSMEM.
-//   table   per channel group j and entry e, LUT[j][e] = <q_j, entry_e's
-//           loop slice> (the query is folded into the codebook once, so a
-//           token's score is D/4 shared-memory lookups and adds);
-//   pass 1  lane = token: its D/4 key indices (one 16-byte load per 16
-//           groups), score = sum_j LUT[j][idx_j], kept in shared memory
-//           (log2 units);
+//   table   T[e][c] = <q_g, entry_e's loop slice> for channel group
+//           g = c mod (D/4), over 64 columns c (each group appears in 2
+//           columns at D = 128, 4 at D = 64): the query is folded into the
+//           codebook once, so a token's score is D/4 shared-memory lookups;
+//   pass 1  lane = token.  At step k a lane reads group (lane + k) mod (D/4)
+//           of its token from column lane + k: the 32 lanes of a warp then
+//           touch 32 consecutive columns, i.e. 32 different banks, whatever
+//           the indices are (a table laid out by group would put a warp's 32
+//           random entries of one group on random banks).  Each lane rotates
+//           its token's D/4 index bytes by its lane number once, so the byte
+//           step k needs sits at a fixed register position; scores stay in
+//           shared memory (log2 units);
 //   softmax the CTA's max and sum of exponentials, merged over the cluster;
-//   pass 2  lane = token: p_t added into W[j][idx_v_j] (a weight histogram
-//           over the value codebook): p_t as a fixed-point integer
-//           (units of 2^-31) with integer shared-memory atomics, which are
-//           native, order-independent and exact; every bin holds at most
-//           the sum of all weights (1), and each token's rounding (<= 2^-32)
+//   pass 2  the same walk adds p_t into a histogram over the value codebook
+//           laid out like the table: p_t as a fixed-point integer (units of
+//           2^-31) with integer shared-memory atomics, which are native,
+//           order-independent and exact; the bins of a (group, entry) are
+//           summed over its columns afterwards; every bin holds at most the
+//           sum of all weights (1), and each token's rounding (<= 2^-32)
 //           lands in one bin, so an output moves by at most n 2^-32 times
 //           the largest codebook magnitude;
-//   output  out[4j + i] = 2^-31 sum_e W[j][e] * entry_e[4l + i].
+//   output  out[4g + i] = 2^-31 sum_e W[g][e] * entry_e[4l + i].
 // The index streams are read once (D/2 bytes per token at D = 128: 32 key
-// and 32 value bytes); the work per token is D/2 random shared-memory
-// accesses, so the kernel is bound by shared-memory bank conflicts of those
-// lookups rather than by HBM.
+// and 32 value bytes); the work per token is D/2 shared-memory accesses,
+// one bank-conflict-free wavefront per warp instruction.
 
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
@@ -47,7 +53,7 @@ constexpr int kVqThreads = 256;
 constexpr int kVqWarps = kVqThreads / 32;
 constexpr int kVqSub = 4;        // channels per sub-vector
 constexpr int kEntries = 256;    // codebook entries (one byte)
-constexpr int kRow = kEntries + 1;  // padded table row: group j's row starts in bank j
+constexpr int kCols = 64;         // table / histogram columns: column c is group c mod (D/4)
 constexpr int kVqSlots = 8448;   // score slots per CTA (two CTAs per SM; 16K + a few hundred tokens in two)
 constexpr int kVqMaxSplit = 8;   // portable cluster size
 
@@ -72,17 +78,47 @@ __device__ __forceinline__ uint4 ld_idx(const uint8_t* p) {
   return r;
 }
 
-// The D/4 indices of a token as D/16 words (index 4k + m in byte m of word k).
+// The D/4 indices of a token as D/16 words, rotated left by r = lane mod
+// (D/4) bytes: byte m of word k holds the index of group (4k + m + r) mod
+// (D/4).  At D = 128 a rotation by four words is the choice of which 16-byte
+// half to load first; the rest is two conditional word rotations and one
+// funnel shift per word.
 template <int D>
-__device__ __forceinline__ void load_indices(uint32_t (&w)[D / 16], const uint8_t* row) {
-#pragma unroll
-  for (int k = 0; k < D / 64; ++k) {
-    const uint4 x = ld_idx(row + 16 * k);
-    w[4 * k] = x.x;
-    w[4 * k + 1] = x.y;
-    w[4 * k + 2] = x.z;
-    w[4 * k + 3] = x.w;
+__device__ __forceinline__ void load_rotated(uint32_t (&w)[D / 16], const uint8_t* row, int lane) {
+  constexpr int NW = D / 16;
+  const int r = lane & (D / 4 - 1);
+  const int a = r >> 2;
+  if constexpr (D == 128) {
+    const int first = (a >> 2) & 1;
+    const uint4 x = ld_idx(row + 16 * first);
+    const uint4 y = ld_idx(row + 16 * (first ^ 1));
+    w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+    w[4] = y.x; w[5] = y.y; w[6] = y.z; w[7] = y.w;
+  } else {
+    const uint4 x = ld_idx(row);
+    w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
   }
+#pragma unroll
+  for (int s = 1; s <= 2; s <<= 1) {
+    const bool take = (a & s) != 0;
+    uint32_t t[NW];
+#pragma unroll
+    for (int i = 0; i < NW; ++i) t[i] = take ? w[(i + s) % NW] : w[i];
+#pragma unroll
+    for (int i = 0; i < NW; ++i) w[i] = t[i];
+  }
+  const int bits = 8 * (r & 3);
+  uint32_t t[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) t[i] = __funnelshift_r(w[i], w[(i + 1) % NW], bits);
+#pragma unroll
+  for (int i = 0; i < NW; ++i) w[i] = t[i];
+}
+
+// Byte offset of entry e's row (e * kCols * 4 = e << 8) for the index in
+// byte k & 3 of a word.
+__device__ __forceinline__ uint32_t entry_row(uint32_t word, int k) {
+  return __byte_perm(word, 0u, 0x4404u | ((k & 3) << 4));
 }
 
 template <int D>
@@ -91,9 +127,8 @@ vq_decode_kernel(const VqParams p) {
   require_ieee_subnormals();
   constexpr int GR = D / kVqSub;  // channel groups
   extern __shared__ __align__(16) float sm[];
-  float* lut = sm;                 // [GR][kRow]
-  uint32_t* wv = reinterpret_cast<uint32_t*>(lut + GR * kRow);  // [GR][kRow] fixed point
-  float* q_s = lut + 2 * GR * kRow;  // [D]
+  float* tab = sm;                 // [kEntries][kCols]: key table, then the value histogram
+  float* q_s = tab + kEntries * kCols;  // [D]
   float* misc = q_s + D;           // [64]
   float* sc = misc + 64;           // [kVqSlots]
 
@@ -115,20 +150,22 @@ vq_decode_kernel(const VqParams p) {
   const float* cbv = p.cb_v + cbo;
 
   for (int d = tid; d < D; d += kVqThreads) q_s[d] = __uint_as_float((uint32_t)p.q[uidx * D + d] << 16);
-  for (int i = tid; i < GR * kRow; i += kVqThreads) wv[i] = 0u;
   __syncthreads();
-  // LUT[j][e] = sum_i q[4j + i] * entry_e[4 loop + i] (thread = entry)
-  for (int i = tid; i < GR * kEntries; i += kVqThreads) {
-    const int j = i / kEntries, e = i % kEntries;
+  // T[e][c] = sum_i q[4g + i] * entry_e[4 loop + i], g = c mod GR (thread = column)
+  for (int i = tid; i < kEntries * kCols; i += kVqThreads) {
+    const int e = i / kCols, g = (i % kCols) % GR;
     const float4 c4 = __ldg(reinterpret_cast<const float4*>(cbk + (size_t)e * W));
-    const float* qq = q_s + kVqSub * j;
+    const float* qq = q_s + kVqSub * g;
     float a = qq[0] * c4.x;
     a = fmaf(qq[1], c4.y, a);
     a = fmaf(qq[2], c4.z, a);
     a = fmaf(qq[3], c4.w, a);
-    lut[j * kRow + e] = a;
+    tab[i] = a;
   }
   __syncthreads();
+  // a lane's column base: step k reads column lane + k of row e at
+  // tb + (e << 8) + 4 k
+  const char* tb = reinterpret_cast<const char*>(tab) + 4 * lane;
 
   // ---------------------------------------------------------------- pass 1
   // two tokens per lane and iteration (t and t + 32): twice the independent
@@ -138,9 +175,9 @@ vq_decode_kernel(const VqParams p) {
   constexpr int STRIDE = 64 * kVqWarps;
   float lmax = -INFINITY;
   uint32_t n0[D / 16], n1[D / 16];
-  if (p0 + 64 * warp + lane < p1) load_indices<D>(n0, ik + (size_t)(p0 + 64 * warp + lane) * GR);
+  if (p0 + 64 * warp + lane < p1) load_rotated<D>(n0, ik + (size_t)(p0 + 64 * warp + lane) * GR, lane);
   if (p0 + 64 * warp + lane + 32 < p1)
-    load_indices<D>(n1, ik + (size_t)(p0 + 64 * warp + lane + 32) * GR);
+    load_rotated<D>(n1, ik + (size_t)(p0 + 64 * warp + lane + 32) * GR, lane);
   for (int base = p0 + 64 * warp; base < p1; base += STRIDE) {
     const int t0 = base + lane, t1 = t0 + 32;
     uint32_t w0[D / 16], w1[D / 16];
@@ -149,30 +186,22 @@ vq_decode_kernel(const VqParams p) {
       w0[k] = n0[k];
       w1[k] = n1[k];
     }
-    if (t0 + STRIDE < p1) load_indices<D>(n0, ik + (size_t)(t0 + STRIDE) * GR);
-    if (t1 + STRIDE < p1) load_indices<D>(n1, ik + (size_t)(t1 + STRIDE) * GR);
+    if (t0 + STRIDE < p1) load_rotated<D>(n0, ik + (size_t)(t0 + STRIDE) * GR, lane);
+    if (t1 + STRIDE < p1) load_rotated<D>(n1, ik + (size_t)(t1 + STRIDE) * GR, lane);
     float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
     if (t1 < p1) {
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t x = w0[k], y = w1[k];
-        a0 += lut[(4 * k) * kRow + (x & 255u)];
-        b0 += lut[(4 * k) * kRow + (y & 255u)];
-        a1 += lut[(4 * k + 1) * kRow + ((x >> 8) & 255u)];
-        b1 += lut[(4 * k + 1) * kRow + ((y >> 8) & 255u)];
-        a0 += lut[(4 * k + 2) * kRow + ((x >> 16) & 255u)];
-        b0 += lut[(4 * k + 2) * kRow + ((y >> 16) & 255u)];
-        a1 += lut[(4 * k + 3) * kRow + (x >> 24)];
-        b1 += lut[(4 * k + 3) * kRow + (y >> 24)];
+      for (int k = 0; k < GR; k += 2) {
+        a0 += *reinterpret_cast<const float*>(tb + entry_row(w0[k >> 2], k) + 4 * k);
+        b0 += *reinterpret_cast<const float*>(tb + entry_row(w1[k >> 2], k) + 4 * k);
+        a1 += *reinterpret_cast<const float*>(tb + entry_row(w0[k >> 2], k + 1) + 4 * (k + 1));
+        b1 += *reinterpret_cast<const float*>(tb + entry_row(w1[k >> 2], k + 1) + 4 * (k + 1));
       }
     } else if (t0 < p1) {
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t x = w0[k];
-        a0 += lut[(4 * k) * kRow + (x & 255u)];
-        a1 += lut[(4 * k + 1) * kRow + ((x >> 8) & 255u)];
-        a0 += lut[(4 * k + 2) * kRow + ((x >> 16) & 255u)];
-        a1 += lut[(4 * k + 3) * kRow + (x >> 24)];
+      for (int k = 0; k < GR; k += 2) {
+        a0 += *reinterpret_cast<const float*>(tb + entry_row(w0[k >> 2], k) + 4 * k);
+        a1 += *reinterpret_cast<const float*>(tb + entry_row(w0[k >> 2], k + 1) + 4 * (k + 1));
       }
     }
     if (t0 < p1) {
@@ -225,10 +254,17 @@ vq_decode_kernel(const VqParams p) {
   const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
 
   // ---------------------------------------------------------------- pass 2
+  // the key table is free (every warp passed the barriers above): it becomes
+  // the value histogram
+  uint32_t* hist = reinterpret_cast<uint32_t*>(tab);
+  for (int i = tid; i < kEntries * kCols / 4; i += kVqThreads)
+    reinterpret_cast<uint4*>(hist)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  char* hb = reinterpret_cast<char*>(hist) + 4 * lane;
   const uint8_t* iv = p.idx_v + uidx * (size_t)p.cap * GR;
-  if (p0 + 64 * warp + lane < p1) load_indices<D>(n0, iv + (size_t)(p0 + 64 * warp + lane) * GR);
+  if (p0 + 64 * warp + lane < p1) load_rotated<D>(n0, iv + (size_t)(p0 + 64 * warp + lane) * GR, lane);
   if (p0 + 64 * warp + lane + 32 < p1)
-    load_indices<D>(n1, iv + (size_t)(p0 + 64 * warp + lane + 32) * GR);
+    load_rotated<D>(n1, iv + (size_t)(p0 + 64 * warp + lane + 32) * GR, lane);
   for (int base = p0 + 64 * warp; base < p1; base += STRIDE) {
     const int t0 = base + lane, t1 = t0 + 32;
     uint32_t w0[D / 16], w1[D / 16];
@@ -237,47 +273,43 @@ vq_decode_kernel(const VqParams p) {
       w0[k] = n0[k];
       w1[k] = n1[k];
     }
-    if (t0 + STRIDE < p1) load_indices<D>(n0, iv + (size_t)(t0 + STRIDE) * GR);
-    if (t1 + STRIDE < p1) load_indices<D>(n1, iv + (size_t)(t1 + STRIDE) * GR);
+    if (t0 + STRIDE < p1) load_rotated<D>(n0, iv + (size_t)(t0 + STRIDE) * GR, lane);
+    if (t1 + STRIDE < p1) load_rotated<D>(n1, iv + (size_t)(t1 + STRIDE) * GR, lane);
     if (t0 < p1) {
       const uint32_t pw = __float2uint_rn(exp2f(sc[t0 - p0] - M) * inv * 2147483648.0f);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t x = w0[k];
-        atomicAdd(&wv[(4 * k) * kRow + (x & 255u)], pw);
-        atomicAdd(&wv[(4 * k + 1) * kRow + ((x >> 8) & 255u)], pw);
-        atomicAdd(&wv[(4 * k + 2) * kRow + ((x >> 16) & 255u)], pw);
-        atomicAdd(&wv[(4 * k + 3) * kRow + (x >> 24)], pw);
-      }
+      for (int k = 0; k < GR; ++k)
+        atomicAdd(reinterpret_cast<uint32_t*>(hb + entry_row(w0[k >> 2], k) + 4 * k), pw);
     }
     if (t1 < p1) {
       const uint32_t pw = __float2uint_rn(exp2f(sc[t1 - p0] - M) * inv * 2147483648.0f);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t x = w1[k];
-        atomicAdd(&wv[(4 * k) * kRow + (x & 255u)], pw);
-        atomicAdd(&wv[(4 * k + 1) * kRow + ((x >> 8) & 255u)], pw);
-        atomicAdd(&wv[(4 * k + 2) * kRow + ((x >> 16) & 255u)], pw);
-        atomicAdd(&wv[(4 * k + 3) * kRow + (x >> 24)], pw);
-      }
+      for (int k = 0; k < GR; ++k)
+        atomicAdd(reinterpret_cast<uint32_t*>(hb + entry_row(w1[k >> 2], k) + 4 * k), pw);
     }
   }
   __syncthreads();
-  // out[4j + i] = sum_e W[j][e] * entry_e[4 loop + i]: PARTS threads per
-  // channel split the entries; the table's rows are free now
+  // out[4g + i] = sum_e W[g][e] * entry_e[4 loop + i] with W[g][e] the sum of
+  // the bins of every column of group g (integers: exact); PARTS threads per
+  // channel split the entries, their partial sums go to the free score slots
   constexpr int PARTS = kVqThreads / D;
+  constexpr int COPIES = kCols / GR;
   {
-    const int d = tid % D, part = tid / D, j = d / kVqSub, i = d % kVqSub;
+    const int d = tid % D, part = tid / D, g = d / kVqSub, i = d % kVqSub;
     float o = 0.f;
-    for (int e = part; e < kEntries; e += PARTS)
-      o = fmaf((float)wv[j * kRow + e], __ldg(cbv + (size_t)e * W + i), o);
-    lut[tid] = o * 4.656612873077393e-10f;  // 2^-31
+    for (int e = part; e < kEntries; e += PARTS) {
+      uint32_t wsum = 0u;
+#pragma unroll
+      for (int c = 0; c < COPIES; ++c) wsum += hist[e * kCols + g + c * GR];
+      o = fmaf((float)wsum, __ldg(cbv + (size_t)e * W + i), o);
+    }
+    sc[tid] = o * 4.656612873077393e-10f;  // 2^-31
   }
   __syncthreads();
   if (tid < D) {
     float o = 0.f;
 #pragma unroll
-    for (int k = 0; k < PARTS; ++k) o += lut[k * D + tid];
+    for (int k = 0; k < PARTS; ++k) o += sc[k * D + tid];
     q_s[tid] = o;  // the query is no longer needed
   }
   __syncthreads();
@@ -369,7 +401,7 @@ vq_encode_kernel(const VqEncodeParams p) {
 
 template <int D>
 constexpr size_t vq_smem() {
-  return sizeof(float) * ((size_t)2 * (D / kVqSub) * kRow + D + 64 + kVqSlots);
+  return sizeof(float) * ((size_t)kEntries * kCols + D + 64 + kVqSlots);
 }
 
 template <int D>

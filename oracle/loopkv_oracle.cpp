@@ -8,9 +8,9 @@
 // Looped Transformers", section 概要 (the abstract):
 //   * each (loop, layer) cell keeps 4-bit codes, 2-bit codes, or reuses the
 //     final loop's KV (SHARE);
-//   * a 4-bit value is read as its high 2 bits, and its low 2 bits are
-//     fetched only where the loop's own attention weights need 4-bit
-//     precision.
+//   * a 4-bit value is held as two 2-bit planes: every loop takes the upper
+//     plane, and the lower plane only for tokens whose weights in that loop
+//     call for 4-bit precision.
 // The abstract leaves the arithmetic open; this file takes these readings:
 //   R1 asymmetric min/max quantization as in "KIVI: A Tuning-Free Asymmetric
 //      2bit Quantization for KV Cache": keys per channel over a group of 32
@@ -728,12 +728,13 @@ int orc_vq_encode(int n_loops, int D, int c, const uint16_t* x, const float* cb,
 }
 
 // ---- planner ---------------------------------------------------------------
-// The plan that minimizes reads under a damage budget and a storage budget,
+// The plan with the fewest reads within a damage budget and a storage budget,
 // by trying every assignment (small instances only).  "LoopKV: Loop-Aware KV
 // Cache Compression for Serving Looped Transformers", section 概要: an offline
 // profile gives each (loop, layer) cell a predicted damage for 4-bit storage,
 // 2-bit storage and reuse of the final loop's KV (damages add); the planner
-// minimizes reads under budgets for predicted damage and storage.  Readings:
+// searches for the least data read while predicted damage and storage each
+// stay within a budget.  Readings:
 //   P1 per cached token and KV head, a 4-bit cell stores its six blocks
 //      (K hi/lo/meta, V hi/lo/meta: 6 x D/4 bytes) and reads five of them plus
 //      the low-plane row of a selected fraction sel of its tokens
