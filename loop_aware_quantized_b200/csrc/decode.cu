@@ -75,6 +75,17 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return r;
 }
 
+__device__ __forceinline__ uint2 ld_stream2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_stream1(const void* p) {
+  uint32_t r;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+
 // Packed fp32 pair arithmetic (sm_100): one instruction for two lanes of
 // work.  Round to nearest, no flush to zero.
 __device__ __forceinline__ float2 add2(float2 a, float2 b) {
@@ -508,6 +519,313 @@ __device__ __forceinline__ void key_pass(const Unit& u, int b_begin, int b_end, 
   }
 }
 
+// ------------------------------------------------- keys of a query group
+//
+// With G >= 2 query heads per KV head the key scores of a 32-token group are
+// a [G x D] by [D x 32] product: a dense contraction, so it goes to the
+// tensor cores (mma.sync m16n8k32, s8 weight digits x u8 code bytes, s32
+// accumulate), exactly, in integers.  One query keeps the FMA-pipe pass
+// above (single-query decode is not a dense contraction).
+//
+// Weights.  For query r the folded weights qs_c = q_c * scale_c of the group
+// share one power of two 2^E chosen from the warp's largest |qs|, so that
+// W_c = rint(qs_c 2^E) has |W_c| < 2^26; the score is then
+// (sum_c W_c code_c) 2^-E + sum_c q_c zero_c.
+//
+// Codes.  The hi / lo planes of a 16-channel word merge into two nibble
+// words (byte b of the even word holds channels 4b (low nibble) and 4b + 2
+// (high), the odd word channels 4b + 1 and 4b + 3): one byte carries two
+// codes, c_lo + 16 c_hi.  With X = 16 W(c_lo's channel) and
+// Y = W(c_hi's channel) - 16 W(c_lo's channel),
+//   byte * X + (byte & 0xF0) * Y = 16 (c_lo W_lo + c_hi W_hi),
+// so two products into one accumulator cover both codes without unpacking
+// them.  X and Y are split into four signed base-256 digits (byte p of
+// v + 0x80808080 as u8, minus 128; exact for |v| < 0x7F7F7F7F, and
+// |X|, |Y| < 17 * 2^26).
+//
+// Tile.  A (16 x 32, s8): row r holds digit d of query q, r = 2q + (d & 1) +
+// 8 (d >> 1), so lane group g (rows g and g + 8) holds digits d0 = g & 1 and
+// d0 + 2 of query g >> 1.  B (32 x 8, u8): column n is token n of an 8-token
+// tile; K byte 4t' + b (b < 4) of K tile kt is byte b of the even word of
+// plane word W = (D / 64) t' + kt, K byte 16 + 4t' + b the same of its odd
+// word.  D (16 x 8, s32) rows and columns follow A and B.  A lane (g, t)
+// loads the plane words W(kt, t) of tokens g + 8j, j = 0..3 (the B
+// fragments of the four token tiles), and after the products combines its
+// two digits, then the digit pair of lanes g and g ^ 1: it ends with the
+// sums of query g >> 1 for tokens 8 (2p + (g & 1)) + 2t + {0, 1}, p = 0, 1.
+
+__device__ __forceinline__ void mma_s8u8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// A lane's plane words of one key group: token g + 8j, plane word W(kt, t).
+template <int D>
+struct KTileMma {
+  uint32_t h[4][D / 64 > 0 ? D / 64 : 1], l[4][D / 64 > 0 ? D / 64 : 1];
+  float4 sc, zr;  // scales / zero points of channels 4 lane .. 4 lane + 3 (lanes < D / 4)
+};
+
+template <int D, bool Q4>
+__device__ __forceinline__ void load_ktile_mma(KTileMma<D>& k, const uint8_t* kb, size_t lo_off,
+                                               const float* km, bool meta) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if constexpr (D == 128) {
+      const uint2 hw = ld_stream2(kb + j * 128);
+      k.h[j][0] = hw.x;
+      k.h[j][1] = hw.y;
+      if constexpr (Q4) {
+        const uint2 lw = ld_stream2(kb + lo_off + j * 128);
+        k.l[j][0] = lw.x;
+        k.l[j][1] = lw.y;
+      } else {
+        k.l[j][0] = 0u;
+        k.l[j][1] = 0u;
+      }
+    } else {
+      k.h[j][0] = ld_stream1(kb + j * 128);
+      k.l[j][0] = Q4 ? ld_stream1(kb + lo_off + j * 128) : 0u;
+    }
+  }
+  if (meta) {
+    k.sc = __ldg(reinterpret_cast<const float4*>(km));
+    k.zr = __ldg(reinterpret_cast<const float4*>(km + D));
+  } else {
+    k.sc = make_float4(0.f, 0.f, 0.f, 0.f);
+    k.zr = k.sc;
+  }
+}
+
+// Nibble words of a 16-channel plane word pair (q = 4 hi + lo for 4-bit
+// keys, q = hi for 2-bit keys).
+template <bool Q4>
+__device__ __forceinline__ void nibble_words(uint32_t hi, uint32_t lo, uint32_t& ev, uint32_t& od) {
+  if constexpr (Q4) {
+    ev = ((hi << 2) & 0xCCCCCCCCu) | (lo & 0x33333333u);
+    od = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
+  } else {
+    ev = hi & 0x33333333u;
+    od = (hi >> 2) & 0x33333333u;
+  }
+}
+
+// Digit d (0..3) of four biased weights, as the signed bytes of one word.
+__device__ __forceinline__ uint32_t digit_word(int4 v, uint32_t sel) {
+  const uint32_t lo2 = __byte_perm((uint32_t)v.x, (uint32_t)v.y, sel);
+  const uint32_t hi2 = __byte_perm((uint32_t)v.z, (uint32_t)v.w, sel);
+  return __byte_perm(lo2, hi2, 0x5410u) ^ 0x80808080u;
+}
+
+// Scores of one group held in registers for the G queries.  st: the warp's
+// staging of the biased weights, [4 arrays][G][D / 4] ints (X even, X odd,
+// Y even, Y odd).  Writes (ADD: adds) the scores of positions below qlim
+// into sc[r * S + pos - p0] and raises lmax[r].
+template <int D, bool Q4, int G, bool ADD>
+__device__ __forceinline__ void key_group_mma(const KTileMma<D>& k, const float* q_s, int* st,
+                                              int gpos0, int qlim, int p0, float* sc, int S,
+                                              float sscale, int lane, float (&lmax)[G]) {
+  constexpr int KT = D / 64 > 0 ? D / 64 : 1;
+  constexpr int Q4W = D / 4;  // weights per array and query
+  const int g = lane >> 2, t = lane & 3;
+  const bool fold = lane < D / 4;
+  // ---- fold each query into the group's scales: integer weights
+  float cpart[G], finv[G];
+#pragma unroll
+  for (int r = 0; r < G; ++r) {
+    const float4 qv = fold ? *reinterpret_cast<const float4*>(q_s + r * D + 4 * lane)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float w0 = qv.x * k.sc.x, w1 = qv.y * k.sc.y, w2 = qv.z * k.sc.z, w3 = qv.w * k.sc.w;
+    cpart[r] = fmaf(qv.w, k.zr.w, fmaf(qv.z, k.zr.z, fmaf(qv.y, k.zr.y, qv.x * k.zr.x)));
+    const float amax = fmaxf(fmaxf(fabsf(w0), fabsf(w1)), fmaxf(fabsf(w2), fabsf(w3)));
+    const uint32_t mbits = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+    const int fexp = min(279 - (int)(mbits >> 23), 253);  // max |w| 2^(fexp - 127) < 2^26
+    const float F = __int_as_float(fexp << 23);
+    finv[r] = __int_as_float((254 - fexp) << 23);
+    if (fold) {
+      const int i0 = __float2int_rn(w0 * F), i1 = __float2int_rn(w1 * F);
+      const int i2 = __float2int_rn(w2 * F), i3 = __float2int_rn(w3 * F);
+      constexpr uint32_t kBias = 0x80808080u;
+      st[(0 * G + r) * Q4W + lane] = (int)((uint32_t)(16 * i0) + kBias);       // X even
+      st[(1 * G + r) * Q4W + lane] = (int)((uint32_t)(16 * i1) + kBias);       // X odd
+      st[(2 * G + r) * Q4W + lane] = (int)((uint32_t)(i2 - 16 * i0) + kBias);  // Y even
+      st[(3 * G + r) * Q4W + lane] = (int)((uint32_t)(i3 - 16 * i1) + kBias);  // Y odd
+    }
+  }
+  // zero-point terms: sum over the warp, every lane gets all G totals
+  {
+    const bool b4 = (lane & 16) != 0;
+    float kk;
+    if constexpr (G == 2) {
+      kk = (b4 ? cpart[1] : cpart[0]) + __shfl_xor_sync(0xffffffffu, b4 ? cpart[0] : cpart[1], 16);
+    } else {
+      const float r0 = __shfl_xor_sync(0xffffffffu, b4 ? cpart[0] : cpart[2], 16);
+      const float r1 = __shfl_xor_sync(0xffffffffu, b4 ? cpart[1] : cpart[3], 16);
+      const float k0 = (b4 ? cpart[2] : cpart[0]) + r0;
+      const float k1 = (b4 ? cpart[3] : cpart[1]) + r1;
+      const bool b3 = (lane & 8) != 0;
+      kk = (b3 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, b3 ? k0 : k1, 8);
+    }
+#pragma unroll
+    for (int o = (G == 2 ? 8 : 4); o > 0; o >>= 1) kk += __shfl_xor_sync(0xffffffffu, kk, o);
+#pragma unroll
+    for (int r = 0; r < G; ++r)
+      cpart[r] = __shfl_sync(0xffffffffu, kk, G == 2 ? 16 * r : 16 * (r >> 1) + 8 * (r & 1));
+  }
+  __syncwarp();
+  // ---- products: lane group g holds digits d0, d0 + 2 of query qg
+  const int qg = g >> 1, d0 = g & 1;
+  const bool qok = qg < G;
+  const uint32_t sel_lo = (uint32_t)d0 | ((uint32_t)(d0 + 4) << 4);
+  const uint32_t sel_hi = (uint32_t)(d0 + 2) | ((uint32_t)(d0 + 6) << 4);
+  int acc[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[j][i] = 0;
+#pragma unroll
+  for (int kt = 0; kt < KT; ++kt) {
+    const int W = (D / 64 > 0 ? D / 64 : 1) * t + kt;
+    uint32_t ax[4] = {0u, 0u, 0u, 0u}, ay[4] = {0u, 0u, 0u, 0u};
+    if (qok) {
+      const int qq = qg < G ? qg : 0;
+      const int4 xe = *reinterpret_cast<const int4*>(st + (0 * G + qq) * Q4W + 4 * W);
+      const int4 xo = *reinterpret_cast<const int4*>(st + (1 * G + qq) * Q4W + 4 * W);
+      const int4 ye = *reinterpret_cast<const int4*>(st + (2 * G + qq) * Q4W + 4 * W);
+      const int4 yo = *reinterpret_cast<const int4*>(st + (3 * G + qq) * Q4W + 4 * W);
+      ax[0] = digit_word(xe, sel_lo);  // row g: even bytes
+      ax[1] = digit_word(xe, sel_hi);  // row g + 8
+      ax[2] = digit_word(xo, sel_lo);  // row g: odd bytes
+      ax[3] = digit_word(xo, sel_hi);
+      ay[0] = digit_word(ye, sel_lo);
+      ay[1] = digit_word(ye, sel_hi);
+      ay[2] = digit_word(yo, sel_lo);
+      ay[3] = digit_word(yo, sel_hi);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t ev, od;
+      nibble_words<Q4>(k.h[j][kt], k.l[j][kt], ev, od);
+      mma_s8u8(acc[j], ax, ev, od);
+      mma_s8u8(acc[j], ay, ev & 0xF0F0F0F0u, od & 0xF0F0F0F0u);
+    }
+  }
+  __syncwarp();  // the staging is read; the next group may overwrite it
+  // ---- digits: rows g (digit d0) and g + 8 (d0 + 2), then lanes g, g ^ 1
+  const float flo = __int_as_float((127 + 8 * d0 - 4) << 23);   // 2^(8 d0) / 16
+  const float fhi = __int_as_float((127 + 8 * d0 + 12) << 23);  // 2^(8 (d0 + 2)) / 16
+  float v[4][2];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) v[j][c] = fmaf((float)acc[j][c + 2], fhi, (float)acc[j][c] * flo);
+  float w[2][2];
+#pragma unroll
+  for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const float keep = d0 ? v[2 * pp + 1][c] : v[2 * pp][c];
+      const float send = d0 ? v[2 * pp][c] : v[2 * pp + 1][c];
+      w[pp][c] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+  if (!qok) return;
+  float fsel = finv[0], csel = cpart[0];
+#pragma unroll
+  for (int r = 1; r < G; ++r) {
+    fsel = qg == r ? finv[r] : fsel;
+    csel = qg == r ? cpart[r] : csel;
+  }
+  const float fs = fsel * sscale, cs = csel * sscale;
+  float mx = -INFINITY;
+#pragma unroll
+  for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int pos = gpos0 + 8 * (2 * pp + d0) + 2 * t + c;
+      if (pos < qlim) {
+        const float sv = fmaf(w[pp][c], fs, cs);
+        float* dst = sc + qg * S + pos - p0;
+        if (ADD) *dst += sv;
+        else *dst = sv;
+        mx = fmaxf(mx, sv);
+      }
+    }
+  if (!ADD) {
+#pragma unroll
+    for (int r = 0; r < G; ++r)
+      if (qg == r) lmax[r] = fmaxf(lmax[r], mx);
+  }
+}
+
+// L2 requests for one key group in the tensor-core layout (see key_pass_mma).
+template <int D, bool Q4>
+__device__ __forceinline__ void prefetch_kgroup_mma(const uint8_t* kb, size_t lo_off, const float* km,
+                                                    bool pon_k, bool pon_m) {
+  if (pon_k) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      prefetch_l2(kb + j * 128);
+      if (Q4) prefetch_l2(kb + lo_off + j * 128);
+    }
+  }
+  if (pon_m) {
+    prefetch_l2(km);
+    prefetch_l2(km + D);
+  }
+}
+
+// Pass 1 for a query group on the tensor cores: as key_pass, with the
+// warp's q * scale rows (G * D floats) as the weight staging.
+template <int D, bool Q4, int G, bool ADD = false>
+__device__ __forceinline__ void key_pass_mma(const Unit& u, int b_begin, int b_end, int p0, int p1,
+                                             const float* q_s, float* qs, float* sc, int S,
+                                             float sscale, int warp, int lane, float (&lmax)[G]) {
+  static_assert(G == 2 || G == 4, "query groups of 2 or 4");
+  const int first = b_begin + warp;
+  if (first >= b_end) return;
+  const int qlim = min(p1, u.nq);
+  const int g = lane >> 2, t = lane & 3;
+  const bool meta = lane < D / 4;
+  constexpr size_t GB = 8 * D;                  // bytes of one group in each block
+  constexpr size_t STEP = (size_t)kWarps * GB;  // a warp's stride between its groups
+  const size_t lane_off = (D == 128) ? (size_t)(t >> 1) * 512 + g * 16 + (t & 1) * 8
+                                     : (size_t)g * 16 + t * 4;
+  const uint8_t* kb = u.data + u.Ld.k_hi + (size_t)first * GB + lane_off;
+  const size_t lo_off = u.Ld.k_lo - u.Ld.k_hi;
+  const float* km = reinterpret_cast<const float*>(u.data + u.Ld.k_meta + (size_t)first * GB) +
+                    (meta ? 4 * lane : 0);
+  int* st = reinterpret_cast<int*>(qs);
+  // L2 requests for the group the registers are loading: the lanes whose
+  // plane pointers start a 128-byte line request the four token rows of
+  // their chunk (K_hi, K_lo), every eighth meta lane its scale and zero lines
+  const bool pon_k = g == 0 && (t & 1) == 0 && (D == 128 || t == 0);
+  const bool pon_m = meta && (lane & 7) == 0;
+  KTileMma<D> a, b;
+  load_ktile_mma<D, Q4>(a, kb, lo_off, km, meta);
+  int bk = first;
+  for (;;) {
+    const bool hasb = bk + kWarps < b_end;
+    if (hasb) load_ktile_mma<D, Q4>(b, kb + STEP, lo_off, km + STEP / 4, meta);
+    if (kAheadK > 0 && hasb) prefetch_kgroup_mma<D, Q4>(kb + STEP, lo_off, km + STEP / 4, pon_k, pon_m);
+    key_group_mma<D, Q4, G, ADD>(a, q_s, st, bk * 32, qlim, p0, sc, S, sscale, lane, lmax);
+    if (!hasb) break;
+    bk += kWarps;
+    kb += STEP;
+    km += STEP / 4;
+    const bool hasa = bk + kWarps < b_end;
+    if (hasa) load_ktile_mma<D, Q4>(a, kb + STEP, lo_off, km + STEP / 4, meta);
+    if (kAheadK > 0 && hasa) prefetch_kgroup_mma<D, Q4>(kb + STEP, lo_off, km + STEP / 4, pon_k, pon_m);
+    key_group_mma<D, Q4, G, ADD>(b, q_s, st, bk * 32, qlim, p0, sc, S, sscale, lane, lmax);
+    if (!hasa) break;
+    bk += kWarps;
+    kb += STEP;
+    km += STEP / 4;
+  }
+}
+
 // A lane's share of a token's value row in pass 2: with G queries per KV
 // head, LPT = (D / 64) * G lanes share a token and each holds CH = 64 / G
 // channels for every query (G * CH / 2 = 32 accumulator pairs): NW plane
@@ -519,16 +837,6 @@ struct VShare {
   static constexpr int NGRP = CH >= 32 ? CH / 32 : 1;
 };
 
-__device__ __forceinline__ uint2 ld_stream2(const void* p) {
-  uint2 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-  return r;
-}
-__device__ __forceinline__ uint32_t ld_stream1(const void* p) {
-  uint32_t r;
-  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
-  return r;
-}
 
 // Asynchronous 16-byte copies global -> shared (L1 bypassed), in groups
 // that a thread waits for; the warp then syncs before reading them.
@@ -754,8 +1062,14 @@ decode_kernel(const DecodeParams p, const CellList cl) {
   float lmax[G];
 #pragma unroll
   for (int r = 0; r < G; ++r) lmax[r] = -INFINITY;
-  if (q4) key_pass<D, true, G>(u, blk0, qend, p0, p1, q_s, qs, sc, S, sscale, warp, lane, lmax);
-  else if (quant) key_pass<D, false, G>(u, blk0, qend, p0, p1, q_s, qs, sc, S, sscale, warp, lane, lmax);
+  if constexpr (G == 1) {
+    if (q4) key_pass<D, true, G>(u, blk0, qend, p0, p1, q_s, qs, sc, S, sscale, warp, lane, lmax);
+    else if (quant) key_pass<D, false, G>(u, blk0, qend, p0, p1, q_s, qs, sc, S, sscale, warp, lane, lmax);
+  } else {
+    if (q4) key_pass_mma<D, true, G>(u, blk0, qend, p0, p1, q_s, qs, sc, S, sscale, warp, lane, lmax);
+    else if (quant)
+      key_pass_mma<D, false, G>(u, blk0, qend, p0, p1, q_s, qs, sc, S, sscale, warp, lane, lmax);
+  }
   // the warp's first value block is requested now, ahead of the softmax merge
   constexpr int LPT = (D / 64) * G;  // lanes per token in pass 2
   constexpr int TPI = 32 / LPT;      // tokens per warp iteration in pass 2
@@ -816,8 +1130,12 @@ decode_kernel(const DecodeParams p, const CellList cl) {
     ur.Ld = u.Lo;
     ur.data_kind = LOOPKV_Q2;
     ur.nq = u.rtok;
-    key_pass<D, false, G, true>(ur, blk0, min(blk1, u.rtok / 32), p0, p1, q_s, qs, sc, S, sscale,
-                                warp, lane, lmax);
+    if constexpr (G == 1)
+      key_pass<D, false, G, true>(ur, blk0, min(blk1, u.rtok / 32), p0, p1, q_s, qs, sc, S, sscale,
+                                  warp, lane, lmax);
+    else
+      key_pass_mma<D, false, G, true>(ur, blk0, min(blk1, u.rtok / 32), p0, p1, q_s, qs, sc, S,
+                                      sscale, warp, lane, lmax);
     __syncthreads();
 #pragma unroll
     for (int r = 0; r < G; ++r) {

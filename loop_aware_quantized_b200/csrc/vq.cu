@@ -70,6 +70,14 @@ struct VqParams {
   int32_t len[LOOPKV_MAX_BATCH];
 };
 
+// L2 requests for the index rows a warp reads kVqAhead iterations from now
+// (the register loads cover only the next one): 64 tokens x D/4 bytes, one
+// 128-byte line per lane.
+constexpr int kVqAhead = 2;
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ uint4 ld_idx(const uint8_t* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -188,6 +196,8 @@ vq_decode_kernel(const VqParams p) {
     }
     if (t0 + STRIDE < p1) load_rotated<D>(n0, ik + (size_t)(t0 + STRIDE) * GR, lane);
     if (t1 + STRIDE < p1) load_rotated<D>(n1, ik + (size_t)(t1 + STRIDE) * GR, lane);
+    if (lane * 128 < 64 * GR && base + kVqAhead * STRIDE + lane * 128 / GR < p1)
+      prefetch_l2(ik + (size_t)(base + kVqAhead * STRIDE) * GR + lane * 128);
     float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
     if (t1 < p1) {
 #pragma unroll
@@ -218,6 +228,17 @@ vq_decode_kernel(const VqParams p) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
   if (lane == 0) misc[warp] = lmax;
+  // the value index rows of the warp's first iterations go to L2 during the
+  // softmax merge
+  {
+    const uint8_t* iv0 = p.idx_v + uidx * (size_t)p.cap * GR;
+#pragma unroll
+    for (int it = 0; it < kVqAhead; ++it) {
+      const int base = p0 + 64 * warp + it * STRIDE;
+      if (lane * 128 < 64 * GR && base + lane * 128 / GR < p1)
+        prefetch_l2(iv0 + (size_t)base * GR + lane * 128);
+    }
+  }
   __syncthreads();
   float m = misc[0];
 #pragma unroll
@@ -275,6 +296,8 @@ vq_decode_kernel(const VqParams p) {
     }
     if (t0 + STRIDE < p1) load_rotated<D>(n0, iv + (size_t)(t0 + STRIDE) * GR, lane);
     if (t1 + STRIDE < p1) load_rotated<D>(n1, iv + (size_t)(t1 + STRIDE) * GR, lane);
+    if (lane * 128 < 64 * GR && base + kVqAhead * STRIDE + lane * 128 / GR < p1)
+      prefetch_l2(iv + (size_t)(base + kVqAhead * STRIDE) * GR + lane * 128);
     if (t0 < p1) {
       const uint32_t pw = __float2uint_rn(exp2f(sc[t0 - p0] - M) * inv * 2147483648.0f);
 #pragma unroll
