@@ -18,6 +18,7 @@ copy bandwidth.  ``--impl reference`` times the CPU oracle instead.
 """
 
 import argparse
+import gc
 import hashlib
 import json
 import os
@@ -54,6 +55,13 @@ def parse():
     ap.add_argument("--batch", type=int, default=0,
                     help="sequences per GPU (default: the workload's batch); smaller "
                          "batches are for profiling captures only")
+    ap.add_argument("--seq-chunks", type=int, default=1,
+                    help="decode the batch as this many sequence sub-batches, one after the "
+                         "other, each with its own cache (for a batch whose KV cache exceeds "
+                         "the GPU); a step's time is the sum over sub-batches")
+    ap.add_argument("--cell-chunks", type=int, default=1,
+                    help="decode the cells as this many loop-aligned chunks, each with its own "
+                         "cache (plans without SHARE / RES2 cells); a step's time is the sum")
     return ap.parse_args()
 
 
@@ -628,6 +636,125 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def time_chunk(args, wl, dev, world, cells_g, seqs, n0, G, total_steps, sampler, keep=False):
+    """Build the cache of `cells_g` (global cell ids, whole loops) for the
+    global sequences `seqs` and time args.steps decode steps on it (append
+    one token to every cell and decode them, in serving order) after
+    args.warmup untimed ones.  Returns the device times, the decode launches'
+    algorithmic bytes and, with keep=True, what the end-to-end leg reuses."""
+    import torch
+    import torch.distributed as dist
+
+    from loop_aware_quantized_b200 import Plan, query_sizes, steps
+    from synth.gpu import DeviceGenerator
+
+    B, H, D = len(seqs), wl.n_heads, wl.head_dim
+    n_loops = len(cells_g) // wl.n_layers
+    kinds = np.asarray(wl.kinds)[cells_g]
+    # each sequence's capacity: its context, the steps' new tokens and a group of headroom
+    cap = (n0.astype(np.int64) + total_steps + 32 + 31) // 32 * 32
+    cap = cap.astype(np.int32)
+    _, need = query_sizes(n_loops, wl.n_layers, H, D, cap, kinds, wl.tau, q_per_kv=G)
+    free, _ = torch.cuda.mem_get_info(dev)
+    if need > 0.92 * free:
+        raise SystemExit("the KV cache of %d sequences needs %.1f GB, %.1f GB are free: decode "
+                         "the batch in sub-batches (--seq-chunks) or the cells in chunks "
+                         "(--cell-chunks)" % (B, need / 1e9, free / 1e9))
+    plan = Plan(n_loops, wl.n_layers, H, D, cap, kinds, wl.tau, device=dev, q_per_kv=G)
+    gen = DeviceGenerator(wl, dev)
+    local_of = {c: i for i, c in enumerate(cells_g)}
+
+    # build the cache: every token of every cell through the append kernel
+    # (the final loop first: RES2 cells quantize against it)
+    t_build = time.perf_counter()
+    kbuf = vbuf = None
+    final = [c for c in cells_g if c // wl.n_layers == wl.n_loops - 1]
+    for c in final + [c for c in cells_g if c not in final]:
+        kbuf, vbuf = gen.kv([c], seqs, np.zeros(B, np.int32), int(n0.max()), k=kbuf, v=vbuf)
+        plan.append([local_of[c]], kbuf, vbuf, n_new=n0)
+    del kbuf, vbuf
+    torch.cuda.synchronize()
+    build_s = time.perf_counter() - t_build
+    torch.cuda.empty_cache()
+
+    phase_l = steps.phases(n_loops, wl.n_layers)
+    phase_g = [[cells_g[i] for i in ph] for ph in phase_l]
+
+    def step_inputs(s):
+        """Inputs of step s: the token at position n0 + s of every cell, and the
+        queries of units holding n0 + s + 1 tokens."""
+        q, k, v = [], [], []
+        for cells in phase_g:
+            kk, vv = gen.kv(list(cells), seqs, n0 + s, 1)
+            k.append(kk)
+            v.append(vv)
+            q.append(gen.queries(list(cells), seqs, np.tile(n0 + s + 1, (len(cells), 1)), g=G))
+        return q, k, v
+
+    n_dev_steps = args.warmup + args.steps
+    inputs = [step_inputs(s) for s in range(n_dev_steps)]
+    oshape = (B, H, G, D) if G > 1 else (B, H, D)
+    outs = [torch.empty((len(c),) + oshape, dtype=torch.float32, device=dev) for c in phase_l]
+    nsels = [[torch.zeros((len(c), B, H), dtype=torch.int32, device=dev) for c in phase_l]
+             for _ in range(args.steps)]
+    stream = torch.cuda.current_stream()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in phase_l] for _ in range(args.steps)]
+
+    for s in range(args.warmup):
+        q, k, v = inputs[s]
+        steps.decode_step(plan, phase_l, q, k, v, outs)
+    torch.cuda.synchronize()
+
+    if sampler.proc is None:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        q, k, v = inputs[args.warmup + i]
+        steps.decode_step(plan, phase_l, q, k, v, outs, nsel=nsels[i], events=ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = sum(a.elapsed_time(b) for row in ev for (a, b) in row)
+    plan.check()
+
+    # algorithmic bytes of every decode launch in the timed region
+    dec_bytes = 0
+    for i in range(args.steps):
+        s = args.warmup + i
+        for pi, cells in enumerate(phase_g):
+            lens_own = n0 + s + 1
+            # non-final loops decode before the final loop's append of this step
+            lens_src = n0 + s if (pi == 0 and len(phase_g) > 1) else n0 + s + 1
+            dec_bytes += decode_bytes(wl, cells, lens_own, lens_src, int(nsels[i][pi].sum()), G)
+    # per phase: an append and a decode launch for the plain cells and one
+    # each for RES2 cells (when the phase has them); the appends commit the
+    # lengths themselves
+    launches_per_step = sum(2 * (int(any(wl.kinds[c] != 4 for c in cells)) +
+                                 int(any(wl.kinds[c] == 4 for c in cells)))
+                            for cells in phase_g)
+    out = {"elapsed_ms": elapsed_ms, "dec_ms": dec_ms, "dec_bytes": dec_bytes,
+           "build_s": build_s, "dec_launches": args.steps * len(phase_g),
+           "launches": launches_per_step * args.steps, "cache_bytes": plan.cache_bytes}
+    if keep:
+        out.update(plan=plan, phase=phase_l, inputs=inputs, outs=outs, step_inputs=step_inputs)
+    else:
+        # give this chunk's cache back to the device before the next chunk
+        plan.close()
+        plan.cache = plan.table = None
+        del plan, gen, inputs, outs, nsels, ev
+        gc.collect()
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -644,9 +771,8 @@ def main():
     import torch.distributed as dist
     from datetime import timedelta
 
-    from loop_aware_quantized_b200 import Plan, steps
+    from loop_aware_quantized_b200 import steps
     from synth import workloads as W
-    from synth.gpu import DeviceGenerator
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -660,106 +786,55 @@ def main():
         wl.lengths = wl.lengths[:args.batch]
         wl.capacity = wl.capacity[:args.batch]
     B, H, D = wl.batch, wl.n_heads, wl.head_dim
-    # weak scaling: every rank serves its own batch of B sequences
-    seqs = shard_sequences(rank, B)
-    n0 = wl.lengths[:B].astype(np.int32)
-    total_steps = args.warmup + args.steps + (0 if args.no_e2e else args.warmup + args.steps)
-    cap = np.full(B, int(n0.max()) + total_steps + 32, np.int32)
-    cap = (cap + 31) // 32 * 32
     G = args.q_per_kv
-    from loop_aware_quantized_b200 import query_sizes
-    _, need = query_sizes(wl.n_loops, wl.n_layers, H, D, cap, wl.kinds, wl.tau, q_per_kv=G)
-    free, _ = torch.cuda.mem_get_info(dev)
-    if need > 0.92 * free:
-        raise SystemExit("the KV cache of %d sequences needs %.1f GB, %.1f GB are free: pass a "
-                         "smaller --batch (the workload is decoded in sequence sub-batches)"
-                         % (B, need / 1e9, free / 1e9))
-    plan = Plan(wl.n_loops, wl.n_layers, H, D, cap, wl.kinds, wl.tau, device=dev, q_per_kv=G)
-    gen = DeviceGenerator(wl, dev)
-
-    # build the cache: every token of every cell through the append kernel
-    # (the final loop first: RES2 cells quantize against it)
-    t_build = time.perf_counter()
-    kbuf = vbuf = None
-    final = list(range((wl.n_loops - 1) * wl.n_layers, wl.n_cells))
-    for c in final + [c for c in range(wl.n_cells) if c not in final]:
-        kbuf, vbuf = gen.kv([c], seqs, np.zeros(B, np.int32), int(n0.max()), k=kbuf, v=vbuf)
-        plan.append([c], kbuf, vbuf, n_new=n0)
-    del kbuf, vbuf
-    torch.cuda.synchronize()
-    build_s = time.perf_counter() - t_build
-    torch.cuda.empty_cache()
-
-    phase = steps.phases(wl.n_loops, wl.n_layers)
-
-    def step_inputs(s):
-        """Inputs of step s: the token at position n0 + s of every cell, and the
-        queries of units holding n0 + s + 1 tokens."""
-        q, k, v = [], [], []
-        for cells in phase:
-            kk, vv = gen.kv(list(cells), seqs, n0 + s, 1)
-            k.append(kk)
-            v.append(vv)
-            q.append(gen.queries(list(cells), seqs, np.tile(n0 + s + 1, (len(cells), 1)), g=G))
-        return q, k, v
-
-    n_dev_steps = args.warmup + args.steps
-    inputs = [step_inputs(s) for s in range(n_dev_steps)]
-    oshape = (B, H, G, D) if G > 1 else (B, H, D)
-    outs = [torch.empty((len(c),) + oshape, dtype=torch.float32, device=dev) for c in phase]
-    nsels = [[torch.zeros((len(c), B, H), dtype=torch.int32, device=dev) for c in phase]
-             for _ in range(args.steps)]
-    stream = torch.cuda.current_stream()
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in phase] for _ in range(args.steps)]
-
-    for s in range(args.warmup):
-        q, k, v = inputs[s]
-        steps.decode_step(plan, phase, q, k, v, outs)
-    torch.cuda.synchronize()
+    # weak scaling: every rank serves its own batch of B sequences
+    seqs_all = shard_sequences(rank, B)
+    if B % args.seq_chunks:
+        raise SystemExit("--seq-chunks must divide the batch (%d)" % B)
+    sb = B // args.seq_chunks
+    if wl.n_loops % args.cell_chunks:
+        raise SystemExit("--cell-chunks must divide the loops (%d)" % wl.n_loops)
+    if args.cell_chunks > 1 and any(int(k) in (2, 4) for k in wl.kinds):
+        raise SystemExit("--cell-chunks needs a plan without SHARE / RES2 cells")
+    lpc = wl.n_loops // args.cell_chunks
+    chunks = []
+    for si in range(args.seq_chunks):
+        for ci in range(args.cell_chunks):
+            cells = list(range(ci * lpc * wl.n_layers, (ci + 1) * lpc * wl.n_layers))
+            chunks.append((cells, list(range(si * sb, (si + 1) * sb))))
+    whole = len(chunks) == 1
+    total_steps = args.warmup + args.steps + (0 if (args.no_e2e or not whole)
+                                              else args.warmup + args.steps)
+    n0_all = wl.lengths[:B].astype(np.int32)
 
     sampler = ClockSampler(local)
-    sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(args.steps):
-        q, k, v = inputs[args.warmup + i]
-        steps.decode_step(plan, phase, q, k, v, outs, nsel=nsels[i], events=ev[i])
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    runs = []
+    for cells_g, idx in chunks:
+        seqs = [seqs_all[i] for i in idx]
+        runs.append(time_chunk(args, wl, dev, world, cells_g, seqs, n0_all[idx], G, total_steps,
+                               sampler, keep=whole))
     clocks = sampler.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    dec_ms = sum(a.elapsed_time(b) for row in ev for (a, b) in row)
-    plan.check()
-
-    # algorithmic bytes of every decode launch in the timed region
-    dec_bytes = 0
-    for i in range(args.steps):
-        s = args.warmup + i
-        for pi, cells in enumerate(phase):
-            lens_own = n0 + s + 1
-            # non-final loops decode before the final loop's append of this step
-            lens_src = n0 + s if pi == 0 else n0 + s + 1
-            dec_bytes += decode_bytes(wl, cells, lens_own, lens_src, int(nsels[i][pi].sum()), G)
+    elapsed_ms = sum(r["elapsed_ms"] for r in runs)
+    dec_ms = sum(r["dec_ms"] for r in runs)
+    dec_bytes = sum(r["dec_bytes"] for r in runs)
+    build_s = sum(r["build_s"] for r in runs)
+    n_dec_launches = sum(r["dec_launches"] for r in runs)
+    launches = sum(r["launches"] for r in runs)
+    cache_gb = max(r["cache_bytes"] for r in runs) / 1e9
+    n0 = n0_all
 
     elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], world, dev)
     ms_per_step = elapsed_ms / args.steps
     value = wl.n_cells * world / (ms_per_step / 1000.0)
-    # per phase: an append and a decode launch for the plain cells and one
-    # each for RES2 cells (when the phase has them), and the length commit
-    launches_per_step = sum(1 + 2 * (int(any(wl.kinds[c] != 4 for c in cells)) +
-                                     int(any(wl.kinds[c] == 4 for c in cells)))
-                            for cells in phase)
 
     # ---- end to end through the API: pinned host inputs in, outputs out
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and whole:
+        r0 = runs[0]
+        plan, phase, inputs, outs, step_inputs = (r0["plan"], r0["phase"], r0["inputs"],
+                                                   r0["outs"], r0["step_inputs"])
+        n_dev_steps = args.warmup + args.steps
+        stream = torch.cuda.current_stream()
         host_in = []
         for s in range(args.steps):
             q, k, v = step_inputs(n_dev_steps + s)
@@ -820,7 +895,6 @@ def main():
 
     peak, peak_kind = measured_peaks()
     achieved = dec_bytes / (dec_ms / 1000.0) / 1e9 if dec_ms > 0 else 0.0
-    n_dec_launches = args.steps * len(phase)
     tr = ncu_traffic()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak,
@@ -832,8 +906,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v1, desc, _ = oracle_baseline(args.config, args.cpu_seconds, seqs, G)
-        v, cores = oracle_all_cores(args.config, seqs, G, cpu_seconds=2 * args.cpu_seconds)
+        v1, desc, _ = oracle_baseline(args.config, args.cpu_seconds, seqs_all, G)
+        v, cores = oracle_all_cores(args.config, seqs_all, G, cpu_seconds=2 * args.cpu_seconds)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": "one process per host core, each timing its own sample like this one: "
                          "%s; on one core alone: %.4g cell-steps/s" % (desc, v1)}
@@ -849,20 +923,27 @@ def main():
                        "global_batch": B * world, "seq_len": int(n0[0]),
                        "parallelism": "dp%d (independent sequences)" % world,
                        "q_per_kv": G,
-                       "l2": "inputs larger than L2 (KV cache %.1f GB)" % (plan.cache_bytes / 1e9),
+                       "l2": "inputs larger than L2 (KV cache %.1f GB)" % cache_gb,
                        "build_s": build_s},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": launches,
             # attended (position, KV head) pairs decoded per second, all cells
             "token_head_cells_per_s": float(wl.n_cells * H * world *
                                             np.sum(n0 + args.warmup + args.steps // 2 + 1)) /
                                       (ms_per_step / 1000.0),
             "clocks": clocks,
         }
+        if not whole:
+            line["config"]["chunks"] = (
+                "%d sequence sub-batch(es) x %d cell chunk(s), decoded one after the other, each "
+                "with its own cache (largest %.1f GB); a step's time is the sum over chunks"
+                % (args.seq_chunks, args.cell_chunks, cache_gb))
         print(json.dumps(line), flush=True)
-    plan.close()
+    for r in runs:
+        if r.get("plan") is not None:
+            r["plan"].close()
     if world > 1:
         dist.destroy_process_group()
 

@@ -10,11 +10,13 @@
 // are done with explicit round-to-nearest intrinsics (no contraction), so the
 // codes are the ones any IEEE implementation of the same steps produces.
 //
-// One CTA per (cell, sequence, head) unit.  New tokens fill the bf16
-// residual; every 32-position group that becomes complete is quantized by
-// one warp through a padded shared-memory tile, then the remaining tokens
-// are written to the residual.  Lengths are advanced by a second, tiny
-// kernel once every head of the unit has read the old length.
+// One CTA per (cell, sequence, head) unit (several for a bulk append).
+// New tokens fill the bf16 residual; every 32-position group that becomes
+// complete is quantized by one warp through a padded shared-memory tile,
+// then the remaining tokens are written to the residual.  The CTAs of a
+// (cell, sequence) pair all read its old length; the last of them to finish
+// stores the new one (an arrival count in the plan table), so no second
+// launch is needed.
 
 #include <cuda_runtime.h>
 
@@ -47,6 +49,21 @@ __device__ __forceinline__ float group_scale(float mn, float mx, int qmax) {
 __device__ __forceinline__ float canon_zero(float mn) { return mn == 0.0f ? 0.0f : mn; }
 
 __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// The length commit of a (cell, sequence) pair: each of its `expected` CTAs
+// arrives once it is done; the last one stores n_old + n_new and resets the
+// count for the next launch.  Every CTA read the old length before it
+// arrived, so none of them sees the new one.
+__device__ __forceinline__ void arrive_commit(DevSeq* e, int n_old, int n_new, unsigned expected) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&e->arrive, 1u) == expected - 1u) {
+      e->len = n_old + n_new;
+      e->arrive = 0u;
+    }
+  }
+}
 
 constexpr int kCodeRow = 16;  // padding bytes of a code-tile row (D + 16 bytes)
 
@@ -171,15 +188,19 @@ append_kernel(const AppendParams p, const CellList cl) {
 
   const TableHeader* hdr = reinterpret_cast<const TableHeader*>(p.table);
   const DevCell* cells = reinterpret_cast<const DevCell*>(p.table + table_cells_offset());
-  const DevSeq* seqs = reinterpret_cast<const DevSeq*>(p.table + table_seqs_offset(hdr->n_cells));
+  DevSeq* seqs = reinterpret_cast<DevSeq*>(p.table + table_seqs_offset(hdr->n_cells));
   const DevCell c = cells[cell];
-  const DevSeq s = seqs[(size_t)cell * hdr->max_batch + b];
+  DevSeq* const entry = seqs + (size_t)cell * hdr->max_batch + b;
+  const DevSeq s = *entry;
   const int kind = c.kind;
   const int n_old = s.len;
   if (n_old < 0 || (kind != LOOPKV_SHARE && n_old + n_new > s.cap)) {
+    // host checks make this unreachable; flag it, leave the unit and its
+    // length alone (every CTA of the pair takes this branch)
     if (threadIdx.x == 0 && chunk == 0) atomicOr(reinterpret_cast<uint32_t*>(p.table), kStatusLength);
     return;
   }
+  const unsigned expected = (unsigned)(H * p.chunks);
   uint8_t* base = p.cache + s.offset + (size_t)h * s.stride;
   const UnitLayout L = unit_layout(kind, D, s.cap);
   const size_t in_off = (((size_t)cl.out[ci] * p.batch + b) * H + h) * (size_t)p.n_new_max * D;
@@ -187,14 +208,16 @@ append_kernel(const AppendParams p, const CellList cl) {
   const uint16_t* vin = p.v + in_off;
 
   if (kind == LOOPKV_SHARE) {
-    if (chunk != 0) return;
-    // keep only the last appended token as the current one
-    const uint4* ks = reinterpret_cast<const uint4*>(kin + (size_t)(n_new - 1) * D);
-    const uint4* vs = reinterpret_cast<const uint4*>(vin + (size_t)(n_new - 1) * D);
-    for (int i = threadIdx.x; i < D / 8; i += kAppendThreads) {
-      reinterpret_cast<uint4*>(base + L.cur_k)[i] = ks[i];
-      reinterpret_cast<uint4*>(base + L.cur_v)[i] = vs[i];
+    if (chunk == 0) {
+      // keep only the last appended token as the current one
+      const uint4* ks = reinterpret_cast<const uint4*>(kin + (size_t)(n_new - 1) * D);
+      const uint4* vs = reinterpret_cast<const uint4*>(vin + (size_t)(n_new - 1) * D);
+      for (int i = threadIdx.x; i < D / 8; i += kAppendThreads) {
+        reinterpret_cast<uint4*>(base + L.cur_k)[i] = ks[i];
+        reinterpret_cast<uint4*>(base + L.cur_v)[i] = vs[i];
+      }
     }
+    arrive_commit(entry, n_old, n_new, expected);
     return;
   }
   if (kind == LOOPKV_BF16) {
@@ -209,6 +232,7 @@ append_kernel(const AppendParams p, const CellList cl) {
       kd[i] = reinterpret_cast<const uint4*>(kin + t * D)[cc];
       vd[i] = reinterpret_cast<const uint4*>(vin + t * D)[cc];
     }
+    arrive_commit(entry, n_old, n_new, expected);
     return;
   }
 
@@ -262,7 +286,10 @@ append_kernel(const AppendParams p, const CellList cl) {
     __syncwarp();
   }
   __syncthreads();  // flushed groups have read the old residual
-  if (chunk != 0) return;
+  if (chunk != 0) {
+    arrive_commit(entry, n_old, n_new, expected);
+    return;
+  }
 
   // remaining tokens go to the residual
   const int r_first = (qtok1 > qtok0) ? qtok1 : n_old;  // first position to write
@@ -278,6 +305,7 @@ append_kernel(const AppendParams p, const CellList cl) {
     reinterpret_cast<uint4*>(rv + (size_t)slot * D * 2)[cc] =
         reinterpret_cast<const uint4*>(vin + (size_t)(pos - n_old) * D)[cc];
   }
+  arrive_commit(entry, n_old, n_new, expected);
 }
 
 // The reference's stored key / value at (pos, d) dequantized in fp32, the
@@ -344,9 +372,10 @@ append_res2_kernel(const AppendParams p, const CellList cl) {
 
   const TableHeader* hdr = reinterpret_cast<const TableHeader*>(p.table);
   const DevCell* cells = reinterpret_cast<const DevCell*>(p.table + table_cells_offset());
-  const DevSeq* seqs = reinterpret_cast<const DevSeq*>(p.table + table_seqs_offset(hdr->n_cells));
+  DevSeq* seqs = reinterpret_cast<DevSeq*>(p.table + table_seqs_offset(hdr->n_cells));
   const DevCell c = cells[cell];
-  const DevSeq s = seqs[(size_t)cell * hdr->max_batch + b];
+  DevSeq* const entry = seqs + (size_t)cell * hdr->max_batch + b;
+  const DevSeq s = *entry;
   const DevCell rc = cells[c.src];
   const DevSeq rs = seqs[(size_t)c.src * hdr->max_batch + b];
   const int rkind = rc.kind;
@@ -360,6 +389,7 @@ append_res2_kernel(const AppendParams p, const CellList cl) {
     if (threadIdx.x == 0 && chunk == 0) atomicOr(reinterpret_cast<uint32_t*>(p.table), kStatusLength);
     return;
   }
+  const unsigned expected = (unsigned)(H * p.chunks);
   uint8_t* base = p.cache + s.offset + (size_t)h * s.stride;
   const uint8_t* rbase = p.cache + rs.offset + (size_t)h * rs.stride;
   const UnitLayout L = unit_layout(LOOPKV_RES2, D, s.cap);
@@ -403,7 +433,10 @@ append_res2_kernel(const AppendParams p, const CellList cl) {
     __syncwarp();
   }
   __syncthreads();  // every group has read its window slots
-  if (chunk != 0) return;
+  if (chunk != 0) {
+    arrive_commit(entry, n_old, n_new, expected);
+    return;
+  }
 
   // new tokens past the residual-coded range go to their window slots
   const int first = n_old > q1 ? n_old : q1;
@@ -418,16 +451,7 @@ append_res2_kernel(const AppendParams p, const CellList cl) {
     reinterpret_cast<uint4*>(rv + slot)[cc] =
         reinterpret_cast<const uint4*>(vin + (size_t)(pos - n_old) * D)[cc];
   }
-}
-
-__global__ void commit_lengths_kernel(uint8_t* table, const CellList cl, int n_cells, int batch,
-                                      const AppendParams p) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n_cells * batch) return;
-  const int ci = i / batch, b = i % batch;
-  const TableHeader* hdr = reinterpret_cast<const TableHeader*>(table);
-  DevSeq* seqs = reinterpret_cast<DevSeq*>(table + table_seqs_offset(hdr->n_cells));
-  seqs[(size_t)cl.cell[ci] * hdr->max_batch + b].len += p.n_new[b];
+  arrive_commit(entry, n_old, n_new, expected);
 }
 
 template <int D>
@@ -457,16 +481,6 @@ int launch_append(const AppendParams& p, const CellList& cells, void* stream, in
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (head_dim == 64) return launch_append_t<64>(p, cells, s, res2);
   return launch_append_t<128>(p, cells, s, res2);
-}
-
-int launch_commit_lengths(uint8_t* table, const CellList& cells, int n_cells, int batch,
-                          const int32_t* n_new, void* stream) {
-  AppendParams p{};
-  for (int b = 0; b < batch; ++b) p.n_new[b] = n_new[b];
-  const int n = n_cells * batch;
-  commit_lengths_kernel<<<(n + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      table, cells, n_cells, batch, p);
-  return (int)cudaGetLastError();
 }
 
 }  // namespace loopkv

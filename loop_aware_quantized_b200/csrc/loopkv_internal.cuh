@@ -42,7 +42,8 @@ struct DevSeq {                // 32 bytes per (cell, sequence)
   uint64_t stride;             // bytes of one head's region
   int32_t cap;                 // capacity in tokens
   int32_t len;                 // tokens stored
-  int32_t pad[2];
+  uint32_t arrive;             // append CTAs done with this pair in the running launch (0 between)
+  int32_t pad;
 };
 static_assert(sizeof(DevSeq) == 32, "seq entry size");
 
@@ -148,8 +149,6 @@ struct DecodeParams {
 // is cell i's index in the caller's list (its slot of the inputs / outputs).
 int launch_append(const AppendParams& p, const CellList& cells, void* stream, int head_dim,
                   bool res2);
-int launch_commit_lengths(uint8_t* table, const CellList& cells, int n_cells, int batch,
-                          const int32_t* n_new, void* stream);
 int launch_decode(const DecodeParams& p, const CellList& cells, void* stream, int head_dim,
                   bool res2);
 int decode_max_slots(int head_dim, int group);  // largest per-query score slots per CTA

@@ -257,7 +257,6 @@ loopkv_status loopkv_append(loopkv_plan* p, const int32_t* h_cells, int32_t n_ce
     ap.n_cells = n_res;
     e = launch_append(ap, res, stream, p->D, true);
   }
-  if (e == 0) e = launch_commit_lengths(p->d_table, cl, n_cells, batch, h_n_new, stream);
   if (e != 0) return LOOPKV_ERR_CUDA;
   for (int i = 0; i < n_cells; ++i)
     for (int b = 0; b < batch; ++b) p->L(cl.cell[i], b) += h_n_new[b];

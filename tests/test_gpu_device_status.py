@@ -115,3 +115,36 @@ def test_append_flags_a_unit_whose_device_length_is_negative(built, cuda_device)
     for h in range(wl.n_heads):
         assert torch.equal(plan.unit_bytes(cell, b, h), before[h])   # nothing written
     assert not torch.equal(plan.unit_bytes(cell, 1, 0), others)      # the rest appended
+
+
+def test_appends_commit_lengths_and_reset_their_arrival_counts(cuda_device):
+    # the CTAs of a (cell, sequence) pair count their arrivals in the table;
+    # the last one stores the new length and resets the count to zero.  A
+    # bulk build of 1000 tokens spreads each unit over three CTAs.
+    import torch
+    from synth.gpu import DeviceGenerator
+    spec = (2, 2, 2, 64, (Q4, SH, Q2, Q4), (1000, 600), (1120, 704), 0.01)
+    wl = W.custom(*spec)
+    seqs = [0, 1]
+    plan = GH.make_plan(wl, seqs)
+    gen = DeviceGenerator(wl, cuda_device)
+    GH.build_cache(wl, plan, gen, seqs, wl.lengths)
+    cells = list(range(wl.n_cells))
+    lens = wl.lengths.astype(np.int32).copy()
+
+    def check():
+        torch.cuda.synchronize()
+        plan.check()
+        host = plan.lengths()
+        for c in cells:
+            for b in seqs:
+                assert _device_length(plan, c, b) == host[c, b] == lens[b]
+                off = _len_offset(plan, c, b) + 4
+                assert int(plan.table[off:off + 4].cpu().view(torch.int32).item()) == 0
+
+    check()
+    for n_new in (1, 1, 5, 31, 60):            # token by token, a flush, a few groups
+        k, v = gen.kv(cells, seqs, lens, n_new)
+        plan.append(cells, k, v)
+        lens += n_new
+        check()
