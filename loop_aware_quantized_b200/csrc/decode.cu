@@ -562,6 +562,14 @@ __device__ __forceinline__ void mma_s8u8(int (&c)[4], const uint32_t (&a)[4], ui
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // A lane's plane words of one key group: token g + 8j, plane word W(kt, t).
 template <int D>
 struct KTileMma {
@@ -620,6 +628,83 @@ __device__ __forceinline__ uint32_t digit_word(int4 v, uint32_t sel) {
   return __byte_perm(lo2, hi2, 0x5410u) ^ 0x80808080u;
 }
 
+// Products and digits of a group for two queries, tokens in the tile's
+// rows: A (16 x 32, u8) = the code bytes of 16 tokens (lane (g, t) holds the
+// even and odd nibble words of plane word W(kt, t) of tokens g and g + 8 of
+// the M tile), B (32 x 8, s8) = the weight digits, column n = digit n & 3 of
+// query n >> 2.  Every row and column is used, so two queries take half the
+// products of the query-digit layout.  Lane (g, t) receives digits
+// 2 (t & 1) and 2 (t & 1) + 1 of query t >> 1 for tokens g and g + 8; with
+// lane t ^ 1 (the other two digits) it completes one token per M tile:
+// token 16 mt + g + 8 (t & 1).
+template <int D, bool Q4, bool ADD>
+__device__ __forceinline__ void key_products_g2(const KTileMma<D>& k, const int* st,
+                                                const float (&finv)[2], const float (&cpart)[2],
+                                                int gpos0, int qlim, int p0, float* sc, int S,
+                                                float sscale, int lane, float (&lmax)[2]) {
+  constexpr int KT = D / 64 > 0 ? D / 64 : 1;
+  constexpr int Q4W = D / 4;
+  const int g = lane >> 2, t = lane & 3;
+  const int qn = g >> 2, dn = g & 3;  // this lane's B column: digit dn of query qn
+  const uint32_t sel = (uint32_t)dn | ((uint32_t)(dn + 4) << 4);
+  int acc[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[mt][i] = 0;
+#pragma unroll
+  for (int kt = 0; kt < KT; ++kt) {
+    const int W = (D / 64 > 0 ? D / 64 : 1) * t + kt;
+    const int4 xe = *reinterpret_cast<const int4*>(st + (0 * 2 + qn) * Q4W + 4 * W);
+    const int4 xo = *reinterpret_cast<const int4*>(st + (1 * 2 + qn) * Q4W + 4 * W);
+    const int4 ye = *reinterpret_cast<const int4*>(st + (2 * 2 + qn) * Q4W + 4 * W);
+    const int4 yo = *reinterpret_cast<const int4*>(st + (3 * 2 + qn) * Q4W + 4 * W);
+    const uint32_t bx0 = digit_word(xe, sel), bx1 = digit_word(xo, sel);
+    const uint32_t by0 = digit_word(ye, sel), by1 = digit_word(yo, sel);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      uint32_t e0, o0, e1, o1;
+      nibble_words<Q4>(k.h[2 * mt][kt], k.l[2 * mt][kt], e0, o0);          // token g + 16 mt
+      nibble_words<Q4>(k.h[2 * mt + 1][kt], k.l[2 * mt + 1][kt], e1, o1);  // token g + 8 + 16 mt
+      const uint32_t ax[4] = {e0, e1, o0, o1};
+      const uint32_t ay[4] = {e0 & 0xF0F0F0F0u, e1 & 0xF0F0F0F0u, o0 & 0xF0F0F0F0u,
+                              o1 & 0xF0F0F0F0u};
+      mma_u8s8(acc[mt], ax, bx0, bx1);
+      mma_u8s8(acc[mt], ay, by0, by1);
+    }
+  }
+  __syncwarp();  // the staging is read; the next group may overwrite it
+  // columns 2t, 2t + 1: digits d1 = 2 (t & 1) and d1 + 1 of query t >> 1
+  const int d1 = 2 * (t & 1);
+  const float f0 = __int_as_float((127 + 8 * d1 - 4) << 23);   // 2^(8 d1) / 16
+  const float f1 = __int_as_float((127 + 8 * d1 + 4) << 23);   // 2^(8 (d1 + 1)) / 16
+  const bool up = (t & 1) != 0;
+  const int qq = t >> 1;
+  const float fs = (qq ? finv[1] : finv[0]) * sscale;
+  const float cs = (qq ? cpart[1] : cpart[0]) * sscale;
+  float mx = -INFINITY;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    const float vg = fmaf((float)acc[mt][1], f1, (float)acc[mt][0] * f0);   // row g
+    const float vg8 = fmaf((float)acc[mt][3], f1, (float)acc[mt][2] * f0);  // row g + 8
+    // lanes t, t ^ 1 hold the other digit pair of the same query: the
+    // lower one completes row g, the upper one row g + 8
+    const float tot = (up ? vg8 : vg) + __shfl_xor_sync(0xffffffffu, up ? vg : vg8, 1);
+    const int pos = gpos0 + 16 * mt + g + (up ? 8 : 0);
+    if (pos < qlim) {
+      const float sv = fmaf(tot, fs, cs);
+      float* dst = sc + qq * S + pos - p0;
+      if (ADD) *dst += sv;
+      else *dst = sv;
+      mx = fmaxf(mx, sv);
+    }
+  }
+  if (!ADD) {
+    if (qq) lmax[1] = fmaxf(lmax[1], mx);
+    else lmax[0] = fmaxf(lmax[0], mx);
+  }
+}
+
 // Scores of one group held in registers for the G queries.  st: the warp's
 // staging of the biased weights, [4 arrays][G][D / 4] ints (X even, X odd,
 // Y even, Y odd).  Writes (ADD: adds) the scores of positions below qlim
@@ -676,6 +761,10 @@ __device__ __forceinline__ void key_group_mma(const KTileMma<D>& k, const float*
       cpart[r] = __shfl_sync(0xffffffffu, kk, G == 2 ? 16 * r : 16 * (r >> 1) + 8 * (r & 1));
   }
   __syncwarp();
+  if constexpr (G == 2) {
+    key_products_g2<D, Q4, ADD>(k, st, finv, cpart, gpos0, qlim, p0, sc, S, sscale, lane, lmax);
+    return;
+  }
   // ---- products: lane group g holds digits d0, d0 + 2 of query qg
   const int qg = g >> 1, d0 = g & 1;
   const bool qok = qg < G;
