@@ -11,17 +11,18 @@
 // One CTA (8 warps) per (layer, sequence, KV head, split); splits of a long
 // sequence form a thread-block cluster and merge through DSMEM.
 //   table   T[e][c] = <q_g, entry_e's loop slice> for channel group
-//           g = c mod (D/4), over 64 columns c (each group appears in 2
-//           columns at D = 128, 4 at D = 64): the query is folded into the
-//           codebook once, so a token's score is D/4 shared-memory lookups;
-//   pass 1  lane = token.  At step k a lane reads group (lane + k) mod (D/4)
-//           of its token from column lane + k: the 32 lanes of a warp then
-//           touch 32 consecutive columns, i.e. 32 different banks, whatever
+//           g = c mod (D/4), over 32 columns c (each group once at D = 128,
+//           twice at D = 64): the query is folded into the codebook once,
+//           so a token's score is D/4 shared-memory lookups;
+//   pass 1  lane = token.  At step k a lane reads group (lane ^ k) mod (D/4)
+//           of its token from column lane ^ k: the 32 lanes of a warp then
+//           touch 32 different columns, i.e. 32 different banks, whatever
 //           the indices are (a table laid out by group would put a warp's 32
-//           random entries of one group on random banks).  Each lane rotates
-//           its token's D/4 index bytes by its lane number once, so the byte
-//           step k needs sits at a fixed register position; scores stay in
-//           shared memory (log2 units);
+//           random entries of one group on random banks).  Each lane
+//           permutes its token's D/4 index bytes by its lane number once, so
+//           the byte step k needs sits at a fixed register position, and the
+//           address is one logic op: (e << 7) | (4 lane ^ 4 k); scores stay
+//           in shared memory (log2 units);
 //   softmax the CTA's max and sum of exponentials, merged over the cluster;
 //   pass 2  the same walk adds p_t into a histogram over the value codebook
 //           laid out like the table: p_t as a fixed-point integer (units of
@@ -34,7 +35,10 @@
 //   output  out[4g + i] = 2^-31 sum_e W[g][e] * entry_e[4l + i].
 // The index streams are read once (D/2 bytes per token at D = 128: 32 key
 // and 32 value bytes); the work per token is D/2 shared-memory accesses,
-// one bank-conflict-free wavefront per warp instruction.
+// one bank-conflict-free wavefront per warp instruction.  The 32-column
+// table (32 KB) keeps a CTA at 66 KB of shared memory and 80 registers, so
+// three CTAs share an SM: the kernel waits on index loads, and the extra
+// warps hide that latency.
 
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
@@ -53,8 +57,8 @@ constexpr int kVqThreads = 256;
 constexpr int kVqWarps = kVqThreads / 32;
 constexpr int kVqSub = 4;        // channels per sub-vector
 constexpr int kEntries = 256;    // codebook entries (one byte)
-constexpr int kCols = 64;         // table / histogram columns: column c is group c mod (D/4)
-constexpr int kVqSlots = 8448;   // score slots per CTA (two CTAs per SM; 16K + a few hundred tokens in two)
+constexpr int kCols = 32;         // table / histogram columns: column c is group c mod (D/4)
+constexpr int kVqSlots = 8448;   // score slots per CTA (16K + a few hundred tokens in a cluster of two)
 constexpr int kVqMaxSplit = 8;   // portable cluster size
 
 struct VqParams {
@@ -86,13 +90,13 @@ __device__ __forceinline__ uint4 ld_idx(const uint8_t* p) {
   return r;
 }
 
-// The D/4 indices of a token as D/16 words, rotated left by r = lane mod
-// (D/4) bytes: byte m of word k holds the index of group (4k + m + r) mod
-// (D/4).  At D = 128 a rotation by four words is the choice of which 16-byte
-// half to load first; the rest is two conditional word rotations and one
-// funnel shift per word.
+// The D/4 indices of a token as D/16 words, permuted by r = lane mod (D/4):
+// byte p of the result (byte p & 3 of word p >> 2) is index p ^ r of the
+// token.  At D = 128 the word permutation's top bit is the choice of which
+// 16-byte half to load first; its other two bits are conditional swaps of
+// word pairs, and one byte permute per word applies r & 3.
 template <int D>
-__device__ __forceinline__ void load_rotated(uint32_t (&w)[D / 16], const uint8_t* row, int lane) {
+__device__ __forceinline__ void load_xored(uint32_t (&w)[D / 16], const uint8_t* row, int lane) {
   constexpr int NW = D / 16;
   const int r = lane & (D / 4 - 1);
   const int a = r >> 2;
@@ -111,26 +115,24 @@ __device__ __forceinline__ void load_rotated(uint32_t (&w)[D / 16], const uint8_
     const bool take = (a & s) != 0;
     uint32_t t[NW];
 #pragma unroll
-    for (int i = 0; i < NW; ++i) t[i] = take ? w[(i + s) % NW] : w[i];
+    for (int i = 0; i < NW; ++i) t[i] = take ? w[i ^ s] : w[i];
 #pragma unroll
     for (int i = 0; i < NW; ++i) w[i] = t[i];
   }
-  const int bits = 8 * (r & 3);
-  uint32_t t[NW];
+  const int b = r & 3;
+  const uint32_t sel = (uint32_t)(b | ((1 ^ b) << 4) | ((2 ^ b) << 8) | ((3 ^ b) << 12));
 #pragma unroll
-  for (int i = 0; i < NW; ++i) t[i] = __funnelshift_r(w[i], w[(i + 1) % NW], bits);
-#pragma unroll
-  for (int i = 0; i < NW; ++i) w[i] = t[i];
+  for (int i = 0; i < NW; ++i) w[i] = __byte_perm(w[i], 0u, sel);
 }
 
-// Byte offset of entry e's row (e * kCols * 4 = e << 8) for the index in
+// Byte offset of entry e's row (e * kCols * 4 = e << 7), e the index in
 // byte k & 3 of a word.
 __device__ __forceinline__ uint32_t entry_row(uint32_t word, int k) {
-  return __byte_perm(word, 0u, 0x4404u | ((k & 3) << 4));
+  return __byte_perm(word, 0u, 0x4404u | ((k & 3) << 4)) >> 1;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kVqThreads, 2)
+__global__ void __launch_bounds__(kVqThreads, 3)
 vq_decode_kernel(const VqParams p) {
   require_ieee_subnormals();
   constexpr int GR = D / kVqSub;  // channel groups
@@ -171,9 +173,9 @@ vq_decode_kernel(const VqParams p) {
     tab[i] = a;
   }
   __syncthreads();
-  // a lane's column base: step k reads column lane + k of row e at
-  // tb + (e << 8) + 4 k
-  const char* tb = reinterpret_cast<const char*>(tab) + 4 * lane;
+  // step k reads column lane ^ k of row e, at byte (e << 7) | (4 lane ^ 4 k)
+  const char* tb = reinterpret_cast<const char*>(tab);
+  const uint32_t l4 = 4u * (uint32_t)lane;
 
   // ---------------------------------------------------------------- pass 1
   // two tokens per lane and iteration (t and t + 32): twice the independent
@@ -183,9 +185,9 @@ vq_decode_kernel(const VqParams p) {
   constexpr int STRIDE = 64 * kVqWarps;
   float lmax = -INFINITY;
   uint32_t n0[D / 16], n1[D / 16];
-  if (p0 + 64 * warp + lane < p1) load_rotated<D>(n0, ik + (size_t)(p0 + 64 * warp + lane) * GR, lane);
+  if (p0 + 64 * warp + lane < p1) load_xored<D>(n0, ik + (size_t)(p0 + 64 * warp + lane) * GR, lane);
   if (p0 + 64 * warp + lane + 32 < p1)
-    load_rotated<D>(n1, ik + (size_t)(p0 + 64 * warp + lane + 32) * GR, lane);
+    load_xored<D>(n1, ik + (size_t)(p0 + 64 * warp + lane + 32) * GR, lane);
   for (int base = p0 + 64 * warp; base < p1; base += STRIDE) {
     const int t0 = base + lane, t1 = t0 + 32;
     uint32_t w0[D / 16], w1[D / 16];
@@ -194,24 +196,24 @@ vq_decode_kernel(const VqParams p) {
       w0[k] = n0[k];
       w1[k] = n1[k];
     }
-    if (t0 + STRIDE < p1) load_rotated<D>(n0, ik + (size_t)(t0 + STRIDE) * GR, lane);
-    if (t1 + STRIDE < p1) load_rotated<D>(n1, ik + (size_t)(t1 + STRIDE) * GR, lane);
+    if (t0 + STRIDE < p1) load_xored<D>(n0, ik + (size_t)(t0 + STRIDE) * GR, lane);
+    if (t1 + STRIDE < p1) load_xored<D>(n1, ik + (size_t)(t1 + STRIDE) * GR, lane);
     if (lane * 128 < 64 * GR && base + kVqAhead * STRIDE + lane * 128 / GR < p1)
       prefetch_l2(ik + (size_t)(base + kVqAhead * STRIDE) * GR + lane * 128);
     float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
     if (t1 < p1) {
 #pragma unroll
       for (int k = 0; k < GR; k += 2) {
-        a0 += *reinterpret_cast<const float*>(tb + entry_row(w0[k >> 2], k) + 4 * k);
-        b0 += *reinterpret_cast<const float*>(tb + entry_row(w1[k >> 2], k) + 4 * k);
-        a1 += *reinterpret_cast<const float*>(tb + entry_row(w0[k >> 2], k + 1) + 4 * (k + 1));
-        b1 += *reinterpret_cast<const float*>(tb + entry_row(w1[k >> 2], k + 1) + 4 * (k + 1));
+        a0 += *reinterpret_cast<const float*>(tb + (entry_row(w0[k >> 2], k) | (l4 ^ (4u * k))));
+        b0 += *reinterpret_cast<const float*>(tb + (entry_row(w1[k >> 2], k) | (l4 ^ (4u * k))));
+        a1 += *reinterpret_cast<const float*>(tb + (entry_row(w0[k >> 2], k + 1) | (l4 ^ (4u * (k + 1)))));
+        b1 += *reinterpret_cast<const float*>(tb + (entry_row(w1[k >> 2], k + 1) | (l4 ^ (4u * (k + 1)))));
       }
     } else if (t0 < p1) {
 #pragma unroll
       for (int k = 0; k < GR; k += 2) {
-        a0 += *reinterpret_cast<const float*>(tb + entry_row(w0[k >> 2], k) + 4 * k);
-        a1 += *reinterpret_cast<const float*>(tb + entry_row(w0[k >> 2], k + 1) + 4 * (k + 1));
+        a0 += *reinterpret_cast<const float*>(tb + (entry_row(w0[k >> 2], k) | (l4 ^ (4u * k))));
+        a1 += *reinterpret_cast<const float*>(tb + (entry_row(w0[k >> 2], k + 1) | (l4 ^ (4u * (k + 1)))));
       }
     }
     if (t0 < p1) {
@@ -281,11 +283,11 @@ vq_decode_kernel(const VqParams p) {
   for (int i = tid; i < kEntries * kCols / 4; i += kVqThreads)
     reinterpret_cast<uint4*>(hist)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
-  char* hb = reinterpret_cast<char*>(hist) + 4 * lane;
+  char* hb = reinterpret_cast<char*>(hist);
   const uint8_t* iv = p.idx_v + uidx * (size_t)p.cap * GR;
-  if (p0 + 64 * warp + lane < p1) load_rotated<D>(n0, iv + (size_t)(p0 + 64 * warp + lane) * GR, lane);
+  if (p0 + 64 * warp + lane < p1) load_xored<D>(n0, iv + (size_t)(p0 + 64 * warp + lane) * GR, lane);
   if (p0 + 64 * warp + lane + 32 < p1)
-    load_rotated<D>(n1, iv + (size_t)(p0 + 64 * warp + lane + 32) * GR, lane);
+    load_xored<D>(n1, iv + (size_t)(p0 + 64 * warp + lane + 32) * GR, lane);
   for (int base = p0 + 64 * warp; base < p1; base += STRIDE) {
     const int t0 = base + lane, t1 = t0 + 32;
     uint32_t w0[D / 16], w1[D / 16];
@@ -294,21 +296,21 @@ vq_decode_kernel(const VqParams p) {
       w0[k] = n0[k];
       w1[k] = n1[k];
     }
-    if (t0 + STRIDE < p1) load_rotated<D>(n0, iv + (size_t)(t0 + STRIDE) * GR, lane);
-    if (t1 + STRIDE < p1) load_rotated<D>(n1, iv + (size_t)(t1 + STRIDE) * GR, lane);
+    if (t0 + STRIDE < p1) load_xored<D>(n0, iv + (size_t)(t0 + STRIDE) * GR, lane);
+    if (t1 + STRIDE < p1) load_xored<D>(n1, iv + (size_t)(t1 + STRIDE) * GR, lane);
     if (lane * 128 < 64 * GR && base + kVqAhead * STRIDE + lane * 128 / GR < p1)
       prefetch_l2(iv + (size_t)(base + kVqAhead * STRIDE) * GR + lane * 128);
     if (t0 < p1) {
       const uint32_t pw = __float2uint_rn(exp2f(sc[t0 - p0] - M) * inv * 2147483648.0f);
 #pragma unroll
       for (int k = 0; k < GR; ++k)
-        atomicAdd(reinterpret_cast<uint32_t*>(hb + entry_row(w0[k >> 2], k) + 4 * k), pw);
+        atomicAdd(reinterpret_cast<uint32_t*>(hb + (entry_row(w0[k >> 2], k) | (l4 ^ (4u * k)))), pw);
     }
     if (t1 < p1) {
       const uint32_t pw = __float2uint_rn(exp2f(sc[t1 - p0] - M) * inv * 2147483648.0f);
 #pragma unroll
       for (int k = 0; k < GR; ++k)
-        atomicAdd(reinterpret_cast<uint32_t*>(hb + entry_row(w1[k >> 2], k) + 4 * k), pw);
+        atomicAdd(reinterpret_cast<uint32_t*>(hb + (entry_row(w1[k >> 2], k) | (l4 ^ (4u * k)))), pw);
     }
   }
   __syncthreads();
