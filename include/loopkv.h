@@ -151,7 +151,9 @@ typedef struct {
 } loopkv_plan_desc;
 
 typedef struct {
-  size_t table_bytes; /* device plan table (cells, lengths, status word) */
+  size_t table_bytes; /* device plan table: the plan's device state (cells,
+                         per-(cell, sequence) regions and lengths, the
+                         appends' arrival counts, the status word) */
   size_t cache_bytes; /* device KV cache in the canonical layout */
 } loopkv_sizes;
 
