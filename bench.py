@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--cell-chunks", type=int, default=1,
                     help="decode the cells as this many loop-aligned chunks, each with its own "
                          "cache (plans without SHARE / RES2 cells); a step's time is the sum")
+    ap.add_argument("--decode-split", type=int, default=0,
+                    help="CTAs per decoded unit at least (0: the library chooses); for "
+                         "launch-shape sweeps")
     return ap.parse_args()
 
 
@@ -660,7 +663,8 @@ def time_chunk(args, wl, dev, world, cells_g, seqs, n0, G, total_steps, sampler,
         raise SystemExit("the KV cache of %d sequences needs %.1f GB, %.1f GB are free: decode "
                          "the batch in sub-batches (--seq-chunks) or the cells in chunks "
                          "(--cell-chunks)" % (B, need / 1e9, free / 1e9))
-    plan = Plan(n_loops, wl.n_layers, H, D, cap, kinds, wl.tau, device=dev, q_per_kv=G)
+    plan = Plan(n_loops, wl.n_layers, H, D, cap, kinds, wl.tau, device=dev, q_per_kv=G,
+                decode_split=args.decode_split)
     gen = DeviceGenerator(wl, dev)
     local_of = {c: i for i, c in enumerate(cells_g)}
 
@@ -935,6 +939,8 @@ def main():
                                       (ms_per_step / 1000.0),
             "clocks": clocks,
         }
+        if args.decode_split:
+            line["config"]["decode_split"] = args.decode_split
         if not whole:
             line["config"]["chunks"] = (
                 "%d sequence sub-batch(es) x %d cell chunk(s), decoded one after the other, each "

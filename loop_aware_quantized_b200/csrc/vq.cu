@@ -21,8 +21,9 @@
 //           random entries of one group on random banks).  Each lane
 //           permutes its token's D/4 index bytes by its lane number once, so
 //           the byte step k needs sits at a fixed register position, and the
-//           address is one logic op: (e << 7) | (4 lane ^ 4 k); scores stay
-//           in shared memory (log2 units);
+//           address is a byte permute and one logic op:
+//           (e << 8) | (4 lane ^ 4 k); scores stay in shared memory (log2
+//           units);
 //   softmax the CTA's max and sum of exponentials, merged over the cluster;
 //   pass 2  the same walk adds p_t into a histogram over the value codebook
 //           laid out like the table: p_t as a fixed-point integer (units of
@@ -33,12 +34,18 @@
 //           lands in one bin, so an output moves by at most n 2^-32 times
 //           the largest codebook magnitude;
 //   output  out[4g + i] = 2^-31 sum_e W[g][e] * entry_e[4l + i].
+// Shared memory is 256-byte rows: row e holds the 32 table (histogram)
+// columns of entry e in its first half and 32 score slots in its second, so
+// an entry's row offset is its index byte moved up one byte (no shift).  The
+// codebooks' loop slices (256 x 16 bytes) are copied to shared memory once
+// (the key slice before the table build, the value slice while the
+// histogram fills), so neither the table build nor the output sum waits on
+// L2 inside its loop.
 // The index streams are read once (D/2 bytes per token at D = 128: 32 key
 // and 32 value bytes); the work per token is D/2 shared-memory accesses,
-// one bank-conflict-free wavefront per warp instruction.  The 32-column
-// table (32 KB) keeps a CTA at 66 KB of shared memory and 80 registers, so
-// three CTAs share an SM: the kernel waits on index loads, and the extra
-// warps hide that latency.
+// one bank-conflict-free wavefront per warp instruction.  A CTA holds 70 KB
+// of shared memory and 80 registers, so three CTAs share an SM: the kernel
+// waits on index loads, and the extra warps hide that latency.
 
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
@@ -80,6 +87,16 @@ struct VqParams {
 constexpr int kVqAhead = 2;
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// 16-byte asynchronous copy global -> shared (L1 bypassed).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+               ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ uint4 ld_idx(const uint8_t* p) {
@@ -125,10 +142,19 @@ __device__ __forceinline__ void load_xored(uint32_t (&w)[D / 16], const uint8_t*
   for (int i = 0; i < NW; ++i) w[i] = __byte_perm(w[i], 0u, sel);
 }
 
-// Byte offset of entry e's row (e * kCols * 4 = e << 7), e the index in
-// byte k & 3 of a word.
+// Shared-memory rows are 256 bytes: row e holds the 32 table (or
+// histogram) columns of entry e in its first 128 bytes and score slots
+// 32 e .. 32 e + 31 in its second 128.  Byte offset of entry e's row
+// (e << 8), e the index in byte k & 3 of a word: one byte permute.
+constexpr int kRow = 256;
+constexpr int kRowSlots = kEntries * 32;  // score slots held in the rows
 __device__ __forceinline__ uint32_t entry_row(uint32_t word, int k) {
-  return __byte_perm(word, 0u, 0x4404u | ((k & 3) << 4)) >> 1;
+  return __byte_perm(word, 0u, 0x4404u | ((k & 3) << 4));
+}
+// Score slot s: in the second half of row s / 32, else in the overflow.
+__device__ __forceinline__ float* slot(char* rows, float* over, int s) {
+  return s < kRowSlots ? reinterpret_cast<float*>(rows + ((s >> 5) << 8) + 128 + ((s & 31) << 2))
+                       : over + (s - kRowSlots);
 }
 
 template <int D>
@@ -137,10 +163,11 @@ vq_decode_kernel(const VqParams p) {
   require_ieee_subnormals();
   constexpr int GR = D / kVqSub;  // channel groups
   extern __shared__ __align__(16) float sm[];
-  float* tab = sm;                 // [kEntries][kCols]: key table, then the value histogram
-  float* q_s = tab + kEntries * kCols;  // [D]
-  float* misc = q_s + D;           // [64]
-  float* sc = misc + 64;           // [kVqSlots]
+  char* rows = reinterpret_cast<char*>(sm);  // [kEntries][kRow]: table / histogram, score slots
+  float* q_s = sm + kEntries * kRow / 4;     // [D]
+  float* misc = q_s + D;                     // [64]
+  float* over = misc + 64;                   // [kVqSlots - kRowSlots] score slots, then partials
+  float* cbs = over + (kVqSlots - kRowSlots);  // [kEntries][4]: a codebook's loop slice
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = p.split;
@@ -159,22 +186,25 @@ vq_decode_kernel(const VqParams p) {
   const float* cbk = p.cb_k + cbo;
   const float* cbv = p.cb_v + cbo;
 
+  static_assert(kVqThreads == kEntries, "one thread per codebook entry stages its slice");
+  cp_async16(cbs + kVqSub * tid, cbk + (size_t)tid * W);
   for (int d = tid; d < D; d += kVqThreads) q_s[d] = __uint_as_float((uint32_t)p.q[uidx * D + d] << 16);
+  cp_async_wait_all();
   __syncthreads();
   // T[e][c] = sum_i q[4g + i] * entry_e[4 loop + i], g = c mod GR (thread = column)
   for (int i = tid; i < kEntries * kCols; i += kVqThreads) {
     const int e = i / kCols, g = (i % kCols) % GR;
-    const float4 c4 = __ldg(reinterpret_cast<const float4*>(cbk + (size_t)e * W));
+    const float4 c4 = *reinterpret_cast<const float4*>(cbs + kVqSub * e);
     const float* qq = q_s + kVqSub * g;
     float a = qq[0] * c4.x;
     a = fmaf(qq[1], c4.y, a);
     a = fmaf(qq[2], c4.z, a);
     a = fmaf(qq[3], c4.w, a);
-    tab[i] = a;
+    *reinterpret_cast<float*>(rows + e * kRow + 4 * (i % kCols)) = a;
   }
   __syncthreads();
-  // step k reads column lane ^ k of row e, at byte (e << 7) | (4 lane ^ 4 k)
-  const char* tb = reinterpret_cast<const char*>(tab);
+  // step k reads column lane ^ k of row e, at byte (e << 8) | (4 lane ^ 4 k)
+  const char* tb = rows;
   const uint32_t l4 = 4u * (uint32_t)lane;
 
   // ---------------------------------------------------------------- pass 1
@@ -218,12 +248,12 @@ vq_decode_kernel(const VqParams p) {
     }
     if (t0 < p1) {
       const float s = (a0 + a1) * p.score_scale;
-      sc[t0 - p0] = s;
+      *slot(rows, over, t0 - p0) = s;
       lmax = fmaxf(lmax, s);
     }
     if (t1 < p1) {
       const float s = (b0 + b1) * p.score_scale;
-      sc[t1 - p0] = s;
+      *slot(rows, over, t1 - p0) = s;
       lmax = fmaxf(lmax, s);
     }
   }
@@ -246,7 +276,7 @@ vq_decode_kernel(const VqParams p) {
 #pragma unroll
   for (int k = 1; k < kVqWarps; ++k) m = fmaxf(m, misc[k]);
   float ls = 0.f;
-  for (int i = tid; i < p1 - p0; i += kVqThreads) ls += exp2f(sc[i] - m);
+  for (int i = tid; i < p1 - p0; i += kVqThreads) ls += exp2f(*slot(rows, over, i) - m);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
   if (lane == 0) misc[8 + warp] = ls;
@@ -279,11 +309,15 @@ vq_decode_kernel(const VqParams p) {
   // ---------------------------------------------------------------- pass 2
   // the key table is free (every warp passed the barriers above): it becomes
   // the value histogram
-  uint32_t* hist = reinterpret_cast<uint32_t*>(tab);
   for (int i = tid; i < kEntries * kCols / 4; i += kVqThreads)
-    reinterpret_cast<uint4*>(hist)[i] = make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(rows + (i >> 3) * kRow + 16 * (i & 7)) = make_uint4(0u, 0u, 0u, 0u);
+  // the value codebook's slice replaces the key one (read by the table build,
+  // which every thread finished before the barriers above); it arrives
+  // while the histogram fills
+  cp_async16(cbs + kVqSub * tid, cbv + (size_t)tid * W);
+  asm volatile("cp.async.commit_group;" ::: "memory");
   __syncthreads();
-  char* hb = reinterpret_cast<char*>(hist);
+  char* hb = rows;
   const uint8_t* iv = p.idx_v + uidx * (size_t)p.cap * GR;
   if (p0 + 64 * warp + lane < p1) load_xored<D>(n0, iv + (size_t)(p0 + 64 * warp + lane) * GR, lane);
   if (p0 + 64 * warp + lane + 32 < p1)
@@ -301,22 +335,23 @@ vq_decode_kernel(const VqParams p) {
     if (lane * 128 < 64 * GR && base + kVqAhead * STRIDE + lane * 128 / GR < p1)
       prefetch_l2(iv + (size_t)(base + kVqAhead * STRIDE) * GR + lane * 128);
     if (t0 < p1) {
-      const uint32_t pw = __float2uint_rn(exp2f(sc[t0 - p0] - M) * inv * 2147483648.0f);
+      const uint32_t pw = __float2uint_rn(exp2f(*slot(rows, over, t0 - p0) - M) * inv * 2147483648.0f);
 #pragma unroll
       for (int k = 0; k < GR; ++k)
         atomicAdd(reinterpret_cast<uint32_t*>(hb + (entry_row(w0[k >> 2], k) | (l4 ^ (4u * k)))), pw);
     }
     if (t1 < p1) {
-      const uint32_t pw = __float2uint_rn(exp2f(sc[t1 - p0] - M) * inv * 2147483648.0f);
+      const uint32_t pw = __float2uint_rn(exp2f(*slot(rows, over, t1 - p0) - M) * inv * 2147483648.0f);
 #pragma unroll
       for (int k = 0; k < GR; ++k)
         atomicAdd(reinterpret_cast<uint32_t*>(hb + (entry_row(w1[k >> 2], k) | (l4 ^ (4u * k)))), pw);
     }
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
   // out[4g + i] = sum_e W[g][e] * entry_e[4 loop + i] with W[g][e] the sum of
   // the bins of every column of group g (integers: exact); PARTS threads per
-  // channel split the entries, their partial sums go to the free score slots
+  // channel split the entries, their partial sums go to the overflow slots
   constexpr int PARTS = kVqThreads / D;
   constexpr int COPIES = kCols / GR;
   {
@@ -325,16 +360,17 @@ vq_decode_kernel(const VqParams p) {
     for (int e = part; e < kEntries; e += PARTS) {
       uint32_t wsum = 0u;
 #pragma unroll
-      for (int c = 0; c < COPIES; ++c) wsum += hist[e * kCols + g + c * GR];
-      o = fmaf((float)wsum, __ldg(cbv + (size_t)e * W + i), o);
+      for (int c = 0; c < COPIES; ++c)
+        wsum += *reinterpret_cast<const uint32_t*>(rows + e * kRow + 4 * (g + c * GR));
+      o = fmaf((float)wsum, cbs[kVqSub * e + i], o);
     }
-    sc[tid] = o * 4.656612873077393e-10f;  // 2^-31
+    over[tid] = o * 4.656612873077393e-10f;  // 2^-31
   }
   __syncthreads();
   if (tid < D) {
     float o = 0.f;
 #pragma unroll
-    for (int k = 0; k < PARTS; ++k) o += sc[k * D + tid];
+    for (int k = 0; k < PARTS; ++k) o += over[k * D + tid];
     q_s[tid] = o;  // the query is no longer needed
   }
   __syncthreads();
@@ -426,7 +462,9 @@ vq_encode_kernel(const VqEncodeParams p) {
 
 template <int D>
 constexpr size_t vq_smem() {
-  return sizeof(float) * ((size_t)kEntries * kCols + D + 64 + kVqSlots);
+  static_assert(kVqSlots - kRowSlots >= kVqThreads, "the overflow slots hold the partial sums");
+  return (size_t)kEntries * kRow +
+         sizeof(float) * ((size_t)D + 64 + (kVqSlots - kRowSlots) + kEntries * kVqSub);
 }
 
 template <int D>
