@@ -1525,22 +1525,42 @@ decode_kernel(const DecodeParams p, const CellList cl) {
       acc[r][i].x = fmaf(acc[r][i].x, pow2(149 - kSub - code2_off(j)), gcon);
       acc[r][i].y = fmaf(acc[r][i].y, pow2(149 - kSub - code2_off(j + 1)), gcon);
     }
-#pragma unroll
-  for (int r = 0; r < G; ++r)
-#pragma unroll
-    for (int i = 0; i < 32 / G; ++i) {
-#pragma unroll
-      for (int o = 16; o >= LPT; o >>= 1) {
-        acc[r][i].x += __shfl_xor_sync(0xffffffffu, acc[r][i].x, o);
-        acc[r][i].y += __shfl_xor_sync(0xffffffffu, acc[r][i].y, o);
-      }
-    }
-  if (lane < LPT) {
+  {
+    // transposed butterfly over the TPI lanes with the same lane % LPT: each
+    // step keeps half of the values (the upper half where the step's lane
+    // bit is set) and adds the partner's copy of them, so the lane ends with
+    // NVL consecutive sums of the flattened [G][CH] slice, from index
+    // 2 (lane - lane % LPT) on
+    constexpr int NV = G * VS::CH;    // 64
+    constexpr int NVL = 2 * LPT;      // = NV / TPI
+    float v[NV];
 #pragma unroll
     for (int r = 0; r < G; ++r)
 #pragma unroll
-      for (int i = 0; i < 32 / G; ++i)
-        reinterpret_cast<float2*>(red + (warp * G + r) * D + lane * VS::CH)[i] = acc[r][i];
+      for (int i = 0; i < VS::CH / 2; ++i) {
+        v[r * VS::CH + 2 * i] = acc[r][i].x;
+        v[r * VS::CH + 2 * i + 1] = acc[r][i].y;
+      }
+#pragma unroll
+    for (int o = 16; o >= LPT; o >>= 1) {
+      const int half = NV * o / 32;
+      const bool up = (lane & o) != 0;
+#pragma unroll
+      for (int j = 0; j < half; ++j) {
+        const float keep = up ? v[j + half] : v[j];
+        const float send = up ? v[j] : v[j + half];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    const int base = 2 * (lane - hf);  // flattened index of v[0]
+    float* dst = red + (warp * G + base / VS::CH) * D + hf * VS::CH + base % VS::CH;
+    if constexpr (NVL == 2) {
+      *reinterpret_cast<float2*>(dst) = make_float2(v[0], v[1]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < NVL / 4; ++k)
+        reinterpret_cast<float4*>(dst)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+    }
   }
   if (lane == 0) misc[80 + warp] = __int_as_float(nsel);
   __syncthreads();

@@ -322,8 +322,10 @@ loopkv_status decode_launch(loopkv_plan* p, const CellList& cl, int n_cells, int
                             float* d_lse, uint32_t* d_mask, int32_t mask_words, int32_t* d_nsel,
                             void* stream) {
   // Split a unit over a cluster of CTAs when its positions do not fit one
-  // CTA's score slots (per query of the group), or when there are too few
-  // units to fill the GPU.
+  // CTA's score slots (per query of the group), or when the units fall short
+  // of one full wave (two CTAs on each of the 148 SMs): every extra CTA of a
+  // unit costs its own start, merge and reduction, which outweighs a fuller
+  // last wave once the first wave is full.
   const int max_slots = decode_max_slots(p->D, p->group);
   const long long units = (long long)n_cells * batch * p->H;
   int split = 1;
@@ -333,7 +335,7 @@ loopkv_status decode_launch(loopkv_plan* p, const CellList& cl, int n_cells, int
   if (p->min_split > 1) {
     split = std::max(split, p->min_split);
   } else {
-    while (units * split < 148 * 4 && split < decode_max_split() && npos_max / (2 * split) >= 512)
+    while (units * split < 148 * 2 && split < decode_max_split() && npos_max / (2 * split) >= 512)
       split *= 2;
   }
   DecodeParams dp{};
