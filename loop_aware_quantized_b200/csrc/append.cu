@@ -31,10 +31,21 @@ constexpr int kAppendThreads = 128;
 constexpr int kAppendWarps = kAppendThreads / 32;
 
 // Quantize x (fp32) of a 32-value group: returns the code, given the
-// group's min and scale.  scale == 0 gives 0.
-__device__ __forceinline__ uint32_t quant_code(float x, float mn, float scale, int qmax) {
+// group's min, scale and inv = rn(1 / scale).  scale == 0 gives 0.
+// The code is rne(q) of the IEEE quotient q = rn(x - mn) / scale without a
+// division per code: with a normal inv, r = rn(rn(x - mn) * inv) differs
+// from q by less than 2^-23 relative, i.e. by less than 2^-19 for
+// q <= 15 (q <= qmax (1 + 2^-24) since scale = rn(range / qmax)), so
+// rne(r) = rne(q) unless r lies within 2^-19 of a half-integer; there (the
+// test uses 2^-16) the exact quotient is taken.  r - floor(r) and its
+// distance to 0.5 are exact (Sterbenz), and a NaN or infinite r falls back
+// too, so the codes equal the division's for every input.
+__device__ __forceinline__ uint32_t quant_code(float x, float mn, float scale, float inv, int qmax) {
   if (scale == 0.0f) return 0u;
-  const float r = __fdiv_rn(__fsub_rn(x, mn), scale);
+  const float d = __fsub_rn(x, mn);
+  float r = __fmul_rn(d, inv);
+  const float f = __fsub_rn(r, floorf(r));
+  if (!(fabsf(__fsub_rn(f, 0.5f)) > 0x1p-16f) || !(inv >= 0x1p-125f)) r = __fdiv_rn(d, scale);
   int c = __float2int_rn(r);  // round half to even
   c = c < 0 ? 0 : (c > qmax ? qmax : c);
   return (uint32_t)c;
@@ -83,7 +94,9 @@ __device__ __forceinline__ void quantize_key_group(X x, uint8_t* codes, float* k
       mx = fmaxf(mx, x(t, d));
     }
     const float sc = group_scale(mn, mx, qmax);
-    for (int t = 0; t < 32; ++t) codes[t * (D + kCodeRow) + d] = (uint8_t)quant_code(x(t, d), mn, sc, qmax);
+    const float inv = sc == 0.0f ? 0.0f : __frcp_rn(sc);
+    for (int t = 0; t < 32; ++t)
+      codes[t * (D + kCodeRow) + d] = (uint8_t)quant_code(x(t, d), mn, sc, inv, qmax);
     kmeta[d] = sc;
     kmeta[D + d] = canon_zero(mn);
   }
@@ -136,10 +149,11 @@ __device__ __forceinline__ void quantize_value_row(V v, bool q4, int qmax, uint4
       mx = fmaxf(mx, v(32 * j + e));
     }
     const float sc = group_scale(mn, mx, qmax);
+    const float inv = sc == 0.0f ? 0.0f : __frcp_rn(sc);
     uint32_t hv0 = 0, lv0 = 0, hv1 = 0, lv1 = 0;
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-      const uint32_t q = quant_code(v(32 * j + e), mn, sc, qmax);
+      const uint32_t q = quant_code(v(32 * j + e), mn, sc, inv, qmax);
       const uint32_t h = (q4 ? (q >> 2) : q) & 3u, l = q & 3u;
       if (e < 16) {
         hv0 |= h << (2 * e);
