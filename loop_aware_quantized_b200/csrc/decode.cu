@@ -887,7 +887,7 @@ __device__ __forceinline__ void key_pass_mma(const Unit& u, int b_begin, int b_e
   const float* km = reinterpret_cast<const float*>(u.data + u.Ld.k_meta + (size_t)first * GB) +
                     (meta ? 4 * lane : 0);
   int* st = reinterpret_cast<int*>(qs);
-  // L2 requests for the group the registers are loading: the lanes whose
+  // L2 requests for a group ahead of the register loads: the lanes whose
   // plane pointers start a 128-byte line request the four token rows of
   // their chunk (K_hi, K_lo), every eighth meta lane its scale and zero lines
   const bool pon_k = g == 0 && (t & 1) == 0 && (D == 128 || t == 0);
@@ -898,7 +898,10 @@ __device__ __forceinline__ void key_pass_mma(const Unit& u, int b_begin, int b_e
   for (;;) {
     const bool hasb = bk + kWarps < b_end;
     if (hasb) load_ktile_mma<D, Q4>(b, kb + STEP, lo_off, km + STEP / 4, meta);
-    if (kAheadK > 0 && hasb) prefetch_kgroup_mma<D, Q4>(kb + STEP, lo_off, km + STEP / 4, pon_k, pon_m);
+    // L2 requests two groups ahead of the register loads (one ahead, the
+    // same group as those loads, measured 1 % slower at two queries)
+    if (kAheadK > 0 && bk + 2 * kWarps < b_end)
+      prefetch_kgroup_mma<D, Q4>(kb + 2 * STEP, lo_off, km + 2 * STEP / 4, pon_k, pon_m);
     key_group_mma<D, Q4, G, ADD>(a, q_s, st, bk * 32, qlim, p0, sc, S, sscale, lane, lmax);
     if (!hasb) break;
     bk += kWarps;
@@ -906,7 +909,8 @@ __device__ __forceinline__ void key_pass_mma(const Unit& u, int b_begin, int b_e
     km += STEP / 4;
     const bool hasa = bk + kWarps < b_end;
     if (hasa) load_ktile_mma<D, Q4>(a, kb + STEP, lo_off, km + STEP / 4, meta);
-    if (kAheadK > 0 && hasa) prefetch_kgroup_mma<D, Q4>(kb + STEP, lo_off, km + STEP / 4, pon_k, pon_m);
+    if (kAheadK > 0 && bk + 2 * kWarps < b_end)
+      prefetch_kgroup_mma<D, Q4>(kb + 2 * STEP, lo_off, km + 2 * STEP / 4, pon_k, pon_m);
     key_group_mma<D, Q4, G, ADD>(b, q_s, st, bk * 32, qlim, p0, sc, S, sscale, lane, lmax);
     if (!hasa) break;
     bk += kWarps;
