@@ -62,6 +62,11 @@ def parse():
     ap.add_argument("--cell-chunks", type=int, default=1,
                     help="decode the cells as this many loop-aligned chunks, each with its own "
                          "cache (plans without SHARE / RES2 cells); a step's time is the sum")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the timed steps one call at a time; by default they are "
+                         "captured (appends and decodes, in serving order) as one CUDA graph "
+                         "after the warm-up and the replay is timed, as a serving engine runs "
+                         "its decode step")
     ap.add_argument("--decode-split", type=int, default=0,
                     help="CTAs per decoded unit at least (0: the library chooses); for "
                          "launch-shape sweeps")
@@ -702,13 +707,31 @@ def time_chunk(args, wl, dev, world, cells_g, seqs, n0, G, total_steps, sampler,
     nsels = [[torch.zeros((len(c), B, H), dtype=torch.int32, device=dev) for c in phase_l]
              for _ in range(args.steps)]
     stream = torch.cuda.current_stream()
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    use_graph = not args.eager
+    # external: inside a captured graph the records become timed event nodes
+    ev = [[(torch.cuda.Event(enable_timing=True, external=use_graph),
+            torch.cuda.Event(enable_timing=True, external=use_graph))
            for _ in phase_l] for _ in range(args.steps)]
 
     for s in range(args.warmup):
         q, k, v = inputs[s]
         steps.decode_step(plan, phase_l, q, k, v, outs)
     torch.cuda.synchronize()
+
+    graph = None
+    if use_graph:
+        # the library only enqueues kernels (lengths advance on the device),
+        # so the K timed steps are captured once and replayed once
+        gstream = torch.cuda.Stream(device=dev)
+        gstream.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gstream):
+            for i in range(args.steps):
+                q, k, v = inputs[args.warmup + i]
+                steps.decode_step(plan, phase_l, q, k, v, outs, nsel=nsels[i], events=ev[i],
+                                  stream=gstream)
+        stream.wait_stream(gstream)
+        torch.cuda.synchronize()
 
     if sampler.proc is None:
         sampler.start()
@@ -718,9 +741,12 @@ def time_chunk(args, wl, dev, world, cells_g, seqs, n0, G, total_steps, sampler,
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for i in range(args.steps):
-        q, k, v = inputs[args.warmup + i]
-        steps.decode_step(plan, phase_l, q, k, v, outs, nsel=nsels[i], events=ev[i])
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(args.steps):
+            q, k, v = inputs[args.warmup + i]
+            steps.decode_step(plan, phase_l, q, k, v, outs, nsel=nsels[i], events=ev[i])
     t_end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -753,7 +779,7 @@ def time_chunk(args, wl, dev, world, cells_g, seqs, n0, G, total_steps, sampler,
         # give this chunk's cache back to the device before the next chunk
         plan.close()
         plan.cache = plan.table = None
-        del plan, gen, inputs, outs, nsels, ev
+        del plan, gen, inputs, outs, nsels, ev, graph
         gc.collect()
         torch.cuda.empty_cache()
     return out
@@ -941,6 +967,10 @@ def main():
         }
         if args.decode_split:
             line["config"]["decode_split"] = args.decode_split
+        line["config"]["launch"] = (
+            "the timed steps launched one call at a time" if args.eager else
+            "the timed steps (appends and decodes) replay as one CUDA graph captured after "
+            "the warm-up")
         if not whole:
             line["config"]["chunks"] = (
                 "%d sequence sub-batch(es) x %d cell chunk(s), decoded one after the other, each "

@@ -219,6 +219,87 @@ def test_decode_replays_from_a_cuda_graph(cuda_device):
     plan.check()
 
 
+def test_serving_steps_replay_from_a_cuda_graph(cuda_device):
+    """A whole serving sequence (three steps of append + decode for the
+    non-final loops, then for the final loop) captured as one CUDA graph and
+    replayed once gives the eager run's outputs, masks, counts and cache
+    bytes, bit for bit: the calls only enqueue kernels, and the appends read
+    and advance the lengths on the device.  The lengths start one token
+    short of a group boundary (31 and 319), so the first captured append
+    quantizes a group."""
+    import torch
+    from loop_aware_quantized_b200 import steps
+    from synth.gpu import DeviceGenerator
+    spec = _spec(128, (Q4, SH, Q2, Q4), (31, 319), 0.01)
+    wl = W.custom(*spec)
+    seqs = [0, 1]
+    n0 = wl.lengths.astype(np.int32)
+    phase = steps.phases(wl.n_loops, wl.n_layers)
+    H, D, B = wl.n_heads, wl.head_dim, len(seqs)
+    n_steps = 3
+    gen = DeviceGenerator(wl, cuda_device)
+    plans = [GH.make_plan(wl, seqs) for _ in range(2)]
+    for plan in plans:
+        plan.cache.zero_()  # bytes the layout leaves undefined start equal too
+        GH.build_cache(wl, plan, gen, seqs, n0)
+    # every step's inputs, shared by both runs
+    ins = []
+    for s in range(n_steps):
+        qs, ks, vs = [], [], []
+        for cells in phase:
+            k, v = gen.kv(list(cells), seqs, n0 + s, 1)
+            ks.append(k)
+            vs.append(v)
+            qs.append(gen.queries(list(cells), seqs, np.tile(n0 + s + 1, (len(cells), 1))))
+        ins.append((qs, ks, vs))
+    mw = int(wl.capacity.max()) // 32 + 1
+
+    def outputs():
+        res = []
+        for _ in range(n_steps):
+            shp = [(len(c), B, H) for c in phase]
+            res.append(dict(out=[torch.zeros(x + (D,), dtype=torch.float32, device=cuda_device)
+                                 for x in shp],
+                            lse=[torch.zeros(x, dtype=torch.float32, device=cuda_device)
+                                 for x in shp],
+                            mask=[torch.zeros(x + (mw,), dtype=torch.int32, device=cuda_device)
+                                  for x in shp],
+                            nsel=[torch.zeros(x, dtype=torch.int32, device=cuda_device)
+                                  for x in shp]))
+        return res
+
+    def run(plan, res, stream=None):
+        for s in range(n_steps):
+            qs, ks, vs = ins[s]
+            r = res[s]
+            steps.decode_step(plan, phase, qs, ks, vs, r["out"], lse=r["lse"], mask=r["mask"],
+                              nsel=r["nsel"], stream=stream)
+
+    eager = outputs()
+    run(plans[0], eager)
+    torch.cuda.synchronize()
+    replay = outputs()
+    s = torch.cuda.Stream(device=cuda_device)
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        run(plans[1], replay, stream=s)
+    # nothing ran during the capture: the cache still holds the bulk build
+    torch.cuda.synchronize()
+    assert not torch.equal(plans[1].cache, plans[0].cache)
+    graph.replay()
+    torch.cuda.synchronize()
+    for s_ in range(n_steps):
+        for key in ("out", "lse", "mask", "nsel"):
+            for i in range(len(phase)):
+                assert torch.equal(eager[s_][key][i], replay[s_][key][i]), (s_, key, i)
+    assert torch.equal(plans[0].cache, plans[1].cache)
+    for plan in plans:
+        plan.check()
+        assert (plan.lengths()[:, :B] == n0 + n_steps).all()
+    del graph
+
+
 def test_kernels_write_only_the_layout_bytes(pool, cuda_device):
     """Guard check (stands in for a memory checker): the cache is filled with
     a sentinel before a bulk build of every kind; afterwards every byte the
