@@ -430,25 +430,40 @@ def bench_vq(args, rank, world):
     ins = [inputs(s) for s in range(n_steps)]
     outs = [torch.empty(ins[0][0][0].shape, dtype=torch.float32, device=dev) for _ in range(L)]
     stream = torch.cuda.current_stream()
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    use_graph = not args.eager
+    # external: inside a captured graph the records become timed event nodes
+    ev = [[(torch.cuda.Event(enable_timing=True, external=use_graph),
+            torch.cuda.Event(enable_timing=True, external=use_graph))
            for _ in range(L)] for _ in range(args.steps)]
 
-    def step(s, inp, events=None):
+    def step(s, inp, events=None, st=None):
         """Encode the token at position n0 + s, then decode over n0 + s + 1."""
         q, xk, xv = inp
-        vq_encode(n0 + s, xk, cbk, ik)
-        vq_encode(n0 + s, xv, cbv, iv)
+        vq_encode(n0 + s, xk, cbk, ik, stream=st)
+        vq_encode(n0 + s, xv, cbv, iv, stream=st)
         lens = n0 + s + 1
         for loop in range(L):
             if events is not None:
-                events[loop][0].record(stream)
-            vq_decode(loop, lens, ik, iv, cbk, cbv, q[loop], out=outs[loop])
+                events[loop][0].record(st or stream)
+            vq_decode(loop, lens, ik, iv, cbk, cbv, q[loop], out=outs[loop], stream=st)
             if events is not None:
-                events[loop][1].record(stream)
+                events[loop][1].record(st or stream)
 
     for s in range(args.warmup):
         step(s, ins[s])
     torch.cuda.synchronize()
+    graph = None
+    if use_graph:
+        # every call takes its lengths and positions by value: the K timed
+        # steps are captured once and replayed once
+        gstream = torch.cuda.Stream(device=dev)
+        gstream.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gstream):
+            for i in range(args.steps):
+                step(args.warmup + i, ins[args.warmup + i], events=ev[i], st=gstream)
+        stream.wait_stream(gstream)
+        torch.cuda.synchronize()
     sampler = ClockSampler(local)
     sampler.start()
     if world > 1:
@@ -457,8 +472,11 @@ def bench_vq(args, rank, world):
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for i in range(args.steps):
-        step(args.warmup + i, ins[args.warmup + i], events=ev[i])
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(args.steps):
+            step(args.warmup + i, ins[args.warmup + i], events=ev[i])
     t_end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -483,7 +501,8 @@ def bench_vq(args, rank, world):
                 "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                 "kernel": "loopkv LoopVQ decode", "bytes_per_launch": launch_bytes,
                 "ms_per_launch": dec_ms / n_launches,
-                "note": "the kernel's shared-memory table lookups bind it before HBM does"}
+                "note": "issue and index-load latency bind the kernel before HBM does (one "
+                        "shared-memory wavefront per table lookup)"}
 
     e2e = None
     if not args.no_e2e:
@@ -540,6 +559,9 @@ def bench_vq(args, rank, world):
                                                  8.0 / (4 * L)),
                        "step": "encode the new token (keys, values), then decode every "
                                "(loop, layer) cell: one launch per loop",
+                       "launch": ("the timed steps launched one call at a time" if args.eager
+                                  else "the timed steps replay as one CUDA graph captured after "
+                                       "the warm-up"),
                        "global_batch": B * world, "seq_len": int(n0[0]),
                        "parallelism": "dp%d (independent sequences)" % world,
                        "l2": "inputs larger than L2 (indices %.1f GB)" % (
