@@ -144,8 +144,9 @@ typedef struct {
                              loopkv_decode for their selection. */
   int32_t decode_split;   /* CTAs (a thread-block cluster) per decoded unit:
                              0 lets the library choose (enough score slots
-                             for the longest unit of a call, more when a call
-                             has too few units to fill the GPU); 1, 2, 4 or
+                             for the longest unit of a call, more while a
+                             call's CTAs fall short of one full wave of two
+                             per SM); 1, 2, 4 or
                              8 asks for at least that many.  The results do
                              not depend on it beyond fp32 rounding order. */
 } loopkv_plan_desc;
