@@ -459,7 +459,7 @@ def bench_vq(args, rank, world):
         gstream = torch.cuda.Stream(device=dev)
         gstream.wait_stream(stream)
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=gstream):
+        with torch.cuda.graph(graph, stream=gstream, capture_error_mode="thread_local"):
             for i in range(args.steps):
                 step(args.warmup + i, ins[args.warmup + i], events=ev[i], st=gstream)
         stream.wait_stream(gstream)
@@ -747,7 +747,7 @@ def time_chunk(args, wl, dev, world, cells_g, seqs, n0, G, total_steps, sampler,
         gstream = torch.cuda.Stream(device=dev)
         gstream.wait_stream(stream)
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=gstream):
+        with torch.cuda.graph(graph, stream=gstream, capture_error_mode="thread_local"):
             for i in range(args.steps):
                 q, k, v = inputs[args.warmup + i]
                 steps.decode_step(plan, phase_l, q, k, v, outs, nsel=nsels[i], events=ev[i],
