@@ -892,6 +892,18 @@ __device__ __forceinline__ void key_pass_mma(const Unit& u, int b_begin, int b_e
   // their chunk (K_hi, K_lo), every eighth meta lane its scale and zero lines
   const bool pon_k = g == 0 && (t & 1) == 0 && (D == 128 || t == 0);
   const bool pon_m = meta && (lane & 7) == 0;
+  if constexpr (G == 4) {
+    // one tile buffer: the registers the second one would hold go to the
+    // value pass; the L2 requests two groups ahead cover the loads' latency
+    for (int bk = first; bk < b_end; bk += kWarps, kb += STEP, km += STEP / 4) {
+      KTileMma<D> a;
+      load_ktile_mma<D, Q4>(a, kb, lo_off, km, meta);
+      if (kAheadK > 0 && bk + 2 * kWarps < b_end)
+        prefetch_kgroup_mma<D, Q4>(kb + 2 * STEP, lo_off, km + 2 * STEP / 4, pon_k, pon_m);
+      key_group_mma<D, Q4, G, ADD>(a, q_s, st, bk * 32, qlim, p0, sc, S, sscale, lane, lmax);
+    }
+    return;
+  }
   KTileMma<D> a, b;
   load_ktile_mma<D, Q4>(a, kb, lo_off, km, meta);
   int bk = first;
