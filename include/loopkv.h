@@ -67,10 +67,13 @@
  *
  * Asynchrony.  loopkv_append, loopkv_decode and loopkv_set_lengths only
  * enqueue work on the given stream and return.  A decode (and the LoopVQ
- * calls) can be captured into a CUDA graph and replayed; an append or
- * set_lengths updates the host copy of the lengths when it is called, so
- * replaying one from a graph would leave that copy behind.  A plan handle
- * must not be used from two host threads at once.
+ * calls) can be captured into a CUDA graph and replayed any number of times.
+ * An append or set_lengths updates the host copy of the lengths when it is
+ * called, i.e. at capture time, while the kernels advance the device lengths
+ * when they run: a graph holding appends (whole serving steps) is to be
+ * replayed once after its capture, which leaves the two copies equal; a
+ * second replay would leave the host copy behind.  A plan handle must not be
+ * used from two host threads at once.
  *
  * Cache layout (canonical, part of the contract).  The cache is one buffer;
  * cell c, sequence b, head h owns a region at loopkv_unit_region().  With
